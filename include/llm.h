@@ -1,0 +1,147 @@
+/*
+ * llm.h -- C ABI of a B200 (sm_100a) library that runs one training step of a
+ * bias-free, pre-norm Llama-style decoder: token embedding -> per layer
+ * [RMSNorm -> causal MHA/GQA attention with RoPE on q,k -> residual -> RMSNorm
+ * -> SwiGLU FFN -> residual] -> final RMSNorm -> untied lm_head -> softmax
+ * cross-entropy, its hand-derived backward pass, and an AdamW update.
+ *
+ * Sources (page title, section):
+ *   Hephaistos, "Architecture at a glance": the block, RMSNorm with cached
+ *     rstd, RoPE on q/k, causal attention with a stable softmax, SwiGLU
+ *     (silu(x W1) * x W3) W2 with hidden floor(8/3 d), untied lm_head, AdamW
+ *     with decoupled weight decay and bias correction; dropout is fixed at 0.
+ *   Hephaistos, "Design notes": parameters in one flat buffer described by
+ *     (offset, len) per tensor; an activation arena cached for backward.
+ *   strata, capability table: n_head and n_kv_head are independent (MHA, GQA,
+ *     MQA); flash-style attention forward and backward with online softmax.
+ *   randyGPT, "Training (Metal GPU path)": cross-entropy over all positions.
+ *
+ * Conventions for every call:
+ *   - Pointers named d_* are DEVICE pointers owned by the caller (for example
+ *     torch tensors passed by data_ptr()).  The library never frees them.
+ *   - Parameters, gradients and Adam moments are flat, unpadded float32
+ *     buffers of llm_param_layout()'s n_params elements, in its order:
+ *     wte[V,d]; per layer g1[d], Wqkv[d, d+2*kvd], Wo[d,d], g2[d],
+ *     W13[d, 2*d_ff] (W1 = columns [0,d_ff), W3 = columns [d_ff, 2*d_ff)),
+ *     W2[d_ff, d]; then gf[d], Wlm[d, V].  Matrices are row-major [in, out],
+ *     so every projection is x W.  kvd = n_kv_head * (d_model / n_head).
+ *     In Wqkv the columns are all q heads, then all k heads, then all v heads;
+ *     query head h uses kv head h / (n_head / n_kv_head).
+ *   - Tokens and targets are int32 [batch, ctx], row-major.
+ *   - All work is enqueued asynchronously on the stream given to llm_create;
+ *     no call synchronises the host except llm_status().
+ *   - Return codes are the LLM_* values below; no exception or abort ever
+ *     crosses this boundary.  LLM_ERR_CONFIG and LLM_ERR_ARG are detected on
+ *     the host before anything is launched.  LLM_ERR_TOKEN and
+ *     LLM_ERR_NONFINITE are detected on the device and reported by
+ *     llm_status(); a step that detects either leaves params, m and v
+ *     unchanged.
+ */
+#ifndef LLM_H_
+#define LLM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  LLM_OK = 0,
+  LLM_ERR_CONFIG = -1,    /* invalid configuration */
+  LLM_ERR_ARG = -2,       /* null/misaligned pointer, workspace too small, bad size */
+  LLM_ERR_TOKEN = -3,     /* a token or target id outside [0, vocab) */
+  LLM_ERR_NONFINITE = -4, /* the loss was not finite */
+  LLM_ERR_CUDA = -5,      /* a CUDA runtime error */
+  LLM_ERR_TIMEOUT = -6    /* a bounded device-side wait gave up */
+};
+
+enum { LLM_FP32 = 0, LLM_BF16 = 1 };
+
+/* Model and optimiser configuration.  d_model must be divisible by n_head,
+ * n_head by n_kv_head, and the head size d_model/n_head must be even (RoPE
+ * rotates pairs (j, j + hd/2)).  compute = LLM_FP32 runs every matmul in
+ * float32; LLM_BF16 runs matmuls and attention with bfloat16 operands and
+ * float32 accumulation, keeping float32 master weights, Adam state and the
+ * residual stream.  rope_base: RoPE base (10000); rms_eps: RMSNorm epsilon
+ * added to the mean square (MicroGPT in Rust, "RMSNorm": 1e-5); beta1, beta2,
+ * adam_eps: AdamW constants (eps is added outside the square root). */
+typedef struct {
+  int32_t vocab, d_model, n_layer, n_head, n_kv_head, d_ff, ctx, batch;
+  float rope_base, rms_eps, beta1, beta2, adam_eps;
+  int32_t compute;
+} llm_config;
+
+/* One tensor of the flat parameter buffer: element (r, c) of a [rows, cols]
+ * tensor sits at offset + r*cols + c.  name is NUL-terminated ("wte",
+ * "l0.g1", "l0.Wqkv", ..., "gf", "Wlm"). */
+typedef struct {
+  char name[32];
+  int64_t offset, rows, cols;
+} llm_tensor_info;
+
+typedef struct llm_ctx llm_ctx;
+
+/* Hephaistos, "Design notes" (flat buffers, named offsets).  On input
+ * *n_tensors is the capacity of out (ignored when out is NULL); on output it
+ * is the number of tensors, and *n_params the total element count.  When out
+ * is non-null and large enough it receives one entry per tensor in buffer
+ * order (LLM_ERR_ARG if too small).  Host-only; LLM_ERR_CONFIG for an invalid
+ * config. */
+int llm_param_layout(const llm_config *cfg, llm_tensor_info *out, int *n_tensors,
+                     int64_t *n_params);
+
+/* Bytes of device workspace llm_create() needs for this config: saved
+ * activations, logits, padded low-precision weight copies, the RoPE table and
+ * scratch.  Host-only. */
+int llm_workspace_bytes(const llm_config *cfg, int64_t *bytes);
+
+/* Builds a context that carves its buffers out of d_workspace (caller-owned,
+ * 256-byte aligned, at least llm_workspace_bytes() long, alive until
+ * llm_destroy) and enqueues work on cuda_stream (a cudaStream_t; NULL = the
+ * legacy default stream).  Enqueues a one-time RoPE table build.  The context
+ * must be used from one host thread at a time. */
+int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void *cuda_stream,
+               llm_ctx **out);
+
+/* Releases host-side state (never the caller's buffers). NULL is ignored. */
+void llm_destroy(llm_ctx *ctx);
+
+/* Fills d_params with a fresh initialisation: every matrix ~ N(0, init_std)
+ * drawn by a counter-based generator keyed by seed; when scale_out_proj != 0,
+ * Wo and W2 use init_std / sqrt(2 n_layer) (randyGPT, Features: GPT-2 style
+ * scaled output projections); RMSNorm gains are 1. */
+int llm_init(llm_ctx *ctx, uint64_t seed, float init_std, int scale_out_proj, float *d_params);
+
+/* Forward pass only: d_logits (float32 [batch, ctx, vocab]) = lm_head output
+ * for d_tokens.  Leaves d_params untouched.  Out-of-range tokens are clamped
+ * for the read and reported by llm_status() as LLM_ERR_TOKEN. */
+int llm_forward(llm_ctx *ctx, const float *d_params, const int32_t *d_tokens, float *d_logits);
+
+/* One training step on the pre-update parameters: loss = mean over all
+ * batch*ctx positions of the cross-entropy of the logits against d_targets,
+ * written to d_loss (one float32 on the device); d_grads is OVERWRITTEN with
+ * d loss / d params; then AdamW updates d_params, d_m and d_v in place
+ * (t = 1-based step count; lr and wd as in p -= lr*wd*p + lr*mhat/(sqrt(vhat)+eps)).
+ * If the step sees an invalid token/target or a non-finite loss, params, m
+ * and v are left untouched and llm_status() reports the error. */
+int llm_step(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,
+             const int32_t *d_tokens, const int32_t *d_targets, float lr, float wd,
+             float *d_loss);
+
+/* Synchronises the context's stream and returns the first error any call on
+ * this context raised on the device since the previous llm_status() (then
+ * clears it), or LLM_ERR_CUDA if the stream reports a CUDA error, else LLM_OK. */
+int llm_status(llm_ctx *ctx);
+
+/* A static, human-readable string for a return code. */
+const char *llm_error_string(int code);
+
+/* Number of kernels the most recent llm_step / llm_forward call enqueued. */
+int llm_last_launch_count(const llm_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLM_H_ */

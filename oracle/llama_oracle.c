@@ -38,6 +38,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+/* Parallel regions only for work large enough to pay for the threads. */
+#define OMP_MIN_WORK (1LL << 18)
+
 typedef struct {
   int32_t V, d, L, H, Hkv, h, T, B;
   double rope_base, eps;
@@ -89,7 +92,7 @@ int orc_param_layout(const orc_cfg *c, int64_t *offs, int64_t *rows, int64_t *co
 /* C[M,N] (=|+=) A[M,K] B[K,N]; leading dimensions given.  Plain definition. */
 void orc_mm_nn(int M, int K, int N, const double *A, int64_t lda, const double *B, int64_t ldb,
                double *C, int64_t ldc, int accumulate) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if ((int64_t)M * K * N > OMP_MIN_WORK)
   for (int i = 0; i < M; i++) {
     double *c = C + (int64_t)i * ldc;
     if (!accumulate) for (int j = 0; j < N; j++) c[j] = 0.0;
@@ -103,7 +106,7 @@ void orc_mm_nn(int M, int K, int N, const double *A, int64_t lda, const double *
 /* C[M,N] (=|+=) A[K,M]^T B[K,N]. */
 void orc_mm_tn(int M, int K, int N, const double *A, int64_t lda, const double *B, int64_t ldb,
                double *C, int64_t ldc, int accumulate) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if ((int64_t)M * K * N > OMP_MIN_WORK)
   for (int i = 0; i < M; i++) {
     double *c = C + (int64_t)i * ldc;
     if (!accumulate) for (int j = 0; j < N; j++) c[j] = 0.0;
@@ -117,7 +120,7 @@ void orc_mm_tn(int M, int K, int N, const double *A, int64_t lda, const double *
 /* C[M,N] (=|+=) A[M,K] B[N,K]^T. */
 void orc_mm_nt(int M, int K, int N, const double *A, int64_t lda, const double *B, int64_t ldb,
                double *C, int64_t ldc, int accumulate) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if ((int64_t)M * K * N > OMP_MIN_WORK)
   for (int i = 0; i < M; i++) {
     const double *a = A + (int64_t)i * lda;
     for (int j = 0; j < N; j++) {
@@ -134,7 +137,7 @@ void orc_mm_nt(int M, int K, int N, const double *A, int64_t lda, const double *
  * no bias, rstd cached.  MicroGPT in Rust, RMSNorm: (mean(x^2) + eps)^-1/2. */
 void orc_rmsnorm_fwd(int n, int d, const double *x, const double *g, double eps, double *y,
                      double *rstd) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if ((int64_t)n * d > OMP_MIN_WORK)
   for (int i = 0; i < n; i++) {
     const double *xi = x + (int64_t)i * d;
     double ss = 0.0;
@@ -148,7 +151,7 @@ void orc_rmsnorm_fwd(int n, int d, const double *x, const double *g, double eps,
  * dg += sum_rows dy * x * r.  dx is written (accumulate=0) or added to. */
 void orc_rmsnorm_bwd(int n, int d, const double *x, const double *rstd, const double *g,
                      const double *dy, double *dx, double *dg, int accumulate) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if ((int64_t)n * d > OMP_MIN_WORK)
   for (int i = 0; i < n; i++) {
     const double *xi = x + (int64_t)i * d, *dyi = dy + (int64_t)i * d;
     double r = rstd[i], dot = 0.0;
@@ -192,7 +195,7 @@ void orc_attention_fwd(int T, int d, int H, int Hkv, const double *qkv, double *
   int hd = d / H, grp = H / Hkv;
   int64_t w = (int64_t)d + 2LL * hd * Hkv;
   double scale = 1.0 / sqrt((double)hd);
-#pragma omp parallel for collapse(2) schedule(static)
+#pragma omp parallel for collapse(2) schedule(static) if ((int64_t)H * T * T * hd > OMP_MIN_WORK)
   for (int hq = 0; hq < H; hq++) {
     for (int i = 0; i < T; i++) {
       int g = hq / grp;
@@ -237,7 +240,7 @@ void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const do
   double *dS = (double *)calloc((size_t)H * T * T, sizeof(double));
   memset(dqkv, 0, sizeof(double) * (size_t)T * w);
   /* P and dS, one (query head, row) per iteration */
-#pragma omp parallel for collapse(2) schedule(static)
+#pragma omp parallel for collapse(2) schedule(static) if ((int64_t)H * T * T * hd > OMP_MIN_WORK)
   for (int hq = 0; hq < H; hq++) {
     for (int i = 0; i < T; i++) {
       int g = hq / grp;
@@ -274,7 +277,7 @@ void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const do
   }
   /* dk_j, dv_j: one (kv head, key row) per iteration, summed over the group's
    * query heads in head order, then over i */
-#pragma omp parallel for collapse(2) schedule(static)
+#pragma omp parallel for collapse(2) schedule(static) if ((int64_t)H * T * T * hd > OMP_MIN_WORK)
   for (int g = 0; g < Hkv; g++) {
     for (int j = 0; j < T; j++) {
       double *dk = dqkv + (int64_t)j * w + d + (int64_t)g * hd;
@@ -300,14 +303,14 @@ void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const do
 /* Hephaistos, Architecture at a glance (Feed-forward): u = silu(a) * b with
  * a = x W1, b = x W3, silu(a) = a / (1 + e^-a). */
 void orc_swiglu_fwd(int64_t n, const double *a, const double *b, double *u) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if (n > OMP_MIN_WORK)
   for (int64_t i = 0; i < n; i++) u[i] = a[i] / (1.0 + exp(-a[i])) * b[i];
 }
 /* da = du * b * silu'(a), db = du * silu(a); silu'(a) = s (1 + a (1 - s)),
  * s = 1/(1+e^-a). */
 void orc_swiglu_bwd(int64_t n, const double *a, const double *b, const double *du, double *da,
                     double *db) {
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if (n > OMP_MIN_WORK)
   for (int64_t i = 0; i < n; i++) {
     double s = 1.0 / (1.0 + exp(-a[i]));
     da[i] = du[i] * b[i] * s * (1.0 + a[i] * (1.0 - s));
@@ -323,7 +326,7 @@ double orc_ce_fwd_bwd(int n, int V, const double *z, const int32_t *y, double in
                       double *dz) {
   double total = 0.0;
   double *row_loss = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if ((int64_t)n * V > OMP_MIN_WORK)
   for (int i = 0; i < n; i++) {
     const double *zi = z + (int64_t)i * V;
     double mx = -INFINITY;
@@ -484,7 +487,7 @@ double orc_forward_backward(const orc_cfg *c, const double *params, const int32_
 void orc_adamw(int64_t n, double *p, const double *g, double *m, double *v, int64_t t, double lr,
                double wd, double b1, double b2, double eps) {
   double bc1 = 1.0 - pow(b1, (double)t), bc2 = 1.0 - pow(b2, (double)t);
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(static) if (n > OMP_MIN_WORK)
   for (int64_t i = 0; i < n; i++) {
     m[i] = b1 * m[i] + (1.0 - b1) * g[i];
     v[i] = b2 * v[i] + (1.0 - b2) * g[i] * g[i];

@@ -1,0 +1,98 @@
+"""ctypes binding of libllm.so (include/llm.h): argument marshalling only.
+
+Every computation runs in the library's CUDA kernels.  Importing this module
+raises if the library has not been built; there is no fallback.
+"""
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libllm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m scratch_llama_decoder_b200.build` "
+        "(nvcc, sm_100a).  There is no CPU fallback.")
+
+lib = C.CDLL(LIB_PATH)
+
+LLM_OK, LLM_ERR_CONFIG, LLM_ERR_ARG, LLM_ERR_TOKEN = 0, -1, -2, -3
+LLM_ERR_NONFINITE, LLM_ERR_CUDA, LLM_ERR_TIMEOUT = -4, -5, -6
+LLM_FP32, LLM_BF16 = 0, 1
+
+
+class llm_config(C.Structure):
+    _fields_ = [("vocab", C.c_int32), ("d_model", C.c_int32), ("n_layer", C.c_int32),
+                ("n_head", C.c_int32), ("n_kv_head", C.c_int32), ("d_ff", C.c_int32),
+                ("ctx", C.c_int32), ("batch", C.c_int32), ("rope_base", C.c_float),
+                ("rms_eps", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float),
+                ("adam_eps", C.c_float), ("compute", C.c_int32)]
+
+
+class llm_tensor_info(C.Structure):
+    _fields_ = [("name", C.c_char * 32), ("offset", C.c_int64), ("rows", C.c_int64),
+                ("cols", C.c_int64)]
+
+
+_vp, _i64, _u64, _f, _i = C.c_void_p, C.c_int64, C.c_uint64, C.c_float, C.c_int
+_cfgp = C.POINTER(llm_config)
+
+EXPORTS = {
+    "llm_param_layout": (_i, [_cfgp, C.POINTER(llm_tensor_info), C.POINTER(_i), C.POINTER(_i64)]),
+    "llm_workspace_bytes": (_i, [_cfgp, C.POINTER(_i64)]),
+    "llm_create": (_i, [_cfgp, _vp, _i64, _vp, C.POINTER(_vp)]),
+    "llm_destroy": (None, [_vp]),
+    "llm_init": (_i, [_vp, _u64, _f, _i, _vp]),
+    "llm_forward": (_i, [_vp, _vp, _vp, _vp]),
+    "llm_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _f, _f, _vp]),
+    "llm_status": (_i, [_vp]),
+    "llm_error_string": (C.c_char_p, [_i]),
+    "llm_last_launch_count": (_i, [_vp]),
+}
+for _name, (_res, _args) in EXPORTS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class LLMError(RuntimeError):
+    def __init__(self, code, where):
+        super().__init__(f"{where}: {lib.llm_error_string(code).decode()} ({code})")
+        self.code = code
+
+
+def check(code, where):
+    if code != LLM_OK:
+        raise LLMError(code, where)
+    return code
+
+
+def make_config(cfg) -> llm_config:
+    """llm_config from a mapping with the field names of include/llm.h
+    (compute given as "fp32"/"bf16" or 0/1)."""
+    comp = cfg.get("compute", 0)
+    if isinstance(comp, str):
+        comp = {"fp32": LLM_FP32, "bf16": LLM_BF16}[comp]
+    return llm_config(cfg["vocab"], cfg["d_model"], cfg["n_layer"], cfg["n_head"],
+                      cfg["n_kv_head"], cfg["d_ff"], cfg["ctx"], cfg["batch"],
+                      float(cfg.get("rope_base", 10000.0)), float(cfg.get("rms_eps", 1e-5)),
+                      float(cfg.get("beta1", 0.9)), float(cfg.get("beta2", 0.999)),
+                      float(cfg.get("adam_eps", 1e-8)), int(comp))
+
+
+def llm_param_layout(cfg):
+    """[(name, offset, rows, cols)], n_params."""
+    c = make_config(cfg)
+    n = C.c_int(0)
+    npar = C.c_int64(0)
+    check(lib.llm_param_layout(C.byref(c), None, C.byref(n), C.byref(npar)), "llm_param_layout")
+    arr = (llm_tensor_info * n.value)()
+    check(lib.llm_param_layout(C.byref(c), arr, C.byref(n), C.byref(npar)), "llm_param_layout")
+    return [(t.name.decode(), t.offset, t.rows, t.cols) for t in arr], npar.value
+
+
+def llm_workspace_bytes(cfg) -> int:
+    c = make_config(cfg)
+    b = C.c_int64(0)
+    check(lib.llm_workspace_bytes(C.byref(c), C.byref(b)), "llm_workspace_bytes")
+    return b.value

@@ -1,0 +1,33 @@
+// Tensor-core (tcgen05 / TMEM / TMA) paths of the training step: the GEMMs with
+// their fused epilogues and the flash-style attention.  A TcPlan exists only
+// for bfloat16 contexts; every entry returns false (or falls back to the SIMT
+// kernels) for shapes it does not tile.
+#pragma once
+#include "internal.h"
+
+namespace llm {
+
+struct TcPlan;
+
+enum TcEpi {
+  TC_EPI_NONE = 0,       // plain output as selected by GemmOut
+  TC_EPI_ROPE = 1,       // QKV forward: rotate q and k columns (RoPE) in the epilogue
+  TC_EPI_SWIGLU = 2,     // W13 forward: store [a|b] and u = silu(a) * b (aux = u)
+  TC_EPI_SWIGLU_BWD = 3  // W2 dgrad: du -> [da|db] using the saved [a|b] (aux = ab)
+};
+
+TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, int hd,
+                       int64_t rot_cols, int64_t hp);
+void tc_plan_destroy(TcPlan *p);
+bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
+             int64_t ldr, int splits, int epi, const void *aux, cudaStream_t s);
+
+// Attention dispatch: tensor-core kernels when the plan covers the head size,
+// else the SIMT kernels.
+void attention_fwd(TcPlan *p, const void *qkv, void *o, float *lse, DType dt, int B, int T, int H,
+                   int Hkv, int hd, cudaStream_t s);
+void attention_bwd(TcPlan *p, const void *qkv, const void *o, const void *dout, const float *lse,
+                   float *Dbuf, void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd,
+                   cudaStream_t s);
+
+}  // namespace llm

@@ -1,0 +1,91 @@
+// Host-side launchers of the training-step kernels (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace llm {
+
+// Error bits of the per-step flag word in device memory.
+enum : int { FLAG_TOKEN = 1, FLAG_NONFINITE = 2, FLAG_TIMEOUT = 4 };
+
+// Activation/operand element type of a launch: float32 or bfloat16.
+enum DType { DT_F32 = 0, DT_BF16 = 1 };
+
+// ------------------------------------------------------------ GEMM (shared)
+// C[M,N] = A[M,K] * B^T where B is given as an [N,K] operand:
+//   A element (m,k) = a_kmajor ? A[m*lda + k] : A[k*lda + m]
+//   B element (n,k) = b_kmajor ? B[n*ldb + k] : B[k*ldb + n]
+struct GemmOperands {
+  int M, N, K;
+  const void *A; int64_t lda; bool a_kmajor;
+  const void *B; int64_t ldb; bool b_kmajor;
+  DType in;  // operand type of A and B
+};
+enum GemmOut {
+  OUT_F32 = 0,      // C (float) = acc
+  OUT_ACT = 1,      // C (operand type) = acc, rounded
+  OUT_ADD_F32 = 2,  // C (float) = R + acc
+  OUT_PARTIAL = 3   // C (float) [split][M][ldc] = partial sum over the split's K range
+};
+// SIMT (CUDA-core) GEMM: any shape, float32 accumulation.  Counts launches.
+void gemm_simt(const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
+               int64_t ldr, int splits, cudaStream_t s);
+
+// ------------------------------------------------------------- elementwise
+void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStream_t s);
+// Low-precision (or float32) padded copy of one weight matrix.
+//   mode 0: dst[r, c] = src[r, c] (zero outside rows x cols), dst [rows_p, cols_p]
+//   mode 1: W13 interleave: src [rows, 2h], dst [rows, 2hp] block-interleaved
+void cast_weight(const float *src, void *dst, DType dt, int64_t rows, int64_t cols,
+                 int64_t rows_p, int64_t cols_p, int mode, int64_t h, int64_t hp, int batch,
+                 int64_t src_batch_stride, int64_t dst_batch_stride, cudaStream_t s);
+void embed_fwd(const float *wte, const int32_t *tok, float *x, int64_t N, int d, int V,
+               int *flag, cudaStream_t s);
+void rmsnorm_fwd(const float *x, const float *g, void *y, DType dt, float *rstd, int64_t N, int d,
+                 float eps, cudaStream_t s);
+// dx = dres + rmsnorm_bwd(dy); optional low-precision copy dx_act; dg partial
+// sums per block into part[nblk, d].  Returns the number of partial blocks.
+int rmsnorm_bwd(const float *x, const float *rstd, const float *g, const float *dy,
+                const float *dres, float *dx, void *dx_act, DType dt, float *part, int64_t N,
+                int d, cudaStream_t s);
+int rmsnorm_bwd_blocks(int64_t N);
+void reduce_partials(const float *part, int nblk, int d, float *out, cudaStream_t s);
+void rope_apply(void *qkv, DType dt, const float *cos_t, const float *sin_t, int64_t N, int T,
+                int ncols_rot, int64_t ld, int hd, int sign, cudaStream_t s);
+void swiglu_fwd(const void *ab, void *u, DType dt, int64_t N, int64_t hp, cudaStream_t s);
+void swiglu_bwd(const void *ab, const void *du, void *dab, DType dt, int64_t N, int64_t hp,
+                cudaStream_t s);
+void cross_entropy(void *logits, DType dt, const int32_t *tgt, float *rowloss, int64_t N, int V,
+                   int64_t ldz, float inv_n, int *flag, cudaStream_t s);
+void loss_reduce(const float *rowloss, int64_t N, float *loss, int *flag, cudaStream_t s);
+void logits_out(const void *logits, DType dt, float *out, int64_t N, int V, int64_t ldz,
+                cudaStream_t s);
+void adamw(float *p, const float *g, float *m, float *v, int64_t n, float lr, float wd, float b1,
+           float b2, float eps, float bc1, float bc2, const int *flag, cudaStream_t s);
+// grad[r, c] (unpadded rows x cols) = sum over splits of part[s][r'][c'].
+//   mode 0: identity; mode 1: W13 de-interleave (cols = 2h, part cols 2hp)
+void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp, float *grad,
+                  int64_t rows, int64_t cols, int mode, int64_t h, cudaStream_t s);
+// Deterministic embedding backward: dwte[v] = sum over i with tok_i = v of dx[i],
+// summed in increasing i; rows without tokens are zero.
+void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int d, int V,
+               int32_t *scratch, cudaStream_t s);
+int64_t embed_bwd_scratch_ints(int64_t N, int V);
+void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, float std,
+                 int constant_one, cudaStream_t s);
+void set_flag_zero(int *flag, cudaStream_t s);
+void or_flag(const int *src, int *dst, cudaStream_t s);
+
+// --------------------------------------------------------------- attention
+// qkv [N, qkvw] (q heads | k heads | v heads, RoPE applied), o [N, H*hd],
+// lse [B, H, T]; SIMT reference kernels for any head size.
+void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
+                   int hd, cudaStream_t s);
+void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
+                   void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s);
+
+// Launch counter (kernels enqueued by the current call).
+extern thread_local int g_launches;
+inline void count_launch(int n = 1) { g_launches += n; }
+
+}  // namespace llm

@@ -1,0 +1,615 @@
+// Memory-bound kernels of the training step: weight casts, embedding gather and
+// scatter-add, RMSNorm forward/backward, RoPE, SwiGLU, cross-entropy, loss
+// reduction, AdamW and initialisation.  Each cites the passage it computes.
+#include "common.cuh"
+#include "internal.h"
+
+namespace llm {
+
+thread_local int g_launches = 0;
+
+static inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
+
+// ------------------------------------------------------------------ RoPE table
+// Hephaistos, Architecture at a glance (Positions): rotary embedding of q and
+// k.  theta_j = base^(-2j/hd); angle = t * theta_j for position t.  The table
+// is built once, in double precision, then rounded to float.
+__global__ void k_rope_table(float *cos_t, float *sin_t, int T, int half, int hd, double base) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= (int64_t)T * half) return;
+  int t = (int)(i / half), j = (int)(i % half);
+  double ang = (double)t * pow(base, -2.0 * j / hd);
+  cos_t[i] = (float)cos(ang);
+  sin_t[i] = (float)sin(ang);
+}
+void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStream_t s) {
+  int64_t n = (int64_t)T * (hd / 2);
+  k_rope_table<<<cdiv(n, 256), 256, 0, s>>>(cos_t, sin_t, T, hd / 2, hd, (double)base);
+  count_launch();
+}
+
+// ------------------------------------------------------------- weight casts
+template <typename A>
+__global__ void k_cast_weight(const float *__restrict__ src, A *__restrict__ dst, int64_t rows,
+                              int64_t cols, int64_t rows_p, int64_t cols_p, int mode, int64_t h,
+                              int64_t hp, int64_t sbs, int64_t dbs) {
+  int64_t n = rows_p * cols_p;
+  src += blockIdx.y * sbs;
+  dst += blockIdx.y * dbs;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t r = i / cols_p, c = i % cols_p;
+    float v = 0.f;
+    if (mode == 0) {
+      if (r < rows && c < cols) v = src[r * cols + c];
+    } else {
+      // interleaved W1|W3 blocks of SWIGLU_BLOCK columns
+      int64_t blk = c / (2 * SWIGLU_BLOCK), w = c % (2 * SWIGLU_BLOCK);
+      int64_t j = blk * SWIGLU_BLOCK + (w % SWIGLU_BLOCK);
+      if (j < h) v = src[r * cols + (w < SWIGLU_BLOCK ? j : h + j)];
+    }
+    dst[i] = from_f<A>(v);
+  }
+}
+void cast_weight(const float *src, void *dst, DType dt, int64_t rows, int64_t cols,
+                 int64_t rows_p, int64_t cols_p, int mode, int64_t h, int64_t hp, int batch,
+                 int64_t sbs, int64_t dbs, cudaStream_t s) {
+  int64_t n = rows_p * cols_p;
+  dim3 grid(min(cdiv(n, 256), 4096u), batch);
+  if (dt == DT_BF16)
+    k_cast_weight<<<grid, 256, 0, s>>>(src, (__nv_bfloat16 *)dst, rows, cols, rows_p, cols_p, mode,
+                                       h, hp, sbs, dbs);
+  else
+    k_cast_weight<<<grid, 256, 0, s>>>(src, (float *)dst, rows, cols, rows_p, cols_p, mode, h, hp,
+                                       sbs, dbs);
+  count_launch();
+}
+
+// ------------------------------------------------------------ embedding fwd
+// Hephaistos, Architecture at a glance: token embedding, no positional table.
+// x[i,:] = wte[tok_i,:].  Out-of-range ids set FLAG_TOKEN and read row 0.
+__global__ void k_embed_fwd(const float *__restrict__ wte, const int32_t *__restrict__ tok,
+                            float *__restrict__ x, int64_t N, int d, int V, int *flag) {
+  int64_t row = blockIdx.x;
+  int t = tok[row];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) atomicOr(flag, FLAG_TOKEN);
+    t = 0;
+  }
+  const float *src = wte + (int64_t)t * d;
+  float *dst = x + row * d;
+  if ((d & 3) == 0) {
+    for (int j = threadIdx.x; j < d / 4; j += blockDim.x)
+      reinterpret_cast<float4 *>(dst)[j] = reinterpret_cast<const float4 *>(src)[j];
+  } else {
+    for (int j = threadIdx.x; j < d; j += blockDim.x) dst[j] = src[j];
+  }
+}
+void embed_fwd(const float *wte, const int32_t *tok, float *x, int64_t N, int d, int V, int *flag,
+               cudaStream_t s) {
+  k_embed_fwd<<<(unsigned)N, min(256, max(32, d / 4)), 0, s>>>(wte, tok, x, N, d, V, flag);
+  count_launch();
+}
+
+// -------------------------------------------------------------- RMSNorm fwd
+// Hephaistos, Architecture at a glance (Normalization); MicroGPT in Rust,
+// RMSNorm: r = (mean_j x_j^2 + eps)^-1/2, y = g * x * r; r is cached.
+// One warp per row.
+template <typename A>
+__global__ void k_rmsnorm_fwd(const float *__restrict__ x, const float *__restrict__ g,
+                              A *__restrict__ y, float *__restrict__ rstd, int64_t N, int d,
+                              float eps) {
+  int64_t row = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
+  int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const float *xr = x + row * d;
+  float ss = 0.f;
+  if ((d & 127) == 0) {
+    for (int j = lane * 4; j < d; j += 128) {
+      float4 v = *reinterpret_cast<const float4 *>(xr + j);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+  } else {
+    for (int j = lane; j < d; j += 32) ss += xr[j] * xr[j];
+  }
+  ss = warp_sum(ss);
+  float r = 1.0f / sqrtf(ss / (float)d + eps);
+  if (lane == 0) rstd[row] = r;
+  A *yr = y + row * d;
+  for (int j = lane; j < d; j += 32) yr[j] = from_f<A>(g[j] * xr[j] * r);
+}
+void rmsnorm_fwd(const float *x, const float *g, void *y, DType dt, float *rstd, int64_t N, int d,
+                 float eps, cudaStream_t s) {
+  unsigned grid = cdiv(N, 8);
+  if (dt == DT_BF16)
+    k_rmsnorm_fwd<<<grid, 256, 0, s>>>(x, g, (__nv_bfloat16 *)y, rstd, N, d, eps);
+  else
+    k_rmsnorm_fwd<<<grid, 256, 0, s>>>(x, g, (float *)y, rstd, N, d, eps);
+  count_launch();
+}
+
+// -------------------------------------------------------------- RMSNorm bwd
+// Backward of y = g x r:  dx = r g dy - x r^3 (1/d) sum_j g_j dy_j x_j, plus
+// the residual gradient dres; dg = sum over rows of dy x r, reduced in a fixed
+// order: each block writes the partial sum of its RMS_ROWS rows, and
+// reduce_partials adds the blocks in index order.
+constexpr int RMS_ROWS = 64;
+int rmsnorm_bwd_blocks(int64_t N) { return (int)cdiv(N, RMS_ROWS); }
+
+template <typename A>
+__global__ void k_rmsnorm_bwd(const float *__restrict__ x, const float *__restrict__ rstd,
+                              const float *__restrict__ g, const float *__restrict__ dy,
+                              const float *dres, float *dx,  // may alias (read then write)
+                              A *__restrict__ dx_act, float *__restrict__ part, int64_t N, int d) {
+  extern __shared__ float sacc[];  // [nwarps][d]
+  int warp = threadIdx.x / 32, lane = threadIdx.x & 31, nw = blockDim.x / 32;
+  float *acc = sacc + (int64_t)warp * d;
+  for (int j = lane; j < d; j += 32) acc[j] = 0.f;
+  int64_t r0 = (int64_t)blockIdx.x * RMS_ROWS;
+  for (int rr = warp; rr < RMS_ROWS; rr += nw) {
+    int64_t row = r0 + rr;
+    if (row >= N) break;
+    const float *xr = x + row * d, *dyr = dy + row * d;
+    float r = rstd[row];
+    float dot = 0.f;
+    for (int j = lane; j < d; j += 32) dot += g[j] * dyr[j] * xr[j];
+    dot = warp_sum(dot);
+    float c = r * r * r * dot / (float)d;
+    for (int j = lane; j < d; j += 32) {
+      float v = r * g[j] * dyr[j] - xr[j] * c;
+      if (dres) v += dres[row * d + j];
+      dx[row * d + j] = v;
+      if (dx_act) dx_act[row * d + j] = from_f<A>(v);
+      acc[j] += dyr[j] * xr[j] * r;
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float s = 0.f;
+    for (int w = 0; w < nw; w++) s += sacc[(int64_t)w * d + j];
+    part[(int64_t)blockIdx.x * d + j] = s;
+  }
+}
+int rmsnorm_bwd(const float *x, const float *rstd, const float *g, const float *dy,
+                const float *dres, float *dx, void *dx_act, DType dt, float *part, int64_t N, int d,
+                cudaStream_t s) {
+  int nblk = rmsnorm_bwd_blocks(N);
+  size_t smem = sizeof(float) * 8 * d;
+  if (dt == DT_BF16)
+    k_rmsnorm_bwd<<<nblk, 256, smem, s>>>(x, rstd, g, dy, dres, dx, (__nv_bfloat16 *)dx_act, part,
+                                          N, d);
+  else
+    k_rmsnorm_bwd<<<nblk, 256, smem, s>>>(x, rstd, g, dy, dres, dx, (float *)dx_act, part, N, d);
+  count_launch();
+  return nblk;
+}
+
+__global__ void k_reduce_partials(const float *__restrict__ part, int nblk, int d,
+                                  float *__restrict__ out) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  float s = 0.f;
+  for (int b = 0; b < nblk; b++) s += part[(int64_t)b * d + j];
+  out[j] = s;
+}
+void reduce_partials(const float *part, int nblk, int d, float *out, cudaStream_t s) {
+  k_reduce_partials<<<cdiv(d, 128), 128, 0, s>>>(part, nblk, d, out);
+  count_launch();
+}
+
+// --------------------------------------------------------------------- RoPE
+// Rotate-half rotation of the q and k columns (the first ncols_rot columns of
+// each row, heads of hd) by +angle (sign 1, forward) or -angle (sign -1, the
+// backward of the forward rotation).  Position = row % T.
+template <typename A>
+__global__ void k_rope_apply(A *__restrict__ qkv, const float *__restrict__ cos_t,
+                             const float *__restrict__ sin_t, int64_t N, int T, int ncols_rot,
+                             int64_t ld, int hd, float sign) {
+  int half = hd / 2;
+  int64_t pairs_per_row = ncols_rot / 2;
+  int64_t n = N * pairs_per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t row = i / pairs_per_row;
+    int p = (int)(i % pairs_per_row);
+    int head = p / half, j = p % half;
+    int t = (int)(row % T);
+    float c = cos_t[(int64_t)t * half + j], sn = sign * sin_t[(int64_t)t * half + j];
+    A *u = qkv + row * ld + (int64_t)head * hd;
+    float a = to_f(u[j]), b = to_f(u[j + half]);
+    u[j] = from_f<A>(a * c - b * sn);
+    u[j + half] = from_f<A>(b * c + a * sn);
+  }
+}
+void rope_apply(void *qkv, DType dt, const float *cos_t, const float *sin_t, int64_t N, int T,
+                int ncols_rot, int64_t ld, int hd, int sign, cudaStream_t s) {
+  int64_t n = N * (ncols_rot / 2);
+  unsigned grid = min(cdiv(n, 256), 148u * 16);
+  if (dt == DT_BF16)
+    k_rope_apply<<<grid, 256, 0, s>>>((__nv_bfloat16 *)qkv, cos_t, sin_t, N, T, ncols_rot, ld, hd,
+                                      (float)sign);
+  else
+    k_rope_apply<<<grid, 256, 0, s>>>((float *)qkv, cos_t, sin_t, N, T, ncols_rot, ld, hd,
+                                      (float)sign);
+  count_launch();
+}
+
+// ------------------------------------------------------------------- SwiGLU
+// Hephaistos, Architecture at a glance (Feed-forward): u = silu(a) * b.
+// ab is [N, 2hp] in interleaved blocks (a columns then b columns per block).
+template <typename A>
+__global__ void k_swiglu_fwd(const A *__restrict__ ab, A *__restrict__ u, int64_t N, int64_t hp) {
+  int64_t n = N * hp;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t row = i / hp, j = i % hp;
+    const A *r = ab + row * 2 * hp;
+    int64_t ca = w1_col(j);
+    float a = to_f(r[ca]), b = to_f(r[ca + SWIGLU_BLOCK]);
+    u[i] = from_f<A>(a * sigmoidf_(a) * b);
+  }
+}
+// da = du * b * silu'(a), db = du * silu(a), silu'(a) = s (1 + a (1 - s)).
+template <typename A>
+__global__ void k_swiglu_bwd(const A *__restrict__ ab, const A *__restrict__ du,
+                             A *__restrict__ dab, int64_t N, int64_t hp) {
+  int64_t n = N * hp;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t row = i / hp, j = i % hp;
+    const A *r = ab + row * 2 * hp;
+    int64_t ca = w1_col(j);
+    float a = to_f(r[ca]), b = to_f(r[ca + SWIGLU_BLOCK]), g = to_f(du[i]);
+    float sg = sigmoidf_(a);
+    dab[row * 2 * hp + ca] = from_f<A>(g * b * sg * (1.f + a * (1.f - sg)));
+    dab[row * 2 * hp + ca + SWIGLU_BLOCK] = from_f<A>(g * a * sg);
+  }
+}
+void swiglu_fwd(const void *ab, void *u, DType dt, int64_t N, int64_t hp, cudaStream_t s) {
+  unsigned grid = min(cdiv(N * hp, 256), 148u * 16);
+  if (dt == DT_BF16)
+    k_swiglu_fwd<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)ab, (__nv_bfloat16 *)u, N, hp);
+  else
+    k_swiglu_fwd<<<grid, 256, 0, s>>>((const float *)ab, (float *)u, N, hp);
+  count_launch();
+}
+void swiglu_bwd(const void *ab, const void *du, void *dab, DType dt, int64_t N, int64_t hp,
+                cudaStream_t s) {
+  unsigned grid = min(cdiv(N * hp, 256), 148u * 16);
+  if (dt == DT_BF16)
+    k_swiglu_bwd<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)ab, (const __nv_bfloat16 *)du,
+                                      (__nv_bfloat16 *)dab, N, hp);
+  else
+    k_swiglu_bwd<<<grid, 256, 0, s>>>((const float *)ab, (const float *)du, (float *)dab, N, hp);
+  count_launch();
+}
+
+// ------------------------------------------------------------ cross-entropy
+// Fused softmax cross-entropy forward and backward over the vocabulary
+// (Hephaistos, "What you'll see": softmax+CE; randyGPT: over all positions).
+// Per row: lse = log sum_v exp(z_v); loss_i = lse - z_{y_i};
+// dz_v = (exp(z_v - lse) - [v = y_i]) * inv_n written over z in place.
+// Probabilities are never stored.  Columns >= V (padding) become 0.
+template <typename A, int NT>
+__global__ void __launch_bounds__(NT) k_cross_entropy(A *__restrict__ z, const int32_t *__restrict__ tgt,
+                                                      float *__restrict__ rowloss, int V,
+                                                      int64_t ldz, float inv_n, int *flag) {
+  __shared__ float sm[NT / 32], ss[NT / 32];
+  int64_t row = blockIdx.x;
+  A *zr = z + row * ldz;
+  float m = -INFINITY, s = 0.f;
+  for (int v = threadIdx.x; v < V; v += NT) {
+    float x = to_f(zr[v]);
+    if (x > m) { s = s * expf(m - x) + 1.f; m = x; }
+    else s += expf(x - m);
+  }
+  // merge (m, s) across the block
+  int lane = threadIdx.x & 31, w = threadIdx.x / 32;
+  for (int o = 16; o > 0; o >>= 1) {
+    float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    float mm = fmaxf(m, m2);
+    s = (mm == -INFINITY) ? 0.f : s * expf(m - mm) + s2 * expf(m2 - mm);
+    m = mm;
+  }
+  if (lane == 0) { sm[w] = m; ss[w] = s; }
+  __syncthreads();
+  float M = -INFINITY;
+  for (int i = 0; i < NT / 32; i++) M = fmaxf(M, sm[i]);
+  float S = 0.f;
+  for (int i = 0; i < NT / 32; i++) S += (sm[i] == -INFINITY) ? 0.f : ss[i] * expf(sm[i] - M);
+  float lse = M + logf(S);
+  int y = tgt[row];
+  if (y < 0 || y >= V) {
+    if (threadIdx.x == 0) atomicOr(flag, FLAG_TOKEN);
+    y = 0;
+  }
+  float zy = to_f(zr[y]);
+  __syncthreads();  // every thread has read z[y] before it is overwritten
+  if (threadIdx.x == 0) rowloss[row] = lse - zy;
+  for (int64_t v = threadIdx.x; v < ldz; v += NT) {
+    float g = 0.f;
+    if (v < V) g = (expf(to_f(zr[v]) - lse) - (v == y ? 1.f : 0.f)) * inv_n;
+    zr[v] = from_f<A>(g);
+  }
+}
+void cross_entropy(void *logits, DType dt, const int32_t *tgt, float *rowloss, int64_t N, int V,
+                   int64_t ldz, float inv_n, int *flag, cudaStream_t s) {
+  if (dt == DT_BF16)
+    k_cross_entropy<__nv_bfloat16, 256><<<(unsigned)N, 256, 0, s>>>((__nv_bfloat16 *)logits, tgt,
+                                                                   rowloss, V, ldz, inv_n, flag);
+  else
+    k_cross_entropy<float, 256><<<(unsigned)N, 256, 0, s>>>((float *)logits, tgt, rowloss, V, ldz,
+                                                           inv_n, flag);
+  count_launch();
+}
+
+// Mean of the row losses in a fixed order; a non-finite mean sets
+// FLAG_NONFINITE.
+__global__ void k_loss_reduce(const float *__restrict__ rowloss, int64_t N, float *loss, int *flag) {
+  __shared__ double sh[1024];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < N; i += blockDim.x) s += (double)rowloss[i];
+  sh[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float l = (float)(sh[0] / (double)N);
+    *loss = l;
+    if (!isfinite(l)) atomicOr(flag, FLAG_NONFINITE);
+  }
+}
+void loss_reduce(const float *rowloss, int64_t N, float *loss, int *flag, cudaStream_t s) {
+  k_loss_reduce<<<1, 1024, 0, s>>>(rowloss, N, loss, flag);
+  count_launch();
+}
+
+template <typename A>
+__global__ void k_logits_out(const A *__restrict__ z, float *__restrict__ out, int64_t N, int V,
+                             int64_t ldz) {
+  int64_t n = N * V;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = to_f(z[(i / V) * ldz + i % V]);
+}
+void logits_out(const void *logits, DType dt, float *out, int64_t N, int V, int64_t ldz,
+                cudaStream_t s) {
+  unsigned grid = min(cdiv(N * V, 256), 148u * 32);
+  if (dt == DT_BF16)
+    k_logits_out<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)logits, out, N, V, ldz);
+  else
+    k_logits_out<<<grid, 256, 0, s>>>((const float *)logits, out, N, V, ldz);
+  count_launch();
+}
+
+// -------------------------------------------------------------------- AdamW
+// Hephaistos, Architecture at a glance (Optimizer); strata (AdamW, decoupled
+// and bias-corrected).  m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+// p -= lr wd p + lr (m/bc1) / (sqrt(v/bc2) + eps), bc = 1 - beta^t.
+// The flat buffers hold every tensor back to back, so one launch covers all.
+// Skipped entirely when the step's flag is non-zero.
+__global__ void k_adamw(float *__restrict__ p, const float *__restrict__ g, float *__restrict__ m,
+                        float *__restrict__ v, int64_t n, float lr, float wd, float b1, float b2,
+                        float eps, float bc1, float bc2, const int *flag) {
+  if (*flag) return;
+  int64_t n4 = n / 4;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 pp = reinterpret_cast<float4 *>(p)[i];
+    float4 gg = reinterpret_cast<const float4 *>(g)[i];
+    float4 mm = reinterpret_cast<float4 *>(m)[i];
+    float4 vv = reinterpret_cast<float4 *>(v)[i];
+#define ADAM1(c)                                                         \
+    mm.c = b1 * mm.c + (1.f - b1) * gg.c;                                \
+    vv.c = b2 * vv.c + (1.f - b2) * gg.c * gg.c;                         \
+    pp.c = pp.c - lr * wd * pp.c - lr * (mm.c / bc1) / (sqrtf(vv.c / bc2) + eps);
+    ADAM1(x) ADAM1(y) ADAM1(z) ADAM1(w)
+#undef ADAM1
+    reinterpret_cast<float4 *>(p)[i] = pp;
+    reinterpret_cast<float4 *>(m)[i] = mm;
+    reinterpret_cast<float4 *>(v)[i] = vv;
+  }
+  for (int64_t i = n4 * 4 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float gi = g[i];
+    float mi = b1 * m[i] + (1.f - b1) * gi;
+    float vi = b2 * v[i] + (1.f - b2) * gi * gi;
+    m[i] = mi;
+    v[i] = vi;
+    p[i] = p[i] - lr * wd * p[i] - lr * (mi / bc1) / (sqrtf(vi / bc2) + eps);
+  }
+}
+void adamw(float *p, const float *g, float *m, float *v, int64_t n, float lr, float wd, float b1,
+           float b2, float eps, float bc1, float bc2, const int *flag, cudaStream_t s) {
+  unsigned grid = min(cdiv(n / 4 + 1, 256), 148u * 8);
+  k_adamw<<<grid, 256, 0, s>>>(p, g, m, v, n, lr, wd, b1, b2, eps, bc1, bc2, flag);
+  count_launch();
+}
+
+// ------------------------------------------------------------ wgrad finish
+__global__ void k_wgrad_finish(const float *__restrict__ part, int splits, int64_t part_rows,
+                               int64_t ldp, float *__restrict__ grad, int64_t rows, int64_t cols,
+                               int mode, int64_t h) {
+  int64_t n = rows * cols;
+  int64_t pstride = part_rows * ldp;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t r = i / cols, c = i % cols, cp = c;
+    if (mode == 1) cp = (c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK;
+    const float *src = part + r * ldp + cp;
+    float s = 0.f;
+    for (int k = 0; k < splits; k++) s += src[k * pstride];
+    grad[i] = s;
+  }
+}
+void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp, float *grad,
+                  int64_t rows, int64_t cols, int mode, int64_t h, cudaStream_t s) {
+  unsigned grid = min(cdiv(rows * cols, 256), 148u * 16);
+  k_wgrad_finish<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode, h);
+  count_launch();
+}
+
+// ------------------------------------------------------- embedding backward
+// dwte[v,:] = sum_{i : tok_i = v} dx[i,:], summed in increasing i, so the
+// result does not depend on scheduling.  The token ids are sorted stably
+// (least-significant-digit radix sort, 8-bit digits) together with their
+// positions; then one block per vocabulary row adds its rows in order.
+constexpr int RADIX_BLOCK = 256;
+
+__global__ void k_radix_hist(const int32_t *__restrict__ keys, int64_t N, int shift,
+                             int32_t *__restrict__ hist, int nblk) {
+  __shared__ int cnt[256];
+  cnt[threadIdx.x] = 0;
+  __syncthreads();
+  int64_t i = (int64_t)blockIdx.x * RADIX_BLOCK + threadIdx.x;
+  if (i < N) atomicAdd(&cnt[(keys[i] >> shift) & 255], 1);
+  __syncthreads();
+  hist[(int64_t)threadIdx.x * nblk + blockIdx.x] = cnt[threadIdx.x];
+}
+// Exclusive scan of n ints in place (one block of 1024 threads).
+__global__ void k_scan_excl(int32_t *a, int64_t n) {
+  __shared__ int32_t sh[1024];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n; base += 1024) {
+    int64_t i = base + threadIdx.x;
+    int32_t v = (i < n) ? a[i] : 0;
+    sh[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      int32_t t = (threadIdx.x >= (unsigned)o) ? sh[threadIdx.x - o] : 0;
+      __syncthreads();
+      sh[threadIdx.x] += t;
+      __syncthreads();
+    }
+    if (i < n) a[i] = carry + sh[threadIdx.x] - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += sh[1023];
+    __syncthreads();
+  }
+}
+__global__ void k_radix_scatter(const int32_t *__restrict__ keys, const int32_t *__restrict__ vals,
+                                int64_t N, int shift, const int32_t *__restrict__ offs, int nblk,
+                                int32_t *__restrict__ keys_out, int32_t *__restrict__ vals_out) {
+  __shared__ int wcnt[RADIX_BLOCK / 32][256];
+  int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < (RADIX_BLOCK / 32) * 256; i += RADIX_BLOCK) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  int64_t i = (int64_t)blockIdx.x * RADIX_BLOCK + threadIdx.x;
+  bool valid = i < N;
+  int key = valid ? keys[i] : 0;
+  int dig = valid ? ((key >> shift) & 255) : 256 + lane;  // invalid lanes never match
+  unsigned peers = __match_any_sync(0xffffffffu, dig);
+  int rank = __popc(peers & ((1u << lane) - 1));
+  if (valid && rank == 0) wcnt[warp][dig] = __popc(peers);
+  __syncthreads();
+  if (valid) {
+    int before = 0;
+    for (int w = 0; w < warp; w++) before += wcnt[w][dig];
+    int pos = offs[(int64_t)dig * nblk + blockIdx.x] + before + rank;
+    keys_out[pos] = key;
+    vals_out[pos] = vals ? vals[i] : (int32_t)i;
+  }
+}
+__global__ void k_clamp_keys(const int32_t *__restrict__ tok, int32_t *__restrict__ keys,
+                             int32_t *__restrict__ counts, int64_t N, int V) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  int t = tok[i];
+  if (t < 0 || t >= V) t = 0;
+  keys[i] = t;
+  atomicAdd(&counts[t], 1);
+}
+__global__ void k_embed_rows(const int32_t *__restrict__ order, const int32_t *__restrict__ offs,
+                             const float *__restrict__ dx, float *__restrict__ dwte, int d) {
+  int v = blockIdx.x;
+  int b = offs[v], e = offs[v + 1];
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float s = 0.f;
+    for (int p = b; p < e; p++) s += dx[(int64_t)order[p] * d + j];
+    dwte[(int64_t)v * d + j] = s;
+  }
+}
+int64_t embed_bwd_scratch_ints(int64_t N, int V) {
+  int64_t nblk = (N + RADIX_BLOCK - 1) / RADIX_BLOCK;
+  return 4 * N + 256 * nblk + (V + 1) + 64;
+}
+void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int d, int V,
+               int32_t *scratch, cudaStream_t s) {
+  int nblk = (int)cdiv(N, RADIX_BLOCK);
+  int32_t *k0 = scratch, *v0 = k0 + N, *k1 = v0 + N, *v1 = k1 + N;
+  int32_t *hist = v1 + N, *offs = hist + 256 * (int64_t)nblk;
+  cudaMemsetAsync(offs, 0, sizeof(int32_t) * (V + 1), s);
+  k_clamp_keys<<<cdiv(N, 256), 256, 0, s>>>(tok, k0, offs, N, V);
+  count_launch();
+  int bits = 1;
+  while ((1 << bits) < V) bits++;
+  const int32_t *kin = k0, *vin = nullptr;
+  int32_t *kout = k1, *vout = v1;
+  for (int shift = 0; shift < bits; shift += 8) {
+    k_radix_hist<<<nblk, RADIX_BLOCK, 0, s>>>(kin, N, shift, hist, nblk);
+    k_scan_excl<<<1, 1024, 0, s>>>(hist, 256 * (int64_t)nblk);
+    k_radix_scatter<<<nblk, RADIX_BLOCK, 0, s>>>(kin, vin, N, shift, hist, nblk, kout, vout);
+    count_launch(3);
+    // ping-pong
+    const int32_t *nk = kout, *nv = vout;
+    kout = (kout == k1) ? k0 : k1;
+    vout = (vout == v1) ? v0 : v1;
+    kin = nk;
+    vin = nv;
+  }
+  k_scan_excl<<<1, 1024, 0, s>>>(offs, V + 1);
+  k_embed_rows<<<V, min(256, ((d + 31) / 32) * 32), 0, s>>>(vin, offs, dx, dwte, d);
+  count_launch(2);
+}
+
+// ------------------------------------------------------------ initialisation
+// Counter-based normal draws for llm_init: Philox4x32-10 (Salmon, Moraes,
+// Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011) keyed
+// by the seed, counter = element index; two 32-bit outputs give one normal by
+// the Box-Muller transform.
+LLM_DEV void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; r++) {
+    uint32_t hi0 = __umulhi(M0, c[0]), lo0 = M0 * c[0];
+    uint32_t hi1 = __umulhi(M1, c[2]), lo1 = M1 * c[2];
+    uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
+    k0 += W0; k1 += W1;
+  }
+}
+__global__ void k_init(float *__restrict__ p, int64_t n, uint32_t k0, uint32_t k1, uint64_t base,
+                       float std, int one) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (one) { p[i] = 1.f; continue; }
+    uint64_t ctr = base + (uint64_t)i;
+    uint32_t c[4] = {(uint32_t)ctr, (uint32_t)(ctr >> 32), 0u, 0u};
+    philox4x32_10(c, k0, k1);
+    double u1 = ((double)c[0] + 1.0) / 4294967296.0;  // (0, 1]
+    double u2 = (double)c[1] / 4294967296.0;          // [0, 1)
+    double z = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+    p[i] = (float)(z * std);
+  }
+}
+void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, float std,
+                 int constant_one, cudaStream_t s) {
+  unsigned grid = min(cdiv(n, 256), 148u * 8);
+  k_init<<<grid, 256, 0, s>>>(p, n, (uint32_t)seed, (uint32_t)(seed >> 32), counter_base, std,
+                              constant_one);
+  count_launch();
+}
+
+// -------------------------------------------------------------------- flags
+__global__ void k_or_flag(const int *src, int *dst) { if (*src) atomicOr(dst, *src); }
+void set_flag_zero(int *flag, cudaStream_t s) { cudaMemsetAsync(flag, 0, sizeof(int), s); }
+void or_flag(const int *src, int *dst, cudaStream_t s) {
+  k_or_flag<<<1, 1, 0, s>>>(src, dst);
+  count_launch();
+}
+
+}  // namespace llm

@@ -1,0 +1,485 @@
+// C ABI (include/llm.h) and host orchestration of one training step: the
+// parameter layout, the carving of the caller's workspace, and the launch
+// sequence forward -> cross-entropy -> backward -> AdamW on one stream.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "../../include/llm.h"
+#include "gemm_tc.h"
+#include "internal.h"
+
+using namespace llm;
+
+namespace {
+
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// Sizes derived from a config.  hp / Vp: hidden and vocabulary padded to the
+// tile multiples of the low-precision weight copies (pad weights are zero, so
+// pad activations are zero and pad gradients are discarded).
+struct Dims {
+  int V, d, L, H, Hkv, hd, kvd, h, T, B;
+  int64_t N, qkvw, hp, Vp, P, layer_sz;
+  DType dt;
+  int ab;  // bytes of one activation element
+};
+
+bool valid_config(const llm_config *c) {
+  if (!c) return false;
+  if (c->vocab < 1 || c->d_model < 4 || c->n_layer < 0 || c->n_head < 1 || c->n_kv_head < 1 ||
+      c->d_ff < 1 || c->ctx < 1 || c->batch < 1)
+    return false;
+  if (c->d_model % c->n_head) return false;
+  if (c->n_head % c->n_kv_head) return false;
+  int hd = c->d_model / c->n_head;
+  if (hd % 2 || hd > 128) return false;
+  if (c->d_model % 4 || c->d_model > 4096) return false;
+  if (c->compute != LLM_FP32 && c->compute != LLM_BF16) return false;
+  if (!(c->rms_eps >= 0.f) || !(c->rope_base > 0.f)) return false;
+  if ((int64_t)c->batch * c->ctx > (int64_t)1 << 30) return false;
+  return true;
+}
+
+Dims make_dims(const llm_config *c) {
+  Dims D;
+  D.V = c->vocab; D.d = c->d_model; D.L = c->n_layer; D.H = c->n_head; D.Hkv = c->n_kv_head;
+  D.hd = D.d / D.H; D.kvd = D.Hkv * D.hd; D.h = c->d_ff; D.T = c->ctx; D.B = c->batch;
+  D.N = (int64_t)D.B * D.T;
+  D.qkvw = D.d + 2LL * D.kvd;
+  D.hp = round_up(D.h, 64);
+  D.Vp = round_up(D.V, 128);
+  D.layer_sz = (int64_t)D.d + (int64_t)D.d * D.qkvw + (int64_t)D.d * D.d + D.d +
+               (int64_t)D.d * 2 * D.h + (int64_t)D.h * D.d;
+  D.P = (int64_t)D.V * D.d + D.L * D.layer_sz + D.d + (int64_t)D.d * D.V;
+  D.dt = c->compute == LLM_BF16 ? DT_BF16 : DT_F32;
+  D.ab = D.dt == DT_BF16 ? 2 : 4;
+  return D;
+}
+
+// Offsets of the flat parameter buffer (Hephaistos, Design notes).
+struct POff {
+  const Dims &D;
+  int64_t layer(int l) const { return (int64_t)D.V * D.d + l * D.layer_sz; }
+  int64_t g1(int l) const { return layer(l); }
+  int64_t wqkv(int l) const { return g1(l) + D.d; }
+  int64_t wo(int l) const { return wqkv(l) + (int64_t)D.d * D.qkvw; }
+  int64_t g2(int l) const { return wo(l) + (int64_t)D.d * D.d; }
+  int64_t w13(int l) const { return g2(l) + D.d; }
+  int64_t w2(int l) const { return w13(l) + (int64_t)D.d * 2 * D.h; }
+  int64_t gf() const { return layer(D.L); }
+  int64_t wlm() const { return gf() + D.d; }
+};
+
+// Split count of a weight-gradient GEMM (K = tokens): enough (tile, split)
+// pairs to fill the GPU twice, each split at least 512 tokens long.
+int wgrad_splits(const Dims &D, int64_t M, int64_t Ncols) {
+  int64_t tiles = ((M + 127) / 128) * ((Ncols + 127) / 128);
+  int64_t want = (2 * 148 + tiles - 1) / tiles;
+  int64_t maxs = std::max<int64_t>(1, D.N / 512);
+  return (int)std::max<int64_t>(1, std::min<int64_t>({want, maxs, 32}));
+}
+
+// Workspace carve: the same sequence of (size) requests both sizes and
+// places the buffers, so llm_workspace_bytes and llm_create agree.
+struct Carver {
+  char *base;
+  int64_t off = 0;
+  void *take(int64_t bytes) {
+    off = round_up(off, 256);
+    void *p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+}  // namespace
+
+struct llm_ctx {
+  llm_config cfg;
+  Dims D;
+  cudaStream_t s;
+  int last_launches = 0;
+  bool use_tc = false;
+  // device buffers (all inside the caller's workspace)
+  int *flag_step, *flag_sticky;
+  float *cos_t, *sin_t;
+  void *w_qkv, *w_o, *w_13, *w_2, *w_lm;  // low-precision copies, layer-strided
+  float *xs;                               // [L+1][N,d] residual stream
+  float *x1;                               // [L][N,d]
+  void *xn1, *qkv, *o, *xn2, *ab, *u;      // [L][...] saved activations
+  float *rstd1, *rstd2, *lse;              // [L][N], [L][N], [L][B,H,T]
+  void *xf, *logits;
+  float *rstdf, *rowloss;
+  float *dx, *dtmp, *Dbuf, *part, *dgpart;
+  void *dxA, *du, *dab, *dO, *dqkv;
+  int32_t *sort_scratch;
+  TcPlan *tc = nullptr;
+  int64_t carve(char *base);
+};
+
+int64_t llm_ctx::carve(char *base) {
+  const Dims &D_ = D;
+  Carver c{base};
+  int64_t N = D_.N, d = D_.d, L = D_.L, ab = D_.ab;
+  flag_step = (int *)c.take(64);
+  flag_sticky = (int *)c.take(64);
+  cos_t = (float *)c.take(4 * (int64_t)D_.T * (D_.hd / 2));
+  sin_t = (float *)c.take(4 * (int64_t)D_.T * (D_.hd / 2));
+  w_qkv = c.take(ab * L * d * D_.qkvw);
+  w_o = c.take(ab * L * d * d);
+  w_13 = c.take(ab * L * d * 2 * D_.hp);
+  w_2 = c.take(ab * L * D_.hp * d);
+  w_lm = c.take(ab * d * D_.Vp);
+  xs = (float *)c.take(4 * (L + 1) * N * d);
+  x1 = (float *)c.take(4 * L * N * d);
+  xn1 = c.take(ab * L * N * d);
+  qkv = c.take(ab * L * N * D_.qkvw);
+  o = c.take(ab * L * N * d);
+  xn2 = c.take(ab * L * N * d);
+  this->ab = c.take(ab * L * N * 2 * D_.hp);
+  u = c.take(ab * L * N * D_.hp);
+  rstd1 = (float *)c.take(4 * L * N);
+  rstd2 = (float *)c.take(4 * L * N);
+  lse = (float *)c.take(4 * L * N * D_.H);
+  xf = c.take(ab * N * d);
+  logits = c.take(ab * N * D_.Vp);
+  rstdf = (float *)c.take(4 * N);
+  rowloss = (float *)c.take(4 * N);
+  dx = (float *)c.take(4 * N * d);
+  dtmp = (float *)c.take(4 * N * d);
+  Dbuf = (float *)c.take(4 * N * D_.H);
+  dxA = c.take(ab * N * d);
+  du = c.take(ab * N * D_.hp);
+  dab = c.take(ab * N * 2 * D_.hp);
+  dO = c.take(ab * N * d);
+  dqkv = c.take(ab * N * D_.qkvw);
+  int64_t part_elems = 0;
+  auto need = [&](int64_t M, int64_t Nc) {
+    part_elems = std::max<int64_t>(part_elems, (int64_t)wgrad_splits(D_, M, Nc) * M * Nc);
+  };
+  need(d, D_.Vp); need(D_.hp, d); need(d, 2 * D_.hp); need(d, d); need(d, D_.qkvw);
+  part = (float *)c.take(4 * part_elems);
+  dgpart = (float *)c.take(4 * (int64_t)rmsnorm_bwd_blocks(N) * d);
+  sort_scratch = (int32_t *)c.take(4 * embed_bwd_scratch_ints(N, D_.V));
+  return round_up(c.off, 256);
+}
+
+// ------------------------------------------------------------- C ABI: host
+extern "C" {
+
+int llm_param_layout(const llm_config *cfg, llm_tensor_info *out, int *n_tensors,
+                     int64_t *n_params) {
+  if (!n_tensors || !n_params) return LLM_ERR_ARG;
+  if (!valid_config(cfg)) return LLM_ERR_CONFIG;
+  Dims D = make_dims(cfg);
+  POff O{D};
+  int cap = *n_tensors;
+  int n = 3 + 6 * D.L;
+  *n_tensors = n;
+  *n_params = D.P;
+  if (!out) return LLM_OK;
+  if (cap < n) return LLM_ERR_ARG;
+  int k = 0;
+  auto put = [&](const char *nm, int64_t off, int64_t r, int64_t c) {
+    memset(out[k].name, 0, sizeof(out[k].name));
+    strncpy(out[k].name, nm, sizeof(out[k].name) - 1);
+    out[k].offset = off; out[k].rows = r; out[k].cols = c;
+    k++;
+  };
+  char nm[32];
+  put("wte", 0, D.V, D.d);
+  for (int l = 0; l < D.L; l++) {
+    snprintf(nm, sizeof nm, "l%d.g1", l);   put(nm, O.g1(l), 1, D.d);
+    snprintf(nm, sizeof nm, "l%d.Wqkv", l); put(nm, O.wqkv(l), D.d, D.qkvw);
+    snprintf(nm, sizeof nm, "l%d.Wo", l);   put(nm, O.wo(l), D.d, D.d);
+    snprintf(nm, sizeof nm, "l%d.g2", l);   put(nm, O.g2(l), 1, D.d);
+    snprintf(nm, sizeof nm, "l%d.W13", l);  put(nm, O.w13(l), D.d, 2LL * D.h);
+    snprintf(nm, sizeof nm, "l%d.W2", l);   put(nm, O.w2(l), D.h, D.d);
+  }
+  put("gf", O.gf(), 1, D.d);
+  put("Wlm", O.wlm(), D.d, D.V);
+  return LLM_OK;
+}
+
+int llm_workspace_bytes(const llm_config *cfg, int64_t *bytes) {
+  if (!bytes) return LLM_ERR_ARG;
+  if (!valid_config(cfg)) return LLM_ERR_CONFIG;
+  llm_ctx tmp;
+  tmp.cfg = *cfg;
+  tmp.D = make_dims(cfg);
+  *bytes = tmp.carve(nullptr);
+  return LLM_OK;
+}
+
+int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void *cuda_stream,
+               llm_ctx **out) {
+  if (!out) return LLM_ERR_ARG;
+  *out = nullptr;
+  if (!valid_config(cfg)) return LLM_ERR_CONFIG;
+  if (!d_workspace || ((uintptr_t)d_workspace & 255)) return LLM_ERR_ARG;
+  llm_ctx *c = new (std::nothrow) llm_ctx();
+  if (!c) return LLM_ERR_ARG;
+  c->cfg = *cfg;
+  c->D = make_dims(cfg);
+  c->s = (cudaStream_t)cuda_stream;
+  int64_t need = c->carve(nullptr);
+  if (ws_bytes < need) { delete c; return LLM_ERR_ARG; }
+  c->carve((char *)d_workspace);
+  g_launches = 0;
+  cudaMemsetAsync(c->flag_step, 0, 64, c->s);
+  cudaMemsetAsync(c->flag_sticky, 0, 64, c->s);
+  rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, cfg->rope_base, c->s);
+  c->tc = tc_plan_create(c->D.dt, c->cos_t, c->sin_t, c->D.T, c->D.hd, c->D.d + c->D.kvd, c->D.hp);
+  if (cudaGetLastError() != cudaSuccess) { delete c; return LLM_ERR_CUDA; }
+  *out = c;
+  return LLM_OK;
+}
+
+void llm_destroy(llm_ctx *c) {
+  if (!c) return;
+  tc_plan_destroy(c->tc);
+  delete c;
+}
+
+const char *llm_error_string(int code) {
+  switch (code) {
+    case LLM_OK: return "ok";
+    case LLM_ERR_CONFIG: return "invalid configuration";
+    case LLM_ERR_ARG: return "invalid argument (null or misaligned pointer, small workspace)";
+    case LLM_ERR_TOKEN: return "token or target id outside [0, vocab)";
+    case LLM_ERR_NONFINITE: return "non-finite loss";
+    case LLM_ERR_CUDA: return "CUDA error";
+    case LLM_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    default: return "unknown error";
+  }
+}
+
+int llm_last_launch_count(const llm_ctx *c) { return c ? c->last_launches : 0; }
+
+int llm_status(llm_ctx *c) {
+  if (!c) return LLM_ERR_ARG;
+  if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+  int f = 0;
+  if (cudaMemcpy(&f, c->flag_sticky, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LLM_ERR_CUDA;
+  if (cudaMemset(c->flag_sticky, 0, sizeof(int)) != cudaSuccess) return LLM_ERR_CUDA;
+  if (f & FLAG_TIMEOUT) return LLM_ERR_TIMEOUT;
+  if (f & FLAG_TOKEN) return LLM_ERR_TOKEN;
+  if (f & FLAG_NONFINITE) return LLM_ERR_NONFINITE;
+  return LLM_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------- step orchestration
+namespace {
+
+bool aligned16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
+
+// C[M,N] = A . B^T with the operand conventions of GemmOperands; routes to
+// the tensor-core kernel when it covers the shape, else to the SIMT kernel.
+void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
+          int64_t ldr, int splits, int epi = 0, const void *aux = nullptr) {
+  if (c->tc && tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, aux, c->s)) return;
+  gemm_simt(g, out, C, ldc, R, ldr, splits, c->s);
+}
+
+// Forward pass; leaves logits (padded, activation type) in c->logits.
+void forward(llm_ctx *c, const float *p, const int32_t *tok) {
+  const Dims &D = c->D;
+  POff O{D};
+  cudaStream_t s = c->s;
+  const int64_t N = D.N, d = D.d;
+  const int ab = D.ab;
+  auto A = [&](void *base, int64_t l, int64_t per) { return (char *)base + l * per * ab; };
+  // low-precision (or float32) padded copies of the weight matrices
+  if (D.L > 0) {
+    cast_weight(p + O.wqkv(0), c->w_qkv, D.dt, d, D.qkvw, d, D.qkvw, 0, 0, 0, D.L, D.layer_sz,
+                d * D.qkvw, s);
+    cast_weight(p + O.wo(0), c->w_o, D.dt, d, d, d, d, 0, 0, 0, D.L, D.layer_sz, d * d, s);
+    cast_weight(p + O.w13(0), c->w_13, D.dt, d, 2LL * D.h, d, 2 * D.hp, 1, D.h, D.hp, D.L,
+                D.layer_sz, d * 2 * D.hp, s);
+    cast_weight(p + O.w2(0), c->w_2, D.dt, D.h, d, D.hp, d, 0, 0, 0, D.L, D.layer_sz, D.hp * d, s);
+  }
+  cast_weight(p + O.wlm(), c->w_lm, D.dt, d, D.V, d, D.Vp, 0, 0, 0, 1, 0, 0, s);
+  embed_fwd(p, tok, c->xs, N, D.d, D.V, c->flag_step, s);
+  for (int l = 0; l < D.L; l++) {
+    float *x = c->xs + l * N * d, *x1 = c->x1 + l * N * d, *x2 = c->xs + (l + 1) * N * d;
+    void *xn1 = A(c->xn1, l, N * d), *qkv = A(c->qkv, l, N * D.qkvw), *o = A(c->o, l, N * d);
+    void *xn2 = A(c->xn2, l, N * d), *abuf = A(c->ab, l, N * 2 * D.hp), *u = A(c->u, l, N * D.hp);
+    float *rstd1 = c->rstd1 + l * N, *rstd2 = c->rstd2 + l * N, *lse = c->lse + l * N * D.H;
+    void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
+    void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
+    // x1 = x + Attn(RMSNorm_g1(x))
+    rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
+    {
+      GemmOperands g{(int)N, (int)D.qkvw, D.d, xn1, d, true, wqkv, D.qkvw, false, D.dt};
+      bool fused = c->tc && tc_gemm(c->tc, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
+                                    nullptr, s);
+      if (!fused) {
+        gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
+        rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
+      }
+    }
+    attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
+    gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d, x,
+         d, 1);
+    // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
+    rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
+    {
+      GemmOperands g{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt};
+      bool fused = c->tc && tc_gemm(c->tc, g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1,
+                                    TC_EPI_SWIGLU, u, s);
+      if (!fused) {
+        gemm_simt(g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, s);
+        swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
+      }
+    }
+    gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_ADD_F32,
+         x2, d, x1, d, 1);
+  }
+  float *xL = c->xs + D.L * N * d;
+  rmsnorm_fwd(xL, p + O.gf(), c->xf, D.dt, c->rstdf, N, D.d, c->cfg.rms_eps, s);
+  gemm(c, GemmOperands{(int)N, (int)D.Vp, D.d, c->xf, d, true, c->w_lm, D.Vp, false, D.dt},
+       OUT_ACT, c->logits, D.Vp, nullptr, 0, 1);
+}
+
+// Weight gradient dW[M, Ncols] = X^T dY (K = tokens), written to the unpadded
+// gradient tensor through the partial buffer (fixed-order split reduction).
+void wgrad(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, int64_t M,
+           int64_t Ncols, float *grad, int64_t rows, int64_t cols, int mode) {
+  const Dims &D = c->D;
+  int splits = wgrad_splits(D, M, Ncols);
+  GemmOperands g{(int)M, (int)Ncols, (int)D.N, X, ldx, false, dY, ldy, false, D.dt};
+  gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits);
+  wgrad_finish(c->part, splits, M, Ncols, grad, rows, cols, mode, D.h, c->s);
+}
+
+void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
+  const Dims &D = c->D;
+  POff O{D};
+  cudaStream_t s = c->s;
+  const int64_t N = D.N, d = D.d;
+  const int ab = D.ab;
+  const bool lp = D.dt == DT_BF16;
+  auto A = [&](void *base, int64_t l, int64_t per) { return (char *)base + l * per * ab; };
+  void *dxop = lp ? c->dxA : (void *)c->dx;  // dx as a GEMM operand
+  void *dxact = lp ? c->dxA : nullptr;
+  int nb;
+  // lm_head: dxf = dz Wlm^T; dWlm = xf^T dz
+  gemm(c, GemmOperands{(int)N, D.d, (int)D.Vp, c->logits, D.Vp, true, c->w_lm, D.Vp, true, D.dt},
+       OUT_F32, c->dtmp, d, nullptr, 0, 1);
+  wgrad(c, c->xf, d, c->logits, D.Vp, d, D.Vp, gr + O.wlm(), d, D.V, 0);
+  float *xL = c->xs + D.L * N * d;
+  nb = rmsnorm_bwd(xL, c->rstdf, p + O.gf(), c->dtmp, nullptr, c->dx, dxact, D.dt, c->dgpart, N,
+                   D.d, s);
+  reduce_partials(c->dgpart, nb, D.d, gr + O.gf(), s);
+  for (int l = D.L - 1; l >= 0; l--) {
+    float *x = c->xs + l * N * d, *x1 = c->x1 + l * N * d;
+    void *xn1 = A(c->xn1, l, N * d), *qkv = A(c->qkv, l, N * D.qkvw), *o = A(c->o, l, N * d);
+    void *xn2 = A(c->xn2, l, N * d), *abuf = A(c->ab, l, N * 2 * D.hp), *u = A(c->u, l, N * D.hp);
+    float *rstd1 = c->rstd1 + l * N, *rstd2 = c->rstd2 + l * N, *lse = c->lse + l * N * D.H;
+    void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
+    void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
+    // FFN branch.  du = dx2 W2^T, then SwiGLU backward into dab.
+    {
+      GemmOperands g{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt};
+      bool fused = c->tc && tc_gemm(c->tc, g, OUT_ACT, c->dab, 2 * D.hp, nullptr, 0, 1,
+                                    TC_EPI_SWIGLU_BWD, abuf, s);
+      if (!fused) {
+        gemm_simt(g, OUT_ACT, c->du, D.hp, nullptr, 0, 1, s);
+        swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
+      }
+    }
+    wgrad(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
+    gemm(c, GemmOperands{(int)N, D.d, (int)(2 * D.hp), c->dab, 2 * D.hp, true, w13, 2 * D.hp,
+                         true, D.dt},
+         OUT_F32, c->dtmp, d, nullptr, 0, 1);
+    wgrad(c, xn2, d, c->dab, 2 * D.hp, d, 2 * D.hp, gr + O.w13(l), d, 2LL * D.h, 1);
+    nb = rmsnorm_bwd(x1, rstd2, p + O.g2(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
+                     D.d, s);
+    reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
+    // attention branch
+    gemm(c, GemmOperands{(int)N, D.d, D.d, dxop, d, true, wo, d, true, D.dt}, OUT_ACT, c->dO, d,
+         nullptr, 0, 1);
+    wgrad(c, o, d, dxop, d, d, d, gr + O.wo(l), d, d, 0);
+    attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
+                  s);
+    rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);
+    gemm(c, GemmOperands{(int)N, D.d, (int)D.qkvw, c->dqkv, D.qkvw, true, wqkv, D.qkvw, true,
+                         D.dt},
+         OUT_F32, c->dtmp, d, nullptr, 0, 1);
+    wgrad(c, xn1, d, c->dqkv, D.qkvw, d, D.qkvw, gr + O.wqkv(l), d, D.qkvw, 0);
+    nb = rmsnorm_bwd(x, rstd1, p + O.g1(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N, D.d,
+                     s);
+    reduce_partials(c->dgpart, nb, D.d, gr + O.g1(l), s);
+  }
+  embed_bwd(tok, c->dx, gr, N, D.d, D.V, c->sort_scratch, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int llm_forward(llm_ctx *c, const float *d_params, const int32_t *d_tokens, float *d_logits) {
+  if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;
+  g_launches = 0;
+  set_flag_zero(c->flag_step, c->s);
+  forward(c, d_params, d_tokens);
+  logits_out(c->logits, c->D.dt, d_logits, c->D.N, c->D.V, c->D.Vp, c->s);
+  or_flag(c->flag_step, c->flag_sticky, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,
+             const int32_t *d_tokens, const int32_t *d_targets, float lr, float wd,
+             float *d_loss) {
+  if (!c || !d_tokens || !d_targets || !d_loss || t < 1) return LLM_ERR_ARG;
+  if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
+    return LLM_ERR_ARG;
+  const Dims &D = c->D;
+  g_launches = 0;
+  set_flag_zero(c->flag_step, c->s);
+  forward(c, d_params, d_tokens);
+  cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
+                c->flag_step, c->s);
+  loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
+  backward(c, d_params, d_grads, d_tokens);
+  double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
+  double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
+  adamw(d_params, d_grads, d_m, d_v, D.P, lr, wd, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps,
+        (float)bc1, (float)bc2, c->flag_step, c->s);
+  or_flag(c->flag_step, c->flag_sticky, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_init(llm_ctx *c, uint64_t seed, float init_std, int scale_out_proj, float *d_params) {
+  if (!c || !d_params || !(init_std >= 0.f)) return LLM_ERR_ARG;
+  const Dims &D = c->D;
+  POff O{D};
+  g_launches = 0;
+  float so = scale_out_proj ? init_std / sqrtf(2.0f * (float)std::max(1, D.L)) : init_std;
+  auto mat = [&](int64_t off, int64_t n, float sd) { init_params(d_params + off, n, seed, off, sd, 0, c->s); };
+  auto one = [&](int64_t off, int64_t n) { init_params(d_params + off, n, seed, off, 0.f, 1, c->s); };
+  mat(0, (int64_t)D.V * D.d, init_std);
+  for (int l = 0; l < D.L; l++) {
+    one(O.g1(l), D.d);
+    mat(O.wqkv(l), (int64_t)D.d * D.qkvw, init_std);
+    mat(O.wo(l), (int64_t)D.d * D.d, so);
+    one(O.g2(l), D.d);
+    mat(O.w13(l), (int64_t)D.d * 2 * D.h, init_std);
+    mat(O.w2(l), (int64_t)D.h * D.d, so);
+  }
+  one(O.gf(), D.d);
+  mat(O.wlm(), (int64_t)D.d * D.V, init_std);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+}  // extern "C"

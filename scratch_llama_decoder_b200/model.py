@@ -1,0 +1,78 @@
+"""LlamaStep: a context of the C ABI bound to torch device memory and stream.
+
+Argument marshalling only: torch tensors are passed to the library by device
+pointer; every step of the computation runs in the library's kernels.
+"""
+import ctypes as C
+
+import torch
+
+from . import _lib as L
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else None
+
+
+class LlamaStep:
+    """Owns the workspace (a torch uint8 tensor) and the llm_ctx for one config.
+
+    cfg: mapping with the llm_config field names (vocab, d_model, n_layer,
+    n_head, n_kv_head, d_ff, ctx, batch, rope_base, rms_eps, beta1, beta2,
+    adam_eps, compute)."""
+
+    def __init__(self, cfg, device="cuda", stream=None):
+        if not torch.cuda.is_available():
+            raise RuntimeError("LlamaStep needs a CUDA device (B200, sm_100a); no CPU fallback")
+        self.cfg = dict(cfg)
+        self.device = torch.device(device)
+        self.layout, self.n_params = L.llm_param_layout(cfg)
+        self.ws_bytes = L.llm_workspace_bytes(cfg)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        self.stream = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self._c = L.make_config(cfg)
+        ctx = C.c_void_p()
+        L.check(L.lib.llm_create(C.byref(self._c), _ptr(self.workspace), self.ws_bytes,
+                                 C.c_void_p(self.stream.cuda_stream), C.byref(ctx)), "llm_create")
+        self.ctx = ctx
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            L.lib.llm_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -------------------------------------------------------------- buffers
+    def new_params(self):
+        return torch.zeros(self.n_params, dtype=torch.float32, device=self.device)
+
+    def init(self, params, seed, init_std, scale_out_proj):
+        L.check(L.lib.llm_init(self.ctx, seed, float(init_std), int(bool(scale_out_proj)),
+                               _ptr(params)), "llm_init")
+
+    def forward(self, params, tokens, logits=None):
+        B, T, V = self.cfg["batch"], self.cfg["ctx"], self.cfg["vocab"]
+        if logits is None:
+            logits = torch.empty(B, T, V, dtype=torch.float32, device=self.device)
+        L.check(L.lib.llm_forward(self.ctx, _ptr(params), _ptr(tokens), _ptr(logits)),
+                "llm_forward")
+        return logits
+
+    def step(self, params, grads, m, v, t, tokens, targets, lr, wd, loss=None):
+        if loss is None:
+            loss = torch.empty(1, dtype=torch.float32, device=self.device)
+        L.check(L.lib.llm_step(self.ctx, _ptr(params), _ptr(grads), _ptr(m), _ptr(v), int(t),
+                               _ptr(tokens), _ptr(targets), float(lr), float(wd), _ptr(loss)),
+                "llm_step")
+        return loss
+
+    def status(self):
+        return L.lib.llm_status(self.ctx)
+
+    def last_launch_count(self):
+        return L.lib.llm_last_launch_count(self.ctx)

@@ -1,0 +1,93 @@
+"""Helpers of the GPU parity tests: run the CUDA path through the C ABI and
+compare with the float64 oracle using norm-wise relative error per tensor."""
+import numpy as np
+import torch
+
+# Tolerances of the training step (norm-wise relative error per tensor).
+#   fp32 configs: loss and logits 1e-4; gradients, updated parameters and the
+#   Adam moments 1e-3.
+#   bf16 configs: loss 5e-3; logits, gradients and m 2e-2; v = (1-b2) g^2
+#   carries twice the relative error of g, so v gets 4e-2.
+TOL = {
+    "fp32": dict(loss=1e-4, logits=1e-4, grads=1e-3, params=1e-3, m=1e-3, v=1e-3, dp=1e-3),
+    "bf16": dict(loss=5e-3, logits=2e-2, grads=2e-2, params=2e-2, m=2e-2, v=4e-2, dp=None),
+}
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    nb = np.linalg.norm(b)
+    if nb == 0.0:
+        return float(np.linalg.norm(a))
+    return float(np.linalg.norm(a - b) / nb)
+
+
+def run_gpu(cfg, params, tok, tgt, steps=1, lr=None, wd=None):
+    """Returns dict with logits (pre-step forward), and per step: loss, grads,
+    params, m, v (numpy float64)."""
+    from scratch_llama_decoder_b200 import LlamaStep
+    lr = cfg["lr"] if lr is None else lr
+    wd = cfg["wd"] if wd is None else wd
+    m = LlamaStep(cfg)
+    P = torch.tensor(params, dtype=torch.float32, device="cuda")
+    G = torch.zeros_like(P)
+    M = torch.zeros_like(P)
+    V = torch.zeros_like(P)
+    td = torch.tensor(tok, dtype=torch.int32, device="cuda").contiguous()
+    yd = torch.tensor(tgt, dtype=torch.int32, device="cuda").contiguous()
+    logits = m.forward(P, td)
+    out = {"logits": logits.double().cpu().numpy().reshape(-1, cfg["vocab"]), "steps": []}
+    assert m.status() == 0
+    for t in range(1, steps + 1):
+        loss = m.step(P, G, M, V, t, td, yd, lr, wd)
+        st = m.status()
+        out["steps"].append(dict(status=st, loss=float(loss.item()),
+                                 grads=G.double().cpu().numpy(), params=P.double().cpu().numpy(),
+                                 m=M.double().cpu().numpy(), v=V.double().cpu().numpy()))
+    out["launches"] = m.last_launch_count()
+    m.close()
+    return out
+
+
+def run_oracle(cfg, params, tok, tgt, steps=1, lr=None, wd=None):
+    import oracle as O
+    lr = cfg["lr"] if lr is None else lr
+    wd = cfg["wd"] if wd is None else wd
+    p = np.asarray(params, np.float64)
+    m = np.zeros_like(p)
+    v = np.zeros_like(p)
+    _, logits, _ = O.forward_backward(cfg, p, tok, tgt, want_grads=False)
+    out = {"logits": logits, "steps": []}
+    for t in range(1, steps + 1):
+        loss, _, g = O.forward_backward(cfg, p, tok, tgt, want_logits=False)
+        p, m, v = O.adamw(p, g, m, v, t, lr, wd, cfg["beta1"], cfg["beta2"], cfg["adam_eps"])
+        out["steps"].append(dict(loss=loss, grads=g, params=p.copy(), m=m.copy(), v=v.copy()))
+    return out
+
+
+def compare(cfg, layout, gpu, ref, prev_params=None, tol=None):
+    """Asserts every gate; returns a dict of the worst errors."""
+    tol = tol or TOL[cfg["compute"]]
+    worst = {"logits": rel(gpu["logits"], ref["logits"])}
+    assert worst["logits"] <= tol["logits"], worst
+    p_prev = prev_params
+    for k, (g, r) in enumerate(zip(gpu["steps"], ref["steps"])):
+        assert g["status"] == 0, g["status"]
+        le = abs(g["loss"] - r["loss"]) / abs(r["loss"])
+        worst["loss"] = max(worst.get("loss", 0.0), le)
+        assert le <= tol["loss"], (k, g["loss"], r["loss"])
+        for key in ("grads", "params", "m", "v"):
+            for name, off, rows, cols in layout:
+                sl = slice(off, off + rows * cols)
+                e = rel(g[key][sl], r[key][sl])
+                worst[key] = max(worst.get(key, 0.0), e)
+                assert e <= tol[key], (k, key, name, e)
+        if tol.get("dp") is not None and p_prev is not None:
+            for name, off, rows, cols in layout:
+                sl = slice(off, off + rows * cols)
+                e = rel(g["params"][sl] - p_prev[sl], r["params"][sl] - p_prev[sl])
+                worst["dp"] = max(worst.get("dp", 0.0), e)
+                assert e <= tol["dp"], (k, "dp", name, e)
+        p_prev = r["params"]
+    return worst

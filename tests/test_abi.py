@@ -1,0 +1,86 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no compute calls).
+
+The library must load, export every function include/llm.h declares, agree
+with the oracle on the flat parameter layout, and reject invalid configs and
+arguments on the host.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import oracle as O
+from synth import CONFIGS, get_config
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared(header):
+    src = open(os.path.join(ROOT, "include", header)).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(llm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    import scratch_llama_decoder_b200 as P
+    headers = [h for h in os.listdir(os.path.join(ROOT, "include")) if h.endswith(".h")]
+    names = [n for h in headers for n in _declared(h)]
+    assert "llm_step" in names and "llm_forward" in names and "llm_init" in names
+    for n in names:
+        assert hasattr(P.lib, n), n  # ctypes resolves the symbol via dlsym
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_layout_matches_oracle(name):
+    from scratch_llama_decoder_b200 import llm_param_layout, llm_workspace_bytes
+    cfg = get_config(name)
+    lay, n = llm_param_layout(cfg)
+    assert lay == O.param_layout(cfg)
+    assert n == O.n_params(cfg)
+    assert llm_workspace_bytes(cfg) > 0
+
+
+def test_gqa_layout_matches_oracle():
+    from scratch_llama_decoder_b200 import llm_param_layout
+    cfg = get_config("c4", n_layer=3)
+    lay, n = llm_param_layout(cfg)
+    assert lay == O.param_layout(cfg) and n == O.n_params(cfg)
+
+
+@pytest.mark.parametrize("bad", [dict(d_model=18, n_head=4), dict(n_head=4, n_kv_head=3),
+                                 dict(d_model=12, n_head=4), dict(vocab=0), dict(compute=7),
+                                 dict(batch=0)])
+def test_invalid_config_rejected(bad):
+    import scratch_llama_decoder_b200 as P
+    cfg = get_config("c1", **bad)
+    c = P.make_config(cfg)
+    b = C.c_int64(0)
+    assert P.lib.llm_workspace_bytes(C.byref(c), C.byref(b)) == P.LLM_ERR_CONFIG
+    n, npar = C.c_int(0), C.c_int64(0)
+    assert P.lib.llm_param_layout(C.byref(c), None, C.byref(n), C.byref(npar)) == P.LLM_ERR_CONFIG
+    ctx = C.c_void_p()
+    assert P.lib.llm_create(C.byref(c), C.c_void_p(256), 1 << 30, None, C.byref(ctx)) == \
+        P.LLM_ERR_CONFIG
+
+
+def test_bad_arguments_rejected_on_host():
+    import scratch_llama_decoder_b200 as P
+    c = P.make_config(get_config("c1"))
+    ctx = C.c_void_p()
+    # null / misaligned workspace, too-small workspace: rejected before any launch
+    assert P.lib.llm_create(C.byref(c), None, 1 << 20, None, C.byref(ctx)) == P.LLM_ERR_ARG
+    assert P.lib.llm_create(C.byref(c), C.c_void_p(0x1001), 1 << 20, None, C.byref(ctx)) == \
+        P.LLM_ERR_ARG
+    assert P.lib.llm_create(C.byref(c), C.c_void_p(0x10000), 16, None, C.byref(ctx)) == \
+        P.LLM_ERR_ARG
+    # layout with too small an output array
+    n, npar = C.c_int(1), C.c_int64(0)
+    arr = (P._lib.llm_tensor_info * 1)()
+    assert P.lib.llm_param_layout(C.byref(c), arr, C.byref(n), C.byref(npar)) == P.LLM_ERR_ARG
+    assert P.lib.llm_step(None, None, None, None, None, 1, None, None, 0.0, 0.0, None) == \
+        P.LLM_ERR_ARG
+    assert P.lib.llm_forward(None, None, None, None) == P.LLM_ERR_ARG
+    assert P.lib.llm_status(None) == P.LLM_ERR_ARG
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert P.lib.llm_error_string(code)
