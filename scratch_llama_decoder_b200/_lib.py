@@ -48,6 +48,9 @@ EXPORTS = {
     "llm_status": (_i, [_vp]),
     "llm_error_string": (C.c_char_p, [_i]),
     "llm_last_launch_count": (_i, [_vp]),
+    # include/llm_kernels.h
+    "llm_kernel_gemm_bf16": (_i, [_i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp,
+                                  _vp]),
 }
 for _name, (_res, _args) in EXPORTS.items():
     _fn = getattr(lib, _name)

@@ -1,20 +1,628 @@
-// tcgen05 GEMM (placeholder: no shapes covered yet; the SIMT kernels run).
+// tcgen05 GEMM for sm_100a: C[M,N] = A[M,K] . B[N,K]^T, bf16 operands, fp32
+// accumulation in tensor memory (TMEM).
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: A and B tiles into a STAGES-deep shared-memory
+//               ring (128-byte swizzle), completion counted on mbarriers;
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               (M=128, N=256, K=16) and commits each stage back to the ring;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row per thread), fused epilogue, stores to global.
+// Two accumulators of 256 columns alternate so the epilogue of one tile
+// overlaps the main loop of the next.  Operands may be K-major or MN-major
+// (both supported by the UMMA descriptors), which covers the forward
+// (x W), data-gradient (dy W^T) and weight-gradient (x^T dy) orientations
+// without transposed copies.  Every mbarrier wait is bounded; on time-out the
+// kernel records FLAG_TIMEOUT, drains its own copies and MMAs, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <unordered_map>
+
+#include "common.cuh"
 #include "gemm_tc.h"
 
 namespace llm {
 
-struct TcPlan {
-  int unused;
+namespace tc {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_BYTES = BN * BK * 2;            // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int TMEM_COLS = 512;
+constexpr int NTHREADS = 192;
+constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on any wait
+
+struct Args {
+  int M, N, K;
+  int tiles_m, tiles_n, splits, kchunk, total;
+  int out, epi;
+  void *C;
+  int64_t ldc;
+  const float *R;
+  int64_t ldr;
+  const void *aux;  // SWIGLU: u output [M, hp]; SWIGLU_BWD: saved ab [M, 2hp]
+  int64_t ld_aux;
+  const float *cos_t, *sin_t;
+  int T, hd, rot_cols;
+  int *flag;
 };
 
-TcPlan *tc_plan_create(DType, const float *, const float *, int, int, int64_t, int64_t) {
-  return nullptr;
+// ------------------------------------------------------------ PTX helpers
+LLM_DEV uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+LLM_DEV unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
+LLM_DEV void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+LLM_DEV bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on the phase of `parity`; false (and FLAG_TIMEOUT) on time-out
+// or when another role of this CTA already gave up.
+LLM_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *gflag) {
+  if (mbar_try(bar, parity)) return true;
+  unsigned long long t0 = gtimer();
+  for (uint32_t it = 1;; it++) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 255) == 0) {
+      if (*abort_flag) return false;
+      if (gtimer() - t0 > WAIT_NS) {
+        *abort_flag = 1;
+        atomicOr(gflag, FLAG_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+LLM_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+LLM_DEV void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+LLM_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+LLM_DEV void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+LLM_DEV void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (UMMA): start address, leading/stride byte
+// offsets (16-byte units), descriptor version 1, 128-byte swizzle (mode 2).
+LLM_DEV uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B,
+// per-operand major-ness, N>>3 and M>>4.
+__host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+LLM_DEV void mma_bf16(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(ad), "l"(bd), "r"(id), "r"(acc)
+      : "memory");
+}
+LLM_DEV void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+LLM_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------ epilogue stores
+LLM_DEV void store32_f32(float *dst, const float (&v)[32], int nvalid) {
+  if (nvalid >= 32) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+      *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  } else {
+    for (int i = 0; i < nvalid; i++) dst[i] = v[i];
+  }
+}
+LLM_DEV uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+LLM_DEV void store32_bf16(__nv_bfloat16 *dst, const float (&v)[32], int nvalid) {
+  if (nvalid >= 32) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      uint4 q = make_uint4(pack_bf16(v[i], v[i + 1]), pack_bf16(v[i + 2], v[i + 3]),
+                           pack_bf16(v[i + 4], v[i + 5]), pack_bf16(v[i + 6], v[i + 7]));
+      *reinterpret_cast<uint4 *>(dst + i) = q;
+    }
+  } else {
+    for (int i = 0; i < nvalid; i++) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+LLM_DEV void load32_bf16(const __nv_bfloat16 *src, float (&v)[32], int nvalid) {
+  if (nvalid >= 32) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      uint4 q = *reinterpret_cast<const uint4 *>(src + i);
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&q);
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        float2 f = __bfloat1622float2(h[k]);
+        v[i + 2 * k] = f.x;
+        v[i + 2 * k + 1] = f.y;
+      }
+    }
+  } else {
+    for (int i = 0; i < 32; i++) v[i] = (i < nvalid) ? __bfloat162float(src[i]) : 0.f;
+  }
+}
+
+// One output tile's epilogue for the thread owning row m (TMEM lane).
+// tm: TMEM address of this lane's accumulator row at column 0.
+// All 32 lanes of the warp execute every tcgen05.ld (warp-uniform control);
+// rows past M only skip their global loads and stores.
+LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split, bool zero) {
+  const bool row_ok = m < a.M;
+  const int N = a.N;
+  auto nval = [&](int n) { return row_ok ? min(32, N - n) : 0; };
+  float v[32];
+  if (a.epi == TC_EPI_ROPE) {
+    // RoPE on q/k heads (columns < rot_cols), plain store of v heads.
+    const int hd = a.hd, half = hd / 2, t = m % a.T;
+    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)m * a.ldc;
+    if (hd == 64) {
+      for (int c0 = 0; c0 < BN; c0 += 64) {
+        int n = n0 + c0;
+        if (n >= N) break;
+        float lo[32], hi[32];
+        if (zero) { for (int i = 0; i < 32; i++) lo[i] = hi[i] = 0.f; }
+        else { tmem_ld32(tm + c0, lo); tmem_ld32(tm + c0 + 32, hi); }
+        if (n < a.rot_cols) {
+          const float *ct = a.cos_t + (int64_t)t * half, *st = a.sin_t + (int64_t)t * half;
+#pragma unroll
+          for (int j = 0; j < 32; j++) {
+            float c = ct[j], s = st[j], x = lo[j], y = hi[j];
+            lo[j] = x * c - y * s;
+            hi[j] = y * c + x * s;
+          }
+        }
+        store32_bf16(C + n, lo, nval(n));
+        store32_bf16(C + n + 32, hi, nval(n + 32));
+      }
+    } else {  // hd == 32: both halves of a head sit in one 32-column chunk
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        int n = n0 + c0;
+        if (n >= N) break;
+        if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
+        else tmem_ld32(tm + c0, v);
+        if (n < a.rot_cols) {
+          const float *ct = a.cos_t + (int64_t)t * half, *st = a.sin_t + (int64_t)t * half;
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            float c = ct[j], s = st[j], x = v[j], y = v[j + 16];
+            v[j] = x * c - y * s;
+            v[j + 16] = y * c + x * s;
+          }
+        }
+        store32_bf16(C + n, v, nval(n));
+      }
+    }
+    return;
+  }
+  if (a.epi == TC_EPI_SWIGLU) {
+    // Interleaved [a|b] blocks of 64+64 columns: store a, b and u = silu(a) b.
+    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)m * a.ldc;
+    __nv_bfloat16 *U = (__nv_bfloat16 *)a.aux + (int64_t)m * a.ld_aux;
+    for (int blk = 0; blk < BN; blk += 2 * SWIGLU_BLOCK) {
+      int n = n0 + blk;
+      if (n >= N) break;
+      for (int q = 0; q < SWIGLU_BLOCK; q += 32) {
+        float av[32], bv[32];
+        if (zero) { for (int i = 0; i < 32; i++) av[i] = bv[i] = 0.f; }
+        else { tmem_ld32(tm + blk + q, av); tmem_ld32(tm + blk + SWIGLU_BLOCK + q, bv); }
+        int nv = row_ok ? 32 : 0;
+        store32_bf16(C + n + q, av, nv);
+        store32_bf16(C + n + SWIGLU_BLOCK + q, bv, nv);
+#pragma unroll
+        for (int i = 0; i < 32; i++) av[i] = av[i] / (1.f + expf(-av[i])) * bv[i];
+        store32_bf16(U + (n / (2 * SWIGLU_BLOCK)) * SWIGLU_BLOCK + q, av, nv);
+      }
+    }
+    return;
+  }
+  if (a.epi == TC_EPI_SWIGLU_BWD) {
+    // acc = du for hidden units [n0, n0+BN); write [da|db] at their
+    // interleaved columns using the saved [a|b].
+    const __nv_bfloat16 *AB = (const __nv_bfloat16 *)a.aux + (int64_t)m * a.ld_aux;
+    __nv_bfloat16 *D = (__nv_bfloat16 *)a.C + (int64_t)m * a.ldc;
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      int j = n0 + c0;
+      if (j >= N) break;
+      if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
+      else tmem_ld32(tm + c0, v);
+      int64_t ca = w1_col(j);
+      int nv = row_ok ? 32 : 0;
+      float av[32], bv[32];
+      load32_bf16(AB + ca, av, nv);
+      load32_bf16(AB + ca + SWIGLU_BLOCK, bv, nv);
+#pragma unroll
+      for (int i = 0; i < 32; i++) {
+        float s = 1.f / (1.f + expf(-av[i]));
+        float du = v[i];
+        float da = du * bv[i] * s * (1.f + av[i] * (1.f - s));
+        bv[i] = du * av[i] * s;
+        av[i] = da;
+      }
+      store32_bf16(D + ca, av, nv);
+      store32_bf16(D + ca + SWIGLU_BLOCK, bv, nv);
+    }
+    return;
+  }
+  // Plain outputs.
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    int n = n0 + c0;
+    if (n >= N) break;
+    int nv = nval(n);
+    if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
+    else tmem_ld32(tm + c0, v);
+    if (a.out == OUT_F32) {
+      store32_f32((float *)a.C + (int64_t)m * a.ldc + n, v, nv);
+    } else if (a.out == OUT_ACT) {
+      store32_bf16((__nv_bfloat16 *)a.C + (int64_t)m * a.ldc + n, v, nv);
+    } else if (a.out == OUT_ADD_F32) {
+      const float *r = a.R + (int64_t)m * a.ldr + n;
+      if (nv >= 32) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float4 q = *reinterpret_cast<const float4 *>(r + i);
+          v[i] += q.x; v[i + 1] += q.y; v[i + 2] += q.z; v[i + 3] += q.w;
+        }
+      } else {
+        for (int i = 0; i < nv; i++) v[i] += r[i];
+      }
+      store32_f32((float *)a.C + (int64_t)m * a.ldc + n, v, nv);
+    } else {  // OUT_PARTIAL
+      store32_f32((float *)a.C + (int64_t)split * a.M * a.ldc + (int64_t)m * a.ldc + n, v, nv);
+    }
+  }
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = (uint64_t *)(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * STAGES;
+  const uint32_t tfull0 = empty0 + 8 * STAGES, tempty0 = tfull0 + 16, drain = tempty0 + 16;
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base_sh)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int tiles_mn = a.tiles_m * a.tiles_n;
+  const int kblocks_total = (a.K + BK - 1) / BK;
+
+  auto kblocks_of = [&](int split, int &kb0) {
+    int kb_per = a.kchunk / BK;
+    kb0 = split * kb_per;
+    int kb1 = min(kblocks_total, kb0 + kb_per);
+    return max(0, kb1 - kb0);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued_parity[STAGES];
+      bool issued[STAGES];
+      for (int i = 0; i < STAGES; i++) issued[i] = false;
+      bool ok = true;
+      for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
+        int split = w / tiles_mn, tile = w % tiles_mn;
+        int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
+        int kb0, nkb = kblocks_of(split, kb0);
+        for (int kb = 0; kb < nkb; kb++) {
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) { ok = false; break; }
+          uint32_t fb = full0 + 8 * s;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
+          int k0 = (kb0 + kb) * BK;
+          if (A_MN) {
+            tma_load_2d(sa, &tmA, m0, k0, fb);
+            tma_load_2d(sa + 8192, &tmA, m0 + 64, k0, fb);
+          } else {
+            tma_load_2d(sa, &tmA, k0, m0, fb);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < 4; j++) tma_load_2d(sb + 8192 * j, &tmB, n0 + 64 * j, k0, fb);
+          } else {
+            tma_load_2d(sb, &tmB, k0, n0, fb);
+          }
+          issued[s] = true;
+          issued_parity[s] = ph;
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      // Our copies must have landed before the CTA exits (normally they were
+      // consumed already; after an abort they may still be in flight).
+      for (int i = 0; i < STAGES; i++)
+        if (issued[i]) {
+          unsigned long long t0 = gtimer();
+          while (!mbar_try(full0 + 8 * i, issued_parity[i]) && gtimer() - t0 < WAIT_NS) {
+          }
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t ID = idesc(A_MN, B_MN);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
+        int split = w / tiles_mn;
+        int kb0, nkb = kblocks_of(split, kb0);
+        if (nkb == 0) continue;  // epilogue writes zeros without waiting
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1, &abort_sh, a.flag)) break;
+        fence_after();
+        uint32_t td = tmem + acc * BN;
+        for (int kb = 0; kb < nkb; kb++) {
+          if (!mbar_wait(full0 + 8 * s, ph, &abort_sh, a.flag)) { ok = false; break; }
+          fence_after();
+          uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
+          uint64_t ad = A_MN ? sdesc(sa, 8192, 1024) : sdesc(sa, 16, 1024);
+          uint64_t bd = B_MN ? sdesc(sb, 8192, 1024) : sdesc(sb, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; kk++) {
+            // advance 16 K elements: 32 bytes inside a K-major swizzle row, or
+            // 16 rows (2048 bytes) of an MN-major tile; >>4 for the descriptor
+            uint64_t da = (uint64_t)(A_MN ? kk * 128 : kk * 2);
+            uint64_t db = (uint64_t)(B_MN ? kk * 128 : kk * 2);
+            mma_bf16(td, ad + da, bd + db, ID, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(empty0 + 8 * s);  // frees the stage when these MMAs finish
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(tfull0 + 8 * acc);  // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; aph ^= 1; }
+      }
+      // drain: every MMA this thread issued has completed
+      mma_commit(drain);
+      unsigned long long t0 = gtimer();
+      while (!mbar_try(drain, 0) && gtimer() - t0 < WAIT_NS) {
+      }
+    }
+  } else {
+    // -------------------------------------------------- epilogue warps
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
+      int split = w / tiles_mn, tile = w % tiles_mn;
+      int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
+      int kb0, nkb = kblocks_of(split, kb0);
+      int m = m0 + quarter * 32 + lane;
+      if (nkb == 0) {
+        epilogue_tile(a, 0, m, n0, split, true);
+        continue;
+      }
+      int got = 0;
+      if (lane == 0) got = mbar_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      fence_after();
+      uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
+      epilogue_tile(a, tm, m, n0, split, false);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; aph ^= 1; }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------ host side
+struct TcPlan {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  int num_sms = 148;
+  const float *cos_t, *sin_t;
+  int T, hd;
+  int64_t rot_cols, hp;
+  int *flag = nullptr;  // device flag word for time-outs (set by the owner)
+  std::mutex mu;
+  struct Key {
+    const void *p;
+    uint64_t d0, d1, s1;
+    uint32_t b0, b1;
+    bool operator==(const Key &o) const {
+      return p == o.p && d0 == o.d0 && d1 == o.d1 && s1 == o.s1 && b0 == o.b0 && b1 == o.b1;
+    }
+  };
+  struct KeyHash {
+    size_t operator()(const Key &k) const {
+      return std::hash<const void *>()(k.p) ^ (k.d0 * 1315423911u) ^ (k.d1 * 2654435761u) ^
+             (k.s1 << 7) ^ ((uint64_t)k.b0 << 20) ^ ((uint64_t)k.b1 << 40);
+    }
+  };
+  std::unordered_map<Key, CUtensorMap, KeyHash> maps;
+
+  // 2-D bf16 tensor map: inner dim d0 (contiguous), outer d1 with row
+  // stride s1 elements; box b0 x b1; 128-byte swizzle; zero fill outside.
+  bool map(const void *p, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0, uint32_t b1,
+           CUtensorMap *out) {
+    Key k{p, d0, d1, s1, b0, b1};
+    std::lock_guard<std::mutex> g(mu);
+    auto it = maps.find(k);
+    if (it != maps.end()) { *out = it->second; return true; }
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {s1 * 2};
+    cuuint32_t box[2] = {b0, b1};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(p), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    maps.emplace(k, *out);
+    return true;
+  }
+};
+
+TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, int hd,
+                       int64_t rot_cols, int64_t hp) {
+  if (dt != DT_BF16) return nullptr;
+  int dev = 0, major = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major != 10) return nullptr;
+  TcPlan *p = new TcPlan();
+  cudaDriverEntryPointQueryResult q;
+  void *fn = nullptr;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                       &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn) {
+    delete p;
+    return nullptr;
+  }
+  p->encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  p->cos_t = cos_t; p->sin_t = sin_t; p->T = T; p->hd = hd; p->rot_cols = rot_cols; p->hp = hp;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(tc::k_gemm_tc<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+    cudaFuncSetAttribute(tc::k_gemm_tc<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+    cudaFuncSetAttribute(tc::k_gemm_tc<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+    cudaFuncSetAttribute(tc::k_gemm_tc<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+    attr_done = true;
+  }
+  return p;
+}
+
+void tc_plan_set_flag(TcPlan *p, int *flag) {
+  if (p) p->flag = flag;
+}
+
 void tc_plan_destroy(TcPlan *p) { delete p; }
-bool tc_gemm(TcPlan *, const GemmOperands &, GemmOut, void *, int64_t, const float *, int64_t, int,
-             int, const void *, cudaStream_t) {
-  return false;
+
+static bool al16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+
+bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
+             int64_t ldr, int splits, int epi, const void *aux, cudaStream_t s) {
+  using namespace tc;
+  if (!p || g.in != DT_BF16 || !p->flag) return false;
+  if (g.M < 1 || g.N < 1 || g.K < 1) return false;
+  if (!al16(g.A) || !al16(g.B) || !al16(C) || (g.lda * 2) % 16 || (g.ldb * 2) % 16) return false;
+  if (out == OUT_ACT ? (ldc % 8) : (ldc % 4)) return false;
+  if (out == OUT_ADD_F32 && (!R || !al16(R) || ldr % 4)) return false;
+  if (epi == TC_EPI_ROPE && !(p->hd == 32 || p->hd == 64)) return false;
+  if ((epi == TC_EPI_SWIGLU || epi == TC_EPI_SWIGLU_BWD) && (g.N % 64 || !aux || !al16(aux)))
+    return false;
+  if (epi != TC_EPI_NONE && out != OUT_ACT) return false;
+  // tensor maps: A as [rows][K] (K-major) or [K][M] (MN-major); same for B
+  CUtensorMap ta, tb;
+  bool ok = g.a_kmajor ? p->map(g.A, g.K, g.M, g.lda, 64, BM, &ta)
+                       : p->map(g.A, g.M, g.K, g.lda, 64, 64, &ta);
+  ok = ok && (g.b_kmajor ? p->map(g.B, g.K, g.N, g.ldb, 64, BN, &tb)
+                         : p->map(g.B, g.N, g.K, g.ldb, 64, 64, &tb));
+  if (!ok) return false;
+  Args a{};
+  a.M = g.M; a.N = g.N; a.K = g.K;
+  a.tiles_m = (g.M + BM - 1) / BM;
+  a.tiles_n = (g.N + BN - 1) / BN;
+  if (out != OUT_PARTIAL) splits = 1;
+  a.splits = max(1, splits);
+  int kc = (g.K + a.splits - 1) / a.splits;
+  a.kchunk = ((kc + BK - 1) / BK) * BK;
+  a.total = a.tiles_m * a.tiles_n * a.splits;
+  a.out = out; a.epi = epi; a.C = C; a.ldc = ldc; a.R = R; a.ldr = ldr;
+  a.aux = aux;
+  a.ld_aux = (epi == TC_EPI_SWIGLU) ? p->hp : 2 * p->hp;
+  a.cos_t = p->cos_t; a.sin_t = p->sin_t; a.T = p->T; a.hd = p->hd; a.rot_cols = (int)p->rot_cols;
+  a.flag = p->flag;
+  int grid = min(a.total, p->num_sms);
+  bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
+  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
+  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
+  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
+  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
+  count_launch();
+  return true;
 }
+
 void attention_fwd(TcPlan *, const void *qkv, void *o, float *lse, DType dt, int B, int T, int H,
                    int Hkv, int hd, cudaStream_t s) {
   attn_fwd_simt(qkv, o, lse, dt, B, T, H, Hkv, hd, s);

@@ -19,6 +19,8 @@ enum TcEpi {
 TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, int hd,
                        int64_t rot_cols, int64_t hp);
 void tc_plan_destroy(TcPlan *p);
+// Device flag word that records a bounded wait giving up (FLAG_TIMEOUT).
+void tc_plan_set_flag(TcPlan *p, int *flag);
 bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
              int64_t ldr, int splits, int epi, const void *aux, cudaStream_t s);
 

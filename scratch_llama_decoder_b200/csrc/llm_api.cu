@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "../../include/llm.h"
@@ -234,6 +235,7 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
   cudaMemsetAsync(c->flag_sticky, 0, 64, c->s);
   rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, cfg->rope_base, c->s);
   c->tc = tc_plan_create(c->D.dt, c->cos_t, c->sin_t, c->D.T, c->D.hd, c->D.d + c->D.kvd, c->D.hp);
+  tc_plan_set_flag(c->tc, c->flag_step);
   if (cudaGetLastError() != cudaSuccess) { delete c; return LLM_ERR_CUDA; }
   *out = c;
   return LLM_OK;
@@ -483,3 +485,29 @@ int llm_init(llm_ctx *c, uint64_t seed, float init_std, int scale_out_proj, floa
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------- single-kernel entries
+#include "../../include/llm_kernels.h"
+
+extern "C" int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_t lda,
+                                    int a_kmajor, const void *d_B, int64_t ldb, int b_kmajor,
+                                    float *d_C, int64_t ldc, int tensor_cores, int *d_flag,
+                                    void *stream) {
+  if (M < 1 || N < 1 || K < 1 || !d_A || !d_B || !d_C || !d_flag) return LLM_ERR_ARG;
+  if (lda < (a_kmajor ? K : M) || ldb < (b_kmajor ? K : N) || ldc < N) return LLM_ERR_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  GemmOperands g{M, N, K, d_A, lda, a_kmajor != 0, d_B, ldb, b_kmajor != 0, DT_BF16};
+  g_launches = 0;
+  if (tensor_cores) {
+    static TcPlan *plan = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] { plan = tc_plan_create(DT_BF16, nullptr, nullptr, 1, 64, 0, 64); });
+    if (!plan) return LLM_ERR_ARG;
+    tc_plan_set_flag(plan, d_flag);
+    if (!tc_gemm(plan, g, OUT_F32, d_C, ldc, nullptr, 0, 1, TC_EPI_NONE, nullptr, s))
+      return LLM_ERR_ARG;
+  } else {
+    gemm_simt(g, OUT_F32, d_C, ldc, nullptr, 0, 1, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}

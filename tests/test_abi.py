@@ -29,6 +29,30 @@ def test_library_exports_every_declared_symbol():
     assert "llm_step" in names and "llm_forward" in names and "llm_init" in names
     for n in names:
         assert hasattr(P.lib, n), n  # ctypes resolves the symbol via dlsym
+        # every entry point has declared argument types: int64_t sizes must
+        # never be passed as 32-bit ints
+        assert n in P._lib.EXPORTS, n
+
+
+def test_binding_argtypes_match_header_arity():
+    import scratch_llama_decoder_b200 as P
+    src = ""
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src += re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", h)).read(),
+                          flags=re.S)
+    for name, (_, args) in P._lib.EXPORTS.items():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", src)
+        assert m, name
+        params = [a for a in m.group(1).split(",") if a.strip() and a.strip() != "void"]
+        assert len(params) == len(args), (name, len(params), len(args))
+        for decl, ct in zip(params, args):
+            if "*" in decl:
+                continue
+            if re.search(r"\buint64_t\b", decl):
+                assert ct is P._lib._u64, (name, decl)
+            elif re.search(r"\bint64_t\b", decl):
+                assert ct is P._lib._i64, (name, decl)
 
 
 @pytest.mark.parametrize("name", sorted(CONFIGS))

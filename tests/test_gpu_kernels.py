@@ -1,0 +1,55 @@
+"""GPU parity of single hot-path kernels (C ABI, include/llm_kernels.h)
+against the float64 oracle's per-operation functions."""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+# (M, N, K): tile multiples, ragged tails in every dimension, the step's shapes
+SHAPES = [(128, 256, 64), (200, 300, 136), (1, 8, 8), (640, 768, 512), (384, 1408, 1024),
+          (256, 2048, 16384 // 8)]
+
+
+def _bf16(rng, shape):
+    x = torch.tensor(rng.standard_normal(shape), dtype=torch.float32).to(torch.bfloat16)
+    return x
+
+
+@pytest.mark.parametrize("a_k,b_k", [(1, 0), (1, 1), (0, 0), (0, 1)])
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("tc", [1, 0])
+def test_gemm_bf16(M, N, K, a_k, b_k, tc):
+    import scratch_llama_decoder_b200 as P
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    # operand storage: K-major A is [M,K]; MN-major A is [K,M]; same for B with N
+    A = _bf16(rng, (M, K) if a_k else (K, M))
+    B = _bf16(rng, (N, K) if b_k else (K, N))
+    lda = A.shape[1]
+    ldb = B.shape[1]
+    if tc and (lda % 8 or ldb % 8):
+        pytest.skip("tensor-core path needs leading dimensions that are multiples of 8")
+    Ad, Bd = A.cuda().contiguous(), B.cuda().contiguous()
+    ldc = (N + 3) // 4 * 4
+    Cd = torch.full((M, ldc), float("nan"), device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = P.lib.llm_kernel_gemm_bf16(M, N, K, C.c_void_p(Ad.data_ptr()), lda, a_k,
+                                    C.c_void_p(Bd.data_ptr()), ldb, b_k,
+                                    C.c_void_p(Cd.data_ptr()), ldc, tc,
+                                    C.c_void_p(flag.data_ptr()), None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    got = Cd[:, :N].double().cpu().numpy()
+    a64 = A.float().double().numpy()
+    b64 = B.float().double().numpy()
+    am = a64 if a_k else a64.T  # [M, K]
+    bm = b64 if b_k else b64.T  # [N, K]
+    ref = O.mm_nt(am, bm)
+    err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    # bf16 products are exact in fp32; only fp32 summation rounding remains
+    assert err < 1e-5, err
