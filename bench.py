@@ -1,0 +1,355 @@
+#!/usr/bin/env python
+"""Throughput of the Llama training step (forward + backward + AdamW) on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Default workload: the ~350M-parameter decoder (vocab 32000, d_model 1024, 20
+layers, 16 heads, SwiGLU 2730, context 2048, batch 8 = 16384 tokens per step),
+bf16 compute with fp32 master weights, synthetic Zipf(1.1) tokens.  Prints one
+JSON line on rank 0.
+
+Our arm: W untimed steps, then K steps timed with CUDA events on the
+library's stream, bracketed by a barrier and a synchronize, max over ranks.
+With N > 1 GPUs every rank runs an independent replica on its own batch
+(weak scaling; no gradient exchange is part of the timed step).
+The roofline object is for the dominant kernel (the tcgen05 GEMM): its
+algorithmic FLOPs over the summed device time of its launches, both taken
+inside the timed region.  e2e repeats the timed loop through the same C ABI
+with the step's tokens and targets copied from pinned host memory each step
+and the loss read back each step.  cpu_baseline times the float64 CPU oracle
+on a bounded sample of the same workload.
+
+Reference arm (--impl reference): the float64 CPU oracle, each step a fixed
+fraction of the workload (a token prefix of one sequence, forward and
+backward, plus AdamW over the same fraction of the parameters), scaled to
+tokens/s of the full step; rank 0 only.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "training tokens/sec (fwd+bwd+AdamW) on 1 B200; % of tensor/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="c5")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_flops(cfg):
+    """Algorithmic FLOPs of one step: 6 * matmul params * tokens plus causal
+    attention (QK^T and PV, forward and twice in backward)."""
+    V, d, L, H, Hkv, h, T, B = (cfg[k] for k in ("vocab", "d_model", "n_layer", "n_head",
+                                                 "n_kv_head", "d_ff", "ctx", "batch"))
+    hd = d // H
+    kvd = Hkv * hd
+    M = L * (d * (d + 2 * kvd) + d * d + 3 * d * h) + d * V
+    N = B * T
+    attn = 12 * L * B * H * (T * (T + 1) / 2) * hd
+    return 6.0 * M * N + attn, attn
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = open(os.devnull if False else f"/tmp/clocks_{os.getpid()}.csv", "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.out.name):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------- oracle leg
+def oracle_sample_rate(cfg, tokens, reps=1, warmup=0):
+    """Tokens/s of the float64 oracle on a fraction f = tokens / (B*T) of the
+    step: forward + backward of the first `tokens` positions of one sequence,
+    plus AdamW over the same fraction of the parameters.  Returns
+    (tokens/s, seconds per sample, cores)."""
+    import numpy as np
+    import oracle as O
+    from synth import make_batch
+    c = dict(cfg, batch=1, ctx=min(cfg["ctx"], tokens))
+    S = c["ctx"]
+    lay = O.param_layout(c)
+    rng = np.random.default_rng(5)
+    n = O.n_params(c)
+    p = rng.standard_normal(n) * cfg["init_std"]
+    for name, off, r, k in lay:
+        if name.split(".")[-1] in ("g1", "g2", "gf"):
+            p[off:off + r * k] = 1.0
+    tok, tgt = make_batch(c, seed=11)
+    frac = S / float(cfg["batch"] * cfg["ctx"])
+    n_adam = max(1, int(n * frac))
+    g = rng.standard_normal(n_adam) * 1e-3
+    m = np.zeros(n_adam)
+    v = np.zeros(n_adam)
+    times = []
+    for it in range(warmup + reps):
+        t0 = time.perf_counter()
+        O.forward_backward(c, p, tok, tgt, want_logits=False)
+        O.adamw(p[:n_adam], g, m, v, 1, cfg["lr"], cfg["wd"])
+        dt = time.perf_counter() - t0
+        if it >= warmup:
+            times.append(dt)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    t = statistics.median(times)
+    return S / t, t, cores, S
+
+
+def sample_tokens_for(cfg, budget_s):
+    """Prefix length whose oracle sample takes about budget_s seconds (probed
+    on a 16-token prefix, assuming linear cost in tokens)."""
+    _, t16, _, _ = oracle_sample_rate(cfg, 16)
+    per_tok = t16 / 16.0
+    S = int(max(16, min(cfg["ctx"], budget_s / max(per_tok, 1e-9))))
+    return S
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from scratch_llama_decoder_b200 import LlamaStep
+    from synth import get_config, make_batch, make_params
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = get_config(args.config)
+    model = LlamaStep(cfg, device=dev)
+    stream = model.stream
+    p_host = make_params(cfg, model.layout, seed=1001 + cfg["index"] + 7919 * rank)
+    tok_h, tgt_h = make_batch(cfg, seed=1000 + cfg["index"] + 7919 * rank)
+    P = torch.tensor(p_host, device=dev)
+    G = torch.zeros_like(P)
+    Mo = torch.zeros_like(P)
+    Vo = torch.zeros_like(P)
+    tok = torch.tensor(tok_h, device=dev)
+    tgt = torch.tensor(tgt_h, device=dev)
+    loss = torch.zeros(1, device=dev)
+    lr, wd = cfg["lr"], cfg["wd"]
+    N = cfg["batch"] * cfg["ctx"]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+    st = model.status()
+    assert st == 0, f"warm-up step failed with status {st}"
+    launches_per_step = model.last_launch_count()
+    model.read_kernel_timing()  # clear
+    model.set_kernel_timing(True)
+
+    clocks = Clocks(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        t += 1
+        model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    g_ms, g_flops, g_launch = model.read_kernel_timing()
+    model.set_kernel_timing(False)
+    st = model.status()
+    assert st == 0, f"timed step failed with status {st}"
+    final_loss = float(loss.item())
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # ---- e2e: same API, host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        tok_pin = torch.tensor(tok_h).pin_memory()
+        tgt_pin = torch.tensor(tgt_h).pin_memory()
+        loss_pin = torch.zeros(1).pin_memory()
+        barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for _ in range(args.steps):
+                t += 1
+                tok.copy_(tok_pin, non_blocking=True)
+                tgt.copy_(tgt_pin, non_blocking=True)
+                model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+                loss_pin.copy_(loss, non_blocking=True)
+                stream.synchronize()
+            f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = f0.elapsed_time(f1)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": N * args.steps * world / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(tok_pin.numel() * 4 + tgt_pin.numel() * 4),
+               "d2h_bytes_per_step": 4}
+
+    if rank != 0:
+        return None
+    pk, src = peaks()
+    F, F_attn = step_flops(cfg)
+    step_s = ms / 1e3 / args.steps
+    value = N * args.steps * world / (ms / 1e3)
+    peak_tc = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    achieved = (g_flops / (g_ms / 1e3)) / 1e12 if g_ms > 0 else 0.0
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+        if cfg["compute"] == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": cfg["name"], "tokens_per_step": N, "batch": cfg["batch"],
+                   "seq_len": cfg["ctx"], "parallelism": f"replicas x{world}" if world > 1
+                   else "single GPU", "l2": "inputs larger than L2 (saved activations of "
+                   "several GB per step; no flush)"},
+        "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM (all projection GEMMs of the "
+                     "step)", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tc if peak_tc else None, "traffic": None,
+                     "launches": g_launch, "ms_total": g_ms,
+                     "peak_source": f"{src} bf16_tflops_sustained"},
+        "step_roofline": {"flops": F, "attention_flops": F_attn,
+                          "t_tensor_ms": F / (peak_tc * 1e12) * 1e3,
+                          "frac_of_tensor_bound": (F / (peak_tc * 1e12)) / step_s},
+        "gpu_launches": launches_per_step * args.steps,
+        "loss": final_loss,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        S = sample_tokens_for(cfg, 12.0)
+        rate, tsec, cores, S = oracle_sample_rate(cfg, S)
+        out["cpu_baseline"] = {
+            "value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"float64 oracle: forward+backward of a {S}-token prefix of one "
+                      f"sequence plus AdamW over {S}/{N} of the parameters "
+                      f"({tsec:.1f} s), scaled to tokens/s"}
+    return out
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    from synth import get_config
+    cfg = get_config(args.config)
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    S = sample_tokens_for(cfg, budget)
+    rate, tsec, cores, S = oracle_sample_rate(cfg, S, reps=args.steps, warmup=args.warmup)
+    N = cfg["batch"] * cfg["ctx"]
+    return {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tsec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": cfg["name"], "tokens_per_step": N, "batch": cfg["batch"],
+                   "seq_len": cfg["ctx"], "parallelism": "host CPU"},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: forward+backward of a {S}-token prefix of one "
+                                   f"sequence plus AdamW over {S}/{N} of the parameters"},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -140,6 +140,17 @@ const char *llm_error_string(int code);
 /* Number of kernels the most recent llm_step / llm_forward call enqueued. */
 int llm_last_launch_count(const llm_ctx *ctx);
 
+/* Measurement hooks (strata, bench harness: time what is claimed).  With
+ * timing enabled, every tensor-core GEMM launch of later calls is bracketed
+ * by CUDA events on the context's stream.  llm_read_kernel_timing()
+ * synchronises that stream and returns, since the previous read, the summed
+ * device time of those launches in milliseconds, their algorithmic FLOPs
+ * (2*M*N*K with unpadded sizes) and their count, then resets the sums.
+ * Events are created on demand (two per pending launch) and kept until
+ * llm_destroy(); reading after every few steps bounds their number. */
+int llm_set_kernel_timing(llm_ctx *ctx, int enable);
+int llm_read_kernel_timing(llm_ctx *ctx, double *ms, double *flops, int64_t *launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,6 +48,9 @@ EXPORTS = {
     "llm_status": (_i, [_vp]),
     "llm_error_string": (C.c_char_p, [_i]),
     "llm_last_launch_count": (_i, [_vp]),
+    "llm_set_kernel_timing": (_i, [_vp, _i]),
+    "llm_read_kernel_timing": (_i, [_vp, C.POINTER(C.c_double), C.POINTER(C.c_double),
+                                    C.POINTER(_i64)]),
     # include/llm_kernels.h
     "llm_kernel_gemm_bf16": (_i, [_i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp,
                                   _vp]),

@@ -119,6 +119,12 @@ struct llm_ctx {
   void *dxA, *du, *dab, *dO, *dqkv;
   int32_t *sort_scratch;
   TcPlan *tc = nullptr;
+  // optional event timing of the tensor-core GEMM launches
+  bool timing = false;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
+  double pending_flops = 0.0;
+  int64_t pending_launches = 0;
   int64_t carve(char *base);
 };
 
@@ -243,6 +249,7 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
 
 void llm_destroy(llm_ctx *c) {
   if (!c) return;
+  for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   tc_plan_destroy(c->tc);
   delete c;
 }
@@ -261,6 +268,31 @@ const char *llm_error_string(int code) {
 }
 
 int llm_last_launch_count(const llm_ctx *c) { return c ? c->last_launches : 0; }
+
+int llm_set_kernel_timing(llm_ctx *c, int enable) {
+  if (!c) return LLM_ERR_ARG;
+  c->timing = enable != 0;
+  return LLM_OK;
+}
+
+int llm_read_kernel_timing(llm_ctx *c, double *ms, double *flops, int64_t *launches) {
+  if (!c || !ms || !flops || !launches) return LLM_ERR_ARG;
+  if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+  double total = 0.0;
+  for (size_t i = 0; i + 1 < c->ev_used; i += 2) {
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, c->ev_pool[i], c->ev_pool[i + 1]) != cudaSuccess)
+      return LLM_ERR_CUDA;
+    total += t;
+  }
+  *ms = total;
+  *flops = c->pending_flops;
+  *launches = c->pending_launches;
+  c->ev_used = 0;
+  c->pending_flops = 0.0;
+  c->pending_launches = 0;
+  return LLM_OK;
+}
 
 int llm_status(llm_ctx *c) {
   if (!c) return LLM_ERR_ARG;
@@ -282,11 +314,41 @@ namespace {
 
 bool aligned16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
 
+// Tensor-core GEMM launch; when timing is on, bracketed by CUDA events on the
+// context's stream and credited with its algorithmic FLOPs (unpadded sizes).
+bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
+            int64_t ldr, int splits, int epi, const void *aux, double alg_flops) {
+  if (!c->tc) return false;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (c->timing) {
+    while (c->ev_pool.size() < c->ev_used + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) break;
+      c->ev_pool.push_back(e);
+    }
+    if (c->ev_pool.size() >= c->ev_used + 2) {
+      e0 = c->ev_pool[c->ev_used];
+      e1 = c->ev_pool[c->ev_used + 1];
+      cudaEventRecord(e0, c->s);
+    }
+  }
+  bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, aux, c->s);
+  if (e0) {
+    cudaEventRecord(e1, c->s);
+    if (ok) {
+      c->ev_used += 2;
+      c->pending_flops += alg_flops;
+      c->pending_launches += 1;
+    }
+  }
+  return ok;
+}
+
 // C[M,N] = A . B^T with the operand conventions of GemmOperands; routes to
 // the tensor-core kernel when it covers the shape, else to the SIMT kernel.
 void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-          int64_t ldr, int splits, int epi = 0, const void *aux = nullptr) {
-  if (c->tc && tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, aux, c->s)) return;
+          int64_t ldr, int splits, double alg_flops) {
+  if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, nullptr, alg_flops)) return;
   gemm_simt(g, out, C, ldc, R, ldr, splits, c->s);
 }
 
@@ -320,8 +382,8 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
     rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
     {
       GemmOperands g{(int)N, (int)D.qkvw, D.d, xn1, d, true, wqkv, D.qkvw, false, D.dt};
-      bool fused = c->tc && tc_gemm(c->tc, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
-                                    nullptr, s);
+      bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE, nullptr,
+                          2.0 * N * d * D.qkvw);
       if (!fused) {
         gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
         rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
@@ -329,25 +391,25 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
     }
     attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
     gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d, x,
-         d, 1);
+         d, 1, 2.0 * N * d * d);
     // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
     rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
     {
       GemmOperands g{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt};
-      bool fused = c->tc && tc_gemm(c->tc, g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1,
-                                    TC_EPI_SWIGLU, u, s);
+      bool fused = run_tc(c, g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, TC_EPI_SWIGLU, u,
+                          2.0 * N * d * 2 * D.h);
       if (!fused) {
         gemm_simt(g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, s);
         swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
       }
     }
     gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_ADD_F32,
-         x2, d, x1, d, 1);
+         x2, d, x1, d, 1, 2.0 * N * D.h * d);
   }
   float *xL = c->xs + D.L * N * d;
   rmsnorm_fwd(xL, p + O.gf(), c->xf, D.dt, c->rstdf, N, D.d, c->cfg.rms_eps, s);
   gemm(c, GemmOperands{(int)N, (int)D.Vp, D.d, c->xf, d, true, c->w_lm, D.Vp, false, D.dt},
-       OUT_ACT, c->logits, D.Vp, nullptr, 0, 1);
+       OUT_ACT, c->logits, D.Vp, nullptr, 0, 1, 2.0 * N * d * D.V);
 }
 
 // Weight gradient dW[M, Ncols] = X^T dY (K = tokens), written to the unpadded
@@ -357,7 +419,7 @@ void wgrad(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, 
   const Dims &D = c->D;
   int splits = wgrad_splits(D, M, Ncols);
   GemmOperands g{(int)M, (int)Ncols, (int)D.N, X, ldx, false, dY, ldy, false, D.dt};
-  gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits);
+  gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits, 2.0 * rows * cols * D.N);
   wgrad_finish(c->part, splits, M, Ncols, grad, rows, cols, mode, D.h, c->s);
 }
 
@@ -374,7 +436,7 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
   int nb;
   // lm_head: dxf = dz Wlm^T; dWlm = xf^T dz
   gemm(c, GemmOperands{(int)N, D.d, (int)D.Vp, c->logits, D.Vp, true, c->w_lm, D.Vp, true, D.dt},
-       OUT_F32, c->dtmp, d, nullptr, 0, 1);
+       OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.V * d);
   wgrad(c, c->xf, d, c->logits, D.Vp, d, D.Vp, gr + O.wlm(), d, D.V, 0);
   float *xL = c->xs + D.L * N * d;
   nb = rmsnorm_bwd(xL, c->rstdf, p + O.gf(), c->dtmp, nullptr, c->dx, dxact, D.dt, c->dgpart, N,
@@ -390,8 +452,8 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
     // FFN branch.  du = dx2 W2^T, then SwiGLU backward into dab.
     {
       GemmOperands g{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt};
-      bool fused = c->tc && tc_gemm(c->tc, g, OUT_ACT, c->dab, 2 * D.hp, nullptr, 0, 1,
-                                    TC_EPI_SWIGLU_BWD, abuf, s);
+      bool fused = run_tc(c, g, OUT_ACT, c->dab, 2 * D.hp, nullptr, 0, 1, TC_EPI_SWIGLU_BWD,
+                          abuf, 2.0 * N * d * D.h);
       if (!fused) {
         gemm_simt(g, OUT_ACT, c->du, D.hp, nullptr, 0, 1, s);
         swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
@@ -400,21 +462,21 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
     wgrad(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
     gemm(c, GemmOperands{(int)N, D.d, (int)(2 * D.hp), c->dab, 2 * D.hp, true, w13, 2 * D.hp,
                          true, D.dt},
-         OUT_F32, c->dtmp, d, nullptr, 0, 1);
+         OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * 2 * D.h * d);
     wgrad(c, xn2, d, c->dab, 2 * D.hp, d, 2 * D.hp, gr + O.w13(l), d, 2LL * D.h, 1);
     nb = rmsnorm_bwd(x1, rstd2, p + O.g2(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
                      D.d, s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
     // attention branch
     gemm(c, GemmOperands{(int)N, D.d, D.d, dxop, d, true, wo, d, true, D.dt}, OUT_ACT, c->dO, d,
-         nullptr, 0, 1);
+         nullptr, 0, 1, 2.0 * N * d * d);
     wgrad(c, o, d, dxop, d, d, d, gr + O.wo(l), d, d, 0);
     attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
                   s);
     rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);
     gemm(c, GemmOperands{(int)N, D.d, (int)D.qkvw, c->dqkv, D.qkvw, true, wqkv, D.qkvw, true,
                          D.dt},
-         OUT_F32, c->dtmp, d, nullptr, 0, 1);
+         OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.qkvw * d);
     wgrad(c, xn1, d, c->dqkv, D.qkvw, d, D.qkvw, gr + O.wqkv(l), d, D.qkvw, 0);
     nb = rmsnorm_bwd(x, rstd1, p + O.g1(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N, D.d,
                      s);

@@ -76,3 +76,13 @@ class LlamaStep:
 
     def last_launch_count(self):
         return L.lib.llm_last_launch_count(self.ctx)
+
+    def set_kernel_timing(self, enable):
+        L.check(L.lib.llm_set_kernel_timing(self.ctx, int(bool(enable))), "llm_set_kernel_timing")
+
+    def read_kernel_timing(self):
+        """(device ms, algorithmic FLOPs, launches) of the timed GEMM launches."""
+        ms, fl, n = C.c_double(0), C.c_double(0), C.c_int64(0)
+        L.check(L.lib.llm_read_kernel_timing(self.ctx, C.byref(ms), C.byref(fl), C.byref(n)),
+                "llm_read_kernel_timing")
+        return ms.value, fl.value, n.value
