@@ -28,6 +28,21 @@ int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_t lda, int 
                          const void *d_B, int64_t ldb, int b_kmajor, float *d_C, int64_t ldc,
                          int tensor_cores, int *d_flag, void *stream);
 
+/* Embedding backward (Hephaistos, Architecture at a glance: token embedding;
+ * its gradient is a scatter-add): dwte[v,:] = sum over positions i with
+ * tokens[i] = v of dx[i,:], summed in increasing i (deterministic), zero for
+ * ids that do not occur.  d_tokens: int32 [n_tokens] (ids outside
+ * [0, vocab) are treated as 0); d_dx: float32 [n_tokens, d_model];
+ * d_dwte: float32 [vocab, d_model], fully overwritten.  d_scratch: device
+ * memory of at least llm_kernel_embed_bwd_scratch_bytes() bytes, 16-byte
+ * aligned, used while the call's kernels run (its contents need no
+ * initialisation).  LLM_ERR_ARG for null pointers, sizes < 1 or a small
+ * scratch. */
+int llm_kernel_embed_bwd_scratch_bytes(int64_t n_tokens, int vocab, int64_t *bytes);
+int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, float *d_dwte,
+                         int64_t n_tokens, int d_model, int vocab, void *d_scratch,
+                         int64_t scratch_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -344,6 +344,18 @@ double orc_ce_fwd_bwd(int n, int V, const double *z, const int32_t *y, double in
   return total;
 }
 
+/* ------------------------------------------------------- embedding bwd */
+/* Gradient of the token-embedding gather (Hephaistos, Architecture at a
+ * glance: token embedding): dwte[v,:] = sum over positions t with tok[t] = v
+ * of dx[t,:], added in position order; rows of absent ids are zero. */
+void orc_embed_bwd(int64_t n, int d, int V, const int32_t *tok, const double *dx, double *dwte) {
+  memset(dwte, 0, sizeof(double) * (size_t)V * d);
+  for (int64_t t = 0; t < n; t++) {
+    double *gw = dwte + (int64_t)tok[t] * d;
+    for (int j = 0; j < d; j++) gw[j] += dx[t * d + j];
+  }
+}
+
 /* -------------------------------------------------------- the whole model */
 typedef struct {
   double *x, *xn1, *rstd1, *qkv, *o, *x1, *xn2, *rstd2, *a, *b, *u;

@@ -68,6 +68,8 @@ _lib.orc_swiglu_bwd.restype = None
 _lib.orc_swiglu_bwd.argtypes = [C.c_int64, _D, _D, _D, _D, _D]
 _lib.orc_ce_fwd_bwd.restype = C.c_double
 _lib.orc_ce_fwd_bwd.argtypes = [C.c_int, C.c_int, _D, _I32, C.c_double, _D]
+_lib.orc_embed_bwd.restype = None
+_lib.orc_embed_bwd.argtypes = [C.c_int64, C.c_int, C.c_int, _I32, _D, _D]
 _lib.orc_forward_backward.restype = C.c_double
 _lib.orc_forward_backward.argtypes = [C.POINTER(OrcCfg), _D, _I32, _I32, _D, _D]
 _lib.orc_adamw.restype = None
@@ -191,6 +193,15 @@ def ce_fwd_bwd(z, y, inv_count=None):
     dz = np.zeros_like(z)
     s = _lib.orc_ce_fwd_bwd(n, V, _dp(z), _ip(y), float(inv_count), _dp(dz))
     return s, dz
+
+
+def embed_bwd(tok, dx, vocab):
+    """dwte [vocab, d] = scatter-add of dx rows by token id, in position order."""
+    tok = np.ascontiguousarray(tok, dtype=np.int32).reshape(-1)
+    dx = _f64(dx)
+    out = np.zeros((vocab, dx.shape[1]))
+    _lib.orc_embed_bwd(tok.size, dx.shape[1], int(vocab), _ip(tok), _dp(dx), _dp(out))
+    return out
 
 
 def forward_backward(cfg, params, tokens, targets=None, want_logits=True, want_grads=True):

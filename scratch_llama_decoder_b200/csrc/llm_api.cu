@@ -573,3 +573,22 @@ extern "C" int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_
   }
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
+
+extern "C" int llm_kernel_embed_bwd_scratch_bytes(int64_t n_tokens, int vocab, int64_t *bytes) {
+  if (!bytes || n_tokens < 1 || vocab < 1 || n_tokens > ((int64_t)1 << 30)) return LLM_ERR_ARG;
+  *bytes = 4 * embed_bwd_scratch_ints(n_tokens, vocab);
+  return LLM_OK;
+}
+
+extern "C" int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, float *d_dwte,
+                                    int64_t n_tokens, int d_model, int vocab, void *d_scratch,
+                                    int64_t scratch_bytes, void *stream) {
+  if (!d_tokens || !d_dx || !d_dwte || !d_scratch || n_tokens < 1 || d_model < 1 || vocab < 1 ||
+      n_tokens > ((int64_t)1 << 30) || ((uintptr_t)d_scratch & 15))
+    return LLM_ERR_ARG;
+  if (scratch_bytes < 4 * embed_bwd_scratch_ints(n_tokens, vocab)) return LLM_ERR_ARG;
+  g_launches = 0;
+  embed_bwd(d_tokens, d_dx, d_dwte, n_tokens, d_model, vocab, (int32_t *)d_scratch,
+            (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}

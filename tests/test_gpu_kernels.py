@@ -53,3 +53,41 @@ def test_gemm_bf16(M, N, K, a_k, b_k, tc):
     err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     # bf16 products are exact in fp32; only fp32 summation rounding remains
     assert err < 1e-5, err
+
+
+@pytest.mark.parametrize("N,d,V", [(16, 16, 27), (16384, 1024, 32000), (1000, 64, 500),
+                                   (300, 48, 70000)])
+def test_embed_bwd_vs_oracle(N, d, V):
+    """Scatter-add of the embedding gradient against the oracle; also
+    bit-for-bit equal to a float32 sum in increasing position order (the
+    kernel's deterministic order); zero rows for absent ids; Zipf ids put
+    thousands of rows on id 0."""
+    import scratch_llama_decoder_b200 as P
+    from synth import zipf_tokens
+    rng = np.random.default_rng(N + V)
+    tok = zipf_tokens(rng, N, V)
+    dx = rng.standard_normal((N, d)).astype(np.float32)
+    nb = C.c_int64(0)
+    assert P.lib.llm_kernel_embed_bwd_scratch_bytes(N, V, C.byref(nb)) == 0
+    scratch = torch.empty(nb.value, dtype=torch.uint8, device="cuda")
+    td = torch.tensor(tok, device="cuda")
+    xd = torch.tensor(dx, device="cuda")
+    out = torch.full((V, d), float("nan"), device="cuda")
+    rc = P.lib.llm_kernel_embed_bwd(C.c_void_p(td.data_ptr()), C.c_void_p(xd.data_ptr()),
+                                    C.c_void_p(out.data_ptr()), N, d, V,
+                                    C.c_void_p(scratch.data_ptr()), nb.value, None)
+    assert rc == 0
+    got = out.cpu().numpy()
+    # float32 sums in increasing position order, done on the host
+    ref = np.zeros((V, d), np.float32)
+    for i in range(N):
+        ref[tok[i]] += dx[i]
+    np.testing.assert_array_equal(got, ref)
+    # and the float64 oracle agrees to float32 rounding
+    ref64 = O.embed_bwd(tok, dx, V)
+    assert np.linalg.norm(got - ref64) <= 1e-6 * max(1e-30, np.linalg.norm(ref64))
+    # too-small scratch is rejected on the host
+    assert P.lib.llm_kernel_embed_bwd(C.c_void_p(td.data_ptr()), C.c_void_p(xd.data_ptr()),
+                                      C.c_void_p(out.data_ptr()), N, d, V,
+                                      C.c_void_p(scratch.data_ptr()), nb.value - 4, None) == \
+        P.LLM_ERR_ARG

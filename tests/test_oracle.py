@@ -224,6 +224,20 @@ def test_swiglu_vs_autograd_and_zero_gate():
     assert np.all(O.swiglu_fwd(np.zeros(5), b[:5]) == 0.0)
 
 
+# ------------------------------------------------------------ embedding bwd
+
+
+def test_embed_bwd_vs_add_at():
+    rng = np.random.default_rng(12)
+    tok = rng.integers(0, 9, 40).astype(np.int32)
+    dx = rng.standard_normal((40, 5))
+    ref = np.zeros((11, 5))
+    np.add.at(ref, tok, dx)
+    got = O.embed_bwd(tok, dx, 11)
+    np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-15)
+    assert np.all(got[9:] == 0.0) and np.all(got[~np.isin(np.arange(11), tok)] == 0.0)
+
+
 # ------------------------------------------------------------ cross-entropy
 
 
