@@ -43,6 +43,26 @@ int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, float *d_dw
                          int64_t n_tokens, int d_model, int vocab, void *d_scratch,
                          int64_t scratch_bytes, void *stream);
 
+/* The embedding backward of llm_kernel_embed_bwd(), for callers that cannot
+ * allocate device memory at call time: code running while a CUDA graph is
+ * being captured, hooks inside an allocator, plug-ins whose host framework
+ * owns all device memory, or loops that forbid allocation after start-up.
+ * The source pages have no counterpart of this call; it exists for such
+ * callers.  Same arguments, layout and result as llm_kernel_embed_bwd(),
+ * without the scratch arguments: the scratch is one library-owned device
+ * array of 1.5 MiB (393,281 int32) on every GPU that loads the library, kept
+ * until the process exits.  Limits: n_tokens <= 65536 and vocab <= 65536,
+ * else LLM_ERR_ARG with nothing launched.  The call allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine).  Its first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, on the
+ * current device) and caches it; make that first call before any stream
+ * capture.  All calls on a device share the array: calls whose kernels
+ * overlap on the GPU (different streams without ordering) race and give
+ * wrong results; calls on one stream are ordered and safe.  Each call
+ * re-initialises what it needs, so no state carries over between calls. */
+int llm_kernel_embed_bwd_noalloc(const int32_t *d_tokens, const float *d_dx, float *d_dwte,
+                                 int64_t n_tokens, int d_model, int vocab, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -56,6 +56,7 @@ EXPORTS = {
                                   _vp]),
     "llm_kernel_embed_bwd_scratch_bytes": (_i, [_i64, _i, C.POINTER(_i64)]),
     "llm_kernel_embed_bwd": (_i, [_vp, _vp, _vp, _i64, _i, _i, _vp, _i64, _vp]),
+    "llm_kernel_embed_bwd_noalloc": (_i, [_vp, _vp, _vp, _i64, _i, _i, _vp]),
 }
 for _name, (_res, _args) in EXPORTS.items():
     _fn = getattr(lib, _name)
