@@ -28,6 +28,27 @@ int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_t lda, int 
                          const void *d_B, int64_t ldb, int b_kmajor, float *d_C, int64_t ldc,
                          int tensor_cores, int *d_flag, void *stream);
 
+/* Causal self-attention of the step, bfloat16 operands and float32 softmax
+ * (Hephaistos, Architecture at a glance: causal multi-head attention with a
+ * numerically stable softmax; strata: n_head and n_kv_head independent,
+ * flash-style forward and backward).  d_qkv: bf16 [batch*ctx, qkvw] with
+ * qkvw = (n_head + 2*n_kv_head)*head_dim, per row all q heads, then k heads,
+ * then v heads (RoPE already applied); query head h uses kv head
+ * h / (n_head/n_kv_head); scale 1/sqrt(head_dim), the diagonal is kept.
+ * Forward: d_o bf16 [batch*ctx, n_head*head_dim] (heads concatenated),
+ * d_lse float32 [batch, n_head, ctx] = natural-log sum of exp of each score
+ * row.  Backward: from d_o, d_lse and d_dout (bf16, like d_o) writes d_dqkv
+ * (bf16, like d_qkv; every element written) and d_D float32 [batch, n_head,
+ * ctx] = rowsum(dout * o) as scratch.  tensor_cores = 1 runs the mma kernels
+ * (head_dim 32 or 64, else LLM_ERR_ARG), 0 the CUDA-core kernels. */
+int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float *d_lse, int batch, int ctx,
+                                  int n_head, int n_kv_head, int head_dim, int tensor_cores,
+                                  void *stream);
+int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o, const void *d_dout,
+                                  const float *d_lse, float *d_D, void *d_dqkv, int batch,
+                                  int ctx, int n_head, int n_kv_head, int head_dim,
+                                  int tensor_cores, void *stream);
+
 /* Embedding backward (Hephaistos, Architecture at a glance: token embedding;
  * its gradient is a scatter-add): dwte[v,:] = sum over positions i with
  * tokens[i] = v of dx[i,:], summed in increasing i (deterministic), zero for

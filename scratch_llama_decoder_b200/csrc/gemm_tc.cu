@@ -625,12 +625,14 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
 
 void attention_fwd(TcPlan *, const void *qkv, void *o, float *lse, DType dt, int B, int T, int H,
                    int Hkv, int hd, cudaStream_t s) {
-  attn_fwd_simt(qkv, o, lse, dt, B, T, H, Hkv, hd, s);
+  if (attn_mma_covers(dt, hd)) attn_fwd_mma(qkv, o, lse, B, T, H, Hkv, hd, s);
+  else attn_fwd_simt(qkv, o, lse, dt, B, T, H, Hkv, hd, s);
 }
 void attention_bwd(TcPlan *, const void *qkv, const void *o, const void *dout, const float *lse,
                    float *Dbuf, void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd,
                    cudaStream_t s) {
-  attn_bwd_simt(qkv, o, dout, lse, Dbuf, dqkv, dt, B, T, H, Hkv, hd, s);
+  if (attn_mma_covers(dt, hd)) attn_bwd_mma(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, hd, s);
+  else attn_bwd_simt(qkv, o, dout, lse, Dbuf, dqkv, dt, B, T, H, Hkv, hd, s);
 }
 
 }  // namespace llm

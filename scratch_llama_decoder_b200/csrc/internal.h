@@ -84,6 +84,13 @@ void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T,
 void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
                    void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s);
 
+// Tensor-core (mma.sync, bf16) kernels for head sizes 32 and 64.
+bool attn_mma_covers(DType dt, int hd);
+void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
+                  cudaStream_t s);
+void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
+                  void *dqkv, int B, int T, int H, int Hkv, int hd, cudaStream_t s);
+
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;
 inline void count_launch(int n = 1) { g_launches += n; }

@@ -592,3 +592,45 @@ extern "C" int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, 
             (cudaStream_t)stream);
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
+
+static bool attn_args_ok(const void *a, const void *b, int B, int T, int H, int Hkv, int hd) {
+  return a && b && B >= 1 && T >= 1 && H >= 1 && Hkv >= 1 && H % Hkv == 0 && hd >= 2 &&
+         hd % 2 == 0 && hd <= 128;
+}
+
+extern "C" int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float *d_lse,
+                                             int batch, int ctx, int n_head, int n_kv_head,
+                                             int head_dim, int tensor_cores, void *stream) {
+  if (!attn_args_ok(d_qkv, d_o, batch, ctx, n_head, n_kv_head, head_dim) || !d_lse)
+    return LLM_ERR_ARG;
+  g_launches = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (tensor_cores) {
+    if (!attn_mma_covers(DT_BF16, head_dim)) return LLM_ERR_ARG;
+    attn_fwd_mma(d_qkv, d_o, d_lse, batch, ctx, n_head, n_kv_head, head_dim, s);
+  } else {
+    attn_fwd_simt(d_qkv, d_o, d_lse, DT_BF16, batch, ctx, n_head, n_kv_head, head_dim, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+extern "C" int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o,
+                                             const void *d_dout, const float *d_lse, float *d_D,
+                                             void *d_dqkv, int batch, int ctx, int n_head,
+                                             int n_kv_head, int head_dim, int tensor_cores,
+                                             void *stream) {
+  if (!attn_args_ok(d_qkv, d_o, batch, ctx, n_head, n_kv_head, head_dim) || !d_dout || !d_lse ||
+      !d_D || !d_dqkv)
+    return LLM_ERR_ARG;
+  g_launches = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (tensor_cores) {
+    if (!attn_mma_covers(DT_BF16, head_dim)) return LLM_ERR_ARG;
+    attn_bwd_mma(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, batch, ctx, n_head, n_kv_head, head_dim,
+                 s);
+  } else {
+    attn_bwd_simt(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, DT_BF16, batch, ctx, n_head, n_kv_head,
+                  head_dim, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}

@@ -91,3 +91,47 @@ def test_embed_bwd_vs_oracle(N, d, V):
                                       C.c_void_p(out.data_ptr()), N, d, V,
                                       C.c_void_p(scratch.data_ptr()), nb.value - 4, None) == \
         P.LLM_ERR_ARG
+
+
+# (batch, ctx, n_head, n_kv_head, head_dim): tile multiples, ragged lengths,
+# one position, MHA/GQA/MQA, both head sizes, the longest context
+ATTN = [(1, 64, 2, 2, 64), (2, 200, 4, 2, 64), (1, 130, 8, 8, 32), (3, 1, 4, 1, 64),
+        (2, 512, 8, 2, 64), (1, 2048, 2, 2, 64), (1, 333, 4, 1, 32)]
+
+
+@pytest.mark.parametrize("tc", [1, 0])
+@pytest.mark.parametrize("B,T,H,Hkv,hd", ATTN)
+def test_attention_fwd_bwd_vs_oracle(B, T, H, Hkv, hd, tc):
+    import scratch_llama_decoder_b200 as P
+    if not tc and T > 600:
+        pytest.skip("CUDA-core reference kernel: long contexts covered by the step tests")
+    rng = np.random.default_rng(B * 1000 + T + H + hd)
+    d, kvd = H * hd, Hkv * hd
+    w = d + 2 * kvd
+    qkv = _bf16(rng, (B * T, w))
+    dout = _bf16(rng, (B * T, d))
+    qd, dd = qkv.cuda(), dout.cuda()
+    o = torch.zeros(B * T, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, T, device="cuda")
+    Dv = torch.zeros(B, H, T, device="cuda")
+    dq = torch.full((B * T, w), float("nan"), dtype=torch.bfloat16, device="cuda")
+    p = lambda t: C.c_void_p(t.data_ptr())
+    assert P.lib.llm_kernel_attention_fwd_bf16(p(qd), p(o), p(lse), B, T, H, Hkv, hd, tc,
+                                               None) == 0
+    assert P.lib.llm_kernel_attention_bwd_bf16(p(qd), p(o), p(dd), p(lse), p(Dv), p(dq), B, T, H,
+                                               Hkv, hd, tc, None) == 0
+    torch.cuda.synchronize()
+    q64 = qkv.float().double().numpy().reshape(B, T, w)
+    d64 = dout.float().double().numpy().reshape(B, T, d)
+    og = o.float().double().cpu().numpy().reshape(B, T, d)
+    lg = lse.double().cpu().numpy()
+    dg = dq.float().double().cpu().numpy().reshape(B, T, w)
+    for b in range(B):
+        o_ref, lse_ref, _ = O.attention_fwd(q64[b], d, H, Hkv)
+        dq_ref = O.attention_bwd(q64[b], d64[b], d, H, Hkv)
+        assert np.linalg.norm(og[b] - o_ref) / np.linalg.norm(o_ref) < 1e-2
+        assert np.abs(lg[b] - lse_ref).max() < 2e-3
+        for lo, hi in ((0, d), (d, d + kvd), (d + kvd, w)):  # dq, dk, dv
+            ref = dq_ref[:, lo:hi]
+            err = np.linalg.norm(dg[b][:, lo:hi] - ref) / max(np.linalg.norm(ref), 1e-30)
+            assert err < 2e-2, (b, lo, err)
