@@ -131,7 +131,11 @@ def test_attention_fwd_bwd_vs_oracle(B, T, H, Hkv, hd, tc):
         dq_ref = O.attention_bwd(q64[b], d64[b], d, H, Hkv)
         assert np.linalg.norm(og[b] - o_ref) / np.linalg.norm(o_ref) < 1e-2
         assert np.abs(lg[b] - lse_ref).max() < 2e-3
-        for lo, hi in ((0, d), (d, d + kvd), (d + kvd, w)):  # dq, dk, dv
+        # dq, dk, dv; a block whose exact value is ~0 (T = 1: dq = dk = 0 since
+        # dS = P (dP - D) vanishes for a single key) is measured against the
+        # scale of the sequence's whole gradient instead
+        full = np.linalg.norm(dq_ref)
+        for lo, hi in ((0, d), (d, d + kvd), (d + kvd, w)):
             ref = dq_ref[:, lo:hi]
-            err = np.linalg.norm(dg[b][:, lo:hi] - ref) / max(np.linalg.norm(ref), 1e-30)
+            err = np.linalg.norm(dg[b][:, lo:hi] - ref) / max(np.linalg.norm(ref), 1e-3 * full)
             assert err < 2e-2, (b, lo, err)
