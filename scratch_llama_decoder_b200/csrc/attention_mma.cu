@@ -11,12 +11,15 @@
 //   fwd : one CTA per (b, h, 64 queries); loops over key blocks up to the
 //         diagonal; online softmax in registers; P goes from the S
 //         accumulator straight into the A fragments of P.V.
-//   D   : D_i = sum_e dO_ie O_ie.
-//   dq  : one CTA per (b, h, 64 queries): recompute P from lse, dP = dO V^T,
-//         dS = P (dP - D), dQ += dS K.
+//   dq  : one CTA per (b, h, 64 queries): D_i = sum_e dO_ie O_ie (saved for
+//         dkv), recompute P from lse, dP = dO V^T, dS = P (dP - D),
+//         dQ += dS K.
 //   dkv : one CTA per (b, kv head, 64 keys): loops over the group's query
 //         heads and the query blocks at or after the keys, in a fixed order:
 //         dV += P^T dO, dK += dS^T Q.  No atomics: deterministic.
+// With cos/sin tables given, dq and dk leave through the inverse RoPE
+// rotation (Hephaistos: RoPE on q and k), so the gradient reaching the QKV
+// projection is with respect to the un-rotated q and k.
 #include "common.cuh"
 #include "gemm_tc.h"
 
@@ -145,6 +148,24 @@ LLM_DEV void c_to_a(const float (&s)[8][4], uint32_t (&p)[4][4]) {
   }
 }
 
+// Rotate one accumulator row (r) of a 16 x HD tile by -angle(pos): columns j
+// and j + HD/2 (n tiles i and i + HD/16) pair up; the backward of the
+// rotate-half RoPE.
+template <int HD>
+LLM_DEV void rope_bwd_row(float (&acc)[HD / 8][4], int r, const float *ct, const float *st) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < HD / 16; i++)
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+      int j = 8 * i + 2 * (lane & 3) + e;
+      float c = ct[j], sn = st[j];
+      float x = acc[i][2 * r + e], y = acc[i + HD / 16][2 * r + e];
+      acc[i][2 * r + e] = x * c + y * sn;
+      acc[i + HD / 16][2 * r + e] = y * c - x * sn;
+    }
+}
+
 // ------------------------------------------------------------------ forward
 template <int HD>
 __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict__ qkv,
@@ -251,29 +272,18 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
 }
 
 // ---------------------------------------------------------------- backward
-// D_i = sum_e dO_ie O_ie (one warp per row).
-template <int HD>
-__global__ void k_attn_D(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dout,
-                         float *__restrict__ D, int B, int T, int H) {
-  int64_t wid = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
-  int lane = threadIdx.x & 31;
-  if (wid >= (int64_t)B * H * T) return;
-  int i = (int)(wid % T), h = (int)((wid / T) % H), b = (int)(wid / ((int64_t)T * H));
-  int64_t off = ((int64_t)b * T + i) * (H * HD) + h * HD;
-  float s = 0.f;
-  for (int e = lane; e < HD; e += 32) s += to_f(o[off + e]) * to_f(dout[off + e]);
-  s = warp_sum(s);
-  if (lane == 0) D[((int64_t)b * H + h) * T + i] = s;
-}
-
 template <int HD>
 __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict__ qkv,
+                                                const __nv_bfloat16 *__restrict__ o,
                                                 const __nv_bfloat16 *__restrict__ dout,
                                                 const float *__restrict__ lse,
-                                                const float *__restrict__ Dv,
-                                                __nv_bfloat16 *__restrict__ dqkv, int T, int H,
+                                                float *__restrict__ Dv,
+                                                __nv_bfloat16 *__restrict__ dqkv,
+                                                const float *__restrict__ cos_t,
+                                                const float *__restrict__ sin_t, int T, int H,
                                                 int Hkv, float scale) {
   __shared__ Tile<HD> Ks[2], Vs[2];
+  __shared__ float Dsh[64];
   const int nqb = gridDim.x;
   const int qb = nqb - 1 - blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -295,6 +305,33 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
   uint32_t qf[HD / 16][4], df[HD / 16][4];
   load_afrag<HD>(Ks[1], w, qf);
   load_afrag<HD>(Vs[1], w, df);
+  {
+    // D_i = sum_e dO_ie O_ie: two threads per row, halves combined by shuffle
+    const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int qi = q0 + r;
+    float acc_d = 0.f;
+    if (qi < T) {
+      const __nv_bfloat16 *orow = o + (roff + qi) * d + h * HD + half * (HD / 2);
+      const __nv_bfloat16 *drow = &Vs[1].v[r * Tile<HD>::LD + half * (HD / 2)];
+#pragma unroll
+      for (int e = 0; e < HD / 2; e += 8) {
+        uint4 a = *reinterpret_cast<const uint4 *>(orow + e);
+        uint4 c = *reinterpret_cast<const uint4 *>(drow + e);
+        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&c);
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          float2 fa = __bfloat1622float2(ha[k]), fc = __bfloat1622float2(hc[k]);
+          acc_d += fa.x * fc.x + fa.y * fc.y;
+        }
+      }
+    }
+    acc_d += __shfl_xor_sync(0xffffffffu, acc_d, 1);
+    if (half == 0) {
+      Dsh[r] = acc_d;
+      if (qi < T) Dv[((int64_t)b * H + h) * T + qi] = acc_d;
+    }
+  }
   __syncthreads();
   const float sl2 = scale * LOG2E;
   const int row0 = q0 + w * 16 + (lane >> 2);
@@ -304,7 +341,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
     int qi = row0 + r * 8;
     bool ok = qi < T;
     L2[r] = ok ? lse[((int64_t)b * H + h) * T + qi] * LOG2E : 0.f;
-    Dr[r] = ok ? Dv[((int64_t)b * H + h) * T + qi] : 0.f;
+    Dr[r] = Dsh[w * 16 + (lane >> 2) + r * 8];
   }
   float acc[HD / 8][4];
 #pragma unroll
@@ -346,6 +383,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
   for (int r = 0; r < 2; r++) {
     int qi = row0 + r * 8;
     if (qi >= T) continue;
+    if (cos_t) rope_bwd_row<HD>(acc, r, cos_t + (int64_t)qi * (HD / 2), sin_t + (int64_t)qi * (HD / 2));
     __nv_bfloat16 *dst = dqkv + ((int64_t)b * T + qi) * ld + h * HD + (lane & 3) * 2;
 #pragma unroll
     for (int i = 0; i < HD / 8; i++)
@@ -359,7 +397,9 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
                                                  const __nv_bfloat16 *__restrict__ dout,
                                                  const float *__restrict__ lse,
                                                  const float *__restrict__ Dv,
-                                                 __nv_bfloat16 *__restrict__ dqkv, int T, int H,
+                                                 __nv_bfloat16 *__restrict__ dqkv,
+                                                 const float *__restrict__ cos_t,
+                                                 const float *__restrict__ sin_t, int T, int H,
                                                  int Hkv, float scale) {
   __shared__ Tile<HD> KVs, Qs[2], dOs[2];
   __shared__ float Ls[2][64], Ds[2][64];
@@ -448,6 +488,7 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
   for (int r = 0; r < 2; r++) {
     int kj = key0 + r * 8;
     if (kj >= T) continue;
+    if (cos_t) rope_bwd_row<HD>(dk, r, cos_t + (int64_t)kj * (HD / 2), sin_t + (int64_t)kj * (HD / 2));
     __nv_bfloat16 *dkr = dqkv + ((int64_t)b * T + kj) * ld + d + g * HD + (lane & 3) * 2;
     __nv_bfloat16 *dvr = dkr + kvd;
 #pragma unroll
@@ -477,24 +518,22 @@ void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int
 }
 
 void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
-                  void *dqkv, int B, int T, int H, int Hkv, int hd, cudaStream_t s) {
+                  void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
+                  const float *sin_t, cudaStream_t s) {
   using namespace attn;
   float scale = 1.0f / sqrtf((float)hd);
   const __nv_bfloat16 *q = (const __nv_bfloat16 *)qkv, *oo = (const __nv_bfloat16 *)o,
                       *dO = (const __nv_bfloat16 *)dout;
   __nv_bfloat16 *dq = (__nv_bfloat16 *)dqkv;
-  unsigned gD = (unsigned)(((int64_t)B * H * T + 7) / 8);
   dim3 gq((T + BQ - 1) / BQ, H, B), gkv((T + BKV - 1) / BKV, Hkv, B);
   if (hd == 64) {
-    k_attn_D<64><<<gD, 256, 0, s>>>(oo, dO, Dbuf, B, T, H);
-    k_attn_dq<64><<<gq, NT, 0, s>>>(q, dO, lse, Dbuf, dq, T, H, Hkv, scale);
-    k_attn_dkv<64><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, T, H, Hkv, scale);
+    k_attn_dq<64><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
+    k_attn_dkv<64><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
   } else {
-    k_attn_D<32><<<gD, 256, 0, s>>>(oo, dO, Dbuf, B, T, H);
-    k_attn_dq<32><<<gq, NT, 0, s>>>(q, dO, lse, Dbuf, dq, T, H, Hkv, scale);
-    k_attn_dkv<32><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, T, H, Hkv, scale);
+    k_attn_dq<32><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
+    k_attn_dkv<32><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
   }
-  count_launch(3);
+  count_launch(2);
 }
 
 }  // namespace llm

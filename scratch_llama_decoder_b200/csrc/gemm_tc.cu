@@ -32,7 +32,8 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int STAGING_BYTES = 4 * 32 * 33 * 4;  // epilogue transpose squares, 4 warps
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + STAGING_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 192;
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on any wait
@@ -147,30 +148,9 @@ LLM_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // ------------------------------------------------------------ epilogue stores
-LLM_DEV void store32_f32(float *dst, const float (&v)[32], int nvalid) {
-  if (nvalid >= 32) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 4)
-      *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-  } else {
-    for (int i = 0; i < nvalid; i++) dst[i] = v[i];
-  }
-}
 LLM_DEV uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
-}
-LLM_DEV void store32_bf16(__nv_bfloat16 *dst, const float (&v)[32], int nvalid) {
-  if (nvalid >= 32) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-      uint4 q = make_uint4(pack_bf16(v[i], v[i + 1]), pack_bf16(v[i + 2], v[i + 3]),
-                           pack_bf16(v[i + 4], v[i + 5]), pack_bf16(v[i + 6], v[i + 7]));
-      *reinterpret_cast<uint4 *>(dst + i) = q;
-    }
-  } else {
-    for (int i = 0; i < nvalid; i++) dst[i] = __float2bfloat16_rn(v[i]);
-  }
 }
 LLM_DEV void load32_bf16(const __nv_bfloat16 *src, float (&v)[32], int nvalid) {
   if (nvalid >= 32) {
@@ -190,19 +170,60 @@ LLM_DEV void load32_bf16(const __nv_bfloat16 *src, float (&v)[32], int nvalid) {
   }
 }
 
-// One output tile's epilogue for the thread owning row m (TMEM lane).
-// tm: TMEM address of this lane's accumulator row at column 0.
-// All 32 lanes of the warp execute every tcgen05.ld (warp-uniform control);
-// rows past M only skip their global loads and stores.
-LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split, bool zero) {
+// Coalesced write-out of a warp's 32 x 32 chunk: lane i holds row i in v;
+// the chunk goes through a padded shared-memory square (33 floats per row, so
+// both the row-wise writes and the column-wise reads hit 32 distinct banks)
+// and leaves one row per store instruction.  rows / cols clip the edges.
+LLM_DEV void put32_f32(float (*stg)[33], const float (&v)[32], float *dst, int64_t ld, int rows,
+                       int cols, const float *R, int64_t ldr) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 32; i++) stg[lane][i] = v[i];
+  __syncwarp();
+  if (lane < cols) {
+    for (int r = 0; r < rows; r++) {
+      float x = stg[r][lane];
+      if (R) x += R[(int64_t)r * ldr + lane];
+      dst[(int64_t)r * ld + lane] = x;
+    }
+  }
+  __syncwarp();
+}
+LLM_DEV void put32_bf16(float (*stg)[33], const float (&v)[32], __nv_bfloat16 *dst, int64_t ld,
+                        int rows, int cols) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 32; i++) stg[lane][i] = v[i];
+  __syncwarp();
+  const int c = 2 * (lane & 15);
+  if (c < cols) {
+    for (int r = lane >> 4; r < rows; r += 2) {
+      if (c + 1 < cols)
+        *reinterpret_cast<uint32_t *>(dst + (int64_t)r * ld + c) = pack_bf16(stg[r][c], stg[r][c + 1]);
+      else
+        dst[(int64_t)r * ld + c] = __float2bfloat16_rn(stg[r][c]);
+    }
+  }
+  __syncwarp();
+}
+
+// One output tile's epilogue for a warp: rows [row0, row0+32) of the tile
+// (TMEM lanes of this warp's quarter, lane i = row row0 + i), columns
+// [n0, n0+BN).  Every lane executes every tcgen05.ld (warp-uniform control);
+// rows past M are clipped only at the stores.
+LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int split, bool zero,
+                           float (*stg)[33]) {
+  const int lane = threadIdx.x & 31;
+  const int m = row0 + lane;
   const bool row_ok = m < a.M;
+  const int rows = max(0, min(32, a.M - row0));
   const int N = a.N;
-  auto nval = [&](int n) { return row_ok ? min(32, N - n) : 0; };
+  auto ncols = [&](int n) { return max(0, min(32, N - n)); };
   float v[32];
   if (a.epi == TC_EPI_ROPE) {
     // RoPE on q/k heads (columns < rot_cols), plain store of v heads.
     const int hd = a.hd, half = hd / 2, t = m % a.T;
-    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)m * a.ldc;
+    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
     if (hd == 64) {
       for (int c0 = 0; c0 < BN; c0 += 64) {
         int n = n0 + c0;
@@ -219,8 +240,8 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split,
             hi[j] = y * c + x * s;
           }
         }
-        store32_bf16(C + n, lo, nval(n));
-        store32_bf16(C + n + 32, hi, nval(n + 32));
+        put32_bf16(stg, lo, C + n, a.ldc, rows, ncols(n));
+        put32_bf16(stg, hi, C + n + 32, a.ldc, rows, ncols(n + 32));
       }
     } else {  // hd == 32: both halves of a head sit in one 32-column chunk
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -237,15 +258,15 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split,
             v[j + 16] = y * c + x * s;
           }
         }
-        store32_bf16(C + n, v, nval(n));
+        put32_bf16(stg, v, C + n, a.ldc, rows, ncols(n));
       }
     }
     return;
   }
   if (a.epi == TC_EPI_SWIGLU) {
     // Interleaved [a|b] blocks of 64+64 columns: store a, b and u = silu(a) b.
-    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)m * a.ldc;
-    __nv_bfloat16 *U = (__nv_bfloat16 *)a.aux + (int64_t)m * a.ld_aux;
+    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
+    __nv_bfloat16 *U = (__nv_bfloat16 *)a.aux + (int64_t)row0 * a.ld_aux;
     for (int blk = 0; blk < BN; blk += 2 * SWIGLU_BLOCK) {
       int n = n0 + blk;
       if (n >= N) break;
@@ -253,12 +274,11 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split,
         float av[32], bv[32];
         if (zero) { for (int i = 0; i < 32; i++) av[i] = bv[i] = 0.f; }
         else { tmem_ld32(tm + blk + q, av); tmem_ld32(tm + blk + SWIGLU_BLOCK + q, bv); }
-        int nv = row_ok ? 32 : 0;
-        store32_bf16(C + n + q, av, nv);
-        store32_bf16(C + n + SWIGLU_BLOCK + q, bv, nv);
+        put32_bf16(stg, av, C + n + q, a.ldc, rows, 32);
+        put32_bf16(stg, bv, C + n + SWIGLU_BLOCK + q, a.ldc, rows, 32);
 #pragma unroll
         for (int i = 0; i < 32; i++) av[i] = av[i] / (1.f + expf(-av[i])) * bv[i];
-        store32_bf16(U + (n / (2 * SWIGLU_BLOCK)) * SWIGLU_BLOCK + q, av, nv);
+        put32_bf16(stg, av, U + (n / (2 * SWIGLU_BLOCK)) * SWIGLU_BLOCK + q, a.ld_aux, rows, 32);
       }
     }
     return;
@@ -267,17 +287,16 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split,
     // acc = du for hidden units [n0, n0+BN); write [da|db] at their
     // interleaved columns using the saved [a|b].
     const __nv_bfloat16 *AB = (const __nv_bfloat16 *)a.aux + (int64_t)m * a.ld_aux;
-    __nv_bfloat16 *D = (__nv_bfloat16 *)a.C + (int64_t)m * a.ldc;
+    __nv_bfloat16 *D = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
     for (int c0 = 0; c0 < BN; c0 += 32) {
       int j = n0 + c0;
       if (j >= N) break;
       if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
       else tmem_ld32(tm + c0, v);
       int64_t ca = w1_col(j);
-      int nv = row_ok ? 32 : 0;
       float av[32], bv[32];
-      load32_bf16(AB + ca, av, nv);
-      load32_bf16(AB + ca + SWIGLU_BLOCK, bv, nv);
+      load32_bf16(AB + ca, av, row_ok ? 32 : 0);
+      load32_bf16(AB + ca + SWIGLU_BLOCK, bv, row_ok ? 32 : 0);
 #pragma unroll
       for (int i = 0; i < 32; i++) {
         float s = 1.f / (1.f + expf(-av[i]));
@@ -286,8 +305,8 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split,
         bv[i] = du * av[i] * s;
         av[i] = da;
       }
-      store32_bf16(D + ca, av, nv);
-      store32_bf16(D + ca + SWIGLU_BLOCK, bv, nv);
+      put32_bf16(stg, av, D + ca, a.ldc, rows, 32);
+      put32_bf16(stg, bv, D + ca + SWIGLU_BLOCK, a.ldc, rows, 32);
     }
     return;
   }
@@ -295,27 +314,15 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int m, int n0, int split,
   for (int c0 = 0; c0 < BN; c0 += 32) {
     int n = n0 + c0;
     if (n >= N) break;
-    int nv = nval(n);
     if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
     else tmem_ld32(tm + c0, v);
-    if (a.out == OUT_F32) {
-      store32_f32((float *)a.C + (int64_t)m * a.ldc + n, v, nv);
-    } else if (a.out == OUT_ACT) {
-      store32_bf16((__nv_bfloat16 *)a.C + (int64_t)m * a.ldc + n, v, nv);
-    } else if (a.out == OUT_ADD_F32) {
-      const float *r = a.R + (int64_t)m * a.ldr + n;
-      if (nv >= 32) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float4 q = *reinterpret_cast<const float4 *>(r + i);
-          v[i] += q.x; v[i + 1] += q.y; v[i + 2] += q.z; v[i + 3] += q.w;
-        }
-      } else {
-        for (int i = 0; i < nv; i++) v[i] += r[i];
-      }
-      store32_f32((float *)a.C + (int64_t)m * a.ldc + n, v, nv);
-    } else {  // OUT_PARTIAL
-      store32_f32((float *)a.C + (int64_t)split * a.M * a.ldc + (int64_t)m * a.ldc + n, v, nv);
+    if (a.out == OUT_ACT) {
+      put32_bf16(stg, v, (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc + n, a.ldc, rows, ncols(n));
+    } else {
+      float *dst = (float *)a.C + (int64_t)row0 * a.ldc + n;
+      if (a.out == OUT_PARTIAL) dst += (int64_t)split * a.M * a.ldc;
+      const float *R = (a.out == OUT_ADD_F32) ? a.R + (int64_t)row0 * a.ldr + n : nullptr;
+      put32_f32(stg, v, dst, a.ldc, rows, ncols(n), R, a.ldr);
     }
   }
 }
@@ -459,15 +466,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // -------------------------------------------------- epilogue warps
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    float (*stg)[33] = reinterpret_cast<float (*)[33]>(smem + STAGES * STAGE_BYTES + 256) +
+                       (warp - 2) * 32;
     int acc = 0;
     uint32_t aph = 0;
     for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
       int split = w / tiles_mn, tile = w % tiles_mn;
       int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
       int kb0, nkb = kblocks_of(split, kb0);
-      int m = m0 + quarter * 32 + lane;
+      const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, 0, m, n0, split, true);
+        epilogue_tile(a, 0, row0, n0, split, true, stg);
         continue;
       }
       int got = 0;
@@ -476,7 +485,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!got) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, tm, m, n0, split, false);
+      epilogue_tile(a, tm, row0, n0, split, false, stg);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -630,9 +639,15 @@ void attention_fwd(TcPlan *, const void *qkv, void *o, float *lse, DType dt, int
 }
 void attention_bwd(TcPlan *, const void *qkv, const void *o, const void *dout, const float *lse,
                    float *Dbuf, void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd,
-                   cudaStream_t s) {
-  if (attn_mma_covers(dt, hd)) attn_bwd_mma(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, hd, s);
-  else attn_bwd_simt(qkv, o, dout, lse, Dbuf, dqkv, dt, B, T, H, Hkv, hd, s);
+                   const float *cos_t, const float *sin_t, cudaStream_t s) {
+  if (attn_mma_covers(dt, hd)) {
+    attn_bwd_mma(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, hd, cos_t, sin_t, s);
+    return;
+  }
+  attn_bwd_simt(qkv, o, dout, lse, Dbuf, dqkv, dt, B, T, H, Hkv, hd, s);
+  if (cos_t)
+    rope_apply(dqkv, dt, cos_t, sin_t, (int64_t)B * T, T, (H + Hkv) * hd,
+               (int64_t)(H + 2 * Hkv) * hd, hd, -1, s);
 }
 
 }  // namespace llm

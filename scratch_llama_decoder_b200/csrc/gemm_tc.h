@@ -28,8 +28,11 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
 // else the SIMT kernels.
 void attention_fwd(TcPlan *p, const void *qkv, void *o, float *lse, DType dt, int B, int T, int H,
                    int Hkv, int hd, cudaStream_t s);
+// attention_bwd also applies the RoPE backward (rotation by -angle) to the dq
+// and dk columns of dqkv: fused into the tensor-core kernels, a separate pass
+// after the SIMT kernels.
 void attention_bwd(TcPlan *p, const void *qkv, const void *o, const void *dout, const float *lse,
                    float *Dbuf, void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd,
-                   cudaStream_t s);
+                   const float *cos_t, const float *sin_t, cudaStream_t s);
 
 }  // namespace llm

@@ -88,8 +88,11 @@ void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float
 bool attn_mma_covers(DType dt, int hd);
 void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
                   cudaStream_t s);
+// With cos_t/sin_t (RoPE tables [T, hd/2]) non-null, dq and dk are rotated
+// back by -angle before they are stored.
 void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
-                  void *dqkv, int B, int T, int H, int Hkv, int hd, cudaStream_t s);
+                  void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
+                  const float *sin_t, cudaStream_t s);
 
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;

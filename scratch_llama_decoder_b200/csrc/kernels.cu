@@ -170,10 +170,102 @@ __global__ void k_rmsnorm_bwd(const float *__restrict__ x, const float *__restri
     part[(int64_t)blockIdx.x * d + j] = s;
   }
 }
+// Vectorised form for d = 128 * VPL: each lane owns VPL float4 columns of a
+// row, keeps its gain-gradient partial sums in registers, and the block adds
+// its 8 warps' partials in warp order.
+template <typename A, int VPL>
+__global__ void __launch_bounds__(256) k_rmsnorm_bwd_v(const float *__restrict__ x,
+                                                       const float *__restrict__ rstd,
+                                                       const float *__restrict__ g,
+                                                       const float *__restrict__ dy,
+                                                       const float *dres, float *dx,
+                                                       A *__restrict__ dx_act,
+                                                       float *__restrict__ part, int64_t N) {
+  constexpr int d = 128 * VPL;
+  __shared__ float4 sred[8][32 * VPL];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  float4 gv[VPL], acc[VPL];
+#pragma unroll
+  for (int k = 0; k < VPL; k++) {
+    gv[k] = reinterpret_cast<const float4 *>(g)[lane + 32 * k];
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int64_t r0 = (int64_t)blockIdx.x * RMS_ROWS;
+  for (int rr = warp; rr < RMS_ROWS; rr += 8) {
+    const int64_t row = r0 + rr;
+    if (row >= N) break;
+    const float4 *xr = reinterpret_cast<const float4 *>(x + row * d);
+    const float4 *dyr = reinterpret_cast<const float4 *>(dy + row * d);
+    float4 xv[VPL], dv[VPL];
+    float dot = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      xv[k] = xr[lane + 32 * k];
+      dv[k] = dyr[lane + 32 * k];
+      dot += gv[k].x * dv[k].x * xv[k].x + gv[k].y * dv[k].y * xv[k].y +
+             gv[k].z * dv[k].z * xv[k].z + gv[k].w * dv[k].w * xv[k].w;
+    }
+    dot = warp_sum(dot);
+    const float r = rstd[row];
+    const float c = r * r * r * dot / (float)d;
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      float4 o;
+      o.x = r * gv[k].x * dv[k].x - xv[k].x * c;
+      o.y = r * gv[k].y * dv[k].y - xv[k].y * c;
+      o.z = r * gv[k].z * dv[k].z - xv[k].z * c;
+      o.w = r * gv[k].w * dv[k].w - xv[k].w * c;
+      if (dres) {
+        float4 q = reinterpret_cast<const float4 *>(dres + row * d)[lane + 32 * k];
+        o.x += q.x; o.y += q.y; o.z += q.z; o.w += q.w;
+      }
+      reinterpret_cast<float4 *>(dx + row * d)[lane + 32 * k] = o;
+      if (dx_act) {
+        A *dst = dx_act + row * d + 4 * (lane + 32 * k);
+        dst[0] = from_f<A>(o.x); dst[1] = from_f<A>(o.y);
+        dst[2] = from_f<A>(o.z); dst[3] = from_f<A>(o.w);
+      }
+      acc[k].x += dv[k].x * xv[k].x * r;
+      acc[k].y += dv[k].y * xv[k].y * r;
+      acc[k].z += dv[k].z * xv[k].z * r;
+      acc[k].w += dv[k].w * xv[k].w * r;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < VPL; k++) sred[warp][lane + 32 * k] = acc[k];
+  __syncthreads();
+  for (int j = threadIdx.x; j < 32 * VPL; j += 256) {
+    float4 t = sred[0][j];
+    for (int w = 1; w < 8; w++) {
+      float4 q = sred[w][j];
+      t.x += q.x; t.y += q.y; t.z += q.z; t.w += q.w;
+    }
+    reinterpret_cast<float4 *>(part + (int64_t)blockIdx.x * d)[j] = t;
+  }
+}
+
 int rmsnorm_bwd(const float *x, const float *rstd, const float *g, const float *dy,
                 const float *dres, float *dx, void *dx_act, DType dt, float *part, int64_t N, int d,
                 cudaStream_t s) {
   int nblk = rmsnorm_bwd_blocks(N);
+  if (d == 128 || d == 256 || d == 512 || d == 1024) {
+#define RB(VPL)                                                                                \
+  do {                                                                                         \
+    if (dt == DT_BF16)                                                                         \
+      k_rmsnorm_bwd_v<__nv_bfloat16, VPL><<<nblk, 256, 0, s>>>(x, rstd, g, dy, dres, dx,       \
+                                                                (__nv_bfloat16 *)dx_act, part, N); \
+    else                                                                                       \
+      k_rmsnorm_bwd_v<float, VPL><<<nblk, 256, 0, s>>>(x, rstd, g, dy, dres, dx, (float *)dx_act, \
+                                                        part, N);                              \
+  } while (0)
+    if (d == 128) RB(1);
+    else if (d == 256) RB(2);
+    else if (d == 512) RB(4);
+    else RB(8);
+#undef RB
+    count_launch();
+    return nblk;
+  }
   size_t smem = sizeof(float) * 8 * d;
   if (dt == DT_BF16)
     k_rmsnorm_bwd<<<nblk, 256, smem, s>>>(x, rstd, g, dy, dres, dx, (__nv_bfloat16 *)dx_act, part,
@@ -184,16 +276,27 @@ int rmsnorm_bwd(const float *x, const float *rstd, const float *g, const float *
   return nblk;
 }
 
+// out[j] = sum over b of part[b][j]: 8 groups of threads add interleaved
+// rows (b = grp, grp+8, ...), then the 8 group sums are added in group order
+// (a fixed order, so the result does not depend on scheduling).
 __global__ void k_reduce_partials(const float *__restrict__ part, int nblk, int d,
                                   float *__restrict__ out) {
-  int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= d) return;
+  __shared__ float sh[8][32];
+  const int c = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const int j = blockIdx.x * 32 + c;
   float s = 0.f;
-  for (int b = 0; b < nblk; b++) s += part[(int64_t)b * d + j];
-  out[j] = s;
+  if (j < d)
+    for (int b = grp; b < nblk; b += 8) s += part[(int64_t)b * d + j];
+  sh[grp][c] = s;
+  __syncthreads();
+  if (grp == 0 && j < d) {
+    float t = sh[0][c];
+    for (int k = 1; k < 8; k++) t += sh[k][c];
+    out[j] = t;
+  }
 }
 void reduce_partials(const float *part, int nblk, int d, float *out, cudaStream_t s) {
-  k_reduce_partials<<<cdiv(d, 128), 128, 0, s>>>(part, nblk, d, out);
+  k_reduce_partials<<<cdiv(d, 32), 256, 0, s>>>(part, nblk, d, out);
   count_launch();
 }
 
@@ -523,14 +626,43 @@ __global__ void k_clamp_keys(const int32_t *__restrict__ tok, int32_t *__restric
   keys[i] = t;
   atomicAdd(&counts[t], 1);
 }
+// One block per (vocabulary row, 256 columns); each thread owns 4 columns
+// (one float4) and adds the rows of its bucket in position order, loading 8
+// rows ahead so a long bucket (the Zipf head) is not latency-bound.
 __global__ void k_embed_rows(const int32_t *__restrict__ order, const int32_t *__restrict__ offs,
                              const float *__restrict__ dx, float *__restrict__ dwte, int d) {
-  int v = blockIdx.x;
-  int b = offs[v], e = offs[v + 1];
+  const int v = blockIdx.x;
+  const int c4 = blockIdx.y * 64 + threadIdx.x;
+  if (4 * c4 >= d) return;
+  const int b = offs[v], e = offs[v + 1];
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  int p = b;
+  for (; p + 8 <= e; p += 8) {
+    float4 t[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++)
+      t[u] = reinterpret_cast<const float4 *>(dx + (int64_t)order[p + u] * d)[c4];
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      s.x += t[u].x; s.y += t[u].y; s.z += t[u].z; s.w += t[u].w;
+    }
+  }
+  for (; p < e; p++) {
+    float4 t = reinterpret_cast<const float4 *>(dx + (int64_t)order[p] * d)[c4];
+    s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+  }
+  reinterpret_cast<float4 *>(dwte + (int64_t)v * d)[c4] = s;
+}
+// Same sums for any d or alignment (one thread per column, rows in order).
+__global__ void k_embed_rows_scalar(const int32_t *__restrict__ order,
+                                    const int32_t *__restrict__ offs, const float *__restrict__ dx,
+                                    float *__restrict__ dwte, int d) {
+  const int v = blockIdx.x;
+  const int b = offs[v], e = offs[v + 1];
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float s = 0.f;
-    for (int p = b; p < e; p++) s += dx[(int64_t)order[p] * d + j];
-    dwte[(int64_t)v * d + j] = s;
+    float sum = 0.f;
+    for (int p = b; p < e; p++) sum += dx[(int64_t)order[p] * d + j];
+    dwte[(int64_t)v * d + j] = sum;
   }
 }
 int64_t embed_bwd_scratch_ints(int64_t N, int V) {
@@ -562,7 +694,10 @@ void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int 
     vin = nv;
   }
   k_scan_excl<<<1, 1024, 0, s>>>(offs, V + 1);
-  k_embed_rows<<<V, min(256, ((d + 31) / 32) * 32), 0, s>>>(vin, offs, dx, dwte, d);
+  if ((d & 3) == 0 && ((uintptr_t)dx & 15) == 0 && ((uintptr_t)dwte & 15) == 0)
+    k_embed_rows<<<dim3(V, cdiv(d, 256)), 64, 0, s>>>(vin, offs, dx, dwte, d);
+  else
+    k_embed_rows_scalar<<<V, min(256, ((d + 31) / 32) * 32), 0, s>>>(vin, offs, dx, dwte, d);
   count_launch(2);
 }
 

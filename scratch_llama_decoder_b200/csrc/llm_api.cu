@@ -472,8 +472,7 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
          nullptr, 0, 1, 2.0 * N * d * d);
     wgrad(c, o, d, dxop, d, d, d, gr + O.wo(l), d, d, 0);
     attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
-                  s);
-    rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);
+                  c->cos_t, c->sin_t, s);
     gemm(c, GemmOperands{(int)N, D.d, (int)D.qkvw, c->dqkv, D.qkvw, true, wqkv, D.qkvw, true,
                          D.dt},
          OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.qkvw * d);
@@ -627,7 +626,7 @@ extern "C" int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o,
   if (tensor_cores) {
     if (!attn_mma_covers(DT_BF16, head_dim)) return LLM_ERR_ARG;
     attn_bwd_mma(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, batch, ctx, n_head, n_kv_head, head_dim,
-                 s);
+                 nullptr, nullptr, s);
   } else {
     attn_bwd_simt(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, DT_BF16, batch, ctx, n_head, n_kv_head,
                   head_dim, s);
