@@ -4,13 +4,18 @@ import numpy as np
 import torch
 
 # Tolerances of the training step (norm-wise relative error per tensor).
-#   fp32 configs: loss and logits 1e-4; gradients, updated parameters and the
-#   Adam moments 1e-3.
+#   fp32 configs: loss and logits 1e-4; gradients, updated parameters, the
+#   Adam moments and the update itself 1e-3.
 #   bf16 configs: loss 5e-3; logits, gradients and m 2e-2; v = (1-b2) g^2
-#   carries twice the relative error of g, so v gets 4e-2.
+#   carries twice the relative error of g, so v gets 4e-2.  The updated
+#   parameters are measured but not gated: at t = 1 AdamW moves each element
+#   by about lr * sign(g), so every gradient element within bf16 rounding of
+#   zero can flip a whole 2*lr step (2% of W2 at the 350M workload, whose
+#   scaled init is 0.003 against lr 3e-4).  AdamW is gated there through m and
+#   v, and exactly through the fp32 workloads.
 TOL = {
     "fp32": dict(loss=1e-4, logits=1e-4, grads=1e-3, params=1e-3, m=1e-3, v=1e-3, dp=1e-3),
-    "bf16": dict(loss=5e-3, logits=2e-2, grads=2e-2, params=2e-2, m=2e-2, v=4e-2, dp=None),
+    "bf16": dict(loss=5e-3, logits=2e-2, grads=2e-2, params=None, m=2e-2, v=4e-2, dp=None),
 }
 
 
@@ -82,7 +87,8 @@ def compare(cfg, layout, gpu, ref, prev_params=None, tol=None):
                 sl = slice(off, off + rows * cols)
                 e = rel(g[key][sl], r[key][sl])
                 worst[key] = max(worst.get(key, 0.0), e)
-                assert e <= tol[key], (k, key, name, e)
+                if tol[key] is not None:
+                    assert e <= tol[key], (k, key, name, e)
         if tol.get("dp") is not None and p_prev is not None:
             for name, off, rows, cols in layout:
                 sl = slice(off, off + rows * cols)

@@ -68,5 +68,6 @@ def test_full_size_step_matches_oracle_samples(name):
                               ("m", mn, z["m_val"]), ("v", vn, z["v_val"])):
             e = _rel(got[sl], ref[sl])
             worst[key] = max(worst[key], e)
-            assert e <= tol[key], (str(z["names"][k]), key, e)
+            if tol[key] is not None:
+                assert e <= tol[key], (str(z["names"][k]), key, e)
     print(cfg["name"], errs, worst)
