@@ -86,10 +86,12 @@ def compare(cfg, layout, gpu, ref, prev_params=None, tol=None):
     gp = np.asarray(prev_params, np.float64)
     gm = np.zeros_like(gp)
     gv = np.zeros_like(gp)
+    # the C ABI passes lr, wd, betas and eps as float32: use those values
+    f32 = lambda x: float(np.float32(x))
+    hyp = [f32(cfg[k]) for k in ("lr", "wd", "beta1", "beta2", "adam_eps")]
     for k, (g, r) in enumerate(zip(gpu["steps"], ref["steps"])):
         # AdamW in isolation: oracle AdamW on the GPU's own inputs
-        ep, em, ev = O.adamw(gp, g["grads"], gm, gv, k + 1, cfg["lr"], cfg["wd"], cfg["beta1"],
-                             cfg["beta2"], cfg["adam_eps"])
+        ep, em, ev = O.adamw(gp, g["grads"], gm, gv, k + 1, *hyp)
         for name, off, rows, cols in layout:
             sl = slice(off, off + rows * cols)
             e = rel(g["params"][sl] - gp[sl], ep[sl] - gp[sl])
