@@ -32,7 +32,7 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int STAGING_BYTES = 4 * 32 * 33 * 4;  // epilogue transpose squares, 4 warps
+constexpr int STAGING_BYTES = 4 * 32 * 36 * 4;  // epilogue transpose squares, 4 warps
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + STAGING_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 192;
@@ -170,38 +170,58 @@ LLM_DEV void load32_bf16(const __nv_bfloat16 *src, float (&v)[32], int nvalid) {
   }
 }
 
-// Coalesced write-out of a warp's 32 x 32 chunk: lane i holds row i in v;
-// the chunk goes through a padded shared-memory square (33 floats per row, so
-// both the row-wise writes and the column-wise reads hit 32 distinct banks)
-// and leaves one row per store instruction.  rows / cols clip the edges.
-LLM_DEV void put32_f32(float (*stg)[33], const float (&v)[32], float *dst, int64_t ld, int rows,
-                       int cols, const float *R, int64_t ldr) {
+// Coalesced write-out of a warp's 32 x 32 chunk: lane i holds row i in v.
+// The chunk goes through a shared-memory square with rows padded to 36 floats
+// (16-byte aligned; the 8 lanes of each 128-bit access phase hit 32 distinct
+// banks), written with 16-byte row-wise stores and read back 4 rows per
+// instruction (8 lanes x 4 floats per row), so each global store instruction
+// covers 4 full row segments.  rows / cols clip the edges.
+constexpr int STG_LD = 36;
+LLM_DEV void stage32(float (*stg)[STG_LD], const float (&v)[32]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < 32; i++) stg[lane][i] = v[i];
+  for (int i = 0; i < 32; i += 4)
+    *reinterpret_cast<float4 *>(&stg[lane][i]) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
   __syncwarp();
-  if (lane < cols) {
-    for (int r = 0; r < rows; r++) {
-      float x = stg[r][lane];
-      if (R) x += R[(int64_t)r * ldr + lane];
-      dst[(int64_t)r * ld + lane] = x;
+}
+LLM_DEV void put32_f32(float (*stg)[STG_LD], const float (&v)[32], float *dst, int64_t ld,
+                       int rows, int cols, const float *R, int64_t ldr) {
+  stage32(stg, v);
+  const int lane = threadIdx.x & 31;
+  const int c = 4 * (lane & 7), rsub = lane >> 3;
+  if (c < cols) {
+    for (int r = rsub; r < rows; r += 4) {
+      float4 x = *reinterpret_cast<const float4 *>(&stg[r][c]);
+      if (c + 4 <= cols) {
+        if (R) {
+          float4 q = *reinterpret_cast<const float4 *>(R + (int64_t)r * ldr + c);
+          x.x += q.x; x.y += q.y; x.z += q.z; x.w += q.w;
+        }
+        *reinterpret_cast<float4 *>(dst + (int64_t)r * ld + c) = x;
+      } else {
+        float e[4] = {x.x, x.y, x.z, x.w};
+        for (int k = 0; c + k < cols; k++)
+          dst[(int64_t)r * ld + c + k] = e[k] + (R ? R[(int64_t)r * ldr + c + k] : 0.f);
+      }
     }
   }
   __syncwarp();
 }
-LLM_DEV void put32_bf16(float (*stg)[33], const float (&v)[32], __nv_bfloat16 *dst, int64_t ld,
+LLM_DEV void put32_bf16(float (*stg)[STG_LD], const float (&v)[32], __nv_bfloat16 *dst, int64_t ld,
                         int rows, int cols) {
+  stage32(stg, v);
   const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int i = 0; i < 32; i++) stg[lane][i] = v[i];
-  __syncwarp();
-  const int c = 2 * (lane & 15);
+  const int c = 4 * (lane & 7), rsub = lane >> 3;
   if (c < cols) {
-    for (int r = lane >> 4; r < rows; r += 2) {
-      if (c + 1 < cols)
-        *reinterpret_cast<uint32_t *>(dst + (int64_t)r * ld + c) = pack_bf16(stg[r][c], stg[r][c + 1]);
-      else
-        dst[(int64_t)r * ld + c] = __float2bfloat16_rn(stg[r][c]);
+    for (int r = rsub; r < rows; r += 4) {
+      float4 x = *reinterpret_cast<const float4 *>(&stg[r][c]);
+      if (c + 4 <= cols) {
+        *reinterpret_cast<uint2 *>(dst + (int64_t)r * ld + c) =
+            make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+      } else {
+        float e[4] = {x.x, x.y, x.z, x.w};
+        for (int k = 0; c + k < cols; k++) dst[(int64_t)r * ld + c + k] = __float2bfloat16_rn(e[k]);
+      }
     }
   }
   __syncwarp();
@@ -212,7 +232,7 @@ LLM_DEV void put32_bf16(float (*stg)[33], const float (&v)[32], __nv_bfloat16 *d
 // [n0, n0+BN).  Every lane executes every tcgen05.ld (warp-uniform control);
 // rows past M are clipped only at the stores.
 LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int split, bool zero,
-                           float (*stg)[33]) {
+                           float (*stg)[STG_LD]) {
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
   const bool row_ok = m < a.M;
@@ -466,7 +486,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // -------------------------------------------------- epilogue warps
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-    float (*stg)[33] = reinterpret_cast<float (*)[33]>(smem + STAGES * STAGE_BYTES + 256) +
+    float (*stg)[STG_LD] = reinterpret_cast<float (*)[STG_LD]>(smem + STAGES * STAGE_BYTES + 256) +
                        (warp - 2) * 32;
     int acc = 0;
     uint32_t aph = 0;
