@@ -49,6 +49,13 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kernel", default=None, choices=["gemm", "attention"],
+                    help="time one hot-path kernel through the C ABI instead of the step")
+    ap.add_argument("--shape", default="16384,3072,1024",
+                    help="gemm: M,N,K; attention: batch,ctx,n_head,n_kv_head,head_dim")
+    ap.add_argument("--orient", default="kn", choices=["kn", "kk", "nn"],
+                    help="gemm operand majorness: kn = x.W (forward), kk = dy.W^T (dgrad), "
+                         "nn = x^T.dy (wgrad)")
     return ap.parse_args()
 
 
@@ -326,8 +333,57 @@ def run_reference(args, rank):
     }
 
 
+def run_kernel(args):
+    """Device time of one hot-path kernel shape (CUDA events, after warm-up)."""
+    import ctypes as C
+    import torch
+    import scratch_llama_decoder_b200 as P
+    torch.cuda.set_device(0)
+    p = lambda t: C.c_void_p(t.data_ptr())
+    g = torch.Generator(device="cuda").manual_seed(0)
+    if args.kernel == "gemm":
+        M, N, K = (int(x) for x in args.shape.split(","))
+        ak, bk = {"kn": (1, 0), "kk": (1, 1), "nn": (0, 0)}[args.orient]
+        A = torch.randn((M, K) if ak else (K, M), device="cuda", generator=g).to(torch.bfloat16)
+        B = torch.randn((N, K) if bk else (K, N), device="cuda", generator=g).to(torch.bfloat16)
+        Cm = torch.empty(M, N, device="cuda")
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+        def call():
+            rc = P.lib.llm_kernel_gemm_bf16(M, N, K, p(A), A.shape[1], ak, p(B), B.shape[1], bk,
+                                            p(Cm), N, 1, p(flag), None)
+            assert rc == 0
+        flops = 2.0 * M * N * K
+    else:
+        Bt, T, H, Hkv, hd = (int(x) for x in args.shape.split(","))
+        w = (H + 2 * Hkv) * hd
+        qkv = torch.randn(Bt * T, w, device="cuda", generator=g).to(torch.bfloat16)
+        o = torch.empty(Bt * T, H * hd, device="cuda", dtype=torch.bfloat16)
+        lse = torch.empty(Bt, H, T, device="cuda")
+
+        def call():
+            assert P.lib.llm_kernel_attention_fwd_bf16(p(qkv), p(o), p(lse), Bt, T, H, Hkv, hd, 1,
+                                                       None) == 0
+        flops = 4.0 * Bt * H * (T * (T + 1) / 2) * hd
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"kernel": args.kernel, "shape": args.shape, "orient": args.orient,
+                      "ms": ms, "tflops": flops / (ms / 1e3) / 1e12}), flush=True)
+
+
 def main():
     args = parse()
+    if args.kernel:
+        run_kernel(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
