@@ -152,24 +152,6 @@ LLM_DEV uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
 }
-LLM_DEV void load32_bf16(const __nv_bfloat16 *src, float (&v)[32], int nvalid) {
-  if (nvalid >= 32) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-      uint4 q = *reinterpret_cast<const uint4 *>(src + i);
-      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&q);
-#pragma unroll
-      for (int k = 0; k < 4; k++) {
-        float2 f = __bfloat1622float2(h[k]);
-        v[i + 2 * k] = f.x;
-        v[i + 2 * k + 1] = f.y;
-      }
-    }
-  } else {
-    for (int i = 0; i < 32; i++) v[i] = (i < nvalid) ? __bfloat162float(src[i]) : 0.f;
-  }
-}
-
 // Coalesced write-out of a warp's 32 x 32 chunk: lane i holds row i in v.
 // The chunk goes through a shared-memory square with rows padded to 36 floats
 // (16-byte aligned; the 8 lanes of each 128-bit access phase hit 32 distinct
@@ -227,6 +209,33 @@ LLM_DEV void put32_bf16(float (*stg)[STG_LD], const float (&v)[32], __nv_bfloat1
   __syncwarp();
 }
 
+// The reverse of put32_*: a warp's 32 rows x 32 bf16 columns of a
+// row-major matrix, read 4 rows per instruction (coalesced) into the staging
+// square, then handed out one row per lane (v[i] = row `lane`, column i).
+LLM_DEV void get32_bf16(float (*stg)[STG_LD], const __nv_bfloat16 *src, int64_t ld, int rows,
+                        float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  const int c = 4 * (lane & 7), rsub = lane >> 3;
+#pragma unroll
+  for (int r = rsub; r < 32; r += 4) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < rows) {
+      uint2 q = *reinterpret_cast<const uint2 *>(src + (int64_t)r * ld + c);
+      float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q.x));
+      float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q.y));
+      x = make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+    *reinterpret_cast<float4 *>(&stg[r][c]) = x;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    float4 x = *reinterpret_cast<const float4 *>(&stg[lane][i]);
+    v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+  }
+  __syncwarp();
+}
+
 // One output tile's epilogue for a warp: rows [row0, row0+32) of the tile
 // (TMEM lanes of this warp's quarter, lane i = row row0 + i), columns
 // [n0, n0+BN).  Every lane executes every tcgen05.ld (warp-uniform control);
@@ -235,7 +244,6 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
                            float (*stg)[STG_LD]) {
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
-  const bool row_ok = m < a.M;
   const int rows = max(0, min(32, a.M - row0));
   const int N = a.N;
   auto ncols = [&](int n) { return max(0, min(32, N - n)); };
@@ -252,12 +260,19 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
         if (zero) { for (int i = 0; i < 32; i++) lo[i] = hi[i] = 0.f; }
         else { tmem_ld32(tm + c0, lo); tmem_ld32(tm + c0 + 32, hi); }
         if (n < a.rot_cols) {
-          const float *ct = a.cos_t + (int64_t)t * half, *st = a.sin_t + (int64_t)t * half;
+          const float4 *ct = reinterpret_cast<const float4 *>(a.cos_t + (int64_t)t * half);
+          const float4 *st = reinterpret_cast<const float4 *>(a.sin_t + (int64_t)t * half);
 #pragma unroll
-          for (int j = 0; j < 32; j++) {
-            float c = ct[j], s = st[j], x = lo[j], y = hi[j];
-            lo[j] = x * c - y * s;
-            hi[j] = y * c + x * s;
+          for (int j4 = 0; j4 < 8; j4++) {
+            float4 c4 = ct[j4], s4 = st[j4];
+            const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+              int j = 4 * j4 + k;
+              float x = lo[j], y = hi[j];
+              lo[j] = x * cc[k] - y * ss[k];
+              hi[j] = y * cc[k] + x * ss[k];
+            }
           }
         }
         put32_bf16(stg, lo, C + n, a.ldc, rows, ncols(n));
@@ -270,12 +285,19 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
         if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
         else tmem_ld32(tm + c0, v);
         if (n < a.rot_cols) {
-          const float *ct = a.cos_t + (int64_t)t * half, *st = a.sin_t + (int64_t)t * half;
+          const float4 *ct = reinterpret_cast<const float4 *>(a.cos_t + (int64_t)t * half);
+          const float4 *st = reinterpret_cast<const float4 *>(a.sin_t + (int64_t)t * half);
 #pragma unroll
-          for (int j = 0; j < 16; j++) {
-            float c = ct[j], s = st[j], x = v[j], y = v[j + 16];
-            v[j] = x * c - y * s;
-            v[j + 16] = y * c + x * s;
+          for (int j4 = 0; j4 < 4; j4++) {
+            float4 c4 = ct[j4], s4 = st[j4];
+            const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+              int j = 4 * j4 + k;
+              float x = v[j], y = v[j + 16];
+              v[j] = x * cc[k] - y * ss[k];
+              v[j + 16] = y * cc[k] + x * ss[k];
+            }
           }
         }
         put32_bf16(stg, v, C + n, a.ldc, rows, ncols(n));
@@ -297,7 +319,7 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
         put32_bf16(stg, av, C + n + q, a.ldc, rows, 32);
         put32_bf16(stg, bv, C + n + SWIGLU_BLOCK + q, a.ldc, rows, 32);
 #pragma unroll
-        for (int i = 0; i < 32; i++) av[i] = av[i] / (1.f + expf(-av[i])) * bv[i];
+        for (int i = 0; i < 32; i++) av[i] = av[i] / (1.f + __expf(-av[i])) * bv[i];
         put32_bf16(stg, av, U + (n / (2 * SWIGLU_BLOCK)) * SWIGLU_BLOCK + q, a.ld_aux, rows, 32);
       }
     }
@@ -306,7 +328,7 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
   if (a.epi == TC_EPI_SWIGLU_BWD) {
     // acc = du for hidden units [n0, n0+BN); write [da|db] at their
     // interleaved columns using the saved [a|b].
-    const __nv_bfloat16 *AB = (const __nv_bfloat16 *)a.aux + (int64_t)m * a.ld_aux;
+    const __nv_bfloat16 *AB = (const __nv_bfloat16 *)a.aux + (int64_t)row0 * a.ld_aux;
     __nv_bfloat16 *D = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
     for (int c0 = 0; c0 < BN; c0 += 32) {
       int j = n0 + c0;
@@ -315,11 +337,11 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
       else tmem_ld32(tm + c0, v);
       int64_t ca = w1_col(j);
       float av[32], bv[32];
-      load32_bf16(AB + ca, av, row_ok ? 32 : 0);
-      load32_bf16(AB + ca + SWIGLU_BLOCK, bv, row_ok ? 32 : 0);
+      get32_bf16(stg, AB + ca, a.ld_aux, rows, av);
+      get32_bf16(stg, AB + ca + SWIGLU_BLOCK, a.ld_aux, rows, bv);
 #pragma unroll
       for (int i = 0; i < 32; i++) {
-        float s = 1.f / (1.f + expf(-av[i]));
+        float s = 1.f / (1.f + __expf(-av[i]));
         float du = v[i];
         float da = du * bv[i] * s * (1.f + av[i] * (1.f - s));
         bv[i] = du * av[i] * s;
