@@ -168,22 +168,32 @@ LLM_DEV void stage32(float (*stg)[STG_LD], const float (&v)[32]) {
 }
 LLM_DEV void put32_f32(float (*stg)[STG_LD], const float (&v)[32], float *dst, int64_t ld,
                        int rows, int cols, const float *R, int64_t ldr) {
-  stage32(stg, v);
   const int lane = threadIdx.x & 31;
   const int c = 4 * (lane & 7), rsub = lane >> 3;
+  const bool full = c + 4 <= cols;
+  // residual rows first: all eight 16-byte loads in flight before any
+  // shared-memory traffic (generic pointers would otherwise serialise them)
+  float4 rv[8];
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const int r = rsub + 4 * k;
+    rv[k] = (R && full && r < rows) ? *reinterpret_cast<const float4 *>(R + (int64_t)r * ldr + c)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  stage32(stg, v);
   if (c < cols) {
-    for (int r = rsub; r < rows; r += 4) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const int r = rsub + 4 * k;
+      if (r >= rows) break;
       float4 x = *reinterpret_cast<const float4 *>(&stg[r][c]);
-      if (c + 4 <= cols) {
-        if (R) {
-          float4 q = *reinterpret_cast<const float4 *>(R + (int64_t)r * ldr + c);
-          x.x += q.x; x.y += q.y; x.z += q.z; x.w += q.w;
-        }
+      if (full) {
+        x.x += rv[k].x; x.y += rv[k].y; x.z += rv[k].z; x.w += rv[k].w;
         *reinterpret_cast<float4 *>(dst + (int64_t)r * ld + c) = x;
       } else {
         float e[4] = {x.x, x.y, x.z, x.w};
-        for (int k = 0; c + k < cols; k++)
-          dst[(int64_t)r * ld + c + k] = e[k] + (R ? R[(int64_t)r * ldr + c + k] : 0.f);
+        for (int q = 0; c + q < cols; q++)
+          dst[(int64_t)r * ld + c + q] = e[q] + (R ? R[(int64_t)r * ldr + c + q] : 0.f);
       }
     }
   }
@@ -195,14 +205,17 @@ LLM_DEV void put32_bf16(float (*stg)[STG_LD], const float (&v)[32], __nv_bfloat1
   const int lane = threadIdx.x & 31;
   const int c = 4 * (lane & 7), rsub = lane >> 3;
   if (c < cols) {
-    for (int r = rsub; r < rows; r += 4) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const int r = rsub + 4 * k;
+      if (r >= rows) break;
       float4 x = *reinterpret_cast<const float4 *>(&stg[r][c]);
       if (c + 4 <= cols) {
         *reinterpret_cast<uint2 *>(dst + (int64_t)r * ld + c) =
             make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
       } else {
         float e[4] = {x.x, x.y, x.z, x.w};
-        for (int k = 0; c + k < cols; k++) dst[(int64_t)r * ld + c + k] = __float2bfloat16_rn(e[k]);
+        for (int q = 0; c + q < cols; q++) dst[(int64_t)r * ld + c + q] = __float2bfloat16_rn(e[q]);
       }
     }
   }
@@ -216,16 +229,18 @@ LLM_DEV void get32_bf16(float (*stg)[STG_LD], const __nv_bfloat16 *src, int64_t 
                         float (&v)[32]) {
   const int lane = threadIdx.x & 31;
   const int c = 4 * (lane & 7), rsub = lane >> 3;
+  uint2 q[8];
 #pragma unroll
-  for (int r = rsub; r < 32; r += 4) {
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < rows) {
-      uint2 q = *reinterpret_cast<const uint2 *>(src + (int64_t)r * ld + c);
-      float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q.x));
-      float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q.y));
-      x = make_float4(lo.x, lo.y, hi.x, hi.y);
-    }
-    *reinterpret_cast<float4 *>(&stg[r][c]) = x;
+  for (int k = 0; k < 8; k++) {  // all loads in flight first
+    const int r = rsub + 4 * k;
+    q[k] = (r < rows) ? *reinterpret_cast<const uint2 *>(src + (int64_t)r * ld + c)
+                      : make_uint2(0u, 0u);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q[k].x));
+    float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q[k].y));
+    *reinterpret_cast<float4 *>(&stg[rsub + 4 * k][c]) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
   __syncwarp();
 #pragma unroll
