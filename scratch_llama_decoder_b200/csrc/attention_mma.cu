@@ -99,14 +99,15 @@ LLM_DEV void load_afrag(const Tile<HD> &t, int w, uint32_t (&f)[HD / 16][4]) {
   }
 }
 
-// acc[16 x 64] += A[16 x HD] . X^T where X is a 64 x HD tile (rows = n):
-// B(k, n) = X[n][k], loaded without transpose.
-template <int HD>
-LLM_DEV void mma_abt(float (&acc)[8][4], const uint32_t (&a)[HD / 16][4], const Tile<HD> &x) {
+// acc[16 x 8*NT] += A[16 x HD] . X^T over rows [x0, x0 + 8*NT) of a 64 x HD
+// tile X (rows = n): B(k, n) = X[x0 + n][k], loaded without transpose.
+template <int HD, int NT = 8>
+LLM_DEV void mma_abt(float (&acc)[NT][4], const uint32_t (&a)[HD / 16][4], const Tile<HD> &x,
+                     int x0 = 0) {
   int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int np = 0; np < 4; np++) {  // pairs of 8-wide n tiles
-    int row = np * 16 + (lane & 7) + (lane >> 4) * 8;
+  for (int np = 0; np < NT / 2; np++) {  // pairs of 8-wide n tiles
+    int row = x0 + np * 16 + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
     for (int k = 0; k < HD / 16; k++) {
       int col = k * 16 + ((lane >> 3) & 1) * 8;
@@ -118,14 +119,16 @@ LLM_DEV void mma_abt(float (&acc)[8][4], const uint32_t (&a)[HD / 16][4], const 
   }
 }
 
-// acc[16 x HD] += P[16 x 64] . Y where Y is a 64 x HD tile (rows = k):
-// B(k, n) = Y[k][n], loaded with transpose.  p: A fragments of P (4 k-steps).
-template <int HD>
-LLM_DEV void mma_ab(float (&acc)[HD / 8][4], const uint32_t (&p)[4][4], const Tile<HD> &y) {
+// acc[16 x HD] += P[16 x 16*KS] . Y over rows [y0, y0 + 16*KS) of a 64 x HD
+// tile Y (rows = k): B(k, n) = Y[y0 + k][n], loaded with transpose.
+// p: A fragments of P (KS k-steps).
+template <int HD, int KS = 4>
+LLM_DEV void mma_ab(float (&acc)[HD / 8][4], const uint32_t (&p)[KS][4], const Tile<HD> &y,
+                    int y0 = 0) {
   int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int k = 0; k < 4; k++) {
-    int row = k * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  for (int k = 0; k < KS; k++) {
+    int row = y0 + k * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
     for (int np = 0; np < HD / 16; np++) {
       int col = np * 16 + (lane >> 4) * 8;
@@ -137,10 +140,11 @@ LLM_DEV void mma_ab(float (&acc)[HD / 8][4], const uint32_t (&p)[4][4], const Ti
   }
 }
 
-// C fragments of a 16 x 64 fp32 tile -> A fragments (bf16) over its 64 columns.
-LLM_DEV void c_to_a(const float (&s)[8][4], uint32_t (&p)[4][4]) {
+// C fragments of a 16 x 8*NT fp32 tile -> A fragments (bf16) over its columns.
+template <int NT = 8>
+LLM_DEV void c_to_a(const float (&s)[NT][4], uint32_t (&p)[NT / 2][4]) {
 #pragma unroll
-  for (int k = 0; k < 4; k++) {
+  for (int k = 0; k < NT / 2; k++) {
     p[k][0] = pack2(s[2 * k][0], s[2 * k][1]);
     p[k][1] = pack2(s[2 * k][2], s[2 * k][3]);
     p[k][2] = pack2(s[2 * k + 1][0], s[2 * k + 1][1]);
@@ -173,9 +177,11 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
                                                  float *__restrict__ lse, int T, int H, int Hkv,
                                                  float scale) {
   __shared__ Tile<HD> Qs, Ks[2], Vs[2];
-  const int nqb = gridDim.x;
-  const int qb = nqb - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (H, B, query blocks): blocks are dispatched x-fastest, so the last
+  // (longest) query blocks of every head start first
+  const int nqb = gridDim.z;
+  const int qb = nqb - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / (H / Hkv);
   const int d = H * HD, kvd = Hkv * HD;
   const int64_t ld = d + 2 * kvd;
@@ -284,9 +290,9 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
                                                 int Hkv, float scale) {
   __shared__ Tile<HD> Ks[2], Vs[2];
   __shared__ float Dsh[64];
-  const int nqb = gridDim.x;
-  const int qb = nqb - 1 - blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int nqb = gridDim.z;
+  const int qb = nqb - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / (H / Hkv);
   const int d = H * HD, kvd = Hkv * HD;
   const int64_t ld = d + 2 * kvd;
@@ -403,9 +409,11 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
                                                  int Hkv, float scale) {
   __shared__ Tile<HD> KVs, Qs[2], dOs[2];
   __shared__ float Ls[2][64], Ds[2][64];
-  const int nkb = gridDim.x;
-  const int kb = blockIdx.x;  // early key blocks see the most query blocks: start them first
-  const int g = blockIdx.y, b = blockIdx.z;
+  // grid (Hkv, B, key blocks): the first key blocks see the most query
+  // blocks, and blocks are dispatched x-fastest, so they start first
+  const int nkb = gridDim.z;
+  const int kb = blockIdx.z;
+  const int g = blockIdx.x, b = blockIdx.y;
   const int grp = H / Hkv;
   const int d = H * HD, kvd = Hkv * HD;
   const int64_t ld = d + 2 * kvd;
@@ -456,32 +464,36 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
     cp_commit();
     cp_wait<1>();
     __syncthreads();
-    // S^T = K Q^T, dP^T = V dO^T  (16 keys x 64 queries per warp)
-    float s[8][4], dp[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; i++)
-#pragma unroll
-      for (int e = 0; e < 4; e++) s[i][e] = dp[i][e] = 0.f;
-    mma_abt<HD>(s, kf, Qs[cur]);
-    mma_abt<HD>(dp, vf, dOs[cur]);
+    // Two halves of 32 queries: S^T = K Q^T and dP^T = V dO^T (16 keys x 32
+    // queries per warp), then dV += P^T dO and dK += dS^T Q over that half.
     const int q0 = qb * BQ;
 #pragma unroll
-    for (int nt = 0; nt < 8; nt++) {
+    for (int hf = 0; hf < 2; hf++) {
+      float s[4][4], dp[4][4];
 #pragma unroll
-      for (int e = 0; e < 4; e++) {
-        int kj = key0 + (e >> 1) * 8;
-        int col = nt * 8 + (lane & 3) * 2 + (e & 1);
-        int qi = q0 + col;
-        float p = (kj > qi || qi >= T || kj >= T) ? 0.f : exp2f(s[nt][e] * sl2 - Ls[cur][col]);
-        s[nt][e] = p;                              // P^T
-        dp[nt][e] = p * (dp[nt][e] - Ds[cur][col]);  // dS^T
+      for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) s[i][e] = dp[i][e] = 0.f;
+      mma_abt<HD, 4>(s, kf, Qs[cur], hf * 32);
+      mma_abt<HD, 4>(dp, vf, dOs[cur], hf * 32);
+#pragma unroll
+      for (int nt = 0; nt < 4; nt++) {
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          int kj = key0 + (e >> 1) * 8;
+          int col = hf * 32 + nt * 8 + (lane & 3) * 2 + (e & 1);
+          int qi = q0 + col;
+          float p = (kj > qi || qi >= T || kj >= T) ? 0.f : exp2f(s[nt][e] * sl2 - Ls[cur][col]);
+          s[nt][e] = p;                                // P^T
+          dp[nt][e] = p * (dp[nt][e] - Ds[cur][col]);  // dS^T
+        }
       }
+      uint32_t pf[2][4], sf[2][4];
+      c_to_a<4>(s, pf);
+      c_to_a<4>(dp, sf);
+      mma_ab<HD, 2>(dv, pf, dOs[cur], hf * 32);
+      mma_ab<HD, 2>(dk, sf, Qs[cur], hf * 32);
     }
-    uint32_t pf[4][4], sf[4][4];
-    c_to_a(s, pf);
-    c_to_a(dp, sf);
-    mma_ab<HD>(dv, pf, dOs[cur]);
-    mma_ab<HD>(dk, sf, Qs[cur]);
     __syncthreads();
   }
 #pragma unroll
@@ -506,7 +518,7 @@ bool attn_mma_covers(DType dt, int hd) { return dt == DT_BF16 && (hd == 32 || hd
 void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
                   cudaStream_t s) {
   using namespace attn;
-  dim3 grid((T + BQ - 1) / BQ, H, B);
+  dim3 grid(H, B, (T + BQ - 1) / BQ);
   float scale = 1.0f / sqrtf((float)hd);
   if (hd == 64)
     k_attn_fwd<64><<<grid, NT, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, T, H,
@@ -525,7 +537,7 @@ void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float 
   const __nv_bfloat16 *q = (const __nv_bfloat16 *)qkv, *oo = (const __nv_bfloat16 *)o,
                       *dO = (const __nv_bfloat16 *)dout;
   __nv_bfloat16 *dq = (__nv_bfloat16 *)dqkv;
-  dim3 gq((T + BQ - 1) / BQ, H, B), gkv((T + BKV - 1) / BKV, Hkv, B);
+  dim3 gq(H, B, (T + BQ - 1) / BQ), gkv(Hkv, B, (T + BKV - 1) / BKV);
   if (hd == 64) {
     k_attn_dq<64><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
     k_attn_dkv<64><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);

@@ -166,21 +166,25 @@ LLM_DEV void stage32(float (*stg)[STG_LD], const float (&v)[32]) {
     *reinterpret_cast<float4 *>(&stg[lane][i]) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
   __syncwarp();
 }
-LLM_DEV void put32_f32(float (*stg)[STG_LD], const float (&v)[32], float *dst, int64_t ld,
-                       int rows, int cols, const float *R, int64_t ldr) {
+// Rows of the warp's 32-row slab, 4 columns per lane (lane&7), 4 rows per
+// instruction: the residual values put32_f32 will add, loaded ahead of use.
+LLM_DEV void ld32_f32(const float *R, int64_t ldr, int rows, int cols, float4 (&rv)[8]) {
   const int lane = threadIdx.x & 31;
   const int c = 4 * (lane & 7), rsub = lane >> 3;
   const bool full = c + 4 <= cols;
-  // residual rows first: all eight 16-byte loads in flight before any
-  // shared-memory traffic (generic pointers would otherwise serialise them)
-  float4 rv[8];
 #pragma unroll
   for (int k = 0; k < 8; k++) {
     const int r = rsub + 4 * k;
     rv[k] = (R && full && r < rows) ? *reinterpret_cast<const float4 *>(R + (int64_t)r * ldr + c)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+LLM_DEV void put32_f32(float (*stg)[STG_LD], const float (&v)[32], float *dst, int64_t ld,
+                       int rows, int cols, const float *R, int64_t ldr, const float4 (&rv)[8]) {
   stage32(stg, v);
+  const int lane = threadIdx.x & 31;
+  const int c = 4 * (lane & 7), rsub = lane >> 3;
+  const bool full = c + 4 <= cols;
   if (c < cols) {
 #pragma unroll
     for (int k = 0; k < 8; k++) {
@@ -225,17 +229,19 @@ LLM_DEV void put32_bf16(float (*stg)[STG_LD], const float (&v)[32], __nv_bfloat1
 // The reverse of put32_*: a warp's 32 rows x 32 bf16 columns of a
 // row-major matrix, read 4 rows per instruction (coalesced) into the staging
 // square, then handed out one row per lane (v[i] = row `lane`, column i).
-LLM_DEV void get32_bf16(float (*stg)[STG_LD], const __nv_bfloat16 *src, int64_t ld, int rows,
-                        float (&v)[32]) {
+LLM_DEV void ld32_bf16(const __nv_bfloat16 *src, int64_t ld, int rows, uint2 (&q)[8]) {
   const int lane = threadIdx.x & 31;
   const int c = 4 * (lane & 7), rsub = lane >> 3;
-  uint2 q[8];
 #pragma unroll
-  for (int k = 0; k < 8; k++) {  // all loads in flight first
+  for (int k = 0; k < 8; k++) {
     const int r = rsub + 4 * k;
     q[k] = (r < rows) ? *reinterpret_cast<const uint2 *>(src + (int64_t)r * ld + c)
                       : make_uint2(0u, 0u);
   }
+}
+LLM_DEV void unstage32_bf16(float (*stg)[STG_LD], const uint2 (&q)[8], float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  const int c = 4 * (lane & 7), rsub = lane >> 3;
 #pragma unroll
   for (int k = 0; k < 8; k++) {
     float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q[k].x));
@@ -342,9 +348,15 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
   }
   if (a.epi == TC_EPI_SWIGLU_BWD) {
     // acc = du for hidden units [n0, n0+BN); write [da|db] at their
-    // interleaved columns using the saved [a|b].
+    // interleaved columns using the saved [a|b].  The saved values of the
+    // next 32-column chunk are loaded while this chunk is computed.
     const __nv_bfloat16 *AB = (const __nv_bfloat16 *)a.aux + (int64_t)row0 * a.ld_aux;
     __nv_bfloat16 *D = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
+    uint2 qa[8], qb[8];
+    if (n0 < N) {
+      ld32_bf16(AB + w1_col(n0), a.ld_aux, rows, qa);
+      ld32_bf16(AB + w1_col(n0) + SWIGLU_BLOCK, a.ld_aux, rows, qb);
+    }
     for (int c0 = 0; c0 < BN; c0 += 32) {
       int j = n0 + c0;
       if (j >= N) break;
@@ -352,8 +364,12 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
       else tmem_ld32(tm + c0, v);
       int64_t ca = w1_col(j);
       float av[32], bv[32];
-      get32_bf16(stg, AB + ca, a.ld_aux, rows, av);
-      get32_bf16(stg, AB + ca + SWIGLU_BLOCK, a.ld_aux, rows, bv);
+      unstage32_bf16(stg, qa, av);
+      unstage32_bf16(stg, qb, bv);
+      if (c0 + 32 < BN && j + 32 < N) {
+        ld32_bf16(AB + w1_col(j + 32), a.ld_aux, rows, qa);
+        ld32_bf16(AB + w1_col(j + 32) + SWIGLU_BLOCK, a.ld_aux, rows, qb);
+      }
 #pragma unroll
       for (int i = 0; i < 32; i++) {
         float s = 1.f / (1.f + __expf(-av[i]));
@@ -367,7 +383,10 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
     }
     return;
   }
-  // Plain outputs.
+  // Plain outputs (a residual is loaded, all eight rows-groups at once, just
+  // before the chunk is staged).
+  const bool add = a.out == OUT_ADD_F32;
+  const float *Rrow = add ? a.R + (int64_t)row0 * a.ldr : nullptr;
   for (int c0 = 0; c0 < BN; c0 += 32) {
     int n = n0 + c0;
     if (n >= N) break;
@@ -378,8 +397,9 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
     } else {
       float *dst = (float *)a.C + (int64_t)row0 * a.ldc + n;
       if (a.out == OUT_PARTIAL) dst += (int64_t)split * a.M * a.ldc;
-      const float *R = (a.out == OUT_ADD_F32) ? a.R + (int64_t)row0 * a.ldr + n : nullptr;
-      put32_f32(stg, v, dst, a.ldc, rows, ncols(n), R, a.ldr);
+      float4 rv[8];
+      ld32_f32(add ? Rrow + n : nullptr, a.ldr, rows, ncols(n), rv);
+      put32_f32(stg, v, dst, a.ldc, rows, ncols(n), add ? Rrow + n : nullptr, a.ldr, rv);
     }
   }
 }

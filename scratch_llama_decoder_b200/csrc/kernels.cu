@@ -170,6 +170,17 @@ __global__ void k_rmsnorm_bwd(const float *__restrict__ x, const float *__restri
     part[(int64_t)blockIdx.x * d + j] = s;
   }
 }
+// Four values to 4 consecutive elements: one 8-byte store for bf16, one
+// 16-byte store for float (dst aligned to the element group).
+LLM_DEV void store4(__nv_bfloat16 *dst, float4 o) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+  uint2 q;
+  q.x = *reinterpret_cast<uint32_t *>(&lo);
+  q.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = q;
+}
+LLM_DEV void store4(float *dst, float4 o) { *reinterpret_cast<float4 *>(dst) = o; }
+
 // Vectorised form for d = 128 * VPL: each lane owns VPL float4 columns of a
 // row, keeps its gain-gradient partial sums in registers, and the block adds
 // its 8 warps' partials in warp order.
@@ -196,12 +207,14 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bwd_v(const float *__restrict__
     if (row >= N) break;
     const float4 *xr = reinterpret_cast<const float4 *>(x + row * d);
     const float4 *dyr = reinterpret_cast<const float4 *>(dy + row * d);
-    float4 xv[VPL], dv[VPL];
+    float4 xv[VPL], dv[VPL], rv[VPL];
     float dot = 0.f;
 #pragma unroll
     for (int k = 0; k < VPL; k++) {
       xv[k] = xr[lane + 32 * k];
       dv[k] = dyr[lane + 32 * k];
+      rv[k] = dres ? reinterpret_cast<const float4 *>(dres + row * d)[lane + 32 * k]
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
       dot += gv[k].x * dv[k].x * xv[k].x + gv[k].y * dv[k].y * xv[k].y +
              gv[k].z * dv[k].z * xv[k].z + gv[k].w * dv[k].w * xv[k].w;
     }
@@ -215,16 +228,9 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bwd_v(const float *__restrict__
       o.y = r * gv[k].y * dv[k].y - xv[k].y * c;
       o.z = r * gv[k].z * dv[k].z - xv[k].z * c;
       o.w = r * gv[k].w * dv[k].w - xv[k].w * c;
-      if (dres) {
-        float4 q = reinterpret_cast<const float4 *>(dres + row * d)[lane + 32 * k];
-        o.x += q.x; o.y += q.y; o.z += q.z; o.w += q.w;
-      }
+      o.x += rv[k].x; o.y += rv[k].y; o.z += rv[k].z; o.w += rv[k].w;
       reinterpret_cast<float4 *>(dx + row * d)[lane + 32 * k] = o;
-      if (dx_act) {
-        A *dst = dx_act + row * d + 4 * (lane + 32 * k);
-        dst[0] = from_f<A>(o.x); dst[1] = from_f<A>(o.y);
-        dst[2] = from_f<A>(o.z); dst[3] = from_f<A>(o.w);
-      }
+      if (dx_act) store4(dx_act + row * d + 4 * (lane + 32 * k), o);
       acc[k].x += dv[k].x * xv[k].x * r;
       acc[k].y += dv[k].y * xv[k].y * r;
       acc[k].z += dv[k].z * xv[k].z * r;
@@ -401,11 +407,20 @@ __global__ void __launch_bounds__(NT) k_cross_entropy(A *__restrict__ z, const i
   int64_t row = blockIdx.x;
   A *zr = z + row * ldz;
   float m = -INFINITY, s = 0.f;
-  for (int v = threadIdx.x; v < V; v += NT) {
-    float x = to_f(zr[v]);
+  auto acc = [&](float x) {
     if (x > m) { s = s * expf(m - x) + 1.f; m = x; }
     else s += expf(x - m);
+  };
+  constexpr int VW = 16 / sizeof(A);  // elements per 16-byte vector
+  const bool vec = (ldz % VW) == 0 && (((uintptr_t)z) & 15) == 0;
+  const int Vv = vec ? V / VW : 0;    // whole vectors inside [0, V)
+  for (int i = threadIdx.x; i < Vv; i += NT) {
+    uint4 q = reinterpret_cast<const uint4 *>(zr)[i];
+    const A *e = reinterpret_cast<const A *>(&q);
+#pragma unroll
+    for (int k = 0; k < VW; k++) acc(to_f(e[k]));
   }
+  for (int v = Vv * VW + threadIdx.x; v < V; v += NT) acc(to_f(zr[v]));
   // merge (m, s) across the block
   int lane = threadIdx.x & 31, w = threadIdx.x / 32;
   for (int o = 16; o > 0; o >>= 1) {
@@ -429,7 +444,20 @@ __global__ void __launch_bounds__(NT) k_cross_entropy(A *__restrict__ z, const i
   float zy = to_f(zr[y]);
   __syncthreads();  // every thread has read z[y] before it is overwritten
   if (threadIdx.x == 0) rowloss[row] = lse - zy;
-  for (int64_t v = threadIdx.x; v < ldz; v += NT) {
+  const int Lv = vec ? (int)(ldz / VW) : 0;
+  for (int i = threadIdx.x; i < Lv; i += NT) {
+    uint4 q = reinterpret_cast<const uint4 *>(zr)[i];
+    A *e = reinterpret_cast<A *>(&q);
+#pragma unroll
+    for (int k = 0; k < VW; k++) {
+      int v = i * VW + k;
+      float g = 0.f;
+      if (v < V) g = (expf(to_f(e[k]) - lse) - (v == y ? 1.f : 0.f)) * inv_n;
+      e[k] = from_f<A>(g);
+    }
+    reinterpret_cast<uint4 *>(zr)[i] = q;
+  }
+  for (int64_t v = (int64_t)Lv * VW + threadIdx.x; v < ldz; v += NT) {
     float g = 0.f;
     if (v < V) g = (expf(to_f(zr[v]) - lse) - (v == y ? 1.f : 0.f)) * inv_n;
     zr[v] = from_f<A>(g);
