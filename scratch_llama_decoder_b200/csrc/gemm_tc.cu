@@ -1,13 +1,15 @@
 // tcgen05 GEMM for sm_100a: C[M,N] = A[M,K] . B[N,K]^T, bf16 operands, fp32
 // accumulation in tensor memory (TMEM).
 //
-// Persistent kernel, one CTA per SM, 6 warps:
+// Persistent kernel, one CTA per SM, 10 warps:
 //   warp 0      TMA producer: A and B tiles into a STAGES-deep shared-memory
 //               ring (128-byte swizzle), completion counted on mbarriers;
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
 //               (M=128, N=256, K=16) and commits each stage back to the ring;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row per thread), fused epilogue, stores to global.
+//   warps 2..9  epilogue, two warps per TMEM lane quarter, each taking half
+//               of the tile's columns: tcgen05.ld of the accumulator (one
+//               TMEM lane = one output row per thread), the fused epilogue,
+//               and row-coalesced stores through a swizzled shared square.
 // Two accumulators of 256 columns alternate so the epilogue of one tile
 // overlaps the main loop of the next.  Operands may be K-major or MN-major
 // (both supported by the UMMA descriptors), which covers the forward
@@ -32,10 +34,11 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int STAGING_BYTES = 4 * 32 * 36 * 4;  // epilogue transpose squares, 4 warps
+constexpr int EPI_WARPS = 8;
+constexpr int STAGING_BYTES = EPI_WARPS * 32 * 32 * 4;  // one 32x32 float square per epilogue warp
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + STAGING_BYTES;
 constexpr int TMEM_COLS = 512;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 64 + 32 * EPI_WARPS;
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on any wait
 
 struct Args {
@@ -46,8 +49,6 @@ struct Args {
   int64_t ldc;
   const float *R;
   int64_t ldr;
-  const void *aux;  // SWIGLU: u output [M, hp]; SWIGLU_BWD: saved ab [M, 2hp]
-  int64_t ld_aux;
   const float *cos_t, *sin_t;
   int T, hd, rot_cols;
   int *flag;
@@ -153,21 +154,22 @@ LLM_DEV uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 // Coalesced write-out of a warp's 32 x 32 chunk: lane i holds row i in v.
-// The chunk goes through a shared-memory square with rows padded to 36 floats
-// (16-byte aligned; the 8 lanes of each 128-bit access phase hit 32 distinct
-// banks), written with 16-byte row-wise stores and read back 4 rows per
-// instruction (8 lanes x 4 floats per row), so each global store instruction
-// covers 4 full row segments.  rows / cols clip the edges.
-constexpr int STG_LD = 36;
-LLM_DEV void stage32(float (*stg)[STG_LD], const float (&v)[32]) {
+// The chunk goes through a 32 x 32 float square in shared memory whose
+// 16-byte groups are XOR-swizzled by the row (group g of row r sits at
+// position g ^ (r & 7)), so both the row-wise 16-byte writes and the
+// 4-rows-per-instruction reads hit 32 distinct banks; each global store
+// instruction then covers 4 full row segments.  rows / cols clip the edges.
+LLM_DEV float4 *sq(float *stg, int r, int g) {
+  return reinterpret_cast<float4 *>(stg + r * 32 + 4 * (g ^ (r & 7)));
+}
+LLM_DEV void stage32(float *stg, const float (&v)[32]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < 32; i += 4)
-    *reinterpret_cast<float4 *>(&stg[lane][i]) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  for (int g = 0; g < 8; g++) *sq(stg, lane, g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
   __syncwarp();
 }
 // Rows of the warp's 32-row slab, 4 columns per lane (lane&7), 4 rows per
-// instruction: the residual values put32_f32 will add, loaded ahead of use.
+// instruction: the residual values put32_f32 adds, all loads in flight first.
 LLM_DEV void ld32_f32(const float *R, int64_t ldr, int rows, int cols, float4 (&rv)[8]) {
   const int lane = threadIdx.x & 31;
   const int c = 4 * (lane & 7), rsub = lane >> 3;
@@ -179,18 +181,18 @@ LLM_DEV void ld32_f32(const float *R, int64_t ldr, int rows, int cols, float4 (&
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
-LLM_DEV void put32_f32(float (*stg)[STG_LD], const float (&v)[32], float *dst, int64_t ld,
-                       int rows, int cols, const float *R, int64_t ldr, const float4 (&rv)[8]) {
+LLM_DEV void put32_f32(float *stg, const float (&v)[32], float *dst, int64_t ld, int rows,
+                       int cols, const float *R, int64_t ldr, const float4 (&rv)[8]) {
   stage32(stg, v);
   const int lane = threadIdx.x & 31;
-  const int c = 4 * (lane & 7), rsub = lane >> 3;
+  const int g = lane & 7, c = 4 * g, rsub = lane >> 3;
   const bool full = c + 4 <= cols;
   if (c < cols) {
 #pragma unroll
     for (int k = 0; k < 8; k++) {
       const int r = rsub + 4 * k;
       if (r >= rows) break;
-      float4 x = *reinterpret_cast<const float4 *>(&stg[r][c]);
+      float4 x = *sq(stg, r, g);
       if (full) {
         x.x += rv[k].x; x.y += rv[k].y; x.z += rv[k].z; x.w += rv[k].w;
         *reinterpret_cast<float4 *>(dst + (int64_t)r * ld + c) = x;
@@ -203,17 +205,17 @@ LLM_DEV void put32_f32(float (*stg)[STG_LD], const float (&v)[32], float *dst, i
   }
   __syncwarp();
 }
-LLM_DEV void put32_bf16(float (*stg)[STG_LD], const float (&v)[32], __nv_bfloat16 *dst, int64_t ld,
-                        int rows, int cols) {
+LLM_DEV void put32_bf16(float *stg, const float (&v)[32], __nv_bfloat16 *dst, int64_t ld, int rows,
+                        int cols) {
   stage32(stg, v);
   const int lane = threadIdx.x & 31;
-  const int c = 4 * (lane & 7), rsub = lane >> 3;
+  const int g = lane & 7, c = 4 * g, rsub = lane >> 3;
   if (c < cols) {
 #pragma unroll
     for (int k = 0; k < 8; k++) {
       const int r = rsub + 4 * k;
       if (r >= rows) break;
-      float4 x = *reinterpret_cast<const float4 *>(&stg[r][c]);
+      float4 x = *sq(stg, r, g);
       if (c + 4 <= cols) {
         *reinterpret_cast<uint2 *>(dst + (int64_t)r * ld + c) =
             make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
@@ -226,43 +228,13 @@ LLM_DEV void put32_bf16(float (*stg)[STG_LD], const float (&v)[32], __nv_bfloat1
   __syncwarp();
 }
 
-// The reverse of put32_*: a warp's 32 rows x 32 bf16 columns of a
-// row-major matrix, read 4 rows per instruction (coalesced) into the staging
-// square, then handed out one row per lane (v[i] = row `lane`, column i).
-LLM_DEV void ld32_bf16(const __nv_bfloat16 *src, int64_t ld, int rows, uint2 (&q)[8]) {
-  const int lane = threadIdx.x & 31;
-  const int c = 4 * (lane & 7), rsub = lane >> 3;
-#pragma unroll
-  for (int k = 0; k < 8; k++) {
-    const int r = rsub + 4 * k;
-    q[k] = (r < rows) ? *reinterpret_cast<const uint2 *>(src + (int64_t)r * ld + c)
-                      : make_uint2(0u, 0u);
-  }
-}
-LLM_DEV void unstage32_bf16(float (*stg)[STG_LD], const uint2 (&q)[8], float (&v)[32]) {
-  const int lane = threadIdx.x & 31;
-  const int c = 4 * (lane & 7), rsub = lane >> 3;
-#pragma unroll
-  for (int k = 0; k < 8; k++) {
-    float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q[k].x));
-    float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q[k].y));
-    *reinterpret_cast<float4 *>(&stg[rsub + 4 * k][c]) = make_float4(lo.x, lo.y, hi.x, hi.y);
-  }
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    float4 x = *reinterpret_cast<const float4 *>(&stg[lane][i]);
-    v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
-  }
-  __syncwarp();
-}
-
 // One output tile's epilogue for a warp: rows [row0, row0+32) of the tile
-// (TMEM lanes of this warp's quarter, lane i = row row0 + i), columns
-// [n0, n0+BN).  Every lane executes every tcgen05.ld (warp-uniform control);
-// rows past M are clipped only at the stores.
-LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int split, bool zero,
-                           float (*stg)[STG_LD]) {
+// (TMEM lanes of this warp's quarter, lane i = row row0 + i) and the warp's
+// half of the columns, [n0 + c_lo, n0 + c_lo + BN/2).  Every lane executes
+// every tcgen05.ld (warp-uniform control); rows past M and columns past N are
+// clipped only at the stores.
+LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int c_lo, int split,
+                           bool zero, float *stg) {
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
   const int rows = max(0, min(32, a.M - row0));
@@ -274,7 +246,7 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
     const int hd = a.hd, half = hd / 2, t = m % a.T;
     __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
     if (hd == 64) {
-      for (int c0 = 0; c0 < BN; c0 += 64) {
+      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 64) {
         int n = n0 + c0;
         if (n >= N) break;
         float lo[32], hi[32];
@@ -300,7 +272,7 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
         put32_bf16(stg, hi, C + n + 32, a.ldc, rows, ncols(n + 32));
       }
     } else {  // hd == 32: both halves of a head sit in one 32-column chunk
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
         int n = n0 + c0;
         if (n >= N) break;
         if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
@@ -326,68 +298,11 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int spl
     }
     return;
   }
-  if (a.epi == TC_EPI_SWIGLU) {
-    // Interleaved [a|b] blocks of 64+64 columns: store a, b and u = silu(a) b.
-    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
-    __nv_bfloat16 *U = (__nv_bfloat16 *)a.aux + (int64_t)row0 * a.ld_aux;
-    for (int blk = 0; blk < BN; blk += 2 * SWIGLU_BLOCK) {
-      int n = n0 + blk;
-      if (n >= N) break;
-      for (int q = 0; q < SWIGLU_BLOCK; q += 32) {
-        float av[32], bv[32];
-        if (zero) { for (int i = 0; i < 32; i++) av[i] = bv[i] = 0.f; }
-        else { tmem_ld32(tm + blk + q, av); tmem_ld32(tm + blk + SWIGLU_BLOCK + q, bv); }
-        put32_bf16(stg, av, C + n + q, a.ldc, rows, 32);
-        put32_bf16(stg, bv, C + n + SWIGLU_BLOCK + q, a.ldc, rows, 32);
-#pragma unroll
-        for (int i = 0; i < 32; i++) av[i] = av[i] / (1.f + __expf(-av[i])) * bv[i];
-        put32_bf16(stg, av, U + (n / (2 * SWIGLU_BLOCK)) * SWIGLU_BLOCK + q, a.ld_aux, rows, 32);
-      }
-    }
-    return;
-  }
-  if (a.epi == TC_EPI_SWIGLU_BWD) {
-    // acc = du for hidden units [n0, n0+BN); write [da|db] at their
-    // interleaved columns using the saved [a|b].  The saved values of the
-    // next 32-column chunk are loaded while this chunk is computed.
-    const __nv_bfloat16 *AB = (const __nv_bfloat16 *)a.aux + (int64_t)row0 * a.ld_aux;
-    __nv_bfloat16 *D = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
-    uint2 qa[8], qb[8];
-    if (n0 < N) {
-      ld32_bf16(AB + w1_col(n0), a.ld_aux, rows, qa);
-      ld32_bf16(AB + w1_col(n0) + SWIGLU_BLOCK, a.ld_aux, rows, qb);
-    }
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-      int j = n0 + c0;
-      if (j >= N) break;
-      if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
-      else tmem_ld32(tm + c0, v);
-      int64_t ca = w1_col(j);
-      float av[32], bv[32];
-      unstage32_bf16(stg, qa, av);
-      unstage32_bf16(stg, qb, bv);
-      if (c0 + 32 < BN && j + 32 < N) {
-        ld32_bf16(AB + w1_col(j + 32), a.ld_aux, rows, qa);
-        ld32_bf16(AB + w1_col(j + 32) + SWIGLU_BLOCK, a.ld_aux, rows, qb);
-      }
-#pragma unroll
-      for (int i = 0; i < 32; i++) {
-        float s = 1.f / (1.f + __expf(-av[i]));
-        float du = v[i];
-        float da = du * bv[i] * s * (1.f + av[i] * (1.f - s));
-        bv[i] = du * av[i] * s;
-        av[i] = da;
-      }
-      put32_bf16(stg, av, D + ca, a.ldc, rows, 32);
-      put32_bf16(stg, bv, D + ca + SWIGLU_BLOCK, a.ldc, rows, 32);
-    }
-    return;
-  }
-  // Plain outputs (a residual is loaded, all eight rows-groups at once, just
+  // Plain outputs (a residual is loaded, all eight row groups at once, just
   // before the chunk is staged).
   const bool add = a.out == OUT_ADD_F32;
   const float *Rrow = add ? a.R + (int64_t)row0 * a.ldr : nullptr;
-  for (int c0 = 0; c0 < BN; c0 += 32) {
+  for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
     int n = n0 + c0;
     if (n >= N) break;
     if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
@@ -426,7 +341,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int b = 0; b < 2; b++) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, 4);
+      mbar_init(tempty0 + 8 * b, EPI_WARPS);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -543,8 +458,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // -------------------------------------------------- epilogue warps
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-    float (*stg)[STG_LD] = reinterpret_cast<float (*)[STG_LD]>(smem + STAGES * STAGE_BYTES + 256) +
-                       (warp - 2) * 32;
+    const int ew = warp - 2;       // epilogue warp 0..7
+    const int c_lo = (ew / 4) * (BN / 2);
+    float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + ew * 32 * 32;
     int acc = 0;
     uint32_t aph = 0;
     for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
@@ -553,7 +469,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, 0, row0, n0, split, true, stg);
+        epilogue_tile(a, 0, row0, n0, c_lo, split, true, stg);
         continue;
       }
       int got = 0;
@@ -562,7 +478,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!got) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, tm, row0, n0, split, false, stg);
+      epilogue_tile(a, tm, row0, n0, c_lo, split, false, stg);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -667,7 +583,7 @@ void tc_plan_destroy(TcPlan *p) { delete p; }
 static bool al16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
 bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-             int64_t ldr, int splits, int epi, const void *aux, cudaStream_t s) {
+             int64_t ldr, int splits, int epi, cudaStream_t s) {
   using namespace tc;
   if (!p || g.in != DT_BF16 || !p->flag) return false;
   if (g.M < 1 || g.N < 1 || g.K < 1) return false;
@@ -675,8 +591,7 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   if (out == OUT_ACT ? (ldc % 8) : (ldc % 4)) return false;
   if (out == OUT_ADD_F32 && (!R || !al16(R) || ldr % 4)) return false;
   if (epi == TC_EPI_ROPE && !(p->hd == 32 || p->hd == 64)) return false;
-  if ((epi == TC_EPI_SWIGLU || epi == TC_EPI_SWIGLU_BWD) && (g.N % 64 || !aux || !al16(aux)))
-    return false;
+  if (epi != TC_EPI_NONE && epi != TC_EPI_ROPE) return false;
   if (epi != TC_EPI_NONE && out != OUT_ACT) return false;
   // tensor maps: A as [rows][K] (K-major) or [K][M] (MN-major); same for B
   CUtensorMap ta, tb;
@@ -695,8 +610,6 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   a.kchunk = ((kc + BK - 1) / BK) * BK;
   a.total = a.tiles_m * a.tiles_n * a.splits;
   a.out = out; a.epi = epi; a.C = C; a.ldc = ldc; a.R = R; a.ldr = ldr;
-  a.aux = aux;
-  a.ld_aux = (epi == TC_EPI_SWIGLU) ? p->hp : 2 * p->hp;
   a.cos_t = p->cos_t; a.sin_t = p->sin_t; a.T = p->T; a.hd = p->hd; a.rot_cols = (int)p->rot_cols;
   a.flag = p->flag;
   int grid = min(a.total, p->num_sms);

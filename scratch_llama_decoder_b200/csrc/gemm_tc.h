@@ -10,10 +10,8 @@ namespace llm {
 struct TcPlan;
 
 enum TcEpi {
-  TC_EPI_NONE = 0,       // plain output as selected by GemmOut
-  TC_EPI_ROPE = 1,       // QKV forward: rotate q and k columns (RoPE) in the epilogue
-  TC_EPI_SWIGLU = 2,     // W13 forward: store [a|b] and u = silu(a) * b (aux = u)
-  TC_EPI_SWIGLU_BWD = 3  // W2 dgrad: du -> [da|db] using the saved [a|b] (aux = ab)
+  TC_EPI_NONE = 0,  // plain output as selected by GemmOut
+  TC_EPI_ROPE = 1   // QKV forward: rotate q and k columns (RoPE) in the epilogue
 };
 
 TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, int hd,
@@ -22,7 +20,7 @@ void tc_plan_destroy(TcPlan *p);
 // Device flag word that records a bounded wait giving up (FLAG_TIMEOUT).
 void tc_plan_set_flag(TcPlan *p, int *flag);
 bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-             int64_t ldr, int splits, int epi, const void *aux, cudaStream_t s);
+             int64_t ldr, int splits, int epi, cudaStream_t s);
 
 // Attention dispatch: tensor-core kernels when the plan covers the head size,
 // else the SIMT kernels.

@@ -374,7 +374,71 @@ __global__ void k_swiglu_bwd(const A *__restrict__ ab, const A *__restrict__ du,
     dab[row * 2 * hp + ca + SWIGLU_BLOCK] = from_f<A>(g * a * sg);
   }
 }
+// bf16, 8 hidden units per thread with 16-byte accesses (8 | 64, so the 8
+// units share one interleave block: a and b are 8 contiguous elements each).
+LLM_DEV void unpack8(uint4 q, float (&f)[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&q);
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    float2 t = __bfloat1622float2(h[k]);
+    f[2 * k] = t.x;
+    f[2 * k + 1] = t.y;
+  }
+}
+LLM_DEV uint4 pack8(const float (&f)[8]) {
+  uint4 q;
+  uint32_t *w = reinterpret_cast<uint32_t *>(&q);
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * k], f[2 * k + 1]);
+    w[k] = *reinterpret_cast<uint32_t *>(&h);
+  }
+  return q;
+}
+__global__ void k_swiglu_fwd_v8(const __nv_bfloat16 *__restrict__ ab, __nv_bfloat16 *__restrict__ u,
+                                int64_t N, int64_t hp) {
+  const int64_t per_row = hp / 8, n = N * per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / per_row, j = (i % per_row) * 8;
+    const __nv_bfloat16 *r = ab + row * 2 * hp + w1_col(j);
+    float a[8], b[8], o[8];
+    unpack8(*reinterpret_cast<const uint4 *>(r), a);
+    unpack8(*reinterpret_cast<const uint4 *>(r + SWIGLU_BLOCK), b);
+#pragma unroll
+    for (int k = 0; k < 8; k++) o[k] = a[k] * sigmoidf_(a[k]) * b[k];
+    *reinterpret_cast<uint4 *>(u + row * hp + j) = pack8(o);
+  }
+}
+__global__ void k_swiglu_bwd_v8(const __nv_bfloat16 *__restrict__ ab, const __nv_bfloat16 *__restrict__ du,
+                                __nv_bfloat16 *__restrict__ dab, int64_t N, int64_t hp) {
+  const int64_t per_row = hp / 8, n = N * per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / per_row, j = (i % per_row) * 8;
+    const int64_t ca = row * 2 * hp + w1_col(j);
+    float a[8], b[8], g[8], da[8], db[8];
+    unpack8(*reinterpret_cast<const uint4 *>(ab + ca), a);
+    unpack8(*reinterpret_cast<const uint4 *>(ab + ca + SWIGLU_BLOCK), b);
+    unpack8(*reinterpret_cast<const uint4 *>(du + row * hp + j), g);
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      float sg = sigmoidf_(a[k]);
+      da[k] = g[k] * b[k] * sg * (1.f + a[k] * (1.f - sg));
+      db[k] = g[k] * a[k] * sg;
+    }
+    *reinterpret_cast<uint4 *>(dab + ca) = pack8(da);
+    *reinterpret_cast<uint4 *>(dab + ca + SWIGLU_BLOCK) = pack8(db);
+  }
+}
+
 void swiglu_fwd(const void *ab, void *u, DType dt, int64_t N, int64_t hp, cudaStream_t s) {
+  if (dt == DT_BF16 && hp % 8 == 0 && ((uintptr_t)ab & 15) == 0 && ((uintptr_t)u & 15) == 0) {
+    k_swiglu_fwd_v8<<<min(cdiv(N * hp / 8, 256), 148u * 16), 256, 0, s>>>(
+        (const __nv_bfloat16 *)ab, (__nv_bfloat16 *)u, N, hp);
+    count_launch();
+    return;
+  }
   unsigned grid = min(cdiv(N * hp, 256), 148u * 16);
   if (dt == DT_BF16)
     k_swiglu_fwd<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)ab, (__nv_bfloat16 *)u, N, hp);
@@ -384,6 +448,13 @@ void swiglu_fwd(const void *ab, void *u, DType dt, int64_t N, int64_t hp, cudaSt
 }
 void swiglu_bwd(const void *ab, const void *du, void *dab, DType dt, int64_t N, int64_t hp,
                 cudaStream_t s) {
+  if (dt == DT_BF16 && hp % 8 == 0 && ((uintptr_t)ab & 15) == 0 && ((uintptr_t)du & 15) == 0 &&
+      ((uintptr_t)dab & 15) == 0) {
+    k_swiglu_bwd_v8<<<min(cdiv(N * hp / 8, 256), 148u * 16), 256, 0, s>>>(
+        (const __nv_bfloat16 *)ab, (const __nv_bfloat16 *)du, (__nv_bfloat16 *)dab, N, hp);
+    count_launch();
+    return;
+  }
   unsigned grid = min(cdiv(N * hp, 256), 148u * 16);
   if (dt == DT_BF16)
     k_swiglu_bwd<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)ab, (const __nv_bfloat16 *)du,

@@ -317,7 +317,7 @@ bool aligned16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
 // Tensor-core GEMM launch; when timing is on, bracketed by CUDA events on the
 // context's stream and credited with its algorithmic FLOPs (unpadded sizes).
 bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-            int64_t ldr, int splits, int epi, const void *aux, double alg_flops) {
+            int64_t ldr, int splits, int epi, double alg_flops) {
   if (!c->tc) return false;
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (c->timing) {
@@ -332,7 +332,7 @@ bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
       cudaEventRecord(e0, c->s);
     }
   }
-  bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, aux, c->s);
+  bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->s);
   if (e0) {
     cudaEventRecord(e1, c->s);
     if (ok) {
@@ -348,7 +348,7 @@ bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
 // the tensor-core kernel when it covers the shape, else to the SIMT kernel.
 void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
           int64_t ldr, int splits, double alg_flops) {
-  if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, nullptr, alg_flops)) return;
+  if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, alg_flops)) return;
   gemm_simt(g, out, C, ldc, R, ldr, splits, c->s);
 }
 
@@ -382,7 +382,7 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
     rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
     {
       GemmOperands g{(int)N, (int)D.qkvw, D.d, xn1, d, true, wqkv, D.qkvw, false, D.dt};
-      bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE, nullptr,
+      bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
                           2.0 * N * d * D.qkvw);
       if (!fused) {
         gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
@@ -394,15 +394,11 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
          d, 1, 2.0 * N * d * d);
     // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
     rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
-    {
-      GemmOperands g{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt};
-      bool fused = run_tc(c, g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, TC_EPI_SWIGLU, u,
-                          2.0 * N * d * 2 * D.h);
-      if (!fused) {
-        gemm_simt(g, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, s);
-        swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
-      }
-    }
+    // W13 GEMM into the interleaved [a|b], then u = silu(a) * b (a separate
+    // full-occupancy pass: cheaper than the same math in the GEMM epilogue)
+    gemm(c, GemmOperands{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt},
+         OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
+    swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
     gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_ADD_F32,
          x2, d, x1, d, 1, 2.0 * N * D.h * d);
   }
@@ -450,15 +446,9 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
     void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
     void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
     // FFN branch.  du = dx2 W2^T, then SwiGLU backward into dab.
-    {
-      GemmOperands g{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt};
-      bool fused = run_tc(c, g, OUT_ACT, c->dab, 2 * D.hp, nullptr, 0, 1, TC_EPI_SWIGLU_BWD,
-                          abuf, 2.0 * N * d * D.h);
-      if (!fused) {
-        gemm_simt(g, OUT_ACT, c->du, D.hp, nullptr, 0, 1, s);
-        swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
-      }
-    }
+    gemm(c, GemmOperands{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt}, OUT_ACT, c->du,
+         D.hp, nullptr, 0, 1, 2.0 * N * d * D.h);
+    swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
     wgrad(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
     gemm(c, GemmOperands{(int)N, D.d, (int)(2 * D.hp), c->dab, 2 * D.hp, true, w13, 2 * D.hp,
                          true, D.dt},
@@ -565,7 +555,7 @@ extern "C" int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_
     std::call_once(once, [] { plan = tc_plan_create(DT_BF16, nullptr, nullptr, 1, 64, 0, 64); });
     if (!plan) return LLM_ERR_ARG;
     tc_plan_set_flag(plan, d_flag);
-    if (!tc_gemm(plan, g, OUT_F32, d_C, ldc, nullptr, 0, 1, TC_EPI_NONE, nullptr, s))
+    if (!tc_gemm(plan, g, OUT_F32, d_C, ldc, nullptr, 0, 1, TC_EPI_NONE, s))
       return LLM_ERR_ARG;
   } else {
     gemm_simt(g, OUT_F32, d_C, ldc, nullptr, 0, 1, s);
