@@ -359,12 +359,18 @@ def run_kernel(args):
         w = (H + 2 * Hkv) * hd
         qkv = torch.randn(Bt * T, w, device="cuda", generator=g).to(torch.bfloat16)
         o = torch.empty(Bt * T, H * hd, device="cuda", dtype=torch.bfloat16)
+        do = torch.randn(Bt * T, H * hd, device="cuda", generator=g).to(torch.bfloat16)
+        dqkv = torch.empty_like(qkv)
         lse = torch.empty(Bt, H, T, device="cuda")
+        Dv = torch.empty(Bt, H, T, device="cuda")
 
         def call():
             assert P.lib.llm_kernel_attention_fwd_bf16(p(qkv), p(o), p(lse), Bt, T, H, Hkv, hd, 1,
                                                        None) == 0
-        flops = 4.0 * Bt * H * (T * (T + 1) / 2) * hd
+            assert P.lib.llm_kernel_attention_bwd_bf16(p(qkv), p(o), p(do), p(lse), p(Dv),
+                                                       p(dqkv), Bt, T, H, Hkv, hd, 1, None) == 0
+        # forward (QK^T, PV) and backward (dV, dP, dQ, dK): 6 causal matmuls
+        flops = 12.0 * Bt * H * (T * (T + 1) / 2) * hd
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()
