@@ -39,8 +39,10 @@ int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_t lda, int 
  * d_lse float32 [batch, n_head, ctx] = natural-log sum of exp of each score
  * row.  Backward: from d_o, d_lse and d_dout (bf16, like d_o) writes d_dqkv
  * (bf16, like d_qkv; every element written) and d_D float32 [batch, n_head,
- * ctx] = rowsum(dout * o) as scratch.  tensor_cores = 1 runs the mma kernels
- * (head_dim 32 or 64, else LLM_ERR_ARG), 0 the CUDA-core kernels. */
+ * ctx] = rowsum(dout * o) as scratch.  tensor_cores selects the kernels:
+ * 2 = the tcgen05/TMEM forward (head_dim 64; the backward then uses the mma
+ * kernels), 1 = the warp-level mma kernels (head_dim 32 or 64), 0 = the
+ * CUDA-core kernels; LLM_ERR_ARG if the selection does not cover head_dim. */
 int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float *d_lse, int batch, int ctx,
                                   int n_head, int n_kv_head, int head_dim, int tensor_cores,
                                   void *stream);

@@ -1,0 +1,334 @@
+// tcgen05 flash-attention forward for head size 64 (bf16 operands, fp32
+// softmax and accumulators): strata's online-softmax attention (no T x T
+// scores in memory, only the row log-sum-exp saved) on the 5th-generation
+// tensor cores.
+//
+// One CTA = 128 queries of one (batch, head); key blocks of 128.  6 warps:
+//   warp 0      TMA producer: the Q tile once, K and V tiles into 2-deep rings;
+//   warp 1      TMEM allocation (256 columns) and the MMA issuer:
+//                 S  = Q K^T     (M 128, N 128, K 64; both operands K-major in
+//                                 shared memory)              -> TMEM [0,128)
+//                 O += P V       (M 128, N 64, K 128; A = P from TMEM, B = V
+//                                 MN-major in shared memory)  -> TMEM [128,192)
+//   warps 2..5  softmax, one query row per thread (TMEM lane): two passes over
+//               the S row (row max, then exp2 and the row sum), P written to
+//               TMEM [192,256) as packed bf16.
+// The running maximum is lazy: the reference maximum of a row moves only when
+// a block's maximum exceeds it by more than 2^8, so P values stay below 256
+// and O (in TMEM) is rescaled only then; O and the row sum always share one
+// reference, so O / l is exact.  256 TMEM columns and ~81 KB of shared memory
+// let two CTAs share an SM and overlap one's softmax with the other's MMAs.
+// Every wait is bounded (FLAG_TIMEOUT, then drain and free TMEM).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm_tc.h"
+#include "tcgen05.cuh"
+
+namespace llm {
+namespace attn_tc {
+
+using namespace tc;
+
+constexpr int BQ = 128, BK = 128, HD = 64;
+constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
+constexpr int STAGES = 2;
+constexpr int NTHREADS = 192;
+constexpr int TMEM_COLS = 256;
+constexpr int COL_S = 0, COL_O = 128, COL_P = 192;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
+// shared memory: Q | K[2] | V[2] | barriers
+constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 1024;
+
+LLM_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bd, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bd), "r"(id), "r"(acc)
+      : "memory");
+}
+LLM_DEV void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+      "r"(w[15])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(NTHREADS, 2)
+    k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16 *__restrict__ o,
+                  float *__restrict__ lse, int T, int H, int Hkv, float scale, int *gflag) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sQ = smem, *sK = smem + TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
+  uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
+  uint32_t *tmem_sh = (uint32_t *)(bars + 24);
+  volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
+  const uint32_t b0 = smem_u32(bars);
+  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
+                 v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
+                 p_full = b0 + 8 * 11, o_done = b0 + 8 * 12, drain = b0 + 8 * 13;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int g = h / (H / Hkv), d = H * HD, kvd = Hkv * HD;
+  const int q0 = qb * BQ;
+  const int nj = min(qb + 1, (T + BK - 1) / BK);  // causal: key blocks up to the diagonal
+  const int row_base = b * T;
+
+  if (threadIdx.x == 0) {
+    *abort_sh = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
+      mbar_init(v_full + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_sh)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, TILE_BYTES);
+      tma_load_2d(smem_u32(sQ), &tm_qkv, h * HD, row_base + q0, q_full);
+      for (int j = 0; j < nj && ok; j++) {
+        const int s = j % STAGES;
+        const uint32_t ph = (j / STAGES) & 1;
+        if (!mbar_wait(k_empty + 8 * s, ph ^ 1, abort_sh, gflag)) { ok = false; break; }
+        mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
+        tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
+                    k_full + 8 * s);
+        if (!mbar_wait(v_empty + 8 * s, ph ^ 1, abort_sh, gflag)) { ok = false; break; }
+        mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
+        tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD, row_base + j * BK,
+                    v_full + 8 * s);
+      }
+      // every copy this thread issued has landed before the CTA may exit
+      unsigned long long t0 = gtimer();
+      while (!mbar_try(q_full, 0) && gtimer() - t0 < WAIT_NS) {
+      }
+      for (int j = max(0, nj - STAGES); j < nj; j++) {
+        const int s = j % STAGES;
+        const uint32_t ph = (j / STAGES) & 1;
+        t0 = gtimer();
+        while (!mbar_try(k_full + 8 * s, ph) && gtimer() - t0 < WAIT_NS) {
+        }
+        while (!mbar_try(v_full + 8 * s, ph) && gtimer() - t0 < WAIT_NS) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
+      constexpr uint32_t ID_O = idesc_mn(128, HD, false, true);
+      const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
+      bool ok = mbar_wait(q_full, 0, abort_sh, gflag);
+      for (int j = 0; j < nj && ok; j++) {
+        const int s = j % STAGES;
+        const uint32_t ph = (j / STAGES) & 1;
+        if (!mbar_wait(k_full + 8 * s, ph, abort_sh, gflag)) { ok = false; break; }
+        if (j > 0 && !mbar_wait(s_free, (j - 1) & 1, abort_sh, gflag)) { ok = false; break; }
+        fence_after();
+        const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; kk++)
+          mma_bf16(tmem + COL_S, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), ID_S,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        mma_commit(k_empty + 8 * s);
+        if (!mbar_wait(p_full, j & 1, abort_sh, gflag)) { ok = false; break; }
+        if (!mbar_wait(v_full + 8 * s, ph, abort_sh, gflag)) { ok = false; break; }
+        fence_after();
+        const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 8192, 1024);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; kk++)
+          mma_ts(tmem + COL_O, tmem + COL_P + kk * 8, vd + (uint64_t)(kk * 128), ID_O,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(v_empty + 8 * s);
+        mma_commit(o_done);
+      }
+      mma_commit(drain);
+      unsigned long long t0 = gtimer();
+      while (!mbar_try(drain, 0) && gtimer() - t0 < WAIT_NS) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row of the tile = TMEM lane
+    const int qi = q0 + r;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = scale * LOG2E;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nj; j++) {
+      int got = 0;
+      if (lane == 0) got = mbar_wait(s_full, j & 1, abort_sh, gflag) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+      fence_after();
+      const int k0 = j * BK;
+      const bool diag = (k0 + BK > q0);  // only blocks touching the diagonal (or T) mask
+      // pass 1: row maximum (log2 units)
+      float mx = -INFINITY;
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        tmem_ld32(tmem + lane_off + COL_S + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          const int kj = k0 + c * 32 + i;
+          const bool masked = diag && (kj > qi || kj >= T);
+          if (!masked) mx = fmaxf(mx, v[i] * sl2);
+        }
+      }
+      const bool need = mx > m_ref + LAZY;  // true on the first block (m_ref = -inf)
+      // P and O of the previous block are free once its P.V has completed
+      if (j > 0) {
+        int got2 = 0;
+        if (lane == 0) got2 = mbar_wait(o_done, (j - 1) & 1, abort_sh, gflag) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got2, 0)) { ok = false; break; }
+        fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+          const float corr = need ? exp2f(m_ref - mx) : 1.f;
+#pragma unroll
+          for (int c = 0; c < 2; c++) {
+            tmem_ld32(tmem + lane_off + COL_O + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[i] *= corr;
+            tmem_st32(tmem + lane_off + COL_O + c * 32, v);
+          }
+        }
+      }
+      if (need) {
+        if (m_ref != -INFINITY) l *= exp2f(m_ref - mx);
+        m_ref = mx;
+      }
+      // pass 2: P = exp2(s - m_ref), packed bf16 into TMEM
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        tmem_ld32(tmem + lane_off + COL_S + c * 32, v);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int kj = k0 + c * 32 + i;
+          const bool m0 = diag && (kj > qi || kj >= T);
+          const bool m1 = diag && (kj + 1 > qi || kj + 1 >= T);
+          const float p0 = m0 ? 0.f : exp2f(v[i] * sl2 - m_ref);
+          const float p1 = m1 ? 0.f : exp2f(v[i + 1] * sl2 - m_ref);
+          l += p0 + p1;
+          w[i / 2] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tmem + lane_off + COL_P + c * 16, w);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(s_free);
+        mbar_arrive(p_full);
+      }
+    }
+    if (ok) {
+      int got = 0;
+      if (lane == 0) got = mbar_wait(o_done, (nj - 1) & 1, abort_sh, gflag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+    }
+    if (ok) {
+      fence_after();
+      float v[32];
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < 2; c++) {
+        tmem_ld32(tmem + lane_off + COL_O + c * 32, v);
+        if (qi < T) {
+          __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 q = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv),
+                                 pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
+                                 pack_bf16(v[i + 4] * inv, v[i + 5] * inv),
+                                 pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
+            *reinterpret_cast<uint4 *>(dst + i) = q;
+          }
+        }
+      }
+      if (qi < T) lse[((int64_t)b * H + h) * T + qi] = (m_ref + log2f(l)) * LN2;
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace attn_tc
+
+bool attn_tc_covers(DType dt, int hd, int T) { return dt == DT_BF16 && hd == 64 && T >= 1; }
+
+// Host side: one tensor map over qkv [B*T rows, qkvw columns] serves the Q, K
+// and V tiles (box 64 x 128, 128-byte swizzle).
+bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
+                 int *flag, cudaStream_t s) {
+  using namespace attn_tc;
+  if (hd != HD || !flag || ((uintptr_t)qkv & 15)) return false;
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static bool init = false;
+  if (!init) {
+    cudaDriverEntryPointQueryResult q;
+    void *fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    init = true;
+  }
+  if (!encode) return false;
+  const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)qkvw, (cuuint64_t)B * T};
+  cuuint64_t strides[1] = {(cuuint64_t)qkvw * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(qkv), dims, strides,
+             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  dim3 grid(H, B, (T + BQ - 1) / BQ);
+  k_attn_fwd_tc<<<grid, NTHREADS, SMEM_BYTES, s>>>(map, (__nv_bfloat16 *)o, lse, T, H, Hkv,
+                                                   1.0f / sqrtf((float)hd), flag);
+  count_launch();
+  return true;
+}
+
+}  // namespace llm

@@ -94,6 +94,12 @@ void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float 
                   void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
                   const float *sin_t, cudaStream_t s);
 
+// tcgen05 flash-attention forward (bf16, head size 64); false when it does not
+// cover the arguments.  flag: device word for FLAG_TIMEOUT.
+bool attn_tc_covers(DType dt, int hd, int T);
+bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
+                 int *flag, cudaStream_t s);
+
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;
 inline void count_launch(int n = 1) { g_launches += n; }

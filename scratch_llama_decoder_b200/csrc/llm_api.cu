@@ -594,7 +594,15 @@ extern "C" int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float
     return LLM_ERR_ARG;
   g_launches = 0;
   cudaStream_t s = (cudaStream_t)stream;
-  if (tensor_cores) {
+  if (tensor_cores == 2) {
+    // tcgen05 kernel: its time-out flag is a library-owned device word
+    static int *flag = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] { cudaMalloc(&flag, sizeof(int)); cudaMemset(flag, 0, sizeof(int)); });
+    if (!flag || !attn_tc_covers(DT_BF16, head_dim, ctx) ||
+        !attn_fwd_tc(d_qkv, d_o, d_lse, batch, ctx, n_head, n_kv_head, head_dim, flag, s))
+      return LLM_ERR_ARG;
+  } else if (tensor_cores == 1) {
     if (!attn_mma_covers(DT_BF16, head_dim)) return LLM_ERR_ARG;
     attn_fwd_mma(d_qkv, d_o, d_lse, batch, ctx, n_head, n_kv_head, head_dim, s);
   } else {
