@@ -53,6 +53,8 @@ def parse():
                     help="time one hot-path kernel through the C ABI instead of the step")
     ap.add_argument("--shape", default="16384,3072,1024",
                     help="gemm: M,N,K; attention: batch,ctx,n_head,n_kv_head,head_dim")
+    ap.add_argument("--fwd-impl", type=int, default=2, choices=[0, 1, 2],
+                    help="attention forward kernels: 2 tcgen05, 1 mma, 0 CUDA cores")
     ap.add_argument("--orient", default="kn", choices=["kn", "kk", "nn"],
                     help="gemm operand majorness: kn = x.W (forward), kk = dy.W^T (dgrad), "
                          "nn = x^T.dy (wgrad)")
@@ -364,13 +366,35 @@ def run_kernel(args):
         lse = torch.empty(Bt, H, T, device="cuda")
         Dv = torch.empty(Bt, H, T, device="cuda")
 
-        def call():
-            assert P.lib.llm_kernel_attention_fwd_bf16(p(qkv), p(o), p(lse), Bt, T, H, Hkv, hd, 1,
-                                                       None) == 0
+        def fwd():
+            assert P.lib.llm_kernel_attention_fwd_bf16(p(qkv), p(o), p(lse), Bt, T, H, Hkv, hd,
+                                                       args.fwd_impl, None) == 0
+
+        def bwd():
             assert P.lib.llm_kernel_attention_bwd_bf16(p(qkv), p(o), p(do), p(lse), p(Dv),
                                                        p(dqkv), Bt, T, H, Hkv, hd, 1, None) == 0
-        # forward (QK^T, PV) and backward (dV, dP, dQ, dK): 6 causal matmuls
-        flops = 12.0 * Bt * H * (T * (T + 1) / 2) * hd
+        causal = Bt * H * (T * (T + 1) / 2) * hd
+        res = {}
+        for name, fn, fl in (("fwd", fwd, 4.0 * causal), ("bwd", bwd, 8.0 * causal)):
+            for _ in range(args.warmup):
+                fwd()
+                fn()
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                if name == "bwd":
+                    fwd()
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1)
+            ms = tot / args.steps
+            res[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12}
+        print(json.dumps({"kernel": "attention", "shape": args.shape, "fwd_impl": args.fwd_impl,
+                          **res}), flush=True)
+        return
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()
