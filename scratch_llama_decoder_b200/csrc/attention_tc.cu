@@ -10,14 +10,17 @@
 //                                 shared memory)              -> TMEM [0,128)
 //                 O += P V       (M 128, N 64, K 128; A = P from TMEM, B = V
 //                                 MN-major in shared memory)  -> TMEM [128,192)
-//   warps 2..5  softmax, one query row per thread (TMEM lane): two passes over
-//               the S row (row max, then exp2 and the row sum), P written to
-//               TMEM [192,256) as packed bf16.
+//   warps 2..5  softmax, one query row per thread (TMEM lane): the whole S
+//               row is loaded into registers with four back-to-back TMEM
+//               loads and one wait, S is released at once (so the MMA warp
+//               runs the next block's Q K^T during this block's exponentials),
+//               and P goes back to TMEM [192,256) as packed bf16 with four
+//               back-to-back stores.
 // The running maximum is lazy: the reference maximum of a row moves only when
 // a block's maximum exceeds it by more than 2^8, so P values stay below 256
 // and O (in TMEM) is rescaled only then; O and the row sum always share one
-// reference, so O / l is exact.  256 TMEM columns and ~81 KB of shared memory
-// let two CTAs share an SM and overlap one's softmax with the other's MMAs.
+// reference, so O / l is exact.  The MMA order per block j is Q K_{j+1}^T, then
+// P_j V_j, so the tensor core works while the softmax of block j runs.
 // Every wait is bounded (FLAG_TIMEOUT, then drain and free TMEM).
 #include <cudaTypedefs.h>
 
@@ -61,7 +64,33 @@ LLM_DEV void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
       : "memory");
 }
 
-__global__ void __launch_bounds__(NTHREADS, 2)
+// Four 32-column TMEM loads in flight, one wait.
+LLM_DEV void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+  uint32_t r[128];
+#define LD32(OFF)                                                                                \
+  asm volatile(                                                                                  \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"  \
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"        \
+      : "=r"(r[OFF + 0]), "=r"(r[OFF + 1]), "=r"(r[OFF + 2]), "=r"(r[OFF + 3]),                \
+        "=r"(r[OFF + 4]), "=r"(r[OFF + 5]), "=r"(r[OFF + 6]), "=r"(r[OFF + 7]),                \
+        "=r"(r[OFF + 8]), "=r"(r[OFF + 9]), "=r"(r[OFF + 10]), "=r"(r[OFF + 11]),              \
+        "=r"(r[OFF + 12]), "=r"(r[OFF + 13]), "=r"(r[OFF + 14]), "=r"(r[OFF + 15]),            \
+        "=r"(r[OFF + 16]), "=r"(r[OFF + 17]), "=r"(r[OFF + 18]), "=r"(r[OFF + 19]),            \
+        "=r"(r[OFF + 20]), "=r"(r[OFF + 21]), "=r"(r[OFF + 22]), "=r"(r[OFF + 23]),            \
+        "=r"(r[OFF + 24]), "=r"(r[OFF + 25]), "=r"(r[OFF + 26]), "=r"(r[OFF + 27]),            \
+        "=r"(r[OFF + 28]), "=r"(r[OFF + 29]), "=r"(r[OFF + 30]), "=r"(r[OFF + 31])             \
+      : "r"(taddr + OFF))
+  LD32(0);
+  LD32(32);
+  LD32(64);
+  LD32(96);
+#undef LD32
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 128; i++) v[i] = __uint_as_float(r[i]);
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16 *__restrict__ o,
                   float *__restrict__ lse, int T, int H, int Hkv, float scale, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
@@ -148,13 +177,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
       constexpr uint32_t ID_O = idesc_mn(128, HD, false, true);
       const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
-      bool ok = mbar_wait(q_full, 0, abort_sh, gflag);
-      for (int j = 0; j < nj && ok; j++) {
+      auto issue_s = [&](int j) {  // S = Q K_j^T into TMEM [0,128)
         const int s = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
-        if (!mbar_wait(k_full + 8 * s, ph, abort_sh, gflag)) { ok = false; break; }
-        if (j > 0 && !mbar_wait(s_free, (j - 1) & 1, abort_sh, gflag)) { ok = false; break; }
-        fence_after();
         const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; kk++)
@@ -162,6 +186,24 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                    kk > 0 ? 1u : 0u);
         mma_commit(s_full);
         mma_commit(k_empty + 8 * s);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_sh, gflag) && mbar_wait(k_full, 0, abort_sh, gflag);
+      if (ok) {
+        fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; j < nj && ok; j++) {
+        const int s = j % STAGES;
+        const uint32_t ph = (j / STAGES) & 1;
+        if (j + 1 < nj) {
+          // next block's scores once the softmax has read this block's S
+          const int s1 = (j + 1) % STAGES;
+          const uint32_t ph1 = ((j + 1) / STAGES) & 1;
+          if (!mbar_wait(k_full + 8 * s1, ph1, abort_sh, gflag)) { ok = false; break; }
+          if (!mbar_wait(s_free, j & 1, abort_sh, gflag)) { ok = false; break; }
+          fence_after();
+          issue_s(j + 1);
+        }
         if (!mbar_wait(p_full, j & 1, abort_sh, gflag)) { ok = false; break; }
         if (!mbar_wait(v_full + 8 * s, ph, abort_sh, gflag)) { ok = false; break; }
         fence_after();
@@ -194,18 +236,18 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       fence_after();
       const int k0 = j * BK;
       const bool diag = (k0 + BK > q0);  // only blocks touching the diagonal (or T) mask
-      // pass 1: row maximum (log2 units)
+      float sv[128];
+      tmem_ld128(tmem + lane_off + COL_S, sv);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
+      // row maximum (log2 units)
       float mx = -INFINITY;
-      float v[32];
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        tmem_ld32(tmem + lane_off + COL_S + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-          const int kj = k0 + c * 32 + i;
-          const bool masked = diag && (kj > qi || kj >= T);
-          if (!masked) mx = fmaxf(mx, v[i] * sl2);
-        }
+      for (int i = 0; i < 128; i++) {
+        sv[i] *= sl2;
+        if (diag && (k0 + i > qi || k0 + i >= T)) sv[i] = -INFINITY;
+        mx = fmaxf(mx, sv[i]);
       }
       const bool need = mx > m_ref + LAZY;  // true on the first block (m_ref = -inf)
       // P and O of the previous block are free once its P.V has completed
@@ -216,6 +258,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         fence_after();
         if (__any_sync(0xffffffffu, need)) {
           const float corr = need ? exp2f(m_ref - mx) : 1.f;
+          float v[32];
 #pragma unroll
           for (int c = 0; c < 2; c++) {
             tmem_ld32(tmem + lane_off + COL_O + c * 32, v);
@@ -229,30 +272,23 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         if (m_ref != -INFINITY) l *= exp2f(m_ref - mx);
         m_ref = mx;
       }
-      // pass 2: P = exp2(s - m_ref), packed bf16 into TMEM
+      // P = exp2(s - m_ref), packed bf16, four stores in flight
+      uint32_t w[64];
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float p0 = exp2f(sv[i] - m_ref), p1 = exp2f(sv[i + 1] - m_ref);
+        l += p0 + p1;
+        w[i / 2] = pack_bf16(p0, p1);
+      }
 #pragma unroll
       for (int c = 0; c < 4; c++) {
-        tmem_ld32(tmem + lane_off + COL_S + c * 32, v);
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int kj = k0 + c * 32 + i;
-          const bool m0 = diag && (kj > qi || kj >= T);
-          const bool m1 = diag && (kj + 1 > qi || kj + 1 >= T);
-          const float p0 = m0 ? 0.f : exp2f(v[i] * sl2 - m_ref);
-          const float p1 = m1 ? 0.f : exp2f(v[i + 1] * sl2 - m_ref);
-          l += p0 + p1;
-          w[i / 2] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tmem + lane_off + COL_P + c * 16, w);
+        uint32_t (&wc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&w[c * 16]);
+        tmem_st16(tmem + lane_off + COL_P + c * 16, wc);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(s_free);
-        mbar_arrive(p_full);
-      }
+      if (lane == 0) mbar_arrive(p_full);
     }
     if (ok) {
       int got = 0;
