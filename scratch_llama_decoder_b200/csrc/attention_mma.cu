@@ -22,6 +22,7 @@
 // projection is with respect to the un-rotated q and k.
 #include "common.cuh"
 #include "gemm_tc.h"
+#include "tcgen05.cuh"
 
 namespace llm {
 namespace attn {
@@ -235,12 +236,12 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
       for (int nt = 0; nt < 8; nt++) mx = fmaxf(mx, fmaxf(s[nt][2 * r], s[nt][2 * r + 1]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      float corr = (m[r] == -INFINITY) ? 0.f : exp2f(m[r] - mx);
+      float corr = (m[r] == -INFINITY) ? 0.f : tc::ex2(m[r] - mx);
       float rs = 0.f;
 #pragma unroll
       for (int nt = 0; nt < 8; nt++) {
-        float p0 = (mx == -INFINITY) ? 0.f : exp2f(s[nt][2 * r] - mx);
-        float p1 = (mx == -INFINITY) ? 0.f : exp2f(s[nt][2 * r + 1] - mx);
+        float p0 = (mx == -INFINITY) ? 0.f : tc::ex2(s[nt][2 * r] - mx);
+        float p1 = (mx == -INFINITY) ? 0.f : tc::ex2(s[nt][2 * r + 1] - mx);
         s[nt][2 * r] = p0;
         s[nt][2 * r + 1] = p1;
         rs += p0 + p1;
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
         int r = e >> 1;
         int qi = row0 + r * 8;
         int kj = k0 + nt * 8 + (lane & 3) * 2 + (e & 1);
-        float p = (kj > qi || kj >= T || qi >= T) ? 0.f : exp2f(s[nt][e] * sl2 - L2[r]);
+        float p = (kj > qi || kj >= T || qi >= T) ? 0.f : tc::ex2(s[nt][e] * sl2 - L2[r]);
         s[nt][e] = p * (dp[nt][e] - Dr[r]);  // dS
       }
     }
@@ -483,7 +484,7 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
           int kj = key0 + (e >> 1) * 8;
           int col = hf * 32 + nt * 8 + (lane & 3) * 2 + (e & 1);
           int qi = q0 + col;
-          float p = (kj > qi || qi >= T || kj >= T) ? 0.f : exp2f(s[nt][e] * sl2 - Ls[cur][col]);
+          float p = (kj > qi || qi >= T || kj >= T) ? 0.f : tc::ex2(s[nt][e] * sl2 - Ls[cur][col]);
           s[nt][e] = p;                                // P^T
           dp[nt][e] = p * (dp[nt][e] - Ds[cur][col]);  // dS^T
         }

@@ -10,12 +10,13 @@
 //                                 shared memory)              -> TMEM [0,128)
 //                 O += P V       (M 128, N 64, K 128; A = P from TMEM, B = V
 //                                 MN-major in shared memory)  -> TMEM [128,192)
-//   warps 2..5  softmax, one query row per thread (TMEM lane): the whole S
-//               row is loaded into registers with four back-to-back TMEM
-//               loads and one wait, S is released at once (so the MMA warp
-//               runs the next block's Q K^T during this block's exponentials),
-//               and P goes back to TMEM [192,256) as packed bf16 with four
-//               back-to-back stores.
+//   warps 2..9  softmax, two warps per TMEM lane quarter: thread = one query
+//               row (TMEM lane) and one half (64 keys) of the block.  The
+//               half-row is loaded into registers in one TMEM round trip and
+//               S is released at once (so the MMA warp runs the next block's
+//               Q K^T during this block's exponentials); the two halves'
+//               maxima meet in shared memory; P goes back to TMEM [192,256)
+//               as packed bf16.
 // The running maximum is lazy: the reference maximum of a row moves only when
 // a block's maximum exceeds it by more than 2^8, so P values stay below 256
 // and O (in TMEM) is rescaled only then; O and the row sum always share one
@@ -38,14 +39,15 @@ using namespace tc;
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 2;
-constexpr int NTHREADS = 192;
+constexpr int SM_WARPS = 8;  // softmax warps
+constexpr int NTHREADS = 64 + 32 * SM_WARPS;
 constexpr int TMEM_COLS = 256;
 constexpr int COL_S = 0, COL_O = 128, COL_P = 192;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
 // shared memory: Q | K[2] | V[2] | barriers
-constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 1024;
+constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 2 * 128 * 4 + 1024;
 
 LLM_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bd, uint32_t id, uint32_t acc) {
   asm volatile(
@@ -64,9 +66,9 @@ LLM_DEV void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
       : "memory");
 }
 
-// Four 32-column TMEM loads in flight, one wait.
-LLM_DEV void tmem_ld128(uint32_t taddr, float (&v)[128]) {
-  uint32_t r[128];
+// Two 32-column TMEM loads in flight, one wait.
+LLM_DEV void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
 #define LD32(OFF)                                                                                \
   asm volatile(                                                                                  \
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"  \
@@ -82,13 +84,13 @@ LLM_DEV void tmem_ld128(uint32_t taddr, float (&v)[128]) {
       : "r"(taddr + OFF))
   LD32(0);
   LD32(32);
-  LD32(64);
-  LD32(96);
 #undef LD32
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 128; i++) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 64; i++) v[i] = __uint_as_float(r[i]);
 }
+// Named barrier of the softmax warps (id 1).
+LLM_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * SM_WARPS) : "memory"); }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16 *__restrict__ o,
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
   uint32_t *tmem_sh = (uint32_t *)(bars + 24);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
+  float *red = (float *)(bars + 32);  // [2][128]: per-half row maxima / sums
   const uint32_t b0 = smem_u32(bars);
   const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
                  v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
@@ -121,8 +124,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(v_empty + 8 * s, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
+    mbar_init(s_free, SM_WARPS);
+    mbar_init(p_full, SM_WARPS);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -223,74 +226,92 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // row of the tile = TMEM lane
+    const int ch = (warp - 2) >> 2;      // which 64-key half of the block
+    const int r = quarter * 32 + lane;   // row of the tile = TMEM lane
     const int qi = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = scale * LOG2E;
     float m_ref = -INFINITY, l = 0.f;
+    // Every softmax warp executes the same named barriers on every path: a
+    // failed wait only turns the remaining work off (ok = false), it never
+    // leaves the loop early (bar.sync has no time-out).
     bool ok = true;
     for (int j = 0; j < nj; j++) {
-      int got = 0;
-      if (lane == 0) got = mbar_wait(s_full, j & 1, abort_sh, gflag) ? 1 : 0;
-      if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-      fence_after();
-      const int k0 = j * BK;
-      const bool diag = (k0 + BK > q0);  // only blocks touching the diagonal (or T) mask
-      float sv[128];
-      tmem_ld128(tmem + lane_off + COL_S, sv);
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
-      // row maximum (log2 units)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 128; i++) {
-        sv[i] *= sl2;
-        if (diag && (k0 + i > qi || k0 + i >= T)) sv[i] = -INFINITY;
-        mx = fmaxf(mx, sv[i]);
+      if (ok) {
+        int got = 0;
+        if (lane == 0) got = mbar_wait(s_full, j & 1, abort_sh, gflag) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, got, 0) != 0;
       }
+      fence_after();
+      const int k0 = j * BK + ch * 64;
+      const bool diag = (j * BK + BK > q0);  // only the diagonal block (or T) masks
+      float sv[64];
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (ok) {
+        tmem_ld64(tmem + lane_off + COL_S + ch * 64, sv);
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
+        // this half's row maximum (log2 units), 4 independent chains
+#pragma unroll
+        for (int i = 0; i < 64; i++) {
+          float x = sv[i] * sl2;
+          if (diag && (k0 + i > qi || k0 + i >= T)) x = -INFINITY;
+          sv[i] = x;
+          m4[i & 3] = fmaxf(m4[i & 3], x);
+        }
+      }
+      red[ch * 128 + r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      softmax_sync();
+      const float mx = fmaxf(red[r], red[128 + r]);
+      softmax_sync();  // both halves read before the next block overwrites red
+      if (!ok) continue;
       const bool need = mx > m_ref + LAZY;  // true on the first block (m_ref = -inf)
       // P and O of the previous block are free once its P.V has completed
       if (j > 0) {
         int got2 = 0;
         if (lane == 0) got2 = mbar_wait(o_done, (j - 1) & 1, abort_sh, gflag) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, got2, 0)) { ok = false; break; }
+        if (!__shfl_sync(0xffffffffu, got2, 0)) { ok = false; continue; }
         fence_after();
         if (__any_sync(0xffffffffu, need)) {
-          const float corr = need ? exp2f(m_ref - mx) : 1.f;
+          // each half-row warp rescales its 32 of O's 64 columns
+          const float corr = need ? ex2(m_ref - mx) : 1.f;
           float v[32];
+          tmem_ld32(tmem + lane_off + COL_O + ch * 32, v);
 #pragma unroll
-          for (int c = 0; c < 2; c++) {
-            tmem_ld32(tmem + lane_off + COL_O + c * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; i++) v[i] *= corr;
-            tmem_st32(tmem + lane_off + COL_O + c * 32, v);
-          }
+          for (int i = 0; i < 32; i++) v[i] *= corr;
+          tmem_st32(tmem + lane_off + COL_O + ch * 32, v);
         }
       }
       if (need) {
-        if (m_ref != -INFINITY) l *= exp2f(m_ref - mx);
+        if (m_ref != -INFINITY) l *= ex2(m_ref - mx);
         m_ref = mx;
       }
-      // P = exp2(s - m_ref), packed bf16, four stores in flight
-      uint32_t w[64];
+      // P = 2^(s - m_ref), packed bf16 into this half's 32 TMEM columns
+      uint32_t w[32];
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        const float p0 = exp2f(sv[i] - m_ref), p1 = exp2f(sv[i + 1] - m_ref);
-        l += p0 + p1;
+      for (int i = 0; i < 64; i += 2) {
+        const float p0 = ex2(sv[i] - m_ref), p1 = ex2(sv[i + 1] - m_ref);
+        l4[(i >> 1) & 3] += p0 + p1;
         w[i / 2] = pack_bf16(p0, p1);
       }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
+      for (int c = 0; c < 2; c++) {
         uint32_t (&wc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&w[c * 16]);
-        tmem_st16(tmem + lane_off + COL_P + c * 16, wc);
+        tmem_st16(tmem + lane_off + COL_P + ch * 32 + c * 16, wc);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
+    // row sum = both halves' sums (same reference maximum)
+    if (ok) red[ch * 128 + r] = l;
+    softmax_sync();
     if (ok) {
+      l = red[r] + red[128 + r];
       int got = 0;
       if (lane == 0) got = mbar_wait(o_done, (nj - 1) & 1, abort_sh, gflag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, got, 0) != 0;
@@ -299,22 +320,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_after();
       float v[32];
       const float inv = 1.f / l;
+      tmem_ld32(tmem + lane_off + COL_O + ch * 32, v);
+      if (qi < T) {
+        __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + ch * 32;
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        tmem_ld32(tmem + lane_off + COL_O + c * 32, v);
-        if (qi < T) {
-          __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + c * 32;
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 q = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv),
-                                 pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
-                                 pack_bf16(v[i + 4] * inv, v[i + 5] * inv),
-                                 pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
-            *reinterpret_cast<uint4 *>(dst + i) = q;
-          }
+        for (int i = 0; i < 32; i += 8) {
+          uint4 q = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv),
+                               pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
+                               pack_bf16(v[i + 4] * inv, v[i + 5] * inv),
+                               pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
+          *reinterpret_cast<uint4 *>(dst + i) = q;
         }
+        if (ch == 0) lse[((int64_t)b * H + h) * T + qi] = (m_ref + log2f(l)) * LN2;
       }
-      if (qi < T) lse[((int64_t)b * H + h) * T + qi] = (m_ref + log2f(l)) * LN2;
     }
   }
   fence_before();

@@ -121,6 +121,13 @@ LLM_DEV void tmem_st32(uint32_t taddr, const float (&v)[32]) {
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// 2^x by the SFU's single ex2.approx instruction (flushes denormals; relative
+// error of a few ulp) -- the softmax exponent.
+LLM_DEV float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 LLM_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
