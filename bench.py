@@ -55,6 +55,8 @@ def parse():
                     help="gemm: M,N,K; attention: batch,ctx,n_head,n_kv_head,head_dim")
     ap.add_argument("--fwd-impl", type=int, default=2, choices=[0, 1, 2],
                     help="attention forward kernels: 2 tcgen05, 1 mma, 0 CUDA cores")
+    ap.add_argument("--bwd-impl", type=int, default=2, choices=[0, 1, 2],
+                    help="attention backward kernels: 2 tcgen05, 1 mma, 0 CUDA cores")
     ap.add_argument("--orient", default="kn", choices=["kn", "kk", "nn"],
                     help="gemm operand majorness: kn = x.W (forward), kk = dy.W^T (dgrad), "
                          "nn = x^T.dy (wgrad)")
@@ -372,7 +374,8 @@ def run_kernel(args):
 
         def bwd():
             assert P.lib.llm_kernel_attention_bwd_bf16(p(qkv), p(o), p(do), p(lse), p(Dv),
-                                                       p(dqkv), Bt, T, H, Hkv, hd, 1, None) == 0
+                                                       p(dqkv), Bt, T, H, Hkv, hd, args.bwd_impl,
+                                                       None) == 0
         causal = Bt * H * (T * (T + 1) / 2) * hd
         res = {}
         for name, fn, fl in (("fwd", fwd, 4.0 * causal), ("bwd", bwd, 8.0 * causal)):
@@ -393,7 +396,7 @@ def run_kernel(args):
             ms = tot / args.steps
             res[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12}
         print(json.dumps({"kernel": "attention", "shape": args.shape, "fwd_impl": args.fwd_impl,
-                          **res}), flush=True)
+                          "bwd_impl": args.bwd_impl, **res}), flush=True)
         return
     for _ in range(args.warmup):
         call()

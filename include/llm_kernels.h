@@ -40,9 +40,13 @@ int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_t lda, int 
  * row.  Backward: from d_o, d_lse and d_dout (bf16, like d_o) writes d_dqkv
  * (bf16, like d_qkv; every element written) and d_D float32 [batch, n_head,
  * ctx] = rowsum(dout * o) as scratch.  tensor_cores selects the kernels:
- * 2 = the tcgen05/TMEM forward (head_dim 64; the backward then uses the mma
- * kernels), 1 = the warp-level mma kernels (head_dim 32 or 64), 0 = the
- * CUDA-core kernels; LLM_ERR_ARG if the selection does not cover head_dim. */
+ * 2 = the tcgen05/TMEM kernels (head_dim 64; pointers 16-byte aligned),
+ * 1 = the warp-level mma kernels (head_dim 32 or 64), 0 = the CUDA-core
+ * kernels; LLM_ERR_ARG if the selection does not cover head_dim.  The calls
+ * are asynchronous on `stream`.  The tcgen05 kernels bound every internal
+ * wait (2 s); a wait that runs out ends the kernel early (outputs incomplete)
+ * and is recorded only in a library-owned device word, which these entries do
+ * not report (the training-step entries do report it, as LLM_ERR_TIMEOUT). */
 int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float *d_lse, int batch, int ctx,
                                   int n_head, int n_kv_head, int head_dim, int tensor_cores,
                                   void *stream);

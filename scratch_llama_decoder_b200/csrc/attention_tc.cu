@@ -23,10 +23,6 @@
 // reference, so O / l is exact.  The MMA order per block j is Q K_{j+1}^T, then
 // P_j V_j, so the tensor core works while the softmax of block j runs.
 // Every wait is bounded (FLAG_TIMEOUT, then drain and free TMEM).
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "tcgen05.cuh"
@@ -49,46 +45,6 @@ constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is re
 // shared memory: Q | K[2] | V[2] | barriers
 constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 2 * 128 * 4 + 1024;
 
-LLM_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bd, uint32_t id, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bd), "r"(id), "r"(acc)
-      : "memory");
-}
-LLM_DEV void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16};" ::"r"(taddr),
-      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
-      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
-      "r"(w[15])
-      : "memory");
-}
-
-// Two 32-column TMEM loads in flight, one wait.
-LLM_DEV void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
-#define LD32(OFF)                                                                                \
-  asm volatile(                                                                                  \
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"  \
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"        \
-      : "=r"(r[OFF + 0]), "=r"(r[OFF + 1]), "=r"(r[OFF + 2]), "=r"(r[OFF + 3]),                \
-        "=r"(r[OFF + 4]), "=r"(r[OFF + 5]), "=r"(r[OFF + 6]), "=r"(r[OFF + 7]),                \
-        "=r"(r[OFF + 8]), "=r"(r[OFF + 9]), "=r"(r[OFF + 10]), "=r"(r[OFF + 11]),              \
-        "=r"(r[OFF + 12]), "=r"(r[OFF + 13]), "=r"(r[OFF + 14]), "=r"(r[OFF + 15]),            \
-        "=r"(r[OFF + 16]), "=r"(r[OFF + 17]), "=r"(r[OFF + 18]), "=r"(r[OFF + 19]),            \
-        "=r"(r[OFF + 20]), "=r"(r[OFF + 21]), "=r"(r[OFF + 22]), "=r"(r[OFF + 23]),            \
-        "=r"(r[OFF + 24]), "=r"(r[OFF + 25]), "=r"(r[OFF + 26]), "=r"(r[OFF + 27]),            \
-        "=r"(r[OFF + 28]), "=r"(r[OFF + 29]), "=r"(r[OFF + 30]), "=r"(r[OFF + 31])             \
-      : "r"(taddr + OFF))
-  LD32(0);
-  LD32(32);
-#undef LD32
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 64; i++) v[i] = __uint_as_float(r[i]);
-}
 // Named barrier of the softmax warps (id 1).
 LLM_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * SM_WARPS) : "memory"); }
 
@@ -354,30 +310,15 @@ bool attn_tc_covers(DType dt, int hd, int T) { return dt == DT_BF16 && hd == 64 
 bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
                  int *flag, cudaStream_t s) {
   using namespace attn_tc;
-  if (hd != HD || !flag || ((uintptr_t)qkv & 15)) return false;
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (hd != HD || !flag) return false;
   static bool init = false;
   if (!init) {
-    cudaDriverEntryPointQueryResult q;
-    void *fn = nullptr;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
     cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     init = true;
   }
-  if (!encode) return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd;
   CUtensorMap map;
-  cuuint64_t dims[2] = {(cuuint64_t)qkvw, (cuuint64_t)B * T};
-  cuuint64_t strides[1] = {(cuuint64_t)qkvw * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t es[2] = {1, 1};
-  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(qkv), dims, strides,
-             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return false;
+  if (!tc::tile_map_bf16(&map, qkv, qkvw, (int64_t)B * T, qkvw, 128)) return false;
   dim3 grid(H, B, (T + BQ - 1) / BQ);
   k_attn_fwd_tc<<<grid, NTHREADS, SMEM_BYTES, s>>>(map, (__nv_bfloat16 *)o, lse, T, H, Hkv,
                                                    1.0f / sqrtf((float)hd), flag);

@@ -1,0 +1,615 @@
+// tcgen05 flash-attention backward for head size 64 (bf16 operands, fp32
+// scores and accumulators).  With the forward's saved row log-sum-exp L and
+// D_i = sum_e dO_ie O_ie, the causal softmax backward of strata's flash
+// attention is, per (query i, key j) pair,
+//     P_ij  = exp(scale * q_i.k_j - L_i)          (0 above the diagonal)
+//     dS_ij = P_ij (dO_i.v_j - D_i)
+//     dQ = scale * dS K,   dK = scale * dS^T Q,   dV = P^T dO,
+// recomputed block by block so no T x T matrix reaches memory.  Two kernels,
+// both with 128 x 128 blocks, one CTA per SM (512 TMEM columns), 10 warps:
+//   warp 0      TMA producer (Q/dO or K/V once, the other pair through a
+//               2-deep ring);
+//   warp 1      TMEM allocation and the MMA issuer;
+//   warps 2..9  elementwise warps, two per TMEM lane quarter: thread = one
+//               row of the block (TMEM lane) and one half (64 columns).
+// dQ kernel (grid H x B x query blocks, longest rows first), per key block j:
+//   S = Q K_j^T and dP = dO V_j^T (M 128, N 128, K 64; operands K-major in
+//   shared memory) into TMEM; the elementwise warps read both rows, release
+//   them (so the next block's products start), form dS in bf16 and put it back
+//   into TMEM; dQ += dS K_j (M 128, N 64, K 128; A = dS from TMEM, B = K_j
+//   MN-major).  The same kernel first forms D (one dot product per row) and
+//   stores it for the second kernel.
+// dK/dV kernel (grid Hkv x B x key blocks, first key blocks first), per (query
+//   head of the group, query block >= this key block):
+//   S^T = K Q^T and dP^T = V dO^T into TMEM; P^T and dS^T back into TMEM as
+//   bf16; dV += P^T dO and dK += dS^T Q (A from TMEM, B = dO / Q MN-major).
+//   The per-query L and D of each step travel with its Q/dO tiles.
+// dQ and dK leave through the backward of the rotate-half RoPE (when tables
+// are given), then scale, bf16.  No atomics: every output element is written
+// once by the CTA that owns its row.  Every wait is bounded (FLAG_TIMEOUT,
+// then drain and free TMEM).
+#include "common.cuh"
+#include "gemm_tc.h"
+#include "tcgen05.cuh"
+
+namespace llm {
+namespace attn_tc_bwd {
+
+using namespace tc;
+
+constexpr int BQ = 128, BK = 128, HD = 64;
+constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
+constexpr int STAGES = 2;
+constexpr int EW_WARPS = 8;  // elementwise warps
+constexpr int NTHREADS = 64 + 32 * EW_WARPS;
+constexpr int TMEM_COLS = 512;
+constexpr float LOG2E = 1.4426950408889634f;
+
+// dQ kernel: TMEM columns; shared memory Q | dO | K[2] | V[2] | barriers | red
+constexpr int DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DS = 256, DQ_COL_DQ = 320;
+constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + 256 + 2 * 128 * 4;
+// dK/dV kernel: TMEM columns; shared memory K | V | Q[2] | dO[2] | L[2] | D[2] | barriers
+constexpr int KV_COL_S = 0, KV_COL_DP = 128, KV_COL_P = 256, KV_COL_DS = 320, KV_COL_DV = 384,
+              KV_COL_DK = 448;
+constexpr int KV_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + 256 + 1024;
+
+// Named barrier of the elementwise warps (id 1).
+LLM_DEV void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EW_WARPS) : "memory"); }
+
+// Lane 0 waits on the phase; the result is shared by the warp, and
+// __syncwarp orders the other lanes' later accesses after lane 0's acquire.
+LLM_DEV bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_sh, int *gflag) {
+  int got = 0;
+  if ((threadIdx.x & 31) == 0) got = mbar_wait(bar, parity, abort_sh, gflag) ? 1 : 0;
+  got = __shfl_sync(0xffffffffu, got, 0);
+  __syncwarp();
+  return got != 0;
+}
+
+// Backward of the rotate-half RoPE on 16 column pairs (c, c + 32) of one row:
+// (x, y) <- (x cos + y sin, y cos - x sin), angle table entries ct[i], st[i].
+LLM_DEV void rope_bwd16(float (&x)[16], float (&y)[16], const float *ct, const float *st) {
+#pragma unroll
+  for (int i = 0; i < 16; i += 4) {
+    const float4 c = *reinterpret_cast<const float4 *>(ct + i);
+    const float4 s = *reinterpret_cast<const float4 *>(st + i);
+    const float cv[4] = {c.x, c.y, c.z, c.w}, sv[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const float a = x[i + e], b = y[i + e];
+      x[i + e] = a * cv[e] + b * sv[e];
+      y[i + e] = b * cv[e] - a * sv[e];
+    }
+  }
+}
+
+// 16 consecutive bf16 values (v * mul) to a 32-byte aligned address.
+LLM_DEV void store16(__nv_bfloat16 *dst, const float (&v)[16], float mul) {
+  uint4 a = make_uint4(pack_bf16(v[0] * mul, v[1] * mul), pack_bf16(v[2] * mul, v[3] * mul),
+                       pack_bf16(v[4] * mul, v[5] * mul), pack_bf16(v[6] * mul, v[7] * mul));
+  uint4 b = make_uint4(pack_bf16(v[8] * mul, v[9] * mul), pack_bf16(v[10] * mul, v[11] * mul),
+                       pack_bf16(v[12] * mul, v[13] * mul), pack_bf16(v[14] * mul, v[15] * mul));
+  reinterpret_cast<uint4 *>(dst)[0] = a;
+  reinterpret_cast<uint4 *>(dst)[1] = b;
+}
+
+LLM_DEV void tmem_alloc_512(uint32_t *dst) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(TMEM_COLS)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+LLM_DEV void tmem_free_512(uint32_t tmem) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+               : "memory");
+}
+// Bounded wait used only on the way out (the copies / MMAs of this thread).
+LLM_DEV void drain_wait(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = gtimer();
+  while (!mbar_try(bar, parity) && gtimer() - t0 < WAIT_NS) {
+  }
+}
+
+// ------------------------------------------------------------------- dQ
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_attn_dq_tc(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                 const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dout,
+                 const float *__restrict__ lse, float *__restrict__ Dv,
+                 __nv_bfloat16 *__restrict__ dqkv, const float *__restrict__ cos_t,
+                 const float *__restrict__ sin_t, int T, int H, int Hkv, float scale, int *gflag) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sQ = smem, *sdO = smem + TILE_BYTES, *sK = smem + 2 * TILE_BYTES,
+          *sV = sK + STAGES * TILE_BYTES;
+  uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
+  uint32_t *tmem_sh = (uint32_t *)(bars + 24);
+  volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
+  float *red = (float *)(bars + 32);  // [2][128] half-row partial dot products
+  const uint32_t b0 = smem_u32(bars);
+  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
+                 v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
+                 ds_full = b0 + 8 * 11, dq_done = b0 + 8 * 12, drain = b0 + 8 * 13;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int g = h / (H / Hkv), d = H * HD, kvd = Hkv * HD;
+  const int64_t ld = d + 2 * kvd;
+  const int q0 = qb * BQ;
+  const int nj = qb + 1;  // causal: key blocks 0..qb (block qb holds the diagonal)
+  const int row_base = b * T;
+
+  if (threadIdx.x == 0) {
+    *abort_sh = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
+      mbar_init(v_full + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, EW_WARPS);
+    mbar_init(ds_full, EW_WARPS);
+    mbar_init(dq_done, 1);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_512(tmem_sh);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int issued = 0;
+      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
+      tma_load_2d(smem_u32(sQ), &tm_qkv, h * HD, row_base + q0, q_full);
+      tma_load_2d(smem_u32(sdO), &tm_do, h * HD, row_base + q0, q_full);
+      for (int j = 0; j < nj; j++) {
+        const int s = j % STAGES;
+        const uint32_t ph = (j / STAGES) & 1;
+        if (!mbar_wait(k_empty + 8 * s, ph ^ 1, abort_sh, gflag)) break;
+        if (!mbar_wait(v_empty + 8 * s, ph ^ 1, abort_sh, gflag)) break;
+        mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
+        tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
+                    k_full + 8 * s);
+        mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
+        tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD, row_base + j * BK,
+                    v_full + 8 * s);
+        issued = j + 1;
+      }
+      // every copy this thread issued has landed before the CTA may exit
+      drain_wait(q_full, 0);
+      for (int j = max(0, issued - STAGES); j < issued; j++) {
+        drain_wait(k_full + 8 * (j % STAGES), (j / STAGES) & 1);
+        drain_wait(v_full + 8 * (j % STAGES), (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
+      constexpr uint32_t ID_DQ = idesc_mn(128, HD, false, true);
+      const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024), dod = sdesc(smem_u32(sdO), 16, 1024);
+      auto issue_sdp = [&](int j) {  // S = Q K_j^T, dP = dO V_j^T
+        const int s = j % STAGES;
+        const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
+        const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; kk++)
+          mma_bf16(tmem + DQ_COL_S, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), ID_S,
+                   kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; kk++)
+          mma_bf16(tmem + DQ_COL_DP, dod + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 2), ID_S,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        mma_commit(v_empty + 8 * s);  // V_j is not read again
+      };
+      bool ok = mbar_wait(q_full, 0, abort_sh, gflag) && mbar_wait(k_full, 0, abort_sh, gflag) &&
+                mbar_wait(v_full, 0, abort_sh, gflag);
+      if (ok) {
+        fence_after();
+        issue_sdp(0);
+      }
+      for (int j = 0; j < nj && ok; j++) {
+        const int s = j % STAGES;
+        if (j + 1 < nj) {
+          // next block's products once the elementwise warps have read S, dP
+          const int s1 = (j + 1) % STAGES;
+          const uint32_t ph1 = ((j + 1) / STAGES) & 1;
+          if (!mbar_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
+              !mbar_wait(v_full + 8 * s1, ph1, abort_sh, gflag) ||
+              !mbar_wait(s_free, j & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          issue_sdp(j + 1);
+        }
+        if (!mbar_wait(ds_full, j & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint64_t kmd = sdesc(smem_u32(sK + s * TILE_BYTES), 8192, 1024);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; kk++)
+          mma_ts(tmem + DQ_COL_DQ, tmem + DQ_COL_DS + kk * 8, kmd + (uint64_t)(kk * 128), ID_DQ,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(k_empty + 8 * s);
+        mma_commit(dq_done);
+      }
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // --------------------------------------------------------- elementwise
+    const int quarter = warp & 3;
+    const int ch = (warp - 2) >> 2;  // which half of the block's columns
+    const int r = quarter * 32 + lane;
+    const int qi = q0 + r;
+    const bool valid = qi < T;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = scale * LOG2E;
+    // D_i = dO_i . O_i, each half-row thread over 32 of the 64 columns
+    float dpart = 0.f;
+    if (valid) {
+      const int64_t off = ((int64_t)row_base + qi) * d + h * HD + ch * 32;
+      const uint4 *po = reinterpret_cast<const uint4 *>(o + off);
+      const uint4 *pd = reinterpret_cast<const uint4 *>(dout + off);
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const uint4 a = po[e], c = pd[e];
+        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&c);
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const float2 fa = __bfloat1622float2(ha[k]), fc = __bfloat1622float2(hc[k]);
+          dpart += fa.x * fc.x + fa.y * fc.y;
+        }
+      }
+    }
+    red[ch * 128 + r] = dpart;
+    ew_sync();
+    const float Di = red[r] + red[128 + r];
+    // rows past T get L = +inf, so every P of theirs is 0
+    const float L2 = valid ? lse[((int64_t)b * H + h) * T + qi] * LOG2E : INFINITY;
+    if (ch == 0 && valid) Dv[((int64_t)b * H + h) * T + qi] = Di;
+    bool ok = true;
+    for (int j = 0; j < nj && ok; j++) {
+      if (!warp_wait(s_full, j & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      float sv[64], dv[64];
+      tmem_ld64(tmem + lane_off + DQ_COL_S + ch * 64, sv);
+      tmem_ld64(tmem + lane_off + DQ_COL_DP + ch * 64, dv);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S and dP now
+      const int k0 = j * BK + ch * 64;
+      const bool diag = (j == qb);  // only the diagonal block masks (keys >= T lie above it)
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
+        if (diag) {
+          if (k0 + i > qi) p0 = 0.f;
+          if (k0 + i + 1 > qi) p1 = 0.f;
+        }
+        w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
+      }
+      // dS of the previous block is free once its dQ product has completed
+      if (j > 0) {
+        if (!warp_wait(dq_done, (j - 1) & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < 2; c++) {
+        uint32_t (&wc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&w[c * 16]);
+        tmem_st16(tmem + lane_off + DQ_COL_DS + ch * 32 + c * 16, wc);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
+    }
+    if (ok) ok = warp_wait(dq_done, (nj - 1) & 1, abort_sh, gflag);
+    if (ok) {
+      fence_after();
+      // column pairs (c, c + 32) of RoPE: this half takes c in [16 ch, 16 ch + 16)
+      float x[16], y[16];
+      tmem_ld16(tmem + lane_off + DQ_COL_DQ + ch * 16, x);
+      tmem_ld16(tmem + lane_off + DQ_COL_DQ + 32 + ch * 16, y);
+      if (valid) {
+        if (cos_t)
+          rope_bwd16(x, y, cos_t + (int64_t)qi * (HD / 2) + ch * 16,
+                     sin_t + (int64_t)qi * (HD / 2) + ch * 16);
+        __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + qi) * ld + h * HD + ch * 16;
+        store16(dst, x, scale);
+        store16(dst + 32, y, scale);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) tmem_free_512(tmem);
+}
+
+// ---------------------------------------------------------------- dK, dV
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_attn_dkv_tc(const __grid_constant__ CUtensorMap tm_qkv,
+                  const __grid_constant__ CUtensorMap tm_do, const float *__restrict__ lse,
+                  const float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
+                  const float *__restrict__ cos_t, const float *__restrict__ sin_t, int T, int H,
+                  int Hkv, float scale, int *gflag) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *sK = smem, *sV = smem + TILE_BYTES, *sQ = smem + 2 * TILE_BYTES,
+          *sdO = sQ + STAGES * TILE_BYTES;
+  float *sL = (float *)(sdO + STAGES * TILE_BYTES);  // [STAGES][128] L * log2(e)
+  float *sD = sL + STAGES * 128;                      // [STAGES][128] D
+  uint64_t *bars = (uint64_t *)(sD + STAGES * 128);
+  uint32_t *tmem_sh = (uint32_t *)(bars + 24);
+  volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
+  const uint32_t b0 = smem_u32(bars);
+  const uint32_t kv_full = b0, q_full = b0 + 8, q_empty = b0 + 8 * 3, ld_full = b0 + 8 * 5,
+                 s_full = b0 + 8 * 7, s_free = b0 + 8 * 8, p_full = b0 + 8 * 9,
+                 pv_done = b0 + 8 * 10, drain = b0 + 8 * 11;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int nkb = gridDim.z, kb = blockIdx.z;
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int grp = H / Hkv, d = H * HD, kvd = Hkv * HD;
+  const int64_t ld = d + 2 * kvd;
+  const int k0 = kb * BK;
+  const int nq = nkb - kb;       // query blocks kb..nkb-1 see this key block
+  const int nsteps = grp * nq;   // (query head of the group, query block) pairs
+  const int row_base = b * T;
+
+  if (threadIdx.x == 0) {
+    *abort_sh = 0;
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(q_full + 8 * s, 1);
+      mbar_init(q_empty + 8 * s, 1);
+      mbar_init(ld_full + 8 * s, 32);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, EW_WARPS);
+    mbar_init(p_full, EW_WARPS);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_512(tmem_sh);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_sh;
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (warp)
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * TILE_BYTES);
+      tma_load_2d(smem_u32(sK), &tm_qkv, d + g * HD, row_base + k0, kv_full);
+      tma_load_2d(smem_u32(sV), &tm_qkv, d + kvd + g * HD, row_base + k0, kv_full);
+    }
+    int issued = 0;
+    for (int st = 0; st < nsteps; st++) {
+      const int s = st % STAGES;
+      const uint32_t ph = (st / STAGES) & 1;
+      const int hq = g * grp + st / nq, qb = kb + st % nq;
+      // the slot (tiles and L, D) of step st - 2 is free once its products completed
+      if (!warp_wait(q_empty + 8 * s, ph ^ 1, abort_sh, gflag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full + 8 * s, 2 * TILE_BYTES);
+        tma_load_2d(smem_u32(sQ + s * TILE_BYTES), &tm_qkv, hq * HD, row_base + qb * BQ,
+                    q_full + 8 * s);
+        tma_load_2d(smem_u32(sdO + s * TILE_BYTES), &tm_do, hq * HD, row_base + qb * BQ,
+                    q_full + 8 * s);
+      }
+      const int64_t base = ((int64_t)b * H + hq) * T;
+#pragma unroll
+      for (int i = lane; i < BQ; i += 32) {
+        const int qi = qb * BQ + i;
+        // queries past T get L = +inf, so every P of theirs is 0
+        sL[s * 128 + i] = qi < T ? lse[base + qi] * LOG2E : INFINITY;
+        sD[s * 128 + i] = qi < T ? Dv[base + qi] : 0.f;
+      }
+      mbar_arrive(ld_full + 8 * s);
+      issued = st + 1;
+    }
+    if (lane == 0) {
+      drain_wait(kv_full, 0);
+      for (int st = max(0, issued - STAGES); st < issued; st++)
+        drain_wait(q_full + 8 * (st % STAGES), (st / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      constexpr uint32_t ID_S = idesc_mn(128, BQ, false, false);
+      constexpr uint32_t ID_KV = idesc_mn(128, HD, false, true);
+      const uint64_t kd = sdesc(smem_u32(sK), 16, 1024), vd = sdesc(smem_u32(sV), 16, 1024);
+      auto issue_s = [&](int st) {  // S^T = K Q^T, dP^T = V dO^T
+        const int s = st % STAGES;
+        const uint64_t qd = sdesc(smem_u32(sQ + s * TILE_BYTES), 16, 1024);
+        const uint64_t dod = sdesc(smem_u32(sdO + s * TILE_BYTES), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; kk++)
+          mma_bf16(tmem + KV_COL_S, kd + (uint64_t)(kk * 2), qd + (uint64_t)(kk * 2), ID_S,
+                   kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; kk++)
+          mma_bf16(tmem + KV_COL_DP, vd + (uint64_t)(kk * 2), dod + (uint64_t)(kk * 2), ID_S,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_sh, gflag) && mbar_wait(q_full, 0, abort_sh, gflag);
+      if (ok) {
+        fence_after();
+        issue_s(0);
+      }
+      for (int st = 0; st < nsteps && ok; st++) {
+        const int s = st % STAGES;
+        if (st + 1 < nsteps) {
+          const int s1 = (st + 1) % STAGES;
+          const uint32_t ph1 = ((st + 1) / STAGES) & 1;
+          if (!mbar_wait(q_full + 8 * s1, ph1, abort_sh, gflag) ||
+              !mbar_wait(s_free, st & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          issue_s(st + 1);
+        }
+        if (!mbar_wait(p_full, st & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint64_t qm = sdesc(smem_u32(sQ + s * TILE_BYTES), 8192, 1024);
+        const uint64_t dom = sdesc(smem_u32(sdO + s * TILE_BYTES), 8192, 1024);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; kk++)
+          mma_ts(tmem + KV_COL_DV, tmem + KV_COL_P + kk * 8, dom + (uint64_t)(kk * 128), ID_KV,
+                 (st > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; kk++)
+          mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DS + kk * 8, qm + (uint64_t)(kk * 128), ID_KV,
+                 (st > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(q_empty + 8 * s);
+        mma_commit(pv_done);
+      }
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // --------------------------------------------------------- elementwise
+    const int quarter = warp & 3;
+    const int ch = (warp - 2) >> 2;  // which half of the block's query columns
+    const int r = quarter * 32 + lane;
+    const int kj = k0 + r;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = scale * LOG2E;
+    bool ok = true;
+    for (int st = 0; st < nsteps && ok; st++) {
+      const int s = st % STAGES;
+      const int qb = kb + st % nq;
+      if (!warp_wait(s_full, st & 1, abort_sh, gflag) ||
+          !warp_wait(ld_full + 8 * s, (st / STAGES) & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      float sv[64], dv[64];
+      tmem_ld64(tmem + lane_off + KV_COL_S + ch * 64, sv);
+      tmem_ld64(tmem + lane_off + KV_COL_DP + ch * 64, dv);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      const int qc0 = qb * BQ + ch * 64;
+      const bool diag = (qb == kb);  // keys >= T occur only in this case, above the diagonal
+      const float *Ls = sL + s * 128 + ch * 64, *Ds = sD + s * 128 + ch * 64;
+      uint32_t wp[32], wd[32];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        float p0 = ex2(fmaf(sv[i], sl2, -Ls[i])), p1 = ex2(fmaf(sv[i + 1], sl2, -Ls[i + 1]));
+        if (diag) {
+          if (kj > qc0 + i) p0 = 0.f;
+          if (kj > qc0 + i + 1) p1 = 0.f;
+        }
+        wp[i / 2] = pack_bf16(p0, p1);
+        wd[i / 2] = pack_bf16(p0 * (dv[i] - Ds[i]), p1 * (dv[i + 1] - Ds[i + 1]));
+      }
+      // P^T and dS^T of the previous step are free once its products completed
+      if (st > 0) {
+        if (!warp_wait(pv_done, (st - 1) & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < 2; c++) {
+        uint32_t (&pc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&wp[c * 16]);
+        uint32_t (&dc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&wd[c * 16]);
+        tmem_st16(tmem + lane_off + KV_COL_P + ch * 32 + c * 16, pc);
+        tmem_st16(tmem + lane_off + KV_COL_DS + ch * 32 + c * 16, dc);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) ok = warp_wait(pv_done, (nsteps - 1) & 1, abort_sh, gflag);
+    if (ok) {
+      fence_after();
+      float x[16], y[16];
+      __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + kj) * ld + d + g * HD + ch * 16;
+      tmem_ld16(tmem + lane_off + KV_COL_DK + ch * 16, x);
+      tmem_ld16(tmem + lane_off + KV_COL_DK + 32 + ch * 16, y);
+      if (kj < T) {
+        if (cos_t)
+          rope_bwd16(x, y, cos_t + (int64_t)kj * (HD / 2) + ch * 16,
+                     sin_t + (int64_t)kj * (HD / 2) + ch * 16);
+        store16(dst, x, scale);
+        store16(dst + 32, y, scale);
+      }
+      tmem_ld16(tmem + lane_off + KV_COL_DV + ch * 16, x);
+      tmem_ld16(tmem + lane_off + KV_COL_DV + 32 + ch * 16, y);
+      if (kj < T) {
+        store16(dst + kvd, x, 1.f);
+        store16(dst + kvd + 32, y, 1.f);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) tmem_free_512(tmem);
+}
+
+}  // namespace attn_tc_bwd
+
+// Host side: tensor maps over qkv [B*T, qkvw] and dout [B*T, H*hd] (box 64 x
+// 128); the dQ kernel runs first (it also writes D), then the dK/dV kernel.
+bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
+                 void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
+                 const float *sin_t, int *flag, cudaStream_t s) {
+  using namespace attn_tc_bwd;
+  if (hd != HD || !flag || ((uintptr_t)o & 15) || ((uintptr_t)dqkv & 15) ||
+      ((uintptr_t)cos_t & 15) || ((uintptr_t)sin_t & 15) || (!cos_t != !sin_t))
+    return false;
+  static bool init = false;
+  if (!init) {
+    cudaFuncSetAttribute(k_attn_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
+    cudaFuncSetAttribute(k_attn_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, KV_SMEM);
+    init = true;
+  }
+  const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd, dw = (int64_t)H * hd;
+  CUtensorMap mq, md;
+  if (!tc::tile_map_bf16(&mq, qkv, qkvw, (int64_t)B * T, qkvw, 128) ||
+      !tc::tile_map_bf16(&md, dout, dw, (int64_t)B * T, dw, 128))
+    return false;
+  const int nb = (T + BQ - 1) / BQ;
+  const float scale = 1.0f / sqrtf((float)hd);
+  k_attn_dq_tc<<<dim3(H, B, nb), NTHREADS, DQ_SMEM, s>>>(
+      mq, md, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dout, lse, Dbuf,
+      (__nv_bfloat16 *)dqkv, cos_t, sin_t, T, H, Hkv, scale, flag);
+  k_attn_dkv_tc<<<dim3(Hkv, B, nb), NTHREADS, KV_SMEM, s>>>(mq, md, lse, Dbuf,
+                                                            (__nv_bfloat16 *)dqkv, cos_t, sin_t,
+                                                            T, H, Hkv, scale, flag);
+  count_launch(2);
+  return true;
+}
+
+}  // namespace llm

@@ -532,9 +532,12 @@ void attention_fwd(TcPlan *p, const void *qkv, void *o, float *lse, DType dt, in
   if (attn_mma_covers(dt, hd)) attn_fwd_mma(qkv, o, lse, B, T, H, Hkv, hd, s);
   else attn_fwd_simt(qkv, o, lse, dt, B, T, H, Hkv, hd, s);
 }
-void attention_bwd(TcPlan *, const void *qkv, const void *o, const void *dout, const float *lse,
+void attention_bwd(TcPlan *p, const void *qkv, const void *o, const void *dout, const float *lse,
                    float *Dbuf, void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd,
                    const float *cos_t, const float *sin_t, cudaStream_t s) {
+  if (p && p->flag && attn_tc_covers(dt, hd, T) &&
+      attn_bwd_tc(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, hd, cos_t, sin_t, p->flag, s))
+    return;
   if (attn_mma_covers(dt, hd)) {
     attn_bwd_mma(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, hd, cos_t, sin_t, s);
     return;

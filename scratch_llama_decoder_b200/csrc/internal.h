@@ -99,6 +99,12 @@ void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float 
 bool attn_tc_covers(DType dt, int hd, int T);
 bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
                  int *flag, cudaStream_t s);
+// tcgen05 backward (dQ kernel, which also writes Dbuf, then dK/dV kernel);
+// same arguments as attn_bwd_mma plus the time-out flag.  False (nothing
+// launched) when it does not cover the arguments.
+bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
+                 void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
+                 const float *sin_t, int *flag, cudaStream_t s);
 
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;

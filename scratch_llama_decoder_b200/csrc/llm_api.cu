@@ -582,6 +582,15 @@ extern "C" int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, 
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
 
+// Time-out flag of the tcgen05 attention kernels called through the kernel
+// entries: one library-owned device word.
+static int *attn_kernel_flag() {
+  static int *flag = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] { cudaMalloc(&flag, sizeof(int)); cudaMemset(flag, 0, sizeof(int)); });
+  return flag;
+}
+
 static bool attn_args_ok(const void *a, const void *b, int B, int T, int H, int Hkv, int hd) {
   return a && b && B >= 1 && T >= 1 && H >= 1 && Hkv >= 1 && H % Hkv == 0 && hd >= 2 &&
          hd % 2 == 0 && hd <= 128;
@@ -595,10 +604,7 @@ extern "C" int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float
   g_launches = 0;
   cudaStream_t s = (cudaStream_t)stream;
   if (tensor_cores == 2) {
-    // tcgen05 kernel: its time-out flag is a library-owned device word
-    static int *flag = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] { cudaMalloc(&flag, sizeof(int)); cudaMemset(flag, 0, sizeof(int)); });
+    int *flag = attn_kernel_flag();
     if (!flag || !attn_tc_covers(DT_BF16, head_dim, ctx) ||
         !attn_fwd_tc(d_qkv, d_o, d_lse, batch, ctx, n_head, n_kv_head, head_dim, flag, s))
       return LLM_ERR_ARG;
@@ -621,7 +627,13 @@ extern "C" int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o,
     return LLM_ERR_ARG;
   g_launches = 0;
   cudaStream_t s = (cudaStream_t)stream;
-  if (tensor_cores) {
+  if (tensor_cores == 2) {
+    int *flag = attn_kernel_flag();
+    if (!flag || !attn_tc_covers(DT_BF16, head_dim, ctx) ||
+        !attn_bwd_tc(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, batch, ctx, n_head, n_kv_head,
+                     head_dim, nullptr, nullptr, flag, s))
+      return LLM_ERR_ARG;
+  } else if (tensor_cores == 1) {
     if (!attn_mma_covers(DT_BF16, head_dim)) return LLM_ERR_ARG;
     attn_bwd_mma(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, batch, ctx, n_head, n_kv_head, head_dim,
                  nullptr, nullptr, s);
