@@ -3,26 +3,30 @@
 // scores in memory, only the row log-sum-exp saved) on the 5th-generation
 // tensor cores.
 //
-// One CTA = 128 queries of one (batch, head); key blocks of 128.  6 warps:
+// One CTA = 128 queries of one (batch, head); key blocks of 128.  11 warps:
 //   warp 0      TMA producer: the Q tile once, K and V tiles into 2-deep rings;
-//   warp 1      TMEM allocation (256 columns) and the MMA issuer:
-//                 S  = Q K^T     (M 128, N 128, K 64; both operands K-major in
-//                                 shared memory)              -> TMEM [0,128)
-//                 O += P V       (M 128, N 64, K 128; A = P from TMEM, B = V
-//                                 MN-major in shared memory)  -> TMEM [128,192)
+//   warp 1      TMEM allocation and MMA issuer A:
+//                 S    = Q K^T          (M 128, N 128, K 64; both operands
+//                                        K-major in shared memory) -> TMEM S
+//                 O_a += P_a V[0:64]    (M 128, N 64, K 64; A = P_a from TMEM,
+//                                        B = V MN-major)           -> TMEM O_a
+//   warp 10     MMA issuer B:  O_b += P_b V[64:128]                -> TMEM O_b
 //   warps 2..9  softmax, two warps per TMEM lane quarter: thread = one query
-//               row (TMEM lane) and one half (64 keys) of the block.  The
-//               half-row is loaded into registers in one TMEM round trip and
-//               S is released at once (so the MMA warp runs the next block's
-//               Q K^T during this block's exponentials); the two halves'
-//               maxima meet in shared memory; P goes back to TMEM [192,256)
-//               as packed bf16.
-// The running maximum is lazy: the reference maximum of a row moves only when
-// a block's maximum exceeds it by more than 2^8, so P values stay below 256
-// and O (in TMEM) is rescaled only then; O and the row sum always share one
-// reference, so O / l is exact.  The MMA order per block j is Q K_{j+1}^T, then
-// P_j V_j, so the tensor core works while the softmax of block j runs.
-// Every wait is bounded (FLAG_TIMEOUT, then drain and free TMEM).
+//               row (TMEM lane) and one half of the block's keys (a: keys
+//               0..63, b: 64..127).
+// The two key halves are two independent online softmaxes (split-K inside the
+// CTA): each half-row thread keeps its own running maximum m, sum l and
+// accumulator O_x, so no thread waits for another inside the key loop; the
+// halves meet once at the end, O = (2^(m_a-m) O_a + 2^(m_b-m) O_b) /
+// (2^(m_a-m) l_a + 2^(m_b-m) l_b) with m = max(m_a, m_b).  The running maximum
+// is lazy: the reference of a half-row moves only when a block's maximum
+// exceeds it by more than 2^8, so P stays below 256 and O_x is rescaled only
+// then; O_x and l_x always share one reference.  The half-row is read from
+// TMEM in one round trip and S is released at once, so Q K_{j+1}^T runs during
+// block j's exponentials.  MMAs are issued by whole converged warps (one
+// elected lane), from two warps because one warp issues a tcgen05.mma only
+// every ~127 cycles whatever N is.  Every wait is bounded (FLAG_TIMEOUT, then
+// drain and free TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "tcgen05.cuh"
@@ -36,17 +40,27 @@ constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 2;
 constexpr int SM_WARPS = 8;  // softmax warps
-constexpr int NTHREADS = 64 + 32 * SM_WARPS;
-constexpr int TMEM_COLS = 256;
-constexpr int COL_S = 0, COL_O = 128, COL_P = 192;
+constexpr int MMA_B_WARP = 2 + SM_WARPS;
+constexpr int NTHREADS = 32 * (MMA_B_WARP + 1);
+constexpr int TMEM_COLS = 512;
+constexpr int COL_S = 0, COL_P = 128, COL_OA = 192, COL_OB = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
-// shared memory: Q | K[2] | V[2] | barriers
-constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 2 * 128 * 4 + 1024;
+// shared memory: Q | K[2] | V[2] | barriers | red
+constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 4 * 128 * 4 + 1024;
 
-// Named barrier of the softmax warps (id 1).
-LLM_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * SM_WARPS) : "memory"); }
+// Named barrier of the softmax warps (id 1) that ANDs a flag over them.
+LLM_DEV bool softmax_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(32 * SM_WARPS)
+      : "memory");
+  return r != 0;
+}
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16 *__restrict__ o,
@@ -57,11 +71,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
   uint32_t *tmem_sh = (uint32_t *)(bars + 24);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
-  float *red = (float *)(bars + 32);  // [2][128]: per-half row maxima / sums
+  float *red = (float *)(bars + 32);  // [4][128]: m_a, m_b, l_a, l_b per row
   const uint32_t b0 = smem_u32(bars);
   const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
                  v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
-                 p_full = b0 + 8 * 11, o_done = b0 + 8 * 12, drain = b0 + 8 * 13;
+                 p_full = b0 + 8 * 11,   // [2]: half a, half b
+                 o_done = b0 + 8 * 13,   // [2]
+                 drain = b0 + 8 * 15;    // [2]: one per MMA warp
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -77,13 +93,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(k_full + 8 * s, 1);
       mbar_init(k_empty + 8 * s, 1);
       mbar_init(v_full + 8 * s, 1);
-      mbar_init(v_empty + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 2);  // both P V halves read V_j
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, SM_WARPS);
-    mbar_init(p_full, SM_WARPS);
-    mbar_init(o_done, 1);
-    mbar_init(drain, 1);
+    for (int x = 0; x < 2; x++) {
+      mbar_init(p_full + 8 * x, SM_WARPS / 2);
+      mbar_init(o_done + 8 * x, 1);
+      mbar_init(drain + 8 * x, 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -130,125 +148,135 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // --------------------------------------------------------- MMA issuer
-      constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
-      constexpr uint32_t ID_O = idesc_mn(128, HD, false, true);
-      const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
-      auto issue_s = [&](int j) {  // S = Q K_j^T into TMEM [0,128)
-        const int s = j % STAGES;
-        const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
+  } else if (warp == 1 || warp == MMA_B_WARP) {
+    // ------------------------------------- MMA issuers (whole warps)
+    const int x = warp == 1 ? 0 : 1;  // which key half's P V this warp issues
+    constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
+    constexpr uint32_t ID_O = idesc_mn(128, HD, false, true);
+    const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
+    auto issue_s = [&](int j) {  // S = Q K_j^T
+      const int s = j % STAGES;
+      const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; kk++)
-          mma_bf16(tmem + COL_S, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), ID_S,
+      for (int kk = 0; kk < HD / 16; kk++)
+        mma_bf16_e(tmem + COL_S, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), ID_S,
                    kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        mma_commit(k_empty + 8 * s);
-      };
-      bool ok = mbar_wait(q_full, 0, abort_sh, gflag) && mbar_wait(k_full, 0, abort_sh, gflag);
+      mma_commit_e(s_full);
+      mma_commit_e(k_empty + 8 * s);
+    };
+    bool ok = true;
+    if (x == 0) {
+      ok = warp_wait(q_full, 0, abort_sh, gflag) && warp_wait(k_full, 0, abort_sh, gflag);
       if (ok) {
         fence_after();
         issue_s(0);
       }
-      for (int j = 0; j < nj && ok; j++) {
-        const int s = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
-        if (j + 1 < nj) {
-          // next block's scores once the softmax has read this block's S
-          const int s1 = (j + 1) % STAGES;
-          const uint32_t ph1 = ((j + 1) / STAGES) & 1;
-          if (!mbar_wait(k_full + 8 * s1, ph1, abort_sh, gflag)) { ok = false; break; }
-          if (!mbar_wait(s_free, j & 1, abort_sh, gflag)) { ok = false; break; }
-          fence_after();
-          issue_s(j + 1);
+    }
+    for (int j = 0; j < nj && ok; j++) {
+      const int s = j % STAGES;
+      const uint32_t ph = (j / STAGES) & 1;
+      if (x == 0 && j + 1 < nj) {
+        // next block's scores once the softmax has read this block's S
+        const int s1 = (j + 1) % STAGES;
+        const uint32_t ph1 = ((j + 1) / STAGES) & 1;
+        if (!warp_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
+            !warp_wait(s_free, j & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
         }
-        if (!mbar_wait(p_full, j & 1, abort_sh, gflag)) { ok = false; break; }
-        if (!mbar_wait(v_full + 8 * s, ph, abort_sh, gflag)) { ok = false; break; }
         fence_after();
-        const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 8192, 1024);
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; kk++)
-          mma_ts(tmem + COL_O, tmem + COL_P + kk * 8, vd + (uint64_t)(kk * 128), ID_O,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(v_empty + 8 * s);
-        mma_commit(o_done);
+        issue_s(j + 1);
       }
-      mma_commit(drain);
+      if (!warp_wait(p_full + 8 * x, j & 1, abort_sh, gflag) ||
+          !warp_wait(v_full + 8 * s, ph, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      // O_x += P_x V[64x : 64x + 64]: 4 K-steps of 16 keys
+      const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 8192, 1024);
+      const uint32_t col_o = x ? COL_OB : COL_OA;
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++)
+        mma_ts_e(tmem + col_o, tmem + COL_P + x * 32 + kk * 8,
+                 vd + (uint64_t)((x * 4 + kk) * 128), ID_O, (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_e(v_empty + 8 * s);
+      mma_commit_e(o_done + 8 * x);
+    }
+    mma_commit_e(drain + 8 * x);
+    if (lane == 0) {
       unsigned long long t0 = gtimer();
-      while (!mbar_try(drain, 0) && gtimer() - t0 < WAIT_NS) {
+      while (!mbar_try(drain + 8 * x, 0) && gtimer() - t0 < WAIT_NS) {
       }
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
-    const int ch = (warp - 2) >> 2;      // which 64-key half of the block
-    const int r = quarter * 32 + lane;   // row of the tile = TMEM lane
+    const int ch = (warp - 2) >> 2;  // which key half of the block
+    const int r = quarter * 32 + lane;  // row of the tile = TMEM lane
     const int qi = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t col_o = ch ? COL_OB : COL_OA;
     const float sl2 = scale * LOG2E;
     float m_ref = -INFINITY, l = 0.f;
-    // Every softmax warp executes the same named barriers on every path: a
-    // failed wait only turns the remaining work off (ok = false), it never
-    // leaves the loop early (bar.sync has no time-out).
     bool ok = true;
-    for (int j = 0; j < nj; j++) {
-      if (ok) {
-        int got = 0;
-        if (lane == 0) got = mbar_wait(s_full, j & 1, abort_sh, gflag) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+    for (int j = 0; j < nj && ok; j++) {
+      if (!warp_wait(s_full, j & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
       }
       fence_after();
       const int k0 = j * BK + ch * 64;
       const bool diag = (j * BK + BK > q0);  // only the diagonal block (or T) masks
       float sv[64];
+      tmem_ld64(tmem + lane_off + COL_S + ch * 64, sv);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
+      // this half-row's block maximum (log2 units), 4 independent chains
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (ok) {
-        tmem_ld64(tmem + lane_off + COL_S + ch * 64, sv);
-        fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
-        // this half's row maximum (log2 units), 4 independent chains
 #pragma unroll
-        for (int i = 0; i < 64; i++) {
-          float x = sv[i] * sl2;
-          if (diag && (k0 + i > qi || k0 + i >= T)) x = -INFINITY;
-          sv[i] = x;
-          m4[i & 3] = fmaxf(m4[i & 3], x);
-        }
+      for (int i = 0; i < 64; i++) {
+        float x = sv[i] * sl2;
+        if (diag && (k0 + i > qi || k0 + i >= T)) x = -INFINITY;
+        sv[i] = x;
+        m4[i & 3] = fmaxf(m4[i & 3], x);
       }
-      red[ch * 128 + r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      softmax_sync();
-      const float mx = fmaxf(red[r], red[128 + r]);
-      softmax_sync();  // both halves read before the next block overwrites red
-      if (!ok) continue;
-      const bool need = mx > m_ref + LAZY;  // true on the first block (m_ref = -inf)
-      // P and O of the previous block are free once its P.V has completed
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // true on the first block with an unmasked key (m_ref = -inf until then)
+      const bool need = mx > m_ref + LAZY;
+      // P_x and O_x of the previous block are free once its P V has completed
       if (j > 0) {
-        int got2 = 0;
-        if (lane == 0) got2 = mbar_wait(o_done, (j - 1) & 1, abort_sh, gflag) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, got2, 0)) { ok = false; continue; }
+        if (!warp_wait(o_done + 8 * ch, (j - 1) & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
         fence_after();
         if (__any_sync(0xffffffffu, need)) {
-          // each half-row warp rescales its 32 of O's 64 columns
-          const float corr = need ? ex2(m_ref - mx) : 1.f;
-          float v[32];
-          tmem_ld32(tmem + lane_off + COL_O + ch * 32, v);
+          const float corr = need ? ex2(m_ref - mx) : 1.f;  // 0 while m_ref = -inf
 #pragma unroll
-          for (int i = 0; i < 32; i++) v[i] *= corr;
-          tmem_st32(tmem + lane_off + COL_O + ch * 32, v);
+          for (int c = 0; c < 2; c++) {
+            float v[32];
+            tmem_ld32(tmem + lane_off + col_o + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[i] *= corr;
+            tmem_st32(tmem + lane_off + col_o + c * 32, v);
+          }
         }
       }
       if (need) {
         if (m_ref != -INFINITY) l *= ex2(m_ref - mx);
         m_ref = mx;
       }
-      // P = 2^(s - m_ref), packed bf16 into this half's 32 TMEM columns
+      // P = 2^(s - m_ref), packed bf16 into this half's 32 TMEM columns; a
+      // half-row with no unmasked key yet (m_ref = -inf) gets P = 0
+      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
       uint32_t w[32];
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
-        const float p0 = ex2(sv[i] - m_ref), p1 = ex2(sv[i + 1] - m_ref);
+        const float p0 = ex2(sv[i] - mr), p1 = ex2(sv[i + 1] - mr);
         l4[(i >> 1) & 3] += p0 + p1;
         w[i / 2] = pack_bf16(p0, p1);
       }
@@ -261,33 +289,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full + 8 * ch);
     }
-    // row sum = both halves' sums (same reference maximum)
-    if (ok) red[ch * 128 + r] = l;
-    softmax_sync();
-    if (ok) {
-      l = red[r] + red[128 + r];
-      int got = 0;
-      if (lane == 0) got = mbar_wait(o_done, (nj - 1) & 1, abort_sh, gflag) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
-    }
-    if (ok) {
+    // the two halves meet: shared reference m, combined sum and output; both
+    // accumulators are complete once both o_done phases of the last block are
+    if (ok)
+      ok = warp_wait(o_done, (nj - 1) & 1, abort_sh, gflag) &&
+           warp_wait(o_done + 8, (nj - 1) & 1, abort_sh, gflag);
+    red[ch * 128 + r] = m_ref;
+    red[256 + ch * 128 + r] = l;
+    // barrier of the softmax warps that also tells whether every one finished
+    if (softmax_all(ok)) {
       fence_after();
-      float v[32];
-      const float inv = 1.f / l;
-      tmem_ld32(tmem + lane_off + COL_O + ch * 32, v);
+      const float ma = red[r], mb = red[128 + r], la = red[256 + r], lb = red[384 + r];
+      const float m = fmaxf(ma, mb);
+      const float fa = ma == -INFINITY ? 0.f : ex2(ma - m);
+      const float fb = mb == -INFINITY ? 0.f : ex2(mb - m);
+      const float lt = la * fa + lb * fb;
+      const float inv = 1.f / lt;
+      float va[32], vb[32];
+      tmem_ld32(tmem + lane_off + COL_OA + ch * 32, va);
+      tmem_ld32(tmem + lane_off + COL_OB + ch * 32, vb);
       if (qi < T) {
         __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + ch * 32;
+        const float ca = fa * inv, cb = fb * inv;
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
-          uint4 q = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv),
-                               pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
-                               pack_bf16(v[i + 4] * inv, v[i + 5] * inv),
-                               pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
-          *reinterpret_cast<uint4 *>(dst + i) = q;
+          uint32_t wv[4];
+#pragma unroll
+          for (int e = 0; e < 4; e++)
+            wv[e] = pack_bf16(va[i + 2 * e] * ca + vb[i + 2 * e] * cb,
+                              va[i + 2 * e + 1] * ca + vb[i + 2 * e + 1] * cb);
+          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
-        if (ch == 0) lse[((int64_t)b * H + h) * T + qi] = (m_ref + log2f(l)) * LN2;
+        if (ch == 0) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
       }
     }
   }

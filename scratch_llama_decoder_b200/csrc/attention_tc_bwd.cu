@@ -6,23 +6,29 @@
 //     dS_ij = P_ij (dO_i.v_j - D_i)
 //     dQ = scale * dS K,   dK = scale * dS^T Q,   dV = P^T dO,
 // recomputed block by block so no T x T matrix reaches memory.  Two kernels,
-// both with 128 x 128 blocks, one CTA per SM (512 TMEM columns), 10 warps:
+// both with 128 x 128 blocks, one CTA per SM (512 TMEM columns), 11 warps:
 //   warp 0      TMA producer (Q/dO or K/V once, the other pair through a
 //               2-deep ring);
-//   warp 1      TMEM allocation and the MMA issuer;
+//   warps 1, 10 MMA issuers A and B (whole converged warps, one elected lane;
+//               one warp issues a tcgen05.mma only every ~127 cycles whatever
+//               N is, so the products are split between two warps); warp 1
+//               also allocates TMEM;
 //   warps 2..9  elementwise warps, two per TMEM lane quarter: thread = one
 //               row of the block (TMEM lane) and one half (64 columns).
 // dQ kernel (grid H x B x query blocks, longest rows first), per key block j:
-//   S = Q K_j^T and dP = dO V_j^T (M 128, N 128, K 64; operands K-major in
-//   shared memory) into TMEM; the elementwise warps read both rows, release
-//   them (so the next block's products start), form dS in bf16 and put it back
-//   into TMEM; dQ += dS K_j (M 128, N 64, K 128; A = dS from TMEM, B = K_j
-//   MN-major).  The same kernel first forms D (one dot product per row) and
-//   stores it for the second kernel.
+//   S = Q K_j^T (issuer A) and dP = dO V_j^T (issuer B) (M 128, N 128, K 64;
+//   operands K-major in shared memory) into TMEM; the elementwise warps read
+//   both rows, release them (so the next block's products start), form dS in
+//   bf16 and put it back into TMEM; dQ_a += dS[:, 0:64] K_j[0:64] (A) and
+//   dQ_b += dS[:, 64:128] K_j[64:128] (B) (M 128, N 64, K 64; A = dS from
+//   TMEM, B = K_j MN-major), dQ = dQ_a + dQ_b at the end, so each key half
+//   of the elementwise warps runs its own pipeline.  The same kernel first
+//   forms D (one dot product per row) and stores it for the second kernel.
 // dK/dV kernel (grid Hkv x B x key blocks, first key blocks first), per (query
 //   head of the group, query block >= this key block):
-//   S^T = K Q^T and dP^T = V dO^T into TMEM; P^T and dS^T back into TMEM as
-//   bf16; dV += P^T dO and dK += dS^T Q (A from TMEM, B = dO / Q MN-major).
+//   S^T = K Q^T (A) and dP^T = V dO^T (B) into TMEM; P^T and dS^T back into
+//   TMEM as bf16; dV += P^T dO (A) and dK += dS^T Q (B) (A operands from
+//   TMEM, B = dO / Q MN-major).
 //   The per-query L and D of each step travel with its Q/dO tiles.
 // dQ and dK leave through the backward of the rotate-half RoPE (when tables
 // are given), then scale, bf16.  No atomics: every output element is written
@@ -41,12 +47,13 @@ constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 2;
 constexpr int EW_WARPS = 8;  // elementwise warps
-constexpr int NTHREADS = 64 + 32 * EW_WARPS;
+constexpr int MMA_B_WARP = 2 + EW_WARPS;  // second MMA-issuing warp
+constexpr int NTHREADS = 32 * (MMA_B_WARP + 1);
 constexpr int TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 
 // dQ kernel: TMEM columns; shared memory Q | dO | K[2] | V[2] | barriers | red
-constexpr int DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DS = 256, DQ_COL_DQ = 320;
+constexpr int DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DS = 256, DQ_COL_DQA = 320, DQ_COL_DQB = 384;
 constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + 256 + 2 * 128 * 4;
 // dK/dV kernel: TMEM columns; shared memory K | V | Q[2] | dO[2] | L[2] | D[2] | barriers
 constexpr int KV_COL_S = 0, KV_COL_DP = 128, KV_COL_P = 256, KV_COL_DS = 320, KV_COL_DV = 384,
@@ -55,16 +62,6 @@ constexpr int KV_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + 2
 
 // Named barrier of the elementwise warps (id 1).
 LLM_DEV void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EW_WARPS) : "memory"); }
-
-// Lane 0 waits on the phase; the result is shared by the warp, and
-// __syncwarp orders the other lanes' later accesses after lane 0's acquire.
-LLM_DEV bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_sh, int *gflag) {
-  int got = 0;
-  if ((threadIdx.x & 31) == 0) got = mbar_wait(bar, parity, abort_sh, gflag) ? 1 : 0;
-  got = __shfl_sync(0xffffffffu, got, 0);
-  __syncwarp();
-  return got != 0;
-}
 
 // Backward of the rotate-half RoPE on 16 column pairs (c, c + 32) of one row:
 // (x, y) <- (x cos + y sin, y cos - x sin), angle table entries ct[i], st[i].
@@ -129,7 +126,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t b0 = smem_u32(bars);
   const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
                  v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
-                 ds_full = b0 + 8 * 11, dq_done = b0 + 8 * 12, drain = b0 + 8 * 13;
+                 ds_full = b0 + 8 * 11,  // [2]: key half a, b
+                 dq_done = b0 + 8 * 13,  // [2]
+                 drain = b0 + 8 * 15;    // [2]: one per MMA warp
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -144,15 +143,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < STAGES; s++) {
       mbar_init(k_full + 8 * s, 1);
-      mbar_init(k_empty + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 2);  // dQ_a and dQ_b read K_j
       mbar_init(v_full + 8 * s, 1);
       mbar_init(v_empty + 8 * s, 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(s_full, 2);  // S and dP
     mbar_init(s_free, EW_WARPS);
-    mbar_init(ds_full, EW_WARPS);
-    mbar_init(dq_done, 1);
-    mbar_init(drain, 1);
+    for (int x = 0; x < 2; x++) {
+      mbar_init(ds_full + 8 * x, EW_WARPS / 2);
+      mbar_init(dq_done + 8 * x, 1);
+      mbar_init(drain + 8 * x, 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_512(tmem_sh);
@@ -188,64 +189,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         drain_wait(v_full + 8 * (j % STAGES), (j / STAGES) & 1);
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // --------------------------------------------------------- MMA issuer
-      constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
-      constexpr uint32_t ID_DQ = idesc_mn(128, HD, false, true);
-      const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024), dod = sdesc(smem_u32(sdO), 16, 1024);
-      auto issue_sdp = [&](int j) {  // S = Q K_j^T, dP = dO V_j^T
-        const int s = j % STAGES;
-        const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
-        const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 16, 1024);
+  } else if (warp == 1 || warp == MMA_B_WARP) {
+    // ------------------------------------- MMA issuers (whole warps)
+    // A: S = Q K_j^T, dQ_a += dS_a K_j[0:64];  B: dP = dO V_j^T, dQ_b += dS_b K_j[64:128]
+    const int x = warp == 1 ? 0 : 1;
+    constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
+    constexpr uint32_t ID_DQ = idesc_mn(128, HD, false, true);
+    const uint64_t ad = sdesc(smem_u32(x ? sdO : sQ), 16, 1024);
+    uint8_t *sB = x ? sV : sK;
+    const uint32_t b_full = x ? v_full : k_full;
+    const uint32_t col = x ? DQ_COL_DP : DQ_COL_S;
+    auto issue_prod = [&](int j) {
+      const int s = j % STAGES;
+      const uint64_t bd = sdesc(smem_u32(sB + s * TILE_BYTES), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; kk++)
-          mma_bf16(tmem + DQ_COL_S, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), ID_S,
+      for (int kk = 0; kk < HD / 16; kk++)
+        mma_bf16_e(tmem + col, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), ID_S,
                    kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; kk++)
-          mma_bf16(tmem + DQ_COL_DP, dod + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 2), ID_S,
-                   kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        mma_commit(v_empty + 8 * s);  // V_j is not read again
-      };
-      bool ok = mbar_wait(q_full, 0, abort_sh, gflag) && mbar_wait(k_full, 0, abort_sh, gflag) &&
-                mbar_wait(v_full, 0, abort_sh, gflag);
-      if (ok) {
-        fence_after();
-        issue_sdp(0);
-      }
-      for (int j = 0; j < nj && ok; j++) {
-        const int s = j % STAGES;
-        if (j + 1 < nj) {
-          // next block's products once the elementwise warps have read S, dP
-          const int s1 = (j + 1) % STAGES;
-          const uint32_t ph1 = ((j + 1) / STAGES) & 1;
-          if (!mbar_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
-              !mbar_wait(v_full + 8 * s1, ph1, abort_sh, gflag) ||
-              !mbar_wait(s_free, j & 1, abort_sh, gflag)) {
-            ok = false;
-            break;
-          }
-          fence_after();
-          issue_sdp(j + 1);
-        }
-        if (!mbar_wait(ds_full, j & 1, abort_sh, gflag)) {
+      mma_commit_e(s_full);
+      if (x) mma_commit_e(v_empty + 8 * s);  // V_j is not read again
+    };
+    bool ok = warp_wait(q_full, 0, abort_sh, gflag) && warp_wait(b_full, 0, abort_sh, gflag);
+    if (ok) {
+      fence_after();
+      issue_prod(0);
+    }
+    for (int j = 0; j < nj && ok; j++) {
+      const int s = j % STAGES;
+      const uint32_t ph = (j / STAGES) & 1;
+      if (j + 1 < nj) {
+        // next block's products once the elementwise warps have read S, dP
+        const int s1 = (j + 1) % STAGES;
+        const uint32_t ph1 = ((j + 1) / STAGES) & 1;
+        if (!warp_wait(b_full + 8 * s1, ph1, abort_sh, gflag) ||
+            !warp_wait(s_free, j & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-        const uint64_t kmd = sdesc(smem_u32(sK + s * TILE_BYTES), 8192, 1024);
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; kk++)
-          mma_ts(tmem + DQ_COL_DQ, tmem + DQ_COL_DS + kk * 8, kmd + (uint64_t)(kk * 128), ID_DQ,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(k_empty + 8 * s);
-        mma_commit(dq_done);
+        issue_prod(j + 1);
       }
-      mma_commit(drain);
-      drain_wait(drain, 0);
+      if (!warp_wait(ds_full + 8 * x, j & 1, abort_sh, gflag) ||
+          (x && !warp_wait(k_full + 8 * s, ph, abort_sh, gflag))) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      const uint64_t kmd = sdesc(smem_u32(sK + s * TILE_BYTES), 8192, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++)
+        mma_ts_e(tmem + (x ? DQ_COL_DQB : DQ_COL_DQA), tmem + DQ_COL_DS + x * 32 + kk * 8,
+                 kmd + (uint64_t)((x * 4 + kk) * 128), ID_DQ, (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_e(k_empty + 8 * s);
+      mma_commit_e(dq_done + 8 * x);
     }
+    mma_commit_e(drain + 8 * x);
+    if (lane == 0) drain_wait(drain + 8 * x, 0);
+    __syncwarp();
   } else {
     // --------------------------------------------------------- elementwise
     const int quarter = warp & 3;
@@ -304,9 +304,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
       }
-      // dS of the previous block is free once its dQ product has completed
+      // this half's dS of the previous block is free once its dQ product completed
       if (j > 0) {
-        if (!warp_wait(dq_done, (j - 1) & 1, abort_sh, gflag)) {
+        if (!warp_wait(dq_done + 8 * ch, (j - 1) & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
@@ -320,15 +320,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) mbar_arrive(ds_full + 8 * ch);
     }
-    if (ok) ok = warp_wait(dq_done, (nj - 1) & 1, abort_sh, gflag);
+    if (ok)
+      ok = warp_wait(dq_done, (nj - 1) & 1, abort_sh, gflag) &&
+           warp_wait(dq_done + 8, (nj - 1) & 1, abort_sh, gflag);
     if (ok) {
       fence_after();
       // column pairs (c, c + 32) of RoPE: this half takes c in [16 ch, 16 ch + 16)
-      float x[16], y[16];
-      tmem_ld16(tmem + lane_off + DQ_COL_DQ + ch * 16, x);
-      tmem_ld16(tmem + lane_off + DQ_COL_DQ + 32 + ch * 16, y);
+      float x[16], y[16], x2[16], y2[16];
+      tmem_ld16(tmem + lane_off + DQ_COL_DQA + ch * 16, x);
+      tmem_ld16(tmem + lane_off + DQ_COL_DQA + 32 + ch * 16, y);
+      tmem_ld16(tmem + lane_off + DQ_COL_DQB + ch * 16, x2);
+      tmem_ld16(tmem + lane_off + DQ_COL_DQB + 32 + ch * 16, y2);
+#pragma unroll
+      for (int i = 0; i < 16; i++) {
+        x[i] += x2[i];
+        y[i] += y2[i];
+      }
       if (valid) {
         if (cos_t)
           rope_bwd16(x, y, cos_t + (int64_t)qi * (HD / 2) + ch * 16,
@@ -364,7 +373,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t b0 = smem_u32(bars);
   const uint32_t kv_full = b0, q_full = b0 + 8, q_empty = b0 + 8 * 3, ld_full = b0 + 8 * 5,
                  s_full = b0 + 8 * 7, s_free = b0 + 8 * 8, p_full = b0 + 8 * 9,
-                 pv_done = b0 + 8 * 10, drain = b0 + 8 * 11;
+                 pv_done = b0 + 8 * 10, drain = b0 + 8 * 11;  // drain [2]: one per MMA warp
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nkb = gridDim.z, kb = blockIdx.z;
   const int g = blockIdx.x, b = blockIdx.y;
@@ -380,14 +389,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < STAGES; s++) {
       mbar_init(q_full + 8 * s, 1);
-      mbar_init(q_empty + 8 * s, 1);
+      mbar_init(q_empty + 8 * s, 2);  // both MMA warps read Q_s and dO_s
       mbar_init(ld_full + 8 * s, 32);
     }
-    mbar_init(s_full, 1);
+    mbar_init(s_full, 2);   // S^T and dP^T
     mbar_init(s_free, EW_WARPS);
     mbar_init(p_full, EW_WARPS);
-    mbar_init(pv_done, 1);
+    mbar_init(pv_done, 2);  // dV and dK
     mbar_init(drain, 1);
+    mbar_init(drain + 8, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_512(tmem_sh);
@@ -433,65 +443,60 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int st = max(0, issued - STAGES); st < issued; st++)
         drain_wait(q_full + 8 * (st % STAGES), (st / STAGES) & 1);
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // --------------------------------------------------------- MMA issuer
-      constexpr uint32_t ID_S = idesc_mn(128, BQ, false, false);
-      constexpr uint32_t ID_KV = idesc_mn(128, HD, false, true);
-      const uint64_t kd = sdesc(smem_u32(sK), 16, 1024), vd = sdesc(smem_u32(sV), 16, 1024);
-      auto issue_s = [&](int st) {  // S^T = K Q^T, dP^T = V dO^T
-        const int s = st % STAGES;
-        const uint64_t qd = sdesc(smem_u32(sQ + s * TILE_BYTES), 16, 1024);
-        const uint64_t dod = sdesc(smem_u32(sdO + s * TILE_BYTES), 16, 1024);
+  } else if (warp == 1 || warp == MMA_B_WARP) {
+    // ------------------------------------- MMA issuers (whole warps)
+    // A: S^T = K Q^T, dV += P^T dO;  B: dP^T = V dO^T, dK += dS^T Q
+    const int x = warp == 1 ? 0 : 1;
+    constexpr uint32_t ID_S = idesc_mn(128, BQ, false, false);
+    constexpr uint32_t ID_KV = idesc_mn(128, HD, false, true);
+    const uint64_t ad = sdesc(smem_u32(x ? sV : sK), 16, 1024);
+    uint8_t *sB = x ? sdO : sQ;    // B of the scores product (K-major)
+    uint8_t *sB2 = x ? sQ : sdO;   // B of the accumulation (MN-major)
+    const uint32_t col = x ? KV_COL_DP : KV_COL_S;
+    const uint32_t col_a2 = x ? KV_COL_DS : KV_COL_P, col_acc = x ? KV_COL_DK : KV_COL_DV;
+    auto issue_prod = [&](int st) {
+      const int s = st % STAGES;
+      const uint64_t bd = sdesc(smem_u32(sB + s * TILE_BYTES), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; kk++)
-          mma_bf16(tmem + KV_COL_S, kd + (uint64_t)(kk * 2), qd + (uint64_t)(kk * 2), ID_S,
+      for (int kk = 0; kk < HD / 16; kk++)
+        mma_bf16_e(tmem + col, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), ID_S,
                    kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; kk++)
-          mma_bf16(tmem + KV_COL_DP, vd + (uint64_t)(kk * 2), dod + (uint64_t)(kk * 2), ID_S,
-                   kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-      };
-      bool ok = mbar_wait(kv_full, 0, abort_sh, gflag) && mbar_wait(q_full, 0, abort_sh, gflag);
-      if (ok) {
-        fence_after();
-        issue_s(0);
-      }
-      for (int st = 0; st < nsteps && ok; st++) {
-        const int s = st % STAGES;
-        if (st + 1 < nsteps) {
-          const int s1 = (st + 1) % STAGES;
-          const uint32_t ph1 = ((st + 1) / STAGES) & 1;
-          if (!mbar_wait(q_full + 8 * s1, ph1, abort_sh, gflag) ||
-              !mbar_wait(s_free, st & 1, abort_sh, gflag)) {
-            ok = false;
-            break;
-          }
-          fence_after();
-          issue_s(st + 1);
-        }
-        if (!mbar_wait(p_full, st & 1, abort_sh, gflag)) {
+      mma_commit_e(s_full);
+    };
+    bool ok = warp_wait(kv_full, 0, abort_sh, gflag) && warp_wait(q_full, 0, abort_sh, gflag);
+    if (ok) {
+      fence_after();
+      issue_prod(0);
+    }
+    for (int st = 0; st < nsteps && ok; st++) {
+      const int s = st % STAGES;
+      if (st + 1 < nsteps) {
+        const int s1 = (st + 1) % STAGES;
+        const uint32_t ph1 = ((st + 1) / STAGES) & 1;
+        if (!warp_wait(q_full + 8 * s1, ph1, abort_sh, gflag) ||
+            !warp_wait(s_free, st & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-        const uint64_t qm = sdesc(smem_u32(sQ + s * TILE_BYTES), 8192, 1024);
-        const uint64_t dom = sdesc(smem_u32(sdO + s * TILE_BYTES), 8192, 1024);
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; kk++)
-          mma_ts(tmem + KV_COL_DV, tmem + KV_COL_P + kk * 8, dom + (uint64_t)(kk * 128), ID_KV,
-                 (st > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; kk++)
-          mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DS + kk * 8, qm + (uint64_t)(kk * 128), ID_KV,
-                 (st > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(q_empty + 8 * s);
-        mma_commit(pv_done);
+        issue_prod(st + 1);
       }
-      mma_commit(drain);
-      drain_wait(drain, 0);
+      if (!warp_wait(p_full, st & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      const uint64_t bm = sdesc(smem_u32(sB2 + s * TILE_BYTES), 8192, 1024);
+#pragma unroll
+      for (int kk = 0; kk < BQ / 16; kk++)
+        mma_ts_e(tmem + col_acc, tmem + col_a2 + kk * 8, bm + (uint64_t)(kk * 128), ID_KV,
+                 (st > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_e(q_empty + 8 * s);
+      mma_commit_e(pv_done);
     }
+    mma_commit_e(drain + 8 * x);
+    if (lane == 0) drain_wait(drain + 8 * x, 0);
+    __syncwarp();
   } else {
     // --------------------------------------------------------- elementwise
     const int quarter = warp & 3;

@@ -270,93 +270,97 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------ TMA producer
-      int s = 0;
-      uint32_t ph = 0;
-      uint32_t issued_parity[STAGES];
-      bool issued[STAGES];
-      for (int i = 0; i < STAGES; i++) issued[i] = false;
-      bool ok = true;
-      for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
-        int split = w / tiles_mn, tile = w % tiles_mn;
-        int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
-        int kb0, nkb = kblocks_of(split, kb0);
-        for (int kb = 0; kb < nkb; kb++) {
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) { ok = false; break; }
-          uint32_t fb = full0 + 8 * s;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
-          int k0 = (kb0 + kb) * BK;
-          if (A_MN) {
-            tma_load_2d(sa, &tmA, m0, k0, fb);
-            tma_load_2d(sa + 8192, &tmA, m0 + 64, k0, fb);
-          } else {
-            tma_load_2d(sa, &tmA, k0, m0, fb);
-          }
-          if (B_MN) {
-#pragma unroll
-            for (int j = 0; j < 4; j++) tma_load_2d(sb + 8192 * j, &tmB, n0 + 64 * j, k0, fb);
-          } else {
-            tma_load_2d(sb, &tmB, k0, n0, fb);
-          }
-          issued[s] = true;
-          issued_parity[s] = ph;
-          if (++s == STAGES) { s = 0; ph ^= 1; }
+    // -------------------------------------------------- TMA producer
+    // whole warp (warp-uniform control flow); one elected lane issues
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t issued_parity[STAGES];
+    bool issued[STAGES];
+    for (int i = 0; i < STAGES; i++) issued[i] = false;
+    bool ok = true;
+    for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
+      int split = w / tiles_mn, tile = w % tiles_mn;
+      int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
+      int kb0, nkb = kblocks_of(split, kb0);
+      for (int kb = 0; kb < nkb; kb++) {
+        if (!warp_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) { ok = false; break; }
+        uint32_t fb = full0 + 8 * s;
+        mbar_arrive_expect_tx_e(fb, STAGE_BYTES);
+        uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
+        int k0 = (kb0 + kb) * BK;
+        if (A_MN) {
+          tma_load_2d_e(sa, &tmA, m0, k0, fb);
+          tma_load_2d_e(sa + 8192, &tmA, m0 + 64, k0, fb);
+        } else {
+          tma_load_2d_e(sa, &tmA, k0, m0, fb);
         }
+        if (B_MN) {
+#pragma unroll
+          for (int j = 0; j < 4; j++) tma_load_2d_e(sb + 8192 * j, &tmB, n0 + 64 * j, k0, fb);
+        } else {
+          tma_load_2d_e(sb, &tmB, k0, n0, fb);
+        }
+        issued[s] = true;
+        issued_parity[s] = ph;
+        if (++s == STAGES) { s = 0; ph ^= 1; }
       }
-      // Our copies must have landed before the CTA exits (normally they were
-      // consumed already; after an abort they may still be in flight).
+    }
+    // Our copies must have landed before the CTA exits (normally they were
+    // consumed already; after an abort they may still be in flight).
+    if (lane == 0)
       for (int i = 0; i < STAGES; i++)
         if (issued[i]) {
           unsigned long long t0 = gtimer();
           while (!mbar_try(full0 + 8 * i, issued_parity[i]) && gtimer() - t0 < WAIT_NS) {
           }
         }
-    }
+    __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      constexpr uint32_t ID = idesc_mn(BM, BN, A_MN, B_MN);
-      int s = 0;
-      uint32_t ph = 0;
-      int acc = 0;
-      uint32_t aph = 0;
-      bool ok = true;
-      for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
-        int split = w / tiles_mn;
-        int kb0, nkb = kblocks_of(split, kb0);
-        if (nkb == 0) continue;  // epilogue writes zeros without waiting
-        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1, &abort_sh, a.flag)) break;
+    // -------------------------------------------------- MMA issuer
+    // The whole warp runs the loop (warp-uniform control flow); one elected
+    // lane issues each MMA and commit.
+    constexpr uint32_t ID = idesc_mn(BM, BN, A_MN, B_MN);
+    int s = 0;
+    uint32_t ph = 0;
+    int acc = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
+      int split = w / tiles_mn;
+      int kb0, nkb = kblocks_of(split, kb0);
+      if (nkb == 0) continue;  // epilogue writes zeros without waiting
+      if (!warp_wait(tempty0 + 8 * acc, aph ^ 1, &abort_sh, a.flag)) break;
+      fence_after();
+      uint32_t td = tmem + acc * BN;
+      for (int kb = 0; kb < nkb; kb++) {
+        if (!warp_wait(full0 + 8 * s, ph, &abort_sh, a.flag)) { ok = false; break; }
         fence_after();
-        uint32_t td = tmem + acc * BN;
-        for (int kb = 0; kb < nkb; kb++) {
-          if (!mbar_wait(full0 + 8 * s, ph, &abort_sh, a.flag)) { ok = false; break; }
-          fence_after();
-          uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
-          uint64_t ad = A_MN ? sdesc(sa, 8192, 1024) : sdesc(sa, 16, 1024);
-          uint64_t bd = B_MN ? sdesc(sb, 8192, 1024) : sdesc(sb, 16, 1024);
+        uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
+        uint64_t ad = A_MN ? sdesc(sa, 8192, 1024) : sdesc(sa, 16, 1024);
+        uint64_t bd = B_MN ? sdesc(sb, 8192, 1024) : sdesc(sb, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; kk++) {
-            // advance 16 K elements: 32 bytes inside a K-major swizzle row, or
-            // 16 rows (2048 bytes) of an MN-major tile; >>4 for the descriptor
-            uint64_t da = (uint64_t)(A_MN ? kk * 128 : kk * 2);
-            uint64_t db = (uint64_t)(B_MN ? kk * 128 : kk * 2);
-            mma_bf16(td, ad + da, bd + db, ID, (kb > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(empty0 + 8 * s);  // frees the stage when these MMAs finish
-          if (++s == STAGES) { s = 0; ph ^= 1; }
+        for (int kk = 0; kk < BK / 16; kk++) {
+          // advance 16 K elements: 32 bytes inside a K-major swizzle row, or
+          // 16 rows (2048 bytes) of an MN-major tile; >>4 for the descriptor
+          uint64_t da = (uint64_t)(A_MN ? kk * 128 : kk * 2);
+          uint64_t db = (uint64_t)(B_MN ? kk * 128 : kk * 2);
+          mma_bf16_e(td, ad + da, bd + db, ID, (kb > 0 || kk > 0) ? 1u : 0u);
         }
-        if (!ok) break;
-        mma_commit(tfull0 + 8 * acc);  // accumulator ready for the epilogue
-        if (++acc == 2) { acc = 0; aph ^= 1; }
+        mma_commit_e(empty0 + 8 * s);  // frees the stage when these MMAs finish
+        if (++s == STAGES) { s = 0; ph ^= 1; }
       }
-      // drain: every MMA this thread issued has completed
-      mma_commit(drain);
+      if (!ok) break;
+      mma_commit_e(tfull0 + 8 * acc);  // accumulator ready for the epilogue
+      if (++acc == 2) { acc = 0; aph ^= 1; }
+    }
+    // drain: every MMA this warp issued has completed
+    mma_commit_e(drain);
+    if (lane == 0) {
       unsigned long long t0 = gtimer();
       while (!mbar_try(drain, 0) && gtimer() - t0 < WAIT_NS) {
       }
     }
+    __syncwarp();
   } else {
     // -------------------------------------------------- epilogue warps
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
