@@ -20,6 +20,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 #include <unordered_map>
 
@@ -37,7 +38,7 @@ constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int EPI_WARPS = 8;
 constexpr int STAGING_BYTES = EPI_WARPS * 32 * 32 * 4;  // one 32x32 float square per epilogue warp
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + STAGING_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + STAGING_BYTES + 256 /*barriers*/;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 64 + 32 * EPI_WARPS;
 
@@ -45,6 +46,7 @@ struct Args {
   int M, N, K;
   int tiles_m, tiles_n, splits, kchunk, total;
   int out, epi;
+  int tma_store;  // 1: the tile leaves through bulk tensor stores of the staging square
   void *C;
   int64_t ldc;
   const float *R;
@@ -130,19 +132,134 @@ LLM_DEV void put32_bf16(float *stg, const float (&v)[32], __nv_bfloat16 *dst, in
   __syncwarp();
 }
 
+// Bulk tensor stores.  The staging square is laid out as the 128-byte-swizzle
+// image of a 32-row x 128-byte box (16-byte group g of row r at g ^ (r & 7)),
+// i.e. exactly what the tensor map of C expects; the copy engine clips rows
+// and columns outside C.  One store group per warp is in flight at a time:
+// stg_acquire waits until the previous store has read the square.
+LLM_DEV void stg_acquire() {
+  if ((threadIdx.x & 31) == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  __syncwarp();
+}
+LLM_DEV void bulk_store(const float *stg, const CUtensorMap *tm, int x, int y, int z, bool three_d) {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    if (three_d)
+      asm volatile(
+          "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+              (uint64_t)tm),
+          "r"(x), "r"(y), "r"(z), "r"(smem_u32(stg))
+          : "memory");
+    else
+      asm volatile(
+          "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+              (uint64_t)tm),
+          "r"(x), "r"(y), "r"(smem_u32(stg))
+          : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  }
+}
+// 64 bf16 columns of the warp's 32 rows (lo = columns 0..31, hi = 32..63):
+// 8 groups of 8 values per row, swizzled like the float square.
+LLM_DEV void stage64_bf16(float *stg, const float (&lo)[32], const float (&hi)[32]) {
+  const int lane = threadIdx.x & 31;
+  uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 32);
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    row[j ^ (lane & 7)] = make_uint4(pack_bf16(lo[8 * j], lo[8 * j + 1]), pack_bf16(lo[8 * j + 2], lo[8 * j + 3]),
+                                     pack_bf16(lo[8 * j + 4], lo[8 * j + 5]), pack_bf16(lo[8 * j + 6], lo[8 * j + 7]));
+    row[(4 + j) ^ (lane & 7)] = make_uint4(pack_bf16(hi[8 * j], hi[8 * j + 1]), pack_bf16(hi[8 * j + 2], hi[8 * j + 3]),
+                                           pack_bf16(hi[8 * j + 4], hi[8 * j + 5]), pack_bf16(hi[8 * j + 6], hi[8 * j + 7]));
+  }
+}
+LLM_DEV void rope32(float (&v)[32], const float *cos_row, const float *sin_row) {
+  // both halves of a 32-wide head in one chunk: (v[j], v[j+16]) rotate by angle j
+  const float4 *ct = reinterpret_cast<const float4 *>(cos_row);
+  const float4 *st = reinterpret_cast<const float4 *>(sin_row);
+#pragma unroll
+  for (int j4 = 0; j4 < 4; j4++) {
+    float4 c4 = ct[j4], s4 = st[j4];
+    const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      int j = 4 * j4 + k;
+      float x = v[j], y = v[j + 16];
+      v[j] = x * cc[k] - y * ss[k];
+      v[j + 16] = y * cc[k] + x * ss[k];
+    }
+  }
+}
+
 // One output tile's epilogue for a warp: rows [row0, row0+32) of the tile
 // (TMEM lanes of this warp's quarter, lane i = row row0 + i) and the warp's
 // half of the columns, [n0 + c_lo, n0 + c_lo + BN/2).  Every lane executes
 // every tcgen05.ld (warp-uniform control); rows past M and columns past N are
 // clipped only at the stores.
-LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int c_lo, int split,
-                           bool zero, float *stg) {
+LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, int row0, int n0,
+                           int c_lo, int split, bool zero, float *stg) {
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
   const int rows = max(0, min(32, a.M - row0));
   const int N = a.N;
   auto ncols = [&](int n) { return max(0, min(32, N - n)); };
   float v[32];
+  if (a.tma_store) {
+    if (rows == 0) return;  // the warp's 32 rows lie past M: nothing to store
+    if (a.out == OUT_ACT) {
+      // bf16, 64 columns per store: plain, or RoPE on q/k head columns
+      const int t = m % a.T, half = a.hd / 2;
+      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 64) {
+        const int n = n0 + c0;
+        if (n >= N) break;
+        float lo[32], hi[32];
+        if (zero) {
+          for (int i = 0; i < 32; i++) lo[i] = hi[i] = 0.f;
+        } else {
+          tmem_ld32(tm + c0, lo);
+          tmem_ld32(tm + c0 + 32, hi);
+        }
+        if (a.epi == TC_EPI_ROPE && n < a.rot_cols) {
+          const float *cr = a.cos_t + (int64_t)t * half, *sr = a.sin_t + (int64_t)t * half;
+          if (a.hd == 64) {
+            const float4 *ct = reinterpret_cast<const float4 *>(cr);
+            const float4 *st = reinterpret_cast<const float4 *>(sr);
+#pragma unroll
+            for (int j4 = 0; j4 < 8; j4++) {
+              float4 c4 = ct[j4], s4 = st[j4];
+              const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+              for (int k = 0; k < 4; k++) {
+                int j = 4 * j4 + k;
+                float x = lo[j], y = hi[j];
+                lo[j] = x * cc[k] - y * ss[k];
+                hi[j] = y * cc[k] + x * ss[k];
+              }
+            }
+          } else {  // hd == 32: each 32-column chunk is one head
+            rope32(lo, cr, sr);
+            if (n + 32 < a.rot_cols) rope32(hi, cr, sr);
+          }
+        }
+        stg_acquire();
+        stage64_bf16(stg, lo, hi);
+        bulk_store(stg, tmC, n, row0, 0, false);
+      }
+    } else {
+      // fp32 (plain, or split-K partial into slab `split`), 32 columns per store
+      const bool part = a.out == OUT_PARTIAL;
+      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
+        const int n = n0 + c0;
+        if (n >= N) break;
+        if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
+        else tmem_ld32(tm + c0, v);
+        stg_acquire();
+        stage32(stg, v);
+        bulk_store(stg, tmC, n, row0, split, part);
+      }
+    }
+    return;
+  }
   if (a.epi == TC_EPI_ROPE) {
     // RoPE on q/k heads (columns < rot_cols), plain store of v heads.
     const int hd = a.hd, half = hd / 2, t = m % a.T;
@@ -224,10 +341,10 @@ LLM_DEV void epilogue_tile(const Args &a, uint32_t tm, int row0, int n0, int c_l
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const Args a) {
+              const __grid_constant__ CUtensorMap tmC, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t *bars = (uint64_t *)(smem + STAGES * STAGE_BYTES);
+  uint64_t *bars = (uint64_t *)(smem + STAGES * STAGE_BYTES + STAGING_BYTES);
   // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
@@ -366,7 +483,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int ew = warp - 2;       // epilogue warp 0..7
     const int c_lo = (ew / 4) * (BN / 2);
-    float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + ew * 32 * 32;
+    float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES) + ew * 32 * 32;
     int acc = 0;
     uint32_t aph = 0;
     for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
@@ -375,7 +492,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, 0, row0, n0, c_lo, split, true, stg);
+        epilogue_tile(a, &tmC, 0, row0, n0, c_lo, split, true, stg);
         continue;
       }
       int got = 0;
@@ -384,12 +501,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!got) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, tm, row0, n0, c_lo, split, false, stg);
+      epilogue_tile(a, &tmC, tm, row0, n0, c_lo, split, false, stg);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; aph ^= 1; }
     }
+    // this warp's bulk stores have completed before the CTA may exit
+    if (a.tma_store && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
   fence_before();
   __syncthreads();
@@ -414,16 +534,18 @@ struct TcPlan {
   std::mutex mu;
   struct Key {
     const void *p;
-    uint64_t d0, d1, s1;
-    uint32_t b0, b1;
+    uint64_t d0, d1, s1, d2;
+    uint32_t b0, b1, esz;
     bool operator==(const Key &o) const {
-      return p == o.p && d0 == o.d0 && d1 == o.d1 && s1 == o.s1 && b0 == o.b0 && b1 == o.b1;
+      return p == o.p && d0 == o.d0 && d1 == o.d1 && s1 == o.s1 && d2 == o.d2 && b0 == o.b0 &&
+             b1 == o.b1 && esz == o.esz;
     }
   };
   struct KeyHash {
     size_t operator()(const Key &k) const {
       return std::hash<const void *>()(k.p) ^ (k.d0 * 1315423911u) ^ (k.d1 * 2654435761u) ^
-             (k.s1 << 7) ^ ((uint64_t)k.b0 << 20) ^ ((uint64_t)k.b1 << 40);
+             (k.s1 << 7) ^ ((uint64_t)k.b0 << 20) ^ ((uint64_t)k.b1 << 40) ^ (k.d2 << 13) ^
+             ((uint64_t)k.esz << 52);
     }
   };
   std::unordered_map<Key, CUtensorMap, KeyHash> maps;
@@ -432,7 +554,7 @@ struct TcPlan {
   // stride s1 elements; box b0 x b1; 128-byte swizzle; zero fill outside.
   bool map(const void *p, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0, uint32_t b1,
            CUtensorMap *out) {
-    Key k{p, d0, d1, s1, b0, b1};
+    Key k{p, d0, d1, s1, 1, b0, b1, 2};
     std::lock_guard<std::mutex> g(mu);
     auto it = maps.find(k);
     if (it != maps.end()) { *out = it->second; return true; }
@@ -444,6 +566,31 @@ struct TcPlan {
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    maps.emplace(k, *out);
+    return true;
+  }
+  // Output map of C: bf16 (esz 2, box 64 x 32) or fp32 (esz 4, box 32 x 32)
+  // over [d1 rows][d0 cols] with row stride s1 elements.  three_d adds a
+  // third dimension of d2 slabs of d1 rows (split-K partial sums; always
+  // three-dimensional, also for d2 = 1, because the kernel's partial-sum
+  // store is), so the edge of one slab never spills into the next.
+  // 128-byte swizzle (one box row = 128 bytes).
+  bool map_out(const void *p, uint64_t d0, uint64_t d1, uint64_t s1, uint64_t d2, bool three_d,
+               uint32_t esz, CUtensorMap *out) {
+    const uint32_t b0 = esz == 2 ? 64 : 32;
+    Key k{p, d0, d1, s1, three_d ? d2 + 1 : 0, b0, 32, esz};
+    std::lock_guard<std::mutex> g(mu);
+    auto it = maps.find(k);
+    if (it != maps.end()) { *out = it->second; return true; }
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1 * esz, s1 * esz * d1};
+    cuuint32_t box[3] = {b0, 32, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = encode(out, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        three_d ? 3 : 2, const_cast<void *>(p), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     maps.emplace(k, *out);
     return true;
@@ -506,11 +653,20 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   ok = ok && (g.b_kmajor ? p->map(g.B, g.K, g.N, g.ldb, 64, BN, &tb)
                          : p->map(g.B, g.N, g.K, g.ldb, 64, 64, &tb));
   if (!ok) return false;
+  if (out != OUT_PARTIAL) splits = 1;
+  // C leaves through bulk tensor stores except for the residual add, which
+  // reads R on the way out
+  CUtensorMap tcm;
+  memset(&tcm, 0, sizeof(tcm));
+  const bool tma_store = out != OUT_ADD_F32;
+  if (tma_store && !p->map_out(C, g.N, g.M, ldc, max(1, splits), out == OUT_PARTIAL,
+                               out == OUT_ACT ? 2 : 4, &tcm))
+    return false;
   Args a{};
+  a.tma_store = tma_store ? 1 : 0;
   a.M = g.M; a.N = g.N; a.K = g.K;
   a.tiles_m = (g.M + BM - 1) / BM;
   a.tiles_n = (g.N + BN - 1) / BN;
-  if (out != OUT_PARTIAL) splits = 1;
   a.splits = max(1, splits);
   int kc = (g.K + a.splits - 1) / a.splits;
   a.kchunk = ((kc + BK - 1) / BK) * BK;
@@ -520,10 +676,10 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   a.flag = p->flag;
   int grid = min(a.total, p->num_sms);
   bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
-  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
-  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
-  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
-  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, a);
+  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
+  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
+  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
+  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
   count_launch();
   return true;
 }
