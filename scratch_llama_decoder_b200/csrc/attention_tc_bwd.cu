@@ -46,7 +46,10 @@ using namespace tc;
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 2;
-constexpr int EW_WARPS = 8;  // elementwise warps
+constexpr int EW_WARPS = 8;  // elementwise warps: 4 lane quarters x NCQ column groups
+constexpr int NCQ = EW_WARPS / 4;  // column groups of a row (2 or 4)
+constexpr int CW = 128 / NCQ;      // score columns per thread
+constexpr int HW = 32 / NCQ;       // head columns per thread in each RoPE half
 constexpr int MMA_B_WARP = 2 + EW_WARPS;  // second MMA-issuing warp
 constexpr int NTHREADS = 32 * (MMA_B_WARP + 1);
 constexpr int TMEM_COLS = 512;
@@ -54,7 +57,7 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 // dQ kernel: TMEM columns; shared memory Q | dO | K[2] | V[2] | barriers | red
 constexpr int DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DS = 256, DQ_COL_DQA = 320, DQ_COL_DQB = 384;
-constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + 256 + 2 * 128 * 4;
+constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + 256 + NCQ * 128 * 4;
 // dK/dV kernel: TMEM columns; shared memory K | V | Q[2] | dO[2] | L[2] | D[2] | barriers
 constexpr int KV_COL_S = 0, KV_COL_DP = 128, KV_COL_P = 256, KV_COL_DS = 320, KV_COL_DV = 384,
               KV_COL_DK = 448;
@@ -63,11 +66,12 @@ constexpr int KV_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + 2
 // Named barrier of the elementwise warps (id 1).
 LLM_DEV void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EW_WARPS) : "memory"); }
 
-// Backward of the rotate-half RoPE on 16 column pairs (c, c + 32) of one row:
+// Backward of the rotate-half RoPE on N column pairs (c, c + 32) of one row:
 // (x, y) <- (x cos + y sin, y cos - x sin), angle table entries ct[i], st[i].
-LLM_DEV void rope_bwd16(float (&x)[16], float (&y)[16], const float *ct, const float *st) {
+template <int N>
+LLM_DEV void rope_bwd_n(float (&x)[N], float (&y)[N], const float *ct, const float *st) {
 #pragma unroll
-  for (int i = 0; i < 16; i += 4) {
+  for (int i = 0; i < N; i += 4) {
     const float4 c = *reinterpret_cast<const float4 *>(ct + i);
     const float4 s = *reinterpret_cast<const float4 *>(st + i);
     const float cv[4] = {c.x, c.y, c.z, c.w}, sv[4] = {s.x, s.y, s.z, s.w};
@@ -80,14 +84,15 @@ LLM_DEV void rope_bwd16(float (&x)[16], float (&y)[16], const float *ct, const f
   }
 }
 
-// 16 consecutive bf16 values (v * mul) to a 32-byte aligned address.
-LLM_DEV void store16(__nv_bfloat16 *dst, const float (&v)[16], float mul) {
-  uint4 a = make_uint4(pack_bf16(v[0] * mul, v[1] * mul), pack_bf16(v[2] * mul, v[3] * mul),
-                       pack_bf16(v[4] * mul, v[5] * mul), pack_bf16(v[6] * mul, v[7] * mul));
-  uint4 b = make_uint4(pack_bf16(v[8] * mul, v[9] * mul), pack_bf16(v[10] * mul, v[11] * mul),
-                       pack_bf16(v[12] * mul, v[13] * mul), pack_bf16(v[14] * mul, v[15] * mul));
-  reinterpret_cast<uint4 *>(dst)[0] = a;
-  reinterpret_cast<uint4 *>(dst)[1] = b;
+// N consecutive bf16 values (v * mul, N a multiple of 8) to a 16-byte
+// aligned address.
+template <int N>
+LLM_DEV void store_n(__nv_bfloat16 *dst, const float (&v)[N], float mul) {
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    reinterpret_cast<uint4 *>(dst)[i / 8] =
+        make_uint4(pack_bf16(v[i] * mul, v[i + 1] * mul), pack_bf16(v[i + 2] * mul, v[i + 3] * mul),
+                   pack_bf16(v[i + 4] * mul, v[i + 5] * mul), pack_bf16(v[i + 6] * mul, v[i + 7] * mul));
 }
 
 LLM_DEV void tmem_alloc_512(uint32_t *dst) {
@@ -249,20 +254,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // --------------------------------------------------------- elementwise
     const int quarter = warp & 3;
-    const int ch = (warp - 2) >> 2;  // which half of the block's columns
+    const int cq = (warp - 2) >> 2;  // column group: keys [cq CW, cq CW + CW) of the block
+    const int x = cq / (NCQ / 2);    // key half (dQ_a or dQ_b) this group feeds
     const int r = quarter * 32 + lane;
     const int qi = q0 + r;
     const bool valid = qi < T;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = scale * LOG2E;
-    // D_i = dO_i . O_i, each half-row thread over 32 of the 64 columns
+    // D_i = dO_i . O_i, each thread over 64 / NCQ of the 64 head columns
     float dpart = 0.f;
     if (valid) {
-      const int64_t off = ((int64_t)row_base + qi) * d + h * HD + ch * 32;
+      const int64_t off = ((int64_t)row_base + qi) * d + h * HD + cq * (HD / NCQ);
       const uint4 *po = reinterpret_cast<const uint4 *>(o + off);
       const uint4 *pd = reinterpret_cast<const uint4 *>(dout + off);
 #pragma unroll
-      for (int e = 0; e < 4; e++) {
+      for (int e = 0; e < HD / NCQ / 8; e++) {
         const uint4 a = po[e], c = pd[e];
         const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
         const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&c);
@@ -273,12 +279,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-    red[ch * 128 + r] = dpart;
+    red[cq * 128 + r] = dpart;
     ew_sync();
-    const float Di = red[r] + red[128 + r];
+    float Di = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCQ; c++) Di += red[c * 128 + r];
     // rows past T get L = +inf, so every P of theirs is 0
     const float L2 = valid ? lse[((int64_t)b * H + h) * T + qi] * LOG2E : INFINITY;
-    if (ch == 0 && valid) Dv[((int64_t)b * H + h) * T + qi] = Di;
+    if (cq == 0 && valid) Dv[((int64_t)b * H + h) * T + qi] = Di;
     bool ok = true;
     for (int j = 0; j < nj && ok; j++) {
       if (!warp_wait(s_full, j & 1, abort_sh, gflag)) {
@@ -286,17 +294,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       fence_after();
-      float sv[64], dv[64];
-      tmem_ld64(tmem + lane_off + DQ_COL_S + ch * 64, sv);
-      tmem_ld64(tmem + lane_off + DQ_COL_DP + ch * 64, dv);
+      float sv[CW], dv[CW];
+      tmem_ldn<CW>(tmem + lane_off + DQ_COL_S + cq * CW, sv);
+      tmem_ldn<CW>(tmem + lane_off + DQ_COL_DP + cq * CW, dv);
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S and dP now
-      const int k0 = j * BK + ch * 64;
+      if (lane == 0) mbar_arrive(s_free);  // the MMA warps may overwrite S and dP now
+      const int k0 = j * BK + cq * CW;
       const bool diag = (j == qb);  // only the diagonal block masks (keys >= T lie above it)
-      uint32_t w[32];
+      uint32_t w[CW / 2];
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
+      for (int i = 0; i < CW; i += 2) {
         float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
         if (diag) {
           if (k0 + i > qi) p0 = 0.f;
@@ -306,45 +314,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // this half's dS of the previous block is free once its dQ product completed
       if (j > 0) {
-        if (!warp_wait(dq_done + 8 * ch, (j - 1) & 1, abort_sh, gflag)) {
+        if (!warp_wait(dq_done + 8 * x, (j - 1) & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
       }
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t (&wc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&w[c * 16]);
-        tmem_st16(tmem + lane_off + DQ_COL_DS + ch * 32 + c * 16, wc);
-      }
+      for (int c = 0; c < CW / 2; c += 16)
+        tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + DQ_COL_DS + cq * (CW / 2) + c, w + c);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full + 8 * ch);
+      if (lane == 0) mbar_arrive(ds_full + 8 * x);
     }
     if (ok)
       ok = warp_wait(dq_done, (nj - 1) & 1, abort_sh, gflag) &&
            warp_wait(dq_done + 8, (nj - 1) & 1, abort_sh, gflag);
     if (ok) {
       fence_after();
-      // column pairs (c, c + 32) of RoPE: this half takes c in [16 ch, 16 ch + 16)
-      float x[16], y[16], x2[16], y2[16];
-      tmem_ld16(tmem + lane_off + DQ_COL_DQA + ch * 16, x);
-      tmem_ld16(tmem + lane_off + DQ_COL_DQA + 32 + ch * 16, y);
-      tmem_ld16(tmem + lane_off + DQ_COL_DQB + ch * 16, x2);
-      tmem_ld16(tmem + lane_off + DQ_COL_DQB + 32 + ch * 16, y2);
+      // column pairs (c, c + 32) of RoPE: this group takes c in [cq HW, cq HW + HW)
+      float xa[HW], ya[HW], xb[HW], yb[HW];
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + cq * HW, xa);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + 32 + cq * HW, ya);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + cq * HW, xb);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + 32 + cq * HW, yb);
 #pragma unroll
-      for (int i = 0; i < 16; i++) {
-        x[i] += x2[i];
-        y[i] += y2[i];
+      for (int i = 0; i < HW; i++) {
+        xa[i] += xb[i];
+        ya[i] += yb[i];
       }
       if (valid) {
         if (cos_t)
-          rope_bwd16(x, y, cos_t + (int64_t)qi * (HD / 2) + ch * 16,
-                     sin_t + (int64_t)qi * (HD / 2) + ch * 16);
-        __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + qi) * ld + h * HD + ch * 16;
-        store16(dst, x, scale);
-        store16(dst + 32, y, scale);
+          rope_bwd_n<HW>(xa, ya, cos_t + (int64_t)qi * (HD / 2) + cq * HW,
+                         sin_t + (int64_t)qi * (HD / 2) + cq * HW);
+        __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + qi) * ld + h * HD + cq * HW;
+        store_n<HW>(dst, xa, scale);
+        store_n<HW>(dst + 32, ya, scale);
       }
     }
   }
@@ -500,7 +506,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // --------------------------------------------------------- elementwise
     const int quarter = warp & 3;
-    const int ch = (warp - 2) >> 2;  // which half of the block's query columns
+    const int cq = (warp - 2) >> 2;  // column group: queries [cq CW, cq CW + CW) of the block
     const int r = quarter * 32 + lane;
     const int kj = k0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -515,18 +521,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       fence_after();
-      float sv[64], dv[64];
-      tmem_ld64(tmem + lane_off + KV_COL_S + ch * 64, sv);
-      tmem_ld64(tmem + lane_off + KV_COL_DP + ch * 64, dv);
+      float sv[CW], dv[CW];
+      tmem_ldn<CW>(tmem + lane_off + KV_COL_S + cq * CW, sv);
+      tmem_ldn<CW>(tmem + lane_off + KV_COL_DP + cq * CW, dv);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
-      const int qc0 = qb * BQ + ch * 64;
+      const int qc0 = qb * BQ + cq * CW;
       const bool diag = (qb == kb);  // keys >= T occur only in this case, above the diagonal
-      const float *Ls = sL + s * 128 + ch * 64, *Ds = sD + s * 128 + ch * 64;
-      uint32_t wp[32], wd[32];
+      const float *Ls = sL + s * 128 + cq * CW, *Ds = sD + s * 128 + cq * CW;
+      uint32_t wp[CW / 2], wd[CW / 2];
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
+      for (int i = 0; i < CW; i += 2) {
         float p0 = ex2(fmaf(sv[i], sl2, -Ls[i])), p1 = ex2(fmaf(sv[i + 1], sl2, -Ls[i + 1]));
         if (diag) {
           if (kj > qc0 + i) p0 = 0.f;
@@ -544,11 +550,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_after();
       }
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t (&pc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&wp[c * 16]);
-        uint32_t (&dc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&wd[c * 16]);
-        tmem_st16(tmem + lane_off + KV_COL_P + ch * 32 + c * 16, pc);
-        tmem_st16(tmem + lane_off + KV_COL_DS + ch * 32 + c * 16, dc);
+      for (int c = 0; c < CW / 2; c += 16) {
+        tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + KV_COL_P + cq * (CW / 2) + c, wp + c);
+        tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + KV_COL_DS + cq * (CW / 2) + c, wd + c);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
@@ -558,22 +562,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok) ok = warp_wait(pv_done, (nsteps - 1) & 1, abort_sh, gflag);
     if (ok) {
       fence_after();
-      float x[16], y[16];
-      __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + kj) * ld + d + g * HD + ch * 16;
-      tmem_ld16(tmem + lane_off + KV_COL_DK + ch * 16, x);
-      tmem_ld16(tmem + lane_off + KV_COL_DK + 32 + ch * 16, y);
+      // column pairs (c, c + 32) of RoPE: this group takes c in [cq HW, cq HW + HW)
+      float xx[HW], yy[HW];
+      __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + kj) * ld + d + g * HD + cq * HW;
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + cq * HW, xx);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + 32 + cq * HW, yy);
       if (kj < T) {
         if (cos_t)
-          rope_bwd16(x, y, cos_t + (int64_t)kj * (HD / 2) + ch * 16,
-                     sin_t + (int64_t)kj * (HD / 2) + ch * 16);
-        store16(dst, x, scale);
-        store16(dst + 32, y, scale);
+          rope_bwd_n<HW>(xx, yy, cos_t + (int64_t)kj * (HD / 2) + cq * HW,
+                         sin_t + (int64_t)kj * (HD / 2) + cq * HW);
+        store_n<HW>(dst, xx, scale);
+        store_n<HW>(dst + 32, yy, scale);
       }
-      tmem_ld16(tmem + lane_off + KV_COL_DV + ch * 16, x);
-      tmem_ld16(tmem + lane_off + KV_COL_DV + 32 + ch * 16, y);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + cq * HW, xx);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + 32 + cq * HW, yy);
       if (kj < T) {
-        store16(dst + kvd, x, 1.f);
-        store16(dst + kvd + 32, y, 1.f);
+        store_n<HW>(dst + kvd, xx, 1.f);
+        store_n<HW>(dst + kvd + 32, yy, 1.f);
       }
     }
   }

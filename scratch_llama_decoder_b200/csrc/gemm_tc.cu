@@ -33,11 +33,12 @@ namespace llm {
 namespace tc {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int STG_BUFS = 1;  // staging squares per epilogue warp (bulk stores in flight)
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int EPI_WARPS = 8;
-constexpr int STAGING_BYTES = EPI_WARPS * 32 * 32 * 4;  // one 32x32 float square per epilogue warp
+constexpr int STAGING_BYTES = EPI_WARPS * STG_BUFS * 32 * 32 * 4;  // 32x32 float squares
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + STAGING_BYTES + 256 /*barriers*/;
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 64 + 32 * EPI_WARPS;
@@ -138,7 +139,8 @@ LLM_DEV void put32_bf16(float *stg, const float (&v)[32], __nv_bfloat16 *dst, in
 // and columns outside C.  One store group per warp is in flight at a time:
 // stg_acquire waits until the previous store has read the square.
 LLM_DEV void stg_acquire() {
-  if ((threadIdx.x & 31) == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  if ((threadIdx.x & 31) == 0)
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(STG_BUFS - 1) : "memory");
   __syncwarp();
 }
 LLM_DEV void bulk_store(const float *stg, const CUtensorMap *tm, int x, int y, int z, bool three_d) {
@@ -197,7 +199,8 @@ LLM_DEV void rope32(float (&v)[32], const float *cos_row, const float *sin_row) 
 // every tcgen05.ld (warp-uniform control); rows past M and columns past N are
 // clipped only at the stores.
 LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, int row0, int n0,
-                           int c_lo, int split, bool zero, float *stg) {
+                           int c_lo, int split, bool zero, float *stg_base, int &sb) {
+  float *stg = stg_base;
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
   const int rows = max(0, min(32, a.M - row0));
@@ -241,6 +244,8 @@ LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, i
             if (n + 32 < a.rot_cols) rope32(hi, cr, sr);
           }
         }
+        stg = stg_base + sb * 32 * 32;
+        sb = sb + 1 == STG_BUFS ? 0 : sb + 1;
         stg_acquire();
         stage64_bf16(stg, lo, hi);
         bulk_store(stg, tmC, n, row0, 0, false);
@@ -253,6 +258,8 @@ LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, i
         if (n >= N) break;
         if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
         else tmem_ld32(tm + c0, v);
+        stg = stg_base + sb * 32 * 32;
+        sb = sb + 1 == STG_BUFS ? 0 : sb + 1;
         stg_acquire();
         stage32(stg, v);
         bulk_store(stg, tmC, n, row0, split, part);
@@ -483,7 +490,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int ew = warp - 2;       // epilogue warp 0..7
     const int c_lo = (ew / 4) * (BN / 2);
-    float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES) + ew * 32 * 32;
+    float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES) + ew * STG_BUFS * 32 * 32;
+    int sb = 0;  // next staging square of this warp
     int acc = 0;
     uint32_t aph = 0;
     for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
@@ -492,7 +500,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, &tmC, 0, row0, n0, c_lo, split, true, stg);
+        epilogue_tile(a, &tmC, 0, row0, n0, c_lo, split, true, stg, sb);
         continue;
       }
       int got = 0;
@@ -501,7 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!got) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, &tmC, tm, row0, n0, c_lo, split, false, stg);
+      epilogue_tile(a, &tmC, tm, row0, n0, c_lo, split, false, stg, sb);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);

@@ -1,6 +1,8 @@
 // Memory-bound kernels of the training step: weight casts, embedding gather and
 // scatter-add, RMSNorm forward/backward, RoPE, SwiGLU, cross-entropy, loss
 // reduction, AdamW and initialisation.  Each cites the passage it computes.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,39 +31,74 @@ void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStrea
 }
 
 // ------------------------------------------------------------- weight casts
+// dst[r, c] (rows_p x cols_p, zero padding) from src [rows x cols]; mode 1
+// interleaves W1 | W3 in blocks of SWIGLU_BLOCK columns.  One block per row
+// (grid-stride), 4 columns per thread: the 4 source columns of an aligned
+// group are contiguous in both modes (SWIGLU_BLOCK and h are multiples of 4),
+// so they move as one 16-byte load when vec is set.
+// 4 consecutive values, one vector store when the address allows it
+LLM_DEV void put4(__nv_bfloat16 *d, const float (&v)[4]) {
+  if (((uintptr_t)d & 7) == 0) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2 *>(d) =
+        make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+  } else {
+    for (int k = 0; k < 4; k++) d[k] = __float2bfloat16_rn(v[k]);
+  }
+}
+LLM_DEV void put4(float *d, const float (&v)[4]) {
+  if (((uintptr_t)d & 15) == 0) *reinterpret_cast<float4 *>(d) = make_float4(v[0], v[1], v[2], v[3]);
+  else for (int k = 0; k < 4; k++) d[k] = v[k];
+}
+LLM_DEV int64_t cast_src_col(int64_t c, int mode, int64_t h) {
+  if (mode == 0) return c;
+  int64_t blk = c / (2 * SWIGLU_BLOCK), w = c % (2 * SWIGLU_BLOCK);
+  int64_t j = blk * SWIGLU_BLOCK + (w % SWIGLU_BLOCK);
+  return j < h ? (w < SWIGLU_BLOCK ? j : h + j) : -1;
+}
 template <typename A>
 __global__ void k_cast_weight(const float *__restrict__ src, A *__restrict__ dst, int64_t rows,
                               int64_t cols, int64_t rows_p, int64_t cols_p, int mode, int64_t h,
-                              int64_t hp, int64_t sbs, int64_t dbs) {
-  int64_t n = rows_p * cols_p;
+                              int64_t hp, int64_t sbs, int64_t dbs, bool vec) {
   src += blockIdx.y * sbs;
   dst += blockIdx.y * dbs;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    int64_t r = i / cols_p, c = i % cols_p;
-    float v = 0.f;
-    if (mode == 0) {
-      if (r < rows && c < cols) v = src[r * cols + c];
-    } else {
-      // interleaved W1|W3 blocks of SWIGLU_BLOCK columns
-      int64_t blk = c / (2 * SWIGLU_BLOCK), w = c % (2 * SWIGLU_BLOCK);
-      int64_t j = blk * SWIGLU_BLOCK + (w % SWIGLU_BLOCK);
-      if (j < h) v = src[r * cols + (w < SWIGLU_BLOCK ? j : h + j)];
+  const int64_t ncols = mode == 0 ? cols : 2 * h;  // valid source columns
+  for (int64_t r = blockIdx.x; r < rows_p; r += gridDim.x) {
+    const float *sr = src + r * cols;
+    A *dr = dst + r * cols_p;
+    for (int64_t c = 4 * (int64_t)threadIdx.x; c < cols_p; c += 4 * (int64_t)blockDim.x) {
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (r < rows) {
+        const int64_t sc = cast_src_col(c, mode, h);
+        if (vec && sc >= 0 && sc + 4 <= ncols && (mode == 0 ? c + 4 <= cols : true)) {
+          const float4 q = *reinterpret_cast<const float4 *>(sr + sc);
+          v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        } else {
+          for (int k = 0; k < 4; k++) {
+            const int64_t cc = c + k;
+            const int64_t sk = cast_src_col(cc, mode, h);
+            if (sk >= 0 && (mode != 0 || cc < cols)) v[k] = sr[sk];
+          }
+        }
+      }
+      if (c + 4 <= cols_p) put4(dr + c, v);
+      else for (int k = 0; c + k < cols_p; k++) dr[c + k] = from_f<A>(v[k]);
     }
-    dst[i] = from_f<A>(v);
   }
 }
 void cast_weight(const float *src, void *dst, DType dt, int64_t rows, int64_t cols,
                  int64_t rows_p, int64_t cols_p, int mode, int64_t h, int64_t hp, int batch,
                  int64_t sbs, int64_t dbs, cudaStream_t s) {
-  int64_t n = rows_p * cols_p;
-  dim3 grid(min(cdiv(n, 256), 4096u), batch);
+  // 16-byte source groups need aligned rows (and for mode 1 a 4-aligned h)
+  const bool vec = ((uintptr_t)src & 15) == 0 && cols % 4 == 0 && sbs % 4 == 0 &&
+                   (mode == 0 || h % 4 == 0) && cols_p % 4 == 0 && dbs % 4 == 0;
+  dim3 grid((unsigned)std::min<int64_t>(rows_p, 148 * 8), batch);
   if (dt == DT_BF16)
     k_cast_weight<<<grid, 256, 0, s>>>(src, (__nv_bfloat16 *)dst, rows, cols, rows_p, cols_p, mode,
-                                       h, hp, sbs, dbs);
+                                       h, hp, sbs, dbs, vec);
   else
     k_cast_weight<<<grid, 256, 0, s>>>(src, (float *)dst, rows, cols, rows_p, cols_p, mode, h, hp,
-                                       sbs, dbs);
+                                       sbs, dbs, vec);
   count_launch();
 }
 
@@ -534,8 +571,119 @@ __global__ void __launch_bounds__(NT) k_cross_entropy(A *__restrict__ z, const i
     zr[v] = from_f<A>(g);
   }
 }
+// bf16 rows held in registers: each thread keeps R 16-byte vectors (8
+// logits each, vector i = threadIdx.x + NT * k) from one read of the row;
+// max, then the sum of 2^(z log2 e - M log2 e), then the gradient, written
+// back once.  Exponentials by the single-instruction ex2 (relative error of a
+// few ulp).  Columns >= V inside the row (padding) get gradient 0.
+LLM_DEV float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <int NT, int R>
+__global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restrict__ z,
+                                                          const int32_t *__restrict__ tgt,
+                                                          float *__restrict__ rowloss, int V,
+                                                          int64_t ldz, float inv_n, int *flag) {
+  constexpr float L2E = 1.4426950408889634f;
+  __shared__ float red[NT / 32];
+  __shared__ float bcast;
+  const int64_t row = blockIdx.x;
+  __nv_bfloat16 *zr = z + row * ldz;
+  const int nvec = (int)(ldz / 8);
+  const int lane = threadIdx.x & 31, w = threadIdx.x / 32;
+  uint4 q[R];
+#pragma unroll
+  for (int k = 0; k < R; k++) {
+    const int i = threadIdx.x + NT * k;
+    q[k] = i < nvec ? reinterpret_cast<const uint4 *>(zr)[i] : make_uint4(0, 0, 0, 0);
+  }
+  int y = tgt[row];
+  if (y < 0 || y >= V) {
+    if (threadIdx.x == 0) atomicOr(flag, FLAG_TOKEN);
+    y = 0;
+  }
+  const float zy = __bfloat162float(zr[y]);
+  // row maximum
+  float m = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < R; k++) {
+    const int v0 = 8 * (threadIdx.x + NT * k);
+    const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&q[k]);
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+      const float2 f = __bfloat1622float2(e[t]);
+      if (v0 + 2 * t < V) m = fmaxf(m, f.x);
+      if (v0 + 2 * t + 1 < V) m = fmaxf(m, f.y);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[w] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float mm = red[0];
+    for (int i = 1; i < NT / 32; i++) mm = fmaxf(mm, red[i]);
+    bcast = mm;
+  }
+  __syncthreads();
+  const float M2 = bcast * L2E;
+  // sum of exponentials (fixed order: thread, then warp shuffle tree, then warps)
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < R; k++) {
+    const int v0 = 8 * (threadIdx.x + NT * k);
+    const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&q[k]);
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+      const float2 f = __bfloat1622float2(e[t]);
+      if (v0 + 2 * t < V) sum += ex2_fast(fmaf(f.x, L2E, -M2));
+      if (v0 + 2 * t + 1 < V) sum += ex2_fast(fmaf(f.y, L2E, -M2));
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  __syncthreads();  // every warp has read bcast before red is reused
+  if (lane == 0) red[w] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float ss = 0.f;
+    for (int i = 0; i < NT / 32; i++) ss += red[i];
+    bcast = ss;
+  }
+  __syncthreads();
+  const float S = bcast;
+  const float lse = M2 / L2E + logf(S);
+  if (threadIdx.x == 0) rowloss[row] = lse - zy;
+  const float LSE2 = lse * L2E;
+  // every thread read z[y] (above) before any vector is written back: the
+  // block barriers of the two reductions order the read before these stores
+#pragma unroll
+  for (int k = 0; k < R; k++) {
+    const int i = threadIdx.x + NT * k;
+    if (i >= nvec) continue;
+    const int v0 = 8 * i;
+    __nv_bfloat162 *e = reinterpret_cast<__nv_bfloat162 *>(&q[k]);
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+      const float2 f = __bfloat1622float2(e[t]);
+      const int va = v0 + 2 * t, vb = va + 1;
+      const float ga = va < V ? (ex2_fast(fmaf(f.x, L2E, -LSE2)) - (va == y ? 1.f : 0.f)) * inv_n : 0.f;
+      const float gb = vb < V ? (ex2_fast(fmaf(f.y, L2E, -LSE2)) - (vb == y ? 1.f : 0.f)) * inv_n : 0.f;
+      e[t] = __floats2bfloat162_rn(ga, gb);
+    }
+    reinterpret_cast<uint4 *>(zr)[i] = q[k];
+  }
+}
+
 void cross_entropy(void *logits, DType dt, const int32_t *tgt, float *rowloss, int64_t N, int V,
                    int64_t ldz, float inv_n, int *flag, cudaStream_t s) {
+  constexpr int NT = 256, R = 16;
+  if (dt == DT_BF16 && ldz % 8 == 0 && ((uintptr_t)logits & 15) == 0 && ldz <= (int64_t)NT * R * 8) {
+    k_cross_entropy_reg<NT, R><<<(unsigned)N, NT, 0, s>>>((__nv_bfloat16 *)logits, tgt, rowloss, V,
+                                                         ldz, inv_n, flag);
+    count_launch();
+    return;
+  }
   if (dt == DT_BF16)
     k_cross_entropy<__nv_bfloat16, 256><<<(unsigned)N, 256, 0, s>>>((__nv_bfloat16 *)logits, tgt,
                                                                    rowloss, V, ldz, inv_n, flag);
@@ -631,25 +779,43 @@ void adamw(float *p, const float *g, float *m, float *v, int64_t n, float lr, fl
 }
 
 // ------------------------------------------------------------ wgrad finish
+// grad[r, c] = sum over splits k (in order) of part[k, r, cp(c)]; mode 1 maps
+// the interleaved W1 | W3 columns back.  One block per row (grid-stride), 4
+// columns per thread: an aligned group of 4 columns has 4 contiguous
+// partial-sum columns in both modes (SWIGLU_BLOCK and h multiples of 4).
 __global__ void k_wgrad_finish(const float *__restrict__ part, int splits, int64_t part_rows,
                                int64_t ldp, float *__restrict__ grad, int64_t rows, int64_t cols,
-                               int mode, int64_t h) {
-  int64_t n = rows * cols;
-  int64_t pstride = part_rows * ldp;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    int64_t r = i / cols, c = i % cols, cp = c;
-    if (mode == 1) cp = (c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK;
-    const float *src = part + r * ldp + cp;
-    float s = 0.f;
-    for (int k = 0; k < splits; k++) s += src[k * pstride];
-    grad[i] = s;
+                               int mode, int64_t h, bool vec) {
+  const int64_t pstride = part_rows * ldp;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float *pr = part + r * ldp;
+    float *gr = grad + r * cols;
+    for (int64_t c = 4 * (int64_t)threadIdx.x; c < cols; c += 4 * (int64_t)blockDim.x) {
+      if (vec && c + 4 <= cols) {
+        const int64_t cp = mode == 1 ? ((c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK) : c;
+        float4 acc = *reinterpret_cast<const float4 *>(pr + cp);
+        for (int k = 1; k < splits; k++) {
+          const float4 q = *reinterpret_cast<const float4 *>(pr + k * pstride + cp);
+          acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+        }
+        *reinterpret_cast<float4 *>(gr + c) = acc;
+      } else {
+        for (int64_t cc = c; cc < c + 4 && cc < cols; cc++) {
+          const int64_t cp = mode == 1 ? ((cc < h) ? w1_col(cc) : w1_col(cc - h) + SWIGLU_BLOCK) : cc;
+          float acc = 0.f;
+          for (int k = 0; k < splits; k++) acc += pr[k * pstride + cp];
+          gr[cc] = acc;
+        }
+      }
+    }
   }
 }
 void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp, float *grad,
                   int64_t rows, int64_t cols, int mode, int64_t h, cudaStream_t s) {
-  unsigned grid = min(cdiv(rows * cols, 256), 148u * 16);
-  k_wgrad_finish<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode, h);
+  const bool vec = ((uintptr_t)part & 15) == 0 && ((uintptr_t)grad & 15) == 0 && ldp % 4 == 0 &&
+                   cols % 4 == 0 && (mode == 0 || h % 4 == 0) && (part_rows * ldp) % 4 == 0;
+  unsigned grid = (unsigned)std::min<int64_t>(rows, 148 * 8);
+  k_wgrad_finish<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode, h, vec);
   count_launch();
 }
 
@@ -728,29 +894,44 @@ __global__ void k_clamp_keys(const int32_t *__restrict__ tok, int32_t *__restric
 // One block per (vocabulary row, 256 columns); each thread owns 4 columns
 // (one float4) and adds the rows of its bucket in position order, loading 8
 // rows ahead so a long bucket (the Zipf head) is not latency-bound.
-__global__ void k_embed_rows(const int32_t *__restrict__ order, const int32_t *__restrict__ offs,
-                             const float *__restrict__ dx, float *__restrict__ dwte, int d) {
-  const int v = blockIdx.x;
-  const int c4 = blockIdx.y * 64 + threadIdx.x;
-  if (4 * c4 >= d) return;
-  const int b = offs[v], e = offs[v + 1];
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  int p = b;
-  for (; p + 8 <= e; p += 8) {
-    float4 t[8];
+// Warp items (vocabulary row v, 128-column chunk), taken in order of v by a
+// grid of whole blocks (the Zipf head -- the longest runs -- starts first);
+// lane = 4 columns.  Each lane adds its run's rows strictly in position
+// order, with the next 16 rows' loads in flight.
+__global__ void __launch_bounds__(256) k_embed_rows(const int32_t *__restrict__ order,
+                                                   const int32_t *__restrict__ offs,
+                                                   const float *__restrict__ dx,
+                                                   float *__restrict__ dwte, int d, int V) {
+  const int nchunk = (d + 127) / 128;
+  const int64_t items = (int64_t)V * nchunk;
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t it = wid; it < items; it += nw) {
+    const int v = (int)(it / nchunk), ch = (int)(it % nchunk);
+    const int c4 = ch * 32 + lane;  // float4 column index
+    const bool on = 4 * c4 < d;
+    const int b = offs[v], e = offs[v + 1];
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    int p = b;
+    for (; p + 16 <= e; p += 16) {
+      float4 t[16];
 #pragma unroll
-    for (int u = 0; u < 8; u++)
-      t[u] = reinterpret_cast<const float4 *>(dx + (int64_t)order[p + u] * d)[c4];
+      for (int u = 0; u < 16; u++)
+        t[u] = on ? reinterpret_cast<const float4 *>(dx + (int64_t)order[p + u] * d)[c4]
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int u = 0; u < 8; u++) {
-      s.x += t[u].x; s.y += t[u].y; s.z += t[u].z; s.w += t[u].w;
+      for (int u = 0; u < 16; u++) {
+        s.x += t[u].x; s.y += t[u].y; s.z += t[u].z; s.w += t[u].w;
+      }
     }
+    for (; p < e; p++) {
+      if (!on) continue;
+      const float4 t = reinterpret_cast<const float4 *>(dx + (int64_t)order[p] * d)[c4];
+      s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+    }
+    if (on) reinterpret_cast<float4 *>(dwte + (int64_t)v * d)[c4] = s;
   }
-  for (; p < e; p++) {
-    float4 t = reinterpret_cast<const float4 *>(dx + (int64_t)order[p] * d)[c4];
-    s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
-  }
-  reinterpret_cast<float4 *>(dwte + (int64_t)v * d)[c4] = s;
 }
 // Same sums for any d or alignment (one thread per column, rows in order).
 __global__ void k_embed_rows_scalar(const int32_t *__restrict__ order,
@@ -794,7 +975,8 @@ void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int 
   }
   k_scan_excl<<<1, 1024, 0, s>>>(offs, V + 1);
   if ((d & 3) == 0 && ((uintptr_t)dx & 15) == 0 && ((uintptr_t)dwte & 15) == 0)
-    k_embed_rows<<<dim3(V, cdiv(d, 256)), 64, 0, s>>>(vin, offs, dx, dwte, d);
+    k_embed_rows<<<(unsigned)std::min<int64_t>(((int64_t)V * cdiv(d, 128) + 7) / 8, 148 * 8), 256,
+                   0, s>>>(vin, offs, dx, dwte, d, V);
   else
     k_embed_rows_scalar<<<V, min(256, ((d + 31) / 32) * 32), 0, s>>>(vin, offs, dx, dwte, d);
   count_launch(2);

@@ -75,13 +75,29 @@ struct POff {
   int64_t wlm() const { return gf() + D.d; }
 };
 
-// Split count of a weight-gradient GEMM (K = tokens): enough (tile, split)
-// pairs to fill the GPU twice, each split at least 512 tokens long.
+// Split count of a weight-gradient GEMM (K = tokens).  The GEMM runs
+// (128 x 256 tile, split) items on 148 SMs in whole waves, so the split count
+// minimises an estimate of waves x k-blocks per item (520 cycles per block of
+// 64 at the tensor rate, 1.9 GHz) plus the partial sums' extra HBM traffic
+// (written by the GEMM, read by the finish pass, 6.5 TB/s); every split keeps
+// at least 8 k-blocks, at most 32 splits.
 int wgrad_splits(const Dims &D, int64_t M, int64_t Ncols) {
-  int64_t tiles = ((M + 127) / 128) * ((Ncols + 127) / 128);
-  int64_t want = (2 * 148 + tiles - 1) / tiles;
-  int64_t maxs = std::max<int64_t>(1, D.N / 512);
-  return (int)std::max<int64_t>(1, std::min<int64_t>({want, maxs, 32}));
+  const int64_t tiles = ((M + 127) / 128) * ((Ncols + 255) / 256);
+  const int64_t kb = (D.N + 63) / 64;
+  int best = 1;
+  double best_us = 1e300;
+  for (int s = 1; s <= 32; s++) {
+    const int64_t kbs = (kb + s - 1) / s;
+    if (s > 1 && kbs < 8) break;
+    const double waves = (double)((tiles * s + 147) / 148);
+    const double us = waves * (double)kbs * 520.0 / 1900.0 +
+                      2.0 * s * (double)M * (double)Ncols * 4.0 / 6.5e6;
+    if (us < best_us * (1.0 - 1e-9)) {
+      best_us = us;
+      best = s;
+    }
+  }
+  return best;
 }
 
 // Workspace carve: the same sequence of (size) requests both sizes and

@@ -249,6 +249,42 @@ LLM_DEV bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_sh, in
     }
   }
 }
+// N consecutive TMEM columns of this thread's lane (N = 8, 16, 32 or 64),
+// one wait for all of them.
+template <int N>
+LLM_DEV void tmem_ldn(uint32_t taddr, float (&v)[N]) {
+  if constexpr (N == 64) {
+    tmem_ld64(taddr, v);
+  } else if constexpr (N == 32) {
+    tmem_ld32(taddr, v);
+  } else if constexpr (N == 16) {
+    tmem_ld16(taddr, v);
+  } else {
+    static_assert(N == 8, "tmem_ldn: 8, 16, 32 or 64 columns");
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; i++) v[i] = __uint_as_float(r[i]);
+  }
+}
+// N packed words (N = 8 or 16) into consecutive TMEM columns, no wait.
+template <int N>
+LLM_DEV void tmem_stn(uint32_t taddr, const uint32_t *w) {
+  if constexpr (N == 16) {
+    tmem_st16(taddr, *reinterpret_cast<const uint32_t (*)[16]>(w));
+  } else {
+    static_assert(N == 8, "tmem_stn: 8 or 16 columns");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                     taddr),
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                 "r"(w[7])
+                 : "memory");
+  }
+}
 LLM_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
