@@ -6,15 +6,17 @@
 //     dS_ij = P_ij (dO_i.v_j - D_i)
 //     dQ = scale * dS K,   dK = scale * dS^T Q,   dV = P^T dO,
 // recomputed block by block so no T x T matrix reaches memory.  Two kernels,
-// both with 128 x 128 blocks, one CTA per SM (512 TMEM columns), 11 warps:
+// both with 128 x 128 blocks, one CTA per SM (512 TMEM columns), 19 warps:
 //   warp 0      TMA producer (Q/dO or K/V once, the other pair through a
 //               2-deep ring);
-//   warps 1, 10 MMA issuers A and B (whole converged warps, one elected lane;
+//   warps 1, 18 MMA issuers A and B (whole converged warps, one elected lane;
 //               one warp issues a tcgen05.mma only every ~127 cycles whatever
 //               N is, so the products are split between two warps); warp 1
 //               also allocates TMEM;
-//   warps 2..9  elementwise warps, two per TMEM lane quarter: thread = one
-//               row of the block (TMEM lane) and one half (64 columns).
+//   warps 2..17 elementwise warps, four per TMEM lane quarter: thread = one
+//               row of the block (TMEM lane) and one column group (32 of the
+//               block's 128 columns); four groups per row keep enough warps
+//               in flight to cover the TMEM, SFU and shared-memory latencies.
 // dQ kernel (grid H x B x query blocks, longest rows first), per key block j:
 //   S = Q K_j^T (issuer A) and dP = dO V_j^T (issuer B) (M 128, N 128, K 64;
 //   operands K-major in shared memory) into TMEM; the elementwise warps read
@@ -46,7 +48,7 @@ using namespace tc;
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 2;
-constexpr int EW_WARPS = 8;  // elementwise warps: 4 lane quarters x NCQ column groups
+constexpr int EW_WARPS = 16;  // elementwise warps: 4 lane quarters x NCQ column groups
 constexpr int NCQ = EW_WARPS / 4;  // column groups of a row (2 or 4)
 constexpr int CW = 128 / NCQ;      // score columns per thread
 constexpr int HW = 32 / NCQ;       // head columns per thread in each RoPE half
