@@ -37,6 +37,29 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "training tokens/sec (fwd+bwd+AdamW) on 1 B200; % of tensor/HBM roofline"
+# DRAM bytes (read + write) per tcgen05 GEMM launch, averaged over the 243
+# GEMM launches of one 350M step (profiles/gemm_dram_traffic_step_350m.md);
+# valid only for the GEMM sources that were captured, identified by hash.
+GEMM_TRAFFIC = {"bytes_per_launch": 256.5e6, "workload": "350m-v32000-d1024-l20-bf16",
+                "sha256": {"gemm_tc.cu": "fbee4d44c173eecd28aa7a64d76c1578fc5bb65d6cd8fac68e5415f3f4d5fde9",
+                           "tcgen05.cuh": "062e7fbd85e8e8eb829ae9081c3849a887fdfcfea2721b394d186b20100514a8"}}
+
+
+def gemm_traffic(workload):
+    """The captured GEMM traffic per launch if the GEMM sources are unchanged
+    since the capture and the workload is the captured one, else None."""
+    import hashlib
+    if workload != GEMM_TRAFFIC["workload"]:
+        return None
+    for name, want in GEMM_TRAFFIC["sha256"].items():
+        path = os.path.join(ROOT, "scratch_llama_decoder_b200", "csrc", name)
+        try:
+            with open(path, "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != want:
+                    return None
+        except OSError:
+            return None
+    return GEMM_TRAFFIC["bytes_per_launch"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -291,7 +314,8 @@ def run_ours(args, rank, world, local_rank):
                    "several GB per step; no flush)"},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM (all projection GEMMs of the "
                      "step)", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
-                     "frac": achieved / peak_tc if peak_tc else None, "traffic": None,
+                     "frac": achieved / peak_tc if peak_tc else None,
+                     "traffic": gemm_traffic(cfg["name"]),
                      "launches": g_launch, "ms_total": g_ms,
                      "peak_source": f"{src} bf16_tflops_sustained"},
         "step_roofline": {"flops": F, "attention_flops": F_attn,

@@ -503,10 +503,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         epilogue_tile(a, &tmC, 0, row0, n0, c_lo, split, true, stg, sb);
         continue;
       }
-      int got = 0;
-      if (lane == 0) got = mbar_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag) ? 1 : 0;
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) break;
+      if (!warp_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag)) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
       epilogue_tile(a, &tmC, tm, row0, n0, c_lo, split, false, stg, sb);
