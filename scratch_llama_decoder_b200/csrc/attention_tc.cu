@@ -3,30 +3,31 @@
 // scores in memory, only the row log-sum-exp saved) on the 5th-generation
 // tensor cores.
 //
-// One CTA = 128 queries of one (batch, head); key blocks of 128.  11 warps:
-//   warp 0      TMA producer: the Q tile once, K and V tiles into 2-deep rings;
-//   warp 1      TMEM allocation and MMA issuer A:
-//                 S    = Q K^T          (M 128, N 128, K 64; both operands
-//                                        K-major in shared memory) -> TMEM S
-//                 O_a += P_a V[0:64]    (M 128, N 64, K 64; A = P_a from TMEM,
-//                                        B = V MN-major)           -> TMEM O_a
-//   warp 10     MMA issuer B:  O_b += P_b V[64:128]                -> TMEM O_b
-//   warps 2..9  softmax, two warps per TMEM lane quarter: thread = one query
-//               row (TMEM lane) and one half of the block's keys (a: keys
-//               0..63, b: 64..127).
-// The two key halves are two independent online softmaxes (split-K inside the
-// CTA): each half-row thread keeps its own running maximum m, sum l and
-// accumulator O_x, so no thread waits for another inside the key loop; the
-// halves meet once at the end, O = (2^(m_a-m) O_a + 2^(m_b-m) O_b) /
-// (2^(m_a-m) l_a + 2^(m_b-m) l_b) with m = max(m_a, m_b).  The running maximum
-// is lazy: the reference of a half-row moves only when a block's maximum
-// exceeds it by more than 2^8, so P stays below 256 and O_x is rescaled only
-// then; O_x and l_x always share one reference.  The half-row is read from
-// TMEM in one round trip and S is released at once, so Q K_{j+1}^T runs during
-// block j's exponentials.  MMAs are issued by whole converged warps (one
-// elected lane), from two warps because one warp issues a tcgen05.mma only
-// every ~127 cycles whatever N is.  Every wait is bounded (FLAG_TIMEOUT, then
-// drain and free TMEM).
+// One CTA = 128 queries of one (batch, head); key blocks of 128, split into
+// NQ key groups of KW = 128 / NQ keys.  Warps:
+//   warp 0          TMA producer: the Q tile once, K and V tiles into 2-deep
+//                   rings;
+//   warp 1          TMEM allocation and MMA issuer A:
+//                     S    = Q K^T       (M 128, N 128, K 64; both operands
+//                                         K-major in shared memory) -> TMEM S
+//                     O_g += P_g V_g     for key groups g < NQ/2 (M 128, N 64,
+//                                         K KW; A = P_g from TMEM, B = the V
+//                                         rows of group g, MN-major) -> TMEM O_g
+//   last warp       MMA issuer B: O_g += P_g V_g for groups g >= NQ/2;
+//   4 NQ warps      softmax, NQ per TMEM lane quarter: thread = one query row
+//                   (TMEM lane) and one key group.
+// The key groups are NQ independent online softmaxes (split-K inside the CTA):
+// each (row, group) thread keeps its own running maximum m_g, sum l_g and
+// accumulator O_g, so no thread waits for another inside the key loop; the
+// groups meet once at the end, O = sum_g 2^(m_g-m) O_g / sum_g 2^(m_g-m) l_g
+// with m = max_g m_g.  The running maximum is lazy: the reference of a
+// (row, group) moves only when a block's maximum exceeds it by more than 2^8,
+// so P stays below 256 and O_g is rescaled only then; O_g and l_g always share
+// one reference.  The group's scores are read from TMEM in one round trip and
+// S is released at once, so Q K_{j+1}^T runs during block j's exponentials.
+// MMAs are issued by whole converged warps (one elected lane), from two warps
+// because one warp issues a tcgen05.mma only every ~127 cycles whatever N is.
+// Every wait is bounded (FLAG_TIMEOUT, then drain and free TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "tcgen05.cuh"
@@ -39,16 +40,21 @@ using namespace tc;
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 2;
-constexpr int SM_WARPS = 8;  // softmax warps
+constexpr int NQ = 4;             // key groups of a block (independent softmaxes)
+constexpr int KW = 128 / NQ;      // keys per group (softmax thread)
+constexpr int SM_WARPS = 4 * NQ;  // softmax warps: 4 lane quarters x NQ groups
 constexpr int MMA_B_WARP = 2 + SM_WARPS;
 constexpr int NTHREADS = 32 * (MMA_B_WARP + 1);
 constexpr int TMEM_COLS = 512;
-constexpr int COL_S = 0, COL_P = 128, COL_OA = 192, COL_OB = 256;
+// TMEM columns: S [0,128), P (packed bf16, group g at COL_P + g KW/2), O_g at
+// COL_O + 64 g
+constexpr int COL_S = 0, COL_P = 128, COL_O = 192;
+static_assert(COL_O + 64 * NQ <= TMEM_COLS, "TMEM columns");
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
 // shared memory: Q | K[2] | V[2] | barriers | red
-constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 4 * 128 * 4 + 1024;
+constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 2 * NQ * 128 * 4 + 1024;
 
 // Named barrier of the softmax warps (id 1) that ANDs a flag over them.
 LLM_DEV bool softmax_all(bool v) {
@@ -71,13 +77,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
   uint32_t *tmem_sh = (uint32_t *)(bars + 24);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
-  float *red = (float *)(bars + 32);  // [4][128]: m_a, m_b, l_a, l_b per row
+  float *red = (float *)(bars + 32);  // [2][NQ][128]: m_g, then l_g per row
   const uint32_t b0 = smem_u32(bars);
   const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
                  v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
-                 p_full = b0 + 8 * 11,   // [2]: half a, half b
-                 o_done = b0 + 8 * 13,   // [2]
-                 drain = b0 + 8 * 15;    // [2]: one per MMA warp
+                 p_full = b0 + 8 * 11,             // [NQ]: one per key group
+                 o_done = p_full + 8 * NQ,         // [NQ]
+                 drain = o_done + 8 * NQ;          // [2]: one per MMA warp
+  static_assert(11 + 2 * NQ + 2 <= 24, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -97,11 +104,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, SM_WARPS);
-    for (int x = 0; x < 2; x++) {
-      mbar_init(p_full + 8 * x, SM_WARPS / 2);
-      mbar_init(o_done + 8 * x, 1);
-      mbar_init(drain + 8 * x, 1);
+    for (int g2 = 0; g2 < NQ; g2++) {
+      mbar_init(p_full + 8 * g2, 4);  // the group's four lane-quarter warps
+      mbar_init(o_done + 8 * g2, 1);
     }
+    mbar_init(drain, 1);
+    mbar_init(drain + 8, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -187,21 +195,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_after();
         issue_s(j + 1);
       }
-      if (!warp_wait(p_full + 8 * x, j & 1, abort_sh, gflag) ||
-          !warp_wait(v_full + 8 * s, ph, abort_sh, gflag)) {
+      if (!warp_wait(v_full + 8 * s, ph, abort_sh, gflag)) {
         ok = false;
         break;
       }
-      fence_after();
-      // O_x += P_x V[64x : 64x + 64]: 4 K-steps of 16 keys
       const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 8192, 1024);
-      const uint32_t col_o = x ? COL_OB : COL_OA;
+      // O_g += P_g V[g KW : g KW + KW] for this warp's groups: KW / 16 K-steps
 #pragma unroll
-      for (int kk = 0; kk < 4; kk++)
-        mma_ts_e(tmem + col_o, tmem + COL_P + x * 32 + kk * 8,
-                 vd + (uint64_t)((x * 4 + kk) * 128), ID_O, (j > 0 || kk > 0) ? 1u : 0u);
+      for (int gg = 0; gg < NQ / 2; gg++) {
+        const int grp = x * (NQ / 2) + gg;
+        if (!warp_wait(p_full + 8 * grp, j & 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+#pragma unroll
+        for (int kk = 0; kk < KW / 16; kk++)
+          mma_ts_e(tmem + COL_O + 64 * grp, tmem + COL_P + grp * (KW / 2) + kk * 8,
+                   vd + (uint64_t)((grp * (KW / 16) + kk) * 128), ID_O,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_e(o_done + 8 * grp);
+      }
+      if (!ok) break;
       mma_commit_e(v_empty + 8 * s);
-      mma_commit_e(o_done + 8 * x);
     }
     mma_commit_e(drain + 8 * x);
     if (lane == 0) {
@@ -213,11 +229,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
-    const int ch = (warp - 2) >> 2;  // which key half of the block
+    const int grp = (warp - 2) >> 2;    // key group: keys [grp KW, grp KW + KW) of a block
     const int r = quarter * 32 + lane;  // row of the tile = TMEM lane
     const int qi = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t col_o = ch ? COL_OB : COL_OA;
+    const uint32_t col_o = COL_O + 64 * grp;
     const float sl2 = scale * LOG2E;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
@@ -227,17 +243,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       fence_after();
-      const int k0 = j * BK + ch * 64;
+      const int k0 = j * BK + grp * KW;
       const bool diag = (j * BK + BK > q0);  // only the diagonal block (or T) masks
-      float sv[64];
-      tmem_ld64(tmem + lane_off + COL_S + ch * 64, sv);
+      float sv[KW];
+      tmem_ldn<KW>(tmem + lane_off + COL_S + grp * KW, sv);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
-      // this half-row's block maximum (log2 units), 4 independent chains
+      // this group's block maximum (log2 units), 4 independent chains
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < 64; i++) {
+      for (int i = 0; i < KW; i++) {
         float x = sv[i] * sl2;
         if (diag && (k0 + i > qi || k0 + i >= T)) x = -INFINITY;
         sv[i] = x;
@@ -246,9 +262,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       // true on the first block with an unmasked key (m_ref = -inf until then)
       const bool need = mx > m_ref + LAZY;
-      // P_x and O_x of the previous block are free once its P V has completed
+      // P_g and O_g of the previous block are free once its P V has completed
       if (j > 0) {
-        if (!warp_wait(o_done + 8 * ch, (j - 1) & 1, abort_sh, gflag)) {
+        if (!warp_wait(o_done + 8 * grp, (j - 1) & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
@@ -256,73 +272,85 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (__any_sync(0xffffffffu, need)) {
           const float corr = need ? ex2(m_ref - mx) : 1.f;  // 0 while m_ref = -inf
 #pragma unroll
-          for (int c = 0; c < 2; c++) {
-            float v[32];
-            tmem_ld32(tmem + lane_off + col_o + c * 32, v);
+          for (int c = 0; c < 4; c++) {
+            float v[16];
+            uint32_t u[16];
+            tmem_ld16(tmem + lane_off + col_o + c * 16, v);
 #pragma unroll
-            for (int i = 0; i < 32; i++) v[i] *= corr;
-            tmem_st32(tmem + lane_off + col_o + c * 32, v);
+            for (int i = 0; i < 16; i++) u[i] = __float_as_uint(v[i] * corr);
+            tmem_st16(tmem + lane_off + col_o + c * 16, u);
           }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         }
       }
       if (need) {
         if (m_ref != -INFINITY) l *= ex2(m_ref - mx);
         m_ref = mx;
       }
-      // P = 2^(s - m_ref), packed bf16 into this half's 32 TMEM columns; a
-      // half-row with no unmasked key yet (m_ref = -inf) gets P = 0
+      // P = 2^(s - m_ref), packed bf16 into this group's KW/2 TMEM columns; a
+      // (row, group) with no unmasked key yet (m_ref = -inf) gets P = 0
       const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-      uint32_t w[32];
+      uint32_t w[KW / 2];
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
+      for (int i = 0; i < KW; i += 2) {
         const float p0 = ex2(sv[i] - mr), p1 = ex2(sv[i + 1] - mr);
         l4[(i >> 1) & 3] += p0 + p1;
         w[i / 2] = pack_bf16(p0, p1);
       }
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t (&wc)[16] = *reinterpret_cast<uint32_t (*)[16]>(&w[c * 16]);
-        tmem_st16(tmem + lane_off + COL_P + ch * 32 + c * 16, wc);
-      }
+      for (int c = 0; c < KW / 2; c += 16)
+        tmem_stn<(KW / 2 < 16 ? KW / 2 : 16)>(tmem + lane_off + COL_P + grp * (KW / 2) + c, w + c);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + 8 * ch);
+      if (lane == 0) mbar_arrive(p_full + 8 * grp);
     }
-    // the two halves meet: shared reference m, combined sum and output; both
-    // accumulators are complete once both o_done phases of the last block are
-    if (ok)
-      ok = warp_wait(o_done, (nj - 1) & 1, abort_sh, gflag) &&
-           warp_wait(o_done + 8, (nj - 1) & 1, abort_sh, gflag);
-    red[ch * 128 + r] = m_ref;
-    red[256 + ch * 128 + r] = l;
+    // the groups meet: shared reference m, combined sum and output; every
+    // accumulator is complete once every o_done phase of the last block is
+#pragma unroll
+    for (int g2 = 0; g2 < NQ; g2++)
+      if (ok) ok = warp_wait(o_done + 8 * g2, (nj - 1) & 1, abort_sh, gflag);
+    red[grp * 128 + r] = m_ref;
+    red[(NQ + grp) * 128 + r] = l;
     // barrier of the softmax warps that also tells whether every one finished
     if (softmax_all(ok)) {
       fence_after();
-      const float ma = red[r], mb = red[128 + r], la = red[256 + r], lb = red[384 + r];
-      const float m = fmaxf(ma, mb);
-      const float fa = ma == -INFINITY ? 0.f : ex2(ma - m);
-      const float fb = mb == -INFINITY ? 0.f : ex2(mb - m);
-      const float lt = la * fa + lb * fb;
-      const float inv = 1.f / lt;
-      float va[32], vb[32];
-      tmem_ld32(tmem + lane_off + COL_OA + ch * 32, va);
-      tmem_ld32(tmem + lane_off + COL_OB + ch * 32, vb);
-      if (qi < T) {
-        __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + ch * 32;
-        const float ca = fa * inv, cb = fb * inv;
+      float m = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
+      for (int g2 = 0; g2 < NQ; g2++) m = fmaxf(m, red[g2 * 128 + r]);
+      float f[NQ], lt = 0.f;
+#pragma unroll
+      for (int g2 = 0; g2 < NQ; g2++) {
+        const float mg = red[g2 * 128 + r];
+        f[g2] = mg == -INFINITY ? 0.f : ex2(mg - m);
+        lt += red[(NQ + g2) * 128 + r] * f[g2];
+      }
+      const float inv = 1.f / lt;
+      // this thread's 64 / NQ output columns: [grp 64/NQ, grp 64/NQ + 64/NQ)
+      constexpr int OW = 64 / NQ;
+      float acc[OW];
+#pragma unroll
+      for (int i = 0; i < OW; i++) acc[i] = 0.f;
+#pragma unroll
+      for (int g2 = 0; g2 < NQ; g2++) {
+        float v[OW];
+        tmem_ldn<OW>(tmem + lane_off + COL_O + 64 * g2 + grp * OW, v);
+        const float cg = f[g2] * inv;
+#pragma unroll
+        for (int i = 0; i < OW; i++) acc[i] += v[i] * cg;
+      }
+      if (qi < T) {
+        __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + grp * OW;
+#pragma unroll
+        for (int i = 0; i < OW; i += 8) {
           uint32_t wv[4];
 #pragma unroll
-          for (int e = 0; e < 4; e++)
-            wv[e] = pack_bf16(va[i + 2 * e] * ca + vb[i + 2 * e] * cb,
-                              va[i + 2 * e + 1] * ca + vb[i + 2 * e + 1] * cb);
+          for (int e = 0; e < 4; e++) wv[e] = pack_bf16(acc[i + 2 * e], acc[i + 2 * e + 1]);
           *reinterpret_cast<uint4 *>(dst + i) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
-        if (ch == 0) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
+        if (grp == 0) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
       }
     }
   }
