@@ -4,12 +4,16 @@
 // Persistent kernel, one CTA per SM, 10 warps:
 //   warp 0      TMA producer: A and B tiles into a STAGES-deep shared-memory
 //               ring (128-byte swizzle), completion counted on mbarriers;
-//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=256, K=16) and commits each stage back to the ring;
+//   warp 1      allocates 512 TMEM columns; issues tcgen05.mma (M=128, N=256,
+//               K=16) and commits each stage back to the ring;
+// (warps 0 and 1 run as whole converged warps; one elected lane issues each
+// copy, MMA and commit)
 //   warps 2..9  epilogue, two warps per TMEM lane quarter, each taking half
 //               of the tile's columns: tcgen05.ld of the accumulator (one
 //               TMEM lane = one output row per thread), the fused epilogue,
-//               and row-coalesced stores through a swizzled shared square.
+//               and bulk tensor stores of a swizzled shared staging square
+//               (a residual comes in through bulk tensor loads of the same
+//               square).
 // Two accumulators of 256 columns alternate so the epilogue of one tile
 // overlaps the main loop of the next.  Operands may be K-major or MN-major
 // (both supported by the UMMA descriptors), which covers the forward
@@ -47,7 +51,6 @@ struct Args {
   int M, N, K;
   int tiles_m, tiles_n, splits, kchunk, total;
   int out, epi;
-  int tma_store;  // 1: the tile leaves through bulk tensor stores of the staging square
   void *C;
   int64_t ldc;
   const float *R;
@@ -58,12 +61,11 @@ struct Args {
 };
 
 // ------------------------------------------------------------ epilogue stores
-// Coalesced write-out of a warp's 32 x 32 chunk: lane i holds row i in v.
-// The chunk goes through a 32 x 32 float square in shared memory whose
-// 16-byte groups are XOR-swizzled by the row (group g of row r sits at
-// position g ^ (r & 7)), so both the row-wise 16-byte writes and the
-// 4-rows-per-instruction reads hit 32 distinct banks; each global store
-// instruction then covers 4 full row segments.  rows / cols clip the edges.
+// A warp's 32 x 32 fp32 chunk (lane i holds row i in v) in the per-warp
+// staging square: 16-byte group g of row r sits at position g ^ (r & 7), the
+// 128-byte-swizzle image of a 32-row x 128-byte box, so the row-wise 16-byte
+// writes spread over all banks and the square is what a bulk tensor copy of
+// that box reads or writes.
 LLM_DEV float4 *sq(float *stg, int r, int g) {
   return reinterpret_cast<float4 *>(stg + r * 32 + 4 * (g ^ (r & 7)));
 }
@@ -73,66 +75,6 @@ LLM_DEV void stage32(float *stg, const float (&v)[32]) {
   for (int g = 0; g < 8; g++) *sq(stg, lane, g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
   __syncwarp();
 }
-// Rows of the warp's 32-row slab, 4 columns per lane (lane&7), 4 rows per
-// instruction: the residual values put32_f32 adds, all loads in flight first.
-LLM_DEV void ld32_f32(const float *R, int64_t ldr, int rows, int cols, float4 (&rv)[8]) {
-  const int lane = threadIdx.x & 31;
-  const int c = 4 * (lane & 7), rsub = lane >> 3;
-  const bool full = c + 4 <= cols;
-#pragma unroll
-  for (int k = 0; k < 8; k++) {
-    const int r = rsub + 4 * k;
-    rv[k] = (R && full && r < rows) ? *reinterpret_cast<const float4 *>(R + (int64_t)r * ldr + c)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-LLM_DEV void put32_f32(float *stg, const float (&v)[32], float *dst, int64_t ld, int rows,
-                       int cols, const float *R, int64_t ldr, const float4 (&rv)[8]) {
-  stage32(stg, v);
-  const int lane = threadIdx.x & 31;
-  const int g = lane & 7, c = 4 * g, rsub = lane >> 3;
-  const bool full = c + 4 <= cols;
-  if (c < cols) {
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      const int r = rsub + 4 * k;
-      if (r >= rows) break;
-      float4 x = *sq(stg, r, g);
-      if (full) {
-        x.x += rv[k].x; x.y += rv[k].y; x.z += rv[k].z; x.w += rv[k].w;
-        *reinterpret_cast<float4 *>(dst + (int64_t)r * ld + c) = x;
-      } else {
-        float e[4] = {x.x, x.y, x.z, x.w};
-        for (int q = 0; c + q < cols; q++)
-          dst[(int64_t)r * ld + c + q] = e[q] + (R ? R[(int64_t)r * ldr + c + q] : 0.f);
-      }
-    }
-  }
-  __syncwarp();
-}
-LLM_DEV void put32_bf16(float *stg, const float (&v)[32], __nv_bfloat16 *dst, int64_t ld, int rows,
-                        int cols) {
-  stage32(stg, v);
-  const int lane = threadIdx.x & 31;
-  const int g = lane & 7, c = 4 * g, rsub = lane >> 3;
-  if (c < cols) {
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      const int r = rsub + 4 * k;
-      if (r >= rows) break;
-      float4 x = *sq(stg, r, g);
-      if (c + 4 <= cols) {
-        *reinterpret_cast<uint2 *>(dst + (int64_t)r * ld + c) =
-            make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
-      } else {
-        float e[4] = {x.x, x.y, x.z, x.w};
-        for (int q = 0; c + q < cols; q++) dst[(int64_t)r * ld + c + q] = __float2bfloat16_rn(e[q]);
-      }
-    }
-  }
-  __syncwarp();
-}
-
 // Bulk tensor stores.  The staging square is laid out as the 128-byte-swizzle
 // image of a 32-row x 128-byte box (16-byte group g of row r at g ^ (r & 7)),
 // i.e. exactly what the tensor map of C expects; the copy engine clips rows
@@ -198,16 +140,17 @@ LLM_DEV void rope32(float (&v)[32], const float *cos_row, const float *sin_row) 
 // half of the columns, [n0 + c_lo, n0 + c_lo + BN/2).  Every lane executes
 // every tcgen05.ld (warp-uniform control); rows past M and columns past N are
 // clipped only at the stores.
-LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, int row0, int n0,
-                           int c_lo, int split, bool zero, float *stg_base, int &sb) {
+LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, const CUtensorMap *tmR,
+                           uint32_t rbar, uint32_t &rph, volatile int *abort_sh, uint32_t tm,
+                           int row0, int n0, int c_lo, int split, bool zero, float *stg_base,
+                           int &sb) {
   float *stg = stg_base;
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
   const int rows = max(0, min(32, a.M - row0));
   const int N = a.N;
-  auto ncols = [&](int n) { return max(0, min(32, N - n)); };
   float v[32];
-  if (a.tma_store) {
+  {
     if (rows == 0) return;  // the warp's 32 rows lie past M: nothing to store
     if (a.out == OUT_ACT) {
       // bf16, 64 columns per store: plain, or RoPE on q/k head columns
@@ -251,96 +194,46 @@ LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, i
         bulk_store(stg, tmC, n, row0, 0, false);
       }
     } else {
-      // fp32 (plain, or split-K partial into slab `split`), 32 columns per store
-      const bool part = a.out == OUT_PARTIAL;
+      // fp32 (plain, residual add, or split-K partial into slab `split`), 32
+      // columns per store; the residual chunk R[rows, n : n + 32] is brought
+      // into the staging square by a bulk tensor load (zero past M and N)
+      // while the accumulator is read from TMEM, then added in place
+      const bool part = a.out == OUT_PARTIAL, add = a.out == OUT_ADD_F32;
       for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
         const int n = n0 + c0;
         if (n >= N) break;
-        if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
-        else tmem_ld32(tm + c0, v);
         stg = stg_base + sb * 32 * 32;
         sb = sb + 1 == STG_BUFS ? 0 : sb + 1;
         stg_acquire();
+        if (add) {
+          mbar_arrive_expect_tx_e(rbar, 32 * 32 * 4);
+          tma_load_2d_e(smem_u32(stg), tmR, n, row0, rbar);
+        }
+        if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
+        else tmem_ld32(tm + c0, v);
+        if (add) {
+          const uint32_t ph = rph;
+          rph ^= 1u;
+          if (!warp_wait(rbar, ph, abort_sh, a.flag)) {
+            // time-out: the load must land before the square is reused or freed
+            if ((threadIdx.x & 31) == 0) {
+              const unsigned long long t0 = gtimer();
+              while (!mbar_try(rbar, ph) && gtimer() - t0 < WAIT_NS) {
+              }
+            }
+            __syncwarp();
+            return;
+          }
+#pragma unroll
+          for (int g = 0; g < 8; g++) {
+            const float4 r4 = *sq(stg, lane, g);
+            v[4 * g] += r4.x; v[4 * g + 1] += r4.y; v[4 * g + 2] += r4.z; v[4 * g + 3] += r4.w;
+          }
+          __syncwarp();
+        }
         stage32(stg, v);
         bulk_store(stg, tmC, n, row0, split, part);
       }
-    }
-    return;
-  }
-  if (a.epi == TC_EPI_ROPE) {
-    // RoPE on q/k heads (columns < rot_cols), plain store of v heads.
-    const int hd = a.hd, half = hd / 2, t = m % a.T;
-    __nv_bfloat16 *C = (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc;
-    if (hd == 64) {
-      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 64) {
-        int n = n0 + c0;
-        if (n >= N) break;
-        float lo[32], hi[32];
-        if (zero) { for (int i = 0; i < 32; i++) lo[i] = hi[i] = 0.f; }
-        else { tmem_ld32(tm + c0, lo); tmem_ld32(tm + c0 + 32, hi); }
-        if (n < a.rot_cols) {
-          const float4 *ct = reinterpret_cast<const float4 *>(a.cos_t + (int64_t)t * half);
-          const float4 *st = reinterpret_cast<const float4 *>(a.sin_t + (int64_t)t * half);
-#pragma unroll
-          for (int j4 = 0; j4 < 8; j4++) {
-            float4 c4 = ct[j4], s4 = st[j4];
-            const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-              int j = 4 * j4 + k;
-              float x = lo[j], y = hi[j];
-              lo[j] = x * cc[k] - y * ss[k];
-              hi[j] = y * cc[k] + x * ss[k];
-            }
-          }
-        }
-        put32_bf16(stg, lo, C + n, a.ldc, rows, ncols(n));
-        put32_bf16(stg, hi, C + n + 32, a.ldc, rows, ncols(n + 32));
-      }
-    } else {  // hd == 32: both halves of a head sit in one 32-column chunk
-      for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
-        int n = n0 + c0;
-        if (n >= N) break;
-        if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
-        else tmem_ld32(tm + c0, v);
-        if (n < a.rot_cols) {
-          const float4 *ct = reinterpret_cast<const float4 *>(a.cos_t + (int64_t)t * half);
-          const float4 *st = reinterpret_cast<const float4 *>(a.sin_t + (int64_t)t * half);
-#pragma unroll
-          for (int j4 = 0; j4 < 4; j4++) {
-            float4 c4 = ct[j4], s4 = st[j4];
-            const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-              int j = 4 * j4 + k;
-              float x = v[j], y = v[j + 16];
-              v[j] = x * cc[k] - y * ss[k];
-              v[j + 16] = y * cc[k] + x * ss[k];
-            }
-          }
-        }
-        put32_bf16(stg, v, C + n, a.ldc, rows, ncols(n));
-      }
-    }
-    return;
-  }
-  // Plain outputs (a residual is loaded, all eight row groups at once, just
-  // before the chunk is staged).
-  const bool add = a.out == OUT_ADD_F32;
-  const float *Rrow = add ? a.R + (int64_t)row0 * a.ldr : nullptr;
-  for (int c0 = c_lo; c0 < c_lo + BN / 2; c0 += 32) {
-    int n = n0 + c0;
-    if (n >= N) break;
-    if (zero) { for (int i = 0; i < 32; i++) v[i] = 0.f; }
-    else tmem_ld32(tm + c0, v);
-    if (a.out == OUT_ACT) {
-      put32_bf16(stg, v, (__nv_bfloat16 *)a.C + (int64_t)row0 * a.ldc + n, a.ldc, rows, ncols(n));
-    } else {
-      float *dst = (float *)a.C + (int64_t)row0 * a.ldc + n;
-      if (a.out == OUT_PARTIAL) dst += (int64_t)split * a.M * a.ldc;
-      float4 rv[8];
-      ld32_f32(add ? Rrow + n : nullptr, a.ldr, rows, ncols(n), rv);
-      put32_f32(stg, v, dst, a.ldc, rows, ncols(n), add ? Rrow + n : nullptr, a.ldr, rv);
     }
   }
 }
@@ -348,16 +241,19 @@ LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, uint32_t tm, i
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmC, const Args a) {
+              const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
+              const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t *bars = (uint64_t *)(smem + STAGES * STAGE_BYTES + STAGING_BYTES);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, rbar[EPI_WARPS]
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * STAGES;
   const uint32_t tfull0 = empty0 + 8 * STAGES, tempty0 = tfull0 + 16, drain = tempty0 + 16;
+  const uint32_t rbar0 = drain + 8;  // residual-load barrier of each epilogue warp
+  static_assert(8 * (2 * STAGES + 5 + EPI_WARPS) <= 256, "barrier space");
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -370,6 +266,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(tempty0 + 8 * b, EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int w = 0; w < EPI_WARPS; w++) mbar_init(rbar0 + 8 * w, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -492,6 +389,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int c_lo = (ew / 4) * (BN / 2);
     float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES) + ew * STG_BUFS * 32 * 32;
     int sb = 0;  // next staging square of this warp
+    uint32_t rph = 0;  // phase of this warp's residual-load barrier
+    const uint32_t rbar = rbar0 + 8 * ew;
     int acc = 0;
     uint32_t aph = 0;
     for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
@@ -500,20 +399,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, &tmC, 0, row0, n0, c_lo, split, true, stg, sb);
+        epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, 0, row0, n0, c_lo, split, true, stg,
+                      sb);
         continue;
       }
       if (!warp_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag)) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, &tmC, tm, row0, n0, c_lo, split, false, stg, sb);
+      epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, tm, row0, n0, c_lo, split, false, stg,
+                    sb);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; aph ^= 1; }
     }
     // this warp's bulk stores have completed before the CTA may exit
-    if (a.tma_store && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     __syncwarp();
   }
   fence_before();
@@ -659,16 +560,16 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
                          : p->map(g.B, g.N, g.K, g.ldb, 64, 64, &tb));
   if (!ok) return false;
   if (out != OUT_PARTIAL) splits = 1;
-  // C leaves through bulk tensor stores except for the residual add, which
-  // reads R on the way out
-  CUtensorMap tcm;
+  // C leaves through bulk tensor stores; a residual R comes in through bulk
+  // tensor loads of the same 32 x 32 fp32 boxes
+  CUtensorMap tcm, trm;
   memset(&tcm, 0, sizeof(tcm));
-  const bool tma_store = out != OUT_ADD_F32;
-  if (tma_store && !p->map_out(C, g.N, g.M, ldc, max(1, splits), out == OUT_PARTIAL,
-                               out == OUT_ACT ? 2 : 4, &tcm))
+  memset(&trm, 0, sizeof(trm));
+  if (!p->map_out(C, g.N, g.M, ldc, max(1, splits), out == OUT_PARTIAL, out == OUT_ACT ? 2 : 4,
+                  &tcm))
     return false;
+  if (out == OUT_ADD_F32 && !p->map_out(R, g.N, g.M, ldr, 1, false, 4, &trm)) return false;
   Args a{};
-  a.tma_store = tma_store ? 1 : 0;
   a.M = g.M; a.N = g.N; a.K = g.K;
   a.tiles_m = (g.M + BM - 1) / BM;
   a.tiles_n = (g.N + BN - 1) / BN;
@@ -681,10 +582,10 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   a.flag = p->flag;
   int grid = min(a.total, p->num_sms);
   bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
-  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
-  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
-  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
-  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, a);
+  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
+  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
+  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
+  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
   count_launch();
   return true;
 }
