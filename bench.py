@@ -10,11 +10,16 @@ JSON line on rank 0.
 
 Our arm: W untimed steps, then K steps timed with CUDA events on the
 library's stream, bracketed by a barrier and a synchronize, max over ranks.
+The library runs on its own stream, where llm_step captures the step into a
+CUDA graph on its second call and replays it afterwards (the warm-up steps
+include the capture).
 With N > 1 GPUs every rank runs an independent replica on its own batch
 (weak scaling; no gradient exchange is part of the timed step).
 The roofline object is for the dominant kernel (the tcgen05 GEMM): its
-algorithmic FLOPs over the summed device time of its launches, both taken
-inside the timed region.  e2e repeats the timed loop through the same C ABI
+algorithmic FLOPs over the summed device time of its launches, taken with CUDA
+events around every GEMM launch over K more steps run right after the timed
+region as individual launches (events cannot time nodes of a replayed graph;
+the kernels are the same).  e2e repeats the timed loop through the same C ABI
 with the step's tokens and targets copied from pinned host memory each step
 and the loss read back each step.  cpu_baseline times the float64 CPU oracle
 on a bounded sample of the same workload.
@@ -211,8 +216,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = get_config(args.config)
-    model = LlamaStep(cfg, device=dev)
-    stream = model.stream
+    # the library's own stream (not the legacy default stream), so llm_step
+    # runs as a replayed CUDA graph after its first two calls
+    stream = torch.cuda.Stream(device=dev)
+    model = LlamaStep(cfg, device=dev, stream=stream)
     p_host = make_params(cfg, model.layout, seed=1001 + cfg["index"] + 7919 * rank)
     tok_h, tgt_h = make_batch(cfg, seed=1000 + cfg["index"] + 7919 * rank)
     P = torch.tensor(p_host, device=dev)
@@ -229,15 +236,16 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    torch.cuda.synchronize()  # inputs written on the default stream are in place
     t = 0
+    # the warm-up steps (>= 3) run the step once as launches, then capture the
+    # step graph and replay it; the timed steps are replays
     for _ in range(args.warmup):
         t += 1
         model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
     st = model.status()
     assert st == 0, f"warm-up step failed with status {st}"
     launches_per_step = model.last_launch_count()
-    model.read_kernel_timing()  # clear
-    model.set_kernel_timing(True)
 
     clocks = Clocks(local_rank)
     barrier()
@@ -254,6 +262,13 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
+    # GEMM roofline: the same K steps again as individual launches, each
+    # tensor-core GEMM bracketed by CUDA events on the library's stream (the
+    # kernels are the ones the graph replays; events cannot time graph nodes)
+    model.set_kernel_timing(True)
+    for _ in range(args.steps):
+        t += 1
+        model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
     g_ms, g_flops, g_launch = model.read_kernel_timing()
     model.set_kernel_timing(False)
     st = model.status()
@@ -275,6 +290,15 @@ def run_ours(args, rank, world, local_rank):
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
+            # two untimed steps: the step graph without timing events is
+            # captured here, outside the timed loop
+            for _ in range(2):
+                t += 1
+                tok.copy_(tok_pin, non_blocking=True)
+                tgt.copy_(tgt_pin, non_blocking=True)
+                model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+                loss_pin.copy_(loss, non_blocking=True)
+                stream.synchronize()
             f0.record(stream)
             for _ in range(args.steps):
                 t += 1

@@ -137,8 +137,21 @@ int llm_status(llm_ctx *ctx);
 /* A static, human-readable string for a return code. */
 const char *llm_error_string(int code);
 
-/* Number of kernels the most recent llm_step / llm_forward call enqueued. */
+/* Number of kernels the most recent llm_step / llm_forward call enqueued
+ * (for a replayed step graph: its kernel nodes plus the scalar write). */
 int llm_last_launch_count(const llm_ctx *ctx);
+
+/* Step graphs (default on).  llm_step writes the step's scalars (lr, wd and
+ * the AdamW bias corrections of t) to device memory with one small kernel,
+ * then runs the step body.  The second llm_step call in a row with the same
+ * buffers (params, grads, m, v, tokens, targets, loss) captures the body
+ * into a CUDA graph on the context's stream and launches it; later calls with
+ * those buffers replay the graph (the buffers' contents may change freely
+ * between calls).  No graph is used on the legacy default stream (stream 0),
+ * while kernel timing is on (llm_set_kernel_timing), or after a capture
+ * failed (the context then runs every step as individual launches).  enable = 0 turns replay off (and frees
+ * the graph after synchronising the stream); enable = 1 turns it back on. */
+int llm_set_graphs(llm_ctx *ctx, int enable);
 
 /* Measurement hooks (strata, bench harness: time what is claimed).  With
  * timing enabled, every tensor-core GEMM launch of later calls is bracketed
@@ -147,7 +160,8 @@ int llm_last_launch_count(const llm_ctx *ctx);
  * device time of those launches in milliseconds, their algorithmic FLOPs
  * (2*M*N*K with unpadded sizes) and their count, then resets the sums.
  * Events are created on demand (two per pending launch) and kept until
- * llm_destroy(); reading after every few steps bounds their number. */
+ * llm_destroy(); reading after every few steps bounds their number.  Steps
+ * run as individual launches while timing is on (no step graph). */
 int llm_set_kernel_timing(llm_ctx *ctx, int enable);
 int llm_read_kernel_timing(llm_ctx *ctx, double *ms, double *flops, int64_t *launches);
 

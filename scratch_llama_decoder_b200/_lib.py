@@ -49,6 +49,7 @@ EXPORTS = {
     "llm_error_string": (C.c_char_p, [_i]),
     "llm_last_launch_count": (_i, [_vp]),
     "llm_set_kernel_timing": (_i, [_vp, _i]),
+    "llm_set_graphs": (_i, [_vp, _i]),
     "llm_read_kernel_timing": (_i, [_vp, C.POINTER(C.c_double), C.POINTER(C.c_double),
                                     C.POINTER(_i64)]),
     # include/llm_kernels.h

@@ -60,8 +60,10 @@ void cross_entropy(void *logits, DType dt, const int32_t *tgt, float *rowloss, i
 void loss_reduce(const float *rowloss, int64_t N, float *loss, int *flag, cudaStream_t s);
 void logits_out(const void *logits, DType dt, float *out, int64_t N, int V, int64_t ldz,
                 cudaStream_t s);
-void adamw(float *p, const float *g, float *m, float *v, int64_t n, float lr, float wd, float b1,
-           float b2, float eps, float bc1, float bc2, const int *flag, cudaStream_t s);
+// hyper: device [lr, wd, bc1, bc2], written by set_hyper.
+void set_hyper(float *hyper, float lr, float wd, float bc1, float bc2, cudaStream_t s);
+void adamw(float *p, const float *g, float *m, float *v, int64_t n, const float *hyper, float b1,
+           float b2, float eps, const int *flag, cudaStream_t s);
 // grad[r, c] (unpadded rows x cols) = sum over splits of part[s][r'][c'].
 //   mode 0: identity; mode 1: W13 de-interleave (cols = 2h, part cols 2hp)
 void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp, float *grad,

@@ -739,11 +739,24 @@ void logits_out(const void *logits, DType dt, float *out, int64_t N, int V, int6
 // and bias-corrected).  m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
 // p -= lr wd p + lr (m/bc1) / (sqrt(v/bc2) + eps), bc = 1 - beta^t.
 // The flat buffers hold every tensor back to back, so one launch covers all.
-// Skipped entirely when the step's flag is non-zero.
+// Skipped entirely when the step's flag is non-zero.  The per-step scalars
+// (lr, wd, bc1, bc2) are read from device memory, written by k_set_hyper
+// before the step, so a captured step graph replays with new values.
+__global__ void k_set_hyper(float *hyper, float lr, float wd, float bc1, float bc2) {
+  hyper[0] = lr;
+  hyper[1] = wd;
+  hyper[2] = bc1;
+  hyper[3] = bc2;
+}
+void set_hyper(float *hyper, float lr, float wd, float bc1, float bc2, cudaStream_t s) {
+  k_set_hyper<<<1, 1, 0, s>>>(hyper, lr, wd, bc1, bc2);
+  count_launch();
+}
 __global__ void k_adamw(float *__restrict__ p, const float *__restrict__ g, float *__restrict__ m,
-                        float *__restrict__ v, int64_t n, float lr, float wd, float b1, float b2,
-                        float eps, float bc1, float bc2, const int *flag) {
+                        float *__restrict__ v, int64_t n, const float *__restrict__ hyper,
+                        float b1, float b2, float eps, const int *flag) {
   if (*flag) return;
+  const float lr = hyper[0], wd = hyper[1], bc1 = hyper[2], bc2 = hyper[3];
   int64_t n4 = n / 4;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -771,10 +784,10 @@ __global__ void k_adamw(float *__restrict__ p, const float *__restrict__ g, floa
     p[i] = p[i] - lr * wd * p[i] - lr * (mi / bc1) / (sqrtf(vi / bc2) + eps);
   }
 }
-void adamw(float *p, const float *g, float *m, float *v, int64_t n, float lr, float wd, float b1,
-           float b2, float eps, float bc1, float bc2, const int *flag, cudaStream_t s) {
+void adamw(float *p, const float *g, float *m, float *v, int64_t n, const float *hyper, float b1,
+           float b2, float eps, const int *flag, cudaStream_t s) {
   unsigned grid = min(cdiv(n / 4 + 1, 256), 148u * 8);
-  k_adamw<<<grid, 256, 0, s>>>(p, g, m, v, n, lr, wd, b1, b2, eps, bc1, bc2, flag);
+  k_adamw<<<grid, 256, 0, s>>>(p, g, m, v, n, hyper, b1, b2, eps, flag);
   count_launch();
 }
 

@@ -135,12 +135,27 @@ struct llm_ctx {
   void *dxA, *du, *dab, *dO, *dqkv;
   int32_t *sort_scratch;
   TcPlan *tc = nullptr;
+  float *hyper;  // device [lr, wd, bc1, bc2] of the current step
   // optional event timing of the tensor-core GEMM launches
   bool timing = false;
   std::vector<cudaEvent_t> ev_pool;
   size_t ev_used = 0;
   double pending_flops = 0.0;
   int64_t pending_launches = 0;
+  // step graph: captured on the second llm_step with the same buffers,
+  // replayed afterwards; steps with kernel timing on run as launches
+  bool graphs = true;  // replay allowed (off after any capture failure)
+  cudaGraphExec_t gexec = nullptr;
+  struct Key {
+    const void *p[7];
+    bool operator==(const Key &o) const {
+      for (int i = 0; i < 7; i++)
+        if (p[i] != o.p[i]) return false;
+      return true;
+    }
+  } gkey{}, prev_key{};
+  bool have_prev = false;
+  int graph_launches = 0;  // kernels per replay
   int64_t carve(char *base);
 };
 
@@ -150,6 +165,7 @@ int64_t llm_ctx::carve(char *base) {
   int64_t N = D_.N, d = D_.d, L = D_.L, ab = D_.ab;
   flag_step = (int *)c.take(64);
   flag_sticky = (int *)c.take(64);
+  hyper = (float *)c.take(64);
   cos_t = (float *)c.take(4 * (int64_t)D_.T * (D_.hd / 2));
   sin_t = (float *)c.take(4 * (int64_t)D_.T * (D_.hd / 2));
   w_qkv = c.take(ab * L * d * D_.qkvw);
@@ -265,6 +281,7 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
 
 void llm_destroy(llm_ctx *c) {
   if (!c) return;
+  if (c->gexec) cudaGraphExecDestroy(c->gexec);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   tc_plan_destroy(c->tc);
   delete c;
@@ -288,6 +305,18 @@ int llm_last_launch_count(const llm_ctx *c) { return c ? c->last_launches : 0; }
 int llm_set_kernel_timing(llm_ctx *c, int enable) {
   if (!c) return LLM_ERR_ARG;
   c->timing = enable != 0;
+  return LLM_OK;
+}
+
+int llm_set_graphs(llm_ctx *c, int enable) {
+  if (!c) return LLM_ERR_ARG;
+  c->graphs = enable != 0;
+  if (!c->graphs && c->gexec) {
+    if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+    cudaGraphExecDestroy(c->gexec);
+    c->gexec = nullptr;
+  }
+  c->have_prev = false;
   return LLM_OK;
 }
 
@@ -513,17 +542,60 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
     return LLM_ERR_ARG;
   const Dims &D = c->D;
   g_launches = 0;
-  set_flag_zero(c->flag_step, c->s);
-  forward(c, d_params, d_tokens);
-  cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
-                c->flag_step, c->s);
-  loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
-  backward(c, d_params, d_grads, d_tokens);
-  double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
-  double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
-  adamw(d_params, d_grads, d_m, d_v, D.P, lr, wd, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps,
-        (float)bc1, (float)bc2, c->flag_step, c->s);
-  or_flag(c->flag_step, c->flag_sticky, c->s);
+  // the step's scalars go to device memory first (outside any graph)
+  const double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
+  const double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
+  set_hyper(c->hyper, lr, wd, (float)bc1, (float)bc2, c->s);
+  auto body = [&]() {
+    set_flag_zero(c->flag_step, c->s);
+    forward(c, d_params, d_tokens);
+    cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
+                  c->flag_step, c->s);
+    loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
+    backward(c, d_params, d_grads, d_tokens);
+    adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2,
+          c->cfg.adam_eps, c->flag_step, c->s);
+    or_flag(c->flag_step, c->flag_sticky, c->s);
+  };
+  const llm_ctx::Key key{{d_params, d_grads, d_m, d_v, d_tokens, d_targets, d_loss}};
+  // graphs need a capturable stream (not the legacy default stream); steps
+  // with kernel timing on run as individual launches
+  if (c->graphs && !c->timing && c->s != nullptr) {
+    if (c->gexec && key == c->gkey) {
+      if (cudaGraphLaunch(c->gexec, c->s) != cudaSuccess) return LLM_ERR_CUDA;
+      c->last_launches = 1 + c->graph_launches;
+      return LLM_OK;
+    }
+    if (c->have_prev && key == c->prev_key) {
+      // second call with these buffers: capture the step, then replay it
+      const int before = g_launches;
+      cudaGraph_t graph = nullptr;
+      bool ok = cudaStreamBeginCapture(c->s, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+      if (ok) {
+        body();
+        ok = cudaStreamEndCapture(c->s, &graph) == cudaSuccess && graph;
+      }
+      cudaGraphExec_t exec = nullptr;
+      if (ok) ok = cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+      if (graph) cudaGraphDestroy(graph);
+      if (ok) {
+        if (c->gexec) cudaGraphExecDestroy(c->gexec);
+        c->gexec = exec;
+        c->gkey = key;
+        c->graph_launches = g_launches - before;
+        if (cudaGraphLaunch(c->gexec, c->s) != cudaSuccess) return LLM_ERR_CUDA;
+        c->last_launches = 1 + c->graph_launches;
+        return LLM_OK;
+      }
+      // the capture did not work out: no more graphs for this context
+      (void)cudaGetLastError();
+      c->graphs = false;
+      g_launches = before;
+    }
+  }
+  c->prev_key = key;
+  c->have_prev = true;
+  body();
   c->last_launches = g_launches;
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }

@@ -80,6 +80,10 @@ class LlamaStep:
     def set_kernel_timing(self, enable):
         L.check(L.lib.llm_set_kernel_timing(self.ctx, int(bool(enable))), "llm_set_kernel_timing")
 
+    def set_graphs(self, enable):
+        """Step graphs on/off (llm_set_graphs)."""
+        L.check(L.lib.llm_set_graphs(self.ctx, int(bool(enable))), "llm_set_graphs")
+
     def read_kernel_timing(self):
         """(device ms, algorithmic FLOPs, launches) of the timed GEMM launches."""
         ms, fl, n = C.c_double(0), C.c_double(0), C.c_int64(0)

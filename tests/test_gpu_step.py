@@ -170,3 +170,54 @@ def test_init_statistics(name):
     P3 = m.new_params()
     m.init(P3, 99, cfg["init_std"], cfg["scale_out_proj"])
     assert torch.equal(P, P2) and not torch.equal(P, P3)
+
+
+def test_step_graph_replay_matches_individual_launches():
+    """On a non-default stream llm_step captures the step into a CUDA graph on
+    its second call with the same buffers and replays it afterwards.  Five
+    steps (step 4 with another token buffer: launched individually, then the
+    graph of the first buffers is captured anew) give bit-identical losses,
+    parameters, gradients and moments with graphs on and off, with the same
+    launch count; with kernel timing on every step runs as launches, so the
+    timed GEMM FLOPs and counts agree."""
+    from scratch_llama_decoder_b200 import LlamaStep
+    cfg = get_config("c3", batch=2, ctx=128, n_layer=2)
+    lay, p, tok, tgt = _inputs(cfg)
+
+    def run(graphs, timing=False):
+        s = torch.cuda.Stream()
+        m = LlamaStep(cfg, stream=s)
+        m.set_graphs(graphs)
+        m.set_kernel_timing(timing)
+        P = torch.tensor(p, device="cuda")
+        G, M, V = (torch.zeros_like(P) for _ in range(3))
+        td = torch.tensor(tok, dtype=torch.int32, device="cuda")
+        td2 = td.flip(1).contiguous()
+        yd = torch.tensor(tgt, dtype=torch.int32, device="cuda")
+        loss = torch.zeros(1, device="cuda")
+        torch.cuda.synchronize()
+        losses, counts = [], []
+        for t in range(1, 6):
+            m.step(P, G, M, V, t, td2 if t == 4 else td, yd, cfg["lr"], cfg["wd"], loss)
+            s.synchronize()
+            losses.append(float(loss.item()))
+            counts.append(m.last_launch_count())
+        st = m.status()
+        timing_read = m.read_kernel_timing() if timing else None
+        out = (losses, counts, st, P.cpu(), G.cpu(), M.cpu(), V.cpu(), timing_read)
+        m.close()
+        return out
+
+    a = run(True)
+    b = run(False)
+    assert a[2] == 0 and b[2] == 0
+    assert a[0] == b[0], (a[0], b[0])
+    assert a[1] == b[1], (a[1], b[1])
+    for x, y in zip(a[3:7], b[3:7]):
+        assert torch.equal(x, y)
+    # timing: the same GEMM FLOPs per step whether launched or replayed
+    ga = run(True, timing=True)[7]
+    gb = run(False, timing=True)[7]
+    assert ga[2] == gb[2] and abs(ga[1] - gb[1]) <= 1e-6 * gb[1], (ga, gb)
+    assert ga[0] > 0 and gb[0] > 0
+
