@@ -45,8 +45,8 @@ METRIC = "training tokens/sec (fwd+bwd+AdamW) on 1 B200; % of tensor/HBM rooflin
 # DRAM bytes (read + write) per tcgen05 GEMM launch, averaged over the 243
 # GEMM launches of one 350M step (profiles/gemm_dram_traffic_step_350m.md);
 # valid only for the GEMM sources that were captured, identified by hash.
-GEMM_TRAFFIC = {"bytes_per_launch": 256.5e6, "workload": "350m-v32000-d1024-l20-bf16",
-                "sha256": {"gemm_tc.cu": "fbee4d44c173eecd28aa7a64d76c1578fc5bb65d6cd8fac68e5415f3f4d5fde9",
+GEMM_TRAFFIC = {"bytes_per_launch": 256.7e6, "workload": "350m-v32000-d1024-l20-bf16",
+                "sha256": {"gemm_tc.cu": "9838f30d7c2ce88eb8d140bce74b03db53dc827e2a0c68d7882854c62a1ca37d",
                            "tcgen05.cuh": "062e7fbd85e8e8eb829ae9081c3849a887fdfcfea2721b394d186b20100514a8"}}
 
 
@@ -132,6 +132,20 @@ class Clocks:
                  "-i", str(self.idx), "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+
+    def wait_first(self, timeout_s=5.0):
+        """Return once the sampler has written its first line (or on time-out),
+        so that a short timed region still gets samples."""
+        if not self.proc:
+            return
+        t0 = time.time()
+        while time.time() - t0 < timeout_s:
+            try:
+                if os.path.getsize(self.out.name) > 0:
+                    return
+            except OSError:
+                pass
+            time.sleep(0.02)
 
     def stop(self):
         if not self.proc:
@@ -251,6 +265,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     clocks.start()
+    clocks.wait_first()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -260,7 +275,6 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     # GEMM roofline: the same K steps again as individual launches, each
     # tensor-core GEMM bracketed by CUDA events on the library's stream (the
@@ -271,6 +285,8 @@ def run_ours(args, rank, world, local_rank):
         model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
     g_ms, g_flops, g_launch = model.read_kernel_timing()
     model.set_kernel_timing(False)
+    # clocks sampled over the timed region and the GEMM-timing pass after it
+    clk = clocks.stop()
     st = model.status()
     assert st == 0, f"timed step failed with status {st}"
     final_loss = float(loss.item())
