@@ -119,6 +119,10 @@ struct llm_ctx {
   llm_config cfg;
   Dims D;
   cudaStream_t s;
+  // weight-gradient GEMMs run on a side stream s2 (forked from / joined to s
+  // with events); cur is the stream the GEMM launchers use
+  cudaStream_t s2 = nullptr, cur = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   int last_launches = 0;
   bool use_tc = false;
   // device buffers (all inside the caller's workspace)
@@ -265,6 +269,14 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
   c->cfg = *cfg;
   c->D = make_dims(cfg);
   c->s = (cudaStream_t)cuda_stream;
+  c->cur = c->s;
+  if (cudaStreamCreateWithFlags(&c->s2, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    // no side stream: every launch stays on the caller's stream
+    (void)cudaGetLastError();
+    c->s2 = nullptr;
+  }
   int64_t need = c->carve(nullptr);
   if (ws_bytes < need) { delete c; return LLM_ERR_ARG; }
   c->carve((char *)d_workspace);
@@ -281,6 +293,12 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
 
 void llm_destroy(llm_ctx *c) {
   if (!c) return;
+  if (c->s2) {
+    cudaStreamSynchronize(c->s2);
+    cudaStreamDestroy(c->s2);
+  }
+  if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+  if (c->ev_join) cudaEventDestroy(c->ev_join);
   if (c->gexec) cudaGraphExecDestroy(c->gexec);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   tc_plan_destroy(c->tc);
@@ -374,12 +392,12 @@ bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
     if (c->ev_pool.size() >= c->ev_used + 2) {
       e0 = c->ev_pool[c->ev_used];
       e1 = c->ev_pool[c->ev_used + 1];
-      cudaEventRecord(e0, c->s);
+      cudaEventRecord(e0, c->cur);
     }
   }
-  bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->s);
+  bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->cur);
   if (e0) {
-    cudaEventRecord(e1, c->s);
+    cudaEventRecord(e1, c->cur);
     if (ok) {
       c->ev_used += 2;
       c->pending_flops += alg_flops;
@@ -394,7 +412,7 @@ bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
 void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
           int64_t ldr, int splits, double alg_flops) {
   if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, alg_flops)) return;
-  gemm_simt(g, out, C, ldc, R, ldr, splits, c->s);
+  gemm_simt(g, out, C, ldc, R, ldr, splits, c->cur);
 }
 
 // Forward pass; leaves logits (padded, activation type) in c->logits.
@@ -461,7 +479,31 @@ void wgrad(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, 
   int splits = wgrad_splits(D, M, Ncols);
   GemmOperands g{(int)M, (int)Ncols, (int)D.N, X, ldx, false, dY, ldy, false, D.dt};
   gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits, 2.0 * rows * cols * D.N);
-  wgrad_finish(c->part, splits, M, Ncols, grad, rows, cols, mode, D.h, c->s);
+  wgrad_finish(c->part, splits, M, Ncols, grad, rows, cols, mode, D.h, c->cur);
+}
+
+// The weight gradients only read saved activations and a dY buffer, and only
+// AdamW reads them, so they run on the side stream: forked after the main
+// stream has produced their dY, joined back before the main stream
+// overwrites that dY (the RMSNorm backwards) and at the end of the backward.
+// They all share the split-K partial buffer, so the side stream runs them in
+// order.  With kernel timing on everything stays on the main stream.
+bool side_on(const llm_ctx *c) { return c->s2 && !c->timing; }
+void fork_side(llm_ctx *c) {
+  if (!side_on(c)) return;
+  cudaEventRecord(c->ev_fork, c->s);
+  cudaStreamWaitEvent(c->s2, c->ev_fork, 0);
+}
+void join_side(llm_ctx *c) {
+  if (!side_on(c)) return;
+  cudaEventRecord(c->ev_join, c->s2);
+  cudaStreamWaitEvent(c->s, c->ev_join, 0);
+}
+void wgrad_side(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, int64_t M,
+                int64_t Ncols, float *grad, int64_t rows, int64_t cols, int mode) {
+  c->cur = side_on(c) ? c->s2 : c->s;
+  wgrad(c, X, ldx, dY, ldy, M, Ncols, grad, rows, cols, mode);
+  c->cur = c->s;
 }
 
 void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
@@ -476,9 +518,10 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
   void *dxact = lp ? c->dxA : nullptr;
   int nb;
   // lm_head: dxf = dz Wlm^T; dWlm = xf^T dz
+  fork_side(c);  // dz (logits) and xf are ready
+  wgrad_side(c, c->xf, d, c->logits, D.Vp, d, D.Vp, gr + O.wlm(), d, D.V, 0);
   gemm(c, GemmOperands{(int)N, D.d, (int)D.Vp, c->logits, D.Vp, true, c->w_lm, D.Vp, true, D.dt},
        OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.V * d);
-  wgrad(c, c->xf, d, c->logits, D.Vp, d, D.Vp, gr + O.wlm(), d, D.V, 0);
   float *xL = c->xs + D.L * N * d;
   nb = rmsnorm_bwd(xL, c->rstdf, p + O.gf(), c->dtmp, nullptr, c->dx, dxact, D.dt, c->dgpart, N,
                    D.d, s);
@@ -491,32 +534,38 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
     void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
     void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
     // FFN branch.  du = dx2 W2^T, then SwiGLU backward into dab.
+    fork_side(c);  // dx2 is ready
+    wgrad_side(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
     gemm(c, GemmOperands{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt}, OUT_ACT, c->du,
          D.hp, nullptr, 0, 1, 2.0 * N * d * D.h);
     swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
-    wgrad(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
+    fork_side(c);  // dab is ready
+    wgrad_side(c, xn2, d, c->dab, 2 * D.hp, d, 2 * D.hp, gr + O.w13(l), d, 2LL * D.h, 1);
     gemm(c, GemmOperands{(int)N, D.d, (int)(2 * D.hp), c->dab, 2 * D.hp, true, w13, 2 * D.hp,
                          true, D.dt},
          OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * 2 * D.h * d);
-    wgrad(c, xn2, d, c->dab, 2 * D.hp, d, 2 * D.hp, gr + O.w13(l), d, 2LL * D.h, 1);
+    join_side(c);  // the RMSNorm backward overwrites dx2 (dxA)
     nb = rmsnorm_bwd(x1, rstd2, p + O.g2(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
                      D.d, s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
     // attention branch
     gemm(c, GemmOperands{(int)N, D.d, D.d, dxop, d, true, wo, d, true, D.dt}, OUT_ACT, c->dO, d,
          nullptr, 0, 1, 2.0 * N * d * d);
-    wgrad(c, o, d, dxop, d, d, d, gr + O.wo(l), d, d, 0);
     attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
                   c->cos_t, c->sin_t, s);
+    fork_side(c);  // dx1 and dqkv are ready (after the attention, so no TMEM contention)
+    wgrad_side(c, o, d, dxop, d, d, d, gr + O.wo(l), d, d, 0);
+    wgrad_side(c, xn1, d, c->dqkv, D.qkvw, d, D.qkvw, gr + O.wqkv(l), d, D.qkvw, 0);
     gemm(c, GemmOperands{(int)N, D.d, (int)D.qkvw, c->dqkv, D.qkvw, true, wqkv, D.qkvw, true,
                          D.dt},
          OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.qkvw * d);
-    wgrad(c, xn1, d, c->dqkv, D.qkvw, d, D.qkvw, gr + O.wqkv(l), d, D.qkvw, 0);
+    join_side(c);  // the RMSNorm backward overwrites dx1 (dxA); the next layer dqkv
     nb = rmsnorm_bwd(x, rstd1, p + O.g1(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N, D.d,
                      s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g1(l), s);
   }
   embed_bwd(tok, c->dx, gr, N, D.d, D.V, c->sort_scratch, s);
+  join_side(c);  // every weight gradient is in place before AdamW
 }
 
 }  // namespace
