@@ -219,6 +219,25 @@ def sample_tokens_for(cfg, budget_s):
     return S
 
 
+# ------------------------------------------------------------ rank helpers
+def max_over_ranks(x, world, device=None):
+    """The largest of a per-rank value over all ranks (all_reduce MAX on
+    `device`: the GPU under NCCL, the CPU under gloo); x itself at world 1."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_step, steps, world, ms):
+    """Whole-job throughput: the units all ranks processed over the time the
+    slowest rank took (ms, already the max over ranks)."""
+    return units_per_step * steps * world / (ms / 1e3)
+
+
 # --------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import numpy as np
@@ -290,10 +309,7 @@ def run_ours(args, rank, world, local_rank):
     st = model.status()
     assert st == 0, f"timed step failed with status {st}"
     final_loss = float(loss.item())
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
 
     # ---- e2e: same API, host buffers, copies inside the timed region
     e2e = None
@@ -327,11 +343,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         ems = f0.elapsed_time(f1)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        e2e = {"value": N * args.steps * world / (ems / 1e3), "unit": "tokens/s",
+        ems = max_over_ranks(ems, world, dev)
+        e2e = {"value": job_rate(N, args.steps, world, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(tok_pin.numel() * 4 + tgt_pin.numel() * 4),
                "d2h_bytes_per_step": 4}
 
@@ -340,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
     pk, src = peaks()
     F, F_attn = step_flops(cfg)
     step_s = ms / 1e3 / args.steps
-    value = N * args.steps * world / (ms / 1e3)
+    value = job_rate(N, args.steps, world, ms)
     peak_tc = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     achieved = (g_flops / (g_ms / 1e3)) / 1e12 if g_ms > 0 else 0.0
     out = {
