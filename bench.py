@@ -401,7 +401,10 @@ def run_reference(args, rank):
     N = cfg["batch"] * cfg["ctx"]
     return {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tsec * 1e3,
+        # a step of this arm is a bounded sample (S tokens); ms_per_step is the
+        # full step's time at the sampled rate, sample_ms the sample's own time
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": N / rate * 1e3,
+        "sample_ms": tsec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": cfg["name"], "tokens_per_step": N, "batch": cfg["batch"],
