@@ -446,9 +446,11 @@ def test_gradcheck_gqa_small():
 # ------------------------------------------------- PyTorch float64 autograd
 
 
-def torch_model_loss(cfg, p, tok, tgt):
+def torch_model_loss(cfg, p, tok, tgt, pairing="half"):
     """Independent forward in PyTorch float64 (library ops: rms_norm, SDPA with
-    GQA, silu, cross_entropy); RoPE is the rotate-half rotation."""
+    GQA, silu, cross_entropy).  RoPE pairs dimension j with j + hd/2
+    (rotate-half, the default) or 2j with 2j + 1 (pairing="interleaved"); pair
+    j turns by t * base^(-2j/hd) either way."""
     V, d, L, H, Hkv, h = (cfg[k] for k in ("vocab", "d_model", "n_layer", "n_head", "n_kv_head",
                                            "d_ff"))
     T, B = cfg["ctx"], cfg["batch"]
@@ -463,6 +465,9 @@ def torch_model_loss(cfg, p, tok, tgt):
     cos, sin = torch.cos(ang), torch.sin(ang)
 
     def rot(u):  # u [B, n, T, hd]
+        if pairing == "interleaved":
+            a, b = u[..., 0::2], u[..., 1::2]
+            return torch.stack([a * cos - b * sin, b * cos + a * sin], -1).flatten(-2)
         a, b = u[..., :hd // 2], u[..., hd // 2:]
         return torch.cat([a * cos - b * sin, b * cos + a * sin], -1)
 
@@ -511,6 +516,45 @@ def test_full_step_vs_torch_autograd_and_adamw(cfgname):
     st = opt.state[P_t]
     np.testing.assert_allclose(M_o, st["exp_avg"].numpy(), rtol=1e-12, atol=1e-18)
     np.testing.assert_allclose(V_o, st["exp_avg_sq"].numpy(), rtol=1e-12, atol=1e-20)
+
+
+def test_rope_pairings_differ_by_a_column_permutation():
+    """The pages pair RoPE dimensions two ways (rotate-half on the Llama page,
+    even-odd pairs on the CodeGen page).  The oracle takes rotate-half; the
+    reading rests on the two being the same model up to one fixed permutation
+    of each head's q and k columns of Wqkv: rotate-half slot j takes
+    interleaved dimension 2j, slot j + hd/2 takes 2j + 1."""
+    cfg = GQA_SMALL
+    lay, p, tok, tgt = _setup(cfg, std=0.3)
+    d, H, Hkv, L = cfg["d_model"], cfg["n_head"], cfg["n_kv_head"], cfg["n_layer"]
+    hd = d // H
+    perm = np.concatenate([np.arange(0, hd, 2), np.arange(1, hd, 2)])
+    cols = np.arange(d + 2 * Hkv * hd)
+    for h in range(H + Hkv):  # q heads, then k heads; v columns keep their place
+        cols[h * hd:(h + 1) * hd] = h * hd + perm
+    pp = p.copy()
+    spans = {n: (o, r, k) for n, o, r, k in lay}
+    for l in range(L):
+        o, r, k = spans[f"l{l}.Wqkv"]
+        pp[o:o + r * k] = p[o:o + r * k].reshape(r, k)[:, cols].reshape(-1)
+    loss_h, z_h, g_h = O.forward_backward(cfg, pp, tok, tgt)
+    pt = torch.tensor(p, requires_grad=True)
+    lt, zt = torch_model_loss(cfg, pt, tok, tgt, pairing="interleaved")
+    lt.backward()
+    assert abs(loss_h - lt.item()) <= 1e-12
+    np.testing.assert_allclose(z_h, zt.detach().numpy(), rtol=1e-10, atol=1e-12)
+    # gradients: the oracle's, with the columns moved back, are the interleaved model's
+    g_back = g_h.copy()
+    for l in range(L):
+        o, r, k = spans[f"l{l}.Wqkv"]
+        blk = np.empty((r, k))
+        blk[:, cols] = g_h[o:o + r * k].reshape(r, k)
+        g_back[o:o + r * k] = blk.reshape(-1)
+    gt = pt.grad.numpy()
+    assert np.linalg.norm(g_back - gt) / np.linalg.norm(gt) <= 1e-10
+    # without the permutation the two pairings are different models
+    loss_plain, _, _ = O.forward_backward(cfg, p, tok, tgt)
+    assert abs(loss_plain - lt.item()) > 1e-6
 
 
 # ------------------------------------------------------------------- AdamW
