@@ -24,6 +24,16 @@ with the step's tokens and targets copied from pinned host memory each step
 and the loss read back each step.  cpu_baseline times the float64 CPU oracle
 on a bounded sample of the same workload.
 
+Decode (--decode): generation throughput of the same workload's model with a
+key/value cache: a forward over the whole context (the prefill), then K timed
+llm_decode steps at positions --pos, --pos + 1, ... (each step one new position
+for every sequence, the weights and every cached key/value row up to it read
+once); value = sequences x K / time.  Its roofline is HBM bytes per step
+(bf16 weights, K/V rows read, K/V row and logits written) over the step's time
+against the measured copy bandwidth; e2e adds top-k sampling with the
+token ids and uniforms copied from pinned host memory and the sampled ids read
+back every step; cpu_baseline is the float64 oracle decoding one sequence.
+
 Reference arm (--impl reference): the float64 CPU oracle, each step a fixed
 fraction of the workload (a token prefix of one sequence, forward and
 backward, plus AdamW over the same fraction of the parameters), scaled to
@@ -85,6 +95,9 @@ def parse():
                     help="attention forward kernels: 2 tcgen05, 1 mma, 0 CUDA cores")
     ap.add_argument("--bwd-impl", type=int, default=2, choices=[0, 1, 2],
                     help="attention backward kernels: 2 tcgen05, 1 mma, 0 CUDA cores")
+    ap.add_argument("--decode", action="store_true",
+                    help="time llm_decode (KV-cache generation) instead of the training step")
+    ap.add_argument("--pos", type=int, default=1024, help="first decoded position (--decode)")
     ap.add_argument("--orient", default="kn", choices=["kn", "kk", "nn"],
                     help="gemm operand majorness: kn = x.W (forward), kk = dy.W^T (dgrad), "
                          "nn = x^T.dy (wgrad)")
@@ -390,6 +403,165 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+def decode_bytes(cfg, pos):
+    """HBM bytes of one decode step at position pos: the unpadded bf16 weight
+    matrices, the float32 embedding rows and RMSNorm gains, every cached key
+    and value row 0..pos (read) and the new row (written), the q row, and the
+    float32 logits (written)."""
+    V, d, L, H, Hkv, h, B = (cfg[k] for k in ("vocab", "d_model", "n_layer", "n_head",
+                                              "n_kv_head", "d_ff", "batch"))
+    hd = d // H
+    kvd = Hkv * hd
+    esz = 2 if cfg["compute"] == "bf16" else 4
+    weights = (L * (d * (d + 2 * kvd) + d * d + 2 * d * h + h * d) + d * V) * esz
+    small = B * d * 4 + (2 * L + 1) * d * 4
+    kv = L * B * ((pos + 1) * 2 * kvd + (d + 2 * kvd)) * esz
+    return weights + small + kv + B * V * 4, weights, kv
+
+
+def oracle_decode_rate(cfg, budget_s=10.0):
+    """The float64 oracle decoding one sequence from position 0 for about
+    budget_s seconds; returns (tokens/s, seconds, cores, positions)."""
+    import numpy as np
+    import oracle as O
+    from oracle import decode as OD
+    from synth import make_batch, make_params
+    c1 = dict(cfg, batch=1)
+    p = make_params(cfg, O.param_layout(cfg)).astype(np.float64)
+    tok, _ = make_batch(cfg)
+    cache = OD.KVCache(c1)
+    n, t0 = 0, time.time()
+    while n < cfg["ctx"] and (time.time() - t0 < budget_s or n < 2):
+        OD.decode_step(c1, p, cache, tok[0, n:n + 1], n)
+        n += 1
+    dt = time.time() - t0
+    return n / dt, dt, os.cpu_count(), n
+
+
+def run_decode(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    from scratch_llama_decoder_b200 import LlamaStep
+    from synth import get_config, make_batch, make_params
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = get_config(args.config)
+    B, T, V = cfg["batch"], cfg["ctx"], cfg["vocab"]
+    if args.pos + args.warmup + args.steps > T:
+        raise SystemExit(f"--pos + --warmup + --steps must be <= ctx ({T})")
+    stream = torch.cuda.Stream(device=dev)
+    model = LlamaStep(cfg, device=dev, stream=stream)
+    p_host = make_params(cfg, model.layout, seed=1001 + cfg["index"] + 7919 * rank)
+    tok_h, _ = make_batch(cfg, seed=1000 + cfg["index"] + 7919 * rank)
+    tok_h = tok_h.reshape(B, T)
+    P = torch.tensor(p_host, device=dev)
+    tok_all = torch.tensor(tok_h, device=dev)
+    cols = torch.tensor(np.ascontiguousarray(tok_h.T), device=dev)  # [T, B]: row t = ids at t
+    tk = torch.empty(B, dtype=torch.int32, device=dev)
+    lg = torch.empty(B, V, device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        model.forward(P, tok_all)  # prefill: every position's keys and values
+        pos = args.pos
+        for _ in range(args.warmup):  # the second call captures the decode graph
+            tk.copy_(cols[pos])
+            model.decode(P, tk, pos, logits=lg)
+            pos += 1
+    st = model.status()
+    assert st == 0, f"warm-up decode failed with status {st}"
+    launches = model.last_launch_count()
+    first = pos
+    clocks = Clocks(local_rank)
+    torch.cuda.synchronize()
+    clocks.start()
+    clocks.wait_first()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            tk.copy_(cols[pos])
+            model.decode(P, tk, pos, logits=lg)
+            pos += 1
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    st = model.status()
+    assert st == 0, f"timed decode failed with status {st}"
+    byt = [decode_bytes(cfg, q) for q in range(first, pos)]
+    alg = sum(b[0] for b in byt) / args.steps
+
+    # e2e: ids and uniforms from pinned host memory, decode + top-k sampling,
+    # sampled ids back to the host every step
+    e2e = None
+    if not args.no_e2e:
+        ids_pin = torch.tensor(tok_h[:, 0]).pin_memory()
+        uni_pin = torch.rand(B).pin_memory()
+        out_pin = torch.zeros(B, dtype=torch.int32).pin_memory()
+        ud = torch.empty(B, device=dev)
+        od = torch.empty(B, dtype=torch.int32, device=dev)
+        with torch.cuda.stream(stream):
+            model.forward(P, tok_all)
+            q = args.pos
+            for _ in range(2):  # untimed: graph capture for these buffers
+                tk.copy_(ids_pin, non_blocking=True)
+                model.decode(P, tk, q, logits=lg)
+                q += 1
+            stream.synchronize()
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            n_e2e = min(args.steps, T - q)
+            f0.record(stream)
+            for _ in range(n_e2e):
+                tk.copy_(ids_pin, non_blocking=True)
+                ud.copy_(uni_pin, non_blocking=True)
+                model.decode(P, tk, q, logits=lg)
+                model.sample(lg, 0.8, 40, ud, out=od)
+                out_pin.copy_(od, non_blocking=True)
+                stream.synchronize()
+                ids_pin.copy_(out_pin)  # the sampled ids are the next step's input
+                q += 1
+            f1.record(stream)
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        e2e = {"value": B * n_e2e / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 8 * B,
+               "d2h_bytes_per_step": 4 * B, "sampling": "temperature 0.8, top-k 40"}
+        assert model.status() == 0
+    if rank != 0:
+        return None
+    pk, src = peaks()
+    peak = pk.get("hbm_gbs")
+    gbs = alg / (ms / 1e3 / args.steps) / 1e9
+    out = {
+        "metric": "decode tokens/sec (KV cache, one position per sequence per step) on 1 B200; "
+                  "% of HBM roofline",
+        "value": job_rate(B, args.steps, world, ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg["compute"] == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": cfg["name"], "batch": B, "ctx": T,
+                   "positions": [first, pos - 1],
+                   "l2": "weights and cache (> 1 GB per step) larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "kernel": "decode step (all kernels)", "achieved": gbs,
+                     "peak": peak, "unit": "GB/s", "frac": gbs / peak if peak else None,
+                     "traffic": None, "bytes_per_step": alg,
+                     "weight_bytes": byt[0][1], "kv_bytes_first": byt[0][2],
+                     "peak_source": f"{src} hbm_gbs"},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, secs, cores, n = oracle_decode_rate(cfg)
+        out["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle",
+                               "sample": f"float64 oracle decoding positions 0..{n - 1} of one "
+                                         f"sequence ({secs:.1f} s)"}
+    return out
+
+
 def run_reference(args, rank):
     if rank != 0:
         return None
@@ -511,7 +683,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = (run_decode if args.decode else run_ours)(args, rank, world, local_rank)
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:

@@ -129,6 +129,48 @@ int llm_step(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d
              const int32_t *d_tokens, const int32_t *d_targets, float lr, float wd,
              float *d_loss);
 
+/* Single-token decode against a key/value cache (Hephaistos, feature list:
+ * "True KV Cache", the prompt is processed once and every later position
+ * costs one pass over a single row per sequence; strata, model table: the
+ * cache holds keys already rotated by RoPE, and decoding position by position
+ * gives the full forward's logits).
+ *
+ * The cache is the context's own saved q|k|v activations: llm_forward (or
+ * llm_step) over d_tokens [batch, ctx] fills positions 0..ctx-1 of every
+ * sequence; that forward over a prompt in positions 0..p-1 is the prefill
+ * (positions >= p may hold any ids: causality keeps them out of positions
+ * < p).  llm_decode then runs position pos for every sequence: d_tokens
+ * [batch] holds each sequence's id at pos, the call writes that position's
+ * rotated keys and values into the cache (so decoding pos, pos+1, ... in
+ * order extends the sequences), and d_logits (float32 [batch, vocab]) gets
+ * the logits of position pos, which attend to cached positions 0..pos.
+ * d_params must be the parameters of that forward: the embedding and the
+ * RMSNorm gains are read from it, the matrices from the low-precision copies
+ * the forward made.  Requires 0 <= pos < ctx and head_dim dividing 128
+ * (LLM_ERR_ARG / LLM_ERR_CONFIG otherwise, nothing launched).  Out-of-range
+ * ids are clamped for the read and reported by llm_status() as
+ * LLM_ERR_TOKEN.  The position goes to device memory first, so the second call
+ * in a row with the same (d_params, d_tokens, d_logits) captures the decode
+ * body into a CUDA graph that later calls replay for any pos (graphs follow
+ * llm_set_graphs).  Results are bit-reproducible. */
+int llm_decode(llm_ctx *ctx, const float *d_params, const int32_t *d_tokens, int pos,
+               float *d_logits);
+
+/* Token sampling (Hephaistos, Sampling: temperature + top-k) for each of
+ * n_rows rows of d_logits (float32, row stride ld >= vocab of the context):
+ *   temperature <= 0 or top_k == 1: greedy, the largest logit (lowest id
+ *     among equal maxima);
+ *   otherwise the top-k set is the first top_k ids ordered by (logit
+ *     descending, id ascending) -- the whole vocabulary when top_k <= 0 or
+ *     top_k >= vocab -- with weights exp((z - max z) / temperature), and the
+ *     token is the smallest id of the set, in increasing id order, whose
+ *     cumulative weight exceeds u * (total weight), u = d_uniform[row]
+ *     clamped to [0, 1).
+ * The uniforms are inputs (device float32 [n_rows]); d_out gets int32
+ * [n_rows] ids.  One block per row; deterministic. */
+int llm_sample(llm_ctx *ctx, const float *d_logits, int64_t ld, int n_rows, float temperature,
+               int top_k, const float *d_uniform, int32_t *d_out);
+
 /* Synchronises the context's stream and returns the first error any call on
  * this context raised on the device since the previous llm_status() (then
  * clears it), or LLM_ERR_CUDA if the stream reports a CUDA error, else LLM_OK. */

@@ -45,6 +45,8 @@ EXPORTS = {
     "llm_init": (_i, [_vp, _u64, _f, _i, _vp]),
     "llm_forward": (_i, [_vp, _vp, _vp, _vp]),
     "llm_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _f, _f, _vp]),
+    "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
+    "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),
     "llm_status": (_i, [_vp]),
     "llm_error_string": (C.c_char_p, [_i]),
     "llm_last_launch_count": (_i, [_vp]),

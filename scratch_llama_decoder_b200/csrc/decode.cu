@@ -1,0 +1,605 @@
+// Single-token decode against the key/value cache, and the token sampler.
+//
+// Hephaistos, feature list ("True KV Cache"): the prompt is run once, then each
+// new position costs one pass of every projection over a single row per
+// sequence; strata, model table: the cached keys are stored already rotated.
+// The cache is the forward pass's own [B*T, q|k|v] activation buffer of every
+// layer (RoPE applied to q and k), so a forward over the prompt is the prefill
+// and a decode call writes row (b, pos) of it.
+//
+// With B rows per call the projections are matrix-vector products bound by
+// reading the weights once: k_gemv streams W in 128-column blocks split over
+// K (about four blocks per SM), each thread multiplying 8 columns of W by the
+// block's B rows held in shared memory, with the RMSNorm of the input row
+// applied while the rows are staged.  The K slices' partial sums are added in
+// slice order by the last block of a column block to finish (a counter per
+// column block), which then applies the epilogue: RoPE + cache store for the
+// q|k|v projection, residual add, SwiGLU, or the fp32 logits.  Attention of
+// the new query against positions 0..pos is split over 128-key chunks
+// (k_attn_decode) and the chunks are merged in order (k_attn_combine).
+// Every sum has a fixed order: a decode call is bit-reproducible.
+#include <limits.h>
+#include <math.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace llm {
+
+namespace {
+
+constexpr int GV_THREADS = 256;
+constexpr int GV_COLS = 128;     // columns of W per block
+constexpr int GV_CG = 16;        // column groups of 8 per block
+constexpr int GV_KL = 16;        // k lanes per block (GV_THREADS / GV_CG)
+constexpr int GV_MB = 8;         // rows of A per pass
+constexpr int GV_UNROLL = 4;     // W rows in flight per thread
+constexpr int GV_KSLICE_MAX = 1024;
+constexpr int GV_SMEM_FLOATS = GV_MB * GV_KSLICE_MAX;  // A slice, then the warp partials
+static_assert(GV_SMEM_FLOATS >= (GV_THREADS / 32) * GV_MB * GV_COLS, "reduction space");
+static_assert(GV_CG * GV_KL == GV_THREADS && 8 * GV_CG == GV_COLS, "thread layout");
+
+constexpr int AT_KEYS = 128;     // keys per attention block (one per thread when scoring)
+constexpr int AT_THREADS = 128;
+constexpr int AT_G = 8;          // query heads of a group per pass
+
+constexpr int SP_THREADS = 1024;
+
+inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
+
+LLM_DEV void bf16x8(uint4 q, float (&f)[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&q);
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const float2 t = __bfloat1622float2(h[k]);
+    f[2 * k] = t.x;
+    f[2 * k + 1] = t.y;
+  }
+}
+// 8 consecutive values from p; one or two 16-byte loads when vec (aligned
+// and all 8 inside the row), else element by element up to n.
+LLM_DEV void load8(const __nv_bfloat16 *p, bool vec, int n, float (&w)[8]) {
+  if (vec && n >= 8) {
+    bf16x8(__ldg(reinterpret_cast<const uint4 *>(p)), w);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; k++) w[k] = k < n ? __bfloat162float(p[k]) : 0.f;
+  }
+}
+LLM_DEV void load8(const float *p, bool vec, int n, float (&w)[8]) {
+  if (vec && n >= 8) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; k++) w[k] = k < n ? p[k] : 0.f;
+  }
+}
+
+// Epilogue of rows [b0, b0 + mb) x columns [n0, n0 + 128) whose sums are in
+// v[r * GV_COLS + c].
+template <typename A>
+LLM_DEV void gemv_epilogue(const GemvArgs &a, const float *v, int b0, int mb, int n0) {
+  for (int idx = threadIdx.x; idx < GV_MB * GV_COLS; idx += GV_THREADS) {
+    const int r = idx / GV_COLS, c = idx % GV_COLS, n = n0 + c;
+    if (r >= mb) continue;
+    const int64_t b = b0 + r;
+    const float y = v[idx];
+    if (a.epi == DEC_QKV) {
+      // Hephaistos, Architecture at a glance (Positions): q and k of head
+      // columns rotate pairs (j, j + hd/2) by pos * theta_j; heads do not
+      // straddle the block (hd divides 128).
+      if (n >= a.nvalid) continue;
+      const int t = *a.pos;
+      float o = y;
+      if (n < a.rot_cols) {
+        const int half = a.hd / 2, e = n % a.hd, j = e % half, cb = c - e;
+        const float cs = a.cos_t[(int64_t)t * half + j], sn = a.sin_t[(int64_t)t * half + j];
+        const float x0 = v[r * GV_COLS + cb + j], x1 = v[r * GV_COLS + cb + j + half];
+        o = e < half ? x0 * cs - x1 * sn : x1 * cs + x0 * sn;
+      }
+      reinterpret_cast<A *>(a.out)[b * a.ldo + (int64_t)t * a.pos_stride + n] = from_f<A>(o);
+    } else if (a.epi == DEC_RESID) {
+      if (n < a.nvalid) reinterpret_cast<float *>(a.out)[b * a.ldo + n] += y;
+    } else if (a.epi == DEC_SWIGLU) {
+      // interleaved W1|W3 blocks of 64 columns: a in the first half of the
+      // block, its b 64 columns further (Hephaistos, Architecture at a
+      // glance: u = silu(a) * b); a and b rounded like the saved activations
+      if (c >= SWIGLU_BLOCK) continue;
+      const int64_t j = (int64_t)(n0 / (2 * SWIGLU_BLOCK)) * SWIGLU_BLOCK + c;
+      if (j >= a.nvalid) continue;
+      const float av = to_f(from_f<A>(y)), bv = to_f(from_f<A>(v[idx + SWIGLU_BLOCK]));
+      reinterpret_cast<A *>(a.out)[b * a.ldo + j] = from_f<A>(av * sigmoidf_(av) * bv);
+    } else {  // DEC_LOGITS
+      if (n < a.nvalid) reinterpret_cast<float *>(a.out)[b * a.ldo + n] = y;
+    }
+  }
+}
+
+// y[b, n] = sum_k A[b, k] W[k, n] for B rows; grid (column blocks, K slices).
+template <typename A>
+__global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
+  __shared__ __align__(16) float sm[GV_SMEM_FLOATS];
+  __shared__ float rs[GV_MB];
+  __shared__ int last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = tid % GV_CG, kl = tid / GV_CG;
+  const int n0 = blockIdx.x * GV_COLS, ksi = blockIdx.y;
+  const int k0 = ksi * a.kslice, k1 = min(a.K, k0 + a.kslice), kn = k1 - k0;
+  const int nc = n0 + 8 * cg;
+  const int ncols = max(0, min(8, a.N - nc));
+  const A *W = reinterpret_cast<const A *>(a.W);
+  const bool vec = a.vec != 0;
+  for (int b0 = 0; b0 < a.B; b0 += GV_MB) {
+    const int mb = min(GV_MB, a.B - b0);
+    // ---- the rows' K slice in shared memory, in operand precision
+    if (a.gain) {
+      // Hephaistos, Architecture at a glance (Normalization): r = (mean x^2 +
+      // eps)^-1/2, A = g * x * r, over the whole row (K = d)
+      if (warp < mb) {
+        const float *xr = a.x + (int64_t)(b0 + warp) * a.ldx;
+        float ss = 0.f;
+        for (int j = lane; j < a.K; j += 32) ss += xr[j] * xr[j];
+        ss = warp_sum(ss);
+        if (lane == 0) rs[warp] = 1.0f / sqrtf(ss / (float)a.K + a.eps);
+      }
+      __syncthreads();
+    }
+    for (int i = tid; i < GV_MB * kn; i += GV_THREADS) {
+      const int r = i / kn, k = k0 + i % kn;
+      float v = 0.f;
+      if (r < mb) {
+        const int64_t row = b0 + r;
+        v = a.gain ? to_f(from_f<A>(a.gain[k] * a.x[row * a.ldx + k] * rs[r]))
+                   : to_f(reinterpret_cast<const A *>(a.xa)[row * a.ldxa + k]);
+      }
+      sm[i] = v;
+    }
+    __syncthreads();
+    // ---- products: this thread's 8 columns over rows k0 + kl, + 16, ...
+    float acc[GV_MB][8];
+#pragma unroll
+    for (int r = 0; r < GV_MB; r++)
+#pragma unroll
+      for (int j = 0; j < 8; j++) acc[r][j] = 0.f;
+    for (int k = k0 + kl; k < k1; k += GV_KL * GV_UNROLL) {
+      float w[GV_UNROLL][8];
+#pragma unroll
+      for (int u = 0; u < GV_UNROLL; u++) {
+        const int kk = k + u * GV_KL;
+        if (kk < k1 && ncols > 0) {
+          load8(W + (int64_t)kk * a.ldw + nc, vec, ncols, w[u]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; j++) w[u][j] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < GV_UNROLL; u++) {
+        const int kk = k + u * GV_KL;
+        if (kk < k1) {
+#pragma unroll
+          for (int r = 0; r < GV_MB; r++) {
+            const float xv = sm[r * kn + (kk - k0)];
+#pragma unroll
+            for (int j = 0; j < 8; j++) acc[r][j] = fmaf(xv, w[u][j], acc[r][j]);
+          }
+        }
+      }
+    }
+    __syncthreads();  // the A slice is no longer read: its space takes the partials
+    // ---- k lanes: the two of a warp by shuffle, then the 8 warps in order
+#pragma unroll
+    for (int r = 0; r < GV_MB; r++)
+#pragma unroll
+      for (int j = 0; j < 8; j++) acc[r][j] += __shfl_xor_sync(0xffffffffu, acc[r][j], 16);
+    if (lane < 16) {
+#pragma unroll
+      for (int r = 0; r < GV_MB; r++)
+#pragma unroll
+        for (int j = 0; j < 8; j++) sm[(warp * GV_MB + r) * GV_COLS + 8 * cg + j] = acc[r][j];
+    }
+    __syncthreads();
+    float fin[GV_MB * GV_COLS / GV_THREADS];
+#pragma unroll
+    for (int i = 0; i < GV_MB * GV_COLS / GV_THREADS; i++) {
+      const int idx = tid + GV_THREADS * i, r = idx / GV_COLS, c = idx % GV_COLS;
+      float s = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < GV_THREADS / 32; w8++) s += sm[(w8 * GV_MB + r) * GV_COLS + c];
+      fin[i] = s;
+    }
+    __syncthreads();
+    if (a.ks == 1) {
+#pragma unroll
+      for (int i = 0; i < GV_MB * GV_COLS / GV_THREADS; i++) sm[tid + GV_THREADS * i] = fin[i];
+      __syncthreads();
+      gemv_epilogue<A>(a, sm, b0, mb, n0);
+    } else {
+#pragma unroll
+      for (int i = 0; i < GV_MB * GV_COLS / GV_THREADS; i++) {
+        const int idx = tid + GV_THREADS * i, r = idx / GV_COLS, c = idx % GV_COLS;
+        if (r < mb && n0 + c < a.N)
+          a.part[((int64_t)ksi * a.B + b0 + r) * a.N + n0 + c] = fin[i];
+      }
+    }
+    __syncthreads();
+  }
+  if (a.ks == 1) return;
+  // ---- the last K slice of this column block to finish adds the partials
+  // in slice order and applies the epilogue
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(&a.count[blockIdx.x], 1u) == (unsigned)(a.ks - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int b0 = 0; b0 < a.B; b0 += GV_MB) {
+    const int mb = min(GV_MB, a.B - b0);
+    for (int idx = tid; idx < GV_MB * GV_COLS; idx += GV_THREADS) {
+      const int r = idx / GV_COLS, c = idx % GV_COLS;
+      float s = 0.f;
+      if (r < mb && n0 + c < a.N)
+        for (int q = 0; q < a.ks; q++)
+          s += __ldcg(a.part + ((int64_t)q * a.B + b0 + r) * a.N + n0 + c);
+      sm[idx] = s;
+    }
+    __syncthreads();
+    gemv_epilogue<A>(a, sm, b0, mb, n0);
+    __syncthreads();
+  }
+  if (tid == 0) a.count[blockIdx.x] = 0u;  // ready for the next launch
+}
+
+// ----------------------------------------------------------- attention
+// Hephaistos, Architecture at a glance (Attention): the query of position pos
+// attends to keys 0..pos with weights softmax(q.k / sqrt(hd)); strata: query
+// head h reads key/value head h / (H / H_kv).  Block (chunk c of 128 keys,
+// key/value head g, sequence b); the group's query heads in passes of 8.
+// Scores are kept in base 2 (q pre-scaled by log2(e) / sqrt(hd)).  Writes per
+// (b, g, chunk, head of group): chunk maximum m, sum l of 2^(s - m), and
+// o = sum 2^(s - m) v.
+template <typename A>
+__global__ void __launch_bounds__(AT_THREADS)
+    k_attn_decode(const A *__restrict__ qkv, int64_t qkvw, int T, const int *__restrict__ pos_p,
+                  int H, int Hkv, int hd, int nch, int vec, float *__restrict__ part) {
+  __shared__ float qs[AT_G][128];
+  __shared__ float ps[AT_G][AT_KEYS];
+  __shared__ float red[AT_G][AT_THREADS];
+  __shared__ float wm[AT_THREADS / 32][AT_G], wl[AT_THREADS / 32][AT_G];
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int pos = *pos_p;
+  const int j0 = c * AT_KEYS;
+  if (j0 > pos) return;
+  const int j1 = min(j0 + AT_KEYS, pos + 1);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = H / Hkv, d = H * hd, kvd = Hkv * hd;
+  const float scale = 1.4426950408889634f / sqrtf((float)hd);
+  const A *rowq = qkv + ((int64_t)b * T + pos) * qkvw;
+  const int j = j0 + tid;
+  const A *kr = qkv + ((int64_t)b * T + j) * qkvw + d + (int64_t)g * hd;
+  for (int r0 = 0; r0 < G; r0 += AT_G) {
+    const int nr = min(AT_G, G - r0);
+    for (int i = tid; i < AT_G * hd; i += AT_THREADS) {
+      const int r = i / hd, e = i % hd;
+      qs[r][e] = r < nr ? to_f(rowq[(int64_t)(g * G + r0 + r) * hd + e]) * scale : 0.f;
+    }
+    __syncthreads();
+    // scores: one key per thread
+    float s[AT_G];
+#pragma unroll
+    for (int r = 0; r < AT_G; r++) s[r] = 0.f;
+    if (j < j1) {
+      for (int e = 0; e < hd; e += 8) {
+        float kv[8];
+        load8(kr + e, vec != 0, hd - e, kv);
+#pragma unroll
+        for (int r = 0; r < AT_G; r++) {
+          float t = s[r];
+#pragma unroll
+          for (int q = 0; q < 8; q++)
+            if (e + q < hd) t = fmaf(qs[r][e + q], kv[q], t);
+          s[r] = t;
+        }
+      }
+    }
+    // chunk maximum and sum per query head (warps, then the 4 warps in order)
+#pragma unroll
+    for (int r = 0; r < AT_G; r++) {
+      const float m = warp_max(j < j1 ? s[r] : -INFINITY);
+      if (lane == 0) wm[warp][r] = m;
+    }
+    __syncthreads();
+    float p[AT_G];
+#pragma unroll
+    for (int r = 0; r < AT_G; r++) {
+      const float m = fmaxf(fmaxf(wm[0][r], wm[1][r]), fmaxf(wm[2][r], wm[3][r]));
+      p[r] = j < j1 ? exp2f(s[r] - m) : 0.f;
+      ps[r][tid] = p[r];
+      const float l = warp_sum(p[r]);
+      if (lane == 0) wl[warp][r] = l;
+    }
+    __syncthreads();
+    // o = sum_j p_j v_j: thread = (dimension e, key lane kq), hd divides 128
+    const int KL = AT_THREADS / hd, e = tid % hd, kq = tid / hd;
+    float o[AT_G];
+#pragma unroll
+    for (int r = 0; r < AT_G; r++) o[r] = 0.f;
+    const A *vb = qkv + (int64_t)b * T * qkvw + d + kvd + (int64_t)g * hd + e;
+    for (int jj = kq; jj < j1 - j0; jj += KL) {
+      const float v = to_f(vb[(int64_t)(j0 + jj) * qkvw]);
+#pragma unroll
+      for (int r = 0; r < AT_G; r++) o[r] = fmaf(ps[r][jj], v, o[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < AT_G; r++) red[r][tid] = o[r];
+    __syncthreads();
+    if (tid < hd) {
+      for (int r = 0; r < nr; r++) {
+        float acc = 0.f;
+        for (int q = 0; q < KL; q++) acc += red[r][q * hd + tid];
+        float *rec = part + ((((int64_t)b * Hkv + g) * nch + c) * G + r0 + r) * (hd + 2);
+        rec[2 + tid] = acc;
+        if (tid == 0) {
+          rec[0] = fmaxf(fmaxf(wm[0][r], wm[1][r]), fmaxf(wm[2][r], wm[3][r]));
+          rec[1] = ((wl[0][r] + wl[1][r]) + wl[2][r]) + wl[3][r];
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// o[b, h*hd + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c over the
+// chunks 0..pos/128 in order.  Block (query head, sequence).
+template <typename A>
+__global__ void k_attn_combine(const float *__restrict__ part, const int *__restrict__ pos_p, int H,
+                               int Hkv, int hd, int nch, A *__restrict__ out) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int G = H / Hkv, g = h / G, r = h % G;
+  const int nc = *pos_p / AT_KEYS + 1;
+  const int64_t stride = (int64_t)G * (hd + 2);
+  const float *rec0 = part + (((int64_t)b * Hkv + g) * nch * G + r) * (hd + 2);
+  float M = -INFINITY;
+  for (int c = 0; c < nc; c++) M = fmaxf(M, rec0[c * stride]);
+  for (int e = threadIdx.x; e < hd; e += blockDim.x) {
+    float L = 0.f, acc = 0.f;
+    for (int c = 0; c < nc; c++) {
+      const float *rc = rec0 + c * stride;
+      const float f = exp2f(rc[0] - M);
+      L = fmaf(f, rc[1], L);
+      acc = fmaf(f, rc[2 + e], acc);
+    }
+    out[(int64_t)b * H * hd + (int64_t)h * hd + e] = from_f<A>(acc / L);
+  }
+}
+
+// ------------------------------------------------------------- sampling
+// Hephaistos, Sampling (temperature + top-k).  Readings: temperature <= 0 or
+// top_k == 1 is greedy (lowest id among equal maxima); the top-k set is the
+// first k ids ordered by (logit descending, id ascending); weights
+// exp((z - max z) / temperature); the draw is the smallest id of the set, in
+// increasing id order, whose cumulative weight exceeds u * total.  One block
+// per row; thread t owns the contiguous ids [t*chunk, (t+1)*chunk).
+LLM_DEV uint32_t order_key(float f) {  // unsigned order = float order
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+LLM_DEV float sample_weight(float z, float zmax, float temperature) {
+  return expf((z - zmax) / temperature);
+}
+__global__ void __launch_bounds__(SP_THREADS)
+    k_sample(const float *__restrict__ logits, int64_t ld, int V, float temperature, int top_k,
+             const float *__restrict__ uni, int32_t *__restrict__ out) {
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned s_prefix, s_rem;
+  __shared__ unsigned eqc[SP_THREADS];
+  __shared__ float wsum[SP_THREADS];
+  __shared__ int s_owner;
+  __shared__ float s_tl;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float *z = logits + (int64_t)b * ld;
+  const int chunk = (V + SP_THREADS - 1) / SP_THREADS;
+  const int lo = min(V, tid * chunk), hi = min(V, lo + chunk);
+  // maximum and its lowest id
+  float bv = -INFINITY;
+  int bi = INT_MAX;
+  for (int i = lo; i < hi; i++) {
+    const float v = z[i];
+    if (bi == INT_MAX || v > bv) { bv = v; bi = i; }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  if (lane == 0) { sv[warp] = bv; si[warp] = bi; }
+  __syncthreads();
+  if (warp == 0) {
+    bv = sv[lane];
+    bi = si[lane];
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) { sv[0] = bv; si[0] = bi; }
+  }
+  __syncthreads();
+  const float zmax = sv[0];
+  if (!(temperature > 0.f) || top_k == 1 || V == 1) {
+    if (tid == 0) out[b] = si[0];
+    return;
+  }
+  // top-k cut: the k-th largest key by an 8-bit-digit radix select (most
+  // significant digit first); the set is every key above it plus the first
+  // `rem` ids holding it
+  const bool all = top_k <= 0 || top_k >= V;
+  uint32_t thr = 0u;
+  unsigned rem = 0u;
+  if (!all) {
+    uint32_t prefix = 0u, mask = 0u;
+    unsigned remaining = (unsigned)top_k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      if (tid < 256) hist[tid] = 0u;
+      __syncthreads();
+      for (int i = lo; i < hi; i++) {
+        const uint32_t k = order_key(z[i]);
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        unsigned cum = 0u;
+        int dsel = 0;
+        for (int dg = 255; dg >= 0; dg--) {
+          if (cum + hist[dg] >= remaining) { dsel = dg; break; }
+          cum += hist[dg];
+        }
+        s_prefix = prefix | ((uint32_t)dsel << shift);
+        s_rem = remaining - cum;
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      remaining = s_rem;
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+    thr = prefix;
+    rem = remaining;
+  }
+  // rank of this thread's first id among the ids holding the cut key
+  unsigned myeq = 0u;
+  if (!all)
+    for (int i = lo; i < hi; i++) myeq += order_key(z[i]) == thr;
+  eqc[tid] = myeq;
+  __syncthreads();
+  if (tid == 0) {
+    unsigned run = 0u;
+    for (int t = 0; t < SP_THREADS; t++) {
+      const unsigned n = eqc[t];
+      eqc[t] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  const unsigned eq0 = eqc[tid];
+  // this thread's weight, ids in increasing order
+  float my = 0.f;
+  {
+    unsigned eq = eq0;
+    for (int i = lo; i < hi; i++) {
+      bool in = all;
+      if (!all) {
+        const uint32_t k = order_key(z[i]);
+        in = k > thr || (k == thr && eq < rem);
+        eq += k == thr;
+      }
+      if (in) my += sample_weight(z[i], zmax, temperature);
+    }
+  }
+  wsum[tid] = my;
+  __syncthreads();
+  if (tid == 0) {
+    float W = 0.f;
+    for (int t = 0; t < SP_THREADS; t++) W += wsum[t];
+    const float u = fminf(fmaxf(uni[b], 0.f), 0.99999994f);
+    const float target = u * W;
+    float c = 0.f, tl = 0.f;
+    int owner = -1;
+    for (int t = 0; t < SP_THREADS; t++) {
+      const float cn = c + wsum[t];
+      if (wsum[t] > 0.f && target < cn) { owner = t; tl = target - c; break; }
+      c = cn;
+    }
+    if (owner < 0)  // rounding put the target past the end: the last weighted id
+      for (int t = SP_THREADS - 1; t >= 0; t--)
+        if (wsum[t] > 0.f) { owner = t; tl = wsum[t]; break; }
+    s_owner = owner;
+    s_tl = tl;
+  }
+  __syncthreads();
+  if (tid == s_owner) {
+    float c = 0.f;
+    int pick = -1, lastin = -1;
+    unsigned eq = eq0;
+    for (int i = lo; i < hi; i++) {
+      bool in = all;
+      if (!all) {
+        const uint32_t k = order_key(z[i]);
+        in = k > thr || (k == thr && eq < rem);
+        eq += k == thr;
+      }
+      if (!in) continue;
+      c += sample_weight(z[i], zmax, temperature);
+      lastin = i;
+      if (c > s_tl) { pick = i; break; }
+    }
+    out[b] = pick >= 0 ? pick : lastin;
+  }
+}
+
+__global__ void k_set_int(int *p, int v) { *p = v; }
+
+}  // namespace
+
+void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice) {
+  const int64_t cb = (N + GV_COLS - 1) / GV_COLS;
+  const int64_t want = std::max<int64_t>(1, (4 * 148 + cb - 1) / cb);  // ~4 blocks per SM
+  const int64_t ks_max = std::max<int64_t>(1, (K + 63) / 64);          // >= 64 rows a slice
+  const int64_t ks_min = (K + GV_KSLICE_MAX - 1) / GV_KSLICE_MAX;
+  int64_t s = std::max(std::min(want, ks_max), ks_min);
+  int64_t sl = (K + s - 1) / s;
+  sl = std::min<int64_t>(GV_KSLICE_MAX, (sl + 15) / 16 * 16);
+  *kslice = (int)sl;
+  *ks = (int)((K + sl - 1) / sl);
+}
+
+int gemv_col_blocks(int64_t N) { return (int)cdiv(N, GV_COLS); }
+
+void gemv(const GemvArgs &a, DType dt, cudaStream_t s) {
+  dim3 grid(cdiv(a.N, GV_COLS), a.ks);
+  if (dt == DT_BF16) k_gemv<__nv_bfloat16><<<grid, GV_THREADS, 0, s>>>(a);
+  else k_gemv<float><<<grid, GV_THREADS, 0, s>>>(a);
+  count_launch();
+}
+
+int attn_decode_chunks(int T) { return (int)cdiv(T, AT_KEYS); }
+
+void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, int H, int Hkv,
+                 int hd, float *part, void *o, DType dt, cudaStream_t s) {
+  const int nch = attn_decode_chunks(T), d = H * hd;
+  const int ve = dt == DT_BF16 ? 8 : 4;
+  const int vec = (hd % 8 == 0 && qkvw % ve == 0 && d % ve == 0) ? 1 : 0;
+  dim3 grid(nch, Hkv, B);
+  if (dt == DT_BF16) {
+    k_attn_decode<<<grid, AT_THREADS, 0, s>>>((const __nv_bfloat16 *)qkv, qkvw, T, pos, H, Hkv,
+                                             hd, nch, vec, part);
+    k_attn_combine<<<dim3(H, B), std::max(32, std::min(128, hd)), 0, s>>>(
+        part, pos, H, Hkv, hd, nch, (__nv_bfloat16 *)o);
+  } else {
+    k_attn_decode<<<grid, AT_THREADS, 0, s>>>((const float *)qkv, qkvw, T, pos, H, Hkv, hd, nch,
+                                             vec, part);
+    k_attn_combine<<<dim3(H, B), std::max(32, std::min(128, hd)), 0, s>>>(part, pos, H, Hkv, hd,
+                                                                         nch, (float *)o);
+  }
+  count_launch(2);
+}
+
+void sample_tokens(const float *logits, int64_t ld, int rows, int V, float temperature, int top_k,
+                   const float *uni, int32_t *out, cudaStream_t s) {
+  k_sample<<<rows, SP_THREADS, 0, s>>>(logits, ld, V, temperature, top_k, uni, out);
+  count_launch();
+}
+
+void set_device_int(int *p, int v, cudaStream_t s) {
+  k_set_int<<<1, 1, 0, s>>>(p, v);
+  count_launch();
+}
+
+}  // namespace llm

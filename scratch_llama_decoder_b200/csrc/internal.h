@@ -108,6 +108,56 @@ bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *
                  void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
                  const float *sin_t, int *flag, cudaStream_t s);
 
+// ------------------------------------------------------------------ decode
+// Matrix-vector products of a decode step: y[b, n] = sum_k A[b, k] W[k, n]
+// for B rows, W [K, ldw] in operand type.  A is either fp32 rows x [B, ldx]
+// normalised on the fly (gain non-null: A = round(g * x * rstd), RMSNorm over
+// the K = d entries of the row) or operand-type rows xa [B, ldxa].  The grid
+// splits K into ks slices of kslice rows (gemv_plan); partial sums go to
+// part [ks, B, N] and the last slice of each 128-column block to finish adds
+// them in slice order (count [column blocks], zero between launches).
+enum DecEpi {
+  DEC_QKV = 0,     // RoPE on columns < rot_cols at position *pos, store out[b*ldo + *pos*pos_stride + n] (n < nvalid)
+  DEC_RESID = 1,   // float out[b*ldo + n] += y (n < nvalid)
+  DEC_SWIGLU = 2,  // interleaved a|b columns -> out[b*ldo + j] = silu(a_j) b_j (j < nvalid)
+  DEC_LOGITS = 3   // float out[b*ldo + n] = y (n < nvalid)
+};
+struct GemvArgs {
+  int B, K, N;
+  const void *W;
+  int64_t ldw;
+  int vec;  // W rows may be read with 16-byte loads
+  const float *x;
+  int64_t ldx;
+  const float *gain;
+  float eps;
+  const void *xa;
+  int64_t ldxa;
+  int ks, kslice;
+  float *part;
+  unsigned *count;
+  int epi;
+  void *out;
+  int64_t ldo, pos_stride;
+  int nvalid;
+  const float *cos_t, *sin_t;
+  const int *pos;
+  int hd, rot_cols;
+};
+void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice);
+int gemv_col_blocks(int64_t N);
+void gemv(const GemvArgs &a, DType dt, cudaStream_t s);
+// Attention of the query at position *pos of every sequence against the
+// cached keys/values 0..*pos of qkv [B*T, qkvw] (one layer), o [B, H*hd];
+// part: B * H * attn_decode_chunks(T) * (hd + 2) floats.  Needs 128 % hd == 0.
+int attn_decode_chunks(int T);
+void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, int H, int Hkv,
+                 int hd, float *part, void *o, DType dt, cudaStream_t s);
+// One token id per row of logits [rows, ld] (V valid columns).
+void sample_tokens(const float *logits, int64_t ld, int rows, int V, float temperature, int top_k,
+                   const float *uni, int32_t *out, cudaStream_t s);
+void set_device_int(int *p, int v, cudaStream_t s);
+
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;
 inline void count_launch(int n = 1) { g_launches += n; }

@@ -160,6 +160,16 @@ struct llm_ctx {
   } gkey{}, prev_key{};
   bool have_prev = false;
   int graph_launches = 0;  // kernels per replay
+  // decode (llm_decode): per-call rows, split-K partials, attention chunk
+  // records, column-block counters, the position word, and its own graph
+  float *dec_x = nullptr, *dec_part = nullptr, *dec_attn = nullptr;
+  void *dec_o = nullptr, *dec_u = nullptr;
+  unsigned *dec_count = nullptr;
+  int *dec_pos = nullptr;
+  cudaGraphExec_t dexec = nullptr;
+  Key dkey{}, dprev_key{};
+  bool dhave_prev = false;
+  int dgraph_launches = 0;
   int64_t carve(char *base);
 };
 
@@ -208,6 +218,23 @@ int64_t llm_ctx::carve(char *base) {
   part = (float *)c.take(4 * part_elems);
   dgpart = (float *)c.take(4 * (int64_t)rmsnorm_bwd_blocks(N) * d);
   sort_scratch = (int32_t *)c.take(4 * embed_bwd_scratch_ints(N, D_.V));
+  // decode: the four matrix-vector shapes of a layer and the lm_head
+  const int64_t B = D_.B;
+  int64_t dpart = 0, dblocks = 0;
+  auto dneed = [&](int64_t K, int64_t Nc) {
+    int ks, sl;
+    gemv_plan(K, Nc, &ks, &sl);
+    if (ks > 1) dpart = std::max<int64_t>(dpart, (int64_t)ks * B * Nc);
+    dblocks = std::max<int64_t>(dblocks, gemv_col_blocks(Nc));
+  };
+  dneed(d, D_.qkvw); dneed(d, d); dneed(d, 2 * D_.hp); dneed(D_.hp, d); dneed(d, D_.Vp);
+  dec_x = (float *)c.take(4 * B * d);
+  dec_o = c.take(ab * B * d);
+  dec_u = c.take(ab * B * D_.hp);
+  dec_part = (float *)c.take(4 * std::max<int64_t>(1, dpart));
+  dec_attn = (float *)c.take(4 * B * D_.H * attn_decode_chunks(D_.T) * (int64_t)(D_.hd + 2));
+  dec_count = (unsigned *)c.take(4 * dblocks);
+  dec_pos = (int *)c.take(64);
   return round_up(c.off, 256);
 }
 
@@ -283,6 +310,11 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
   g_launches = 0;
   cudaMemsetAsync(c->flag_step, 0, 64, c->s);
   cudaMemsetAsync(c->flag_sticky, 0, 64, c->s);
+  cudaMemsetAsync(c->dec_count, 0, 4 * (size_t)gemv_col_blocks(std::max<int64_t>(
+                                           std::max<int64_t>(c->D.qkvw, 2 * c->D.hp),
+                                           std::max<int64_t>(c->D.d, c->D.Vp))),
+                  c->s);
+  cudaMemsetAsync(c->dec_pos, 0, 64, c->s);
   rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, cfg->rope_base, c->s);
   c->tc = tc_plan_create(c->D.dt, c->cos_t, c->sin_t, c->D.T, c->D.hd, c->D.d + c->D.kvd, c->D.hp);
   tc_plan_set_flag(c->tc, c->flag_step);
@@ -300,6 +332,7 @@ void llm_destroy(llm_ctx *c) {
   if (c->ev_fork) cudaEventDestroy(c->ev_fork);
   if (c->ev_join) cudaEventDestroy(c->ev_join);
   if (c->gexec) cudaGraphExecDestroy(c->gexec);
+  if (c->dexec) cudaGraphExecDestroy(c->dexec);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
   tc_plan_destroy(c->tc);
   delete c;
@@ -329,12 +362,15 @@ int llm_set_kernel_timing(llm_ctx *c, int enable) {
 int llm_set_graphs(llm_ctx *c, int enable) {
   if (!c) return LLM_ERR_ARG;
   c->graphs = enable != 0;
-  if (!c->graphs && c->gexec) {
+  if (!c->graphs && (c->gexec || c->dexec)) {
     if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
-    cudaGraphExecDestroy(c->gexec);
+    if (c->gexec) cudaGraphExecDestroy(c->gexec);
+    if (c->dexec) cudaGraphExecDestroy(c->dexec);
     c->gexec = nullptr;
+    c->dexec = nullptr;
   }
   c->have_prev = false;
+  c->dhave_prev = false;
   return LLM_OK;
 }
 
@@ -568,6 +604,70 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
   join_side(c);  // every weight gradient is in place before AdamW
 }
 
+// One decode position for every sequence (position in c->dec_pos): the
+// layers of the forward on one row per sequence, reading keys and values of
+// positions 0..pos from the saved q|k|v activations and writing position
+// pos's row of them.  Logits go to logits [B, V] (float32).
+void decode_body(llm_ctx *c, const float *p, const int32_t *tok, float *logits) {
+  const Dims &D = c->D;
+  POff O{D};
+  cudaStream_t s = c->s;
+  const int64_t N = D.N, d = D.d;
+  const int ab = D.ab, esz_vec = 16 / ab;
+  auto A = [&](void *base, int64_t l, int64_t per) { return (char *)base + l * per * ab; };
+  auto mv = [&](int64_t K, int64_t Ncols, const void *W, int64_t ldw, int epi, void *out,
+                int64_t ldo, int nvalid) {
+    GemvArgs a{};
+    a.B = D.B;
+    a.K = (int)K;
+    a.N = (int)Ncols;
+    a.W = W;
+    a.ldw = ldw;
+    a.vec = (ldw % esz_vec == 0 && ((uintptr_t)W & 15) == 0) ? 1 : 0;
+    a.eps = c->cfg.rms_eps;
+    gemv_plan(K, Ncols, &a.ks, &a.kslice);
+    a.part = c->dec_part;
+    a.count = c->dec_count;
+    a.epi = epi;
+    a.out = out;
+    a.ldo = ldo;
+    a.nvalid = nvalid;
+    a.cos_t = c->cos_t;
+    a.sin_t = c->sin_t;
+    a.pos = c->dec_pos;
+    a.hd = D.hd;
+    a.rot_cols = D.d + D.kvd;
+    return a;
+  };
+  embed_fwd(p, tok, c->dec_x, D.B, D.d, D.V, c->flag_step, s);
+  for (int l = 0; l < D.L; l++) {
+    void *qkv = A(c->qkv, l, N * D.qkvw);
+    // q|k|v of position pos (RMSNorm g1 on the fly, RoPE on q and k) into
+    // row (b, pos) of the layer's saved activations
+    GemvArgs a = mv(d, D.qkvw, A(c->w_qkv, l, d * D.qkvw), D.qkvw, DEC_QKV, qkv,
+                    (int64_t)D.T * D.qkvw, (int)D.qkvw);
+    a.x = c->dec_x; a.ldx = d; a.gain = p + O.g1(l); a.pos_stride = D.qkvw;
+    gemv(a, D.dt, s);
+    attn_decode(qkv, D.qkvw, D.B, D.T, c->dec_pos, D.H, D.Hkv, D.hd, c->dec_attn, c->dec_o, D.dt,
+                s);
+    // x += o Wo
+    a = mv(d, d, A(c->w_o, l, d * d), d, DEC_RESID, c->dec_x, d, D.d);
+    a.xa = c->dec_o; a.ldxa = d;
+    gemv(a, D.dt, s);
+    // u = SwiGLU(RMSNorm_g2(x) W13); x += u W2
+    a = mv(d, 2 * D.hp, A(c->w_13, l, d * 2 * D.hp), 2 * D.hp, DEC_SWIGLU, c->dec_u, D.hp,
+           (int)D.hp);
+    a.x = c->dec_x; a.ldx = d; a.gain = p + O.g2(l);
+    gemv(a, D.dt, s);
+    a = mv(D.hp, d, A(c->w_2, l, D.hp * d), d, DEC_RESID, c->dec_x, d, D.d);
+    a.xa = c->dec_u; a.ldxa = D.hp;
+    gemv(a, D.dt, s);
+  }
+  GemvArgs a = mv(d, D.Vp, c->w_lm, D.Vp, DEC_LOGITS, logits, D.V, D.V);
+  a.x = c->dec_x; a.ldx = d; a.gain = p + O.gf();
+  gemv(a, D.dt, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -645,6 +745,70 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
   c->prev_key = key;
   c->have_prev = true;
   body();
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_decode(llm_ctx *c, const float *d_params, const int32_t *d_tokens, int pos,
+               float *d_logits) {
+  if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;
+  const Dims &D = c->D;
+  if (pos < 0 || pos >= D.T) return LLM_ERR_ARG;
+  if (128 % D.hd) return LLM_ERR_CONFIG;
+  if (((uintptr_t)d_params & 3) || ((uintptr_t)d_tokens & 3) || ((uintptr_t)d_logits & 3))
+    return LLM_ERR_ARG;
+  g_launches = 0;
+  set_device_int(c->dec_pos, pos, c->s);  // outside any graph
+  const int before = g_launches;
+  auto body = [&]() {
+    set_flag_zero(c->flag_step, c->s);
+    decode_body(c, d_params, d_tokens, d_logits);
+    or_flag(c->flag_step, c->flag_sticky, c->s);
+  };
+  const llm_ctx::Key key{{d_params, d_tokens, d_logits, nullptr, nullptr, nullptr, nullptr}};
+  if (c->graphs && c->s != nullptr) {
+    if (c->dexec && key == c->dkey) {
+      if (cudaGraphLaunch(c->dexec, c->s) != cudaSuccess) return LLM_ERR_CUDA;
+      c->last_launches = before + c->dgraph_launches;
+      return LLM_OK;
+    }
+    if (c->dhave_prev && key == c->dprev_key) {
+      cudaGraph_t graph = nullptr;
+      bool ok = cudaStreamBeginCapture(c->s, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+      if (ok) {
+        body();
+        ok = cudaStreamEndCapture(c->s, &graph) == cudaSuccess && graph;
+      }
+      cudaGraphExec_t exec = nullptr;
+      if (ok) ok = cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+      if (graph) cudaGraphDestroy(graph);
+      if (ok) {
+        if (c->dexec) cudaGraphExecDestroy(c->dexec);
+        c->dexec = exec;
+        c->dkey = key;
+        c->dgraph_launches = g_launches - before;
+        if (cudaGraphLaunch(c->dexec, c->s) != cudaSuccess) return LLM_ERR_CUDA;
+        c->last_launches = before + c->dgraph_launches;
+        return LLM_OK;
+      }
+      (void)cudaGetLastError();
+      c->graphs = false;
+      g_launches = before;
+    }
+  }
+  c->dprev_key = key;
+  c->dhave_prev = true;
+  body();
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_sample(llm_ctx *c, const float *d_logits, int64_t ld, int n_rows, float temperature,
+               int top_k, const float *d_uniform, int32_t *d_out) {
+  if (!c || !d_logits || !d_uniform || !d_out || n_rows < 1 || ld < c->D.V) return LLM_ERR_ARG;
+  if (!(temperature == temperature)) return LLM_ERR_ARG;  // NaN
+  g_launches = 0;
+  sample_tokens(d_logits, ld, n_rows, c->D.V, temperature, top_k, d_uniform, d_out, c->s);
   c->last_launches = g_launches;
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }

@@ -71,6 +71,25 @@ class LlamaStep:
                 "llm_step")
         return loss
 
+    def decode(self, params, tokens, pos, logits=None):
+        """Logits [B, V] of position pos (llm_decode); tokens: int32 [B]."""
+        B, V = self.cfg["batch"], self.cfg["vocab"]
+        if logits is None:
+            logits = torch.empty(B, V, dtype=torch.float32, device=self.device)
+        L.check(L.lib.llm_decode(self.ctx, _ptr(params), _ptr(tokens), int(pos), _ptr(logits)),
+                "llm_decode")
+        return logits
+
+    def sample(self, logits, temperature, top_k, uniforms, out=None):
+        """int32 token ids [rows] from float32 logits [rows, ld] (llm_sample)."""
+        rows = logits.shape[0]
+        if out is None:
+            out = torch.empty(rows, dtype=torch.int32, device=self.device)
+        L.check(L.lib.llm_sample(self.ctx, _ptr(logits), logits.stride(0), rows,
+                                 float(temperature), int(top_k), _ptr(uniforms), _ptr(out)),
+                "llm_sample")
+        return out
+
     def status(self):
         return L.lib.llm_status(self.ctx)
 
