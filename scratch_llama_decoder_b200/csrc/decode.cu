@@ -9,14 +9,14 @@
 //
 // With B rows per call the projections are matrix-vector products bound by
 // reading the weights once: k_gemv streams W in 128-column blocks split over
-// K (about four blocks per SM), each thread multiplying 8 columns of W by the
+// K (one wave of two blocks per SM), each thread multiplying 8 columns of W by the
 // block's B rows held in shared memory, with the RMSNorm of the input row
 // applied while the rows are staged.  The K slices' partial sums are added in
 // slice order by the last block of a column block to finish (a counter per
 // column block), which then applies the epilogue: RoPE + cache store for the
 // q|k|v projection, residual add, SwiGLU, or the fp32 logits.  Attention of
-// the new query against positions 0..pos is split over 128-key chunks
-// (k_attn_decode) and the chunks are merged in order (k_attn_combine).
+// the new query against positions 0..pos is split over 128-key chunks; the
+// last chunk of a (sequence, key/value head) to finish merges them in order.
 // Every sum has a fixed order: a decode call is bit-reproducible.
 #include <limits.h>
 #include <math.h>
@@ -37,6 +37,7 @@ constexpr int GV_KL = 16;        // k lanes per block (GV_THREADS / GV_CG)
 constexpr int GV_MB = 8;         // rows of A per pass
 constexpr int GV_UNROLL = 4;     // W rows in flight per thread
 constexpr int GV_KSLICE_MAX = 1024;
+constexpr int GV_KS_MAX = 16;    // K slices (partials the finishing block adds)
 constexpr int GV_SMEM_FLOATS = GV_MB * GV_KSLICE_MAX;  // A slice, then the warp partials
 static_assert(GV_SMEM_FLOATS >= (GV_THREADS / 32) * GV_MB * GV_COLS, "reduction space");
 static_assert(GV_CG * GV_KL == GV_THREADS && 8 * GV_CG == GV_COLS, "thread layout");
@@ -48,6 +49,14 @@ constexpr int AT_G = 8;          // query heads of a group per pass
 constexpr int SP_THREADS = 1024;
 
 inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
+
+// Programmatic dependent launch: the next kernel of the stream may be
+// scheduled once every block of this one has passed pdl_release(); it runs
+// its independent prologue (weight loads) and then pdl_wait() blocks until
+// this grid has completed and its writes are visible.  Without the launch
+// attribute both are no-ops.
+LLM_DEV void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+LLM_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 LLM_DEV void bf16x8(uint4 q, float (&f)[8]) {
   const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&q);
@@ -134,21 +143,45 @@ __global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
   const int ncols = max(0, min(8, a.N - nc));
   const A *W = reinterpret_cast<const A *>(a.W);
   const bool vec = a.vec != 0;
+  float w[GV_UNROLL][8];
+  auto load_w = [&](int k) {
+#pragma unroll
+    for (int u = 0; u < GV_UNROLL; u++) {
+      const int kk = k + u * GV_KL;
+      if (kk < k1 && ncols > 0) {
+        load8(W + (int64_t)kk * a.ldw + nc, vec, ncols, w[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; j++) w[u][j] = 0.f;
+      }
+    }
+  };
+  pdl_release();
+  // the weights are never written by the kernels before this one: the first
+  // batch of this thread's rows is in flight before waiting for them
+  load_w(k0 + kl);
+  pdl_wait();
   for (int b0 = 0; b0 < a.B; b0 += GV_MB) {
     const int mb = min(GV_MB, a.B - b0);
     // ---- the rows' K slice in shared memory, in operand precision
     if (a.gain) {
       // Hephaistos, Architecture at a glance (Normalization): r = (mean x^2 +
       // eps)^-1/2, A = g * x * r, over the whole row (K = d)
+      // (x rows are 16-byte aligned and K = d is a multiple of 4)
       if (warp < mb) {
-        const float *xr = a.x + (int64_t)(b0 + warp) * a.ldx;
+        const float4 *xr = reinterpret_cast<const float4 *>(a.x + (int64_t)(b0 + warp) * a.ldx);
         float ss = 0.f;
-        for (int j = lane; j < a.K; j += 32) ss += xr[j] * xr[j];
+#pragma unroll 8
+        for (int j = lane; j < a.K / 4; j += 32) {
+          const float4 v = xr[j];
+          ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        }
         ss = warp_sum(ss);
         if (lane == 0) rs[warp] = 1.0f / sqrtf(ss / (float)a.K + a.eps);
       }
       __syncthreads();
     }
+#pragma unroll 4
     for (int i = tid; i < GV_MB * kn; i += GV_THREADS) {
       const int r = i / kn, k = k0 + i % kn;
       float v = 0.f;
@@ -167,17 +200,7 @@ __global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
 #pragma unroll
       for (int j = 0; j < 8; j++) acc[r][j] = 0.f;
     for (int k = k0 + kl; k < k1; k += GV_KL * GV_UNROLL) {
-      float w[GV_UNROLL][8];
-#pragma unroll
-      for (int u = 0; u < GV_UNROLL; u++) {
-        const int kk = k + u * GV_KL;
-        if (kk < k1 && ncols > 0) {
-          load8(W + (int64_t)kk * a.ldw + nc, vec, ncols, w[u]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; j++) w[u][j] = 0.f;
-        }
-      }
+      if (b0 > 0 || k > k0 + kl) load_w(k);  // the first batch was loaded up front
 #pragma unroll
       for (int u = 0; u < GV_UNROLL; u++) {
         const int kk = k + u * GV_KL;
@@ -238,16 +261,36 @@ __global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
   __syncthreads();
   if (!last) return;
   __threadfence();
+  constexpr int PER = GV_MB * GV_COLS / GV_THREADS;
+  const int64_t qstride = (int64_t)a.B * a.N;
   for (int b0 = 0; b0 < a.B; b0 += GV_MB) {
     const int mb = min(GV_MB, a.B - b0);
-    for (int idx = tid; idx < GV_MB * GV_COLS; idx += GV_THREADS) {
-      const int r = idx / GV_COLS, c = idx % GV_COLS;
-      float s = 0.f;
-      if (r < mb && n0 + c < a.N)
-        for (int q = 0; q < a.ks; q++)
-          s += __ldcg(a.part + ((int64_t)q * a.B + b0 + r) * a.N + n0 + c);
-      sm[idx] = s;
+    const float *pp[PER];
+    bool ok[PER];
+    float sum[PER];
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+      const int idx = tid + GV_THREADS * i, r = idx / GV_COLS, c = idx % GV_COLS;
+      ok[i] = r < mb && n0 + c < a.N;
+      pp[i] = a.part + ((int64_t)b0 + r) * a.N + n0 + c;
+      sum[i] = 0.f;
     }
+    // slices in order; four slices of every output in flight at a time
+    // (past the last slice a zero is added, which leaves the sum unchanged)
+    for (int q0 = 0; q0 < a.ks; q0 += 4) {
+      float v[PER][4];
+#pragma unroll
+      for (int i = 0; i < PER; i++)
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+          v[i][u] = (ok[i] && q0 + u < a.ks) ? __ldcg(pp[i] + (q0 + u) * qstride) : 0.f;
+#pragma unroll
+      for (int i = 0; i < PER; i++)
+#pragma unroll
+        for (int u = 0; u < 4; u++) sum[i] += v[i][u];
+    }
+#pragma unroll
+    for (int i = 0; i < PER; i++) sm[tid + GV_THREADS * i] = sum[i];
     __syncthreads();
     gemv_epilogue<A>(a, sm, b0, mb, n0);
     __syncthreads();
@@ -260,28 +303,34 @@ __global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
 // attends to keys 0..pos with weights softmax(q.k / sqrt(hd)); strata: query
 // head h reads key/value head h / (H / H_kv).  Block (chunk c of 128 keys,
 // key/value head g, sequence b); the group's query heads in passes of 8.
-// Scores are kept in base 2 (q pre-scaled by log2(e) / sqrt(hd)).  Writes per
-// (b, g, chunk, head of group): chunk maximum m, sum l of 2^(s - m), and
-// o = sum 2^(s - m) v.
+// Scores are kept in base 2 (q pre-scaled by log2(e) / sqrt(hd)).  Each block
+// writes per head of the group its chunk maximum m, sum l of 2^(s - m) and
+// o = sum 2^(s - m) v; the last chunk of (b, g) to finish merges the chunks
+// in order: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+constexpr int AT_HDMAX = 128;
 template <typename A>
 __global__ void __launch_bounds__(AT_THREADS)
     k_attn_decode(const A *__restrict__ qkv, int64_t qkvw, int T, const int *__restrict__ pos_p,
-                  int H, int Hkv, int hd, int nch, int vec, float *__restrict__ part) {
-  __shared__ float qs[AT_G][128];
+                  int H, int Hkv, int hd, int nch, int vec, float *__restrict__ part,
+                  unsigned *__restrict__ count, A *__restrict__ out) {
+  __shared__ __align__(16) float qs[AT_G][AT_HDMAX];
   __shared__ float ps[AT_G][AT_KEYS];
-  __shared__ float red[AT_G][AT_THREADS];
+  __shared__ __align__(16) float red[AT_G * AT_KEYS * 8];  // [r][key lane][hd], <= 8*1024
   __shared__ float wm[AT_THREADS / 32][AT_G], wl[AT_THREADS / 32][AT_G];
+  __shared__ int last;
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  pdl_release();
+  pdl_wait();  // the new row (b, pos) comes from the kernel before
   const int pos = *pos_p;
   const int j0 = c * AT_KEYS;
   if (j0 > pos) return;
-  const int j1 = min(j0 + AT_KEYS, pos + 1);
+  const int nk = min(AT_KEYS, pos + 1 - j0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = H / Hkv, d = H * hd, kvd = Hkv * hd;
   const float scale = 1.4426950408889634f / sqrtf((float)hd);
   const A *rowq = qkv + ((int64_t)b * T + pos) * qkvw;
-  const int j = j0 + tid;
-  const A *kr = qkv + ((int64_t)b * T + j) * qkvw + d + (int64_t)g * hd;
+  const A *kr = qkv + ((int64_t)b * T + j0 + tid) * qkvw + d + (int64_t)g * hd;
+  const A *vb = qkv + ((int64_t)b * T + j0) * qkvw + d + kvd + (int64_t)g * hd;
   for (int r0 = 0; r0 < G; r0 += AT_G) {
     const int nr = min(AT_G, G - r0);
     for (int i = tid; i < AT_G * hd; i += AT_THREADS) {
@@ -289,93 +338,131 @@ __global__ void __launch_bounds__(AT_THREADS)
       qs[r][e] = r < nr ? to_f(rowq[(int64_t)(g * G + r0 + r) * hd + e]) * scale : 0.f;
     }
     __syncthreads();
-    // scores: one key per thread
+    // scores: one key per thread, its row loaded 64 dimensions at a time
     float s[AT_G];
 #pragma unroll
     for (int r = 0; r < AT_G; r++) s[r] = 0.f;
-    if (j < j1) {
-      for (int e = 0; e < hd; e += 8) {
-        float kv[8];
-        load8(kr + e, vec != 0, hd - e, kv);
+    if (tid < nk) {
+      for (int e0 = 0; e0 < hd; e0 += 64) {
+        float kv[8][8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+          const int e = e0 + 8 * u;
+          if (e < hd) {
+            load8(kr + e, vec != 0, hd - e, kv[u]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; q++) kv[u][q] = 0.f;
+          }
+        }
 #pragma unroll
         for (int r = 0; r < AT_G; r++) {
-          float t = s[r];
+          if (r < nr) {
+            float t = s[r];
 #pragma unroll
-          for (int q = 0; q < 8; q++)
-            if (e + q < hd) t = fmaf(qs[r][e + q], kv[q], t);
-          s[r] = t;
+            for (int u = 0; u < 8; u++)
+#pragma unroll
+              for (int q = 0; q < 8; q++)
+                if (e0 + 8 * u + q < hd) t = fmaf(qs[r][e0 + 8 * u + q], kv[u][q], t);
+            s[r] = t;
+          }
         }
       }
     }
     // chunk maximum and sum per query head (warps, then the 4 warps in order)
 #pragma unroll
     for (int r = 0; r < AT_G; r++) {
-      const float m = warp_max(j < j1 ? s[r] : -INFINITY);
+      const float m = warp_max(tid < nk ? s[r] : -INFINITY);
       if (lane == 0) wm[warp][r] = m;
     }
     __syncthreads();
-    float p[AT_G];
 #pragma unroll
     for (int r = 0; r < AT_G; r++) {
       const float m = fmaxf(fmaxf(wm[0][r], wm[1][r]), fmaxf(wm[2][r], wm[3][r]));
-      p[r] = j < j1 ? exp2f(s[r] - m) : 0.f;
-      ps[r][tid] = p[r];
-      const float l = warp_sum(p[r]);
+      const float p = tid < nk ? exp2f(s[r] - m) : 0.f;
+      ps[r][tid] = p;
+      const float l = warp_sum(p);
       if (lane == 0) wl[warp][r] = l;
     }
     __syncthreads();
-    // o = sum_j p_j v_j: thread = (dimension e, key lane kq), hd divides 128
-    const int KL = AT_THREADS / hd, e = tid % hd, kq = tid / hd;
-    float o[AT_G];
+    // o = sum_j p_j v_j.  Thread = (group of VW dimensions, key lane); VW = 8
+    // with 16-byte loads when rows allow, else 1
+    const int VW = vec ? 8 : 1;
+    const int DG = hd / VW, KLN = AT_THREADS / DG, dg = tid % DG, kq = tid / DG;
+    float acc[AT_G][8];
 #pragma unroll
-    for (int r = 0; r < AT_G; r++) o[r] = 0.f;
-    const A *vb = qkv + (int64_t)b * T * qkvw + d + kvd + (int64_t)g * hd + e;
-    for (int jj = kq; jj < j1 - j0; jj += KL) {
-      const float v = to_f(vb[(int64_t)(j0 + jj) * qkvw]);
+    for (int r = 0; r < AT_G; r++)
 #pragma unroll
-      for (int r = 0; r < AT_G; r++) o[r] = fmaf(ps[r][jj], v, o[r]);
-    }
+      for (int q = 0; q < 8; q++) acc[r][q] = 0.f;
+    for (int jj0 = kq; jj0 < nk; jj0 += 4 * KLN) {
+      float v[4][8];
 #pragma unroll
-    for (int r = 0; r < AT_G; r++) red[r][tid] = o[r];
-    __syncthreads();
-    if (tid < hd) {
-      for (int r = 0; r < nr; r++) {
-        float acc = 0.f;
-        for (int q = 0; q < KL; q++) acc += red[r][q * hd + tid];
-        float *rec = part + ((((int64_t)b * Hkv + g) * nch + c) * G + r0 + r) * (hd + 2);
-        rec[2 + tid] = acc;
-        if (tid == 0) {
-          rec[0] = fmaxf(fmaxf(wm[0][r], wm[1][r]), fmaxf(wm[2][r], wm[3][r]));
-          rec[1] = ((wl[0][r] + wl[1][r]) + wl[2][r]) + wl[3][r];
+      for (int u = 0; u < 4; u++) {
+        const int jj = jj0 + u * KLN;
+        if (jj < nk) {
+          load8(vb + (int64_t)jj * qkvw + dg * VW, vec != 0, VW, v[u]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; q++) v[u][q] = 0.f;
         }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const int jj = jj0 + u * KLN;
+        if (jj < nk) {
+#pragma unroll
+          for (int r = 0; r < AT_G; r++) {
+            if (r < nr) {
+              const float pj = ps[r][jj];
+#pragma unroll
+              for (int q = 0; q < 8; q++) acc[r][q] = fmaf(pj, v[u][q], acc[r][q]);
+            }
+          }
+        }
+      }
+    }
+    for (int r = 0; r < nr; r++)
+      for (int q = 0; q < VW; q++) red[(r * KLN + kq) * hd + dg * VW + q] = acc[r][q];
+    __syncthreads();
+    for (int idx = tid; idx < nr * hd; idx += AT_THREADS) {
+      const int r = idx / hd, e = idx % hd;
+      float o = 0.f;
+      for (int q = 0; q < KLN; q++) o += red[(r * KLN + q) * hd + e];
+      float *rec = part + ((((int64_t)b * Hkv + g) * nch + c) * G + r0 + r) * (hd + 2);
+      rec[2 + e] = o;
+      if (e == 0) {
+        rec[0] = fmaxf(fmaxf(wm[0][r], wm[1][r]), fmaxf(wm[2][r], wm[3][r]));
+        rec[1] = ((wl[0][r] + wl[1][r]) + wl[2][r]) + wl[3][r];
       }
     }
     __syncthreads();
   }
-}
-
-// o[b, h*hd + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c over the
-// chunks 0..pos/128 in order.  Block (query head, sequence).
-template <typename A>
-__global__ void k_attn_combine(const float *__restrict__ part, const int *__restrict__ pos_p, int H,
-                               int Hkv, int hd, int nch, A *__restrict__ out) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int G = H / Hkv, g = h / G, r = h % G;
-  const int nc = *pos_p / AT_KEYS + 1;
+  // ---- the last chunk of (b, g) to finish merges the chunks in order
+  const int nc = pos / AT_KEYS + 1;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(&count[b * Hkv + g], 1u) == (unsigned)(nc - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
   const int64_t stride = (int64_t)G * (hd + 2);
-  const float *rec0 = part + (((int64_t)b * Hkv + g) * nch * G + r) * (hd + 2);
-  float M = -INFINITY;
-  for (int c = 0; c < nc; c++) M = fmaxf(M, rec0[c * stride]);
-  for (int e = threadIdx.x; e < hd; e += blockDim.x) {
-    float L = 0.f, acc = 0.f;
-    for (int c = 0; c < nc; c++) {
-      const float *rc = rec0 + c * stride;
-      const float f = exp2f(rc[0] - M);
-      L = fmaf(f, rc[1], L);
-      acc = fmaf(f, rc[2 + e], acc);
+  for (int idx = tid; idx < G * hd; idx += AT_THREADS) {
+    const int r = idx / hd, e = idx % hd;
+    const float *rec0 = part + (((int64_t)b * Hkv + g) * nch * G + r) * (hd + 2);
+    float M = -INFINITY;
+#pragma unroll 4
+    for (int cc = 0; cc < nc; cc++) M = fmaxf(M, __ldcg(rec0 + cc * stride));
+    float L = 0.f, o = 0.f;
+#pragma unroll 4
+    for (int cc = 0; cc < nc; cc++) {
+      const float *rc = rec0 + cc * stride;
+      const float f = exp2f(__ldcg(rc) - M);
+      L = fmaf(f, __ldcg(rc + 1), L);
+      o = fmaf(f, __ldcg(rc + 2 + e), o);
     }
-    out[(int64_t)b * H * hd + (int64_t)h * hd + e] = from_f<A>(acc / L);
+    out[(int64_t)b * H * hd + (int64_t)(g * G + r) * hd + e] = from_f<A>(o / L);
   }
+  if (tid == 0) count[b * Hkv + g] = 0u;  // ready for the next launch
 }
 
 // ------------------------------------------------------------- sampling
@@ -550,8 +637,9 @@ __global__ void k_set_int(int *p, int v) { *p = v; }
 
 void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice) {
   const int64_t cb = (N + GV_COLS - 1) / GV_COLS;
-  const int64_t want = std::max<int64_t>(1, (4 * 148 + cb - 1) / cb);  // ~4 blocks per SM
-  const int64_t ks_max = std::max<int64_t>(1, (K + 63) / 64);          // >= 64 rows a slice
+  // one wave: two blocks of this kernel fit on each of the 148 SMs
+  const int64_t want = std::max<int64_t>(1, (2 * 148) / cb);
+  const int64_t ks_max = std::min<int64_t>(GV_KS_MAX, std::max<int64_t>(1, (K + 63) / 64));
   const int64_t ks_min = (K + GV_KSLICE_MAX - 1) / GV_KSLICE_MAX;
   int64_t s = std::max(std::min(want, ks_max), ks_min);
   int64_t sl = (K + s - 1) / s;
@@ -562,33 +650,45 @@ void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice) {
 
 int gemv_col_blocks(int64_t N) { return (int)cdiv(N, GV_COLS); }
 
+// Launch with programmatic stream serialisation (see pdl_release / pdl_wait).
+template <typename... P, typename... Q>
+static void launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, cudaStream_t s, Q... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 void gemv(const GemvArgs &a, DType dt, cudaStream_t s) {
   dim3 grid(cdiv(a.N, GV_COLS), a.ks);
-  if (dt == DT_BF16) k_gemv<__nv_bfloat16><<<grid, GV_THREADS, 0, s>>>(a);
-  else k_gemv<float><<<grid, GV_THREADS, 0, s>>>(a);
+  if (dt == DT_BF16) launch_pdl(k_gemv<__nv_bfloat16>, grid, dim3(GV_THREADS), s, a);
+  else launch_pdl(k_gemv<float>, grid, dim3(GV_THREADS), s, a);
   count_launch();
 }
 
 int attn_decode_chunks(int T) { return (int)cdiv(T, AT_KEYS); }
 
 void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, int H, int Hkv,
-                 int hd, float *part, void *o, DType dt, cudaStream_t s) {
+                 int hd, float *part, unsigned *count, void *o, DType dt, cudaStream_t s) {
   const int nch = attn_decode_chunks(T), d = H * hd;
   const int ve = dt == DT_BF16 ? 8 : 4;
   const int vec = (hd % 8 == 0 && qkvw % ve == 0 && d % ve == 0) ? 1 : 0;
   dim3 grid(nch, Hkv, B);
-  if (dt == DT_BF16) {
-    k_attn_decode<<<grid, AT_THREADS, 0, s>>>((const __nv_bfloat16 *)qkv, qkvw, T, pos, H, Hkv,
-                                             hd, nch, vec, part);
-    k_attn_combine<<<dim3(H, B), std::max(32, std::min(128, hd)), 0, s>>>(
-        part, pos, H, Hkv, hd, nch, (__nv_bfloat16 *)o);
-  } else {
-    k_attn_decode<<<grid, AT_THREADS, 0, s>>>((const float *)qkv, qkvw, T, pos, H, Hkv, hd, nch,
-                                             vec, part);
-    k_attn_combine<<<dim3(H, B), std::max(32, std::min(128, hd)), 0, s>>>(part, pos, H, Hkv, hd,
-                                                                         nch, (float *)o);
-  }
-  count_launch(2);
+  if (dt == DT_BF16)
+    launch_pdl(k_attn_decode<__nv_bfloat16>, grid, dim3(AT_THREADS), s,
+               (const __nv_bfloat16 *)qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part, count,
+               (__nv_bfloat16 *)o);
+  else
+    launch_pdl(k_attn_decode<float>, grid, dim3(AT_THREADS), s, (const float *)qkv, qkvw, T, pos,
+               H, Hkv, hd, nch, vec, part, count, (float *)o);
+  count_launch();
 }
 
 void sample_tokens(const float *logits, int64_t ld, int rows, int V, float temperature, int top_k,

@@ -149,10 +149,11 @@ int gemv_col_blocks(int64_t N);
 void gemv(const GemvArgs &a, DType dt, cudaStream_t s);
 // Attention of the query at position *pos of every sequence against the
 // cached keys/values 0..*pos of qkv [B*T, qkvw] (one layer), o [B, H*hd];
-// part: B * H * attn_decode_chunks(T) * (hd + 2) floats.  Needs 128 % hd == 0.
+// part: B * H * attn_decode_chunks(T) * (hd + 2) floats; count: B * Hkv
+// counters, zero between launches.  Needs 128 % hd == 0.
 int attn_decode_chunks(int T);
 void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, int H, int Hkv,
-                 int hd, float *part, void *o, DType dt, cudaStream_t s);
+                 int hd, float *part, unsigned *count, void *o, DType dt, cudaStream_t s);
 // One token id per row of logits [rows, ld] (V valid columns).
 void sample_tokens(const float *logits, int64_t ld, int rows, int V, float temperature, int top_k,
                    const float *uni, int32_t *out, cudaStream_t s);

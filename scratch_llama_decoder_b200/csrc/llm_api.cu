@@ -164,7 +164,7 @@ struct llm_ctx {
   // records, column-block counters, the position word, and its own graph
   float *dec_x = nullptr, *dec_part = nullptr, *dec_attn = nullptr;
   void *dec_o = nullptr, *dec_u = nullptr;
-  unsigned *dec_count = nullptr;
+  unsigned *dec_count = nullptr, *dec_acount = nullptr;
   int *dec_pos = nullptr;
   cudaGraphExec_t dexec = nullptr;
   Key dkey{}, dprev_key{};
@@ -234,6 +234,7 @@ int64_t llm_ctx::carve(char *base) {
   dec_part = (float *)c.take(4 * std::max<int64_t>(1, dpart));
   dec_attn = (float *)c.take(4 * B * D_.H * attn_decode_chunks(D_.T) * (int64_t)(D_.hd + 2));
   dec_count = (unsigned *)c.take(4 * dblocks);
+  dec_acount = (unsigned *)c.take(4 * B * D_.Hkv);
   dec_pos = (int *)c.take(64);
   return round_up(c.off, 256);
 }
@@ -314,6 +315,7 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
                                            std::max<int64_t>(c->D.qkvw, 2 * c->D.hp),
                                            std::max<int64_t>(c->D.d, c->D.Vp))),
                   c->s);
+  cudaMemsetAsync(c->dec_acount, 0, 4 * (size_t)c->D.B * c->D.Hkv, c->s);
   cudaMemsetAsync(c->dec_pos, 0, 64, c->s);
   rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, cfg->rope_base, c->s);
   c->tc = tc_plan_create(c->D.dt, c->cos_t, c->sin_t, c->D.T, c->D.hd, c->D.d + c->D.kvd, c->D.hp);
@@ -648,8 +650,8 @@ void decode_body(llm_ctx *c, const float *p, const int32_t *tok, float *logits) 
                     (int64_t)D.T * D.qkvw, (int)D.qkvw);
     a.x = c->dec_x; a.ldx = d; a.gain = p + O.g1(l); a.pos_stride = D.qkvw;
     gemv(a, D.dt, s);
-    attn_decode(qkv, D.qkvw, D.B, D.T, c->dec_pos, D.H, D.Hkv, D.hd, c->dec_attn, c->dec_o, D.dt,
-                s);
+    attn_decode(qkv, D.qkvw, D.B, D.T, c->dec_pos, D.H, D.Hkv, D.hd, c->dec_attn, c->dec_acount,
+                c->dec_o, D.dt, s);
     // x += o Wo
     a = mv(d, d, A(c->w_o, l, d * d), d, DEC_RESID, c->dec_x, d, D.d);
     a.xa = c->dec_o; a.ldxa = d;
