@@ -15,8 +15,9 @@
 // slice order by the last block of a column block to finish (a counter per
 // column block), which then applies the epilogue: RoPE + cache store for the
 // q|k|v projection, residual add, SwiGLU, or the fp32 logits.  Attention of
-// the new query against positions 0..pos is split over 128-key chunks; the
-// last chunk of a (sequence, key/value head) to finish merges them in order.
+// the new query against positions 0..pos is split over 128-key chunks staged
+// in shared memory by asynchronous copies; the last chunk of a (sequence,
+// key/value head) to finish merges them in order.
 // Every sum has a fixed order: a decode call is bit-reproducible.
 #include <limits.h>
 #include <math.h>
@@ -44,7 +45,6 @@ static_assert(GV_CG * GV_KL == GV_THREADS && 8 * GV_CG == GV_COLS, "thread layou
 
 constexpr int AT_KEYS = 128;     // keys per attention block (one per thread when scoring)
 constexpr int AT_THREADS = 128;
-constexpr int AT_G = 8;          // query heads of a group per pass
 
 constexpr int SP_THREADS = 1024;
 
@@ -275,20 +275,18 @@ __global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
       pp[i] = a.part + ((int64_t)b0 + r) * a.N + n0 + c;
       sum[i] = 0.f;
     }
-    // slices in order; four slices of every output in flight at a time
-    // (past the last slice a zero is added, which leaves the sum unchanged)
-    for (int q0 = 0; q0 < a.ks; q0 += 4) {
-      float v[PER][4];
+    // every slice of this thread's outputs in flight at once, then added in
+    // slice order (past the last slice a zero is added: the sum is unchanged)
+    float v[PER][GV_KS_MAX];
 #pragma unroll
-      for (int i = 0; i < PER; i++)
+    for (int i = 0; i < PER; i++)
 #pragma unroll
-        for (int u = 0; u < 4; u++)
-          v[i][u] = (ok[i] && q0 + u < a.ks) ? __ldcg(pp[i] + (q0 + u) * qstride) : 0.f;
+      for (int q = 0; q < GV_KS_MAX; q++)
+        v[i][q] = (ok[i] && q < a.ks) ? __ldcg(pp[i] + q * qstride) : 0.f;
 #pragma unroll
-      for (int i = 0; i < PER; i++)
+    for (int i = 0; i < PER; i++)
 #pragma unroll
-        for (int u = 0; u < 4; u++) sum[i] += v[i][u];
-    }
+      for (int q = 0; q < GV_KS_MAX; q++) sum[i] += v[i][q];
 #pragma unroll
     for (int i = 0; i < PER; i++) sm[tid + GV_THREADS * i] = sum[i];
     __syncthreads();
@@ -302,82 +300,133 @@ __global__ void __launch_bounds__(GV_THREADS) k_gemv(const GemvArgs a) {
 // Hephaistos, Architecture at a glance (Attention): the query of position pos
 // attends to keys 0..pos with weights softmax(q.k / sqrt(hd)); strata: query
 // head h reads key/value head h / (H / H_kv).  Block (chunk c of 128 keys,
-// key/value head g, sequence b); the group's query heads in passes of 8.
-// Scores are kept in base 2 (q pre-scaled by log2(e) / sqrt(hd)).  Each block
-// writes per head of the group its chunk maximum m, sum l of 2^(s - m) and
-// o = sum 2^(s - m) v; the last chunk of (b, g) to finish merges the chunks
-// in order: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+// key/value head g, sequence b).  The chunk's key and value rows are staged in
+// shared memory (rows padded by 16 bytes) by asynchronous 16-byte copies: the
+// rows before pos were written by earlier calls, so their copies are issued
+// before waiting for the kernel before (which writes q and row pos).  The
+// group's query heads go in passes of GT; scores are kept in base 2 (q
+// pre-scaled by log2(e) / sqrt(hd)).  Each block writes per head its chunk
+// maximum m, sum l of 2^(s - m) and o = sum 2^(s - m) v; the last chunk of
+// (b, g) to finish merges the chunks in order:
+// o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
 constexpr int AT_HDMAX = 128;
-template <typename A>
-__global__ void __launch_bounds__(AT_THREADS)
+constexpr int AT_MERGE = 16;  // chunks whose records are loaded together in the merge
+
+LLM_DEV uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+LLM_DEV void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+LLM_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// 8 values of a staged row (16-byte aligned when vec), element by element up to n
+LLM_DEV void smem8(const __nv_bfloat16 *p, bool vec, int n, float (&w)[8]) {
+  if (vec && n >= 8) {
+    bf16x8(*reinterpret_cast<const uint4 *>(p), w);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; k++) w[k] = k < n ? __bfloat162float(p[k]) : 0.f;
+  }
+}
+LLM_DEV void smem8(const float *p, bool vec, int n, float (&w)[8]) {
+  if (vec && n >= 8) {
+    const float4 a = reinterpret_cast<const float4 *>(p)[0];
+    const float4 b = reinterpret_cast<const float4 *>(p)[1];
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; k++) w[k] = k < n ? p[k] : 0.f;
+  }
+}
+// Bytes of one staged row (a multiple of 16, plus 16 so rows fall on
+// different banks) and of the block's dynamic shared memory.
+__host__ __device__ inline int attn_row_bytes(int hd, int esz) {
+  return (hd * esz + 15) / 16 * 16 + 16;
+}
+
+template <typename A, int GT>
+__global__ void __launch_bounds__(AT_THREADS, 4)
     k_attn_decode(const A *__restrict__ qkv, int64_t qkvw, int T, const int *__restrict__ pos_p,
                   int H, int Hkv, int hd, int nch, int vec, float *__restrict__ part,
                   unsigned *__restrict__ count, A *__restrict__ out) {
-  __shared__ __align__(16) float qs[AT_G][AT_HDMAX];
-  __shared__ float ps[AT_G][AT_KEYS];
-  __shared__ __align__(16) float red[AT_G * AT_KEYS * 8];  // [r][key lane][hd], <= 8*1024
-  __shared__ float wm[AT_THREADS / 32][AT_G], wl[AT_THREADS / 32][AT_G];
+  extern __shared__ __align__(16) uint8_t kv_sm[];
+  __shared__ __align__(16) float qs[GT][AT_HDMAX];
+  __shared__ float ps[GT][AT_KEYS];
+  __shared__ float wm[AT_THREADS / 32][GT], wl[AT_THREADS / 32][GT];
   __shared__ int last;
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   pdl_release();
-  pdl_wait();  // the new row (b, pos) comes from the kernel before
+  // the position word is written before the decode kernels start
   const int pos = *pos_p;
   const int j0 = c * AT_KEYS;
   if (j0 > pos) return;
   const int nk = min(AT_KEYS, pos + 1 - j0);
+  const int nold = min(nk, pos - j0);  // rows of this chunk written by earlier calls
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = H / Hkv, d = H * hd, kvd = Hkv * hd;
+  const int esz = (int)sizeof(A), RS = attn_row_bytes(hd, esz);
+  uint8_t *Ks = kv_sm, *Vs = kv_sm + AT_KEYS * RS;
+  const A *kb = qkv + ((int64_t)b * T + j0) * qkvw + d + (int64_t)g * hd;
+  const A *vb = kb + kvd;
+  const int cpr = hd * esz / 16;  // 16-byte pieces of a row (vec)
+  auto stage = [&](int ja, int jb) {  // rows [ja, jb) of the chunk
+    if (vec) {
+      for (int i = tid; i < (jb - ja) * cpr; i += AT_THREADS) {
+        const int j = ja + i / cpr, q = i % cpr;
+        cp_async16(Ks + j * RS + 16 * q, reinterpret_cast<const uint8_t *>(kb + (int64_t)j * qkvw) + 16 * q);
+        cp_async16(Vs + j * RS + 16 * q, reinterpret_cast<const uint8_t *>(vb + (int64_t)j * qkvw) + 16 * q);
+      }
+    } else {
+      for (int i = tid; i < (jb - ja) * hd; i += AT_THREADS) {
+        const int j = ja + i / hd, e = i % hd;
+        reinterpret_cast<A *>(Ks + j * RS)[e] = kb[(int64_t)j * qkvw + e];
+        reinterpret_cast<A *>(Vs + j * RS)[e] = vb[(int64_t)j * qkvw + e];
+      }
+    }
+  };
+  stage(0, nold);
+  pdl_wait();  // q and row pos come from the kernel before
+  stage(nold, nk);
+  cp_async_wait_all();
   const float scale = 1.4426950408889634f / sqrtf((float)hd);
   const A *rowq = qkv + ((int64_t)b * T + pos) * qkvw;
-  const A *kr = qkv + ((int64_t)b * T + j0 + tid) * qkvw + d + (int64_t)g * hd;
-  const A *vb = qkv + ((int64_t)b * T + j0) * qkvw + d + kvd + (int64_t)g * hd;
-  for (int r0 = 0; r0 < G; r0 += AT_G) {
-    const int nr = min(AT_G, G - r0);
-    for (int i = tid; i < AT_G * hd; i += AT_THREADS) {
+  for (int r0 = 0; r0 < G; r0 += GT) {
+    const int nr = min(GT, G - r0);
+    for (int i = tid; i < GT * hd; i += AT_THREADS) {
       const int r = i / hd, e = i % hd;
       qs[r][e] = r < nr ? to_f(rowq[(int64_t)(g * G + r0 + r) * hd + e]) * scale : 0.f;
     }
-    __syncthreads();
-    // scores: one key per thread, its row loaded 64 dimensions at a time
-    float s[AT_G];
+    __syncthreads();  // q, and every thread's staged rows
+    // scores: one key per thread
+    float s[GT];
 #pragma unroll
-    for (int r = 0; r < AT_G; r++) s[r] = 0.f;
+    for (int r = 0; r < GT; r++) s[r] = 0.f;
     if (tid < nk) {
-      for (int e0 = 0; e0 < hd; e0 += 64) {
-        float kv[8][8];
+      const A *kr = reinterpret_cast<const A *>(Ks + tid * RS);
+      for (int e = 0; e < hd; e += 8) {
+        float kv[8];
+        smem8(kr + e, vec != 0, hd - e, kv);
 #pragma unroll
-        for (int u = 0; u < 8; u++) {
-          const int e = e0 + 8 * u;
-          if (e < hd) {
-            load8(kr + e, vec != 0, hd - e, kv[u]);
-          } else {
+        for (int r = 0; r < GT; r++) {
+          float t = s[r];
 #pragma unroll
-            for (int q = 0; q < 8; q++) kv[u][q] = 0.f;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < AT_G; r++) {
-          if (r < nr) {
-            float t = s[r];
-#pragma unroll
-            for (int u = 0; u < 8; u++)
-#pragma unroll
-              for (int q = 0; q < 8; q++)
-                if (e0 + 8 * u + q < hd) t = fmaf(qs[r][e0 + 8 * u + q], kv[u][q], t);
-            s[r] = t;
-          }
+          for (int q = 0; q < 8; q++)
+            if (e + q < hd) t = fmaf(qs[r][e + q], kv[q], t);
+          s[r] = t;
         }
       }
     }
     // chunk maximum and sum per query head (warps, then the 4 warps in order)
 #pragma unroll
-    for (int r = 0; r < AT_G; r++) {
+    for (int r = 0; r < GT; r++) {
       const float m = warp_max(tid < nk ? s[r] : -INFINITY);
       if (lane == 0) wm[warp][r] = m;
     }
     __syncthreads();
 #pragma unroll
-    for (int r = 0; r < AT_G; r++) {
+    for (int r = 0; r < GT; r++) {
       const float m = fmaxf(fmaxf(wm[0][r], wm[1][r]), fmaxf(wm[2][r], wm[3][r]));
       const float p = tid < nk ? exp2f(s[r] - m) : 0.f;
       ps[r][tid] = p;
@@ -385,49 +434,14 @@ __global__ void __launch_bounds__(AT_THREADS)
       if (lane == 0) wl[warp][r] = l;
     }
     __syncthreads();
-    // o = sum_j p_j v_j.  Thread = (group of VW dimensions, key lane); VW = 8
-    // with 16-byte loads when rows allow, else 1
-    const int VW = vec ? 8 : 1;
-    const int DG = hd / VW, KLN = AT_THREADS / DG, dg = tid % DG, kq = tid / DG;
-    float acc[AT_G][8];
-#pragma unroll
-    for (int r = 0; r < AT_G; r++)
-#pragma unroll
-      for (int q = 0; q < 8; q++) acc[r][q] = 0.f;
-    for (int jj0 = kq; jj0 < nk; jj0 += 4 * KLN) {
-      float v[4][8];
-#pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const int jj = jj0 + u * KLN;
-        if (jj < nk) {
-          load8(vb + (int64_t)jj * qkvw + dg * VW, vec != 0, VW, v[u]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; q++) v[u][q] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const int jj = jj0 + u * KLN;
-        if (jj < nk) {
-#pragma unroll
-          for (int r = 0; r < AT_G; r++) {
-            if (r < nr) {
-              const float pj = ps[r][jj];
-#pragma unroll
-              for (int q = 0; q < 8; q++) acc[r][q] = fmaf(pj, v[u][q], acc[r][q]);
-            }
-          }
-        }
-      }
-    }
-    for (int r = 0; r < nr; r++)
-      for (int q = 0; q < VW; q++) red[(r * KLN + kq) * hd + dg * VW + q] = acc[r][q];
-    __syncthreads();
+    // o[r][e] = sum_j p_j v_j[e], keys in order, one output per thread
     for (int idx = tid; idx < nr * hd; idx += AT_THREADS) {
       const int r = idx / hd, e = idx % hd;
+      const uint8_t *vc = Vs + e * esz;
       float o = 0.f;
-      for (int q = 0; q < KLN; q++) o += red[(r * KLN + q) * hd + e];
+#pragma unroll 8
+      for (int jj = 0; jj < nk; jj++)
+        o = fmaf(ps[r][jj], to_f(*reinterpret_cast<const A *>(vc + jj * RS)), o);
       float *rec = part + ((((int64_t)b * Hkv + g) * nch + c) * G + r0 + r) * (hd + 2);
       rec[2 + e] = o;
       if (e == 0) {
@@ -450,15 +464,33 @@ __global__ void __launch_bounds__(AT_THREADS)
     const int r = idx / hd, e = idx % hd;
     const float *rec0 = part + (((int64_t)b * Hkv + g) * nch * G + r) * (hd + 2);
     float M = -INFINITY;
-#pragma unroll 4
-    for (int cc = 0; cc < nc; cc++) M = fmaxf(M, __ldcg(rec0 + cc * stride));
+    for (int c0 = 0; c0 < nc; c0 += AT_MERGE) {
+      float mv[AT_MERGE];
+#pragma unroll
+      for (int u = 0; u < AT_MERGE; u++)
+        mv[u] = c0 + u < nc ? __ldcg(rec0 + (c0 + u) * stride) : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < AT_MERGE; u++) M = fmaxf(M, mv[u]);
+    }
     float L = 0.f, o = 0.f;
-#pragma unroll 4
-    for (int cc = 0; cc < nc; cc++) {
-      const float *rc = rec0 + cc * stride;
-      const float f = exp2f(__ldcg(rc) - M);
-      L = fmaf(f, __ldcg(rc + 1), L);
-      o = fmaf(f, __ldcg(rc + 2 + e), o);
+    for (int c0 = 0; c0 < nc; c0 += AT_MERGE) {
+      float mv[AT_MERGE], lv[AT_MERGE], ov[AT_MERGE];
+#pragma unroll
+      for (int u = 0; u < AT_MERGE; u++) {
+        const bool in = c0 + u < nc;
+        const float *rc = rec0 + (c0 + u) * stride;
+        mv[u] = in ? __ldcg(rc) : 0.f;
+        lv[u] = in ? __ldcg(rc + 1) : 0.f;
+        ov[u] = in ? __ldcg(rc + 2 + e) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < AT_MERGE; u++) {
+        if (c0 + u < nc) {
+          const float f = exp2f(mv[u] - M);
+          L = fmaf(f, lv[u], L);
+          o = fmaf(f, ov[u], o);
+        }
+      }
     }
     out[(int64_t)b * H * hd + (int64_t)(g * G + r) * hd + e] = from_f<A>(o / L);
   }
@@ -641,7 +673,10 @@ void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice) {
   const int64_t want = std::max<int64_t>(1, (2 * 148) / cb);
   const int64_t ks_max = std::min<int64_t>(GV_KS_MAX, std::max<int64_t>(1, (K + 63) / 64));
   const int64_t ks_min = (K + GV_KSLICE_MAX - 1) / GV_KSLICE_MAX;
-  int64_t s = std::max(std::min(want, ks_max), ks_min);
+  // at most 128 rows a slice (two batches of loads per thread) where the
+  // slice cap allows, else as few waves as the cap gives
+  const int64_t want_rows = (K + 127) / 128;
+  int64_t s = std::max(std::min(std::max(want, want_rows), ks_max), ks_min);
   int64_t sl = (K + s - 1) / s;
   sl = std::min<int64_t>(GV_KSLICE_MAX, (sl + 15) / 16 * 16);
   *kslice = (int)sl;
@@ -652,11 +687,12 @@ int gemv_col_blocks(int64_t N) { return (int)cdiv(N, GV_COLS); }
 
 // Launch with programmatic stream serialisation (see pdl_release / pdl_wait).
 template <typename... P, typename... Q>
-static void launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, cudaStream_t s, Q... args) {
+static void launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Q... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -668,26 +704,51 @@ static void launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, cudaStream_t
 
 void gemv(const GemvArgs &a, DType dt, cudaStream_t s) {
   dim3 grid(cdiv(a.N, GV_COLS), a.ks);
-  if (dt == DT_BF16) launch_pdl(k_gemv<__nv_bfloat16>, grid, dim3(GV_THREADS), s, a);
-  else launch_pdl(k_gemv<float>, grid, dim3(GV_THREADS), s, a);
+  if (dt == DT_BF16) launch_pdl(k_gemv<__nv_bfloat16>, grid, dim3(GV_THREADS), 0, s, a);
+  else launch_pdl(k_gemv<float>, grid, dim3(GV_THREADS), 0, s, a);
   count_launch();
 }
 
 int attn_decode_chunks(int T) { return (int)cdiv(T, AT_KEYS); }
 
+template <typename A, int GT>
+static void attn_launch(dim3 grid, size_t smem, cudaStream_t s, const void *qkv, int64_t qkvw,
+                        int T, const int *pos, int H, int Hkv, int hd, int nch, int vec,
+                        float *part, unsigned *count, void *o) {
+  static bool attr = false;  // opt in to the largest staged tile once per kernel
+  if (!attr) {
+    cudaFuncSetAttribute(k_attn_decode<A, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         2 * AT_KEYS * attn_row_bytes(AT_HDMAX, 4));
+    attr = true;
+  }
+  launch_pdl(k_attn_decode<A, GT>, grid, dim3(AT_THREADS), smem, s, (const A *)qkv, qkvw, T, pos,
+             H, Hkv, hd, nch, vec, part, count, (A *)o);
+}
+template <typename A>
+static void attn_dispatch(int G, dim3 grid, size_t smem, cudaStream_t s, const void *qkv,
+                          int64_t qkvw, int T, const int *pos, int H, int Hkv, int hd, int nch,
+                          int vec, float *part, unsigned *count, void *o) {
+  if (G <= 1) attn_launch<A, 1>(grid, smem, s, qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part, count, o);
+  else if (G <= 2) attn_launch<A, 2>(grid, smem, s, qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part, count, o);
+  else if (G <= 4) attn_launch<A, 4>(grid, smem, s, qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part, count, o);
+  else attn_launch<A, 8>(grid, smem, s, qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part, count, o);
+}
+
 void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, int H, int Hkv,
                  int hd, float *part, unsigned *count, void *o, DType dt, cudaStream_t s) {
-  const int nch = attn_decode_chunks(T), d = H * hd;
-  const int ve = dt == DT_BF16 ? 8 : 4;
-  const int vec = (hd % 8 == 0 && qkvw % ve == 0 && d % ve == 0) ? 1 : 0;
+  const int nch = attn_decode_chunks(T), d = H * hd, kvd = Hkv * hd;
+  const int esz = dt == DT_BF16 ? 2 : 4, ve = 16 / esz;
+  // 16-byte copies: whole pieces per row, every row start 16-byte aligned
+  const int vec = ((hd * esz) % 16 == 0 && qkvw % ve == 0 && d % ve == 0 && kvd % ve == 0 &&
+                   ((uintptr_t)qkv & 15) == 0) ? 1 : 0;
+  const size_t smem = 2 * (size_t)AT_KEYS * attn_row_bytes(hd, esz);
   dim3 grid(nch, Hkv, B);
   if (dt == DT_BF16)
-    launch_pdl(k_attn_decode<__nv_bfloat16>, grid, dim3(AT_THREADS), s,
-               (const __nv_bfloat16 *)qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part, count,
-               (__nv_bfloat16 *)o);
+    attn_dispatch<__nv_bfloat16>(H / Hkv, grid, smem, s, qkv, qkvw, T, pos, H, Hkv, hd, nch, vec,
+                                 part, count, o);
   else
-    launch_pdl(k_attn_decode<float>, grid, dim3(AT_THREADS), s, (const float *)qkv, qkvw, T, pos,
-               H, Hkv, hd, nch, vec, part, count, (float *)o);
+    attn_dispatch<float>(H / Hkv, grid, smem, s, qkv, qkvw, T, pos, H, Hkv, hd, nch, vec, part,
+                         count, o);
   count_launch();
 }
 
