@@ -673,10 +673,9 @@ void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice) {
   const int64_t want = std::max<int64_t>(1, (2 * 148) / cb);
   const int64_t ks_max = std::min<int64_t>(GV_KS_MAX, std::max<int64_t>(1, (K + 63) / 64));
   const int64_t ks_min = (K + GV_KSLICE_MAX - 1) / GV_KSLICE_MAX;
-  // at most 128 rows a slice (two batches of loads per thread) where the
-  // slice cap allows, else as few waves as the cap gives
-  const int64_t want_rows = (K + 127) / 128;
-  int64_t s = std::max(std::min(std::max(want, want_rows), ks_max), ks_min);
+  // (measured: more slices than one wave, or slices under 128 rows bought
+  // with a second wave, made the W13 and lm_head products slower)
+  int64_t s = std::max(std::min(want, ks_max), ks_min);
   int64_t sl = (K + s - 1) / s;
   sl = std::min<int64_t>(GV_KSLICE_MAX, (sl + 15) / 16 * 16);
   *kslice = (int)sl;
