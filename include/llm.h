@@ -171,6 +171,45 @@ int llm_decode(llm_ctx *ctx, const float *d_params, const int32_t *d_tokens, int
 int llm_sample(llm_ctx *ctx, const float *d_logits, int64_t ld, int n_rows, float temperature,
                int top_k, const float *d_uniform, int32_t *d_out);
 
+/* Learning-rate schedule (host only: needs no context and no GPU; the value
+ * is passed to llm_step as lr).  Transformer-In-Rust, Features: cosine decay
+ * with linear warmup, and cosine / linear / constant schedulers; randyGPT,
+ * Training: constant at max_lr, then cosine decay to min_lr over the final
+ * 40%; strata: cosine + warmup.  For 1-based step t:
+ *   t <= warmup_steps (when > 0):  lr = max_lr * t / warmup_steps
+ *   t <= decay_start:               lr = max_lr
+ *   else, p = min(1, (t - decay_start) / (total_steps - decay_start)), or 1
+ *   when total_steps <= decay_start:
+ *     LLM_LR_COSINE:   min_lr + (max_lr - min_lr) * (1 + cos(pi p)) / 2
+ *     LLM_LR_LINEAR:   max_lr + (min_lr - max_lr) * p
+ *     LLM_LR_CONSTANT: max_lr
+ * computed in double precision and rounded to float into *lr.  LLM_ERR_ARG
+ * for a null pointer, t < 1, warmup_steps < 0, decay_start < warmup_steps, an
+ * unknown shape or a non-finite rate. */
+enum { LLM_LR_CONSTANT = 0, LLM_LR_COSINE = 1, LLM_LR_LINEAR = 2 };
+typedef struct {
+  float max_lr, min_lr;
+  int64_t warmup_steps, decay_start, total_steps;
+  int32_t shape;
+} llm_lr_schedule;
+int llm_lr_at(const llm_lr_schedule *sched, int64_t t, float *lr);
+
+/* Global-norm gradient clipping inside llm_step (MicroGPT in Rust, Gradient
+ * Clipping: when the gradient norm exceeds max_norm every gradient is scaled
+ * by max_norm / norm; Transformer-In-Rust: clipping by global norm).  With
+ * max_norm > 0, every later llm_step computes the Euclidean norm of the whole
+ * gradient buffer (double-precision sums in a fixed order), scales d_grads in
+ * place by max_norm / norm when norm > max_norm, and AdamW then uses the
+ * clipped gradient (d_grads holds it after the step).  max_norm <= 0 turns
+ * clipping off (the default).  A change frees the captured step graph
+ * (synchronising the stream first).  LLM_ERR_ARG for NaN. */
+int llm_set_grad_clip(llm_ctx *ctx, float max_norm);
+
+/* Synchronises the context's stream and returns in *norm the gradient norm
+ * (before clipping) of the most recent llm_step run with clipping on;
+ * LLM_ERR_ARG if no such step has run on this context. */
+int llm_read_grad_norm(llm_ctx *ctx, double *norm);
+
 /* Synchronises the context's stream and returns the first error any call on
  * this context raised on the device since the previous llm_status() (then
  * clears it), or LLM_ERR_CUDA if the stream reports a CUDA error, else LLM_OK. */

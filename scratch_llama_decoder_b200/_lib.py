@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(HERE, "libllm.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m scratch_llama_decoder_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python scratch_llama_decoder_b200/build.py` "
         "(nvcc, sm_100a).  There is no CPU fallback.")
 
 lib = C.CDLL(LIB_PATH)
@@ -34,6 +34,15 @@ class llm_tensor_info(C.Structure):
                 ("cols", C.c_int64)]
 
 
+LLM_LR_CONSTANT, LLM_LR_COSINE, LLM_LR_LINEAR = 0, 1, 2
+LR_SHAPES = {"constant": LLM_LR_CONSTANT, "cosine": LLM_LR_COSINE, "linear": LLM_LR_LINEAR}
+
+
+class llm_lr_schedule(C.Structure):
+    _fields_ = [("max_lr", C.c_float), ("min_lr", C.c_float), ("warmup_steps", C.c_int64),
+                ("decay_start", C.c_int64), ("total_steps", C.c_int64), ("shape", C.c_int32)]
+
+
 _vp, _i64, _u64, _f, _i = C.c_void_p, C.c_int64, C.c_uint64, C.c_float, C.c_int
 _cfgp = C.POINTER(llm_config)
 
@@ -47,6 +56,9 @@ EXPORTS = {
     "llm_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _f, _f, _vp]),
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
     "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),
+    "llm_set_grad_clip": (_i, [_vp, _f]),
+    "llm_read_grad_norm": (_i, [_vp, C.POINTER(C.c_double)]),
+    "llm_lr_at": (_i, [C.POINTER(llm_lr_schedule), _i64, C.POINTER(_f)]),
     "llm_status": (_i, [_vp]),
     "llm_error_string": (C.c_char_p, [_i]),
     "llm_last_launch_count": (_i, [_vp]),
@@ -111,3 +123,11 @@ def llm_workspace_bytes(cfg) -> int:
     b = C.c_int64(0)
     check(lib.llm_workspace_bytes(C.byref(c), C.byref(b)), "llm_workspace_bytes")
     return b.value
+
+
+def lr_at(t, max_lr, min_lr, warmup, decay_start, total, shape="cosine") -> float:
+    """Learning rate of 1-based step t (llm_lr_at)."""
+    sc = llm_lr_schedule(max_lr, min_lr, warmup, decay_start, total, LR_SHAPES[shape])
+    out = C.c_float(0.0)
+    check(lib.llm_lr_at(C.byref(sc), int(t), C.byref(out)), "llm_lr_at")
+    return out.value

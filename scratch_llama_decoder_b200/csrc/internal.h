@@ -75,6 +75,12 @@ void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int 
 int64_t embed_bwd_scratch_ints(int64_t N, int V);
 void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, float std,
                  int constant_one, cudaStream_t s);
+// Global-norm clipping of g [n] (16-byte aligned) in place: part holds
+// clip_part_blocks() doubles; *norm gets the norm before clipping, *scale the
+// factor applied (max_norm / norm when norm > max_norm, else 1).
+int clip_part_blocks();
+void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm, float *scale,
+                cudaStream_t s);
 void set_flag_zero(int *flag, cudaStream_t s);
 void or_flag(const int *src, int *dst, cudaStream_t s);
 

@@ -1034,6 +1034,80 @@ void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, floa
 }
 
 // -------------------------------------------------------------------- flags
+// ------------------------------------------------------- gradient clipping
+// MicroGPT in Rust, Gradient Clipping: the norm of all gradients together;
+// when it exceeds max_norm every gradient is scaled by max_norm / norm.
+// Squares are summed in double: per block in a fixed order over a fixed grid,
+// then the block sums in order by one block, so the norm is reproducible.
+constexpr int CLIP_BLOCKS = 148 * 4, CLIP_THREADS = 256;
+LLM_DEV double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+LLM_DEV double block_sum_d(double v, double *ws) {  // ws: CLIP_THREADS / 32 doubles
+  v = warp_sum_d(v);
+  if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double s = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < CLIP_THREADS / 32; w++) s += ws[w];
+  return s;  // valid in thread 0
+}
+// g is 16-byte aligned; elements past the last whole float4 go to block 0.
+__global__ void __launch_bounds__(CLIP_THREADS)
+    k_sumsq(const float *__restrict__ g, int64_t n, double *__restrict__ part) {
+  __shared__ double ws[CLIP_THREADS / 32];
+  const int64_t n4 = n / 4;
+  const float4 *g4 = reinterpret_cast<const float4 *>(g);
+  double acc = 0.0;
+  for (int64_t i = blockIdx.x * (int64_t)CLIP_THREADS + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * CLIP_THREADS) {
+    const float4 v = g4[i];
+    acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (int)(n & 3)) {
+    const double v = g[n4 * 4 + threadIdx.x];
+    acc += v * v;
+  }
+  const double s = block_sum_d(acc, ws);
+  if (threadIdx.x == 0) part[blockIdx.x] = s;
+}
+__global__ void __launch_bounds__(CLIP_THREADS)
+    k_clip_scale(const double *__restrict__ part, int nblk, float max_norm,
+                 double *__restrict__ norm, float *__restrict__ scale) {
+  __shared__ double ws[CLIP_THREADS / 32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nblk; i += CLIP_THREADS) acc += part[i];
+  const double s = block_sum_d(acc, ws);
+  if (threadIdx.x == 0) {
+    const double nm = sqrt(s);
+    *norm = nm;
+    *scale = nm > (double)max_norm ? (float)((double)max_norm / nm) : 1.0f;
+  }
+}
+__global__ void __launch_bounds__(CLIP_THREADS)
+    k_scale_grads(float *__restrict__ g, int64_t n, const float *__restrict__ scale) {
+  const float sc = *scale;
+  const int64_t n4 = n / 4;
+  float4 *g4 = reinterpret_cast<float4 *>(g);
+  for (int64_t i = blockIdx.x * (int64_t)CLIP_THREADS + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * CLIP_THREADS) {
+    float4 v = g4[i];
+    v.x *= sc; v.y *= sc; v.z *= sc; v.w *= sc;
+    g4[i] = v;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (int)(n & 3)) g[n4 * 4 + threadIdx.x] *= sc;
+}
+int clip_part_blocks() { return CLIP_BLOCKS; }
+void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm, float *scale,
+                cudaStream_t s) {
+  k_sumsq<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, part);
+  k_clip_scale<<<1, CLIP_THREADS, 0, s>>>(part, CLIP_BLOCKS, max_norm, norm, scale);
+  k_scale_grads<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, scale);
+  count_launch(3);
+}
+
 __global__ void k_or_flag(const int *src, int *dst) { if (*src) atomicOr(dst, *src); }
 void set_flag_zero(int *flag, cudaStream_t s) { cudaMemsetAsync(flag, 0, sizeof(int), s); }
 void or_flag(const int *src, int *dst, cudaStream_t s) {

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -170,6 +171,11 @@ struct llm_ctx {
   Key dkey{}, dprev_key{};
   bool dhave_prev = false;
   int dgraph_launches = 0;
+  // gradient clipping (llm_set_grad_clip): threshold, block sums, norm, scale
+  float clip = 0.f;
+  bool have_norm = false;
+  double *clip_part = nullptr, *clip_norm = nullptr;
+  float *clip_scale = nullptr;
   int64_t carve(char *base);
 };
 
@@ -236,6 +242,9 @@ int64_t llm_ctx::carve(char *base) {
   dec_count = (unsigned *)c.take(4 * dblocks);
   dec_acount = (unsigned *)c.take(4 * B * D_.Hkv);
   dec_pos = (int *)c.take(64);
+  clip_part = (double *)c.take(8 * (int64_t)clip_part_blocks());
+  clip_norm = (double *)c.take(64);
+  clip_scale = (float *)c.take(64);
   return round_up(c.off, 256);
 }
 
@@ -373,6 +382,54 @@ int llm_set_graphs(llm_ctx *c, int enable) {
   }
   c->have_prev = false;
   c->dhave_prev = false;
+  return LLM_OK;
+}
+
+int llm_set_grad_clip(llm_ctx *c, float max_norm) {
+  if (!c || max_norm != max_norm) return LLM_ERR_ARG;
+  const float v = max_norm > 0.f ? max_norm : 0.f;
+  if (v != c->clip) {
+    // the threshold is baked into a captured step: drop the graph
+    if (c->gexec) {
+      if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+      cudaGraphExecDestroy(c->gexec);
+      c->gexec = nullptr;
+    }
+    c->have_prev = false;
+    c->clip = v;
+  }
+  return LLM_OK;
+}
+
+int llm_read_grad_norm(llm_ctx *c, double *norm) {
+  if (!c || !norm || !c->have_norm) return LLM_ERR_ARG;
+  if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+  if (cudaMemcpy(norm, c->clip_norm, sizeof(double), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LLM_ERR_CUDA;
+  return LLM_OK;
+}
+
+int llm_lr_at(const llm_lr_schedule *sc, int64_t t, float *lr) {
+  if (!sc || !lr || t < 1 || sc->warmup_steps < 0 || sc->decay_start < sc->warmup_steps)
+    return LLM_ERR_ARG;
+  if (sc->shape != LLM_LR_CONSTANT && sc->shape != LLM_LR_COSINE && sc->shape != LLM_LR_LINEAR)
+    return LLM_ERR_ARG;
+  if (!std::isfinite(sc->max_lr) || !std::isfinite(sc->min_lr)) return LLM_ERR_ARG;
+  const double mx = sc->max_lr, mn = sc->min_lr;
+  double v;
+  if (sc->warmup_steps > 0 && t <= sc->warmup_steps) {
+    v = mx * (double)t / (double)sc->warmup_steps;
+  } else if (t <= sc->decay_start || sc->shape == LLM_LR_CONSTANT) {
+    v = mx;
+  } else {
+    double p = 1.0;
+    if (sc->total_steps > sc->decay_start)
+      p = std::min(1.0, (double)(t - sc->decay_start) /
+                            (double)(sc->total_steps - sc->decay_start));
+    v = sc->shape == LLM_LR_COSINE ? mn + (mx - mn) * (1.0 + cos(M_PI * p)) / 2.0
+                                   : mx + (mn - mx) * p;
+  }
+  *lr = (float)v;
   return LLM_OK;
 }
 
@@ -704,10 +761,13 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
                   c->flag_step, c->s);
     loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
     backward(c, d_params, d_grads, d_tokens);
+    if (c->clip > 0.f)
+      clip_grads(d_grads, D.P, c->clip, c->clip_part, c->clip_norm, c->clip_scale, c->s);
     adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2,
           c->cfg.adam_eps, c->flag_step, c->s);
     or_flag(c->flag_step, c->flag_sticky, c->s);
   };
+  if (c->clip > 0.f) c->have_norm = true;
   const llm_ctx::Key key{{d_params, d_grads, d_m, d_v, d_tokens, d_targets, d_loss}};
   // graphs need a capturable stream (not the legacy default stream); steps
   // with kernel timing on run as individual launches

@@ -90,6 +90,16 @@ class LlamaStep:
                 "llm_sample")
         return out
 
+    def set_grad_clip(self, max_norm):
+        """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
+        L.check(L.lib.llm_set_grad_clip(self.ctx, float(max_norm)), "llm_set_grad_clip")
+
+    def read_grad_norm(self):
+        """Gradient norm before clipping of the last clipped step (llm_read_grad_norm)."""
+        v = C.c_double(0.0)
+        L.check(L.lib.llm_read_grad_norm(self.ctx, C.byref(v)), "llm_read_grad_norm")
+        return v.value
+
     def status(self):
         return L.lib.llm_status(self.ctx)
 

@@ -33,13 +33,16 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / nb)
 
 
-def run_gpu(cfg, params, tok, tgt, steps=1, lr=None, wd=None):
+def run_gpu(cfg, params, tok, tgt, steps=1, lr=None, wd=None, clip=None):
     """Returns dict with logits (pre-step forward), and per step: loss, grads,
-    params, m, v (numpy float64)."""
+    params, m, v (numpy float64), and with clip (global-norm clipping
+    threshold) the norm before clipping."""
     from scratch_llama_decoder_b200 import LlamaStep
     lr = cfg["lr"] if lr is None else lr
     wd = cfg["wd"] if wd is None else wd
     m = LlamaStep(cfg)
+    if clip is not None:
+        m.set_grad_clip(clip)
     P = torch.tensor(params, dtype=torch.float32, device="cuda")
     G = torch.zeros_like(P)
     M = torch.zeros_like(P)
@@ -54,14 +57,16 @@ def run_gpu(cfg, params, tok, tgt, steps=1, lr=None, wd=None):
         st = m.status()
         out["steps"].append(dict(status=st, loss=float(loss.item()),
                                  grads=G.double().cpu().numpy(), params=P.double().cpu().numpy(),
-                                 m=M.double().cpu().numpy(), v=V.double().cpu().numpy()))
+                                 m=M.double().cpu().numpy(), v=V.double().cpu().numpy(),
+                                 norm=m.read_grad_norm() if clip is not None else None))
     out["launches"] = m.last_launch_count()
     m.close()
     return out
 
 
-def run_oracle(cfg, params, tok, tgt, steps=1, lr=None, wd=None):
+def run_oracle(cfg, params, tok, tgt, steps=1, lr=None, wd=None, clip=None):
     import oracle as O
+    from oracle import train_terms as TT
     lr = cfg["lr"] if lr is None else lr
     wd = cfg["wd"] if wd is None else wd
     p = np.asarray(params, np.float64)
@@ -71,8 +76,12 @@ def run_oracle(cfg, params, tok, tgt, steps=1, lr=None, wd=None):
     out = {"logits": logits, "steps": []}
     for t in range(1, steps + 1):
         loss, _, g = O.forward_backward(cfg, p, tok, tgt, want_logits=False)
+        norm = None
+        if clip is not None:
+            g, norm, _ = TT.clip(g, clip)
         p, m, v = O.adamw(p, g, m, v, t, lr, wd, cfg["beta1"], cfg["beta2"], cfg["adam_eps"])
-        out["steps"].append(dict(loss=loss, grads=g, params=p.copy(), m=m.copy(), v=v.copy()))
+        out["steps"].append(dict(loss=loss, grads=g, params=p.copy(), m=m.copy(), v=v.copy(),
+                                 norm=norm))
     return out
 
 

@@ -1,0 +1,46 @@
+"""llm_lr_at (host-only C ABI) against the float64 schedule of the oracle:
+equal to within float32 rounding at every step of several schedules, and
+invalid arguments rejected.  Runs without a GPU (the library loads on the
+host; the schedule launches nothing)."""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+from oracle import train_terms as TT
+
+SCHEDULES = [
+    # max_lr, min_lr, warmup, decay_start, total, shape
+    (3e-4, 3e-5, 100, 100, 1000, "cosine"),   # linear warm-up, then cosine
+    (1e-4, 1e-5, 0, 600, 1000, "cosine"),     # randyGPT: hold, cosine over the final 40%
+    (1e-3, 0.0, 10, 50, 300, "linear"),
+    (2e-4, 1e-6, 7, 7, 7, "cosine"),          # total <= decay start: min_lr after warm-up
+    (5e-4, 5e-5, 0, 0, 64, "constant"),
+]
+
+
+@pytest.mark.parametrize("sched", SCHEDULES)
+def test_lr_at_matches_oracle(sched):
+    import scratch_llama_decoder_b200 as P
+    mx, mn, W, S, T, shape = sched
+    for t in list(range(1, T + 40)):
+        got = P.lr_at(t, mx, mn, W, S, T, shape)
+        want = np.float32(TT.lr_at(t, float(np.float32(mx)), float(np.float32(mn)), W, S, T,
+                                   shape))
+        assert got == pytest.approx(float(want), rel=1.2e-7, abs=1e-30), (t, got, want)
+
+
+def test_lr_at_rejects_bad_arguments():
+    import scratch_llama_decoder_b200 as P
+    from scratch_llama_decoder_b200._lib import llm_lr_schedule
+    out = C.c_float(0.0)
+    bad = [
+        (llm_lr_schedule(1e-3, 1e-4, 10, 10, 100, 1), 0),       # t < 1
+        (llm_lr_schedule(1e-3, 1e-4, -1, 10, 100, 1), 1),       # negative warm-up
+        (llm_lr_schedule(1e-3, 1e-4, 10, 5, 100, 1), 1),        # decay before warm-up ends
+        (llm_lr_schedule(1e-3, 1e-4, 10, 10, 100, 7), 1),       # unknown shape
+        (llm_lr_schedule(float("nan"), 1e-4, 10, 10, 100, 1), 1),
+    ]
+    for sc, t in bad:
+        assert P.lib.llm_lr_at(C.byref(sc), t, C.byref(out)) == P.LLM_ERR_ARG
+    assert P.lib.llm_lr_at(None, 1, C.byref(out)) == P.LLM_ERR_ARG
