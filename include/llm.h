@@ -129,6 +129,30 @@ int llm_step(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d
              const int32_t *d_tokens, const int32_t *d_targets, float lr, float wd,
              float *d_loss);
 
+/* llm_step in two halves, for data parallelism with one process per GPU and
+ * the batch split across ranks (each rank a context over its share):
+ *   llm_grad:  the step's forward, loss and backward without the update:
+ *              d_grads = d loss / d params and d_loss = the mean loss over
+ *              this context's batch*ctx positions.
+ *   llm_adamw: the step's update: d_grads *= grad_scale in place (1/ranks after
+ *              a summing all-reduce turns the sum of the ranks' mean gradients
+ *              into the mean over the whole batch), then global-norm clipping
+ *              when llm_set_grad_clip is on, then AdamW as in llm_step.  It is
+ *              skipped (params, m, v untouched) when the error word holds an
+ *              error: the word the last llm_grad set, ORed with llm_flag_in.
+ *   llm_flag_out copies that int32 error word (0 = none) to d_flag (device);
+ *   llm_flag_in ORs d_flag into it, so ranks that all-reduce their words (MAX)
+ *   skip or take the update together.
+ * llm_grad then llm_adamw(grad_scale = 1) gives llm_step's results bit for
+ * bit.  These run as individual launches (no graph).  LLM_ERR_ARG for null or
+ * misaligned (16-byte) buffers, t < 1 or a non-finite grad_scale. */
+int llm_grad(llm_ctx *ctx, const float *d_params, float *d_grads, const int32_t *d_tokens,
+             const int32_t *d_targets, float *d_loss);
+int llm_adamw(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,
+              float lr, float wd, float grad_scale);
+int llm_flag_out(llm_ctx *ctx, int32_t *d_flag);
+int llm_flag_in(llm_ctx *ctx, const int32_t *d_flag);
+
 /* Single-token decode against a key/value cache (Hephaistos, feature list:
  * "True KV Cache", the prompt is processed once and every later position
  * costs one pass over a single row per sequence; strata, model table: the

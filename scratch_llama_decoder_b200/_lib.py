@@ -54,6 +54,10 @@ EXPORTS = {
     "llm_init": (_i, [_vp, _u64, _f, _i, _vp]),
     "llm_forward": (_i, [_vp, _vp, _vp, _vp]),
     "llm_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _f, _f, _vp]),
+    "llm_grad": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "llm_adamw": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _f, _f, _f]),
+    "llm_flag_out": (_i, [_vp, _vp]),
+    "llm_flag_in": (_i, [_vp, _vp]),
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
     "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),
     "llm_set_grad_clip": (_i, [_vp, _f]),

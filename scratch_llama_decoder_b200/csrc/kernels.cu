@@ -1099,6 +1099,23 @@ __global__ void __launch_bounds__(CLIP_THREADS)
   }
   if (blockIdx.x == 0 && threadIdx.x < (int)(n & 3)) g[n4 * 4 + threadIdx.x] *= sc;
 }
+// g *= sc (the mean of summed gradients: sc = 1 / ranks)
+__global__ void __launch_bounds__(CLIP_THREADS)
+    k_scale_grads_by(float *__restrict__ g, int64_t n, float sc) {
+  const int64_t n4 = n / 4;
+  float4 *g4 = reinterpret_cast<float4 *>(g);
+  for (int64_t i = blockIdx.x * (int64_t)CLIP_THREADS + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * CLIP_THREADS) {
+    float4 v = g4[i];
+    v.x *= sc; v.y *= sc; v.z *= sc; v.w *= sc;
+    g4[i] = v;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (int)(n & 3)) g[n4 * 4 + threadIdx.x] *= sc;
+}
+void scale_grads(float *g, int64_t n, float sc, cudaStream_t s) {
+  k_scale_grads_by<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, sc);
+  count_launch();
+}
 int clip_part_blocks() { return CLIP_BLOCKS; }
 void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm, float *scale,
                 cudaStream_t s) {

@@ -811,6 +811,60 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
 
+int llm_grad(llm_ctx *c, const float *d_params, float *d_grads, const int32_t *d_tokens,
+             const int32_t *d_targets, float *d_loss) {
+  if (!c || !d_tokens || !d_targets || !d_loss) return LLM_ERR_ARG;
+  if (!aligned16(d_params) || !aligned16(d_grads)) return LLM_ERR_ARG;
+  const Dims &D = c->D;
+  g_launches = 0;
+  set_flag_zero(c->flag_step, c->s);
+  forward(c, d_params, d_tokens);
+  cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
+                c->flag_step, c->s);
+  loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
+  backward(c, d_params, d_grads, d_tokens);
+  or_flag(c->flag_step, c->flag_sticky, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_adamw(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,
+              float lr, float wd, float grad_scale) {
+  if (!c || t < 1 || !std::isfinite(grad_scale)) return LLM_ERR_ARG;
+  if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
+    return LLM_ERR_ARG;
+  const Dims &D = c->D;
+  g_launches = 0;
+  const double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
+  const double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
+  set_hyper(c->hyper, lr, wd, (float)bc1, (float)bc2, c->s);
+  if (grad_scale != 1.0f) scale_grads(d_grads, D.P, grad_scale, c->s);
+  if (c->clip > 0.f) {
+    clip_grads(d_grads, D.P, c->clip, c->clip_part, c->clip_norm, c->clip_scale, c->s);
+    c->have_norm = true;
+  }
+  adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps,
+        c->flag_step, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_flag_out(llm_ctx *c, int32_t *d_flag) {
+  if (!c || !d_flag) return LLM_ERR_ARG;
+  if (cudaMemcpyAsync(d_flag, c->flag_step, sizeof(int32_t), cudaMemcpyDeviceToDevice, c->s) !=
+      cudaSuccess)
+    return LLM_ERR_CUDA;
+  return LLM_OK;
+}
+
+int llm_flag_in(llm_ctx *c, const int32_t *d_flag) {
+  if (!c || !d_flag) return LLM_ERR_ARG;
+  g_launches = 0;
+  or_flag(d_flag, c->flag_step, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
 int llm_decode(llm_ctx *c, const float *d_params, const int32_t *d_tokens, int pos,
                float *d_logits) {
   if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;

@@ -71,6 +71,27 @@ class LlamaStep:
                 "llm_step")
         return loss
 
+    def grad(self, params, grads, tokens, targets, loss=None):
+        """Forward, loss and backward without the update (llm_grad)."""
+        if loss is None:
+            loss = torch.empty(1, dtype=torch.float32, device=self.device)
+        L.check(L.lib.llm_grad(self.ctx, _ptr(params), _ptr(grads), _ptr(tokens), _ptr(targets),
+                               _ptr(loss)), "llm_grad")
+        return loss
+
+    def adamw(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
+        """grads *= grad_scale, optional clipping, AdamW (llm_adamw)."""
+        L.check(L.lib.llm_adamw(self.ctx, _ptr(params), _ptr(grads), _ptr(m), _ptr(v), int(t),
+                                float(lr), float(wd), float(grad_scale)), "llm_adamw")
+
+    def flag_out(self, flag):
+        """Copy the step's int32 error word to flag (llm_flag_out)."""
+        L.check(L.lib.llm_flag_out(self.ctx, _ptr(flag)), "llm_flag_out")
+
+    def flag_in(self, flag):
+        """OR the int32 word flag into the step's error word (llm_flag_in)."""
+        L.check(L.lib.llm_flag_in(self.ctx, _ptr(flag)), "llm_flag_in")
+
     def decode(self, params, tokens, pos, logits=None):
         """Logits [B, V] of position pos (llm_decode); tokens: int32 [B]."""
         B, V = self.cfg["batch"], self.cfg["vocab"]

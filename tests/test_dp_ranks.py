@@ -1,0 +1,146 @@
+"""The data-parallel step's host logic on CPU: two gloo ranks (spawned
+processes, rendezvous on 127.0.0.1), each with half of the batch, driven
+through DataParallelStep with an engine that computes on the float64 oracle.
+Two ranks must give the single-process step on the whole batch (the mean of
+the ranks' mean gradients is the batch-mean gradient when the shares are
+equal), and an error on one rank must make both skip the update."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+class OracleEngine:
+    """grad / adamw / flag_out / flag_in of the C ABI, computed by the oracle
+    on float64 CPU tensors."""
+    device = torch.device("cpu")
+
+    def __init__(self, cfg, fail_at=None):
+        self.cfg = cfg
+        self.flag = 0
+        self.fail_at = fail_at
+        self.calls = 0
+
+    def grad(self, params, grads, tokens, targets, loss):
+        import oracle as O
+        self.calls += 1
+        lv, _, g = O.forward_backward(self.cfg, params.numpy(), tokens.numpy(), targets.numpy(),
+                                      want_logits=False)
+        grads.copy_(torch.from_numpy(g))
+        loss.fill_(lv)
+        self.flag = 1 if self.calls == self.fail_at else 0
+
+    def flag_out(self, f):
+        f.fill_(self.flag)
+
+    def flag_in(self, f):
+        self.flag |= int(f.item())
+
+    def adamw(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
+        import oracle as O
+        grads.mul_(grad_scale)
+        if self.flag:
+            return
+        p2, m2, v2 = O.adamw(params.numpy(), grads.numpy(), m.numpy(), v.numpy(), t, lr, wd)
+        params.copy_(torch.from_numpy(p2))
+        m.copy_(torch.from_numpy(m2))
+        v.copy_(torch.from_numpy(v2))
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _setup(full_cfg):
+    import oracle as O
+    from synth import make_batch, make_params
+    p = make_params(full_cfg, O.param_layout(full_cfg)).astype(np.float64)
+    tok, tgt = make_batch(full_cfg)
+    return p, tok.reshape(full_cfg["batch"], -1), tgt.reshape(full_cfg["batch"], -1)
+
+
+def _run(engine, dp, p, tok, tgt, steps, lr, wd):
+    P = torch.tensor(p)
+    G, M, V = (torch.zeros_like(P) for _ in range(3))
+    loss = torch.zeros(1, dtype=torch.float64)
+    losses = []
+    for t in range(1, steps + 1):
+        dp.step(P, G, M, V, t, torch.tensor(tok), torch.tensor(tgt), lr, wd, loss)
+        losses.append(float(loss.item()))
+    return P.numpy(), M.numpy(), V.numpy(), losses
+
+
+def _rank_main(rank, world, port, full_cfg, steps, fail_rank, fail_at, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        p, tok, tgt = _setup(full_cfg)
+        share = full_cfg["batch"] // world
+        cfg = dict(full_cfg, batch=share)
+        eng = OracleEngine(cfg, fail_at=fail_at if rank == fail_rank else None)
+        dp = DataParallelStep(eng)
+        out = _run(eng, dp, p, tok[rank * share:(rank + 1) * share],
+                   tgt[rank * share:(rank + 1) * share], steps, full_cfg["lr"], full_cfg["wd"])
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+def _two_ranks(full_cfg, steps, fail_rank=-1, fail_at=None):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, full_cfg, steps, fail_rank, fail_at, q))
+             for r in range(2)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=300) for _ in range(2))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    return res
+
+
+def test_two_ranks_equal_one_process_on_the_whole_batch():
+    from synth import get_config
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    full = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_head=2, d_ff=42,
+                      ctx=5, batch=2, init_std=0.3, name="gqa-small", index=9)
+    res = _two_ranks(full, steps=3)
+    p, tok, tgt = _setup(full)
+    # DataParallelStep with one rank (no process group) is the plain step
+    eng = OracleEngine(full)
+    ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 3, full["lr"], full["wd"])
+    for r in (0, 1):
+        P, M, V, losses = res[r]
+        np.testing.assert_allclose(P, ref[0], rtol=1e-12, atol=1e-15)
+        np.testing.assert_allclose(M, ref[1], rtol=1e-10, atol=1e-18)
+        np.testing.assert_allclose(V, ref[2], rtol=1e-10, atol=1e-22)
+        # the summed mean losses over 2 ranks = 2 x the batch-mean loss
+        np.testing.assert_allclose(np.array(losses) / 2, ref[3], rtol=1e-12)
+    np.testing.assert_array_equal(res[0][0], res[1][0])  # the ranks agree bit for bit
+
+
+def test_an_error_on_one_rank_skips_the_update_on_both():
+    from synth import get_config
+    full = get_config("c1", batch=2)
+    res = _two_ranks(full, steps=2, fail_rank=1, fail_at=2)
+    res_ok = _two_ranks(full, steps=1)
+    for r in (0, 1):
+        # step 2 was skipped everywhere: parameters stay at their step-1 values
+        np.testing.assert_array_equal(res[r][0], res_ok[r][0])
