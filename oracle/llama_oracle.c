@@ -46,6 +46,46 @@ typedef struct {
   double rope_base, eps;
 } orc_cfg;
 
+/* ----------------------------------------------------------------- dropout */
+/* Inverted dropout (Hephaistos, Architecture at a glance: dropout on the
+ * embeddings, the attention weights and the attention and MLP outputs; masks
+ * drawn by the training forward and reused by its backward).  The masks come
+ * from Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+ * easy as 1, 2, 3", SC 2011): key = the seed's two 32-bit halves, counter =
+ * (element index low word, element index high word, site + 4 * layer, step),
+ * with sites 0 embedding output [B*T, d], 1 attention probabilities
+ * [B, H, T, T], 2 attention branch output [B*T, d], 3 MLP branch output
+ * [B*T, d] (element index row-major over those shapes).  An element is kept
+ * when the first output word is >= floor(p * 2^32); kept elements are scaled
+ * by 1 / (1 - p). */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3], k0 = key[0], k1 = key[1];
+  for (int r = 0; r < 10; r++) {
+    uint64_t p0 = (uint64_t)0xD2511F53u * c0, p1 = (uint64_t)0xCD9E8D57u * c2;
+    uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n1 = (uint32_t)p1;
+    uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1, n3 = (uint32_t)p0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+typedef struct {
+  double p;       /* drop probability in [0, 1) */
+  uint64_t seed;
+  uint32_t step;  /* training forward number */
+} orc_dropout;
+
+/* 0 or 1/(1-p) for element e of (site, layer) */
+static double drop_factor(const orc_dropout *dr, int site, int layer, uint64_t e) {
+  uint32_t ctr[4] = {(uint32_t)e, (uint32_t)(e >> 32), (uint32_t)(site + 4 * layer), dr->step};
+  uint32_t key[2] = {(uint32_t)dr->seed, (uint32_t)(dr->seed >> 32)}, out[4];
+  orc_philox4x32_10(ctr, key, out);
+  const uint64_t thr = (uint64_t)floor(dr->p * 4294967296.0);
+  return (uint64_t)out[0] >= thr ? 1.0 / (1.0 - dr->p) : 0.0;
+}
+
 /* ------------------------------------------------------------------ layout */
 /* Flat parameter buffer ("Hephaistos", Design notes: flat buffers, named
  * offsets).  Order: wte[V,d]; per layer g1[d], Wqkv[d, d+2kvd], Wo[d,d], g2[d],
@@ -190,8 +230,16 @@ void orc_rope(double *u, int hd, int t, double base, int sign) {
  * heads), RoPE already applied.  o is [T, d] (heads concatenated).
  * lse[H,T] (optional) is the log-sum-exp of each score row; P[H,T,T]
  * (optional) receives the probabilities (zero above the diagonal). */
+static void attention_fwd_do(int T, int d, int H, int Hkv, const double *qkv, double *o,
+                             double *lse, double *P, const orc_dropout *dr, int layer, int b);
 void orc_attention_fwd(int T, int d, int H, int Hkv, const double *qkv, double *o, double *lse,
                        double *P) {
+  attention_fwd_do(T, d, H, Hkv, qkv, o, lse, P, NULL, 0, 0);
+}
+/* With dr: o_i = sum_j P_ij f_ij v_j, f the dropout factor of probability
+ * (b, head, i, j); P and lse stay the undropped softmax. */
+static void attention_fwd_do(int T, int d, int H, int Hkv, const double *qkv, double *o,
+                             double *lse, double *P, const orc_dropout *dr, int layer, int b) {
   int hd = d / H, grp = H / Hkv;
   int64_t w = (int64_t)d + 2LL * hd * Hkv;
   double scale = 1.0 / sqrt((double)hd);
@@ -216,7 +264,9 @@ void orc_attention_fwd(int T, int d, int H, int Hkv, const double *qkv, double *
       for (int j = 0; j <= i; j++) {
         double p = s[j] / sum;
         const double *v = qkv + (int64_t)j * w + d + (int64_t)hd * Hkv + (int64_t)g * hd;
-        for (int e = 0; e < hd; e++) oi[e] += p * v[e];
+        const double pd =
+            dr ? p * drop_factor(dr, 1, layer, (((uint64_t)b * H + hq) * T + i) * T + j) : p;
+        for (int e = 0; e < hd; e++) oi[e] += pd * v[e];
         if (P) P[((int64_t)hq * T + i) * T + j] = p;
       }
       if (P) for (int j = i + 1; j < T; j++) P[((int64_t)hq * T + i) * T + j] = 0.0;
@@ -231,13 +281,32 @@ void orc_attention_fwd(int T, int d, int H, int Hkv, const double *qkv, double *
  * dS = P (dP - rowsum(dP P)); dq = dS k / sqrt(hd); dk = dS^T q / sqrt(hd).
  * GQA: dk and dv sum over the query heads of the group, in head order.
  * dqkv [T, d+2kvd] is written. */
+static void attention_bwd_do(int T, int d, int H, int Hkv, const double *qkv,
+                             const double *dout, double *dqkv, const orc_dropout *dr, int layer,
+                             int b);
 void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const double *dout,
                        double *dqkv) {
+  attention_bwd_do(T, d, H, Hkv, qkv, dout, dqkv, NULL, 0, 0);
+}
+/* With dr (the mask of attention_fwd_do): dv_j = sum_i P_ij f_ij do_i;
+ * dP_ij = f_ij (do_i . v_j); dS = P (dP - rowsum(dP P)). */
+static void attention_bwd_do(int T, int d, int H, int Hkv, const double *qkv,
+                             const double *dout, double *dqkv, const orc_dropout *dr, int layer,
+                             int b) {
   int hd = d / H, grp = H / Hkv;
   int64_t w = (int64_t)d + 2LL * hd * Hkv;
   double scale = 1.0 / sqrt((double)hd);
   double *P = (double *)calloc((size_t)H * T * T, sizeof(double));
   double *dS = (double *)calloc((size_t)H * T * T, sizeof(double));
+  double *F = NULL; /* dropout factors [H, T, T] */
+  if (dr) {
+    F = (double *)calloc((size_t)H * T * T, sizeof(double));
+    for (int hq = 0; hq < H; hq++)
+      for (int i = 0; i < T; i++)
+        for (int j = 0; j <= i; j++)
+          F[((int64_t)hq * T + i) * T + j] =
+              drop_factor(dr, 1, layer, (((uint64_t)b * H + hq) * T + i) * T + j);
+  }
   memset(dqkv, 0, sizeof(double) * (size_t)T * w);
   /* P and dS, one (query head, row) per iteration */
 #pragma omp parallel for collapse(2) schedule(static) if ((int64_t)H * T * T * hd > OMP_MIN_WORK)
@@ -263,6 +332,7 @@ void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const do
         const double *v = qkv + (int64_t)j * w + d + (int64_t)hd * Hkv + (int64_t)g * hd;
         double dp = 0.0;
         for (int e = 0; e < hd; e++) dp += doi[e] * v[e];
+        if (F) dp *= F[((int64_t)hq * T + i) * T + j];
         dSi[j] = dp;
         rs += dp * Pi[j];
       }
@@ -287,6 +357,7 @@ void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const do
           const double *q = qkv + (int64_t)i * w + (int64_t)hq * hd;
           const double *doi = dout + (int64_t)i * d + (int64_t)hq * hd;
           double ds = dS[((int64_t)hq * T + i) * T + j], p = P[((int64_t)hq * T + i) * T + j];
+          if (F) p *= F[((int64_t)hq * T + i) * T + j];
           for (int e = 0; e < hd; e++) {
             dk[e] += ds * q[e] * scale;
             dv[e] += p * doi[e];
@@ -297,6 +368,7 @@ void orc_attention_bwd(int T, int d, int H, int Hkv, const double *qkv, const do
   }
   free(P);
   free(dS);
+  free(F);
 }
 
 /* ------------------------------------------------------------------ SwiGLU */
@@ -364,8 +436,28 @@ typedef struct {
 /* Forward (and optionally backward) of one sequence.  Logits are written to
  * logits_out[T,V] if non-null; grads (if non-null) are accumulated with the
  * loss scale inv_count.  Returns the sum of this sequence's row losses. */
+/* out[t, j] = x[t, j] + f(site, layer, (b*T + t)*d + j) * y[t, j] */
+static void add_dropped(const orc_dropout *dr, int site, int layer, int b, int T, int d,
+                        const double *x, const double *y, double *out) {
+  for (int t = 0; t < T; t++)
+    for (int j = 0; j < d; j++) {
+      const int64_t i = (int64_t)t * d + j;
+      out[i] = x[i] + drop_factor(dr, site, layer, ((uint64_t)b * T + t) * d + j) * y[i];
+    }
+}
+/* dy[t, j] = f(site, layer, (b*T + t)*d + j) * dx[t, j] */
+static void mask_rows(const orc_dropout *dr, int site, int layer, int b, int T, int d,
+                      const double *dx, double *dy) {
+  for (int t = 0; t < T; t++)
+    for (int j = 0; j < d; j++) {
+      const int64_t i = (int64_t)t * d + j;
+      dy[i] = drop_factor(dr, site, layer, ((uint64_t)b * T + t) * d + j) * dx[i];
+    }
+}
+
 static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, const int32_t *tgt,
-                       double inv_count, double *logits_out, double *grads) {
+                       double inv_count, double *logits_out, double *grads,
+                       const orc_dropout *dr, int bseq) {
   const int T = c->T, d = c->d, L = c->L, H = c->H, Hkv = c->Hkv, h = c->h, V = c->V;
   const int hd = d / H;
   const int64_t w = qkvw(c);
@@ -374,6 +466,8 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
   /* embedding gather (Hephaistos: token embedding, no positional table) */
   for (int t = 0; t < T; t++)
     memcpy(x + (int64_t)t * d, p + (int64_t)tok[t] * d, sizeof(double) * d);
+  if (dr) mask_rows(dr, 0, 0, bseq, T, d, x, x);
+  double *ybr = dr ? (double *)malloc(sizeof(double) * (size_t)T * d) : NULL;
   for (int l = 0; l < L; l++) {
     layer_acts *A = &acts[l];
     A->x = x;
@@ -394,9 +488,14 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
       for (int hq = 0; hq < H; hq++) orc_rope(A->qkv + (int64_t)t * w + (int64_t)hq * hd, hd, t, c->rope_base, 1);
       for (int g = 0; g < Hkv; g++) orc_rope(A->qkv + (int64_t)t * w + d + (int64_t)g * hd, hd, t, c->rope_base, 1);
     }
-    orc_attention_fwd(T, d, H, Hkv, A->qkv, A->o, NULL, NULL);
-    memcpy(A->x1, A->x, sizeof(double) * (size_t)T * d);
-    orc_mm_nn(T, d, d, A->o, d, p + off_wo(c, l), d, A->x1, d, 1);
+    attention_fwd_do(T, d, H, Hkv, A->qkv, A->o, NULL, NULL, dr, l, bseq);
+    if (dr) {
+      orc_mm_nn(T, d, d, A->o, d, p + off_wo(c, l), d, ybr, d, 0);
+      add_dropped(dr, 2, l, bseq, T, d, A->x, ybr, A->x1);
+    } else {
+      memcpy(A->x1, A->x, sizeof(double) * (size_t)T * d);
+      orc_mm_nn(T, d, d, A->o, d, p + off_wo(c, l), d, A->x1, d, 1);
+    }
     /* x2 = x1 + SwiGLU(RMSNorm_g2(x1)) */
     orc_rmsnorm_fwd(T, d, A->x1, p + off_g2(c, l), c->eps, A->xn2, A->rstd2);
     const double *w13 = p + off_w13(c, l);
@@ -404,8 +503,13 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
     orc_mm_nn(T, d, h, A->xn2, d, w13 + h, 2LL * h, A->b, h, 0);
     orc_swiglu_fwd((int64_t)T * h, A->a, A->b, A->u);
     double *x2 = (double *)malloc(sizeof(double) * (size_t)T * d);
-    memcpy(x2, A->x1, sizeof(double) * (size_t)T * d);
-    orc_mm_nn(T, h, d, A->u, h, p + off_w2(c, l), d, x2, d, 1);
+    if (dr) {
+      orc_mm_nn(T, h, d, A->u, h, p + off_w2(c, l), d, ybr, d, 0);
+      add_dropped(dr, 3, l, bseq, T, d, A->x1, ybr, x2);
+    } else {
+      memcpy(x2, A->x1, sizeof(double) * (size_t)T * d);
+      orc_mm_nn(T, h, d, A->u, h, p + off_w2(c, l), d, x2, d, 1);
+    }
     x = x2;
   }
   /* final RMSNorm, untied lm_head, cross-entropy */
@@ -433,9 +537,15 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
     double *dqkv = (double *)malloc(sizeof(double) * (size_t)T * w);
     for (int l = L - 1; l >= 0; l--) {
       layer_acts *A = &acts[l];
-      /* dx holds d loss / d x2 (layer output). FFN branch: */
-      orc_mm_tn(h, T, d, A->u, h, dx, d, grads + off_w2(c, l), d, 1);
-      orc_mm_nt(T, d, h, dx, d, p + off_w2(c, l), d, du, h, 0);
+      /* dx holds d loss / d x2 (layer output). FFN branch (its output's
+       * gradient is dx through the dropout mask): */
+      const double *dyf = dx;
+      if (dr) {
+        mask_rows(dr, 3, l, bseq, T, d, dx, ybr);
+        dyf = ybr;
+      }
+      orc_mm_tn(h, T, d, A->u, h, dyf, d, grads + off_w2(c, l), d, 1);
+      orc_mm_nt(T, d, h, dyf, d, p + off_w2(c, l), d, du, h, 0);
       orc_swiglu_bwd((int64_t)T * h, A->a, A->b, du, da, db);
       double *g13 = grads + off_w13(c, l);
       const double *w13 = p + off_w13(c, l);
@@ -446,9 +556,14 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
       /* residual: dx1 = dx2 + RMSNorm_bwd(dxn) */
       orc_rmsnorm_bwd(T, d, A->x1, A->rstd2, p + off_g2(c, l), dxn, dx, grads + off_g2(c, l), 1);
       /* attention branch */
-      orc_mm_tn(d, T, d, A->o, d, dx, d, grads + off_wo(c, l), d, 1);
-      orc_mm_nt(T, d, d, dx, d, p + off_wo(c, l), d, dO, d, 0);
-      orc_attention_bwd(T, d, H, Hkv, A->qkv, dO, dqkv);
+      const double *dya = dx;
+      if (dr) {
+        mask_rows(dr, 2, l, bseq, T, d, dx, ybr);
+        dya = ybr;
+      }
+      orc_mm_tn(d, T, d, A->o, d, dya, d, grads + off_wo(c, l), d, 1);
+      orc_mm_nt(T, d, d, dya, d, p + off_wo(c, l), d, dO, d, 0);
+      attention_bwd_do(T, d, H, Hkv, A->qkv, dO, dqkv, dr, l, bseq);
       for (int t = 0; t < T; t++) {
         for (int hq = 0; hq < H; hq++) orc_rope(dqkv + (int64_t)t * w + (int64_t)hq * hd, hd, t, c->rope_base, -1);
         for (int g = 0; g < Hkv; g++) orc_rope(dqkv + (int64_t)t * w + d + (int64_t)g * hd, hd, t, c->rope_base, -1);
@@ -457,7 +572,9 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
       orc_mm_nt(T, (int)w, d, dqkv, w, p + off_wqkv(c, l), w, dxn, d, 0);
       orc_rmsnorm_bwd(T, d, A->x, A->rstd1, p + off_g1(c, l), dxn, dx, grads + off_g1(c, l), 1);
     }
-    /* embedding scatter-add: dwte[tok_t] += dx0_t, in token order */
+    /* embedding scatter-add: dwte[tok_t] += dx0_t, in token order (through
+     * the embedding dropout mask) */
+    if (dr) mask_rows(dr, 0, 0, bseq, T, d, dx, dx);
     for (int t = 0; t < T; t++) {
       double *gw = grads + (int64_t)tok[t] * d;
       for (int j = 0; j < d; j++) gw[j] += dx[(int64_t)t * d + j];
@@ -473,22 +590,43 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
   }
   free(x);
   if (L == 0) { /* x was never handed to a layer record */ }
-  free(xf); free(rstdf); free(z); free(dz); free(acts);
+  free(xf); free(rstdf); free(z); free(dz); free(acts); free(ybr);
   return loss;
 }
 
 /* Loss (mean over all B*T positions), logits[B*T, V] (optional) and grads[P]
  * (optional, overwritten) for tokens/targets [B, T] and params[P]. */
-double orc_forward_backward(const orc_cfg *c, const double *params, const int32_t *tokens,
-                            const int32_t *targets, double *logits, double *grads) {
+static double forward_backward(const orc_cfg *c, const double *params, const int32_t *tokens,
+                               const int32_t *targets, double *logits, double *grads,
+                               const orc_dropout *dr) {
   int64_t P = orc_n_params(c);
   int64_t N = (int64_t)c->B * c->T;
   if (grads) memset(grads, 0, sizeof(double) * (size_t)P);
   double total = 0.0;
   for (int b = 0; b < c->B; b++)
     total += seq_step(c, params, tokens + (int64_t)b * c->T, targets ? targets + (int64_t)b * c->T : NULL,
-                      1.0 / (double)N, logits ? logits + (int64_t)b * c->T * c->V : NULL, grads);
+                      1.0 / (double)N, logits ? logits + (int64_t)b * c->T * c->V : NULL, grads,
+                      dr, b);
   return total / (double)N;
+}
+double orc_forward_backward(const orc_cfg *c, const double *params, const int32_t *tokens,
+                            const int32_t *targets, double *logits, double *grads) {
+  return forward_backward(c, params, tokens, targets, logits, grads, NULL);
+}
+/* The training forward and backward with inverted dropout of rate p at the
+ * four sites (see orc_philox4x32_10 above); masks keyed by seed and step. */
+double orc_forward_backward_dropout(const orc_cfg *c, const double *params,
+                                    const int32_t *tokens, const int32_t *targets,
+                                    double *logits, double *grads, double p, uint64_t seed,
+                                    uint32_t step) {
+  orc_dropout dr = {p, seed, step};
+  return forward_backward(c, params, tokens, targets, logits, grads, &dr);
+}
+/* Dropout factors (0 or 1/(1-p)) of elements [e0, e0 + n) of (site, layer). */
+void orc_dropout_factors(double p, uint64_t seed, uint32_t step, int site, int layer,
+                         uint64_t e0, int64_t n, double *out) {
+  orc_dropout dr = {p, seed, step};
+  for (int64_t i = 0; i < n; i++) out[i] = drop_factor(&dr, site, layer, e0 + (uint64_t)i);
 }
 
 /* ------------------------------------------------------------------- AdamW */

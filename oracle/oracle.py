@@ -72,6 +72,15 @@ _lib.orc_embed_bwd.restype = None
 _lib.orc_embed_bwd.argtypes = [C.c_int64, C.c_int, C.c_int, _I32, _D, _D]
 _lib.orc_forward_backward.restype = C.c_double
 _lib.orc_forward_backward.argtypes = [C.POINTER(OrcCfg), _D, _I32, _I32, _D, _D]
+_lib.orc_forward_backward_dropout.restype = C.c_double
+_lib.orc_forward_backward_dropout.argtypes = [C.POINTER(OrcCfg), _D, _I32, _I32, _D, _D,
+                                              C.c_double, C.c_uint64, C.c_uint32]
+_lib.orc_philox4x32_10.restype = None
+_lib.orc_philox4x32_10.argtypes = [C.POINTER(C.c_uint32), C.POINTER(C.c_uint32),
+                                   C.POINTER(C.c_uint32)]
+_lib.orc_dropout_factors.restype = None
+_lib.orc_dropout_factors.argtypes = [C.c_double, C.c_uint64, C.c_uint32, C.c_int, C.c_int,
+                                     C.c_uint64, C.c_int64, _D]
 _lib.orc_adamw.restype = None
 _lib.orc_adamw.argtypes = [C.c_int64, _D, _D, _D, _D, C.c_int64, C.c_double, C.c_double,
                            C.c_double, C.c_double, C.c_double]
@@ -204,8 +213,27 @@ def embed_bwd(tok, dx, vocab):
     return out
 
 
-def forward_backward(cfg, params, tokens, targets=None, want_logits=True, want_grads=True):
-    """Returns (loss, logits [B*T, V] or None, grads [P] or None)."""
+def philox4x32_10(counter, key):
+    """Philox4x32-10 of four 32-bit counter words and two key words."""
+    c = (C.c_uint32 * 4)(*[int(x) & 0xffffffff for x in counter])
+    k = (C.c_uint32 * 2)(*[int(x) & 0xffffffff for x in key])
+    out = (C.c_uint32 * 4)()
+    _lib.orc_philox4x32_10(c, k, out)
+    return [int(x) for x in out]
+
+
+def dropout_factors(p, seed, step, site, layer, n, e0=0):
+    """Factors (0 or 1/(1-p)) of elements [e0, e0+n) of a dropout site."""
+    out = np.zeros(n)
+    _lib.orc_dropout_factors(float(p), int(seed), int(step), int(site), int(layer), int(e0),
+                             int(n), _dp(out))
+    return out
+
+
+def forward_backward(cfg, params, tokens, targets=None, want_logits=True, want_grads=True,
+                     dropout=None):
+    """Returns (loss, logits [B*T, V] or None, grads [P] or None).  dropout:
+    None or (p, seed, step) for the training forward with inverted dropout."""
     c = _cfg(cfg)
     params = _f64(params)
     tokens = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
@@ -214,8 +242,14 @@ def forward_backward(cfg, params, tokens, targets=None, want_logits=True, want_g
     assert tokens.size == N and params.size == n_params(cfg)
     logits = np.zeros((N, cfg["vocab"])) if want_logits else None
     grads = np.zeros(params.size) if (want_grads and tg is not None) else None
-    loss = _lib.orc_forward_backward(C.byref(c), _dp(params), _ip(tokens), _ip(tg), _dp(logits),
-                                     _dp(grads))
+    if dropout is None:
+        loss = _lib.orc_forward_backward(C.byref(c), _dp(params), _ip(tokens), _ip(tg),
+                                         _dp(logits), _dp(grads))
+    else:
+        pd, seed, stp = dropout
+        loss = _lib.orc_forward_backward_dropout(C.byref(c), _dp(params), _ip(tokens), _ip(tg),
+                                                 _dp(logits), _dp(grads), float(pd), int(seed),
+                                                 int(stp))
     return float(loss), logits, grads
 
 
