@@ -159,9 +159,10 @@ int llm_flag_in(llm_ctx *ctx, const int32_t *d_flag);
  * cache holds keys already rotated by RoPE, and decoding position by position
  * gives the full forward's logits).
  *
- * The cache is the context's own saved q|k|v activations: llm_forward (or
- * llm_step) over d_tokens [batch, ctx] fills positions 0..ctx-1 of every
- * sequence; that forward over a prompt in positions 0..p-1 is the prefill
+ * The cache is the context's own saved q|k|v activations: llm_forward over
+ * d_tokens [batch, ctx] fills positions 0..ctx-1 of every sequence (llm_step's
+ * forward does too, but with dropout on it holds a training forward's
+ * values); that forward over a prompt in positions 0..p-1 is the prefill
  * (positions >= p may hold any ids: causality keeps them out of positions
  * < p).  llm_decode then runs position pos for every sequence: d_tokens
  * [batch] holds each sequence's id at pos, the call writes that position's
@@ -228,6 +229,26 @@ int llm_lr_at(const llm_lr_schedule *sched, int64_t t, float *lr);
  * clipping off (the default).  A change frees the captured step graph
  * (synchronising the stream first).  LLM_ERR_ARG for NaN. */
 int llm_set_grad_clip(llm_ctx *ctx, float max_norm);
+
+/* Inverted dropout in the training forward and backward of llm_step and
+ * llm_grad (Hephaistos, Architecture at a glance: dropout on the embeddings,
+ * the attention weights and the attention and MLP outputs; masks drawn by the
+ * training forward and reused by its backward).  With 0 < p < 1 each element
+ * of the embedding output [B*T, d], the attention probabilities [B, H, T, T],
+ * and the attention and MLP branch outputs [B*T, d] (before their residual
+ * adds) is kept with probability 1 - p and scaled by 1 / (1 - p).  The masks
+ * come from Philox4x32-10 (Salmon et al., SC 2011): key = the seed's two
+ * 32-bit halves, counter = (element index low word, high word, site + 4 *
+ * layer, n) with sites 0 embedding, 1 attention probabilities, 2 attention
+ * output, 3 MLP output, element indices row-major over those shapes, n = the
+ * number of training calls (llm_step or llm_grad) since the last
+ * llm_set_dropout; an element is kept when the first output word is >=
+ * floor(p * 2^32).  llm_forward and llm_decode never drop.  While dropout is
+ * on, attention runs in the CUDA-core kernels (the tensor-core kernels draw no
+ * masks).  p = 0 turns it off (the default).  A changed setting frees the
+ * captured step graph; every call restarts n at 0.  LLM_ERR_ARG unless
+ * 0 <= p < 1. */
+int llm_set_dropout(llm_ctx *ctx, float p, uint64_t seed);
 
 /* Synchronises the context's stream and returns in *norm the gradient norm
  * (before clipping) of the most recent llm_step run with clipping on;

@@ -61,6 +61,7 @@ EXPORTS = {
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
     "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),
     "llm_set_grad_clip": (_i, [_vp, _f]),
+    "llm_set_dropout": (_i, [_vp, _f, _u64]),
     "llm_read_grad_norm": (_i, [_vp, C.POINTER(C.c_double)]),
     "llm_lr_at": (_i, [C.POINTER(llm_lr_schedule), _i64, C.POINTER(_f)]),
     "llm_status": (_i, [_vp]),

@@ -3,7 +3,9 @@
 // reference of the tensor-core kernels.  One warp per query row (forward, dq)
 // or per key row (dk, dv); the softmax is the online (running max and sum)
 // form of strata's flash-style attention, and only the row log-sum-exp is
-// saved for the backward.
+// saved for the backward.  With dropout (drop.on) the value sums use the
+// dropped probabilities P f while the softmax statistics stay those of P
+// (Hephaistos: inverted dropout on the attention weights).
 #include "common.cuh"
 #include "internal.h"
 
@@ -17,7 +19,8 @@ constexpr int MAXR = 4;  // head sizes up to 128 (4 values per lane)
 // s_ij = q_i . k_j / sqrt(hd) for j <= i; o_i = sum_j softmax_j(s_ij) v_j.
 template <typename A>
 __global__ void k_attn_fwd_simt(const A *__restrict__ qkv, A *__restrict__ o,
-                                float *__restrict__ lse, int B, int T, int H, int Hkv, int hd) {
+                                float *__restrict__ lse, int B, int T, int H, int Hkv, int hd,
+                                const DropArgs drop) {
   int64_t wid = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * H * T) return;
@@ -36,6 +39,8 @@ __global__ void k_attn_fwd_simt(const A *__restrict__ qkv, A *__restrict__ o,
     acc[r] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
+  const uint32_t step = drop.on ? (uint32_t)*drop.step : 0u;
+  const uint64_t erow = (((uint64_t)b * H + hq) * T + i) * T;
   for (int j = 0; j <= i; j++) {
     const A *kr = qkv + ((int64_t)b * T + j) * w + d + (int64_t)g * hd;
     const A *vr = kr + kvd;
@@ -49,10 +54,11 @@ __global__ void k_attn_fwd_simt(const A *__restrict__ qkv, A *__restrict__ o,
     float mn = fmaxf(m, s);
     float corr = expf(m - mn), p = expf(s - mn);
     l = l * corr + p;
+    const float pv = drop.on ? p * drop_factor(drop, erow + j, step) : p;
 #pragma unroll
     for (int r = 0; r < MAXR; r++) {
       int e = lane + 32 * r;
-      acc[r] = acc[r] * corr + ((e < hd) ? p * to_f(vr[e]) : 0.f);
+      acc[r] = acc[r] * corr + ((e < hd) ? pv * to_f(vr[e]) : 0.f);
     }
     m = mn;
   }
@@ -68,11 +74,13 @@ __global__ void k_attn_fwd_simt(const A *__restrict__ qkv, A *__restrict__ o,
 // Backward (strata: attention backward; P recomputed from the saved lse):
 // D_i = do_i . o_i; P_ij = exp(s_ij - lse_i); dP_ij = do_i . v_j;
 // dS_ij = P_ij (dP_ij - D_i); dq_i = sum_j dS_ij k_j / sqrt(hd).
+// With dropout, dP_ij = f_ij (do_i . v_j) and D_i = do_i . o_i still equals
+// sum_j P_ij dP_ij.
 template <typename A>
 __global__ void k_attn_bwd_dq_simt(const A *__restrict__ qkv, const A *__restrict__ o,
                                    const A *__restrict__ dout, const float *__restrict__ lse,
                                    float *__restrict__ Dbuf, A *__restrict__ dqkv, int B, int T,
-                                   int H, int Hkv, int hd) {
+                                   int H, int Hkv, int hd, const DropArgs drop) {
   int64_t wid = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * H * T) return;
@@ -99,6 +107,8 @@ __global__ void k_attn_bwd_dq_simt(const A *__restrict__ qkv, const A *__restric
   D = warp_sum(D);
   float L = lse[((int64_t)b * H + hq) * T + i];
   if (lane == 0) Dbuf[((int64_t)b * H + hq) * T + i] = D;
+  const uint32_t step = drop.on ? (uint32_t)*drop.step : 0u;
+  const uint64_t erow = (((uint64_t)b * H + hq) * T + i) * T;
   for (int j = 0; j <= i; j++) {
     const A *kr = qkv + ((int64_t)b * T + j) * w + d + (int64_t)g * hd;
     const A *vr = kr + kvd;
@@ -110,6 +120,7 @@ __global__ void k_attn_bwd_dq_simt(const A *__restrict__ qkv, const A *__restric
     }
     s = warp_sum(s) * scale;
     dp = warp_sum(dp);
+    if (drop.on) dp *= drop_factor(drop, erow + j, step);
     float p = expf(s - L);
     float ds = p * (dp - D) * scale;
 #pragma unroll
@@ -131,7 +142,8 @@ __global__ void k_attn_bwd_dq_simt(const A *__restrict__ qkv, const A *__restric
 template <typename A>
 __global__ void k_attn_bwd_dkv_simt(const A *__restrict__ qkv, const A *__restrict__ dout,
                                     const float *__restrict__ lse, const float *__restrict__ Dbuf,
-                                    A *__restrict__ dqkv, int B, int T, int H, int Hkv, int hd) {
+                                    A *__restrict__ dqkv, int B, int T, int H, int Hkv, int hd,
+                                    const DropArgs drop) {
   int64_t wid = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * Hkv * T) return;
@@ -151,6 +163,7 @@ __global__ void k_attn_bwd_dkv_simt(const A *__restrict__ qkv, const A *__restri
     v[r] = (e < hd) ? to_f(vr[e]) : 0.f;
     dk[r] = dv[r] = 0.f;
   }
+  const uint32_t step = drop.on ? (uint32_t)*drop.step : 0u;
   for (int hq = g * grp; hq < (g + 1) * grp; hq++) {
     for (int i = j; i < T; i++) {
       int64_t row = (int64_t)b * T + i;
@@ -170,11 +183,17 @@ __global__ void k_attn_bwd_dkv_simt(const A *__restrict__ qkv, const A *__restri
       dp = warp_sum(dp);
       int64_t li = ((int64_t)b * H + hq) * T + i;
       float p = expf(s - lse[li]);
+      float pv = p;  // the probability the forward multiplied v by
+      if (drop.on) {
+        const float f = drop_factor(drop, (uint64_t)li * T + j, step);
+        dp *= f;
+        pv = p * f;
+      }
       float ds = p * (dp - Dbuf[li]) * scale;
 #pragma unroll
       for (int r = 0; r < MAXR; r++) {
         dk[r] += ds * qv[r];
-        dv[r] += p * dov[r];
+        dv[r] += pv * dov[r];
       }
     }
   }
@@ -188,33 +207,35 @@ __global__ void k_attn_bwd_dkv_simt(const A *__restrict__ qkv, const A *__restri
 }
 
 void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
-                   int hd, cudaStream_t s) {
+                   int hd, cudaStream_t s, DropArgs drop) {
   int64_t warps = (int64_t)B * H * T;
   unsigned grid = (unsigned)((warps + 7) / 8);
   if (dt == DT_BF16)
     k_attn_fwd_simt<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, B, T,
-                                         H, Hkv, hd);
+                                         H, Hkv, hd, drop);
   else
-    k_attn_fwd_simt<<<grid, 256, 0, s>>>((const float *)qkv, (float *)o, lse, B, T, H, Hkv, hd);
+    k_attn_fwd_simt<<<grid, 256, 0, s>>>((const float *)qkv, (float *)o, lse, B, T, H, Hkv, hd,
+                                         drop);
   count_launch();
 }
 
 void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
-                   void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s) {
+                   void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s,
+                   DropArgs drop) {
   unsigned g1 = (unsigned)(((int64_t)B * H * T + 7) / 8);
   unsigned g2 = (unsigned)(((int64_t)B * Hkv * T + 7) / 8);
   if (dt == DT_BF16) {
     using T_ = __nv_bfloat16;
     k_attn_bwd_dq_simt<<<g1, 256, 0, s>>>((const T_ *)qkv, (const T_ *)o, (const T_ *)dout, lse,
-                                          Dbuf, (T_ *)dqkv, B, T, H, Hkv, hd);
+                                          Dbuf, (T_ *)dqkv, B, T, H, Hkv, hd, drop);
     k_attn_bwd_dkv_simt<<<g2, 256, 0, s>>>((const T_ *)qkv, (const T_ *)dout, lse, Dbuf,
-                                           (T_ *)dqkv, B, T, H, Hkv, hd);
+                                           (T_ *)dqkv, B, T, H, Hkv, hd, drop);
   } else {
     k_attn_bwd_dq_simt<<<g1, 256, 0, s>>>((const float *)qkv, (const float *)o,
                                           (const float *)dout, lse, Dbuf, (float *)dqkv, B, T, H,
-                                          Hkv, hd);
+                                          Hkv, hd, drop);
     k_attn_bwd_dkv_simt<<<g2, 256, 0, s>>>((const float *)qkv, (const float *)dout, lse, Dbuf,
-                                           (float *)dqkv, B, T, H, Hkv, hd);
+                                           (float *)dqkv, B, T, H, Hkv, hd, drop);
   }
   count_launch(2);
 }

@@ -36,3 +36,25 @@ LLM_DEV float sigmoidf_(float a) { return 1.0f / (1.0f + expf(-a)); }
 // at (j/64)*128 + j%64 and its W3 column 64 further.
 constexpr int SWIGLU_BLOCK = 64;
 __host__ __device__ __forceinline__ int64_t w1_col(int64_t j) { return (j / SWIGLU_BLOCK) * (2 * SWIGLU_BLOCK) + (j % SWIGLU_BLOCK); }
+
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+// as 1, 2, 3", SC 2011): ten rounds of two 32x32 -> 64-bit products with the
+// round keys bumped by the Weyl constants.
+LLM_DEV void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; r++) {
+    uint32_t hi0 = __umulhi(M0, c[0]), lo0 = M0 * c[0];
+    uint32_t hi1 = __umulhi(M1, c[2]), lo1 = M1 * c[2];
+    uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
+    k0 += W0; k1 += W1;
+  }
+}
+// 0 or a.scale for element e of the dropout site a (step: *a.step, read once
+// by the caller).
+LLM_DEV float drop_factor(const llm::DropArgs &a, uint64_t e, uint32_t step) {
+  uint32_t c[4] = {(uint32_t)e, (uint32_t)(e >> 32), a.site, step};
+  philox4x32_10(c, a.k0, a.k1);
+  return c[0] >= a.thr ? a.scale : 0.f;
+}

@@ -11,6 +11,19 @@ enum : int { FLAG_TOKEN = 1, FLAG_NONFINITE = 2, FLAG_TIMEOUT = 4 };
 // Activation/operand element type of a launch: float32 or bfloat16.
 enum DType { DT_F32 = 0, DT_BF16 = 1 };
 
+// Inverted-dropout masks of one site (Hephaistos: dropout on the embeddings,
+// the attention weights and the attention and MLP outputs; masks drawn by the
+// training forward and reused by its backward).  Element e of the site is kept
+// when word 0 of Philox4x32-10(counter = (e low, e high, site, *step), key =
+// (k0, k1)) is >= thr = floor(p * 2^32); kept elements are scaled by `scale`
+// = 1 / (1 - p).  on = 0: no dropout.
+struct DropArgs {
+  int on = 0;
+  uint32_t thr = 0, k0 = 0, k1 = 0, site = 0;
+  float scale = 1.f;
+  const int *step = nullptr;  // device word: the training forward's number
+};
+
 // ------------------------------------------------------------ GEMM (shared)
 // C[M,N] = A[M,K] * B^T where B is given as an [N,K] operand:
 //   A element (m,k) = a_kmajor ? A[m*lda + k] : A[k*lda + m]
@@ -83,16 +96,27 @@ int clip_part_blocks();
 void scale_grads(float *g, int64_t n, float sc, cudaStream_t s);
 void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm, float *scale,
                 cudaStream_t s);
+// Dropout of [n] row-major elements of a site (element index = position):
+//   drop_rows: x *= f in place;  drop_add: out = x + f y;
+//   drop_to_act: out (operand type) = f dx.
+void drop_rows(float *x, int64_t n, const DropArgs &a, cudaStream_t s);
+void drop_add(const float *x, const float *y, float *out, int64_t n, const DropArgs &a,
+              cudaStream_t s);
+void drop_to_act(const float *dx, void *out, DType dt, int64_t n, const DropArgs &a,
+                 cudaStream_t s);
 void set_flag_zero(int *flag, cudaStream_t s);
 void or_flag(const int *src, int *dst, cudaStream_t s);
 
 // --------------------------------------------------------------- attention
 // qkv [N, qkvw] (q heads | k heads | v heads, RoPE applied), o [N, H*hd],
 // lse [B, H, T]; SIMT reference kernels for any head size.
+// With drop.on, the probabilities are dropped (element ((b*H + h)*T + i)*T + j
+// of the site): o uses P f, the backward uses the same f.
 void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
-                   int hd, cudaStream_t s);
+                   int hd, cudaStream_t s, DropArgs drop = DropArgs{});
 void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
-                   void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s);
+                   void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s,
+                   DropArgs drop = DropArgs{});
 
 // Tensor-core (mma.sync, bf16) kernels for head sizes 32 and 64.
 bool attn_mma_covers(DType dt, int hd);

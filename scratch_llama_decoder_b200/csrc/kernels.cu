@@ -1000,17 +1000,6 @@ void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int 
 // Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011) keyed
 // by the seed, counter = element index; two 32-bit outputs give one normal by
 // the Box-Muller transform.
-LLM_DEV void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
-  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
-#pragma unroll
-  for (int r = 0; r < 10; r++) {
-    uint32_t hi0 = __umulhi(M0, c[0]), lo0 = M0 * c[0];
-    uint32_t hi1 = __umulhi(M1, c[2]), lo1 = M1 * c[2];
-    uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
-    c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
-    k0 += W0; k1 += W1;
-  }
-}
 __global__ void k_init(float *__restrict__ p, int64_t n, uint32_t k0, uint32_t k1, uint64_t base,
                        float std, int one) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
@@ -1033,7 +1022,48 @@ void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, floa
   count_launch();
 }
 
-// -------------------------------------------------------------------- flags
+// ------------------------------------------------------------------ dropout
+// Hephaistos, Architecture at a glance (Regularization): inverted dropout,
+// masks reused by the backward (the factor of an element is a pure function
+// of its index, the site and the step, so the backward draws it again).
+__global__ void k_drop_rows(float *__restrict__ x, int64_t n, const DropArgs a) {
+  const uint32_t step = (uint32_t)*a.step;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    x[i] *= drop_factor(a, (uint64_t)i, step);
+}
+__global__ void k_drop_add(const float *__restrict__ x, const float *__restrict__ y,
+                           float *__restrict__ out, int64_t n, const DropArgs a) {
+  const uint32_t step = (uint32_t)*a.step;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = x[i] + drop_factor(a, (uint64_t)i, step) * y[i];
+}
+template <typename A>
+__global__ void k_drop_to_act(const float *__restrict__ dx, A *__restrict__ out, int64_t n,
+                              const DropArgs a) {
+  const uint32_t step = (uint32_t)*a.step;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = from_f<A>(drop_factor(a, (uint64_t)i, step) * dx[i]);
+}
+void drop_rows(float *x, int64_t n, const DropArgs &a, cudaStream_t s) {
+  k_drop_rows<<<min(cdiv(n, 256), 148u * 16), 256, 0, s>>>(x, n, a);
+  count_launch();
+}
+void drop_add(const float *x, const float *y, float *out, int64_t n, const DropArgs &a,
+              cudaStream_t s) {
+  k_drop_add<<<min(cdiv(n, 256), 148u * 16), 256, 0, s>>>(x, y, out, n, a);
+  count_launch();
+}
+void drop_to_act(const float *dx, void *out, DType dt, int64_t n, const DropArgs &a,
+                 cudaStream_t s) {
+  const unsigned grid = min(cdiv(n, 256), 148u * 16);
+  if (dt == DT_BF16) k_drop_to_act<<<grid, 256, 0, s>>>(dx, (__nv_bfloat16 *)out, n, a);
+  else k_drop_to_act<<<grid, 256, 0, s>>>(dx, (float *)out, n, a);
+  count_launch();
+}
+
 // ------------------------------------------------------- gradient clipping
 // MicroGPT in Rust, Gradient Clipping: the norm of all gradients together;
 // when it exceeds max_norm every gradient is scaled by max_norm / norm.
@@ -1125,6 +1155,7 @@ void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm,
   count_launch(3);
 }
 
+// -------------------------------------------------------------------- flags
 __global__ void k_or_flag(const int *src, int *dst) { if (*src) atomicOr(dst, *src); }
 void set_flag_zero(int *flag, cudaStream_t s) { cudaMemsetAsync(flag, 0, sizeof(int), s); }
 void or_flag(const int *src, int *dst, cudaStream_t s) {

@@ -171,6 +171,12 @@ struct llm_ctx {
   Key dkey{}, dprev_key{};
   bool dhave_prev = false;
   int dgraph_launches = 0;
+  // dropout (llm_set_dropout): rate, seed, training calls so far, and the
+  // device word holding the current call's number
+  float drop_p = 0.f;
+  uint64_t drop_seed = 0;
+  int64_t train_calls = 0;
+  int *drop_step = nullptr;
   // gradient clipping (llm_set_grad_clip): threshold, block sums, norm, scale
   float clip = 0.f;
   bool have_norm = false;
@@ -242,6 +248,7 @@ int64_t llm_ctx::carve(char *base) {
   dec_count = (unsigned *)c.take(4 * dblocks);
   dec_acount = (unsigned *)c.take(4 * B * D_.Hkv);
   dec_pos = (int *)c.take(64);
+  drop_step = (int *)c.take(64);
   clip_part = (double *)c.take(8 * (int64_t)clip_part_blocks());
   clip_norm = (double *)c.take(64);
   clip_scale = (float *)c.take(64);
@@ -326,6 +333,7 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
                   c->s);
   cudaMemsetAsync(c->dec_acount, 0, 4 * (size_t)c->D.B * c->D.Hkv, c->s);
   cudaMemsetAsync(c->dec_pos, 0, 64, c->s);
+  cudaMemsetAsync(c->drop_step, 0, 64, c->s);
   rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, cfg->rope_base, c->s);
   c->tc = tc_plan_create(c->D.dt, c->cos_t, c->sin_t, c->D.T, c->D.hd, c->D.d + c->D.kvd, c->D.hp);
   tc_plan_set_flag(c->tc, c->flag_step);
@@ -398,6 +406,23 @@ int llm_set_grad_clip(llm_ctx *c, float max_norm) {
     c->have_prev = false;
     c->clip = v;
   }
+  return LLM_OK;
+}
+
+int llm_set_dropout(llm_ctx *c, float p, uint64_t seed) {
+  if (!c || !(p >= 0.f) || !(p < 1.f)) return LLM_ERR_ARG;
+  if (p != c->drop_p || seed != c->drop_seed) {
+    // the rate is baked into a captured step: drop the graph
+    if (c->gexec) {
+      if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+      cudaGraphExecDestroy(c->gexec);
+      c->gexec = nullptr;
+    }
+    c->have_prev = false;
+    c->drop_p = p;
+    c->drop_seed = seed;
+  }
+  c->train_calls = 0;
   return LLM_OK;
 }
 
@@ -510,8 +535,28 @@ void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, 
   gemm_simt(g, out, C, ldc, R, ldr, splits, c->cur);
 }
 
-// Forward pass; leaves logits (padded, activation type) in c->logits.
-void forward(llm_ctx *c, const float *p, const int32_t *tok) {
+// Dropout masks of (site, layer) for the current training call (sites: 0
+// embedding output, 1 attention probabilities, 2 attention branch output, 3
+// MLP branch output).
+DropArgs drop_args(const llm_ctx *c, int site, int layer) {
+  DropArgs a;
+  a.on = 1;
+  a.thr = (uint32_t)floor((double)c->drop_p * 4294967296.0);
+  a.scale = (float)(1.0 / (1.0 - (double)c->drop_p));
+  a.k0 = (uint32_t)c->drop_seed;
+  a.k1 = (uint32_t)(c->drop_seed >> 32);
+  a.site = (uint32_t)(site + 4 * layer);
+  a.step = c->drop_step;
+  return a;
+}
+bool dropping(const llm_ctx *c) { return c->drop_p > 0.f; }
+
+// Forward pass; leaves logits (padded, activation type) in c->logits.  train:
+// a training forward (dropout applies when set; evaluation never drops).
+// With dropout on, attention runs in the CUDA-core kernels, which draw the
+// probability masks.
+void forward(llm_ctx *c, const float *p, const int32_t *tok, bool train) {
+  const bool drop = train && dropping(c);
   const Dims &D = c->D;
   POff O{D};
   cudaStream_t s = c->s;
@@ -529,6 +574,7 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
   }
   cast_weight(p + O.wlm(), c->w_lm, D.dt, d, D.V, d, D.Vp, 0, 0, 0, 1, 0, 0, s);
   embed_fwd(p, tok, c->xs, N, D.d, D.V, c->flag_step, s);
+  if (drop) drop_rows(c->xs, N * d, drop_args(c, 0, 0), s);
   for (int l = 0; l < D.L; l++) {
     float *x = c->xs + l * N * d, *x1 = c->x1 + l * N * d, *x2 = c->xs + (l + 1) * N * d;
     void *xn1 = A(c->xn1, l, N * d), *qkv = A(c->qkv, l, N * D.qkvw), *o = A(c->o, l, N * d);
@@ -547,9 +593,16 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
         rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
       }
     }
-    attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
-    gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d, x,
-         d, 1, 2.0 * N * d * d);
+    if (drop) {  // x1 = x + f * (o Wo), o from dropped probabilities
+      attn_fwd_simt(qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
+      gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_F32, c->dtmp, d,
+           nullptr, 0, 1, 2.0 * N * d * d);
+      drop_add(x, c->dtmp, x1, N * d, drop_args(c, 2, l), s);
+    } else {
+      attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
+      gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d,
+           x, d, 1, 2.0 * N * d * d);
+    }
     // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
     rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
     // W13 GEMM into the interleaved [a|b], then u = silu(a) * b (a separate
@@ -557,8 +610,14 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok) {
     gemm(c, GemmOperands{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt},
          OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
     swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
-    gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_ADD_F32,
-         x2, d, x1, d, 1, 2.0 * N * D.h * d);
+    if (drop) {  // x2 = x1 + f * (u W2)
+      gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_F32,
+           c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.h * d);
+      drop_add(x1, c->dtmp, x2, N * d, drop_args(c, 3, l), s);
+    } else {
+      gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt},
+           OUT_ADD_F32, x2, d, x1, d, 1, 2.0 * N * D.h * d);
+    }
   }
   float *xL = c->xs + D.L * N * d;
   rmsnorm_fwd(xL, p + O.gf(), c->xf, D.dt, c->rstdf, N, D.d, c->cfg.rms_eps, s);
@@ -609,7 +668,10 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
   const int ab = D.ab;
   const bool lp = D.dt == DT_BF16;
   auto A = [&](void *base, int64_t l, int64_t per) { return (char *)base + l * per * ab; };
-  void *dxop = lp ? c->dxA : (void *)c->dx;  // dx as a GEMM operand
+  const bool drop = dropping(c);
+  // dx as a GEMM operand; with dropout the masked copy of the branch
+  // output's gradient (dxA, operand type at both precisions)
+  void *dxop = (lp || drop) ? c->dxA : (void *)c->dx;
   void *dxact = lp ? c->dxA : nullptr;
   int nb;
   // lm_head: dxf = dz Wlm^T; dWlm = xf^T dz
@@ -629,6 +691,7 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
     void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
     void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
     // FFN branch.  du = dx2 W2^T, then SwiGLU backward into dab.
+    if (drop) drop_to_act(c->dx, c->dxA, D.dt, N * d, drop_args(c, 3, l), s);
     fork_side(c);  // dx2 is ready
     wgrad_side(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
     gemm(c, GemmOperands{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt}, OUT_ACT, c->du,
@@ -644,10 +707,17 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
                      D.d, s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
     // attention branch
+    if (drop) drop_to_act(c->dx, c->dxA, D.dt, N * d, drop_args(c, 2, l), s);
     gemm(c, GemmOperands{(int)N, D.d, D.d, dxop, d, true, wo, d, true, D.dt}, OUT_ACT, c->dO, d,
          nullptr, 0, 1, 2.0 * N * d * d);
-    attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
-                  c->cos_t, c->sin_t, s);
+    if (drop) {  // the same probability masks, then RoPE backward on dq, dk
+      attn_bwd_simt(qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s,
+                    drop_args(c, 1, l));
+      rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);
+    } else {
+      attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
+                    c->cos_t, c->sin_t, s);
+    }
     fork_side(c);  // dx1 and dqkv are ready (after the attention, so no TMEM contention)
     wgrad_side(c, o, d, dxop, d, d, d, gr + O.wo(l), d, d, 0);
     wgrad_side(c, xn1, d, c->dqkv, D.qkvw, d, D.qkvw, gr + O.wqkv(l), d, D.qkvw, 0);
@@ -659,6 +729,7 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
                      s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g1(l), s);
   }
+  if (drop) drop_rows(c->dx, N * d, drop_args(c, 0, 0), s);
   embed_bwd(tok, c->dx, gr, N, D.d, D.V, c->sort_scratch, s);
   join_side(c);  // every weight gradient is in place before AdamW
 }
@@ -735,7 +806,7 @@ int llm_forward(llm_ctx *c, const float *d_params, const int32_t *d_tokens, floa
   if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;
   g_launches = 0;
   set_flag_zero(c->flag_step, c->s);
-  forward(c, d_params, d_tokens);
+  forward(c, d_params, d_tokens, false);
   logits_out(c->logits, c->D.dt, d_logits, c->D.N, c->D.V, c->D.Vp, c->s);
   or_flag(c->flag_step, c->flag_sticky, c->s);
   c->last_launches = g_launches;
@@ -754,9 +825,11 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
   const double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
   const double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
   set_hyper(c->hyper, lr, wd, (float)bc1, (float)bc2, c->s);
+  // the mask step word also goes to device memory outside any graph
+  if (dropping(c)) set_device_int(c->drop_step, (int)(c->train_calls++), c->s);
   auto body = [&]() {
     set_flag_zero(c->flag_step, c->s);
-    forward(c, d_params, d_tokens);
+    forward(c, d_params, d_tokens, true);
     cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
                   c->flag_step, c->s);
     loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
@@ -817,8 +890,9 @@ int llm_grad(llm_ctx *c, const float *d_params, float *d_grads, const int32_t *d
   if (!aligned16(d_params) || !aligned16(d_grads)) return LLM_ERR_ARG;
   const Dims &D = c->D;
   g_launches = 0;
+  if (dropping(c)) set_device_int(c->drop_step, (int)(c->train_calls++), c->s);
   set_flag_zero(c->flag_step, c->s);
-  forward(c, d_params, d_tokens);
+  forward(c, d_params, d_tokens, true);
   cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
                 c->flag_step, c->s);
   loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);

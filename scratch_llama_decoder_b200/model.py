@@ -111,6 +111,10 @@ class LlamaStep:
                 "llm_sample")
         return out
 
+    def set_dropout(self, p, seed):
+        """Inverted dropout in later training calls (llm_set_dropout)."""
+        L.check(L.lib.llm_set_dropout(self.ctx, float(p), int(seed)), "llm_set_dropout")
+
     def set_grad_clip(self, max_norm):
         """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
         L.check(L.lib.llm_set_grad_clip(self.ctx, float(max_norm)), "llm_set_grad_clip")
