@@ -9,3 +9,18 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA B200 GPU (sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+# Collection order for a run that stops at the first failure (-x): the parity
+# tests of the training step, its kernels and decode first, then the tests of
+# the entry points built on them (data parallelism, dropout), and last the
+# allocation-free entry, whose file sets up per-device state on first use.
+_LATE = ("test_gpu_dp.py", "test_gpu_dropout.py")
+_LAST = ("test_zz_no_alloc.py",)
+
+
+def pytest_collection_modifyitems(session, config, items):
+    def rank(item):
+        name = os.path.basename(str(item.fspath))
+        return 2 if name in _LAST else 1 if name in _LATE else 0
+    items.sort(key=rank)  # stable: the order inside each group is kept
