@@ -12,9 +12,10 @@ Keys enter the cache already rotated by RoPE at their own position and are
 never rotated again.  strata's gate is that decoding a sequence position by
 position reproduces the full forward's logits (to ~1e-9 in float64).
 
-Sampler (Hephaistos, Sampling: temperature + top-k; strata, sampler row;
-Transformer-In-Rust, inference pipeline: temperature scaling, then top-k
-filtering).  Readings taken where the pages are silent:
+Sampler (Hephaistos, Sampling: temperature + top-k; strata, sampler row:
+temperature / top-k / top-p; randyGPT: top-p (nucleus) + temperature;
+Transformer-In-Rust, sampling pipeline: repetition penalty, temperature,
+top-k, top-p, random sample).  Readings taken where the pages are silent:
   * temperature 0 (or top_k = 1) is greedy: the largest logit, the lowest id
     among equal maxima;
   * the top-k set is the first k ids in the order (logit descending, id
@@ -26,6 +27,14 @@ filtering).  Readings taken where the pages are silent:
     supplied by the caller (random numbers are inputs, not drawn here).
 The distribution is softmax(z / temperature) restricted to the set and
 renormalised, whatever order the CDF walks; id order needs no sort.
+  * repetition penalty r (the usual form, Keskar et al. 2019): before
+    anything else, every id present in the sequence's history has its logit
+    divided by r when positive and multiplied by r otherwise, in float32 (the
+    logits' own precision, so both sides see the same penalised logits);
+  * top-p (nucleus) applies inside the top-k set: walking the set in the
+    (logit descending, id ascending) order, keep the shortest prefix whose
+    weight reaches top_p of the set's total (at least one id), then draw
+    from that prefix as above.
 """
 import numpy as np
 
@@ -111,11 +120,40 @@ def sample_cdf(z, temperature, top_k):
     return S, C, C[-1]
 
 
-def sample(z, temperature, top_k, u):
+def penalise(z, penalty, history):
+    """Logits after the repetition penalty (float32 arithmetic)."""
+    z = np.array(z, dtype=np.float32)
+    if penalty == 1.0:
+        return z
+    r = np.float32(penalty)
+    for i in sorted({int(h) for h in history if 0 <= int(h) < z.size}):
+        z[i] = z[i] / r if z[i] > 0 else z[i] * r
+    return z
+
+
+def nucleus(z, temperature, top_k, top_p):
+    """Ids of the top-p prefix of the top-k set, in increasing id order, and
+    the float64 cumulative weights along the (logit desc, id asc) walk."""
+    S = topk_set(z, top_k)
+    zf = np.asarray(z, dtype=np.float64)
+    order = S[np.lexsort((S, -zf[S]))]  # logit descending, then id ascending
+    w = np.exp((zf[order] - zf.max()) / temperature)
+    C = np.cumsum(w)
+    n = 1 + int(np.searchsorted(C, top_p * C[-1], side="left"))
+    return np.sort(order[:min(n, order.size)]), C
+
+
+def sample(z, temperature, top_k, u, top_p=1.0, penalty=1.0, history=()):
     """Token id drawn from logits z [V] with uniform u in [0, 1)."""
-    z = np.asarray(z)
+    z = penalise(z, penalty, history) if penalty != 1.0 else np.asarray(z)
     if temperature <= 0 or top_k == 1:
         return int(np.argmax(z))  # first maximum = lowest id among ties
+    if top_p < 1.0:
+        S, _ = nucleus(z, temperature, top_k, top_p)
+        zf = np.asarray(z, dtype=np.float64)
+        C = np.cumsum(np.exp((zf[S] - zf.max()) / temperature))
+        i = int(np.searchsorted(C, float(u) * C[-1], side="right"))
+        return int(S[min(i, S.size - 1)])
     S, C, W = sample_cdf(z, temperature, top_k)
     i = int(np.searchsorted(C, float(u) * W, side="right"))
     return int(S[min(i, S.size - 1)])

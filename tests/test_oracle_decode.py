@@ -120,3 +120,50 @@ def test_sampler_empirical_frequencies():
     chi2 = n * np.sum((freq[S] - p[S]) ** 2 / p[S])
     assert chi2 < 25.0, chi2
     assert math.isclose(freq.sum(), 1.0)
+
+
+def test_sampler_top_p_worked_example():
+    # probabilities 0.5, 0.3, 0.2 (ids 2, 0, 1 by logit): top_p 0.7 keeps the
+    # first two by probability (0.5 + 0.3 >= 0.7), renormalised 0.625 / 0.375
+    z = np.log(np.array([0.3, 0.2, 0.5]))
+    S, _ = OD.nucleus(z, 1.0, 3, 0.7)
+    np.testing.assert_array_equal(S, [0, 2])
+    # id order: id 0 (0.375) then id 2 (0.625)
+    assert [OD.sample(z, 1.0, 3, u, top_p=0.7) for u in (0.0, 0.37, 0.38, 0.99)] == [0, 0, 2, 2]
+    # a prefix reaching top_p exactly stops there; top_p 1 keeps the set
+    np.testing.assert_array_equal(OD.nucleus(z, 1.0, 3, 0.5)[0], [2])
+    np.testing.assert_array_equal(OD.nucleus(z, 1.0, 3, 1.0)[0], [0, 1, 2])
+    # a tiny top_p keeps the single most likely id (greedy-like)
+    assert {OD.sample(z, 1.0, 3, u, top_p=1e-6) for u in np.linspace(0, 0.99, 20)} == {2}
+    # top-p inside top-k: top-2 set {2, 0}; top_p 0.7 of its 0.8 total keeps both
+    np.testing.assert_array_equal(OD.nucleus(z, 1.0, 2, 0.7)[0], [0, 2])
+    np.testing.assert_array_equal(OD.nucleus(z, 1.0, 2, 0.6)[0], [2])
+
+
+def test_sampler_repetition_penalty():
+    z = np.array([2.0, -1.0, 0.5, 3.0], dtype=np.float32)
+    pz = OD.penalise(z, 2.0, [0, 1, 1, 7, -1])
+    np.testing.assert_array_equal(pz, np.array([1.0, -2.0, 0.5, 3.0], dtype=np.float32))
+    np.testing.assert_array_equal(OD.penalise(z, 1.0, [0, 1]), z)
+    # the penalty can move the greedy choice
+    z = np.array([2.0, 1.5], dtype=np.float32)
+    assert OD.sample(z, 0.0, 0, 0.5) == 0
+    assert OD.sample(z, 0.0, 0, 0.5, penalty=1.5, history=[0]) == 1
+
+
+def test_sampler_top_p_frequencies():
+    rng = np.random.default_rng(21)
+    z = (rng.standard_normal(12) * 1.5).astype(np.float32)
+    temp, k, tp, n = 0.9, 8, 0.8, 20000
+    S, _ = OD.nucleus(z, temp, k, tp)
+    draws = np.array([OD.sample(z, temp, k, u, top_p=tp) for u in rng.random(n)])
+    p = np.zeros(12)
+    p[S] = np.exp(z[S].astype(np.float64) / temp)
+    p /= p.sum()
+    freq = np.bincount(draws, minlength=12) / n
+    assert set(np.unique(draws).tolist()) <= set(S.tolist())
+    assert np.all(np.abs(freq - p) <= 4.5 * np.sqrt(p * (1 - p) / n) + 1e-12)
+    # the nucleus is the shortest prefix reaching top_p of the top-k weight
+    w = np.sort(np.exp(z.astype(np.float64) / temp))[::-1][:k]
+    m = int(np.argmax(np.cumsum(w) >= tp * w.sum())) + 1
+    assert S.size == m
