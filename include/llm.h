@@ -196,6 +196,25 @@ int llm_decode(llm_ctx *ctx, const float *d_params, const int32_t *d_tokens, int
 int llm_sample(llm_ctx *ctx, const float *d_logits, int64_t ld, int n_rows, float temperature,
                int top_k, const float *d_uniform, int32_t *d_out);
 
+/* llm_sample with the rest of the sampling pipeline (Transformer-In-Rust,
+ * Features: repetition penalty -> temperature -> top-k -> top-p -> random
+ * sample; strata and randyGPT: top-p nucleus sampling).  First, when
+ * repetition_penalty != 1, every id present among the first history_len
+ * entries of the row's history (device int32, row b at d_history + b *
+ * history_ld; entries outside [0, vocab) ignored) has its logit divided by
+ * repetition_penalty when positive and multiplied by it otherwise (float32).
+ * Then temperature and top-k as in llm_sample; then, when top_p < 1, only the
+ * shortest prefix of the top-k set walked in (logit descending, id
+ * ascending) order whose weight reaches top_p of the set's total is kept
+ * (at least one id), and the draw is made from it as in llm_sample.
+ * top_p = 1 and repetition_penalty = 1 give llm_sample's ids.  LLM_ERR_ARG
+ * unless 0 < top_p <= 1 (top_p < 1 needs 1 <= top_k <= 1024),
+ * repetition_penalty > 0 and finite, history_len >= 0, and with a penalty a
+ * history, history_ld >= history_len and vocab <= 524288. */
+int llm_sample_ex(llm_ctx *ctx, const float *d_logits, int64_t ld, int n_rows, float temperature,
+                  int top_k, float top_p, float repetition_penalty, const int32_t *d_history,
+                  int64_t history_ld, int history_len, const float *d_uniform, int32_t *d_out);
+
 /* Learning-rate schedule (host only: needs no context and no GPU; the value
  * is passed to llm_step as lr).  Transformer-In-Rust, Features: cosine decay
  * with linear warmup, and cosine / linear / constant schedulers; randyGPT,

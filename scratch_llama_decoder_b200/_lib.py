@@ -60,6 +60,7 @@ EXPORTS = {
     "llm_flag_in": (_i, [_vp, _vp]),
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
     "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),
+    "llm_sample_ex": (_i, [_vp, _vp, _i64, _i, _f, _i, _f, _f, _vp, _i64, _i, _vp, _vp]),
     "llm_set_grad_clip": (_i, [_vp, _f]),
     "llm_set_dropout": (_i, [_vp, _f, _u64]),
     "llm_read_grad_norm": (_i, [_vp, C.POINTER(C.c_double)]),

@@ -47,6 +47,7 @@ constexpr int AT_KEYS = 128;     // keys per attention block (one per thread whe
 constexpr int AT_THREADS = 128;
 
 constexpr int SP_THREADS = 1024;
+constexpr int SP_PEN_BYTES = 64 * 1024;  // history bitmap of the penalty: ids < 524288
 
 inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
 
@@ -511,9 +512,31 @@ LLM_DEV uint32_t order_key(float f) {  // unsigned order = float order
 LLM_DEV float sample_weight(float z, float zmax, float temperature) {
   return expf((z - zmax) / temperature);
 }
+// Extensions (llm_sample_ex), applied only by the EXT instantiation
+// (Transformer-In-Rust, sampling pipeline: repetition penalty, temperature,
+// top-k, top-p; strata and randyGPT: top-p).  The penalty divides a positive
+// logit of an id present in the row's history by `penalty` and multiplies a
+// negative one, before everything else (float32, the logits' precision).  Top-p
+// keeps, inside the top-k set walked in (logit descending, id ascending)
+// order, the shortest prefix whose weight reaches top_p of the set's total;
+// the set is sorted in shared memory, so top_k <= SP_NUC_MAX.
+constexpr int SP_NUC_MAX = 1024;
+struct SampleExt {
+  float top_p = 1.f;
+  float penalty = 1.f;
+  const int32_t *hist = nullptr;
+  int64_t hist_ld = 0;
+  int hist_len = 0;
+};
+LLM_DEV unsigned long long sort_composite(uint32_t key, int id) {  // (key desc, id asc) = desc
+  return ((unsigned long long)key << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)id);
+}
+
+template <bool EXT>
 __global__ void __launch_bounds__(SP_THREADS)
     k_sample(const float *__restrict__ logits, int64_t ld, int V, float temperature, int top_k,
-             const float *__restrict__ uni, int32_t *__restrict__ out) {
+             const float *__restrict__ uni, int32_t *__restrict__ out, const SampleExt ext) {
+  extern __shared__ uint32_t pen_bits[];  // EXT with a penalty: one bit per id of the history
   __shared__ float sv[32];
   __shared__ int si[32];
   __shared__ unsigned hist[256];
@@ -526,11 +549,33 @@ __global__ void __launch_bounds__(SP_THREADS)
   const float *z = logits + (int64_t)b * ld;
   const int chunk = (V + SP_THREADS - 1) / SP_THREADS;
   const int lo = min(V, tid * chunk), hi = min(V, lo + chunk);
+  bool pen = false;
+  if constexpr (EXT) {
+    pen = ext.penalty != 1.f && ext.hist_len > 0;
+    if (pen) {
+      for (int w = tid; w < (V + 31) / 32; w += SP_THREADS) pen_bits[w] = 0u;
+      __syncthreads();
+      const int32_t *h = ext.hist + (int64_t)b * ext.hist_ld;
+      for (int j = tid; j < ext.hist_len; j += SP_THREADS) {
+        const int id = h[j];
+        if (id >= 0 && id < V) atomicOr(&pen_bits[id >> 5], 1u << (id & 31));
+      }
+      __syncthreads();
+    }
+  }
+  auto zval = [&](int i) -> float {  // the (penalised) logit of id i
+    float v = z[i];
+    if constexpr (EXT) {
+      if (pen && ((pen_bits[i >> 5] >> (i & 31)) & 1u))
+        v = v > 0.f ? v / ext.penalty : v * ext.penalty;
+    }
+    return v;
+  };
   // maximum and its lowest id
   float bv = -INFINITY;
   int bi = INT_MAX;
   for (int i = lo; i < hi; i++) {
-    const float v = z[i];
+    const float v = zval(i);
     if (bi == INT_MAX || v > bv) { bv = v; bi = i; }
   }
   for (int o = 16; o > 0; o >>= 1) {
@@ -569,7 +614,7 @@ __global__ void __launch_bounds__(SP_THREADS)
       if (tid < 256) hist[tid] = 0u;
       __syncthreads();
       for (int i = lo; i < hi; i++) {
-        const uint32_t k = order_key(z[i]);
+        const uint32_t k = order_key(zval(i));
         if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
       }
       __syncthreads();
@@ -595,7 +640,7 @@ __global__ void __launch_bounds__(SP_THREADS)
   // rank of this thread's first id among the ids holding the cut key
   unsigned myeq = 0u;
   if (!all)
-    for (int i = lo; i < hi; i++) myeq += order_key(z[i]) == thr;
+    for (int i = lo; i < hi; i++) myeq += order_key(zval(i)) == thr;
   eqc[tid] = myeq;
   __syncthreads();
   if (tid == 0) {
@@ -608,20 +653,104 @@ __global__ void __launch_bounds__(SP_THREADS)
   }
   __syncthreads();
   const unsigned eq0 = eqc[tid];
+  // top-p: the composites of the top-k set sorted descending; members are the
+  // composites >= the cut (0: no cut)
+  unsigned long long cut = 0ull;
+  if constexpr (EXT) {
+    if (ext.top_p < 1.f) {
+      __shared__ unsigned long long sortv[SP_NUC_MAX];
+      __shared__ unsigned scnt[SP_THREADS];
+      __shared__ unsigned s_n;
+      __shared__ unsigned long long s_cut;
+      unsigned cnt = 0u;
+      {
+        unsigned eq = eq0;
+        for (int i = lo; i < hi; i++) {
+          const uint32_t k = order_key(zval(i));
+          cnt += all || k > thr || (k == thr && eq < rem);
+          if (!all) eq += k == thr;
+        }
+      }
+      scnt[tid] = cnt;
+      __syncthreads();
+      if (tid == 0) {
+        unsigned run = 0u;
+        for (int t = 0; t < SP_THREADS; t++) {
+          const unsigned n = scnt[t];
+          scnt[t] = run;
+          run += n;
+        }
+        s_n = run;  // <= SP_NUC_MAX: top_k <= SP_NUC_MAX, or V itself when top_k >= V
+      }
+      __syncthreads();
+      const int n = (int)s_n;
+      {
+        unsigned pos = scnt[tid], eq = eq0;
+        for (int i = lo; i < hi; i++) {
+          const uint32_t k = order_key(zval(i));
+          const bool in = all || k > thr || (k == thr && eq < rem);
+          if (!all) eq += k == thr;
+          if (in) sortv[pos++] = sort_composite(k, i);
+        }
+      }
+      int n2 = 1;
+      while (n2 < n) n2 <<= 1;
+      for (int t = n + tid; t < n2; t += SP_THREADS) sortv[t] = 0ull;  // below every member
+      __syncthreads();
+      // bitonic sort, descending
+      for (int size = 2; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          for (int t = tid; t < n2; t += SP_THREADS) {
+            const int q = t ^ stride;
+            if (q > t) {
+              const unsigned long long x = sortv[t], y = sortv[q];
+              if (((t & size) == 0) ? (x < y) : (x > y)) { sortv[t] = y; sortv[q] = x; }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      // weights along the walk (one per thread), then the prefix by one thread
+      for (int t = tid; t < n; t += SP_THREADS) {
+        const int id = (int)(0xFFFFFFFFu - (uint32_t)sortv[t]);
+        wsum[t] = sample_weight(zval(id), zmax, temperature);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        float W = 0.f;
+        for (int t = 0; t < n; t++) W += wsum[t];
+        const float goal = ext.top_p * W;
+        float c = 0.f;
+        int m = n;
+        for (int t = 0; t < n; t++) {
+          c += wsum[t];
+          if (c >= goal) { m = t + 1; break; }
+        }
+        s_cut = sortv[m - 1];
+      }
+      __syncthreads();
+      cut = s_cut;
+    }
+  }
+  auto member = [&](int i, unsigned &eq) -> bool {  // in the top-k set (and the nucleus)
+    bool in = all;
+    uint32_t k = 0u;
+    if (!all || EXT) k = order_key(zval(i));
+    if (!all) {
+      in = k > thr || (k == thr && eq < rem);
+      eq += k == thr;
+    }
+    if constexpr (EXT) in = in && sort_composite(k, i) >= cut;
+    return in;
+  };
   // this thread's weight, ids in increasing order
   float my = 0.f;
   {
     unsigned eq = eq0;
-    for (int i = lo; i < hi; i++) {
-      bool in = all;
-      if (!all) {
-        const uint32_t k = order_key(z[i]);
-        in = k > thr || (k == thr && eq < rem);
-        eq += k == thr;
-      }
-      if (in) my += sample_weight(z[i], zmax, temperature);
-    }
+    for (int i = lo; i < hi; i++)
+      if (member(i, eq)) my += sample_weight(zval(i), zmax, temperature);
   }
+  __syncthreads();  // the top-p walk's weights are no longer read
   wsum[tid] = my;
   __syncthreads();
   if (tid == 0) {
@@ -648,14 +777,8 @@ __global__ void __launch_bounds__(SP_THREADS)
     int pick = -1, lastin = -1;
     unsigned eq = eq0;
     for (int i = lo; i < hi; i++) {
-      bool in = all;
-      if (!all) {
-        const uint32_t k = order_key(z[i]);
-        in = k > thr || (k == thr && eq < rem);
-        eq += k == thr;
-      }
-      if (!in) continue;
-      c += sample_weight(z[i], zmax, temperature);
+      if (!member(i, eq)) continue;
+      c += sample_weight(zval(i), zmax, temperature);
       lastin = i;
       if (c > s_tl) { pick = i; break; }
     }
@@ -753,7 +876,33 @@ void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, in
 
 void sample_tokens(const float *logits, int64_t ld, int rows, int V, float temperature, int top_k,
                    const float *uni, int32_t *out, cudaStream_t s) {
-  k_sample<<<rows, SP_THREADS, 0, s>>>(logits, ld, V, temperature, top_k, uni, out);
+  k_sample<false><<<rows, SP_THREADS, 0, s>>>(logits, ld, V, temperature, top_k, uni, out,
+                                              SampleExt{});
+  count_launch();
+}
+
+int sample_ex_max_top_k() { return SP_NUC_MAX; }
+int64_t sample_ex_max_vocab_penalty() { return (int64_t)SP_PEN_BYTES * 8; }
+
+void sample_tokens_ex(const float *logits, int64_t ld, int rows, int V, float temperature,
+                      int top_k, float top_p, float penalty, const int32_t *hist,
+                      int64_t hist_ld, int hist_len, const float *uni, int32_t *out,
+                      cudaStream_t s) {
+  static bool attr = false;  // room for the largest history bitmap, once
+  if (!attr) {
+    cudaFuncSetAttribute(k_sample<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         SP_PEN_BYTES);
+    attr = true;
+  }
+  SampleExt e;
+  e.top_p = top_p;
+  e.penalty = penalty;
+  e.hist = hist;
+  e.hist_ld = hist_ld;
+  e.hist_len = hist_len;
+  const bool pen = penalty != 1.f && hist_len > 0;
+  const size_t smem = pen ? (size_t)((V + 31) / 32) * 4 : 0;
+  k_sample<true><<<rows, SP_THREADS, smem, s>>>(logits, ld, V, temperature, top_k, uni, out, e);
   count_launch();
 }
 

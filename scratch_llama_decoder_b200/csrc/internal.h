@@ -189,6 +189,15 @@ void attn_decode(const void *qkv, int64_t qkvw, int B, int T, const int *pos, in
 // One token id per row of logits [rows, ld] (V valid columns).
 void sample_tokens(const float *logits, int64_t ld, int rows, int V, float temperature, int top_k,
                    const float *uni, int32_t *out, cudaStream_t s);
+// The same with the repetition penalty (ids of hist [rows, hist_ld], first
+// hist_len used; penalty != 1 needs V <= sample_ex_max_vocab_penalty()) and
+// top-p inside the top-k set (top_p < 1 needs 1 <= top_k <= sample_ex_max_top_k()).
+int sample_ex_max_top_k();
+int64_t sample_ex_max_vocab_penalty();
+void sample_tokens_ex(const float *logits, int64_t ld, int rows, int V, float temperature,
+                      int top_k, float top_p, float penalty, const int32_t *hist,
+                      int64_t hist_ld, int hist_len, const float *uni, int32_t *out,
+                      cudaStream_t s);
 void set_device_int(int *p, int v, cudaStream_t s);
 
 // Launch counter (kernels enqueued by the current call).

@@ -1003,6 +1003,25 @@ int llm_sample(llm_ctx *c, const float *d_logits, int64_t ld, int n_rows, float 
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
 
+int llm_sample_ex(llm_ctx *c, const float *d_logits, int64_t ld, int n_rows, float temperature,
+                  int top_k, float top_p, float repetition_penalty, const int32_t *d_history,
+                  int64_t history_ld, int history_len, const float *d_uniform, int32_t *d_out) {
+  if (!c || !d_logits || !d_uniform || !d_out || n_rows < 1 || ld < c->D.V) return LLM_ERR_ARG;
+  if (!(temperature == temperature) || !(top_p > 0.f) || !(top_p <= 1.f)) return LLM_ERR_ARG;
+  if (top_p < 1.f && (top_k < 1 || top_k > sample_ex_max_top_k())) return LLM_ERR_ARG;
+  if (!(repetition_penalty > 0.f) || !std::isfinite(repetition_penalty) || history_len < 0)
+    return LLM_ERR_ARG;
+  const bool pen = repetition_penalty != 1.f && history_len > 0;
+  if (pen && (!d_history || history_ld < history_len ||
+              (int64_t)c->D.V > sample_ex_max_vocab_penalty()))
+    return LLM_ERR_ARG;
+  g_launches = 0;
+  sample_tokens_ex(d_logits, ld, n_rows, c->D.V, temperature, top_k, top_p, repetition_penalty,
+                   d_history, history_ld, pen ? history_len : 0, d_uniform, d_out, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
 int llm_init(llm_ctx *c, uint64_t seed, float init_std, int scale_out_proj, float *d_params) {
   if (!c || !d_params || !(init_std >= 0.f)) return LLM_ERR_ARG;
   const Dims &D = c->D;

@@ -71,6 +71,21 @@ class LlamaStep:
                 "llm_step")
         return loss
 
+    def sample_ex(self, logits, temperature, top_k, uniforms, top_p=1.0, penalty=1.0,
+                  history=None, out=None):
+        """llm_sample_ex: repetition penalty over history (int32 [rows, n]),
+        temperature, top-k, top-p."""
+        rows = logits.shape[0]
+        if out is None:
+            out = torch.empty(rows, dtype=torch.int32, device=self.device)
+        hl = 0 if history is None else history.shape[1]
+        hld = 0 if history is None else history.stride(0)
+        L.check(L.lib.llm_sample_ex(self.ctx, _ptr(logits), logits.stride(0), rows,
+                                    float(temperature), int(top_k), float(top_p), float(penalty),
+                                    _ptr(history), hld, hl, _ptr(uniforms), _ptr(out)),
+                "llm_sample_ex")
+        return out
+
     def grad(self, params, grads, tokens, targets, loss=None):
         """Forward, loss and backward without the update (llm_grad)."""
         if loss is None:
