@@ -67,6 +67,7 @@ def decode_step(cfg, params, cache, tokens, pos):
     V, d, L = cfg["vocab"], cfg["d_model"], cfg["n_layer"]
     H, Hkv, h = cfg["n_head"], cfg["n_kv_head"], cfg["d_ff"]
     hd, eps, base = d // H, cfg["rms_eps"], cfg["rope_base"]
+    rs = cfg.get("rope_scale", 1.0)
     kvd, G = Hkv * hd, H // Hkv
     P = _tensors(cfg, params)
     tok = np.asarray(tokens, dtype=np.int64).reshape(-1)
@@ -80,9 +81,9 @@ def decode_step(cfg, params, cache, tokens, pos):
         v = qkv[:, d + kvd:].reshape(B, Hkv, hd)
         for b in range(B):
             for hh in range(H):
-                q[b, hh] = rope(q[b, hh], pos, base)
+                q[b, hh] = rope(q[b, hh], pos, base, scale=rs)
             for g in range(Hkv):
-                cache.K[l][b, g, pos] = rope(k[b, g], pos, base)
+                cache.K[l][b, g, pos] = rope(k[b, g], pos, base, scale=rs)
                 cache.V[l][b, g, pos] = v[b, g]
         o = np.zeros((B, H, hd))
         for b in range(B):

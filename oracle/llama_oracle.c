@@ -44,6 +44,7 @@
 typedef struct {
   int32_t V, d, L, H, Hkv, h, T, B;
   double rope_base, eps;
+  double rope_scale; /* position interpolation: RoPE position = t / rope_scale */
 } orc_cfg;
 
 /* ----------------------------------------------------------------- dropout */
@@ -211,16 +212,22 @@ void orc_rmsnorm_bwd(int n, int d, const double *x, const double *rstd, const do
  * theta_j = base^(-2j/hd); u'_j = u_j cos - u_{j+hd/2} sin,
  * u'_{j+hd/2} = u_{j+hd/2} cos + u_j sin.  sign = -1 applies the inverse
  * rotation (the backward of the forward rotation). */
-void orc_rope(double *u, int hd, int t, double base, int sign) {
+/* Rotation at a (possibly fractional) position (strata, RoPE row: position
+ * interpolation folds extended positions into the trained range, position
+ * t / scale). */
+void orc_rope_pos(double *u, int hd, double pos, double base, int sign) {
   int half = hd / 2;
   for (int j = 0; j < half; j++) {
     double theta = pow(base, -2.0 * j / hd);
-    double phi = (double)t * theta;
+    double phi = pos * theta;
     double c = cos(phi), s = sign * sin(phi);
     double a = u[j], b = u[j + half];
     u[j] = a * c - b * s;
     u[j + half] = b * c + a * s;
   }
+}
+void orc_rope(double *u, int hd, int t, double base, int sign) {
+  orc_rope_pos(u, hd, (double)t, base, sign);
 }
 
 /* --------------------------------------------------------------- attention */
@@ -485,8 +492,9 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
     orc_rmsnorm_fwd(T, d, A->x, p + off_g1(c, l), c->eps, A->xn1, A->rstd1);
     orc_mm_nn(T, d, (int)w, A->xn1, d, p + off_wqkv(c, l), w, A->qkv, w, 0);
     for (int t = 0; t < T; t++) {
-      for (int hq = 0; hq < H; hq++) orc_rope(A->qkv + (int64_t)t * w + (int64_t)hq * hd, hd, t, c->rope_base, 1);
-      for (int g = 0; g < Hkv; g++) orc_rope(A->qkv + (int64_t)t * w + d + (int64_t)g * hd, hd, t, c->rope_base, 1);
+      const double pos = (double)t / c->rope_scale;
+      for (int hq = 0; hq < H; hq++) orc_rope_pos(A->qkv + (int64_t)t * w + (int64_t)hq * hd, hd, pos, c->rope_base, 1);
+      for (int g = 0; g < Hkv; g++) orc_rope_pos(A->qkv + (int64_t)t * w + d + (int64_t)g * hd, hd, pos, c->rope_base, 1);
     }
     attention_fwd_do(T, d, H, Hkv, A->qkv, A->o, NULL, NULL, dr, l, bseq);
     if (dr) {
@@ -565,8 +573,9 @@ static double seq_step(const orc_cfg *c, const double *p, const int32_t *tok, co
       orc_mm_nt(T, d, d, dya, d, p + off_wo(c, l), d, dO, d, 0);
       attention_bwd_do(T, d, H, Hkv, A->qkv, dO, dqkv, dr, l, bseq);
       for (int t = 0; t < T; t++) {
-        for (int hq = 0; hq < H; hq++) orc_rope(dqkv + (int64_t)t * w + (int64_t)hq * hd, hd, t, c->rope_base, -1);
-        for (int g = 0; g < Hkv; g++) orc_rope(dqkv + (int64_t)t * w + d + (int64_t)g * hd, hd, t, c->rope_base, -1);
+        const double pos = (double)t / c->rope_scale;
+        for (int hq = 0; hq < H; hq++) orc_rope_pos(dqkv + (int64_t)t * w + (int64_t)hq * hd, hd, pos, c->rope_base, -1);
+        for (int g = 0; g < Hkv; g++) orc_rope_pos(dqkv + (int64_t)t * w + d + (int64_t)g * hd, hd, pos, c->rope_base, -1);
       }
       orc_mm_tn(d, T, (int)w, A->xn1, d, dqkv, w, grads + off_wqkv(c, l), w, 1);
       orc_mm_nt(T, (int)w, d, dqkv, w, p + off_wqkv(c, l), w, dxn, d, 0);

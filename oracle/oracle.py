@@ -19,7 +19,7 @@ _I64 = C.POINTER(C.c_int64)
 class OrcCfg(C.Structure):
     _fields_ = [("V", C.c_int32), ("d", C.c_int32), ("L", C.c_int32), ("H", C.c_int32),
                 ("Hkv", C.c_int32), ("h", C.c_int32), ("T", C.c_int32), ("B", C.c_int32),
-                ("rope_base", C.c_double), ("eps", C.c_double)]
+                ("rope_base", C.c_double), ("eps", C.c_double), ("rope_scale", C.c_double)]
 
 
 def _cfg(cfg) -> OrcCfg:
@@ -27,7 +27,7 @@ def _cfg(cfg) -> OrcCfg:
     ctx, batch, rope_base, rms_eps."""
     return OrcCfg(cfg["vocab"], cfg["d_model"], cfg["n_layer"], cfg["n_head"], cfg["n_kv_head"],
                   cfg["d_ff"], cfg["ctx"], cfg["batch"], float(cfg.get("rope_base", 10000.0)),
-                  float(cfg.get("rms_eps", 1e-5)))
+                  float(cfg.get("rms_eps", 1e-5)), float(cfg.get("rope_scale", 1.0)))
 
 
 def _dp(a):
@@ -58,6 +58,8 @@ _lib.orc_rmsnorm_bwd.restype = None
 _lib.orc_rmsnorm_bwd.argtypes = [C.c_int, C.c_int, _D, _D, _D, _D, _D, _D, C.c_int]
 _lib.orc_rope.restype = None
 _lib.orc_rope.argtypes = [_D, C.c_int, C.c_int, C.c_double, C.c_int]
+_lib.orc_rope_pos.restype = None
+_lib.orc_rope_pos.argtypes = [_D, C.c_int, C.c_double, C.c_double, C.c_int]
 _lib.orc_attention_fwd.restype = None
 _lib.orc_attention_fwd.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, _D, _D, _D, _D]
 _lib.orc_attention_bwd.restype = None
@@ -155,9 +157,13 @@ def rmsnorm_bwd(x, rstd, g, dy):
     return dx, dg
 
 
-def rope(u, t, base=10000.0, sign=1):
+def rope(u, t, base=10000.0, sign=1, scale=1.0):
+    """RoPE of head vector u at position t (t / scale with interpolation)."""
     u = _f64(u).copy()
-    _lib.orc_rope(_dp(u), u.shape[0], int(t), float(base), int(sign))
+    if scale == 1.0:
+        _lib.orc_rope(_dp(u), u.shape[0], int(t), float(base), int(sign))
+    else:
+        _lib.orc_rope_pos(_dp(u), u.shape[0], float(t) / float(scale), float(base), int(sign))
     return u
 
 

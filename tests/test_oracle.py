@@ -446,7 +446,7 @@ def test_gradcheck_gqa_small():
 # ------------------------------------------------- PyTorch float64 autograd
 
 
-def torch_model_loss(cfg, p, tok, tgt, pairing="half"):
+def torch_model_loss(cfg, p, tok, tgt, pairing="half", rope_scale=1.0):
     """Independent forward in PyTorch float64 (library ops: rms_norm, SDPA with
     GQA, silu, cross_entropy).  RoPE pairs dimension j with j + hd/2
     (rotate-half, the default) or 2j with 2j + 1 (pairing="interleaved"); pair
@@ -459,7 +459,7 @@ def torch_model_loss(cfg, p, tok, tgt, pairing="half"):
     P = {n: p[o:o + r * k].view(r, k) if r > 1 else p[o:o + k] for n, o, r, k in lay}
     tok_t = torch.tensor(tok, dtype=torch.long)
     x = P["wte"][tok_t]  # [B,T,d]
-    pos = torch.arange(T, dtype=torch.float64)
+    pos = torch.arange(T, dtype=torch.float64) / rope_scale
     inv = cfg["rope_base"] ** (-torch.arange(0, hd // 2, dtype=torch.float64) * 2 / hd)
     ang = pos[:, None] * inv[None, :]
     cos, sin = torch.cos(ang), torch.sin(ang)
@@ -555,6 +555,37 @@ def test_rope_pairings_differ_by_a_column_permutation():
     # without the permutation the two pairings are different models
     loss_plain, _, _ = O.forward_backward(cfg, p, tok, tgt)
     assert abs(loss_plain - lt.item()) > 1e-6
+
+
+def test_rope_position_interpolation():
+    """strata, RoPE row: position interpolation folds extended positions into
+    the trained range (position t / scale)."""
+    rng = np.random.default_rng(12)
+    hd = 16
+    u, k = rng.standard_normal(hd), rng.standard_normal(hd)
+    for t in (0, 1, 5, 1023):
+        np.testing.assert_array_equal(O.rope(u, 2 * t, scale=2.0), O.rope(u, t))
+    half = O.rope(u, 1, scale=2.0)  # two half steps make one step
+    np.testing.assert_allclose(O.rope(half, 1, scale=2.0), O.rope(u, 1), atol=1e-14)
+    # relative positions survive the scaling
+    a = O.rope(u, 7, scale=4.0) @ O.rope(k, 3, scale=4.0)
+    b = O.rope(u, 107, scale=4.0) @ O.rope(k, 103, scale=4.0)
+    assert abs(a - b) < 1e-11
+    # the model with a scale against PyTorch float64 autograd with scaled positions
+    cfg = dict(GQA_SMALL, ctx=7, rope_scale=2.5)
+    lay, p, tok, tgt = _setup(cfg, std=0.2)
+    loss, z, g = O.forward_backward(cfg, p, tok, tgt)
+    pt = torch.tensor(p, requires_grad=True)
+    lt, zt = torch_model_loss(cfg, pt, tok, tgt, rope_scale=2.5)
+    lt.backward()
+    assert abs(loss - lt.item()) <= 1e-12
+    np.testing.assert_allclose(z, zt.detach().numpy(), rtol=1e-10, atol=1e-12)
+    assert np.linalg.norm(g - pt.grad.numpy()) / np.linalg.norm(pt.grad.numpy()) <= 1e-10
+    # and scale 1 is the plain model
+    l1, _, _ = O.forward_backward(dict(cfg, rope_scale=1.0), p, tok, tgt, want_grads=False)
+    plain = {k_: v for k_, v in cfg.items() if k_ != "rope_scale"}
+    l0, _, _ = O.forward_backward(plain, p, tok, tgt, want_grads=False)
+    assert l1 == l0 and abs(l1 - loss) > 1e-9
 
 
 # ------------------------------------------------------------------- AdamW

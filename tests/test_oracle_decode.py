@@ -19,12 +19,14 @@ GQA_SMALL = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_hea
                        ctx=6, batch=2, init_std=0.3, name="gqa-small", index=9)
 
 
-@pytest.mark.parametrize("cfgname", ["c1", "gqa", "mqa"])
+@pytest.mark.parametrize("cfgname", ["c1", "gqa", "mqa", "gqa_interp"])
 def test_decode_equals_full_forward_at_every_position(cfgname):
     if cfgname == "c1":
         cfg = get_config("c1", batch=2)
     elif cfgname == "gqa":
         cfg = GQA_SMALL
+    elif cfgname == "gqa_interp":  # RoPE position interpolation, scale 2
+        cfg = dict(GQA_SMALL, rope_scale=2.0, name="gqa-small-interp")
     else:
         cfg = dict(GQA_SMALL, n_kv_head=1, name="mqa-small")
     c = dict(cfg, init_std=0.3)
