@@ -249,6 +249,15 @@ int llm_lr_at(const llm_lr_schedule *sched, int64_t t, float *lr);
  * (synchronising the stream first).  LLM_ERR_ARG for NaN. */
 int llm_set_grad_clip(llm_ctx *ctx, float max_norm);
 
+/* RoPE position interpolation (strata, RoPE row: context scaling folds
+ * extended positions into the trained range): every later call rotates q and
+ * k at position t by the angles (t / factor) * base^(-2j/hd) -- the forward,
+ * the backward and decode alike (the context's one angle table is rebuilt,
+ * on its stream).  factor = 1 is plain RoPE (the default); a model trained at
+ * context L runs at context factor * L with its positions in [0, L).
+ * LLM_ERR_ARG unless factor > 0 and finite. */
+int llm_set_rope_scale(llm_ctx *ctx, float factor);
+
 /* Inverted dropout in the training forward and backward of llm_step and
  * llm_grad (Hephaistos, Architecture at a glance: dropout on the embeddings,
  * the attention weights and the attention and MLP outputs; masks drawn by the

@@ -45,7 +45,9 @@ void gemm_simt(const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const f
                int64_t ldr, int splits, cudaStream_t s);
 
 // ------------------------------------------------------------- elementwise
-void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStream_t s);
+// cos/sin [T, hd/2] of the angles (t / scale) * base^(-2j/hd).
+void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStream_t s,
+                double scale = 1.0);
 // Low-precision (or float32) padded copy of one weight matrix.
 //   mode 0: dst[r, c] = src[r, c] (zero outside rows x cols), dst [rows_p, cols_p]
 //   mode 1: W13 interleave: src [rows, 2h], dst [rows, 2hp] block-interleaved

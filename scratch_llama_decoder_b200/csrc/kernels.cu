@@ -14,19 +14,23 @@ static inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1
 
 // ------------------------------------------------------------------ RoPE table
 // Hephaistos, Architecture at a glance (Positions): rotary embedding of q and
-// k.  theta_j = base^(-2j/hd); angle = t * theta_j for position t.  The table
-// is built once, in double precision, then rounded to float.
-__global__ void k_rope_table(float *cos_t, float *sin_t, int T, int half, int hd, double base) {
+// k.  theta_j = base^(-2j/hd); angle = (t / scale) * theta_j for position t
+// (scale 1; strata, RoPE row: position interpolation folds extended positions
+// into the trained range with scale > 1).  The table is built in double
+// precision, then rounded to float.
+__global__ void k_rope_table(float *cos_t, float *sin_t, int T, int half, int hd, double base,
+                             double scale) {
   int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= (int64_t)T * half) return;
   int t = (int)(i / half), j = (int)(i % half);
-  double ang = (double)t * pow(base, -2.0 * j / hd);
+  double ang = ((double)t / scale) * pow(base, -2.0 * j / hd);
   cos_t[i] = (float)cos(ang);
   sin_t[i] = (float)sin(ang);
 }
-void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStream_t s) {
+void rope_table(float *cos_t, float *sin_t, int T, int hd, float base, cudaStream_t s,
+                double scale) {
   int64_t n = (int64_t)T * (hd / 2);
-  k_rope_table<<<cdiv(n, 256), 256, 0, s>>>(cos_t, sin_t, T, hd / 2, hd, (double)base);
+  k_rope_table<<<cdiv(n, 256), 256, 0, s>>>(cos_t, sin_t, T, hd / 2, hd, (double)base, scale);
   count_launch();
 }
 

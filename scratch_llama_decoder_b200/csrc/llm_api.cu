@@ -409,6 +409,14 @@ int llm_set_grad_clip(llm_ctx *c, float max_norm) {
   return LLM_OK;
 }
 
+int llm_set_rope_scale(llm_ctx *c, float factor) {
+  if (!c || !(factor > 0.f) || !std::isfinite(factor)) return LLM_ERR_ARG;
+  g_launches = 0;
+  rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, c->cfg.rope_base, c->s, (double)factor);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
 int llm_set_dropout(llm_ctx *c, float p, uint64_t seed) {
   if (!c || !(p >= 0.f) || !(p < 1.f)) return LLM_ERR_ARG;
   if (p != c->drop_p || seed != c->drop_seed) {

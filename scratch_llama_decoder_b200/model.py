@@ -126,6 +126,10 @@ class LlamaStep:
                 "llm_sample")
         return out
 
+    def set_rope_scale(self, factor):
+        """RoPE position interpolation: positions t / factor (llm_set_rope_scale)."""
+        L.check(L.lib.llm_set_rope_scale(self.ctx, float(factor)), "llm_set_rope_scale")
+
     def set_dropout(self, p, seed):
         """Inverted dropout in later training calls (llm_set_dropout)."""
         L.check(L.lib.llm_set_dropout(self.ctx, float(p), int(seed)), "llm_set_dropout")

@@ -14,9 +14,10 @@ def pytest_configure(config):
 # Collection order for a run that stops at the first failure (-x): the parity
 # tests of the training step, its kernels and decode first, then the tests of
 # the entry points built on them (data parallelism, dropout, the extended
-# sampler), and last the
+# sampler, longer contexts), and last the
 # allocation-free entry, whose file sets up per-device state on first use.
-_LATE = ("test_gpu_dp.py", "test_gpu_dropout.py", "test_gpu_sample_ext.py")
+_LATE = ("test_gpu_dp.py", "test_gpu_dropout.py", "test_gpu_sample_ext.py",
+         "test_gpu_long_context.py")
 _LAST = ("test_zz_no_alloc.py",)
 
 

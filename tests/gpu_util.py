@@ -43,6 +43,8 @@ def run_gpu(cfg, params, tok, tgt, steps=1, lr=None, wd=None, clip=None):
     m = LlamaStep(cfg)
     if clip is not None:
         m.set_grad_clip(clip)
+    if cfg.get("rope_scale", 1.0) != 1.0:
+        m.set_rope_scale(cfg["rope_scale"])
     P = torch.tensor(params, dtype=torch.float32, device="cuda")
     G = torch.zeros_like(P)
     M = torch.zeros_like(P)
