@@ -150,6 +150,16 @@ int llm_grad(llm_ctx *ctx, const float *d_params, float *d_grads, const int32_t 
              const int32_t *d_targets, float *d_loss);
 int llm_adamw(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,
               float lr, float wd, float grad_scale);
+/* The update of llm_adamw over `count` consecutive elements for a sharded
+ * optimiser (each rank updates its 1/ranks of the parameters after a
+ * reduce-scatter of the gradient, then the ranks all-gather the parameters):
+ * d_params, d_grads, d_m and d_v each point at the range's first element
+ * (16-byte aligned); d_grads *= grad_scale, then AdamW with the context's
+ * betas and eps, skipped on the error word like llm_adamw.  No clipping (the
+ * global norm needs the whole gradient).  LLM_ERR_ARG for misaligned
+ * pointers, count < 0, t < 1 or a non-finite grad_scale. */
+int llm_adamw_range(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d_v,
+                    int64_t count, int64_t t, float lr, float wd, float grad_scale);
 int llm_flag_out(llm_ctx *ctx, int32_t *d_flag);
 int llm_flag_in(llm_ctx *ctx, const int32_t *d_flag);
 

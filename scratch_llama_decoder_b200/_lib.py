@@ -56,6 +56,7 @@ EXPORTS = {
     "llm_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _f, _f, _vp]),
     "llm_grad": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "llm_adamw": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _f, _f, _f]),
+    "llm_adamw_range": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _f, _f, _f]),
     "llm_flag_out": (_i, [_vp, _vp]),
     "llm_flag_in": (_i, [_vp, _vp]),
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),

@@ -931,6 +931,24 @@ int llm_adamw(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
 
+int llm_adamw_range(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v,
+                    int64_t count, int64_t t, float lr, float wd, float grad_scale) {
+  if (!c || t < 1 || count < 0 || !std::isfinite(grad_scale)) return LLM_ERR_ARG;
+  if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
+    return LLM_ERR_ARG;
+  g_launches = 0;
+  const double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
+  const double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
+  set_hyper(c->hyper, lr, wd, (float)bc1, (float)bc2, c->s);
+  if (count > 0) {
+    if (grad_scale != 1.0f) scale_grads(d_grads, count, grad_scale, c->s);
+    adamw(d_params, d_grads, d_m, d_v, count, c->hyper, c->cfg.beta1, c->cfg.beta2,
+          c->cfg.adam_eps, c->flag_step, c->s);
+  }
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
 int llm_flag_out(llm_ctx *c, int32_t *d_flag) {
   if (!c || !d_flag) return LLM_ERR_ARG;
   if (cudaMemcpyAsync(d_flag, c->flag_step, sizeof(int32_t), cudaMemcpyDeviceToDevice, c->s) !=

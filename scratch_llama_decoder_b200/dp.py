@@ -51,3 +51,64 @@ class DataParallelStep:
                 dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=self.group)
             e.adamw(params, grads, m, v, t, lr, wd, grad_scale=1.0 / self.world)
         return loss
+
+
+class ShardedDataParallelStep(DataParallelStep):
+    """The data-parallel step with the optimiser state sharded across ranks
+    (the parameters' Adam moments live only on the rank that updates them):
+      1. llm_grad on the rank's share of the batch, into a flat gradient
+         buffer padded to ranks x chunk elements (chunk a multiple of 4;
+         llm_grad writes the first n_params, the pad stays zero);
+      2. reduce-scatter (sum): each rank receives the summed gradient of its
+         chunk of the parameters;
+      3. the error words are combined (max) as in DataParallelStep;
+      4. llm_adamw_range on the rank's chunk with grad_scale = 1 / ranks;
+      5. all-gather of the updated chunks into every rank's parameters.
+    Per rank that moves a reduce-scatter plus an all-gather of the gradient's
+    size (together one all-reduce's traffic) and keeps 1 / ranks of m and v.
+    Clipping is not applied here (its norm needs the whole gradient).
+    buffers() allocates the padded parameter and gradient buffers and the
+    chunk-sized m and v."""
+
+    def __init__(self, engine, n_params, group=None):
+        super().__init__(engine, group)
+        self.rank = dist.get_rank(group) if self.world > 1 else 0
+        self.n = int(n_params)
+        self.chunk = ((self.n + self.world - 1) // self.world + 3) // 4 * 4
+        self.lo = self.rank * self.chunk
+        self.count = max(0, min(self.chunk, self.n - self.lo))
+        self._gshard = None
+
+    def buffers(self, dtype=torch.float32):
+        dev = self.engine.device
+        padded = self.world * self.chunk
+        return (torch.zeros(padded, dtype=dtype, device=dev),
+                torch.zeros(padded, dtype=dtype, device=dev),
+                torch.zeros(self.chunk, dtype=dtype, device=dev),
+                torch.zeros(self.chunk, dtype=dtype, device=dev))
+
+    def step(self, params, grads, m, v, t, tokens, targets, lr, wd, loss):
+        e = self.engine
+        C, lo, cnt = self.chunk, self.lo, self.count
+        with self._stream():
+            e.grad(params, grads, tokens, targets, loss)
+            if self.world > 1:
+                if self._gshard is None:
+                    self._gshard = torch.zeros(C, dtype=grads.dtype, device=grads.device)
+                dist.reduce_scatter_tensor(self._gshard, grads, op=dist.ReduceOp.SUM,
+                                           group=self.group)
+                e.flag_out(self.flag)
+                dist.all_reduce(self.flag, op=dist.ReduceOp.MAX, group=self.group)
+                e.flag_in(self.flag)
+                dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=self.group)
+                gs = self._gshard
+            else:
+                gs = grads
+            e.adamw_range(params[lo:lo + cnt], gs[:cnt], m[:cnt], v[:cnt], t, lr, wd,
+                          grad_scale=1.0 / self.world)
+            if self.world > 1:
+                src = params[lo:lo + C]
+                if dist.get_backend(self.group) != "nccl":
+                    src = src.clone()  # in place only where the backend documents it
+                dist.all_gather_into_tensor(params, src, group=self.group)
+        return loss

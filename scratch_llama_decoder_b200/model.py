@@ -99,6 +99,15 @@ class LlamaStep:
         L.check(L.lib.llm_adamw(self.ctx, _ptr(params), _ptr(grads), _ptr(m), _ptr(v), int(t),
                                 float(lr), float(wd), float(grad_scale)), "llm_adamw")
 
+    def adamw_range(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
+        """AdamW over the elements of 1-D views params, grads, m, v (equal
+        lengths; llm_adamw_range)."""
+        n = params.numel()
+        assert grads.numel() == n and m.numel() == n and v.numel() == n
+        L.check(L.lib.llm_adamw_range(self.ctx, _ptr(params), _ptr(grads), _ptr(m), _ptr(v), n,
+                                      int(t), float(lr), float(wd), float(grad_scale)),
+                "llm_adamw_range")
+
     def flag_out(self, flag):
         """Copy the step's int32 error word to flag (llm_flag_out)."""
         L.check(L.lib.llm_flag_out(self.ctx, _ptr(flag)), "llm_flag_out")

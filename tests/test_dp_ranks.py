@@ -31,9 +31,10 @@ class OracleEngine:
     def grad(self, params, grads, tokens, targets, loss):
         import oracle as O
         self.calls += 1
-        lv, _, g = O.forward_backward(self.cfg, params.numpy(), tokens.numpy(), targets.numpy(),
-                                      want_logits=False)
-        grads.copy_(torch.from_numpy(g))
+        n = O.n_params(self.cfg)  # buffers may be padded past the parameters
+        lv, _, g = O.forward_backward(self.cfg, params.numpy()[:n], tokens.numpy(),
+                                      targets.numpy(), want_logits=False)
+        grads[:n].copy_(torch.from_numpy(g))
         loss.fill_(lv)
         self.flag = 1 if self.calls == self.fail_at else 0
 
@@ -42,6 +43,16 @@ class OracleEngine:
 
     def flag_in(self, f):
         self.flag |= int(f.item())
+
+    def adamw_range(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
+        import oracle as O
+        grads.mul_(grad_scale)
+        if self.flag or params.numel() == 0:
+            return
+        p2, m2, v2 = O.adamw(params.numpy(), grads.numpy(), m.numpy(), v.numpy(), t, lr, wd)
+        params.copy_(torch.from_numpy(p2))
+        m.copy_(torch.from_numpy(m2))
+        v.copy_(torch.from_numpy(v2))
 
     def adamw(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
         import oracle as O
@@ -77,6 +88,35 @@ def _run(engine, dp, p, tok, tgt, steps, lr, wd):
         dp.step(P, G, M, V, t, torch.tensor(tok), torch.tensor(tgt), lr, wd, loss)
         losses.append(float(loss.item()))
     return P.numpy(), M.numpy(), V.numpy(), losses
+
+
+def _rank_main_sharded(rank, world, port, full_cfg, steps, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    from scratch_llama_decoder_b200.dp import ShardedDataParallelStep
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        p, tok, tgt = _setup(full_cfg)
+        share = full_cfg["batch"] // world
+        cfg = dict(full_cfg, batch=share)
+        eng = OracleEngine(cfg)
+        dp = ShardedDataParallelStep(eng, O.n_params(cfg))
+        P, G, M, V = dp.buffers(torch.float64)
+        P[:p.size].copy_(torch.from_numpy(p))
+        loss = torch.zeros(1, dtype=torch.float64)
+        for t in range(1, steps + 1):
+            dp.step(P, G, M, V, t, torch.tensor(tok[rank * share:(rank + 1) * share]),
+                    torch.tensor(tgt[rank * share:(rank + 1) * share]), full_cfg["lr"],
+                    full_cfg["wd"], loss)
+        q.put((rank, (P[:p.size].numpy().copy(), M[:dp.count].numpy().copy(),
+                      V[:dp.count].numpy().copy(), dp.lo, dp.count)))
+    finally:
+        dist.destroy_process_group()
 
 
 def _rank_main(rank, world, port, full_cfg, steps, fail_rank, fail_at, q):
@@ -144,3 +184,34 @@ def test_an_error_on_one_rank_skips_the_update_on_both():
     for r in (0, 1):
         # step 2 was skipped everywhere: parameters stay at their step-1 values
         np.testing.assert_array_equal(res[r][0], res_ok[r][0])
+
+
+def test_sharded_optimiser_two_ranks_equal_one_process():
+    """Reduce-scatter, AdamW on each rank's chunk, all-gather: the parameters
+    of the one-process step on the whole batch, and the ranks' moment chunks
+    are that step's moments."""
+    from synth import get_config
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    full = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_head=2, d_ff=42,
+                      ctx=5, batch=2, init_std=0.3, name="gqa-small", index=9)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_sharded, args=(r, 2, port, full, 3, q))
+             for r in range(2)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=300) for _ in range(2))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    p, tok, tgt = _setup(full)
+    eng = OracleEngine(full)
+    ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 3, full["lr"], full["wd"])
+    for r in (0, 1):
+        P, Mc, Vc, lo, cnt = res[r]
+        np.testing.assert_allclose(P, ref[0], rtol=1e-12, atol=1e-15)
+        np.testing.assert_allclose(Mc, ref[1][lo:lo + cnt], rtol=1e-10, atol=1e-18)
+        np.testing.assert_allclose(Vc, ref[2][lo:lo + cnt], rtol=1e-10, atol=1e-22)
+    np.testing.assert_array_equal(res[0][0], res[1][0])
+    assert res[0][4] + res[1][4] == p.size  # the chunks cover every parameter once

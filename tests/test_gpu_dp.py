@@ -100,3 +100,30 @@ def test_error_word_in_and_out():
     assert L.lib.llm_adamw(m.ctx, P.data_ptr(), G.data_ptr(), M.data_ptr(), V.data_ptr(), 1,
                            1e-3, 0.1, float("inf")) == L.LLM_ERR_ARG
     m.close()
+
+
+def test_sharded_step_on_one_rank_is_step():
+    """ShardedDataParallelStep without a process group (one chunk holding
+    every parameter) gives llm_step's parameters, gradient and moments bit
+    for bit; its buffers are padded past the parameters."""
+    from scratch_llama_decoder_b200.dp import ShardedDataParallelStep
+    cfg, m, P, G, M, V, td, yd = _setup()
+    loss = torch.zeros(1, device="cuda")
+    for t in range(1, 3):
+        m.step(P, G, M, V, t, td, yd, cfg["lr"], cfg["wd"], loss)
+    ref = _state(P, G, M, V, loss)
+    m.close()
+    cfg, m, P, G, M, V, td, yd = _setup()
+    dp = ShardedDataParallelStep(m, m.n_params)
+    assert dp.world == 1 and dp.count == m.n_params and dp.chunk % 4 == 0
+    Pp, Gp, Mp, Vp = dp.buffers()
+    n = m.n_params
+    Pp[:n].copy_(P)
+    for t in range(1, 3):
+        dp.step(Pp, Gp, Mp, Vp, t, td, yd, cfg["lr"], cfg["wd"], loss)
+    torch.cuda.synchronize()
+    got = [Pp[:n].cpu(), Gp[:n].cpu(), Mp[:n].cpu(), Vp[:n].cpu(), loss.cpu()]
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    assert not Gp[n:].any()  # the pad past the parameters stays zero
+    m.close()
