@@ -215,3 +215,24 @@ def test_sharded_optimiser_two_ranks_equal_one_process():
         np.testing.assert_allclose(Vc, ref[2][lo:lo + cnt], rtol=1e-10, atol=1e-22)
     np.testing.assert_array_equal(res[0][0], res[1][0])
     assert res[0][4] + res[1][4] == p.size  # the chunks cover every parameter once
+
+
+def test_sharded_wrapper_on_one_rank_is_the_plain_wrapper():
+    import oracle as O
+    from synth import get_config
+    from scratch_llama_decoder_b200.dp import DataParallelStep, ShardedDataParallelStep
+    cfg = get_config("c1", batch=2)
+    p, tok, tgt = _setup(cfg)
+    eng = OracleEngine(cfg)
+    ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 2, cfg["lr"], cfg["wd"])
+    eng = OracleEngine(cfg)
+    dp = ShardedDataParallelStep(eng, O.n_params(cfg))
+    assert dp.world == 1 and dp.count == p.size and dp.chunk >= p.size and dp.chunk % 4 == 0
+    P, G, M, V = dp.buffers(torch.float64)
+    P[:p.size].copy_(torch.from_numpy(p))
+    loss = torch.zeros(1, dtype=torch.float64)
+    for t in (1, 2):
+        dp.step(P, G, M, V, t, torch.tensor(tok), torch.tensor(tgt), cfg["lr"], cfg["wd"], loss)
+    np.testing.assert_array_equal(P[:p.size].numpy(), ref[0])
+    np.testing.assert_array_equal(M[:p.size].numpy(), ref[1])
+    assert not G[p.size:].any() and not P[p.size:].any()
