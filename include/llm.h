@@ -65,11 +65,18 @@ enum { LLM_FP32 = 0, LLM_BF16 = 1 };
  * float32 accumulation, keeping float32 master weights, Adam state and the
  * residual stream.  rope_base: RoPE base (10000); rms_eps: RMSNorm epsilon
  * added to the mean square (MicroGPT in Rust, "RMSNorm": 1e-5); beta1, beta2,
- * adam_eps: AdamW constants (eps is added outside the square root). */
+ * adam_eps: AdamW constants (eps is added outside the square root).
+ * recompute = 1 keeps only each layer's input between the forward and the
+ * backward and recomputes the layer's other activations from it in the
+ * backward (the same kernels, so the gradients do not change); it cuts the
+ * workspace by the saved activations of all but one layer at the cost of a
+ * second forward of every layer, and llm_decode (whose cache is every layer's
+ * saved q|k|v) returns LLM_ERR_CONFIG.  0 keeps them (the default). */
 typedef struct {
   int32_t vocab, d_model, n_layer, n_head, n_kv_head, d_ff, ctx, batch;
   float rope_base, rms_eps, beta1, beta2, adam_eps;
   int32_t compute;
+  int32_t recompute;
 } llm_config;
 
 /* One tensor of the flat parameter buffer: element (r, c) of a [rows, cols]

@@ -26,7 +26,7 @@ class llm_config(C.Structure):
                 ("n_head", C.c_int32), ("n_kv_head", C.c_int32), ("d_ff", C.c_int32),
                 ("ctx", C.c_int32), ("batch", C.c_int32), ("rope_base", C.c_float),
                 ("rms_eps", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float),
-                ("adam_eps", C.c_float), ("compute", C.c_int32)]
+                ("adam_eps", C.c_float), ("compute", C.c_int32), ("recompute", C.c_int32)]
 
 
 class llm_tensor_info(C.Structure):
@@ -112,7 +112,8 @@ def make_config(cfg) -> llm_config:
                       cfg["n_kv_head"], cfg["d_ff"], cfg["ctx"], cfg["batch"],
                       float(cfg.get("rope_base", 10000.0)), float(cfg.get("rms_eps", 1e-5)),
                       float(cfg.get("beta1", 0.9)), float(cfg.get("beta2", 0.999)),
-                      float(cfg.get("adam_eps", 1e-8)), int(comp))
+                      float(cfg.get("adam_eps", 1e-8)), int(comp),
+                      int(cfg.get("recompute", 0)))
 
 
 def llm_param_layout(cfg):

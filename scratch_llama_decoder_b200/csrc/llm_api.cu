@@ -28,6 +28,8 @@ struct Dims {
   int64_t N, qkvw, hp, Vp, P, layer_sz;
   DType dt;
   int ab;  // bytes of one activation element
+  bool rc;  // recompute: one slot of per-layer activations
+  int LS;   // slots of per-layer activations (L, or 1 with recompute)
 };
 
 bool valid_config(const llm_config *c) {
@@ -41,6 +43,7 @@ bool valid_config(const llm_config *c) {
   if (hd % 2 || hd > 128) return false;
   if (c->d_model % 4 || c->d_model > 4096) return false;
   if (c->compute != LLM_FP32 && c->compute != LLM_BF16) return false;
+  if (c->recompute != 0 && c->recompute != 1) return false;
   if (!(c->rms_eps >= 0.f) || !(c->rope_base > 0.f)) return false;
   if ((int64_t)c->batch * c->ctx > (int64_t)1 << 30) return false;
   return true;
@@ -59,6 +62,8 @@ Dims make_dims(const llm_config *c) {
   D.P = (int64_t)D.V * D.d + D.L * D.layer_sz + D.d + (int64_t)D.d * D.V;
   D.dt = c->compute == LLM_BF16 ? DT_BF16 : DT_F32;
   D.ab = D.dt == DT_BF16 ? 2 : 4;
+  D.rc = c->recompute != 0;
+  D.LS = D.rc ? std::min(1, D.L) : D.L;
   return D;
 }
 
@@ -200,16 +205,17 @@ int64_t llm_ctx::carve(char *base) {
   w_2 = c.take(ab * L * D_.hp * d);
   w_lm = c.take(ab * d * D_.Vp);
   xs = (float *)c.take(4 * (L + 1) * N * d);
-  x1 = (float *)c.take(4 * L * N * d);
-  xn1 = c.take(ab * L * N * d);
-  qkv = c.take(ab * L * N * D_.qkvw);
-  o = c.take(ab * L * N * d);
-  xn2 = c.take(ab * L * N * d);
-  this->ab = c.take(ab * L * N * 2 * D_.hp);
-  u = c.take(ab * L * N * D_.hp);
-  rstd1 = (float *)c.take(4 * L * N);
-  rstd2 = (float *)c.take(4 * L * N);
-  lse = (float *)c.take(4 * L * N * D_.H);
+  const int64_t LS = D_.LS;  // per-layer activation slots
+  x1 = (float *)c.take(4 * LS * N * d);
+  xn1 = c.take(ab * LS * N * d);
+  qkv = c.take(ab * LS * N * D_.qkvw);
+  o = c.take(ab * LS * N * d);
+  xn2 = c.take(ab * LS * N * d);
+  this->ab = c.take(ab * LS * N * 2 * D_.hp);
+  u = c.take(ab * LS * N * D_.hp);
+  rstd1 = (float *)c.take(4 * LS * N);
+  rstd2 = (float *)c.take(4 * LS * N);
+  lse = (float *)c.take(4 * LS * N * D_.H);
   xf = c.take(ab * N * d);
   logits = c.take(ab * N * D_.Vp);
   rstdf = (float *)c.take(4 * N);
@@ -559,6 +565,61 @@ DropArgs drop_args(const llm_ctx *c, int site, int layer) {
 }
 bool dropping(const llm_ctx *c) { return c->drop_p > 0.f; }
 
+// One layer of the forward from its input xs[l]: the activations the
+// backward reads go to slot sl (l, or 0 with recompute), and with `out` the
+// layer output xs[l + 1] too.
+void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
+  const Dims &D = c->D;
+  POff O{D};
+  cudaStream_t s = c->s;
+  const int64_t N = D.N, d = D.d;
+  const int ab = D.ab;
+  auto A = [&](void *base, int64_t k, int64_t per) { return (char *)base + k * per * ab; };
+  float *x = c->xs + l * N * d, *x1 = c->x1 + sl * N * d, *x2 = c->xs + (l + 1) * N * d;
+  void *xn1 = A(c->xn1, sl, N * d), *qkv = A(c->qkv, sl, N * D.qkvw), *o = A(c->o, sl, N * d);
+  void *xn2 = A(c->xn2, sl, N * d), *abuf = A(c->ab, sl, N * 2 * D.hp), *u = A(c->u, sl, N * D.hp);
+  float *rstd1 = c->rstd1 + sl * N, *rstd2 = c->rstd2 + sl * N, *lse = c->lse + sl * N * D.H;
+  void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
+  void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
+  // x1 = x + Attn(RMSNorm_g1(x))
+  rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
+  {
+    GemmOperands g{(int)N, (int)D.qkvw, D.d, xn1, d, true, wqkv, D.qkvw, false, D.dt};
+    bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
+                        2.0 * N * d * D.qkvw);
+    if (!fused) {
+      gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
+      rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
+    }
+  }
+  if (drop) {  // x1 = x + f * (o Wo), o from dropped probabilities
+    attn_fwd_simt(qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
+    gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_F32, c->dtmp, d,
+         nullptr, 0, 1, 2.0 * N * d * d);
+    drop_add(x, c->dtmp, x1, N * d, drop_args(c, 2, l), s);
+  } else {
+    attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
+    gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d,
+         x, d, 1, 2.0 * N * d * d);
+  }
+  // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
+  rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
+  // W13 GEMM into the interleaved [a|b], then u = silu(a) * b (a separate
+  // full-occupancy pass: cheaper than the same math in the GEMM epilogue)
+  gemm(c, GemmOperands{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt},
+       OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
+  swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
+  if (!out) return;  // the recomputation stops here: x2 exists
+  if (drop) {  // x2 = x1 + f * (u W2)
+    gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_F32,
+         c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.h * d);
+    drop_add(x1, c->dtmp, x2, N * d, drop_args(c, 3, l), s);
+  } else {
+    gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt},
+         OUT_ADD_F32, x2, d, x1, d, 1, 2.0 * N * D.h * d);
+  }
+}
+
 // Forward pass; leaves logits (padded, activation type) in c->logits.  train:
 // a training forward (dropout applies when set; evaluation never drops).
 // With dropout on, attention runs in the CUDA-core kernels, which draw the
@@ -569,8 +630,6 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok, bool train) {
   POff O{D};
   cudaStream_t s = c->s;
   const int64_t N = D.N, d = D.d;
-  const int ab = D.ab;
-  auto A = [&](void *base, int64_t l, int64_t per) { return (char *)base + l * per * ab; };
   // low-precision (or float32) padded copies of the weight matrices
   if (D.L > 0) {
     cast_weight(p + O.wqkv(0), c->w_qkv, D.dt, d, D.qkvw, d, D.qkvw, 0, 0, 0, D.L, D.layer_sz,
@@ -583,50 +642,7 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok, bool train) {
   cast_weight(p + O.wlm(), c->w_lm, D.dt, d, D.V, d, D.Vp, 0, 0, 0, 1, 0, 0, s);
   embed_fwd(p, tok, c->xs, N, D.d, D.V, c->flag_step, s);
   if (drop) drop_rows(c->xs, N * d, drop_args(c, 0, 0), s);
-  for (int l = 0; l < D.L; l++) {
-    float *x = c->xs + l * N * d, *x1 = c->x1 + l * N * d, *x2 = c->xs + (l + 1) * N * d;
-    void *xn1 = A(c->xn1, l, N * d), *qkv = A(c->qkv, l, N * D.qkvw), *o = A(c->o, l, N * d);
-    void *xn2 = A(c->xn2, l, N * d), *abuf = A(c->ab, l, N * 2 * D.hp), *u = A(c->u, l, N * D.hp);
-    float *rstd1 = c->rstd1 + l * N, *rstd2 = c->rstd2 + l * N, *lse = c->lse + l * N * D.H;
-    void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
-    void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
-    // x1 = x + Attn(RMSNorm_g1(x))
-    rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
-    {
-      GemmOperands g{(int)N, (int)D.qkvw, D.d, xn1, d, true, wqkv, D.qkvw, false, D.dt};
-      bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
-                          2.0 * N * d * D.qkvw);
-      if (!fused) {
-        gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
-        rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
-      }
-    }
-    if (drop) {  // x1 = x + f * (o Wo), o from dropped probabilities
-      attn_fwd_simt(qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
-      gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_F32, c->dtmp, d,
-           nullptr, 0, 1, 2.0 * N * d * d);
-      drop_add(x, c->dtmp, x1, N * d, drop_args(c, 2, l), s);
-    } else {
-      attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
-      gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d,
-           x, d, 1, 2.0 * N * d * d);
-    }
-    // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
-    rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
-    // W13 GEMM into the interleaved [a|b], then u = silu(a) * b (a separate
-    // full-occupancy pass: cheaper than the same math in the GEMM epilogue)
-    gemm(c, GemmOperands{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt},
-         OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
-    swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
-    if (drop) {  // x2 = x1 + f * (u W2)
-      gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_F32,
-           c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.h * d);
-      drop_add(x1, c->dtmp, x2, N * d, drop_args(c, 3, l), s);
-    } else {
-      gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt},
-           OUT_ADD_F32, x2, d, x1, d, 1, 2.0 * N * D.h * d);
-    }
-  }
+  for (int l = 0; l < D.L; l++) layer_fwd(c, p, l, D.rc ? 0 : l, drop, true);
   float *xL = c->xs + D.L * N * d;
   rmsnorm_fwd(xL, p + O.gf(), c->xf, D.dt, c->rstdf, N, D.d, c->cfg.rms_eps, s);
   gemm(c, GemmOperands{(int)N, (int)D.Vp, D.d, c->xf, d, true, c->w_lm, D.Vp, false, D.dt},
@@ -692,10 +708,14 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
                    D.d, s);
   reduce_partials(c->dgpart, nb, D.d, gr + O.gf(), s);
   for (int l = D.L - 1; l >= 0; l--) {
-    float *x = c->xs + l * N * d, *x1 = c->x1 + l * N * d;
-    void *xn1 = A(c->xn1, l, N * d), *qkv = A(c->qkv, l, N * D.qkvw), *o = A(c->o, l, N * d);
-    void *xn2 = A(c->xn2, l, N * d), *abuf = A(c->ab, l, N * 2 * D.hp), *u = A(c->u, l, N * D.hp);
-    float *rstd1 = c->rstd1 + l * N, *rstd2 = c->rstd2 + l * N, *lse = c->lse + l * N * D.H;
+    // with recompute, the layer's activations come back from its input first
+    // (the side stream finished with the slot at the end of layer l + 1)
+    const int sl = D.rc ? 0 : l;
+    if (D.rc) layer_fwd(c, p, l, 0, drop, false);
+    float *x = c->xs + l * N * d, *x1 = c->x1 + sl * N * d;
+    void *xn1 = A(c->xn1, sl, N * d), *qkv = A(c->qkv, sl, N * D.qkvw), *o = A(c->o, sl, N * d);
+    void *xn2 = A(c->xn2, sl, N * d), *abuf = A(c->ab, sl, N * 2 * D.hp), *u = A(c->u, sl, N * D.hp);
+    float *rstd1 = c->rstd1 + sl * N, *rstd2 = c->rstd2 + sl * N, *lse = c->lse + sl * N * D.H;
     void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
     void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
     // FFN branch.  du = dx2 W2^T, then SwiGLU backward into dab.
@@ -970,7 +990,7 @@ int llm_decode(llm_ctx *c, const float *d_params, const int32_t *d_tokens, int p
   if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;
   const Dims &D = c->D;
   if (pos < 0 || pos >= D.T) return LLM_ERR_ARG;
-  if (128 % D.hd) return LLM_ERR_CONFIG;
+  if (128 % D.hd || D.rc) return LLM_ERR_CONFIG;
   if (((uintptr_t)d_params & 3) || ((uintptr_t)d_tokens & 3) || ((uintptr_t)d_logits & 3))
     return LLM_ERR_ARG;
   g_launches = 0;

@@ -108,3 +108,23 @@ def test_bad_arguments_rejected_on_host():
     assert P.lib.llm_status(None) == P.LLM_ERR_ARG
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert P.lib.llm_error_string(code)
+
+
+def test_recompute_workspace_keeps_one_layer_of_activations():
+    """recompute = 1 drops the saved activations of all but one layer: the
+    workspace shrinks by (L - 1) x (x1 in float32; xn1, q|k|v, o, xn2, [a|b],
+    u in the operand type; rstd1, rstd2, lse in float32), up to alignment."""
+    from scratch_llama_decoder_b200 import llm_workspace_bytes
+    from synth import get_config
+    cfg = get_config("c5")
+    w0 = llm_workspace_bytes(cfg)
+    w1 = llm_workspace_bytes(dict(cfg, recompute=1))
+    N, d, L, H = cfg["batch"] * cfg["ctx"], cfg["d_model"], cfg["n_layer"], cfg["n_head"]
+    hp = (cfg["d_ff"] + 63) // 64 * 64
+    qkvw = d + 2 * cfg["n_kv_head"] * (d // H)
+    per_layer = 4 * N * d + 2 * N * (d + qkvw + d + d + 2 * hp + hp) + 4 * N * (2 + H)
+    assert abs((w0 - w1) - (L - 1) * per_layer) <= 11 * 256
+    assert w1 < w0 / 3  # the 350M step's workspace is mostly saved activations
+    import scratch_llama_decoder_b200 as P
+    with pytest.raises(P.LLMError):
+        llm_workspace_bytes(dict(cfg, recompute=2))

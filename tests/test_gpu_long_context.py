@@ -69,3 +69,32 @@ def test_decode_with_rope_scale_matches_full_forward():
     assert L.lib.llm_set_rope_scale(m.ctx, 0.0) == L.LLM_ERR_ARG
     assert L.lib.llm_set_rope_scale(m.ctx, float("inf")) == L.LLM_ERR_ARG
     m.close()
+
+
+@pytest.mark.parametrize("dropout", [0.0, 0.2])
+def test_recompute_is_bit_identical_to_stored_activations(dropout):
+    from scratch_llama_decoder_b200 import LlamaStep
+    res = []
+    for rc in (0, 1):
+        cfg = get_config("c3", batch=2, ctx=96, n_layer=3, recompute=rc)
+        p = make_params(cfg, O.param_layout(cfg))
+        tok, tgt = make_batch(cfg)
+        m = LlamaStep(cfg)
+        if dropout:
+            m.set_dropout(dropout, 77)
+        P = torch.tensor(p, device="cuda")
+        G, M, V = (torch.zeros_like(P) for _ in range(3))
+        loss = torch.zeros(1, device="cuda")
+        td, yd = torch.tensor(tok, device="cuda"), torch.tensor(tgt, device="cuda")
+        for t in (1, 2):
+            m.step(P, G, M, V, t, td, yd, cfg["lr"], cfg["wd"], loss)
+        assert m.status() == 0
+        res.append([x.cpu() for x in (P, G, M, V, loss)])
+        if rc:
+            import scratch_llama_decoder_b200 as L
+            lg = torch.empty(2, cfg["vocab"], device="cuda")
+            assert L.lib.llm_decode(m.ctx, P.data_ptr(), td[:, 0].contiguous().data_ptr(), 0,
+                                    lg.data_ptr()) == L.LLM_ERR_CONFIG
+        m.close()
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
