@@ -255,6 +255,27 @@ typedef struct {
 } llm_lr_schedule;
 int llm_lr_at(const llm_lr_schedule *sched, int64_t t, float *lr);
 
+/* Learning-rate reduction on a plateau (host only; randyGPT, Training:
+ * ReduceLROnPlateau halves max_lr on stagnation, up to 3 times, patience 30).
+ * llm_plateau_init sets factor, patience, max_reductions and a relative
+ * threshold and starts the scale at 1.  llm_plateau_update takes one
+ * evaluation's metric (lower is better): a metric below best * (1 -
+ * threshold) becomes the best and restarts the count; otherwise the count
+ * grows, and once it exceeds patience the scale is multiplied by factor (at
+ * most max_reductions times) and the count restarts.  *scale receives the
+ * current scale, to multiply the schedule's rate by.  LLM_ERR_ARG for a null
+ * pointer, factor outside (0, 1], a negative patience or max_reductions, a
+ * threshold outside [0, 1) or a NaN metric. */
+typedef struct {
+  double best, threshold, scale;
+  int64_t bad, patience;
+  int32_t reductions, max_reductions;
+  float factor;
+} llm_plateau;
+int llm_plateau_init(llm_plateau *pl, float factor, int64_t patience, int32_t max_reductions,
+                     double threshold);
+int llm_plateau_update(llm_plateau *pl, double metric, float *scale);
+
 /* Global-norm gradient clipping inside llm_step (MicroGPT in Rust, Gradient
  * Clipping: when the gradient norm exceeds max_norm every gradient is scaled
  * by max_norm / norm; Transformer-In-Rust: clipping by global norm).  With

@@ -22,6 +22,12 @@ Clipping (MicroGPT in Rust, Gradient Clipping: when the gradient norm exceeds
 max_norm every gradient is scaled by max_norm / norm, else left alone;
 Transformer-In-Rust: by global norm).  The norm is the Euclidean norm of all
 gradient elements together.
+
+Plateau (randyGPT, Training: ReduceLROnPlateau halves max_lr on stagnation, up
+to 3 times, patience 30).  Readings: a metric counts as better when it is
+below best * (1 - threshold) (threshold 0: strictly below); after more than
+`patience` evaluations in a row without a better one the scale is multiplied
+by `factor` (at most `max_reductions` times) and the count restarts.
 """
 import math
 
@@ -57,3 +63,23 @@ def clip(g, max_norm):
     n = grad_norm(g)
     s = clip_scale(n, max_norm)
     return np.asarray(g, dtype=np.float64) * s, n, s
+
+
+class Plateau:
+    """Learning-rate scale after each evaluation (starts at 1)."""
+
+    def __init__(self, factor=0.5, patience=30, max_reductions=3, threshold=0.0):
+        self.factor, self.patience = factor, patience
+        self.max_reductions, self.threshold = max_reductions, threshold
+        self.best, self.bad, self.reductions, self.scale = math.inf, 0, 0, 1.0
+
+    def update(self, metric):
+        if metric < self.best * (1.0 - self.threshold):
+            self.best, self.bad = metric, 0
+        else:
+            self.bad += 1
+            if self.bad > self.patience and self.reductions < self.max_reductions:
+                self.reductions += 1
+                self.scale *= self.factor
+                self.bad = 0
+        return self.scale

@@ -38,6 +38,12 @@ LLM_LR_CONSTANT, LLM_LR_COSINE, LLM_LR_LINEAR = 0, 1, 2
 LR_SHAPES = {"constant": LLM_LR_CONSTANT, "cosine": LLM_LR_COSINE, "linear": LLM_LR_LINEAR}
 
 
+class llm_plateau(C.Structure):
+    _fields_ = [("best", C.c_double), ("threshold", C.c_double), ("scale", C.c_double),
+                ("bad", C.c_int64), ("patience", C.c_int64), ("reductions", C.c_int32),
+                ("max_reductions", C.c_int32), ("factor", C.c_float)]
+
+
 class llm_lr_schedule(C.Structure):
     _fields_ = [("max_lr", C.c_float), ("min_lr", C.c_float), ("warmup_steps", C.c_int64),
                 ("decay_start", C.c_int64), ("total_steps", C.c_int64), ("shape", C.c_int32)]
@@ -67,6 +73,8 @@ EXPORTS = {
     "llm_set_rope_scale": (_i, [_vp, _f]),
     "llm_read_grad_norm": (_i, [_vp, C.POINTER(C.c_double)]),
     "llm_lr_at": (_i, [C.POINTER(llm_lr_schedule), _i64, C.POINTER(_f)]),
+    "llm_plateau_init": (_i, [C.POINTER(llm_plateau), _f, _i64, C.c_int32, C.c_double]),
+    "llm_plateau_update": (_i, [C.POINTER(llm_plateau), C.c_double, C.POINTER(_f)]),
     "llm_status": (_i, [_vp]),
     "llm_error_string": (C.c_char_p, [_i]),
     "llm_last_launch_count": (_i, [_vp]),
@@ -140,3 +148,18 @@ def lr_at(t, max_lr, min_lr, warmup, decay_start, total, shape="cosine") -> floa
     out = C.c_float(0.0)
     check(lib.llm_lr_at(C.byref(sc), int(t), C.byref(out)), "llm_lr_at")
     return out.value
+
+
+class Plateau:
+    """Learning-rate reduction on a plateau (llm_plateau_init / _update)."""
+
+    def __init__(self, factor=0.5, patience=30, max_reductions=3, threshold=0.0):
+        self._s = llm_plateau()
+        check(lib.llm_plateau_init(C.byref(self._s), float(factor), int(patience),
+                                   int(max_reductions), float(threshold)), "llm_plateau_init")
+
+    def update(self, metric) -> float:
+        out = C.c_float(1.0)
+        check(lib.llm_plateau_update(C.byref(self._s), float(metric), C.byref(out)),
+              "llm_plateau_update")
+        return out.value

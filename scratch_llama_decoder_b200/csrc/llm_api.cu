@@ -472,6 +472,36 @@ int llm_lr_at(const llm_lr_schedule *sc, int64_t t, float *lr) {
   return LLM_OK;
 }
 
+int llm_plateau_init(llm_plateau *pl, float factor, int64_t patience, int32_t max_reductions,
+                     double threshold) {
+  if (!pl || !(factor > 0.f) || !(factor <= 1.f) || patience < 0 || max_reductions < 0 ||
+      !(threshold >= 0.0) || !(threshold < 1.0))
+    return LLM_ERR_ARG;
+  pl->best = INFINITY;
+  pl->threshold = threshold;
+  pl->scale = 1.0;
+  pl->bad = 0;
+  pl->patience = patience;
+  pl->reductions = 0;
+  pl->max_reductions = max_reductions;
+  pl->factor = factor;
+  return LLM_OK;
+}
+
+int llm_plateau_update(llm_plateau *pl, double metric, float *scale) {
+  if (!pl || !scale || metric != metric) return LLM_ERR_ARG;
+  if (metric < pl->best * (1.0 - pl->threshold)) {
+    pl->best = metric;
+    pl->bad = 0;
+  } else if (++pl->bad > pl->patience && pl->reductions < pl->max_reductions) {
+    pl->reductions++;
+    pl->scale *= (double)pl->factor;
+    pl->bad = 0;
+  }
+  *scale = (float)pl->scale;
+  return LLM_OK;
+}
+
 int llm_read_kernel_timing(llm_ctx *c, double *ms, double *flops, int64_t *launches) {
   if (!c || !ms || !flops || !launches) return LLM_ERR_ARG;
   if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;

@@ -1,6 +1,6 @@
-"""llm_lr_at (host-only C ABI) against the float64 schedule of the oracle:
-equal to within float32 rounding at every step of several schedules, and
-invalid arguments rejected.  Runs without a GPU (the library loads on the
+"""llm_lr_at and llm_plateau_* (host-only C ABI) against the oracle's
+schedule and plateau rule: equal to within float32 rounding at every step,
+and invalid arguments rejected.  Runs without a GPU (the library loads on the
 host; the schedule launches nothing)."""
 import ctypes as C
 
@@ -44,3 +44,23 @@ def test_lr_at_rejects_bad_arguments():
     for sc, t in bad:
         assert P.lib.llm_lr_at(C.byref(sc), t, C.byref(out)) == P.LLM_ERR_ARG
     assert P.lib.llm_lr_at(None, 1, C.byref(out)) == P.LLM_ERR_ARG
+
+
+def test_plateau_matches_oracle():
+    import scratch_llama_decoder_b200 as P
+    rng = np.random.default_rng(9)
+    losses = np.concatenate([np.linspace(5, 3, 40), 3 + 0.01 * rng.random(200),
+                             np.linspace(2.9, 2.5, 20), 2.6 + 0.01 * rng.random(150)])
+    for args in ((0.5, 30, 3, 0.0), (0.3, 5, 10, 1e-3), (1.0, 0, 2, 0.0)):
+        # the C ABI takes the factor as float32: the oracle gets that value
+        a, b = P.Plateau(*args), TT.Plateau(float(np.float32(args[0])), *args[1:])
+        for v in losses:
+            assert a.update(v) == np.float32(b.update(float(v)))
+    from scratch_llama_decoder_b200._lib import llm_plateau
+    s = llm_plateau()
+    for bad in ((0.0, 30, 3, 0.0), (1.5, 30, 3, 0.0), (0.5, -1, 3, 0.0), (0.5, 30, -1, 0.0),
+                (0.5, 30, 3, 1.0)):
+        assert P.lib.llm_plateau_init(C.byref(s), *bad) == P.LLM_ERR_ARG
+    assert P.lib.llm_plateau_init(C.byref(s), 0.5, 30, 3, 0.0) == 0
+    out = C.c_float()
+    assert P.lib.llm_plateau_update(C.byref(s), float("nan"), C.byref(out)) == P.LLM_ERR_ARG

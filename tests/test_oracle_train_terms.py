@@ -90,3 +90,28 @@ def test_clip_against_torch_clip_grad_norm():
         got = np.concatenate([p.grad.numpy() for p in ps])
         np.testing.assert_allclose(got, c, rtol=1e-6 / max(n, 1e-30) * 10, atol=0)
         assert math.isclose(s, 1.0) == (n <= max_norm)
+
+
+def test_plateau_against_torch_reduce_lr_on_plateau():
+    """randyGPT's schedule: halve on stagnation (patience 30), at most 3 times;
+    PyTorch's ReduceLROnPlateau (mode min, rel threshold 0, cooldown 0) with
+    min_lr = lr * 0.5^3 gives the same rates."""
+    rng = np.random.default_rng(9)
+    losses = np.concatenate([np.linspace(5, 3, 40), 3 + 0.01 * rng.random(200),
+                             np.linspace(2.9, 2.5, 20), 2.6 + 0.01 * rng.random(150)])
+    pl = TT.Plateau(0.5, 30, 3, 0.0)
+    p = torch.nn.Parameter(torch.zeros(1, dtype=torch.float64))
+    opt = torch.optim.SGD([p], lr=1.0)
+    sch = torch.optim.lr_scheduler.ReduceLROnPlateau(opt, mode="min", factor=0.5, patience=30,
+                                                     threshold=0.0, threshold_mode="rel",
+                                                     cooldown=0, min_lr=0.125, eps=0.0)
+    scales = []
+    for v in losses:
+        scales.append(pl.update(float(v)))
+        sch.step(float(v))
+        assert scales[-1] == pytest.approx(opt.param_groups[0]["lr"], rel=1e-15)
+    assert pl.reductions == 3 and scales[-1] == 0.125
+    # the first reduction comes on the 31st evaluation without a better one
+    first = next(i for i, x in enumerate(scales) if x < 1.0)
+    best_i = int(np.argmin(losses[:first]))
+    assert first - best_i == 31
