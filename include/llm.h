@@ -316,6 +316,14 @@ int llm_set_rope_scale(llm_ctx *ctx, float factor);
  * 0 <= p < 1. */
 int llm_set_dropout(llm_ctx *ctx, float p, uint64_t seed);
 
+/* The norm clipping uses: LLM_CLIP_L2, the Euclidean norm of the whole
+ * gradient (the default), or LLM_CLIP_LINF, its largest absolute element
+ * (randyGPT, Training: gradient clipping by the L-infinity norm at 1.0); the
+ * rule is the same, scale = max_norm / norm when norm > max_norm.  A change
+ * frees the captured step graph.  LLM_ERR_ARG for another mode. */
+enum { LLM_CLIP_L2 = 0, LLM_CLIP_LINF = 1 };
+int llm_set_grad_clip_mode(llm_ctx *ctx, int mode);
+
 /* Synchronises the context's stream and returns in *norm the gradient norm
  * (before clipping) of the most recent llm_step run with clipping on;
  * LLM_ERR_ARG if no such step has run on this context. */

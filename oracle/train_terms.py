@@ -21,7 +21,8 @@ total <= decay_start.
 Clipping (MicroGPT in Rust, Gradient Clipping: when the gradient norm exceeds
 max_norm every gradient is scaled by max_norm / norm, else left alone;
 Transformer-In-Rust: by global norm).  The norm is the Euclidean norm of all
-gradient elements together.
+gradient elements together; randyGPT's "L-infinity norm clipped at 1.0" is
+the same rule with the largest absolute gradient element as the norm.
 
 Plateau (randyGPT, Training: ReduceLROnPlateau halves max_lr on stagnation, up
 to 3 times, patience 30).  Readings: a metric counts as better when it is
@@ -48,9 +49,12 @@ def lr_at(t, max_lr, min_lr, warmup, decay_start, total, shape="cosine"):
     return max_lr + (min_lr - max_lr) * p
 
 
-def grad_norm(g):
-    """Euclidean norm of every gradient element together."""
+def grad_norm(g, kind="l2"):
+    """Euclidean norm of every gradient element together ("l2"), or the
+    largest absolute element ("linf")."""
     g = np.asarray(g, dtype=np.float64)
+    if kind == "linf":
+        return float(np.max(np.abs(g))) if g.size else 0.0
     return float(np.sqrt(np.sum(g * g)))
 
 
@@ -58,9 +62,9 @@ def clip_scale(norm, max_norm):
     return max_norm / norm if norm > max_norm else 1.0
 
 
-def clip(g, max_norm):
+def clip(g, max_norm, kind="l2"):
     """(clipped gradient, norm before clipping, scale)."""
-    n = grad_norm(g)
+    n = grad_norm(g, kind)
     s = clip_scale(n, max_norm)
     return np.asarray(g, dtype=np.float64) * s, n, s
 

@@ -35,6 +35,7 @@ class llm_tensor_info(C.Structure):
 
 
 LLM_LR_CONSTANT, LLM_LR_COSINE, LLM_LR_LINEAR = 0, 1, 2
+LLM_CLIP_L2, LLM_CLIP_LINF = 0, 1
 LR_SHAPES = {"constant": LLM_LR_CONSTANT, "cosine": LLM_LR_COSINE, "linear": LLM_LR_LINEAR}
 
 
@@ -70,6 +71,7 @@ EXPORTS = {
     "llm_sample_ex": (_i, [_vp, _vp, _i64, _i, _f, _i, _f, _f, _vp, _i64, _i, _vp, _vp]),
     "llm_set_grad_clip": (_i, [_vp, _f]),
     "llm_set_dropout": (_i, [_vp, _f, _u64]),
+    "llm_set_grad_clip_mode": (_i, [_vp, _i]),
     "llm_set_rope_scale": (_i, [_vp, _f]),
     "llm_read_grad_norm": (_i, [_vp, C.POINTER(C.c_double)]),
     "llm_lr_at": (_i, [C.POINTER(llm_lr_schedule), _i64, C.POINTER(_f)]),

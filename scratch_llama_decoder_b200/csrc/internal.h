@@ -94,6 +94,9 @@ void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, floa
 // clip_part_blocks() doubles; *norm gets the norm before clipping, *scale the
 // factor applied (max_norm / norm when norm > max_norm, else 1).
 int clip_part_blocks();
+// The same with the L-infinity norm (the largest |g|).
+void clip_grads_inf(float *g, int64_t n, float max_norm, double *part, double *norm,
+                    float *scale, cudaStream_t s);
 // g [n] (16-byte aligned) *= sc in place.
 void scale_grads(float *g, int64_t n, float sc, cudaStream_t s);
 void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm, float *scale,

@@ -1133,6 +1133,41 @@ __global__ void __launch_bounds__(CLIP_THREADS)
   }
   if (blockIdx.x == 0 && threadIdx.x < (int)(n & 3)) g[n4 * 4 + threadIdx.x] *= sc;
 }
+// randyGPT, Training: clipping by the L-infinity norm -- the largest |g| --
+// with the same rule.  A maximum does not depend on the order it is taken in.
+__global__ void __launch_bounds__(CLIP_THREADS)
+    k_absmax(const float *__restrict__ g, int64_t n, float *__restrict__ part) {
+  __shared__ float ws[CLIP_THREADS / 32];
+  float mx = 0.f;
+  for (int64_t i = blockIdx.x * (int64_t)CLIP_THREADS + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * CLIP_THREADS)
+    mx = fmaxf(mx, fabsf(g[i]));
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int w = 0; w < CLIP_THREADS / 32; w++) m = fmaxf(m, ws[w]);
+    part[blockIdx.x] = m;
+  }
+}
+__global__ void k_clip_scale_inf(const float *__restrict__ part, int nblk, float max_norm,
+                                 double *__restrict__ norm, float *__restrict__ scale) {
+  if (threadIdx.x != 0) return;
+  float m = 0.f;
+  for (int i = 0; i < nblk; i++) m = fmaxf(m, part[i]);
+  *norm = (double)m;
+  *scale = m > max_norm ? (float)((double)max_norm / (double)m) : 1.0f;
+}
+void clip_grads_inf(float *g, int64_t n, float max_norm, double *part, double *norm,
+                    float *scale, cudaStream_t s) {
+  float *fpart = reinterpret_cast<float *>(part);  // CLIP_BLOCKS floats fit in the doubles
+  k_absmax<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, fpart);
+  k_clip_scale_inf<<<1, 32, 0, s>>>(fpart, CLIP_BLOCKS, max_norm, norm, scale);
+  k_scale_grads<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, scale);
+  count_launch(3);
+}
+
 // g *= sc (the mean of summed gradients: sc = 1 / ranks)
 __global__ void __launch_bounds__(CLIP_THREADS)
     k_scale_grads_by(float *__restrict__ g, int64_t n, float sc) {

@@ -184,6 +184,7 @@ struct llm_ctx {
   int *drop_step = nullptr;
   // gradient clipping (llm_set_grad_clip): threshold, block sums, norm, scale
   float clip = 0.f;
+  int clip_mode = 0;  // LLM_CLIP_L2 or LLM_CLIP_LINF
   bool have_norm = false;
   double *clip_part = nullptr, *clip_norm = nullptr;
   float *clip_scale = nullptr;
@@ -440,6 +441,21 @@ int llm_set_dropout(llm_ctx *c, float p, uint64_t seed) {
   return LLM_OK;
 }
 
+int llm_set_grad_clip_mode(llm_ctx *c, int mode) {
+  if (!c || (mode != LLM_CLIP_L2 && mode != LLM_CLIP_LINF)) return LLM_ERR_ARG;
+  if (mode != c->clip_mode) {
+    // the norm is part of a captured step: drop the graph
+    if (c->gexec) {
+      if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+      cudaGraphExecDestroy(c->gexec);
+      c->gexec = nullptr;
+    }
+    c->have_prev = false;
+    c->clip_mode = mode;
+  }
+  return LLM_OK;
+}
+
 int llm_read_grad_norm(llm_ctx *c, double *norm) {
   if (!c || !norm || !c->have_norm) return LLM_ERR_ARG;
   if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
@@ -577,6 +593,14 @@ void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, 
           int64_t ldr, int splits, double alg_flops) {
   if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, alg_flops)) return;
   gemm_simt(g, out, C, ldc, R, ldr, splits, c->cur);
+}
+
+// Gradient clipping of the whole gradient buffer with the context's norm.
+void clip_step(llm_ctx *c, float *g) {
+  if (c->clip_mode == LLM_CLIP_LINF)
+    clip_grads_inf(g, c->D.P, c->clip, c->clip_part, c->clip_norm, c->clip_scale, c->s);
+  else
+    clip_grads(g, c->D.P, c->clip, c->clip_part, c->clip_norm, c->clip_scale, c->s);
 }
 
 // Dropout masks of (site, layer) for the current training call (sites: 0
@@ -892,8 +916,7 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
                   c->flag_step, c->s);
     loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
     backward(c, d_params, d_grads, d_tokens);
-    if (c->clip > 0.f)
-      clip_grads(d_grads, D.P, c->clip, c->clip_part, c->clip_norm, c->clip_scale, c->s);
+    if (c->clip > 0.f) clip_step(c, d_grads);
     adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2,
           c->cfg.adam_eps, c->flag_step, c->s);
     or_flag(c->flag_step, c->flag_sticky, c->s);
@@ -972,7 +995,7 @@ int llm_adamw(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_
   set_hyper(c->hyper, lr, wd, (float)bc1, (float)bc2, c->s);
   if (grad_scale != 1.0f) scale_grads(d_grads, D.P, grad_scale, c->s);
   if (c->clip > 0.f) {
-    clip_grads(d_grads, D.P, c->clip, c->clip_part, c->clip_norm, c->clip_scale, c->s);
+    clip_step(c, d_grads);
     c->have_norm = true;
   }
   adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps,

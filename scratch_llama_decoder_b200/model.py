@@ -147,6 +147,10 @@ class LlamaStep:
         """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
         L.check(L.lib.llm_set_grad_clip(self.ctx, float(max_norm)), "llm_set_grad_clip")
 
+    def set_grad_clip_mode(self, mode):
+        """0: global L2 norm (default); 1: L-infinity norm (llm_set_grad_clip_mode)."""
+        L.check(L.lib.llm_set_grad_clip_mode(self.ctx, int(mode)), "llm_set_grad_clip_mode")
+
     def read_grad_norm(self):
         """Gradient norm before clipping of the last clipped step (llm_read_grad_norm)."""
         v = C.c_double(0.0)

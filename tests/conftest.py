@@ -17,7 +17,7 @@ def pytest_configure(config):
 # sampler, longer contexts), and last the
 # allocation-free entry, whose file sets up per-device state on first use.
 _LATE = ("test_gpu_dp.py", "test_gpu_dropout.py", "test_gpu_sample_ext.py",
-         "test_gpu_long_context.py")
+         "test_gpu_long_context.py", "test_gpu_clip_linf.py")
 _LAST = ("test_zz_no_alloc.py",)
 
 

@@ -115,3 +115,20 @@ def test_plateau_against_torch_reduce_lr_on_plateau():
     first = next(i for i, x in enumerate(scales) if x < 1.0)
     best_i = int(np.argmin(losses[:first]))
     assert first - best_i == 31
+
+
+def test_linf_clip_closed_form_and_torch():
+    g, n, sc = TT.clip([3.0, -4.0, 0.5], 1.0, "linf")
+    assert n == 4.0 and sc == 0.25
+    np.testing.assert_allclose(g, [0.75, -1.0, 0.125], rtol=1e-15)
+    g, n, sc = TT.clip([0.3, -0.4], 1.0, "linf")
+    assert sc == 1.0 and n == 0.4
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(3000)
+    pt = torch.nn.Parameter(torch.zeros(3000, dtype=torch.float64))
+    pt.grad = torch.tensor(x)
+    total = torch.nn.utils.clip_grad_norm_([pt], 1.5, norm_type=float("inf"))
+    c, n, sc = TT.clip(x, 1.5, "linf")
+    assert float(total) == n  # the largest |g|, exactly
+    np.testing.assert_allclose(pt.grad.numpy(), c, rtol=1e-5)
+    assert np.abs(c).max() == pytest.approx(1.5, rel=1e-15)
