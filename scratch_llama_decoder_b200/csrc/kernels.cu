@@ -1135,19 +1135,21 @@ __global__ void __launch_bounds__(CLIP_THREADS)
 }
 // randyGPT, Training: clipping by the L-infinity norm -- the largest |g| --
 // with the same rule.  A maximum does not depend on the order it is taken in.
+// A NaN anywhere makes the norm NaN (as the L2 sum does), so the scale stays 1.
+LLM_DEV float nan_max(float a, float b) { return a != a ? a : ((b != b || b > a) ? b : a); }
 __global__ void __launch_bounds__(CLIP_THREADS)
     k_absmax(const float *__restrict__ g, int64_t n, float *__restrict__ part) {
   __shared__ float ws[CLIP_THREADS / 32];
   float mx = 0.f;
   for (int64_t i = blockIdx.x * (int64_t)CLIP_THREADS + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * CLIP_THREADS)
-    mx = fmaxf(mx, fabsf(g[i]));
-  mx = warp_max(mx);
+    mx = nan_max(mx, fabsf(g[i]));
+  for (int o = 16; o > 0; o >>= 1) mx = nan_max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = mx;
   __syncthreads();
   if (threadIdx.x == 0) {
     float m = 0.f;
-    for (int w = 0; w < CLIP_THREADS / 32; w++) m = fmaxf(m, ws[w]);
+    for (int w = 0; w < CLIP_THREADS / 32; w++) m = nan_max(m, ws[w]);
     part[blockIdx.x] = m;
   }
 }
@@ -1155,7 +1157,7 @@ __global__ void k_clip_scale_inf(const float *__restrict__ part, int nblk, float
                                  double *__restrict__ norm, float *__restrict__ scale) {
   if (threadIdx.x != 0) return;
   float m = 0.f;
-  for (int i = 0; i < nblk; i++) m = fmaxf(m, part[i]);
+  for (int i = 0; i < nblk; i++) m = nan_max(m, part[i]);
   *norm = (double)m;
   *scale = m > max_norm ? (float)((double)max_norm / (double)m) : 1.0f;
 }

@@ -132,3 +132,13 @@ def test_linf_clip_closed_form_and_torch():
     assert float(total) == n  # the largest |g|, exactly
     np.testing.assert_allclose(pt.grad.numpy(), c, rtol=1e-5)
     assert np.abs(c).max() == pytest.approx(1.5, rel=1e-15)
+
+
+def test_nan_gradient_leaves_the_scale_at_one():
+    """A NaN gradient makes either norm NaN; NaN > max_norm is false, so the
+    clipping rule leaves the gradient unscaled (the step's non-finite-loss
+    check is what stops such an update)."""
+    for kind in ("l2", "linf"):
+        n = TT.grad_norm([1.0, float("nan"), -3.0], kind)
+        assert math.isnan(n)
+        assert TT.clip_scale(n, 1.0) == 1.0
