@@ -12,17 +12,18 @@ def pytest_configure(config):
 
 
 # Collection order for a run that stops at the first failure (-x): the parity
-# tests of the training step, its kernels and decode first, then the tests of
-# the entry points built on them (data parallelism, dropout, the extended
-# sampler, longer contexts), and last the
-# allocation-free entry, whose file sets up per-device state on first use.
+# tests of the training step, its kernels and decode first, then the
+# allocation-free entry (its file sets up per-device state on first use, which
+# no other test reads), and last the tests of the entry points built on the
+# step (data parallelism, dropout, the extended sampler, longer contexts,
+# L-infinity clipping).
+_NEXT = ("test_zz_no_alloc.py",)
 _LATE = ("test_gpu_dp.py", "test_gpu_dropout.py", "test_gpu_sample_ext.py",
          "test_gpu_long_context.py", "test_gpu_clip_linf.py")
-_LAST = ("test_zz_no_alloc.py",)
 
 
 def pytest_collection_modifyitems(session, config, items):
     def rank(item):
         name = os.path.basename(str(item.fspath))
-        return 2 if name in _LAST else 1 if name in _LATE else 0
+        return 2 if name in _LATE else 1 if name in _NEXT else 0
     items.sort(key=rank)  # stable: the order inside each group is kept
