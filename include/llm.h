@@ -30,6 +30,14 @@
  *   - Tokens and targets are int32 [batch, ctx], row-major.
  *   - All work is enqueued asynchronously on the stream given to llm_create;
  *     no call synchronises the host except llm_status().
+ *   - One device per process: a context belongs to the CUDA device current
+ *     when llm_create is called (its stream, workspace and every buffer
+ *     passed to it are on that device), and every call on it must be made
+ *     with that device current.  The first context (or llm_kernels.h entry)
+ *     of a process fixes the process's device; creating a context, or calling
+ *     a kernel entry, with another device current returns LLM_ERR_ARG, and so
+ *     does a call on a context with another device current.  Run one process
+ *     per GPU (torch.distributed) to use several.
  *   - Return codes are the LLM_* values below; no exception or abort ever
  *     crosses this boundary.  LLM_ERR_CONFIG and LLM_ERR_ARG are detected on
  *     the host before anything is launched.  LLM_ERR_TOKEN and
@@ -49,7 +57,8 @@ extern "C" {
 enum {
   LLM_OK = 0,
   LLM_ERR_CONFIG = -1,    /* invalid configuration */
-  LLM_ERR_ARG = -2,       /* null/misaligned pointer, workspace too small, bad size */
+  LLM_ERR_ARG = -2,       /* null/misaligned pointer, workspace too small, bad size,
+                             another device current (one device per process) */
   LLM_ERR_TOKEN = -3,     /* a token or target id outside [0, vocab) */
   LLM_ERR_NONFINITE = -4, /* the loss was not finite */
   LLM_ERR_CUDA = -5,      /* a CUDA runtime error */

@@ -2,7 +2,9 @@
  * llm_kernels.h -- single hot-path kernels of the training step exposed for
  * parity tests and micro-benchmarks.  Same conventions as llm.h: d_* are
  * caller-owned DEVICE pointers, work is enqueued on `stream` (a cudaStream_t),
- * return codes are the LLM_* values of llm.h, nothing is allocated.
+ * return codes are the LLM_* values of llm.h, nothing is allocated.  The
+ * one-device-per-process rule of llm.h holds here too (LLM_ERR_ARG when
+ * another device than the process's is current).
  */
 #ifndef LLM_KERNELS_H_
 #define LLM_KERNELS_H_

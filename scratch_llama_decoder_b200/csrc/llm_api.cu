@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <vector>
@@ -124,6 +125,7 @@ struct Carver {
 struct llm_ctx {
   llm_config cfg;
   Dims D;
+  int dev = -1;  // the device current at llm_create
   cudaStream_t s;
   // weight-gradient GEMMs run on a side stream s2 (forked from / joined to s
   // with events); cur is the stream the GEMM launchers use
@@ -309,6 +311,28 @@ int llm_workspace_bytes(const llm_config *cfg, int64_t *bytes) {
   return LLM_OK;
 }
 
+// Every context and kernel entry of a process runs on one device (the
+// kernels opt in to their shared-memory sizes once per process): the first
+// call that needs a device fixes it, later calls with another device current
+// are refused.
+static std::atomic<int> g_device{-1};
+static bool claim_device(int *dev) {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  int first = -1;
+  if (!g_device.compare_exchange_strong(first, d) && first != d) return false;
+  if (dev) *dev = d;
+  return true;
+}
+// The context's device is the current one.
+static bool on_device(const llm_ctx *c) {
+  int d = -1;
+  return cudaGetDevice(&d) == cudaSuccess && d == c->dev;
+}
+
 int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void *cuda_stream,
                llm_ctx **out) {
   if (!out) return LLM_ERR_ARG;
@@ -319,6 +343,7 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
   if (!c) return LLM_ERR_ARG;
   c->cfg = *cfg;
   c->D = make_dims(cfg);
+  if (ws_bytes < c->carve(nullptr) || !claim_device(&c->dev)) { delete c; return LLM_ERR_ARG; }
   c->s = (cudaStream_t)cuda_stream;
   c->cur = c->s;
   if (cudaStreamCreateWithFlags(&c->s2, cudaStreamNonBlocking) != cudaSuccess ||
@@ -328,8 +353,6 @@ int llm_create(const llm_config *cfg, void *d_workspace, int64_t ws_bytes, void 
     (void)cudaGetLastError();
     c->s2 = nullptr;
   }
-  int64_t need = c->carve(nullptr);
-  if (ws_bytes < need) { delete c; return LLM_ERR_ARG; }
   c->carve((char *)d_workspace);
   g_launches = 0;
   cudaMemsetAsync(c->flag_step, 0, 64, c->s);
@@ -381,12 +404,14 @@ int llm_last_launch_count(const llm_ctx *c) { return c ? c->last_launches : 0; }
 
 int llm_set_kernel_timing(llm_ctx *c, int enable) {
   if (!c) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   c->timing = enable != 0;
   return LLM_OK;
 }
 
 int llm_set_graphs(llm_ctx *c, int enable) {
   if (!c) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   c->graphs = enable != 0;
   if (!c->graphs && (c->gexec || c->dexec)) {
     if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
@@ -402,6 +427,7 @@ int llm_set_graphs(llm_ctx *c, int enable) {
 
 int llm_set_grad_clip(llm_ctx *c, float max_norm) {
   if (!c || max_norm != max_norm) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   const float v = max_norm > 0.f ? max_norm : 0.f;
   if (v != c->clip) {
     // the threshold is baked into a captured step: drop the graph
@@ -418,6 +444,7 @@ int llm_set_grad_clip(llm_ctx *c, float max_norm) {
 
 int llm_set_rope_scale(llm_ctx *c, float factor) {
   if (!c || !(factor > 0.f) || !std::isfinite(factor)) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   g_launches = 0;
   rope_table(c->cos_t, c->sin_t, c->D.T, c->D.hd, c->cfg.rope_base, c->s, (double)factor);
   c->last_launches = g_launches;
@@ -426,6 +453,7 @@ int llm_set_rope_scale(llm_ctx *c, float factor) {
 
 int llm_set_dropout(llm_ctx *c, float p, uint64_t seed) {
   if (!c || !(p >= 0.f) || !(p < 1.f)) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (p != c->drop_p || seed != c->drop_seed) {
     // the rate is baked into a captured step: drop the graph
     if (c->gexec) {
@@ -443,6 +471,7 @@ int llm_set_dropout(llm_ctx *c, float p, uint64_t seed) {
 
 int llm_set_grad_clip_mode(llm_ctx *c, int mode) {
   if (!c || (mode != LLM_CLIP_L2 && mode != LLM_CLIP_LINF)) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (mode != c->clip_mode) {
     // the norm is part of a captured step: drop the graph
     if (c->gexec) {
@@ -458,6 +487,7 @@ int llm_set_grad_clip_mode(llm_ctx *c, int mode) {
 
 int llm_read_grad_norm(llm_ctx *c, double *norm) {
   if (!c || !norm || !c->have_norm) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
   if (cudaMemcpy(norm, c->clip_norm, sizeof(double), cudaMemcpyDeviceToHost) != cudaSuccess)
     return LLM_ERR_CUDA;
@@ -520,6 +550,7 @@ int llm_plateau_update(llm_plateau *pl, double metric, float *scale) {
 
 int llm_read_kernel_timing(llm_ctx *c, double *ms, double *flops, int64_t *launches) {
   if (!c || !ms || !flops || !launches) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
   double total = 0.0;
   for (size_t i = 0; i + 1 < c->ev_used; i += 2) {
@@ -539,6 +570,7 @@ int llm_read_kernel_timing(llm_ctx *c, double *ms, double *flops, int64_t *launc
 
 int llm_status(llm_ctx *c) {
   if (!c) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
   int f = 0;
   if (cudaMemcpy(&f, c->flag_sticky, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
@@ -886,6 +918,7 @@ extern "C" {
 
 int llm_forward(llm_ctx *c, const float *d_params, const int32_t *d_tokens, float *d_logits) {
   if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   g_launches = 0;
   set_flag_zero(c->flag_step, c->s);
   forward(c, d_params, d_tokens, false);
@@ -899,6 +932,7 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
              const int32_t *d_tokens, const int32_t *d_targets, float lr, float wd,
              float *d_loss) {
   if (!c || !d_tokens || !d_targets || !d_loss || t < 1) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
     return LLM_ERR_ARG;
   const Dims &D = c->D;
@@ -968,6 +1002,7 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
 int llm_grad(llm_ctx *c, const float *d_params, float *d_grads, const int32_t *d_tokens,
              const int32_t *d_targets, float *d_loss) {
   if (!c || !d_tokens || !d_targets || !d_loss) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (!aligned16(d_params) || !aligned16(d_grads)) return LLM_ERR_ARG;
   const Dims &D = c->D;
   g_launches = 0;
@@ -986,6 +1021,7 @@ int llm_grad(llm_ctx *c, const float *d_params, float *d_grads, const int32_t *d
 int llm_adamw(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,
               float lr, float wd, float grad_scale) {
   if (!c || t < 1 || !std::isfinite(grad_scale)) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
     return LLM_ERR_ARG;
   const Dims &D = c->D;
@@ -1007,6 +1043,7 @@ int llm_adamw(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_
 int llm_adamw_range(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v,
                     int64_t count, int64_t t, float lr, float wd, float grad_scale) {
   if (!c || t < 1 || count < 0 || !std::isfinite(grad_scale)) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
     return LLM_ERR_ARG;
   g_launches = 0;
@@ -1024,6 +1061,7 @@ int llm_adamw_range(llm_ctx *c, float *d_params, float *d_grads, float *d_m, flo
 
 int llm_flag_out(llm_ctx *c, int32_t *d_flag) {
   if (!c || !d_flag) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (cudaMemcpyAsync(d_flag, c->flag_step, sizeof(int32_t), cudaMemcpyDeviceToDevice, c->s) !=
       cudaSuccess)
     return LLM_ERR_CUDA;
@@ -1032,6 +1070,7 @@ int llm_flag_out(llm_ctx *c, int32_t *d_flag) {
 
 int llm_flag_in(llm_ctx *c, const int32_t *d_flag) {
   if (!c || !d_flag) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   g_launches = 0;
   or_flag(d_flag, c->flag_step, c->s);
   c->last_launches = g_launches;
@@ -1041,6 +1080,7 @@ int llm_flag_in(llm_ctx *c, const int32_t *d_flag) {
 int llm_decode(llm_ctx *c, const float *d_params, const int32_t *d_tokens, int pos,
                float *d_logits) {
   if (!c || !d_params || !d_tokens || !d_logits) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   const Dims &D = c->D;
   if (pos < 0 || pos >= D.T) return LLM_ERR_ARG;
   if (128 % D.hd || D.rc) return LLM_ERR_CONFIG;
@@ -1095,6 +1135,7 @@ int llm_decode(llm_ctx *c, const float *d_params, const int32_t *d_tokens, int p
 int llm_sample(llm_ctx *c, const float *d_logits, int64_t ld, int n_rows, float temperature,
                int top_k, const float *d_uniform, int32_t *d_out) {
   if (!c || !d_logits || !d_uniform || !d_out || n_rows < 1 || ld < c->D.V) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (!(temperature == temperature)) return LLM_ERR_ARG;  // NaN
   g_launches = 0;
   sample_tokens(d_logits, ld, n_rows, c->D.V, temperature, top_k, d_uniform, d_out, c->s);
@@ -1106,6 +1147,7 @@ int llm_sample_ex(llm_ctx *c, const float *d_logits, int64_t ld, int n_rows, flo
                   int top_k, float top_p, float repetition_penalty, const int32_t *d_history,
                   int64_t history_ld, int history_len, const float *d_uniform, int32_t *d_out) {
   if (!c || !d_logits || !d_uniform || !d_out || n_rows < 1 || ld < c->D.V) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   if (!(temperature == temperature) || !(top_p > 0.f) || !(top_p <= 1.f)) return LLM_ERR_ARG;
   if (top_p < 1.f && (top_k < 1 || top_k > sample_ex_max_top_k())) return LLM_ERR_ARG;
   if (!(repetition_penalty > 0.f) || !std::isfinite(repetition_penalty) || history_len < 0)
@@ -1123,6 +1165,7 @@ int llm_sample_ex(llm_ctx *c, const float *d_logits, int64_t ld, int n_rows, flo
 
 int llm_init(llm_ctx *c, uint64_t seed, float init_std, int scale_out_proj, float *d_params) {
   if (!c || !d_params || !(init_std >= 0.f)) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
   const Dims &D = c->D;
   POff O{D};
   g_launches = 0;
@@ -1157,6 +1200,7 @@ extern "C" int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_
   if (lda < (a_kmajor ? K : M) || ldb < (b_kmajor ? K : N) || ldc < N) return LLM_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   GemmOperands g{M, N, K, d_A, lda, a_kmajor != 0, d_B, ldb, b_kmajor != 0, DT_BF16};
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
   g_launches = 0;
   if (tensor_cores) {
     static TcPlan *plan = nullptr;
@@ -1185,6 +1229,7 @@ extern "C" int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, 
       n_tokens > ((int64_t)1 << 30) || ((uintptr_t)d_scratch & 15))
     return LLM_ERR_ARG;
   if (scratch_bytes < 4 * embed_bwd_scratch_ints(n_tokens, vocab)) return LLM_ERR_ARG;
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
   g_launches = 0;
   embed_bwd(d_tokens, d_dx, d_dwte, n_tokens, d_model, vocab, (int32_t *)d_scratch,
             (cudaStream_t)stream);
@@ -1210,6 +1255,7 @@ extern "C" int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float
                                              int head_dim, int tensor_cores, void *stream) {
   if (!attn_args_ok(d_qkv, d_o, batch, ctx, n_head, n_kv_head, head_dim) || !d_lse)
     return LLM_ERR_ARG;
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
   g_launches = 0;
   cudaStream_t s = (cudaStream_t)stream;
   if (tensor_cores == 2) {
@@ -1234,6 +1280,7 @@ extern "C" int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o,
   if (!attn_args_ok(d_qkv, d_o, batch, ctx, n_head, n_kv_head, head_dim) || !d_dout || !d_lse ||
       !d_D || !d_dqkv)
     return LLM_ERR_ARG;
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
   g_launches = 0;
   cudaStream_t s = (cudaStream_t)stream;
   if (tensor_cores == 2) {

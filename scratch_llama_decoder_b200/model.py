@@ -4,6 +4,7 @@ Argument marshalling only: torch tensors are passed to the library by device
 pointer; every step of the computation runs in the library's kernels.
 """
 import ctypes as C
+import functools
 
 import torch
 
@@ -12,6 +13,16 @@ from . import _lib as L
 
 def _ptr(t):
     return C.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _on_device(fn):
+    """Runs a method with the context's device current: the library refuses
+    calls on a context made with another device current."""
+    @functools.wraps(fn)
+    def call(self, *args, **kwargs):
+        with torch.cuda.device(self.device):
+            return fn(self, *args, **kwargs)
+    return call
 
 
 class LlamaStep:
@@ -25,15 +36,22 @@ class LlamaStep:
         if not torch.cuda.is_available():
             raise RuntimeError("LlamaStep needs a CUDA device (B200, sm_100a); no CPU fallback")
         self.cfg = dict(cfg)
-        self.device = torch.device(device)
+        dev = torch.device(device)
+        if dev.type != "cuda":
+            raise ValueError(f"LlamaStep runs on a CUDA device, not {dev}")
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
         self.layout, self.n_params = L.llm_param_layout(cfg)
         self.ws_bytes = L.llm_workspace_bytes(cfg)
-        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
-        self.stream = stream if stream is not None else torch.cuda.current_stream(self.device)
         self._c = L.make_config(cfg)
-        ctx = C.c_void_p()
-        L.check(L.lib.llm_create(C.byref(self._c), _ptr(self.workspace), self.ws_bytes,
-                                 C.c_void_p(self.stream.cuda_stream), C.byref(ctx)), "llm_create")
+        with torch.cuda.device(self.device):
+            self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+            self.stream = stream if stream is not None else torch.cuda.current_stream(self.device)
+            ctx = C.c_void_p()
+            L.check(L.lib.llm_create(C.byref(self._c), _ptr(self.workspace), self.ws_bytes,
+                                     C.c_void_p(self.stream.cuda_stream), C.byref(ctx)),
+                    "llm_create")
         self.ctx = ctx
 
     def close(self):
@@ -51,10 +69,12 @@ class LlamaStep:
     def new_params(self):
         return torch.zeros(self.n_params, dtype=torch.float32, device=self.device)
 
+    @_on_device
     def init(self, params, seed, init_std, scale_out_proj):
         L.check(L.lib.llm_init(self.ctx, seed, float(init_std), int(bool(scale_out_proj)),
                                _ptr(params)), "llm_init")
 
+    @_on_device
     def forward(self, params, tokens, logits=None):
         B, T, V = self.cfg["batch"], self.cfg["ctx"], self.cfg["vocab"]
         if logits is None:
@@ -63,6 +83,7 @@ class LlamaStep:
                 "llm_forward")
         return logits
 
+    @_on_device
     def step(self, params, grads, m, v, t, tokens, targets, lr, wd, loss=None):
         if loss is None:
             loss = torch.empty(1, dtype=torch.float32, device=self.device)
@@ -71,6 +92,7 @@ class LlamaStep:
                 "llm_step")
         return loss
 
+    @_on_device
     def sample_ex(self, logits, temperature, top_k, uniforms, top_p=1.0, penalty=1.0,
                   history=None, out=None):
         """llm_sample_ex: repetition penalty over history (int32 [rows, n]),
@@ -86,6 +108,7 @@ class LlamaStep:
                 "llm_sample_ex")
         return out
 
+    @_on_device
     def grad(self, params, grads, tokens, targets, loss=None):
         """Forward, loss and backward without the update (llm_grad)."""
         if loss is None:
@@ -94,11 +117,13 @@ class LlamaStep:
                                _ptr(loss)), "llm_grad")
         return loss
 
+    @_on_device
     def adamw(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
         """grads *= grad_scale, optional clipping, AdamW (llm_adamw)."""
         L.check(L.lib.llm_adamw(self.ctx, _ptr(params), _ptr(grads), _ptr(m), _ptr(v), int(t),
                                 float(lr), float(wd), float(grad_scale)), "llm_adamw")
 
+    @_on_device
     def adamw_range(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
         """AdamW over the elements of 1-D views params, grads, m, v (equal
         lengths; llm_adamw_range)."""
@@ -108,14 +133,17 @@ class LlamaStep:
                                       int(t), float(lr), float(wd), float(grad_scale)),
                 "llm_adamw_range")
 
+    @_on_device
     def flag_out(self, flag):
         """Copy the step's int32 error word to flag (llm_flag_out)."""
         L.check(L.lib.llm_flag_out(self.ctx, _ptr(flag)), "llm_flag_out")
 
+    @_on_device
     def flag_in(self, flag):
         """OR the int32 word flag into the step's error word (llm_flag_in)."""
         L.check(L.lib.llm_flag_in(self.ctx, _ptr(flag)), "llm_flag_in")
 
+    @_on_device
     def decode(self, params, tokens, pos, logits=None):
         """Logits [B, V] of position pos (llm_decode); tokens: int32 [B]."""
         B, V = self.cfg["batch"], self.cfg["vocab"]
@@ -125,6 +153,7 @@ class LlamaStep:
                 "llm_decode")
         return logits
 
+    @_on_device
     def sample(self, logits, temperature, top_k, uniforms, out=None):
         """int32 token ids [rows] from float32 logits [rows, ld] (llm_sample)."""
         rows = logits.shape[0]
@@ -135,41 +164,51 @@ class LlamaStep:
                 "llm_sample")
         return out
 
+    @_on_device
     def set_rope_scale(self, factor):
         """RoPE position interpolation: positions t / factor (llm_set_rope_scale)."""
         L.check(L.lib.llm_set_rope_scale(self.ctx, float(factor)), "llm_set_rope_scale")
 
+    @_on_device
     def set_dropout(self, p, seed):
         """Inverted dropout in later training calls (llm_set_dropout)."""
         L.check(L.lib.llm_set_dropout(self.ctx, float(p), int(seed)), "llm_set_dropout")
 
+    @_on_device
     def set_grad_clip(self, max_norm):
         """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
         L.check(L.lib.llm_set_grad_clip(self.ctx, float(max_norm)), "llm_set_grad_clip")
 
+    @_on_device
     def set_grad_clip_mode(self, mode):
         """0: global L2 norm (default); 1: L-infinity norm (llm_set_grad_clip_mode)."""
         L.check(L.lib.llm_set_grad_clip_mode(self.ctx, int(mode)), "llm_set_grad_clip_mode")
 
+    @_on_device
     def read_grad_norm(self):
         """Gradient norm before clipping of the last clipped step (llm_read_grad_norm)."""
         v = C.c_double(0.0)
         L.check(L.lib.llm_read_grad_norm(self.ctx, C.byref(v)), "llm_read_grad_norm")
         return v.value
 
+    @_on_device
     def status(self):
         return L.lib.llm_status(self.ctx)
 
+    @_on_device
     def last_launch_count(self):
         return L.lib.llm_last_launch_count(self.ctx)
 
+    @_on_device
     def set_kernel_timing(self, enable):
         L.check(L.lib.llm_set_kernel_timing(self.ctx, int(bool(enable))), "llm_set_kernel_timing")
 
+    @_on_device
     def set_graphs(self, enable):
         """Step graphs on/off (llm_set_graphs)."""
         L.check(L.lib.llm_set_graphs(self.ctx, int(bool(enable))), "llm_set_graphs")
 
+    @_on_device
     def read_kernel_timing(self):
         """(device ms, algorithmic FLOPs, launches) of the timed GEMM launches."""
         ms, fl, n = C.c_double(0), C.c_double(0), C.c_int64(0)
