@@ -44,6 +44,17 @@ def test_param_count_matches_page():
     assert O.n_params(cfg) == g["printed_params"]
 
 
+def test_param_count_matches_page_scaled_model():
+    """Hephaistos' scaled run prints its size to two decimals in millions; the
+    layout with SwiGLU hidden floor(8/3 d) = 1024 gives 15,735,168."""
+    g = json.load(open(GOLDEN))["param_count_hephaistos_scaled"]
+    d = g["d_model"]
+    cfg = get_config("c1", vocab=g["vocab"], d_model=d, n_layer=g["n_layer"],
+                     n_head=g["n_head"], n_kv_head=g["n_head"], d_ff=(8 * d) // 3, ctx=g["ctx"])
+    n = O.n_params(cfg)
+    assert round(n / 1e6, g["digits_after_point"]) == g["printed_params_millions"], n
+
+
 @pytest.mark.parametrize("name,expect", [("c1", 3952), ("c2", 1702016), ("c3", 5742848),
                                          ("c4", 30413312), ("c5", 317195264)])
 def test_param_count_closed_form(name, expect):
