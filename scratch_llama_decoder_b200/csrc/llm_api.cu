@@ -575,7 +575,8 @@ int llm_status(llm_ctx *c) {
   int f = 0;
   if (cudaMemcpy(&f, c->flag_sticky, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return LLM_ERR_CUDA;
-  if (cudaMemset(c->flag_sticky, 0, sizeof(int)) != cudaSuccess) return LLM_ERR_CUDA;
+  // cleared on the context's stream, so it lands before any later call's work
+  if (cudaMemsetAsync(c->flag_sticky, 0, sizeof(int), c->s) != cudaSuccess) return LLM_ERR_CUDA;
   if (f & FLAG_TIMEOUT) return LLM_ERR_TIMEOUT;
   if (f & FLAG_TOKEN) return LLM_ERR_TOKEN;
   if (f & FLAG_NONFINITE) return LLM_ERR_NONFINITE;

@@ -9,7 +9,7 @@ import torch
 import oracle as O
 from oracle import train_terms as TT
 from synth import get_config, make_batch, make_params
-from tests.gpu_util import TOL, compare, rel
+from tests.gpu_util import TOL, compare
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,7 @@ def test_linf_clipped_steps_match_oracle(name, over):
     p = make_params(cfg, lay)
     tok, tgt = make_batch(cfg)
     _, _, g = O.forward_backward(cfg, p, tok, tgt, want_logits=False)
-    clip = 0.5 * float(np.abs(g).max())
+    clip = 0.25 * float(np.abs(g).max())  # inside the clipping regime at both steps
     gpu = _run(cfg, p, tok, tgt, clip, 2, 1)
     # the oracle with L-infinity clipping before each AdamW
     pp = p.astype(np.float64)
@@ -57,9 +57,10 @@ def test_linf_clipped_steps_match_oracle(name, over):
                                  norm=n))
     compare(cfg, lay, gpu, ref, prev_params=p.astype(np.float64))
     for gs, rs in zip(gpu["steps"], ref["steps"]):
-        # the GPU's norm is exactly the largest |g| of its own gradient
+        # the reported norm is the largest |g| before clipping
         assert abs(gs["norm"] - rs["norm"]) <= TOL[cfg["compute"]]["grads"] * rs["norm"]
-        assert np.abs(gs["grads"]).max() == pytest.approx(clip, rel=1e-6)
+        if rs["norm"] > clip:  # clipped: the largest stored |g| is the threshold
+            assert np.abs(gs["grads"]).max() == pytest.approx(clip, rel=1e-6)
 
 
 def test_clip_mode_arguments():
