@@ -197,8 +197,9 @@ int llm_flag_in(llm_ctx *ctx, const int32_t *d_flag);
  * the logits of position pos, which attend to cached positions 0..pos.
  * d_params must be the parameters of that forward: the embedding and the
  * RMSNorm gains are read from it, the matrices from the low-precision copies
- * the forward made.  Requires 0 <= pos < ctx and head_dim dividing 128
- * (LLM_ERR_ARG / LLM_ERR_CONFIG otherwise, nothing launched).  Out-of-range
+ * the forward made.  Requires 0 <= pos < ctx (LLM_ERR_ARG otherwise), and
+ * head_dim dividing 128, d_ff at most 16384 and a context made without
+ * recompute (LLM_ERR_CONFIG otherwise); nothing is launched on an error.  Out-of-range
  * ids are clamped for the read and reported by llm_status() as
  * LLM_ERR_TOKEN.  The position goes to device memory first, so the second call
  * in a row with the same (d_params, d_tokens, d_logits) captures the decode

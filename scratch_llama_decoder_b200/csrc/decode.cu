@@ -807,6 +807,12 @@ void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice) {
 
 int gemv_col_blocks(int64_t N) { return (int)cdiv(N, GV_COLS); }
 
+bool gemv_fits(int64_t K, int64_t N) {
+  int ks = 0, sl = 0;
+  gemv_plan(K, N, &ks, &sl);
+  return ks >= 1 && ks <= GV_KS_MAX && sl >= 1 && sl <= GV_KSLICE_MAX;
+}
+
 // Launch with programmatic stream serialisation (see pdl_release / pdl_wait).
 template <typename... P, typename... Q>
 static void launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,

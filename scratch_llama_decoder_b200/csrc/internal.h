@@ -182,6 +182,9 @@ struct GemvArgs {
   int hd, rot_cols;
 };
 void gemv_plan(int64_t K, int64_t N, int *ks, int *kslice);
+// The plan of a [K, N] product stays within the K slices the finishing
+// block adds (K up to 16 slices of 1024 rows).
+bool gemv_fits(int64_t K, int64_t N);
 int gemv_col_blocks(int64_t N);
 void gemv(const GemvArgs &a, DType dt, cudaStream_t s);
 // Attention of the query at position *pos of every sequence against the

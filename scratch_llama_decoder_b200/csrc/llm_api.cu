@@ -1085,6 +1085,10 @@ int llm_decode(llm_ctx *c, const float *d_params, const int32_t *d_tokens, int p
   const Dims &D = c->D;
   if (pos < 0 || pos >= D.T) return LLM_ERR_ARG;
   if (128 % D.hd || D.rc) return LLM_ERR_CONFIG;
+  // every projection's K (d_model, or the padded d_ff of W2) in 16 slices
+  if (!gemv_fits(D.d, D.qkvw) || !gemv_fits(D.d, 2 * D.hp) || !gemv_fits(D.hp, D.d) ||
+      !gemv_fits(D.d, D.Vp))
+    return LLM_ERR_CONFIG;
   if (((uintptr_t)d_params & 3) || ((uintptr_t)d_tokens & 3) || ((uintptr_t)d_logits & 3))
     return LLM_ERR_ARG;
   g_launches = 0;

@@ -98,3 +98,21 @@ def test_recompute_is_bit_identical_to_stored_activations(dropout):
         m.close()
     for a, b in zip(*res):
         assert torch.equal(a, b)
+
+
+def test_decode_refuses_a_hidden_size_past_its_split_plan():
+    """Decode adds at most 16 K slices of 1024 rows per product: a d_ff past
+    16384 is refused on the host (nothing launched); training still runs."""
+    import scratch_llama_decoder_b200 as L
+    from scratch_llama_decoder_b200 import LlamaStep
+    cfg = get_config("c1", batch=1, ctx=8, d_ff=16448)
+    m = LlamaStep(cfg)
+    P = torch.tensor(make_params(cfg, O.param_layout(cfg)), device="cuda")
+    tok, _ = make_batch(cfg)
+    td = torch.tensor(tok, device="cuda")
+    m.forward(P, td)
+    lg = torch.empty(1, cfg["vocab"], device="cuda")
+    assert L.lib.llm_decode(m.ctx, P.data_ptr(), td[:, 0].contiguous().data_ptr(), 0,
+                            lg.data_ptr()) == L.LLM_ERR_CONFIG
+    assert m.status() == 0
+    m.close()
