@@ -78,7 +78,7 @@ def gemm_traffic(workload):
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -101,7 +101,52 @@ def parse():
     ap.add_argument("--orient", default="kn", choices=["kn", "kk", "nn"],
                     help="gemm operand majorness: kn = x.W (forward), kk = dy.W^T (dgrad), "
                          "nn = x^T.dy (wgrad)")
-    return ap.parse_args()
+    # options of the training step (defaults: the step as benchmarked)
+    ap.add_argument("--clip", type=float, default=0.0,
+                    help="gradient clipping threshold (0: off)")
+    ap.add_argument("--clip-mode", default="l2", choices=["l2", "linf"])
+    ap.add_argument("--dropout", type=float, default=0.0, help="inverted dropout rate")
+    ap.add_argument("--rope-scale", type=float, default=1.0,
+                    help="RoPE position interpolation factor")
+    ap.add_argument("--recompute", action="store_true",
+                    help="keep only layer inputs; recompute activations in the backward")
+    ap.add_argument("--ctx", type=int, default=None, help="override the context length")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch")
+    return ap.parse_args(argv)
+
+
+def step_options(args):
+    """(config overrides, options applied to the context, label suffix) of the
+    step's options; empty for the step as benchmarked."""
+    over, opts = {}, {}
+    if args.ctx is not None:
+        over["ctx"] = int(args.ctx)
+    if args.batch is not None:
+        over["batch"] = int(args.batch)
+    if args.recompute:
+        over["recompute"] = 1
+    if args.clip > 0:
+        opts["clip"] = (float(args.clip), args.clip_mode)
+    if args.dropout > 0:
+        opts["dropout"] = float(args.dropout)
+    if args.rope_scale != 1.0:
+        opts["rope_scale"] = float(args.rope_scale)
+    parts = [f"{k}{v}" for k, v in over.items()]
+    if "clip" in opts:
+        parts.append(f"clip-{opts['clip'][1]}{opts['clip'][0]:g}")
+    parts += [f"{k}{opts[k]:g}" for k in ("dropout", "rope_scale") if k in opts]
+    return over, opts, ("+" + "+".join(parts)) if parts else ""
+
+
+def apply_options(model, opts):
+    if "clip" in opts:
+        thr, mode = opts["clip"]
+        model.set_grad_clip_mode(1 if mode == "linf" else 0)
+        model.set_grad_clip(thr)
+    if "dropout" in opts:
+        model.set_dropout(opts["dropout"], 0x5EED)
+    if "rope_scale" in opts:
+        model.set_rope_scale(opts["rope_scale"])
 
 
 def peaks():
@@ -187,15 +232,20 @@ class Clocks:
 
 
 # --------------------------------------------------------------- oracle leg
-def oracle_sample_rate(cfg, tokens, reps=1, warmup=0):
+def oracle_sample_rate(cfg, tokens, reps=1, warmup=0, opts=None):
     """Tokens/s of the float64 oracle on a fraction f = tokens / (B*T) of the
     step: forward + backward of the first `tokens` positions of one sequence,
-    plus AdamW over the same fraction of the parameters.  Returns
+    plus AdamW over the same fraction of the parameters, with the step's
+    options (dropout, RoPE scaling, clipping of that gradient share).  Returns
     (tokens/s, seconds per sample, cores)."""
     import numpy as np
     import oracle as O
+    from oracle import train_terms as TT
     from synth import make_batch
+    opts = opts or {}
     c = dict(cfg, batch=1, ctx=min(cfg["ctx"], tokens))
+    if "rope_scale" in opts:
+        c["rope_scale"] = opts["rope_scale"]
     S = c["ctx"]
     lay = O.param_layout(c)
     rng = np.random.default_rng(5)
@@ -213,8 +263,10 @@ def oracle_sample_rate(cfg, tokens, reps=1, warmup=0):
     times = []
     for it in range(warmup + reps):
         t0 = time.perf_counter()
-        O.forward_backward(c, p, tok, tgt, want_logits=False)
-        O.adamw(p[:n_adam], g, m, v, 1, cfg["lr"], cfg["wd"])
+        drop = (float(np.float32(opts["dropout"])), 0x5EED, it) if "dropout" in opts else None
+        O.forward_backward(c, p, tok, tgt, want_logits=False, dropout=drop)
+        gc = TT.clip(g, opts["clip"][0], opts["clip"][1])[0] if "clip" in opts else g
+        O.adamw(p[:n_adam], gc, m, v, 1, cfg["lr"], cfg["wd"])
         dt = time.perf_counter() - t0
         if it >= warmup:
             times.append(dt)
@@ -223,10 +275,10 @@ def oracle_sample_rate(cfg, tokens, reps=1, warmup=0):
     return S / t, t, cores, S
 
 
-def sample_tokens_for(cfg, budget_s):
+def sample_tokens_for(cfg, budget_s, opts=None):
     """Prefix length whose oracle sample takes about budget_s seconds (probed
     on a 16-token prefix, assuming linear cost in tokens)."""
-    _, t16, _, _ = oracle_sample_rate(cfg, 16)
+    _, t16, _, _ = oracle_sample_rate(cfg, 16, opts=opts)
     per_tok = t16 / 16.0
     S = int(max(16, min(cfg["ctx"], budget_s / max(per_tok, 1e-9))))
     return S
@@ -261,11 +313,14 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = get_config(args.config)
+    over, opts, suffix = step_options(args)
+    cfg = get_config(args.config, **over)
+    workload = cfg["name"] + suffix
     # the library's own stream (not the legacy default stream), so llm_step
     # runs as a replayed CUDA graph after its first two calls
     stream = torch.cuda.Stream(device=dev)
     model = LlamaStep(cfg, device=dev, stream=stream)
+    apply_options(model, opts)
     p_host = make_params(cfg, model.layout, seed=1001 + cfg["index"] + 7919 * rank)
     tok_h, tgt_h = make_batch(cfg, seed=1000 + cfg["index"] + 7919 * rank)
     P = torch.tensor(p_host, device=dev)
@@ -374,14 +429,14 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
         if cfg["compute"] == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": cfg["name"], "tokens_per_step": N, "batch": cfg["batch"],
+        "config": {"workload": workload, "tokens_per_step": N, "batch": cfg["batch"],
                    "seq_len": cfg["ctx"], "parallelism": f"replicas x{world}" if world > 1
                    else "single GPU", "l2": "inputs larger than L2 (saved activations of "
                    "several GB per step; no flush)"},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM (all projection GEMMs of the "
                      "step)", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
                      "frac": achieved / peak_tc if peak_tc else None,
-                     "traffic": gemm_traffic(cfg["name"]),
+                     "traffic": gemm_traffic(workload),
                      "launches": g_launch, "ms_total": g_ms,
                      "peak_source": f"{src} bf16_tflops_sustained"},
         "step_roofline": {"flops": F, "attention_flops": F_attn,
@@ -393,8 +448,8 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
     }
     if world == 1 and not args.no_cpu_baseline:
-        S = sample_tokens_for(cfg, 12.0)
-        rate, tsec, cores, S = oracle_sample_rate(cfg, S)
+        S = sample_tokens_for(cfg, 12.0, opts)
+        rate, tsec, cores, S = oracle_sample_rate(cfg, S, opts=opts)
         out["cpu_baseline"] = {
             "value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"float64 oracle: forward+backward of a {S}-token prefix of one "
@@ -566,10 +621,12 @@ def run_reference(args, rank):
     if rank != 0:
         return None
     from synth import get_config
-    cfg = get_config(args.config)
+    over, opts, suffix = step_options(args)
+    cfg = get_config(args.config, **over)
     budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
-    S = sample_tokens_for(cfg, budget)
-    rate, tsec, cores, S = oracle_sample_rate(cfg, S, reps=args.steps, warmup=args.warmup)
+    S = sample_tokens_for(cfg, budget, opts)
+    rate, tsec, cores, S = oracle_sample_rate(cfg, S, reps=args.steps, warmup=args.warmup,
+                                              opts=opts)
     N = cfg["batch"] * cfg["ctx"]
     return {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": 1,
@@ -579,8 +636,8 @@ def run_reference(args, rank):
         "sample_ms": tsec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": cfg["name"], "tokens_per_step": N, "batch": cfg["batch"],
-                   "seq_len": cfg["ctx"], "parallelism": "host CPU"},
+        "config": {"workload": cfg["name"] + suffix, "tokens_per_step": N,
+                   "batch": cfg["batch"], "seq_len": cfg["ctx"], "parallelism": "host CPU"},
         "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: forward+backward of a {S}-token prefix of one "
                                    f"sequence plus AdamW over {S}/{N} of the parameters"},
