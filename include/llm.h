@@ -152,8 +152,9 @@ int llm_step(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d
  *              this context's batch*ctx positions.
  *   llm_adamw: the step's update: d_grads *= grad_scale in place (1/ranks after
  *              a summing all-reduce turns the sum of the ranks' mean gradients
- *              into the mean over the whole batch), then global-norm clipping
- *              when llm_set_grad_clip is on, then AdamW as in llm_step.  It is
+ *              into the mean over the whole batch), then clipping when
+ *              llm_set_grad_clip is on (by the norm llm_set_grad_clip_mode
+ *              selects), then AdamW as in llm_step.  It is
  *              skipped (params, m, v untouched) when the error word holds an
  *              error: the word the last llm_grad set, ORed with llm_flag_in.
  *   llm_flag_out copies that int32 error word (0 = none) to d_flag (device);
@@ -289,8 +290,9 @@ int llm_plateau_update(llm_plateau *pl, double metric, float *scale);
 /* Global-norm gradient clipping inside llm_step (MicroGPT in Rust, Gradient
  * Clipping: when the gradient norm exceeds max_norm every gradient is scaled
  * by max_norm / norm; Transformer-In-Rust: clipping by global norm).  With
- * max_norm > 0, every later llm_step computes the Euclidean norm of the whole
- * gradient buffer (double-precision sums in a fixed order), scales d_grads in
+ * max_norm > 0, every later llm_step (and llm_adamw) computes the norm of the
+ * whole gradient buffer -- Euclidean by default, from double-precision sums in
+ * a fixed order, or the L-infinity norm (llm_set_grad_clip_mode) --, scales d_grads in
  * place by max_norm / norm when norm > max_norm, and AdamW then uses the
  * clipped gradient (d_grads holds it after the step).  max_norm <= 0 turns
  * clipping off (the default).  A change frees the captured step graph
@@ -335,13 +337,17 @@ enum { LLM_CLIP_L2 = 0, LLM_CLIP_LINF = 1 };
 int llm_set_grad_clip_mode(llm_ctx *ctx, int mode);
 
 /* Synchronises the context's stream and returns in *norm the gradient norm
- * (before clipping) of the most recent llm_step run with clipping on;
- * LLM_ERR_ARG if no such step has run on this context. */
+ * (before clipping, in the selected norm) of the most recent llm_step or
+ * llm_adamw run with clipping on; LLM_ERR_ARG if no such call has run on this
+ * context. */
 int llm_read_grad_norm(llm_ctx *ctx, double *norm);
 
-/* Synchronises the context's stream and returns the first error any call on
+/* Synchronises the context's stream and returns the errors that calls on
  * this context raised on the device since the previous llm_status() (then
- * clears it), or LLM_ERR_CUDA if the stream reports a CUDA error, else LLM_OK. */
+ * clears them): LLM_ERR_TIMEOUT before LLM_ERR_TOKEN before LLM_ERR_NONFINITE
+ * when several were raised; LLM_ERR_CUDA if the stream reports a CUDA error;
+ * else LLM_OK.  An error word brought in by llm_flag_in is not reported here
+ * (it only skips the update). */
 int llm_status(llm_ctx *ctx);
 
 /* A static, human-readable string for a return code. */
