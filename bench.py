@@ -353,16 +353,18 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clocks.start()
     clocks.wait_first()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    # one event before the first step and one after each: the headline is
+    # first to last, the per-step times give the median and best step
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for k in range(args.steps):
         t += 1
         model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
-    e1.record(stream)
+        ev[k + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
+    ms = ev[0].elapsed_time(ev[-1])
+    per_step = sorted(ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps))
     # GEMM roofline: the same K steps again as individual launches, each
     # tensor-core GEMM bracketed by CUDA events on the library's stream (the
     # kernels are the ones the graph replays; events cannot time graph nodes)
@@ -443,6 +445,10 @@ def run_ours(args, rank, world, local_rank):
                           "t_tensor_ms": F / (peak_tc * 1e12) * 1e3,
                           "frac_of_tensor_bound": (F / (peak_tc * 1e12)) / step_s},
         "gpu_launches": launches_per_step * args.steps,
+        # this rank's steps (rank 0): median and best step, as tokens/s per GPU
+        "per_step": {"median_ms": per_step[len(per_step) // 2], "best_ms": per_step[0],
+                     "median_tokens_per_s_per_gpu": N / (per_step[len(per_step) // 2] / 1e3),
+                     "best_tokens_per_s_per_gpu": N / (per_step[0] / 1e3)},
         "loss": final_loss,
         "clocks": clk,
         "e2e": e2e,
@@ -723,6 +729,8 @@ def run_kernel(args):
 
 def main():
     args = parse()
+    if args.steps < 1 or args.warmup < 0:
+        raise SystemExit("bench.py: --steps must be >= 1 and --warmup >= 0")
     if args.kernel:
         run_kernel(args)
         return
