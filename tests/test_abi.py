@@ -128,3 +128,26 @@ def test_recompute_workspace_keeps_one_layer_of_activations():
     import scratch_llama_decoder_b200 as P
     with pytest.raises(P.LLMError):
         llm_workspace_bytes(dict(cfg, recompute=2))
+
+
+def test_every_context_call_refuses_a_null_context():
+    """Every entry point taking an llm_ctx (read from include/llm.h) returns
+    LLM_ERR_ARG for a null context before touching a device; llm_destroy
+    ignores it and llm_last_launch_count reports 0."""
+    import re
+    import scratch_llama_decoder_b200 as P
+    hdr = open(os.path.join(ROOT, "include", "llm.h")).read()
+    names = re.findall(r"^\w[\w ]*?\**\s*(llm_\w+)\((?:const )?llm_ctx \*", hdr, re.M)
+    assert len(names) >= 20
+    fill = {C.c_void_p: None, C.c_int: 1, C.c_int64: 1, C.c_uint64: 1, C.c_float: 1.0,
+            C.c_double: 1.0}
+    for name in names:
+        fn = getattr(P.lib, name)
+        args = [None] + [fill.get(t) for t in fn.argtypes[1:]]
+        rc = fn(*args)
+        if name == "llm_destroy":
+            assert rc is None
+        elif name == "llm_last_launch_count":
+            assert rc == 0
+        else:
+            assert rc == P.LLM_ERR_ARG, name
