@@ -180,6 +180,27 @@ int llm_adamw_range(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, f
 int llm_flag_out(llm_ctx *ctx, int32_t *d_flag);
 int llm_flag_in(llm_ctx *ctx, const int32_t *d_flag);
 
+/* Gradient buckets, so that a data-parallel exchange of the gradient overlaps
+ * the backward that produces it (one process per GPU; the exchange, e.g. an
+ * NCCL all-reduce per bucket, runs on the caller's own stream).  The flat
+ * gradient splits into n_layer + 2 contiguous buckets, numbered in the order
+ * the backward finishes them: 0 = gf and Wlm (the end of the buffer), k = 1 ..
+ * n_layer = layer n_layer - k, n_layer + 1 = wte (the start of the buffer).
+ *   llm_grad_bucket_range (host only): offset and element count of bucket k
+ *     in the flat buffer; LLM_ERR_CONFIG for an invalid config, LLM_ERR_ARG
+ *     for k outside [0, n_layer + 1] or a null pointer.
+ *   llm_set_grad_buckets: with enable = 1 every later llm_grad records one
+ *     event per bucket on the context's stream once that bucket's gradients
+ *     are final (nothing else changes: the gradients are bit-identical);
+ *     0 turns it off (the default).  llm_step never records them.
+ *   llm_grad_bucket_wait: makes `stream` (a cudaStream_t on the context's
+ *     device) wait until bucket k of the most recent llm_grad is final.
+ *     LLM_ERR_ARG for k out of range or when that llm_grad ran without
+ *     buckets. */
+int llm_grad_bucket_range(const llm_config *cfg, int k, int64_t *offset, int64_t *count);
+int llm_set_grad_buckets(llm_ctx *ctx, int enable);
+int llm_grad_bucket_wait(llm_ctx *ctx, int k, void *stream);
+
 /* Single-token decode against a key/value cache (Hephaistos, feature list:
  * "True KV Cache", the prompt is processed once and every later position
  * costs one pass over a single row per sequence; strata, model table: the

@@ -66,6 +66,9 @@ EXPORTS = {
     "llm_adamw_range": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _f, _f, _f]),
     "llm_flag_out": (_i, [_vp, _vp]),
     "llm_flag_in": (_i, [_vp, _vp]),
+    "llm_grad_bucket_range": (_i, [_cfgp, _i, C.POINTER(_i64), C.POINTER(_i64)]),
+    "llm_set_grad_buckets": (_i, [_vp, _i]),
+    "llm_grad_bucket_wait": (_i, [_vp, _i, _vp]),
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
     "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),
     "llm_sample_ex": (_i, [_vp, _vp, _i64, _i, _f, _i, _f, _f, _vp, _i64, _i, _vp, _vp]),
@@ -142,6 +145,21 @@ def llm_workspace_bytes(cfg) -> int:
     b = C.c_int64(0)
     check(lib.llm_workspace_bytes(C.byref(c), C.byref(b)), "llm_workspace_bytes")
     return b.value
+
+
+def grad_buckets(cfg):
+    """[(offset, count)] of the gradient buckets in the order the backward
+    finishes them (llm_grad_bucket_range; host only)."""
+    c = make_config(cfg)
+    out, k = [], 0
+    off, cnt = C.c_int64(0), C.c_int64(0)
+    while True:
+        rc = lib.llm_grad_bucket_range(C.byref(c), k, C.byref(off), C.byref(cnt))
+        if rc == LLM_ERR_ARG and k > 0:
+            return out
+        check(rc, "llm_grad_bucket_range")
+        out.append((off.value, cnt.value))
+        k += 1
 
 
 def lr_at(t, max_lr, min_lr, warmup, decay_start, total, shape="cosine") -> float:

@@ -184,6 +184,10 @@ struct llm_ctx {
   uint64_t drop_seed = 0;
   int64_t train_calls = 0;
   int *drop_step = nullptr;
+  // gradient buckets (llm_set_grad_buckets): one event per bucket, recorded by
+  // llm_grad's backward on the main stream once the bucket's gradients are final
+  std::vector<cudaEvent_t> ev_bucket;
+  bool buckets_on = false, buckets_recorded = false;
   // gradient clipping (llm_set_grad_clip): threshold, block sums, norm, scale
   float clip = 0.f;
   int clip_mode = 0;  // LLM_CLIP_L2 or LLM_CLIP_LINF
@@ -383,6 +387,7 @@ void llm_destroy(llm_ctx *c) {
   if (c->gexec) cudaGraphExecDestroy(c->gexec);
   if (c->dexec) cudaGraphExecDestroy(c->dexec);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
+  for (cudaEvent_t e : c->ev_bucket) cudaEventDestroy(e);
   tc_plan_destroy(c->tc);
   delete c;
 }
@@ -771,7 +776,12 @@ void wgrad_side(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t 
   c->cur = c->s;
 }
 
-void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
+// With `buckets`, an event per gradient bucket is recorded on the main stream
+// as soon as the bucket is final (bucket 0: gf and Wlm, after the first join
+// of the side stream; bucket L - l: layer l, after its g1 reduction, the
+// layer's weight gradients having been joined before; bucket L + 1: wte,
+// after the embedding scatter and the last join).
+void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool buckets = false) {
   const Dims &D = c->D;
   POff O{D};
   cudaStream_t s = c->s;
@@ -818,6 +828,7 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
                          true, D.dt},
          OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * 2 * D.h * d);
     join_side(c);  // the RMSNorm backward overwrites dx2 (dxA)
+    if (buckets && l == D.L - 1) cudaEventRecord(c->ev_bucket[0], s);  // gf, Wlm
     nb = rmsnorm_bwd(x1, rstd2, p + O.g2(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
                      D.d, s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
@@ -843,10 +854,15 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok) {
     nb = rmsnorm_bwd(x, rstd1, p + O.g1(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N, D.d,
                      s);
     reduce_partials(c->dgpart, nb, D.d, gr + O.g1(l), s);
+    if (buckets) cudaEventRecord(c->ev_bucket[D.L - l], s);  // layer l
   }
   if (drop) drop_rows(c->dx, N * d, drop_args(c, 0, 0), s);
   embed_bwd(tok, c->dx, gr, N, D.d, D.V, c->sort_scratch, s);
   join_side(c);  // every weight gradient is in place before AdamW
+  if (buckets) {
+    if (D.L == 0) cudaEventRecord(c->ev_bucket[0], s);
+    cudaEventRecord(c->ev_bucket[D.L + 1], s);  // wte
+  }
 }
 
 // One decode position for every sequence (position in c->dec_pos): the
@@ -1013,10 +1029,58 @@ int llm_grad(llm_ctx *c, const float *d_params, float *d_grads, const int32_t *d
   cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
                 c->flag_step, c->s);
   loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
-  backward(c, d_params, d_grads, d_tokens);
+  backward(c, d_params, d_grads, d_tokens, c->buckets_on);
+  c->buckets_recorded = c->buckets_on;
   or_flag(c->flag_step, c->flag_sticky, c->s);
   c->last_launches = g_launches;
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_set_grad_buckets(llm_ctx *c, int enable) {
+  if (!c) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
+  if (enable && c->ev_bucket.empty()) {
+    for (int k = 0; k < c->D.L + 2; k++) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+        for (cudaEvent_t x : c->ev_bucket) cudaEventDestroy(x);
+        c->ev_bucket.clear();
+        return LLM_ERR_CUDA;
+      }
+      c->ev_bucket.push_back(e);
+    }
+  }
+  c->buckets_on = enable != 0;
+  c->buckets_recorded = false;
+  return LLM_OK;
+}
+
+int llm_grad_bucket_range(const llm_config *cfg, int k, int64_t *offset, int64_t *count) {
+  if (!offset || !count) return LLM_ERR_ARG;
+  if (!valid_config(cfg)) return LLM_ERR_CONFIG;
+  const Dims D = make_dims(cfg);
+  if (k < 0 || k > D.L + 1) return LLM_ERR_ARG;
+  POff O{D};
+  if (k == 0) {  // gf, Wlm
+    *offset = O.gf();
+    *count = D.P - O.gf();
+  } else if (k <= D.L) {  // layer L - k
+    *offset = O.layer(D.L - k);
+    *count = D.layer_sz;
+  } else {  // wte
+    *offset = 0;
+    *count = (int64_t)D.V * D.d;
+  }
+  return LLM_OK;
+}
+
+int llm_grad_bucket_wait(llm_ctx *c, int k, void *stream) {
+  if (!c) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
+  if (!c->buckets_recorded || k < 0 || k > c->D.L + 1) return LLM_ERR_ARG;
+  return cudaStreamWaitEvent((cudaStream_t)stream, c->ev_bucket[k], 0) == cudaSuccess
+             ? LLM_OK
+             : LLM_ERR_CUDA;
 }
 
 int llm_adamw(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v, int64_t t,

@@ -18,6 +18,14 @@ ranks' mean losses (divided by the rank count it is the batch mean).
 The engine is a LlamaStep (or any object with its grad / adamw / flag_out /
 flag_in methods, a device and, for CUDA, a stream); collectives are issued on
 the engine's stream so that they follow its kernels in order.
+
+With overlap=True the gradient is exchanged in buckets while the backward
+still runs: the engine records an event per bucket as its backward finishes
+it (layers from the last to the first), a communication stream waits for each
+bucket's event and all-reduces that bucket, and the engine's stream waits for
+the communication stream before the update.  The sums are the same numbers as
+one all-reduce of the whole buffer (the reduction of each element is the same
+over the same ranks).
 """
 import contextlib
 
@@ -26,12 +34,33 @@ import torch.distributed as dist
 
 
 class DataParallelStep:
-    def __init__(self, engine, group=None):
+    def __init__(self, engine, group=None, overlap=False):
         self.engine = engine
         self.group = group
         self.world = (dist.get_world_size(group)
                       if dist.is_available() and dist.is_initialized() else 1)
         self.flag = torch.zeros(1, dtype=torch.int32, device=engine.device)
+        self.overlap = bool(overlap) and self.world > 1
+        self._comm = None
+        if self.overlap:
+            engine.set_grad_buckets(True)
+            self.buckets = engine.grad_buckets()
+            if engine.device.type == "cuda":
+                self._comm = torch.cuda.Stream(device=engine.device)
+
+    def _exchange_buckets(self, grads):
+        """One all-reduce per bucket, each after the backward has finished it."""
+        e = self.engine
+        for k, (off, cnt) in enumerate(self.buckets):
+            if self._comm is not None:
+                e.grad_bucket_wait(k, self._comm)
+                with torch.cuda.stream(self._comm):
+                    dist.all_reduce(grads[off:off + cnt], op=dist.ReduceOp.SUM, group=self.group)
+            else:
+                e.grad_bucket_wait(k, None)
+                dist.all_reduce(grads[off:off + cnt], op=dist.ReduceOp.SUM, group=self.group)
+        if self._comm is not None:
+            e.stream.wait_stream(self._comm)
 
     def _stream(self):
         e = self.engine
@@ -44,7 +73,10 @@ class DataParallelStep:
         with self._stream():
             e.grad(params, grads, tokens, targets, loss)
             if self.world > 1:
-                dist.all_reduce(grads, op=dist.ReduceOp.SUM, group=self.group)
+                if self.overlap:
+                    self._exchange_buckets(grads)
+                else:
+                    dist.all_reduce(grads, op=dist.ReduceOp.SUM, group=self.group)
                 e.flag_out(self.flag)
                 dist.all_reduce(self.flag, op=dist.ReduceOp.MAX, group=self.group)
                 e.flag_in(self.flag)

@@ -143,6 +143,22 @@ class LlamaStep:
         """OR the int32 word flag into the step's error word (llm_flag_in)."""
         L.check(L.lib.llm_flag_in(self.ctx, _ptr(flag)), "llm_flag_in")
 
+    def grad_buckets(self):
+        """[(offset, count)] of the gradient buckets, in the order llm_grad's
+        backward finishes them."""
+        return L.grad_buckets(self.cfg)
+
+    @_on_device
+    def set_grad_buckets(self, enable):
+        L.check(L.lib.llm_set_grad_buckets(self.ctx, int(bool(enable))), "llm_set_grad_buckets")
+
+    @_on_device
+    def grad_bucket_wait(self, k, stream):
+        """Makes torch stream `stream` wait until bucket k of the last
+        llm_grad is final."""
+        L.check(L.lib.llm_grad_bucket_wait(self.ctx, int(k), C.c_void_p(stream.cuda_stream)),
+                "llm_grad_bucket_wait")
+
     @_on_device
     def decode(self, params, tokens, pos, logits=None):
         """Logits [B, V] of position pos (llm_decode); tokens: int32 [B]."""

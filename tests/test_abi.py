@@ -151,3 +151,37 @@ def test_every_context_call_refuses_a_null_context():
             assert rc == 0
         else:
             assert rc == P.LLM_ERR_ARG, name
+
+
+@pytest.mark.parametrize("name,over", [("c1", {}), ("c4", {}), ("c5", {}), ("c1", dict(n_layer=0))])
+def test_grad_buckets_tile_the_gradient_in_backward_order(name, over):
+    """llm_grad_bucket_range: n_layer + 2 contiguous buckets covering the flat
+    gradient exactly once, numbered in the order the backward finishes them
+    (head, layers from the last, embedding)."""
+    import scratch_llama_decoder_b200 as P
+    cfg = get_config(name, **over)
+    b = P.grad_buckets(cfg)
+    L = cfg["n_layer"]
+    assert len(b) == L + 2
+    lay = {nm: (off, r * k) for nm, off, r, k in O.param_layout(cfg)}
+    n = O.n_params(cfg)
+    assert sorted(b) == [(o, c) for o, c in sorted(b)]
+    pos = 0
+    for off, cnt in sorted(b):  # a tiling of [0, n)
+        assert off == pos and cnt > 0
+        pos += cnt
+    assert pos == n
+    assert b[-1] == (0, lay["wte"][1])                    # the embedding comes last
+    assert b[0] == (lay["gf"][0], n - lay["gf"][0])       # the head first
+    for k in range(1, L + 1):                              # then layers L-1 .. 0
+        mine = [v for nm, v in lay.items() if nm.startswith(f"l{L - k}.")]
+        assert b[k] == (lay[f"l{L - k}.g1"][0], sum(c for _, c in mine))
+    c = P.make_config(cfg)
+    off, cnt = C.c_int64(0), C.c_int64(0)
+    assert P.lib.llm_grad_bucket_range(C.byref(c), L + 2, C.byref(off), C.byref(cnt)) == \
+        P.LLM_ERR_ARG
+    assert P.lib.llm_grad_bucket_range(C.byref(c), -1, C.byref(off), C.byref(cnt)) == \
+        P.LLM_ERR_ARG
+    bad = P.make_config(get_config(name, **dict(over, n_head=3)))
+    assert P.lib.llm_grad_bucket_range(C.byref(bad), 0, C.byref(off), C.byref(cnt)) == \
+        P.LLM_ERR_CONFIG

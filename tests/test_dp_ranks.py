@@ -41,6 +41,18 @@ class OracleEngine:
     def flag_out(self, f):
         f.fill_(self.flag)
 
+    # gradient buckets: the library's ranges (host only); the oracle's
+    # gradient is complete when grad returns, so waiting is a no-op
+    def set_grad_buckets(self, enable):
+        self.buckets_on = bool(enable)
+
+    def grad_buckets(self):
+        import scratch_llama_decoder_b200 as P
+        return P.grad_buckets(self.cfg)
+
+    def grad_bucket_wait(self, k, stream):
+        assert self.buckets_on and stream is None
+
     def flag_in(self, f):
         self.flag |= int(f.item())
 
@@ -119,7 +131,7 @@ def _rank_main_sharded(rank, world, port, full_cfg, steps, q):
         dist.destroy_process_group()
 
 
-def _rank_main(rank, world, port, full_cfg, steps, fail_rank, fail_at, q):
+def _rank_main(rank, world, port, full_cfg, steps, fail_rank, fail_at, q, overlap=False):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -133,7 +145,8 @@ def _rank_main(rank, world, port, full_cfg, steps, fail_rank, fail_at, q):
         share = full_cfg["batch"] // world
         cfg = dict(full_cfg, batch=share)
         eng = OracleEngine(cfg, fail_at=fail_at if rank == fail_rank else None)
-        dp = DataParallelStep(eng)
+        dp = DataParallelStep(eng, overlap=overlap)
+        assert dp.overlap == overlap
         out = _run(eng, dp, p, tok[rank * share:(rank + 1) * share],
                    tgt[rank * share:(rank + 1) * share], steps, full_cfg["lr"], full_cfg["wd"])
         q.put((rank, out))
@@ -141,11 +154,12 @@ def _rank_main(rank, world, port, full_cfg, steps, fail_rank, fail_at, q):
         dist.destroy_process_group()
 
 
-def _two_ranks(full_cfg, steps, fail_rank=-1, fail_at=None):
+def _two_ranks(full_cfg, steps, fail_rank=-1, fail_at=None, overlap=False):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, full_cfg, steps, fail_rank, fail_at, q))
+    procs = [ctx.Process(target=_rank_main,
+                         args=(r, 2, port, full_cfg, steps, fail_rank, fail_at, q, overlap))
              for r in range(2)]
     for pr in procs:
         pr.start()
@@ -236,3 +250,23 @@ def test_sharded_wrapper_on_one_rank_is_the_plain_wrapper():
     np.testing.assert_array_equal(P[:p.size].numpy(), ref[0])
     np.testing.assert_array_equal(M[:p.size].numpy(), ref[1])
     assert not G[p.size:].any() and not P[p.size:].any()
+
+
+def test_bucketed_exchange_equals_the_whole_buffer_exchange():
+    """overlap=True: one all-reduce per gradient bucket (the library's ranges)
+    gives the same parameters, moments and losses as one all-reduce of the
+    whole buffer, bit for bit, and the one-process step on the whole batch."""
+    from synth import get_config
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    full = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_head=2, d_ff=42,
+                      ctx=5, batch=2, init_std=0.3, name="gqa-small", index=9)
+    whole = _two_ranks(full, steps=2)
+    bucketed = _two_ranks(full, steps=2, overlap=True)
+    p, tok, tgt = _setup(full)
+    eng = OracleEngine(full)
+    ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 2, full["lr"], full["wd"])
+    for r in (0, 1):
+        for a, b in zip(bucketed[r][:3], whole[r][:3]):
+            np.testing.assert_array_equal(a, b)
+        assert bucketed[r][3] == whole[r][3]
+        np.testing.assert_allclose(bucketed[r][0], ref[0], rtol=1e-12, atol=1e-15)

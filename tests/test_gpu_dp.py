@@ -127,3 +127,39 @@ def test_sharded_step_on_one_rank_is_step():
         assert torch.equal(a, b)
     assert not Gp[n:].any()  # the pad past the parameters stays zero
     m.close()
+
+
+def test_grad_buckets_events_and_identical_gradient():
+    """llm_set_grad_buckets: the gradient is bit-identical with the bucket
+    events on, and a second stream that waits for bucket k (llm_grad_bucket_wait)
+    reads that bucket's final values; waiting before a bucketed llm_grad is
+    refused."""
+    import scratch_llama_decoder_b200 as L
+    cfg, m, P, G, M, V, td, yd = _setup()
+    loss = torch.zeros(1, device="cuda")
+    side = torch.cuda.Stream()
+    with pytest.raises(L.LLMError):
+        m.grad_bucket_wait(0, side)
+    m.grad(P, G, td, yd, loss)
+    ref = G.clone()
+    m.set_grad_buckets(True)
+    buckets = m.grad_buckets()
+    assert len(buckets) == cfg["n_layer"] + 2
+    G.zero_()
+    m.grad(P, G, td, yd, loss)
+    copies = []
+    for k, (off, cnt) in enumerate(buckets):
+        m.grad_bucket_wait(k, side)
+        with torch.cuda.stream(side):
+            copies.append(G[off:off + cnt].clone())
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    assert torch.equal(G, ref)
+    for (off, cnt), c in zip(buckets, copies):
+        assert torch.equal(c, ref[off:off + cnt])
+    with pytest.raises(L.LLMError):
+        m.grad_bucket_wait(len(buckets), side)
+    m.set_grad_buckets(False)
+    with pytest.raises(L.LLMError):
+        m.grad_bucket_wait(0, side)
+    m.close()
