@@ -537,18 +537,18 @@ def run_decode(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clocks.start()
     clocks.wait_first()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(args.steps):
+        ev[0].record(stream)
+        for k in range(args.steps):
             tk.copy_(cols[pos])
             model.decode(P, tk, pos, logits=lg)
             pos += 1
-        e1.record(stream)
+            ev[k + 1].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
+    per_step = sorted(ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps))
     st = model.status()
     assert st == 0, f"timed decode failed with status {st}"
     byt = [decode_bytes(cfg, q) for q in range(first, pos)]
@@ -611,6 +611,9 @@ def run_decode(args, rank, world, local_rank):
                      "weight_bytes": byt[0][1], "kv_bytes_first": byt[0][2],
                      "peak_source": f"{src} hbm_gbs"},
         "gpu_launches": launches * args.steps,
+        # this rank's positions: median and best decode step (the later
+        # positions read more cached keys and values)
+        "per_step": {"median_ms": per_step[len(per_step) // 2], "best_ms": per_step[0]},
         "clocks": clk,
         "e2e": e2e,
     }
