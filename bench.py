@@ -14,7 +14,11 @@ The library runs on its own stream, where llm_step captures the step into a
 CUDA graph on its second call and replays it afterwards (the warm-up steps
 include the capture).
 With N > 1 GPUs every rank runs an independent replica on its own batch
-(weak scaling; no gradient exchange is part of the timed step).
+(weak scaling; no gradient exchange is part of the timed step), or, with
+--dp allreduce|overlap|sharded, one model trained data-parallel: the same
+weights on every rank, each rank's own batch, and the NCCL gradient exchange
+(one all-reduce, one per layer bucket overlapped with the backward, or
+reduce-scatter + sharded AdamW + all-gather) inside every timed step.
 The roofline object is for the dominant kernel (the tcgen05 GEMM): its
 algorithmic FLOPs over the summed device time of its launches, taken with CUDA
 events around every GEMM launch over K more steps run right after the timed
@@ -112,6 +116,10 @@ def parse(argv=None):
                     help="keep only layer inputs; recompute activations in the backward")
     ap.add_argument("--ctx", type=int, default=None, help="override the context length")
     ap.add_argument("--batch", type=int, default=None, help="override the batch")
+    ap.add_argument("--dp", default="none", choices=["none", "allreduce", "overlap", "sharded"],
+                    help="with --gpus N > 1: one model trained data-parallel (gradient "
+                         "all-reduce, the same per layer bucket overlapped with the backward, or "
+                         "a sharded optimiser) instead of N independent replicas")
     return ap.parse_args(argv)
 
 
@@ -321,12 +329,26 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     model = LlamaStep(cfg, device=dev, stream=stream)
     apply_options(model, opts)
-    p_host = make_params(cfg, model.layout, seed=1001 + cfg["index"] + 7919 * rank)
+    dp_mode = args.dp if world > 1 else "none"
+    # replicas start from their own weights; a data-parallel model is one
+    # model, the same weights on every rank (each rank its own data)
+    p_host = make_params(cfg, model.layout,
+                         seed=1001 + cfg["index"] + (7919 * rank if dp_mode == "none" else 0))
     tok_h, tgt_h = make_batch(cfg, seed=1000 + cfg["index"] + 7919 * rank)
-    P = torch.tensor(p_host, device=dev)
-    G = torch.zeros_like(P)
-    Mo = torch.zeros_like(P)
-    Vo = torch.zeros_like(P)
+    stepper = None
+    if dp_mode == "sharded":
+        from scratch_llama_decoder_b200.dp import ShardedDataParallelStep
+        stepper = ShardedDataParallelStep(model, model.n_params)
+        P, G, Mo, Vo = stepper.buffers()  # padded; the moments are this rank's chunk
+        P[:model.n_params].copy_(torch.from_numpy(p_host))
+    else:
+        if dp_mode != "none":
+            from scratch_llama_decoder_b200.dp import DataParallelStep
+            stepper = DataParallelStep(model, overlap=dp_mode == "overlap")
+        P = torch.tensor(p_host, device=dev)
+        G = torch.zeros_like(P)
+        Mo = torch.zeros_like(P)
+        Vo = torch.zeros_like(P)
     tok = torch.tensor(tok_h, device=dev)
     tgt = torch.tensor(tgt_h, device=dev)
     loss = torch.zeros(1, device=dev)
@@ -337,16 +359,28 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    def train_step(t):
+        # every step of this run, timed or not, goes through here (with a
+        # sharded optimiser the moments are chunk-sized: llm_step must not
+        # see them)
+        if stepper is None:
+            model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+        else:
+            stepper.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+
+    def step_launches():
+        return model.last_launch_count() if stepper is None else stepper.last_launches
+
     torch.cuda.synchronize()  # inputs written on the default stream are in place
     t = 0
     # the warm-up steps (>= 3) run the step once as launches, then capture the
     # step graph and replay it; the timed steps are replays
     for _ in range(args.warmup):
         t += 1
-        model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+        train_step(t)
     st = model.status()
     assert st == 0, f"warm-up step failed with status {st}"
-    launches_per_step = model.last_launch_count()
+    launches_per_step = step_launches()
 
     clocks = Clocks(local_rank)
     barrier()
@@ -359,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
     ev[0].record(stream)
     for k in range(args.steps):
         t += 1
-        model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+        train_step(t)
         ev[k + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -371,7 +405,7 @@ def run_ours(args, rank, world, local_rank):
     model.set_kernel_timing(True)
     for _ in range(args.steps):
         t += 1
-        model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+        train_step(t)
     g_ms, g_flops, g_launch = model.read_kernel_timing()
     model.set_kernel_timing(False)
     # clocks sampled over the timed region and the GEMM-timing pass after it
@@ -398,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
                 t += 1
                 tok.copy_(tok_pin, non_blocking=True)
                 tgt.copy_(tgt_pin, non_blocking=True)
-                model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+                train_step(t)
                 loss_pin.copy_(loss, non_blocking=True)
                 stream.synchronize()
             f0.record(stream)
@@ -406,7 +440,7 @@ def run_ours(args, rank, world, local_rank):
                 t += 1
                 tok.copy_(tok_pin, non_blocking=True)
                 tgt.copy_(tgt_pin, non_blocking=True)
-                model.step(P, G, Mo, Vo, t, tok, tgt, lr, wd, loss)
+                train_step(t)
                 loss_pin.copy_(loss, non_blocking=True)
                 stream.synchronize()
             f1.record(stream)
@@ -432,8 +466,9 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
         if cfg["compute"] == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": workload, "tokens_per_step": N, "batch": cfg["batch"],
-                   "seq_len": cfg["ctx"], "parallelism": f"replicas x{world}" if world > 1
-                   else "single GPU", "l2": "inputs larger than L2 (saved activations of "
+                   "seq_len": cfg["ctx"],
+                   "parallelism": ("single GPU" if world == 1 else f"replicas x{world}"
+                                   if dp_mode == "none" else f"dp{world} ({dp_mode})"), "l2": "inputs larger than L2 (saved activations of "
                    "several GB per step; no flush)"},
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM (all projection GEMMs of the "
                      "step)", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",

@@ -68,10 +68,15 @@ class DataParallelStep:
             return torch.cuda.stream(e.stream)
         return contextlib.nullcontext()
 
+    def _launches(self):
+        n = getattr(self.engine, "last_launch_count", None)
+        return n() if n else 0
+
     def step(self, params, grads, m, v, t, tokens, targets, lr, wd, loss):
         e = self.engine
         with self._stream():
             e.grad(params, grads, tokens, targets, loss)
+            launches = self._launches()
             if self.world > 1:
                 if self.overlap:
                     self._exchange_buckets(grads)
@@ -82,6 +87,8 @@ class DataParallelStep:
                 e.flag_in(self.flag)
                 dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=self.group)
             e.adamw(params, grads, m, v, t, lr, wd, grad_scale=1.0 / self.world)
+            # the library's kernels of this step (llm_grad and llm_adamw)
+            self.last_launches = launches + self._launches()
         return loss
 
 
@@ -124,6 +131,7 @@ class ShardedDataParallelStep(DataParallelStep):
         C, lo, cnt = self.chunk, self.lo, self.count
         with self._stream():
             e.grad(params, grads, tokens, targets, loss)
+            launches = self._launches()
             if self.world > 1:
                 if self._gshard is None:
                     self._gshard = torch.zeros(C, dtype=grads.dtype, device=grads.device)
@@ -138,6 +146,7 @@ class ShardedDataParallelStep(DataParallelStep):
                 gs = grads
             e.adamw_range(params[lo:lo + cnt], gs[:cnt], m[:cnt], v[:cnt], t, lr, wd,
                           grad_scale=1.0 / self.world)
+            self.last_launches = launches + self._launches()
             if self.world > 1:
                 src = params[lo:lo + C]
                 if dist.get_backend(self.group) != "nccl":

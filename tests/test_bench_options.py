@@ -33,3 +33,9 @@ def test_oracle_sample_runs_with_every_option():
                                            "--dropout", "0.2", "--rope-scale", "2"]))[1]
     rate, t, cores, S = bench.oracle_sample_rate(cfg, 8, reps=2, warmup=1, opts=opts)
     assert rate > 0 and S == 8 and cores >= 1
+
+
+def test_data_parallel_modes_parse():
+    assert bench.parse([]).dp == "none"
+    for mode in ("allreduce", "overlap", "sharded"):
+        assert bench.parse(["--dp", mode]).dp == mode
