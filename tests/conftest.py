@@ -19,7 +19,7 @@ def pytest_configure(config):
 # L-infinity clipping).
 _NEXT = ("test_zz_no_alloc.py",)
 _LATE = ("test_gpu_dp.py", "test_gpu_dropout.py", "test_gpu_sample_ext.py",
-         "test_gpu_long_context.py", "test_gpu_clip_linf.py")
+         "test_gpu_long_context.py", "test_gpu_clip_linf.py", "test_gpu_c_abi.py")
 
 
 def pytest_collection_modifyitems(session, config, items):
