@@ -15,15 +15,17 @@ def pytest_configure(config):
 # tests of the training step, its kernels and decode first, then the
 # allocation-free entry (its file sets up per-device state on first use, which
 # no other test reads), and last the tests of the entry points built on the
-# step (data parallelism, dropout, the extended sampler, longer contexts,
-# L-infinity clipping).
+# step, in this order: L-infinity clipping, data parallelism, the C program,
+# the extended sampler, longer contexts, dropout.
 _NEXT = ("test_zz_no_alloc.py",)
-_LATE = ("test_gpu_dp.py", "test_gpu_dropout.py", "test_gpu_sample_ext.py",
-         "test_gpu_long_context.py", "test_gpu_clip_linf.py", "test_gpu_c_abi.py")
+_LATE = ("test_gpu_clip_linf.py", "test_gpu_dp.py", "test_gpu_c_abi.py",
+         "test_gpu_sample_ext.py", "test_gpu_long_context.py", "test_gpu_dropout.py")
 
 
 def pytest_collection_modifyitems(session, config, items):
     def rank(item):
         name = os.path.basename(str(item.fspath))
-        return 2 if name in _LATE else 1 if name in _NEXT else 0
+        if name in _LATE:
+            return 2 + _LATE.index(name)
+        return 1 if name in _NEXT else 0
     items.sort(key=rank)  # stable: the order inside each group is kept
