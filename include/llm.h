@@ -349,6 +349,15 @@ int llm_set_rope_scale(llm_ctx *ctx, float factor);
  * 0 <= p < 1. */
 int llm_set_dropout(llm_ctx *ctx, float p, uint64_t seed);
 
+/* The mask counter n of llm_set_dropout: the number the next training call
+ * draws its masks with.  Host only (no device work, no synchronisation).  A
+ * run checkpointed by saving params, m, v, t and n, and resumed in a new
+ * context with the same llm_set_dropout(p, seed) then llm_set_dropout_calls(n),
+ * continues with the masks the uninterrupted run would have drawn.
+ * LLM_ERR_ARG for a null pointer or n outside [0, 2^31). */
+int llm_get_dropout_calls(llm_ctx *ctx, int64_t *n);
+int llm_set_dropout_calls(llm_ctx *ctx, int64_t n);
+
 /* The norm clipping uses: LLM_CLIP_L2, the Euclidean norm of the whole
  * gradient (the default), or LLM_CLIP_LINF, its largest absolute element
  * (randyGPT, Training: gradient clipping by the L-infinity norm at 1.0); the

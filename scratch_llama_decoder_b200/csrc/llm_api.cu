@@ -474,6 +474,18 @@ int llm_set_dropout(llm_ctx *c, float p, uint64_t seed) {
   return LLM_OK;
 }
 
+int llm_get_dropout_calls(llm_ctx *c, int64_t *n) {
+  if (!c || !n) return LLM_ERR_ARG;
+  *n = c->train_calls;
+  return LLM_OK;
+}
+
+int llm_set_dropout_calls(llm_ctx *c, int64_t n) {
+  if (!c || n < 0 || n > INT32_MAX) return LLM_ERR_ARG;
+  c->train_calls = n;
+  return LLM_OK;
+}
+
 int llm_set_grad_clip_mode(llm_ctx *c, int mode) {
   if (!c || (mode != LLM_CLIP_L2 && mode != LLM_CLIP_LINF)) return LLM_ERR_ARG;
   if (!on_device(c)) return LLM_ERR_ARG;

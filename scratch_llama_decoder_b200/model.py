@@ -190,6 +190,15 @@ class LlamaStep:
         """Inverted dropout in later training calls (llm_set_dropout)."""
         L.check(L.lib.llm_set_dropout(self.ctx, float(p), int(seed)), "llm_set_dropout")
 
+    def dropout_calls(self):
+        """The mask counter: the number the next training call draws with."""
+        n = C.c_int64(0)
+        L.check(L.lib.llm_get_dropout_calls(self.ctx, C.byref(n)), "llm_get_dropout_calls")
+        return n.value
+
+    def set_dropout_calls(self, n):
+        L.check(L.lib.llm_set_dropout_calls(self.ctx, int(n)), "llm_set_dropout_calls")
+
     @_on_device
     def set_grad_clip(self, max_norm):
         """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
