@@ -9,7 +9,6 @@ import socket
 import sys
 
 import numpy as np
-import pytest
 import torch
 import torch.multiprocessing as mp
 

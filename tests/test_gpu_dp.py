@@ -4,7 +4,6 @@ undoes an exact scaling of the gradient, DataParallelStep without a process
 group is the plain step, and an error word brought in by llm_flag_in skips the
 update.  (Every call in this environment has one GPU; the rank logic with two
 ranks is tested on CPU in test_dp_ranks.py.)"""
-import numpy as np
 import pytest
 import torch
 

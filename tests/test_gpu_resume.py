@@ -4,7 +4,6 @@ beyond the caller's params, m, v and the step count t -- and, with dropout,
 the mask counter (llm_get_dropout_calls / llm_set_dropout_calls) -- so steps
 1..4 in one context equal steps 1..2, a checkpoint of those to host memory, a
 new context and steps 3..4, bit for bit."""
-import numpy as np
 import pytest
 import torch
 

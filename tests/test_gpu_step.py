@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from synth import get_config, make_batch, make_params
-from tests.gpu_util import TOL, compare, rel, run_gpu, run_oracle
+from tests.gpu_util import compare, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 

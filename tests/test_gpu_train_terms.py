@@ -9,7 +9,7 @@ import torch
 
 import oracle as O
 from synth import get_config, make_batch, make_params
-from tests.gpu_util import TOL, compare, rel, run_gpu, run_oracle
+from tests.gpu_util import TOL, compare, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
