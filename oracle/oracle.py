@@ -5,11 +5,15 @@ benchmark's CPU-baseline leg, never by the product library.  Arrays in and
 out are numpy float64 / int32; everything is computed on the host CPU.
 """
 import ctypes as C
+import os
+
 import numpy as np
 
 from .build import build
 
-_lib = C.CDLL(build())
+# LLM_ORACLE_LIB: another build of llama_oracle.c to load (the sanitizer test
+# loads one built with AddressSanitizer and UBSan)
+_lib = C.CDLL(os.environ.get("LLM_ORACLE_LIB") or build())
 
 _D = C.POINTER(C.c_double)
 _I32 = C.POINTER(C.c_int32)
