@@ -7,7 +7,9 @@ import ctypes as C
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libllm.so")
+# LLM_LIB: another build of the library to load (the sanitizer test loads one
+# whose host code is built with AddressSanitizer and UBSan)
+LIB_PATH = os.environ.get("LLM_LIB") or os.path.join(HERE, "libllm.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
