@@ -15,10 +15,11 @@ CUDA graph on its second call and replays it afterwards (the warm-up steps
 include the capture).
 With N > 1 GPUs every rank runs an independent replica on its own batch
 (weak scaling; no gradient exchange is part of the timed step), or, with
---dp allreduce|overlap|sharded, one model trained data-parallel: the same
-weights on every rank, each rank's own batch, and the NCCL gradient exchange
-(one all-reduce, one per layer bucket overlapped with the backward, or
-reduce-scatter + sharded AdamW + all-gather) inside every timed step.
+--dp allreduce|overlap|sharded|sharded-overlap, one model trained
+data-parallel: the same weights on every rank, each rank's own batch, and the
+NCCL gradient exchange (one all-reduce, one per layer bucket overlapped with
+the backward, reduce-scatter + sharded AdamW + all-gather, or that per bucket
+overlapped with the backward) inside every timed step.
 The roofline object is for the dominant kernel (the tcgen05 GEMM): its
 algorithmic FLOPs over the summed device time of its launches, taken with CUDA
 events around every GEMM launch over K more steps run right after the timed
@@ -116,10 +117,13 @@ def parse(argv=None):
                     help="keep only layer inputs; recompute activations in the backward")
     ap.add_argument("--ctx", type=int, default=None, help="override the context length")
     ap.add_argument("--batch", type=int, default=None, help="override the batch")
-    ap.add_argument("--dp", default="none", choices=["none", "allreduce", "overlap", "sharded"],
+    ap.add_argument("--dp", default="none",
+                    choices=["none", "allreduce", "overlap", "sharded", "sharded-overlap"],
                     help="with --gpus N > 1: one model trained data-parallel (gradient "
-                         "all-reduce, the same per layer bucket overlapped with the backward, or "
-                         "a sharded optimiser) instead of N independent replicas")
+                         "all-reduce, the same per layer bucket overlapped with the backward, a "
+                         "sharded optimiser, or that sharded optimiser with per-bucket "
+                         "reduce-scatters overlapped with the backward) instead of N independent "
+                         "replicas")
     return ap.parse_args(argv)
 
 
@@ -336,9 +340,10 @@ def run_ours(args, rank, world, local_rank):
                          seed=1001 + cfg["index"] + (7919 * rank if dp_mode == "none" else 0))
     tok_h, tgt_h = make_batch(cfg, seed=1000 + cfg["index"] + 7919 * rank)
     stepper = None
-    if dp_mode == "sharded":
+    if dp_mode in ("sharded", "sharded-overlap"):
         from scratch_llama_decoder_b200.dp import ShardedDataParallelStep
-        stepper = ShardedDataParallelStep(model, model.n_params)
+        stepper = ShardedDataParallelStep(model, model.n_params,
+                                          overlap=dp_mode == "sharded-overlap")
         P, G, Mo, Vo = stepper.buffers()  # padded; the moments are this rank's chunk
         P[:model.n_params].copy_(torch.from_numpy(p_host))
     else:

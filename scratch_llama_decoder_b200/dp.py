@@ -107,27 +107,93 @@ class ShardedDataParallelStep(DataParallelStep):
     size (together one all-reduce's traffic) and keeps 1 / ranks of m and v.
     Clipping is not applied here (its norm needs the whole gradient).
     buffers() allocates the padded parameter and gradient buffers and the
-    chunk-sized m and v."""
+    chunk-sized m and v.
 
-    def __init__(self, engine, n_params, group=None):
-        super().__init__(engine, group)
+    With overlap=True the exchange runs per gradient bucket while the
+    backward goes on: rank r owns piece r of every bucket (q = the bucket's
+    count / ranks rounded up to a multiple of 4; bucket offsets are multiples
+    of 4, so every piece is 16-byte aligned), each bucket is reduce-scattered
+    on a communication stream as soon as the backward has finished it, and
+    after the update each bucket's pieces are all-gathered.  A bucket's last
+    piece may reach up to 4 x ranks elements past the bucket: into the bucket
+    finished just before it (buckets complete from the end of the buffer
+    backwards, so those gradients are final when read, and the all-gathers,
+    in the same order, write back values that are already final and the same
+    on every rank) or, for the head, into the buffers' padding.  pieces lists
+    (bucket offset, q, elements kept, moment offset) of this rank."""
+
+    def __init__(self, engine, n_params, group=None, overlap=False):
+        super().__init__(engine, group, overlap)
         self.rank = dist.get_rank(group) if self.world > 1 else 0
         self.n = int(n_params)
-        self.chunk = ((self.n + self.world - 1) // self.world + 3) // 4 * 4
-        self.lo = self.rank * self.chunk
-        self.count = max(0, min(self.chunk, self.n - self.lo))
         self._gshard = None
+        if self.overlap:
+            self.pieces, mo = [], 0
+            for off, cnt in self.buckets:
+                assert off % 4 == 0
+                q = ((cnt + self.world - 1) // self.world + 3) // 4 * 4
+                self.pieces.append((off, q, max(0, min(q, cnt - self.rank * q)), mo))
+                mo += q
+            self.chunk = mo  # this rank's moments: one piece per bucket
+            end = max(off + self.world * q for off, q, _, _ in self.pieces)
+            self.padded = (max(self.n, end) + 3) // 4 * 4
+            self.lo, self.count = None, sum(k for _, _, k, _ in self.pieces)
+        else:
+            self.chunk = ((self.n + self.world - 1) // self.world + 3) // 4 * 4
+            self.padded = self.world * self.chunk
+            self.lo = self.rank * self.chunk
+            self.count = max(0, min(self.chunk, self.n - self.lo))
 
     def buffers(self, dtype=torch.float32):
         dev = self.engine.device
-        padded = self.world * self.chunk
+        padded = self.padded
         return (torch.zeros(padded, dtype=dtype, device=dev),
                 torch.zeros(padded, dtype=dtype, device=dev),
                 torch.zeros(self.chunk, dtype=dtype, device=dev),
                 torch.zeros(self.chunk, dtype=dtype, device=dev))
 
+    def _step_buckets(self, params, grads, m, v, t, tokens, targets, lr, wd, loss):
+        e, W = self.engine, self.world
+        if self._gshard is None:
+            self._gshard = torch.zeros(self.chunk, dtype=grads.dtype, device=grads.device)
+        gs = self._gshard
+        e.grad(params, grads, tokens, targets, loss)
+        launches = self._launches()
+        for k, (off, q, _, mo) in enumerate(self.pieces):
+            if self._comm is not None:
+                e.grad_bucket_wait(k, self._comm)
+                with torch.cuda.stream(self._comm):
+                    dist.reduce_scatter_tensor(gs[mo:mo + q], grads[off:off + W * q],
+                                               op=dist.ReduceOp.SUM, group=self.group)
+            else:
+                e.grad_bucket_wait(k, None)
+                dist.reduce_scatter_tensor(gs[mo:mo + q], grads[off:off + W * q],
+                                           op=dist.ReduceOp.SUM, group=self.group)
+        if self._comm is not None:
+            e.stream.wait_stream(self._comm)
+        e.flag_out(self.flag)
+        dist.all_reduce(self.flag, op=dist.ReduceOp.MAX, group=self.group)
+        e.flag_in(self.flag)
+        dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=self.group)
+        for off, q, keep, mo in self.pieces:
+            if keep:
+                a = off + self.rank * q
+                e.adamw_range(params[a:a + keep], gs[mo:mo + keep], m[mo:mo + keep],
+                              v[mo:mo + keep], t, lr, wd, grad_scale=1.0 / W)
+                launches += self._launches()
+        self.last_launches = launches
+        nccl = dist.get_backend(self.group) == "nccl"
+        for off, q, _, _ in self.pieces:
+            a = off + self.rank * q
+            src = params[a:a + q] if nccl else params[a:a + q].clone()
+            dist.all_gather_into_tensor(params[off:off + W * q], src, group=self.group)
+
     def step(self, params, grads, m, v, t, tokens, targets, lr, wd, loss):
         e = self.engine
+        if self.overlap:
+            with self._stream():
+                self._step_buckets(params, grads, m, v, t, tokens, targets, lr, wd, loss)
+            return loss
         C, lo, cnt = self.chunk, self.lo, self.count
         with self._stream():
             e.grad(params, grads, tokens, targets, loss)

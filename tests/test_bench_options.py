@@ -37,5 +37,5 @@ def test_oracle_sample_runs_with_every_option():
 
 def test_data_parallel_modes_parse():
     assert bench.parse([]).dp == "none"
-    for mode in ("allreduce", "overlap", "sharded"):
+    for mode in ("allreduce", "overlap", "sharded", "sharded-overlap"):
         assert bench.parse(["--dp", mode]).dp == mode

@@ -9,6 +9,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -101,7 +102,7 @@ def _run(engine, dp, p, tok, tgt, steps, lr, wd):
     return P.numpy(), M.numpy(), V.numpy(), losses
 
 
-def _rank_main_sharded(rank, world, port, full_cfg, steps, q):
+def _rank_main_sharded(rank, world, port, full_cfg, steps, q, overlap=False):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -116,7 +117,8 @@ def _rank_main_sharded(rank, world, port, full_cfg, steps, q):
         share = full_cfg["batch"] // world
         cfg = dict(full_cfg, batch=share)
         eng = OracleEngine(cfg)
-        dp = ShardedDataParallelStep(eng, O.n_params(cfg))
+        dp = ShardedDataParallelStep(eng, O.n_params(cfg), overlap=overlap)
+        assert dp.overlap == overlap
         P, G, M, V = dp.buffers(torch.float64)
         P[:p.size].copy_(torch.from_numpy(p))
         loss = torch.zeros(1, dtype=torch.float64)
@@ -124,8 +126,16 @@ def _rank_main_sharded(rank, world, port, full_cfg, steps, q):
             dp.step(P, G, M, V, t, torch.tensor(tok[rank * share:(rank + 1) * share]),
                     torch.tensor(tgt[rank * share:(rank + 1) * share]), full_cfg["lr"],
                     full_cfg["wd"], loss)
-        q.put((rank, (P[:p.size].numpy().copy(), M[:dp.count].numpy().copy(),
-                      V[:dp.count].numpy().copy(), dp.lo, dp.count)))
+        if overlap:  # the rank's pieces of every bucket, placed in the full layout
+            Mf, Vf = np.full(p.size, np.nan), np.full(p.size, np.nan)
+            for off, qq, keep, mo in dp.pieces:
+                a = off + rank * qq
+                Mf[a:a + keep] = M[mo:mo + keep].numpy()
+                Vf[a:a + keep] = V[mo:mo + keep].numpy()
+            q.put((rank, (P[:p.size].numpy().copy(), Mf, Vf, None, None)))
+        else:
+            q.put((rank, (P[:p.size].numpy().copy(), M[:dp.count].numpy().copy(),
+                          V[:dp.count].numpy().copy(), dp.lo, dp.count)))
     finally:
         dist.destroy_process_group()
 
@@ -269,3 +279,41 @@ def test_bucketed_exchange_equals_the_whole_buffer_exchange():
             np.testing.assert_array_equal(a, b)
         assert bucketed[r][3] == whole[r][3]
         np.testing.assert_allclose(bucketed[r][0], ref[0], rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_bucketed_sharded_optimiser_equals_one_process(world):
+    """ShardedDataParallelStep(overlap=True): per-bucket reduce-scatter (each
+    rank owning one piece of every bucket), AdamW on the pieces, per-bucket
+    all-gather.  The ranks' parameters agree bit for bit and equal the
+    one-process step on the whole batch; the pieces' moments, placed back,
+    cover every parameter exactly once and equal that step's moments."""
+    from synth import get_config
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    full = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_head=2, d_ff=42,
+                      ctx=5, batch=world, init_std=0.3, name="gqa-small", index=9)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_sharded, args=(r, world, port, full, 3, q, True))
+             for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=300) for _ in range(world))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    p, tok, tgt = _setup(full)
+    eng = OracleEngine(full)
+    ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 3, full["lr"], full["wd"])
+    Mf = np.full(p.size, np.nan)
+    Vf = np.full(p.size, np.nan)
+    for r in range(world):
+        np.testing.assert_array_equal(res[r][0], res[0][0])
+        np.testing.assert_allclose(res[r][0], ref[0], rtol=1e-12, atol=1e-15)
+        have = ~np.isnan(res[r][1])
+        assert not np.any(~np.isnan(Mf[have]))  # each element owned by one rank
+        Mf[have], Vf[have] = res[r][1][have], res[r][2][have]
+    assert not np.any(np.isnan(Mf))
+    np.testing.assert_allclose(Mf, ref[1], rtol=1e-10, atol=1e-18)
+    np.testing.assert_allclose(Vf, ref[2], rtol=1e-10, atol=1e-22)
