@@ -16,10 +16,12 @@ def pytest_configure(config):
 # allocation-free entry (its file sets up per-device state on first use, which
 # no other test reads), and last the tests of the entry points built on the
 # step, in this order: L-infinity clipping, data parallelism, the C program,
-# resume, the extended sampler, longer contexts, dropout.
+# resume, the extended sampler, longer contexts, the configuration limits,
+# dropout.
 _NEXT = ("test_zz_no_alloc.py",)
 _LATE = ("test_gpu_clip_linf.py", "test_gpu_dp.py", "test_gpu_c_abi.py", "test_gpu_resume.py",
-         "test_gpu_sample_ext.py", "test_gpu_long_context.py", "test_gpu_dropout.py")
+         "test_gpu_sample_ext.py", "test_gpu_long_context.py", "test_gpu_limits.py",
+         "test_gpu_dropout.py")
 
 
 def pytest_collection_modifyitems(session, config, items):
