@@ -25,7 +25,7 @@
  *     n_kv_head independently (MHA/GQA/MQA); AdamW decoupled, bias-corrected.
  *   randyGPT, "Training (Metal GPU path)": cross-entropy over all positions.
  *
- * Readings taken where the pages are silent (each listed in the design notes):
+ * Readings taken where the pages are silent:
  *   - attention scale 1/sqrt(head_dim); the causal mask keeps the diagonal;
  *   - GQA groups are contiguous: query head hq uses kv head hq / (H/Hkv);
  *   - RoPE: theta_j = base^(-2j/hd), position = index within the sequence,

@@ -374,11 +374,7 @@ bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int 
                  int *flag, cudaStream_t s) {
   using namespace attn_tc;
   if (hd != HD || !flag) return false;
-  static bool init = false;
-  if (!init) {
-    cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    init = true;
-  }
+  if (!smem_optin((const void *)k_attn_fwd_tc, SMEM_BYTES)) return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd;
   CUtensorMap map;
   if (!tc::tile_map_bf16(&map, qkv, qkvw, (int64_t)B * T, qkvw, 128)) return false;

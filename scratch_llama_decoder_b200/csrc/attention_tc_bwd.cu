@@ -601,12 +601,9 @@ bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *
   if (hd != HD || !flag || ((uintptr_t)o & 15) || ((uintptr_t)dqkv & 15) ||
       ((uintptr_t)cos_t & 15) || ((uintptr_t)sin_t & 15) || (!cos_t != !sin_t))
     return false;
-  static bool init = false;
-  if (!init) {
-    cudaFuncSetAttribute(k_attn_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
-    cudaFuncSetAttribute(k_attn_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, KV_SMEM);
-    init = true;
-  }
+  if (!smem_optin((const void *)k_attn_dq_tc, DQ_SMEM) ||
+      !smem_optin((const void *)k_attn_dkv_tc, KV_SMEM))
+    return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd, dw = (int64_t)H * hd;
   CUtensorMap mq, md;
   if (!tc::tile_map_bf16(&mq, qkv, qkvw, (int64_t)B * T, qkvw, 128) ||

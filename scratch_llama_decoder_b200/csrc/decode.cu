@@ -843,12 +843,8 @@ template <typename A, int GT>
 static void attn_launch(dim3 grid, size_t smem, cudaStream_t s, const void *qkv, int64_t qkvw,
                         int T, const int *pos, int H, int Hkv, int hd, int nch, int vec,
                         float *part, unsigned *count, void *o) {
-  static bool attr = false;  // opt in to the largest staged tile once per kernel
-  if (!attr) {
-    cudaFuncSetAttribute(k_attn_decode<A, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         2 * AT_KEYS * attn_row_bytes(AT_HDMAX, 4));
-    attr = true;
-  }
+  // room for the largest staged tile (a refusal fails the launch)
+  smem_optin((const void *)k_attn_decode<A, GT>, (int)(2 * AT_KEYS * attn_row_bytes(AT_HDMAX, 4)));
   launch_pdl(k_attn_decode<A, GT>, grid, dim3(AT_THREADS), smem, s, (const A *)qkv, qkvw, T, pos,
              H, Hkv, hd, nch, vec, part, count, (A *)o);
 }
@@ -894,12 +890,7 @@ void sample_tokens_ex(const float *logits, int64_t ld, int rows, int V, float te
                       int top_k, float top_p, float penalty, const int32_t *hist,
                       int64_t hist_ld, int hist_len, const float *uni, int32_t *out,
                       cudaStream_t s) {
-  static bool attr = false;  // room for the largest history bitmap, once
-  if (!attr) {
-    cudaFuncSetAttribute(k_sample<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         SP_PEN_BYTES);
-    attr = true;
-  }
+  smem_optin((const void *)k_sample<true>, SP_PEN_BYTES);  // room for the largest history bitmap
   SampleExt e;
   e.top_p = top_p;
   e.penalty = penalty;

@@ -522,13 +522,13 @@ TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, 
   p->encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
   cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, dev);
   p->cos_t = cos_t; p->sin_t = sin_t; p->T = T; p->hd = hd; p->rot_cols = rot_cols; p->hp = hp;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(tc::k_gemm_tc<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
-    cudaFuncSetAttribute(tc::k_gemm_tc<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
-    cudaFuncSetAttribute(tc::k_gemm_tc<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
-    cudaFuncSetAttribute(tc::k_gemm_tc<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
-    attr_done = true;
+  // the plan's device is current here: opt every variant in on it
+  if (!smem_optin((const void *)tc::k_gemm_tc<false, false>, tc::SMEM_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc<false, true>, tc::SMEM_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc<true, false>, tc::SMEM_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc<true, true>, tc::SMEM_BYTES)) {
+    delete p;
+    return nullptr;
   }
   return p;
 }

@@ -208,6 +208,11 @@ void sample_tokens_ex(const float *logits, int64_t ld, int rows, int V, float te
                       cudaStream_t s);
 void set_device_int(int *p, int v, cudaStream_t s);
 
+// Opts `func` into `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to the device's context, so it is set once per
+// (device, kernel), under a lock; false when the runtime refuses it.
+bool smem_optin(const void *func, int bytes);
+
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;
 inline void count_launch(int n = 1) { g_launches += n; }

@@ -2,6 +2,9 @@
 // scatter-add, RMSNorm forward/backward, RoPE, SwiGLU, cross-entropy, loss
 // reduction, AdamW and initialisation.  Each cites the passage it computes.
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -9,6 +12,21 @@
 namespace llm {
 
 thread_local int g_launches = 0;
+
+bool smem_optin(const void *func, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::mutex mu;
+  static std::map<std::pair<int, const void *>, int> done;  // largest size set per (device, kernel)
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, func);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done[key] = bytes;
+  return true;
+}
 
 static inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
 
@@ -313,12 +331,17 @@ int rmsnorm_bwd(const float *x, const float *rstd, const float *g, const float *
     count_launch();
     return nblk;
   }
-  size_t smem = sizeof(float) * 8 * d;
-  if (dt == DT_BF16)
+  // generic width: 8 warps' gain-gradient rows in shared memory (128 KiB at
+  // the largest accepted width, 4096), so opt in above the 48 KiB default
+  const int smem = (int)(sizeof(float) * 8 * d);
+  if (dt == DT_BF16) {
+    smem_optin((const void *)k_rmsnorm_bwd<__nv_bfloat16>, smem);  // a refusal fails the launch
     k_rmsnorm_bwd<<<nblk, 256, smem, s>>>(x, rstd, g, dy, dres, dx, (__nv_bfloat16 *)dx_act, part,
                                           N, d);
-  else
+  } else {
+    smem_optin((const void *)k_rmsnorm_bwd<float>, smem);
     k_rmsnorm_bwd<<<nblk, 256, smem, s>>>(x, rstd, g, dy, dres, dx, (float *)dx_act, part, N, d);
+  }
   count_launch();
   return nblk;
 }

@@ -56,7 +56,6 @@ extern "C" int llm_kernel_embed_bwd_noalloc(const int32_t *d_tokens, const float
     }
     scratch = g_scratch_dev_ptr[dev];
   }
-  llm::g_launches = 0;
   llm::embed_bwd(d_tokens, d_dx, d_dwte, n_tokens, d_model, vocab, scratch, (cudaStream_t)stream);
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
