@@ -92,6 +92,8 @@ def parse(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads' step timings (per_config)")
     ap.add_argument("--kernel", default=None, choices=["gemm", "attention"],
                     help="time one hot-path kernel through the C ABI instead of the step")
     ap.add_argument("--shape", default="16384,3072,1024",
@@ -180,6 +182,56 @@ def step_flops(cfg):
     N = B * T
     attn = 12 * L * B * H * (T * (T + 1) / 2) * hd
     return 6.0 * M * N + attn, attn
+
+
+def step_bytes(cfg):
+    """HBM bytes of one step in the roofline's memory term (a model: what a
+    step must move at least once with the activations it keeps for the
+    backward).  Per token and layer: the saved activations -- the float32
+    residual inputs x and x1, and in the activation type xn1, q|k|v, o, xn2,
+    a|b and u, plus the float32 rstd pair and the log-sum-exps -- written once
+    by the forward and read once by the backward, and the float32 residual
+    gradient read and written at each of the layer's two residual joins.  Per
+    step: the low-precision weights read by the forward and by the data
+    gradients, the float32 weight gradients written, AdamW's 28 bytes per
+    parameter, the logits written, read by the cross-entropy, its gradient
+    written and read by the two lm_head GEMMs (four passes), and the embedding
+    rows gathered and their gradient rows read and written."""
+    V, d, L, H, Hkv, h, T, B = (cfg[k] for k in ("vocab", "d_model", "n_layer", "n_head",
+                                                 "n_kv_head", "d_ff", "ctx", "batch"))
+    hd = d // H
+    kvd = Hkv * hd
+    ab = 2 if cfg["compute"] == "bf16" else 4
+    N = B * T
+    saved = 8 * d + ab * (d + (d + 2 * kvd) + d + d + 2 * h + h) + 8 + 4 * H
+    per_tok_layer = 2 * saved + 16 * d
+    M = L * (d * (d + 2 * kvd) + d * d + 3 * d * h) + d * V
+    P = V * d + L * (2 * d + d * (d + 2 * kvd) + d * d + 3 * d * h) + d + d * V
+    per_step = 2 * ab * M + 4 * M + 28 * P + 4 * N * V * ab + 2 * N * d * 4 + V * d * 4
+    return N * L * per_tok_layer + per_step
+
+
+# nominal dense TF32 / BF16 tensor rates (1.1 and 2.25 PFLOP/s): a float32
+# workload's contractions are bounded by the TF32 rate at best
+TF32_OF_BF16 = 1.1 / 2.25
+
+
+def step_roofline(cfg, pk, step_ms):
+    """The step against max(FLOPs / tensor peak, bytes / HBM bandwidth)."""
+    F, F_attn = step_flops(cfg)
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    if cfg["compute"] != "bf16":
+        peak = peak * TF32_OF_BF16
+    byt = step_bytes(cfg)
+    t_tensor = F / (peak * 1e12) * 1e3
+    t_hbm = byt / (pk["hbm_gbs"] * 1e9) * 1e3
+    t_roof = max(t_tensor, t_hbm)
+    return {"flops": F, "attention_flops": F_attn, "bytes": byt,
+            "t_tensor_ms": t_tensor, "t_hbm_ms": t_hbm,
+            "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+            "tensor_peak_tflops": peak,
+            "frac_of_tensor_bound": t_tensor / step_ms,
+            "frac_of_roofline": t_roof / step_ms}
 
 
 # ------------------------------------------------------------------ clocks
@@ -481,9 +533,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": gemm_traffic(workload),
                      "launches": g_launch, "ms_total": g_ms,
                      "peak_source": f"{src} bf16_tflops_sustained"},
-        "step_roofline": {"flops": F, "attention_flops": F_attn,
-                          "t_tensor_ms": F / (peak_tc * 1e12) * 1e3,
-                          "frac_of_tensor_bound": (F / (peak_tc * 1e12)) / step_s},
+        "step_roofline": step_roofline(cfg, pk, step_s * 1e3),
         "gpu_launches": launches_per_step * args.steps,
         # this rank's steps (rank 0): median and best step, as tokens/s per GPU
         "per_step": {"median_ms": per_step[len(per_step) // 2], "best_ms": per_step[0],
@@ -493,6 +543,16 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "e2e": e2e,
     }
+    if world == 1 and not args.no_per_config and args.config == "c5" and not suffix:
+        # the other workloads, each timed the same way in this process (their
+        # own context, stream and clock record)
+        model.close()
+        del P, G, Mo, Vo, model
+        torch.cuda.empty_cache()
+        out["per_config"] = {}
+        for name in PER_CONFIG:
+            r = time_workload(name, args.steps, max(3, args.warmup), dev, local_rank, pk)
+            out["per_config"][r.pop("workload")] = r
     if world == 1 and not args.no_cpu_baseline:
         S = sample_tokens_for(cfg, 12.0, opts)
         rate, tsec, cores, S = oracle_sample_rate(cfg, S, opts=opts)
@@ -501,6 +561,61 @@ def run_ours(args, rank, world, local_rank):
             "sample": f"float64 oracle: forward+backward of a {S}-token prefix of one "
                       f"sequence plus AdamW over {S}/{N} of the parameters "
                       f"({tsec:.1f} s), scaled to tokens/s"}
+    return out
+
+
+PER_CONFIG = ("c2", "c3", "c4")
+
+
+def time_workload(name, steps, warmup, dev, local_rank, pk):
+    """One workload's training step timed as the headline is: its own stream
+    (graph replays after the warm-up), an event before the first timed step
+    and after each, clocks sampled over the timed region."""
+    import torch
+    from scratch_llama_decoder_b200 import LlamaStep
+    from synth import get_config, make_batch, make_params
+    cfg = get_config(name)
+    stream = torch.cuda.Stream(device=dev)
+    model = LlamaStep(cfg, device=dev, stream=stream)
+    P = torch.tensor(make_params(cfg, model.layout), device=dev)
+    G, Mo, Vo = (torch.zeros_like(P) for _ in range(3))
+    tok_h, tgt_h = make_batch(cfg)
+    tok, tgt = torch.tensor(tok_h, device=dev), torch.tensor(tgt_h, device=dev)
+    loss = torch.zeros(1, device=dev)
+    N = cfg["batch"] * cfg["ctx"]
+    torch.cuda.synchronize()
+    t = 0
+    for _ in range(warmup):
+        t += 1
+        model.step(P, G, Mo, Vo, t, tok, tgt, cfg["lr"], cfg["wd"], loss)
+    assert model.status() == 0, name
+    launches = model.last_launch_count()
+    clocks = Clocks(local_rank)
+    torch.cuda.synchronize()
+    clocks.start()
+    clocks.wait_first()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for k in range(steps):
+        t += 1
+        model.step(P, G, Mo, Vo, t, tok, tgt, cfg["lr"], cfg["wd"], loss)
+        ev[k + 1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert model.status() == 0, name
+    ms = ev[0].elapsed_time(ev[-1]) / steps
+    per_step = sorted(ev[k].elapsed_time(ev[k + 1]) for k in range(steps))
+    roof = step_roofline(cfg, pk, ms)
+    out = {"workload": cfg["name"], "ms_per_step": ms, "value": N / (ms / 1e3),
+           "unit": "tokens/s", "dtype": "bf16" if cfg["compute"] == "bf16" else "f32",
+           "tokens_per_step": N, "frac_of_roofline": roof["frac_of_roofline"],
+           "step_roofline": roof, "median_ms": per_step[len(per_step) // 2],
+           "best_ms": per_step[0], "gpu_launches": launches * steps,
+           "loss": float(loss.item()), "clocks": clk,
+           "l2": "inputs larger than L2 (saved activations of the step); no flush"}
+    model.close()
+    del P, G, Mo, Vo, model
+    torch.cuda.empty_cache()
     return out
 
 

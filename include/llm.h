@@ -173,10 +173,42 @@ int llm_adamw(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *
  * d_params, d_grads, d_m and d_v each point at the range's first element
  * (16-byte aligned); d_grads *= grad_scale, then AdamW with the context's
  * betas and eps, skipped on the error word like llm_adamw.  No clipping (the
- * global norm needs the whole gradient).  LLM_ERR_ARG for misaligned
+ * global norm needs the whole gradient: llm_adamw_range_clip below).  LLM_ERR_ARG for misaligned
  * pointers, count < 0, t < 1 or a non-finite grad_scale. */
 int llm_adamw_range(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d_v,
                     int64_t count, int64_t t, float lr, float wd, float grad_scale);
+
+/* Clipping for the sharded optimiser, where no rank holds the whole gradient
+ * (MicroGPT in Rust, "Gradient Clipping"; Transformer-In-Rust, "Gradient
+ * Clipping -- By global norm": the threshold applies to the norm of every
+ * gradient element together).  Per step, on each rank:
+ *   llm_grad_norm_part: d_grads[0, count) *= grad_scale in place (1/ranks, as
+ *     llm_adamw_range's grad_scale), then the range's part of the norm is
+ *     written to d_part (one float64 on the device, 8-byte aligned; with
+ *     accumulate = 1 combined with the value already there): the sum of
+ *     squares, in float64 and a fixed order, for the L2 norm, or the largest
+ *     |g| for the L-infinity norm (llm_set_grad_clip_mode).  A rank whose
+ *     share is several ranges calls it once per range, accumulating.
+ *   the caller combines the ranks' parts: all-reduce SUM (L2) or MAX
+ *     (L-infinity) of the float64;
+ *   llm_adamw_range_clip: from the combined part d_total the norm (its square
+ *     root for L2) and the scale of llm_set_grad_clip's rule (threshold /
+ *     norm when the norm exceeds the threshold, else 1; a NaN norm gives 1),
+ *     d_grads[0, count) *= scale, then AdamW over the range as
+ *     llm_adamw_range does with grad_scale 1 (skipped on the error word).
+ *     The norm is what llm_read_grad_norm returns afterwards.  With clipping
+ *     off (threshold 0) d_total is not read (may be NULL) and nothing is
+ *     clipped.  A rank with several ranges calls it once per range with the
+ *     same d_total.
+ * Every rank then applies the same scale, the one the whole-gradient
+ * clipping of llm_adamw would apply to the same summed gradient (equal up to
+ * the order of the float64 sum).  LLM_ERR_ARG for null or misaligned
+ * buffers, count < 0, t < 1, accumulate not 0 or 1 or a non-finite
+ * grad_scale. */
+int llm_grad_norm_part(llm_ctx *ctx, float *d_grads, int64_t count, float grad_scale,
+                       int accumulate, double *d_part);
+int llm_adamw_range_clip(llm_ctx *ctx, float *d_params, float *d_grads, float *d_m, float *d_v,
+                         int64_t count, int64_t t, float lr, float wd, const double *d_total);
 int llm_flag_out(llm_ctx *ctx, int32_t *d_flag);
 int llm_flag_in(llm_ctx *ctx, const int32_t *d_flag);
 

@@ -79,7 +79,7 @@ int llm_kernel_embed_bwd(const int32_t *d_tokens, const float *d_dx, float *d_dw
  * The source pages have no counterpart of this call; it exists for such
  * callers.  Same arguments, layout and result as llm_kernel_embed_bwd(),
  * without the scratch arguments: the scratch is one library-owned device
- * array of 1.5 MiB (393,281 int32) on every GPU that loads the library, kept
+ * array of 1.5 MiB (394,307 int32) on every GPU that loads the library, kept
  * until the process exits.  Limits: n_tokens <= 65536 and vocab <= 65536,
  * else LLM_ERR_ARG with nothing launched.  The call allocates nothing (no
  * cudaMalloc, cudaFree or allocating library routine).  Its first call on a

@@ -66,6 +66,8 @@ EXPORTS = {
     "llm_grad": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "llm_adamw": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _f, _f, _f]),
     "llm_adamw_range": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _f, _f, _f]),
+    "llm_grad_norm_part": (_i, [_vp, _vp, _i64, _f, _i, _vp]),
+    "llm_adamw_range_clip": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _f, _f, _vp]),
     "llm_flag_out": (_i, [_vp, _vp]),
     "llm_flag_in": (_i, [_vp, _vp]),
     "llm_grad_bucket_range": (_i, [_cfgp, _i, C.POINTER(_i64), C.POINTER(_i64)]),

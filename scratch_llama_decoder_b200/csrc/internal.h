@@ -101,6 +101,16 @@ void clip_grads_inf(float *g, int64_t n, float max_norm, double *part, double *n
 void scale_grads(float *g, int64_t n, float sc, cudaStream_t s);
 void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm, float *scale,
                 cudaStream_t s);
+// The norm of a gradient spread over ranks: g [n] *= sc in place, then the
+// range's part -- sum of squares (L2) or largest |g| (linf), float64 -- is
+// written to *out, or with accumulate added to it (L2) or maxed into it.
+// part: clip_part_blocks() doubles of scratch.
+void grad_norm_part(float *g, int64_t n, float sc, int linf, int accumulate, double *part,
+                    double *out, cudaStream_t s);
+// From the ranks' combined part *total: *norm (sqrt of it for L2), *scale
+// (max_norm / norm when norm > max_norm, else 1), then g [n] *= scale.
+void clip_from_total(float *g, int64_t n, const double *total, int linf, float max_norm,
+                     double *norm, float *scale, cudaStream_t s);
 // Dropout of [n] row-major elements of a site (element index = position):
 //   drop_rows: x *= f in place;  drop_add: out = x + f y;
 //   drop_to_act: out (operand type) = f dx.

@@ -860,11 +860,17 @@ void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp,
 }
 
 // ------------------------------------------------------- embedding backward
-// dwte[v,:] = sum_{i : tok_i = v} dx[i,:], summed in increasing i, so the
-// result does not depend on scheduling.  The token ids are sorted stably
+// dwte[v,:] = sum_{i : tok_i = v} dx[i,:] in a fixed order, so the result
+// does not depend on scheduling.  The token ids are sorted stably
 // (least-significant-digit radix sort, 8-bit digits) together with their
-// positions; then one block per vocabulary row adds its rows in order.
+// positions, giving each vocabulary row its run of positions in increasing
+// order.  A run of at most EMB_LONG rows is summed in that order; a longer run
+// (the frequent ids: Zipf puts thousands of rows on id 0) is cut into
+// EMB_PARTS contiguous parts (part k = rows [c k / P, c (k + 1) / P) of its c
+// rows), each part summed in order from zero, and the part sums are added in
+// part order -- a fixed order with a dependent-load chain P times shorter.
 constexpr int RADIX_BLOCK = 256;
+constexpr int EMB_LONG = 64, EMB_PARTS = 8;
 
 __global__ void k_radix_hist(const int32_t *__restrict__ keys, int64_t N, int shift,
                              int32_t *__restrict__ hist, int nblk) {
@@ -931,13 +937,39 @@ __global__ void k_clamp_keys(const int32_t *__restrict__ tok, int32_t *__restric
   keys[i] = t;
   atomicAdd(&counts[t], 1);
 }
-// One block per (vocabulary row, 256 columns); each thread owns 4 columns
-// (one float4) and adds the rows of its bucket in position order, loading 8
-// rows ahead so a long bucket (the Zipf head) is not latency-bound.
+// The vocabulary rows whose run is longer than EMB_LONG, listed in any order
+// (each is summed the same way wherever it is listed).
+__global__ void k_long_runs(const int32_t *__restrict__ offs, int V, int32_t *__restrict__ list,
+                            int32_t *__restrict__ count) {
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v < V && offs[v + 1] - offs[v] > EMB_LONG) list[atomicAdd(count, 1)] = v;
+}
+// Rows [p, e) of a run, in order, into s: lane = 4 columns (float4 c4), with
+// the next 16 rows' loads in flight.
+LLM_DEV float4 run_sum4(const int32_t *__restrict__ order, const float *__restrict__ dx, int d,
+                        int c4, bool on, int p, int e) {
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (; p + 16 <= e; p += 16) {
+    float4 t[16];
+#pragma unroll
+    for (int u = 0; u < 16; u++)
+      t[u] = on ? reinterpret_cast<const float4 *>(dx + (int64_t)order[p + u] * d)[c4]
+                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 16; u++) {
+      s.x += t[u].x; s.y += t[u].y; s.z += t[u].z; s.w += t[u].w;
+    }
+  }
+  for (; p < e; p++) {
+    if (!on) continue;
+    const float4 t = reinterpret_cast<const float4 *>(dx + (int64_t)order[p] * d)[c4];
+    s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+  }
+  return s;
+}
 // Warp items (vocabulary row v, 128-column chunk), taken in order of v by a
-// grid of whole blocks (the Zipf head -- the longest runs -- starts first);
-// lane = 4 columns.  Each lane adds its run's rows strictly in position
-// order, with the next 16 rows' loads in flight.
+// grid of whole blocks; lane = 4 columns.  Runs of at most EMB_LONG rows
+// (and absent ids: zero rows); longer runs are left to k_embed_long.
 __global__ void __launch_bounds__(256) k_embed_rows(const int32_t *__restrict__ order,
                                                    const int32_t *__restrict__ offs,
                                                    const float *__restrict__ dx,
@@ -952,49 +984,68 @@ __global__ void __launch_bounds__(256) k_embed_rows(const int32_t *__restrict__ 
     const int c4 = ch * 32 + lane;  // float4 column index
     const bool on = 4 * c4 < d;
     const int b = offs[v], e = offs[v + 1];
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    int p = b;
-    for (; p + 16 <= e; p += 16) {
-      float4 t[16];
-#pragma unroll
-      for (int u = 0; u < 16; u++)
-        t[u] = on ? reinterpret_cast<const float4 *>(dx + (int64_t)order[p + u] * d)[c4]
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 16; u++) {
-        s.x += t[u].x; s.y += t[u].y; s.z += t[u].z; s.w += t[u].w;
-      }
-    }
-    for (; p < e; p++) {
-      if (!on) continue;
-      const float4 t = reinterpret_cast<const float4 *>(dx + (int64_t)order[p] * d)[c4];
-      s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
-    }
+    if (e - b > EMB_LONG) continue;
+    const float4 s = run_sum4(order, dx, d, c4, on, b, e);
     if (on) reinterpret_cast<float4 *>(dwte + (int64_t)v * d)[c4] = s;
   }
 }
-// Same sums for any d or alignment (one thread per column, rows in order).
+// Block (listed long run, 128-column chunk): warp k sums part k of the run,
+// warp 0 adds the part sums in part order.
+__global__ void __launch_bounds__(32 * EMB_PARTS)
+    k_embed_long(const int32_t *__restrict__ list, const int32_t *__restrict__ count,
+                 const int32_t *__restrict__ order, const int32_t *__restrict__ offs,
+                 const float *__restrict__ dx, float *__restrict__ dwte, int d) {
+  __shared__ float4 part[EMB_PARTS][32];
+  if ((int)blockIdx.x >= *count) return;
+  const int v = list[blockIdx.x];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int c4 = blockIdx.y * 32 + lane;
+  const bool on = 4 * c4 < d;
+  const int b = offs[v];
+  const int64_t c = offs[v + 1] - b;
+  const int p0 = b + (int)(c * warp / EMB_PARTS), p1 = b + (int)(c * (warp + 1) / EMB_PARTS);
+  part[warp][lane] = run_sum4(order, dx, d, c4, on, p0, p1);
+  __syncthreads();
+  if (warp == 0 && on) {
+    float4 t = part[0][lane];
+#pragma unroll
+    for (int k = 1; k < EMB_PARTS; k++) {
+      const float4 q = part[k][lane];
+      t.x += q.x; t.y += q.y; t.z += q.z; t.w += q.w;
+    }
+    reinterpret_cast<float4 *>(dwte + (int64_t)v * d)[c4] = t;
+  }
+}
+// Same sums and order for any d or alignment (one thread per column).
 __global__ void k_embed_rows_scalar(const int32_t *__restrict__ order,
                                     const int32_t *__restrict__ offs, const float *__restrict__ dx,
                                     float *__restrict__ dwte, int d) {
   const int v = blockIdx.x;
   const int b = offs[v], e = offs[v + 1];
+  const int64_t c = e - b;
+  const int np = c > EMB_LONG ? EMB_PARTS : 1;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float sum = 0.f;
-    for (int p = b; p < e; p++) sum += dx[(int64_t)order[p] * d + j];
-    dwte[(int64_t)v * d + j] = sum;
+    float total = 0.f;
+    for (int k = 0; k < np; k++) {
+      float sum = 0.f;
+      for (int p = b + (int)(c * k / np); p < b + (int)(c * (k + 1) / np); p++)
+        sum += dx[(int64_t)order[p] * d + j];
+      total = k == 0 ? sum : total + sum;
+    }
+    dwte[(int64_t)v * d + j] = total;
   }
 }
 int64_t embed_bwd_scratch_ints(int64_t N, int V) {
   int64_t nblk = (N + RADIX_BLOCK - 1) / RADIX_BLOCK;
-  return 4 * N + 256 * nblk + (V + 1) + 64;
+  return 4 * N + 256 * nblk + (V + 1) + 1 + (N / EMB_LONG + 1) + 64;
 }
 void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int d, int V,
                int32_t *scratch, cudaStream_t s) {
   int nblk = (int)cdiv(N, RADIX_BLOCK);
   int32_t *k0 = scratch, *v0 = k0 + N, *k1 = v0 + N, *v1 = k1 + N;
   int32_t *hist = v1 + N, *offs = hist + 256 * (int64_t)nblk;
-  cudaMemsetAsync(offs, 0, sizeof(int32_t) * (V + 1), s);
+  int32_t *nlong = offs + V + 1, *list = nlong + 1;  // long runs: count, then vocabulary ids
+  cudaMemsetAsync(offs, 0, sizeof(int32_t) * (V + 2), s);  // counts and the long-run count
   k_clamp_keys<<<cdiv(N, 256), 256, 0, s>>>(tok, k0, offs, N, V);
   count_launch();
   int bits = 1;
@@ -1014,12 +1065,19 @@ void embed_bwd(const int32_t *tok, const float *dx, float *dwte, int64_t N, int 
     vin = nv;
   }
   k_scan_excl<<<1, 1024, 0, s>>>(offs, V + 1);
-  if ((d & 3) == 0 && ((uintptr_t)dx & 15) == 0 && ((uintptr_t)dwte & 15) == 0)
+  count_launch();
+  if ((d & 3) == 0 && ((uintptr_t)dx & 15) == 0 && ((uintptr_t)dwte & 15) == 0) {
+    k_long_runs<<<cdiv(V, 256), 256, 0, s>>>(offs, V, list, nlong);
     k_embed_rows<<<(unsigned)std::min<int64_t>(((int64_t)V * cdiv(d, 128) + 7) / 8, 148 * 8), 256,
                    0, s>>>(vin, offs, dx, dwte, d, V);
-  else
+    const int64_t slots = std::max<int64_t>(1, N / EMB_LONG);  // at most N / EMB_LONG long runs
+    k_embed_long<<<dim3((unsigned)slots, cdiv(d, 128)), 32 * EMB_PARTS, 0, s>>>(
+        list, nlong, vin, offs, dx, dwte, d);
+    count_launch(3);
+  } else {
     k_embed_rows_scalar<<<V, min(256, ((d + 31) / 32) * 32), 0, s>>>(vin, offs, dx, dwte, d);
-  count_launch(2);
+    count_launch();
+  }
 }
 
 // ------------------------------------------------------------ initialisation
@@ -1217,6 +1275,56 @@ void clip_grads(float *g, int64_t n, float max_norm, double *part, double *norm,
   k_clip_scale<<<1, CLIP_THREADS, 0, s>>>(part, CLIP_BLOCKS, max_norm, norm, scale);
   k_scale_grads<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, scale);
   count_launch(3);
+}
+
+// Clipping with the gradient spread over ranks (sharded optimiser): each rank
+// reduces its own range to one double -- the sum of squares (L2) or the
+// largest |g| (L-infinity) -- the ranks combine those (sum or max), and every
+// rank derives the same norm and scale from the combined value.
+__global__ void __launch_bounds__(CLIP_THREADS)
+    k_part_total(const double *__restrict__ part, int nblk, int accumulate, double *out) {
+  __shared__ double ws[CLIP_THREADS / 32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nblk; i += CLIP_THREADS) acc += part[i];
+  const double s = block_sum_d(acc, ws);
+  if (threadIdx.x == 0) *out = accumulate ? *out + s : s;
+}
+__global__ void k_part_max(const float *__restrict__ part, int nblk, int accumulate, double *out) {
+  if (threadIdx.x != 0) return;
+  float m = 0.f;
+  for (int i = 0; i < nblk; i++) m = nan_max(m, part[i]);
+  const double dm = (double)m;
+  if (!accumulate) *out = dm;
+  else {
+    const double o = *out;  // NaN wins, as in nan_max
+    *out = o != o ? o : ((dm != dm || dm > o) ? dm : o);
+  }
+}
+void grad_norm_part(float *g, int64_t n, float sc, int linf, int accumulate, double *part,
+                    double *out, cudaStream_t s) {
+  if (sc != 1.0f) scale_grads(g, n, sc, s);
+  if (linf) {
+    float *fpart = reinterpret_cast<float *>(part);
+    k_absmax<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, fpart);
+    k_part_max<<<1, 32, 0, s>>>(fpart, CLIP_BLOCKS, accumulate, out);
+  } else {
+    k_sumsq<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, part);
+    k_part_total<<<1, CLIP_THREADS, 0, s>>>(part, CLIP_BLOCKS, accumulate, out);
+  }
+  count_launch(2);
+}
+__global__ void k_clip_from_total(const double *__restrict__ total, int linf, float max_norm,
+                                  double *__restrict__ norm, float *__restrict__ scale) {
+  if (threadIdx.x != 0) return;
+  const double nm = linf ? *total : sqrt(*total);
+  *norm = nm;
+  *scale = nm > (double)max_norm ? (float)((double)max_norm / nm) : 1.0f;
+}
+void clip_from_total(float *g, int64_t n, const double *total, int linf, float max_norm,
+                     double *norm, float *scale, cudaStream_t s) {
+  k_clip_from_total<<<1, 32, 0, s>>>(total, linf, max_norm, norm, scale);
+  k_scale_grads<<<CLIP_BLOCKS, CLIP_THREADS, 0, s>>>(g, n, scale);
+  count_launch(2);
 }
 
 // -------------------------------------------------------------------- flags

@@ -1136,6 +1136,42 @@ int llm_adamw_range(llm_ctx *c, float *d_params, float *d_grads, float *d_m, flo
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
 
+int llm_grad_norm_part(llm_ctx *c, float *d_grads, int64_t count, float grad_scale,
+                       int accumulate, double *d_part) {
+  if (!c || count < 0 || !std::isfinite(grad_scale) || (accumulate != 0 && accumulate != 1))
+    return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
+  if (!aligned16(d_grads) || !d_part || ((uintptr_t)d_part & 7)) return LLM_ERR_ARG;
+  g_launches = 0;
+  grad_norm_part(d_grads, count, grad_scale, c->clip_mode == LLM_CLIP_LINF ? 1 : 0, accumulate,
+                 c->clip_part, d_part, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+int llm_adamw_range_clip(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v,
+                         int64_t count, int64_t t, float lr, float wd, const double *d_total) {
+  if (!c || t < 1 || count < 0) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
+  if (!aligned16(d_params) || !aligned16(d_grads) || !aligned16(d_m) || !aligned16(d_v))
+    return LLM_ERR_ARG;
+  if (c->clip > 0.f && (!d_total || ((uintptr_t)d_total & 7))) return LLM_ERR_ARG;
+  g_launches = 0;
+  const double bc1 = 1.0 - pow((double)c->cfg.beta1, (double)t);
+  const double bc2 = 1.0 - pow((double)c->cfg.beta2, (double)t);
+  set_hyper(c->hyper, lr, wd, (float)bc1, (float)bc2, c->s);
+  if (c->clip > 0.f) {
+    clip_from_total(d_grads, count, d_total, c->clip_mode == LLM_CLIP_LINF ? 1 : 0, c->clip,
+                    c->clip_norm, c->clip_scale, c->s);
+    c->have_norm = true;
+  }
+  if (count > 0)
+    adamw(d_params, d_grads, d_m, d_v, count, c->hyper, c->cfg.beta1, c->cfg.beta2,
+          c->cfg.adam_eps, c->flag_step, c->s);
+  c->last_launches = g_launches;
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
 int llm_flag_out(llm_ctx *c, int32_t *d_flag) {
   if (!c || !d_flag) return LLM_ERR_ARG;
   if (!on_device(c)) return LLM_ERR_ARG;

@@ -23,8 +23,10 @@ constexpr int64_t kMaxTokens = 65536;
 constexpr int kMaxVocab = 65536;
 // int32 words the embedding backward needs at the maximum sizes: keys and
 // positions twice (ping-pong of the radix sort), 256 digit counters per
-// 256-token block, vocab+1 row offsets, and slack.
-constexpr int64_t kScratchInts = 4 * kMaxTokens + 256 * (kMaxTokens / 256) + (kMaxVocab + 1) + 64;
+// 256-token block, vocab+1 row offsets, the count and list of the runs longer
+// than 64 rows (at most tokens / 64 of them), and slack.
+constexpr int64_t kScratchInts = 4 * kMaxTokens + 256 * (kMaxTokens / 256) + (kMaxVocab + 1) + 1 +
+                                 (kMaxTokens / 64 + 1) + 64;
 
 static __device__ __align__(256) int32_t g_embed_bwd_scratch[kScratchInts];
 

@@ -105,7 +105,13 @@ class ShardedDataParallelStep(DataParallelStep):
       5. all-gather of the updated chunks into every rank's parameters.
     Per rank that moves a reduce-scatter plus an all-gather of the gradient's
     size (together one all-reduce's traffic) and keeps 1 / ranks of m and v.
-    Clipping is not applied here (its norm needs the whole gradient).
+    With clipping on (the engine's grad_clip > 0), step 4 becomes: each rank
+    scales its chunk by 1 / ranks and reduces it to its part of the norm
+    (llm_grad_norm_part: sum of squares in float64, or the largest |g|), one
+    all-reduce of that float64 (SUM, or MAX for the L-infinity norm) gives
+    every rank the whole gradient's part, and llm_adamw_range_clip clips the
+    chunk by the resulting norm and updates it -- the same scale on every
+    rank, the one llm_adamw applies to the whole summed gradient.
     buffers() allocates the padded parameter and gradient buffers and the
     chunk-sized m and v.
 
@@ -144,6 +150,23 @@ class ShardedDataParallelStep(DataParallelStep):
             self.lo = self.rank * self.chunk
             self.count = max(0, min(self.chunk, self.n - self.lo))
 
+    def _clipping(self):
+        return getattr(self.engine, "grad_clip", 0.0) > 0.0
+
+    def _norm_part(self):
+        """One float64 on the engine's device: this rank's part of the norm."""
+        if getattr(self, "_part", None) is None:
+            self._part = torch.zeros(1, dtype=torch.float64, device=self.engine.device)
+        return self._part
+
+    def _combine(self, part):
+        """Every rank's part of the norm, combined: the sum of the ranks' sums
+        of squares, or the largest of their largest |g|."""
+        if self.world > 1:
+            linf = getattr(self.engine, "grad_clip_mode", 0) == 1
+            dist.all_reduce(part, op=dist.ReduceOp.MAX if linf else dist.ReduceOp.SUM,
+                            group=self.group)
+
     def buffers(self, dtype=torch.float32):
         dev = self.engine.device
         padded = self.padded
@@ -175,11 +198,23 @@ class ShardedDataParallelStep(DataParallelStep):
         dist.all_reduce(self.flag, op=dist.ReduceOp.MAX, group=self.group)
         e.flag_in(self.flag)
         dist.all_reduce(loss, op=dist.ReduceOp.SUM, group=self.group)
+        if self._clipping():
+            part = self._norm_part()
+            part.zero_()
+            for off, q, keep, mo in self.pieces:
+                if keep:
+                    e.grad_norm_part(gs[mo:mo + keep], 1.0 / W, part, accumulate=True)
+                    launches += self._launches()
+            self._combine(part)
         for off, q, keep, mo in self.pieces:
             if keep:
                 a = off + self.rank * q
-                e.adamw_range(params[a:a + keep], gs[mo:mo + keep], m[mo:mo + keep],
-                              v[mo:mo + keep], t, lr, wd, grad_scale=1.0 / W)
+                if self._clipping():
+                    e.adamw_range_clip(params[a:a + keep], gs[mo:mo + keep], m[mo:mo + keep],
+                                       v[mo:mo + keep], t, lr, wd, part)
+                else:
+                    e.adamw_range(params[a:a + keep], gs[mo:mo + keep], m[mo:mo + keep],
+                                  v[mo:mo + keep], t, lr, wd, grad_scale=1.0 / W)
                 launches += self._launches()
         self.last_launches = launches
         nccl = dist.get_backend(self.group) == "nccl"
@@ -210,8 +245,16 @@ class ShardedDataParallelStep(DataParallelStep):
                 gs = self._gshard
             else:
                 gs = grads
-            e.adamw_range(params[lo:lo + cnt], gs[:cnt], m[:cnt], v[:cnt], t, lr, wd,
-                          grad_scale=1.0 / self.world)
+            if self._clipping():
+                part = self._norm_part()
+                e.grad_norm_part(gs[:cnt], 1.0 / self.world, part)
+                launches += self._launches()
+                self._combine(part)
+                e.adamw_range_clip(params[lo:lo + cnt], gs[:cnt], m[:cnt], v[:cnt], t, lr, wd,
+                                   part)
+            else:
+                e.adamw_range(params[lo:lo + cnt], gs[:cnt], m[:cnt], v[:cnt], t, lr, wd,
+                              grad_scale=1.0 / self.world)
             self.last_launches = launches + self._launches()
             if self.world > 1:
                 src = params[lo:lo + C]

@@ -53,6 +53,7 @@ class LlamaStep:
                                      C.c_void_p(self.stream.cuda_stream), C.byref(ctx)),
                     "llm_create")
         self.ctx = ctx
+        self.grad_clip, self.grad_clip_mode = 0.0, 0  # as llm_create leaves them
 
     def close(self):
         if getattr(self, "ctx", None):
@@ -134,6 +135,24 @@ class LlamaStep:
                 "llm_adamw_range")
 
     @_on_device
+    def grad_norm_part(self, grads, grad_scale, part, accumulate=False):
+        """grads (1-D view) *= grad_scale, then its part of the clipping norm
+        into part (one float64 on the device; llm_grad_norm_part)."""
+        L.check(L.lib.llm_grad_norm_part(self.ctx, _ptr(grads), grads.numel(), float(grad_scale),
+                                         int(bool(accumulate)), _ptr(part)),
+                "llm_grad_norm_part")
+
+    @_on_device
+    def adamw_range_clip(self, params, grads, m, v, t, lr, wd, total):
+        """Clip by the ranks' combined norm part total, then AdamW over the
+        elements of 1-D views params, grads, m, v (llm_adamw_range_clip)."""
+        n = params.numel()
+        assert grads.numel() == n and m.numel() == n and v.numel() == n
+        L.check(L.lib.llm_adamw_range_clip(self.ctx, _ptr(params), _ptr(grads), _ptr(m), _ptr(v),
+                                           n, int(t), float(lr), float(wd), _ptr(total)),
+                "llm_adamw_range_clip")
+
+    @_on_device
     def flag_out(self, flag):
         """Copy the step's int32 error word to flag (llm_flag_out)."""
         L.check(L.lib.llm_flag_out(self.ctx, _ptr(flag)), "llm_flag_out")
@@ -203,11 +222,13 @@ class LlamaStep:
     def set_grad_clip(self, max_norm):
         """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
         L.check(L.lib.llm_set_grad_clip(self.ctx, float(max_norm)), "llm_set_grad_clip")
+        self.grad_clip = float(max_norm)
 
     @_on_device
     def set_grad_clip_mode(self, mode):
         """0: global L2 norm (default); 1: L-infinity norm (llm_set_grad_clip_mode)."""
         L.check(L.lib.llm_set_grad_clip_mode(self.ctx, int(mode)), "llm_set_grad_clip_mode")
+        self.grad_clip_mode = int(mode)
 
     @_on_device
     def read_grad_norm(self):

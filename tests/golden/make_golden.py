@@ -11,7 +11,15 @@ stores, in tests/golden/step_<config>.npz:
                              (all of a smaller tensor) with the gradient and the
                              post-AdamW parameter, m and v there
   g_norm                     full L2 norm of each tensor's gradient
-Usage: python tests/golden/make_golden.py c2 [c3 ...]
+and, with --rows, in tests/golden/logit_rows_<config>.npz:
+  rows, vals                 full logit rows (float32) from the first and the
+                             last 128-row block of the [B*T, V] logits (the
+                             first and last output tiles of the lm_head GEMM),
+                             computed by the oracle's forward on the one
+                             sequence each row belongs to (up to the row's
+                             block): by causality (pinned in the oracle's
+                             tests) those rows equal the whole batch's.
+Usage: python tests/golden/make_golden.py [--rows] c2 [c3 ...]
 """
 import os
 import sys
@@ -70,6 +78,41 @@ def golden(name):
     print(f"{cfg['name']}: loss {loss:.6f}  oracle {t1 - t0:.1f}s -> {out}", flush=True)
 
 
+def _block_rows(T, N):
+    """Global row ids: four from the first 128-row block, four from the last."""
+    first = [0, 1, 64, 127]
+    last = [N - 128, N - 65, N - 2, N - 1]
+    return [r for r in first + last if 0 <= r < N]
+
+
+def logit_rows(name):
+    cfg = get_config(name)
+    tok, _ = make_batch(cfg)
+    B, T = tok.shape
+    p = make_params(cfg, O.param_layout(cfg)).astype(np.float64)
+    rows = _block_rows(T, B * T)
+    vals = np.zeros((len(rows), cfg["vocab"]), np.float32)
+    t0 = time.time()
+    for b in sorted({r // T for r in rows}):
+        mine = [k for k, r in enumerate(rows) if r // T == b]
+        upto = max(rows[k] % T for k in mine) + 1  # positions after the last row are not needed
+        sub = dict(cfg, batch=1, ctx=upto)
+        _, z, _ = O.forward_backward(sub, p, np.ascontiguousarray(tok[b:b + 1, :upto]),
+                                     want_grads=False)
+        for k in mine:
+            vals[k] = z[rows[k] % T]
+    out = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                       f"logit_rows_{cfg['name']}.npz")
+    np.savez_compressed(out, rows=np.array(rows, np.int64), vals=vals,
+                        oracle_seconds=np.float64(time.time() - t0))
+    print(f"{cfg['name']}: {len(rows)} logit rows in {time.time() - t0:.1f}s -> {out}", flush=True)
+
+
 if __name__ == "__main__":
-    for nm in sys.argv[1:]:
-        golden(nm)
+    args = sys.argv[1:]
+    if args and args[0] == "--rows":
+        for nm in args[1:]:
+            logit_rows(nm)
+    else:
+        for nm in args:
+            golden(nm)

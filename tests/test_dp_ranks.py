@@ -22,11 +22,48 @@ class OracleEngine:
     on float64 CPU tensors."""
     device = torch.device("cpu")
 
-    def __init__(self, cfg, fail_at=None):
+    def __init__(self, cfg, fail_at=None, clip=0.0, clip_mode=0):
         self.cfg = cfg
         self.flag = 0
         self.fail_at = fail_at
         self.calls = 0
+        self.grad_clip, self.grad_clip_mode = float(clip), int(clip_mode)
+        self.norms = []  # the norm before clipping of every clipped update
+
+    def _kind(self):
+        return "linf" if self.grad_clip_mode == 1 else "l2"
+
+    def _clip_whole(self, grads):
+        from oracle import train_terms as TT
+        if self.grad_clip > 0.0:
+            g, n, _ = TT.clip(grads.numpy(), self.grad_clip, self._kind())
+            grads.copy_(torch.from_numpy(g))
+            self.norms.append(n)
+
+    # the sharded form's clipping: a part of the norm per range, combined by
+    # the caller across ranks, then the clipping rule on the combined value
+    def grad_norm_part(self, grads, grad_scale, part, accumulate=False):
+        grads.mul_(grad_scale)
+        g = grads.numpy()
+        if self.grad_clip_mode == 1:
+            v = float(np.max(np.abs(g))) if g.size else 0.0
+            part.fill_(max(float(part.item()), v) if accumulate else v)
+        else:
+            v = float(np.sum(g * g))
+            part.fill_(float(part.item()) + v if accumulate else v)
+
+    def adamw_range_clip(self, params, grads, m, v, t, lr, wd, total):
+        from oracle import train_terms as TT
+        if self.grad_clip > 0.0:
+            tv = float(total.item())
+            n = tv if self.grad_clip_mode == 1 else float(np.sqrt(tv))
+            grads.mul_(TT.clip_scale(n, self.grad_clip))
+            if getattr(self, "_norm_t", None) != t:  # one norm per step, however many ranges
+                self.norms.append(n)
+                self._norm_t = t
+            else:
+                assert n == self.norms[-1]  # every range of a step sees the same norm
+        self.adamw_range(params, grads, m, v, t, lr, wd)
 
     def grad(self, params, grads, tokens, targets, loss):
         import oracle as O
@@ -69,6 +106,7 @@ class OracleEngine:
     def adamw(self, params, grads, m, v, t, lr, wd, grad_scale=1.0):
         import oracle as O
         grads.mul_(grad_scale)
+        self._clip_whole(grads)
         if self.flag:
             return
         p2, m2, v2 = O.adamw(params.numpy(), grads.numpy(), m.numpy(), v.numpy(), t, lr, wd)
@@ -102,7 +140,8 @@ def _run(engine, dp, p, tok, tgt, steps, lr, wd):
     return P.numpy(), M.numpy(), V.numpy(), losses
 
 
-def _rank_main_sharded(rank, world, port, full_cfg, steps, q, overlap=False):
+def _rank_main_sharded(rank, world, port, full_cfg, steps, q, overlap=False, clip=0.0,
+                       clip_mode=0):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -116,7 +155,7 @@ def _rank_main_sharded(rank, world, port, full_cfg, steps, q, overlap=False):
         p, tok, tgt = _setup(full_cfg)
         share = full_cfg["batch"] // world
         cfg = dict(full_cfg, batch=share)
-        eng = OracleEngine(cfg)
+        eng = OracleEngine(cfg, clip=clip, clip_mode=clip_mode)
         dp = ShardedDataParallelStep(eng, O.n_params(cfg), overlap=overlap)
         assert dp.overlap == overlap
         P, G, M, V = dp.buffers(torch.float64)
@@ -132,10 +171,10 @@ def _rank_main_sharded(rank, world, port, full_cfg, steps, q, overlap=False):
                 a = off + rank * qq
                 Mf[a:a + keep] = M[mo:mo + keep].numpy()
                 Vf[a:a + keep] = V[mo:mo + keep].numpy()
-            q.put((rank, (P[:p.size].numpy().copy(), Mf, Vf, None, None)))
+            q.put((rank, (P[:p.size].numpy().copy(), Mf, Vf, None, None, eng.norms)))
         else:
             q.put((rank, (P[:p.size].numpy().copy(), M[:dp.count].numpy().copy(),
-                          V[:dp.count].numpy().copy(), dp.lo, dp.count)))
+                          V[:dp.count].numpy().copy(), dp.lo, dp.count, eng.norms)))
     finally:
         dist.destroy_process_group()
 
@@ -232,7 +271,7 @@ def test_sharded_optimiser_two_ranks_equal_one_process():
     eng = OracleEngine(full)
     ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 3, full["lr"], full["wd"])
     for r in (0, 1):
-        P, Mc, Vc, lo, cnt = res[r]
+        P, Mc, Vc, lo, cnt, _ = res[r]
         np.testing.assert_allclose(P, ref[0], rtol=1e-12, atol=1e-15)
         np.testing.assert_allclose(Mc, ref[1][lo:lo + cnt], rtol=1e-10, atol=1e-18)
         np.testing.assert_allclose(Vc, ref[2][lo:lo + cnt], rtol=1e-10, atol=1e-22)
@@ -317,3 +356,67 @@ def test_bucketed_sharded_optimiser_equals_one_process(world):
     assert not np.any(np.isnan(Mf))
     np.testing.assert_allclose(Mf, ref[1], rtol=1e-10, atol=1e-18)
     np.testing.assert_allclose(Vf, ref[2], rtol=1e-10, atol=1e-22)
+
+
+def _sharded_ranks(full, world, steps, overlap, clip, clip_mode):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_sharded,
+                         args=(r, world, port, full, steps, q, overlap, clip, clip_mode))
+             for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=300) for _ in range(world))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    return res
+
+
+@pytest.mark.parametrize("world,overlap,clip_mode", [(2, False, 0), (3, True, 0), (2, True, 1),
+                                                     (3, False, 1)],
+                         ids=["2ranks-whole-l2", "3ranks-buckets-l2", "2ranks-buckets-linf",
+                              "3ranks-whole-linf"])
+def test_sharded_optimiser_clips_like_the_whole_gradient(world, overlap, clip_mode):
+    """Clipping in the sharded forms (MicroGPT in Rust, Gradient Clipping;
+    Transformer-In-Rust: by global norm; randyGPT: the L-infinity form): each
+    rank's part of the norm, combined across ranks, gives the norm of the
+    whole summed gradient, so the ranks clip as the one-process oracle step
+    with the same threshold does.  The threshold sits below the norm of every
+    step (checked), so every step is clipped."""
+    from synth import get_config
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    full = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_head=2, d_ff=42,
+                      ctx=5, batch=world, init_std=0.3, name="gqa-small", index=9)
+    clip = 0.05 if clip_mode == 1 else 0.5
+    res = _sharded_ranks(full, world, 3, overlap, clip, clip_mode)
+    p, tok, tgt = _setup(full)
+    eng = OracleEngine(full, clip=clip, clip_mode=clip_mode)
+    ref = _run(eng, DataParallelStep(eng), p, tok, tgt, 3, full["lr"], full["wd"])
+    assert len(eng.norms) == 3 and min(eng.norms) > clip  # every step clipped
+    for r in range(world):
+        P, Mr, Vr = res[r][0], res[r][1], res[r][2]
+        np.testing.assert_array_equal(P, res[0][0])  # the ranks agree bit for bit
+        np.testing.assert_allclose(P, ref[0], rtol=1e-12, atol=1e-15)
+        if overlap:
+            have = ~np.isnan(Mr)
+            np.testing.assert_allclose(Mr[have], ref[1][have], rtol=1e-10, atol=1e-18)
+            np.testing.assert_allclose(Vr[have], ref[2][have], rtol=1e-10, atol=1e-22)
+        else:
+            lo, cnt = res[r][3], res[r][4]
+            np.testing.assert_allclose(Mr, ref[1][lo:lo + cnt], rtol=1e-10, atol=1e-18)
+            np.testing.assert_allclose(Vr, ref[2][lo:lo + cnt], rtol=1e-10, atol=1e-22)
+        # every rank saw the whole gradient's norm
+        np.testing.assert_allclose(res[r][5], eng.norms, rtol=1e-12)
+
+
+def test_sharded_clipping_with_an_unclipping_threshold_is_the_unclipped_step():
+    """A threshold above every norm leaves the sharded step unchanged."""
+    from synth import get_config
+    full = get_config("c1", vocab=11, d_model=16, n_layer=2, n_head=4, n_kv_head=2, d_ff=42,
+                      ctx=5, batch=2, init_std=0.3, name="gqa-small", index=9)
+    clipped = _sharded_ranks(full, 2, 2, False, 1e9, 0)
+    plain = _sharded_ranks(full, 2, 2, False, 0.0, 0)
+    for r in (0, 1):
+        np.testing.assert_allclose(clipped[r][0], plain[r][0], rtol=1e-15, atol=0)

@@ -6,10 +6,9 @@ all device memory).  Its scratch is a library-owned device array, so this
 test checks it against the scratch-taking entry point llm_kernel_embed_bwd
 on the same inputs, on two calls in a row with different sizes (the second
 call must not see the first call's leftovers), and that sizes beyond its
-limits are refused on the host.  This file is collected after the step,
-kernel and decode parity tests and before the tests of the entry points built
-on the step; it also passes alone in a fresh process, where its first call
-does the per-device set-up.
+limits are refused on the host.  This file is collected after every other
+test file; it also passes alone in a fresh process, where its first call does
+the per-device set-up.
 """
 import ctypes as C
 
