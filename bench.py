@@ -463,6 +463,7 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.steps):
         t += 1
         train_step(t)
+    classes = model.read_kernel_class_timing()
     g_ms, g_flops, g_launch = model.read_kernel_timing()
     model.set_kernel_timing(False)
     # clocks sampled over the timed region and the GEMM-timing pass after it
@@ -534,6 +535,7 @@ def run_ours(args, rank, world, local_rank):
                      "launches": g_launch, "ms_total": g_ms,
                      "peak_source": f"{src} bf16_tflops_sustained"},
         "step_roofline": step_roofline(cfg, pk, step_s * 1e3),
+        "kernels": kernel_rates(classes, args.steps, pk, src),
         "gpu_launches": launches_per_step * args.steps,
         # this rank's steps (rank 0): median and best step, as tokens/s per GPU
         "per_step": {"median_ms": per_step[len(per_step) // 2], "best_ms": per_step[0],
@@ -561,6 +563,32 @@ def run_ours(args, rank, world, local_rank):
             "sample": f"float64 oracle: forward+backward of a {S}-token prefix of one "
                       f"sequence plus AdamW over {S}/{N} of the parameters "
                       f"({tsec:.1f} s), scaled to tokens/s"}
+    return out
+
+
+def kernel_rates(classes, steps, pk, src):
+    """Per kernel class: device time per step (CUDA events around every
+    launch, individual launches on one stream), algorithmic work per step and
+    the rate against the class's bound (TFLOP/s against the sustained bf16
+    peak for the contractions, GB/s against the measured copy bandwidth for
+    the memory-bound passes)."""
+    from scratch_llama_decoder_b200._lib import KERNEL_CLASSES
+    peak_tc = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    out = {}
+    for name, unit in KERNEL_CLASSES:
+        ms, work, n = classes.get(name, (0.0, 0.0, 0))
+        if n == 0 or ms <= 0:
+            continue
+        if unit == "flop":
+            rate, peak, u = work / (ms / 1e3) / 1e12, peak_tc, "TFLOP/s"
+            ps = f"{src} bf16_tflops_sustained"
+        else:
+            rate, peak, u = work / (ms / 1e3) / 1e9, pk["hbm_gbs"], "GB/s"
+            ps = f"{src} hbm_gbs"
+        out[name] = {"ms_per_step": ms / steps, "launches_per_step": n / steps,
+                     "work_per_step": work / steps, "work_unit": unit, "achieved": rate,
+                     "peak": peak, "unit": u, "frac": rate / peak if peak else None,
+                     "peak_source": ps}
     return out
 
 

@@ -432,16 +432,48 @@ int llm_last_launch_count(const llm_ctx *ctx);
 int llm_set_graphs(llm_ctx *ctx, int enable);
 
 /* Measurement hooks (strata, bench harness: time what is claimed).  With
- * timing enabled, every tensor-core GEMM launch of later calls is bracketed
- * by CUDA events on the context's stream.  llm_read_kernel_timing()
- * synchronises that stream and returns, since the previous read, the summed
- * device time of those launches in milliseconds, their algorithmic FLOPs
- * (2*M*N*K with unpadded sizes) and their count, then resets the sums.
- * Events are created on demand (two per pending launch) and kept until
+ * timing enabled, the launches of later llm_step calls are bracketed by CUDA
+ * events on the context's stream, per kernel class, and each bracket is
+ * credited with its algorithmic work: FLOPs for the contractions (GEMM:
+ * 2*M*N*K with unpadded sizes; attention: the causal T(T+1)/2 (query, key)
+ * pairs per (sequence, head) times 4 hd FLOPs forward, 8 hd backward), bytes
+ * for the memory-bound passes (what the pass must read and write once:
+ * RMSNorm forward 4 + ab bytes per element plus the rstd, backward the float32
+ * input, upstream gradient, residual gradient (when added) and output plus
+ * the activation-type copy; SwiGLU a, b, u (forward) and a, b, du, da, db
+ * (backward) at ab bytes; cross-entropy the logits read and written once;
+ * embedding gather 8 bytes per element read and written; embedding scatter
+ * the upstream rows and the whole table; AdamW 28 bytes per parameter; the
+ * weight copies 4 + ab bytes per weight; the split-K finish its partials and
+ * outputs).  ab = bytes of an activation element (2 bf16, 4 fp32).
+ * llm_read_kernel_class_timing() synchronises the stream and returns, for
+ * class cls (LLM_KT_*), the summed device time in milliseconds, the credited
+ * work and the number of brackets since the last reset;
+ * llm_read_kernel_timing() does the same for LLM_KT_GEMM, then resets every
+ * class.  Events are created on demand (two per bracket) and kept until
  * llm_destroy(); reading after every few steps bounds their number.  Steps
- * run as individual launches while timing is on (no step graph). */
+ * run as individual launches on the one stream while timing is on (no step
+ * graph, no side stream).  LLM_ERR_ARG for a class out of range. */
+enum {
+  LLM_KT_GEMM = 0,           /* tcgen05 projection GEMMs (FLOPs) */
+  LLM_KT_ATTN_FWD = 1,       /* attention forward (FLOPs) */
+  LLM_KT_ATTN_BWD = 2,       /* attention backward (FLOPs) */
+  LLM_KT_RMSNORM_FWD = 3,    /* bytes from here on */
+  LLM_KT_RMSNORM_BWD = 4,    /* with the gain-gradient reduction */
+  LLM_KT_SWIGLU_FWD = 5,
+  LLM_KT_SWIGLU_BWD = 6,
+  LLM_KT_CROSS_ENTROPY = 7,  /* with the loss reduction */
+  LLM_KT_EMBED_FWD = 8,
+  LLM_KT_EMBED_BWD = 9,
+  LLM_KT_ADAMW = 10,
+  LLM_KT_WEIGHT_CAST = 11,
+  LLM_KT_WGRAD_FINISH = 12,
+  LLM_KT_CLASSES = 13
+};
 int llm_set_kernel_timing(llm_ctx *ctx, int enable);
 int llm_read_kernel_timing(llm_ctx *ctx, double *ms, double *flops, int64_t *launches);
+int llm_read_kernel_class_timing(llm_ctx *ctx, int cls, double *ms, double *work,
+                                 int64_t *launches);
 
 #ifdef __cplusplus
 }

@@ -38,6 +38,13 @@ class llm_tensor_info(C.Structure):
 
 LLM_LR_CONSTANT, LLM_LR_COSINE, LLM_LR_LINEAR = 0, 1, 2
 LLM_CLIP_L2, LLM_CLIP_LINF = 0, 1
+# kernel classes of llm_read_kernel_class_timing (LLM_KT_*), with the unit of
+# the work each is credited with
+KERNEL_CLASSES = [("gemm", "flop"), ("attention_fwd", "flop"), ("attention_bwd", "flop"),
+                  ("rmsnorm_fwd", "byte"), ("rmsnorm_bwd", "byte"), ("swiglu_fwd", "byte"),
+                  ("swiglu_bwd", "byte"), ("cross_entropy", "byte"), ("embed_fwd", "byte"),
+                  ("embed_bwd", "byte"), ("adamw", "byte"), ("weight_cast", "byte"),
+                  ("wgrad_finish", "byte")]
 LR_SHAPES = {"constant": LLM_LR_CONSTANT, "cosine": LLM_LR_COSINE, "linear": LLM_LR_LINEAR}
 
 
@@ -93,6 +100,8 @@ EXPORTS = {
     "llm_set_graphs": (_i, [_vp, _i]),
     "llm_read_kernel_timing": (_i, [_vp, C.POINTER(C.c_double), C.POINTER(C.c_double),
                                     C.POINTER(_i64)]),
+    "llm_read_kernel_class_timing": (_i, [_vp, _i, C.POINTER(C.c_double), C.POINTER(C.c_double),
+                                          C.POINTER(_i64)]),
     # include/llm_kernels.h
     "llm_kernel_gemm_bf16": (_i, [_i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp,
                                   _vp]),

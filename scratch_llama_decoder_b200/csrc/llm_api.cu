@@ -148,12 +148,15 @@ struct llm_ctx {
   int32_t *sort_scratch;
   TcPlan *tc = nullptr;
   float *hyper;  // device [lr, wd, bc1, bc2] of the current step
-  // optional event timing of the tensor-core GEMM launches
+  // optional event timing of the step's launches by kernel class
+  // (llm_set_kernel_timing): event pairs in order, the class of each pair,
+  // and per class the algorithmic work credited (FLOPs or bytes)
   bool timing = false;
   std::vector<cudaEvent_t> ev_pool;
+  std::vector<int> ev_class;  // class of pair k (events 2k, 2k + 1)
   size_t ev_used = 0;
-  double pending_flops = 0.0;
-  int64_t pending_launches = 0;
+  double pending_work[LLM_KT_CLASSES] = {};
+  int64_t pending_count[LLM_KT_CLASSES] = {};
   // step graph: captured on the second llm_step with the same buffers,
   // replayed afterwards; steps with kernel timing on run as launches
   bool graphs = true;  // replay allowed (off after any capture failure)
@@ -565,23 +568,34 @@ int llm_plateau_update(llm_plateau *pl, double metric, float *scale) {
   return LLM_OK;
 }
 
-int llm_read_kernel_timing(llm_ctx *c, double *ms, double *flops, int64_t *launches) {
-  if (!c || !ms || !flops || !launches) return LLM_ERR_ARG;
+int llm_read_kernel_class_timing(llm_ctx *c, int cls, double *ms, double *work,
+                                 int64_t *launches) {
+  if (!c || !ms || !work || !launches || cls < 0 || cls >= LLM_KT_CLASSES) return LLM_ERR_ARG;
   if (!on_device(c)) return LLM_ERR_ARG;
   if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
   double total = 0.0;
   for (size_t i = 0; i + 1 < c->ev_used; i += 2) {
+    if (c->ev_class[i / 2] != cls) continue;
     float t = 0.f;
     if (cudaEventElapsedTime(&t, c->ev_pool[i], c->ev_pool[i + 1]) != cudaSuccess)
       return LLM_ERR_CUDA;
     total += t;
   }
   *ms = total;
-  *flops = c->pending_flops;
-  *launches = c->pending_launches;
+  *work = c->pending_work[cls];
+  *launches = c->pending_count[cls];
+  return LLM_OK;
+}
+
+int llm_read_kernel_timing(llm_ctx *c, double *ms, double *flops, int64_t *launches) {
+  if (!c || !ms || !flops || !launches) return LLM_ERR_ARG;
+  const int rc = llm_read_kernel_class_timing(c, LLM_KT_GEMM, ms, flops, launches);
+  if (rc != LLM_OK) return rc;
   c->ev_used = 0;
-  c->pending_flops = 0.0;
-  c->pending_launches = 0;
+  for (int k = 0; k < LLM_KT_CLASSES; k++) {
+    c->pending_work[k] = 0.0;
+    c->pending_count[k] = 0;
+  }
   return LLM_OK;
 }
 
@@ -607,33 +621,55 @@ namespace {
 
 bool aligned16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
 
-// Tensor-core GEMM launch; when timing is on, bracketed by CUDA events on the
-// context's stream and credited with its algorithmic FLOPs (unpadded sizes).
+// With kernel timing on, brackets the launches of its scope with CUDA events
+// on the context's current stream and credits them to a kernel class with
+// their algorithmic work (FLOPs or bytes); drop() takes back a scope that
+// launched nothing.
+struct KTimer {
+  llm_ctx *c;
+  int cls;
+  double work;
+  cudaEvent_t e1 = nullptr;
+  KTimer(llm_ctx *c_, int cls_, double work_) : c(c_), cls(cls_), work(work_) {
+    if (!c->timing) return;
+    while (c->ev_pool.size() < c->ev_used + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return;
+      c->ev_pool.push_back(e);
+    }
+    cudaEventRecord(c->ev_pool[c->ev_used], c->cur);
+    e1 = c->ev_pool[c->ev_used + 1];
+  }
+  void drop() { e1 = nullptr; }
+  ~KTimer() {
+    if (!e1) return;
+    cudaEventRecord(e1, c->cur);
+    if (c->ev_class.size() < c->ev_used / 2 + 1) c->ev_class.resize(c->ev_used / 2 + 1);
+    c->ev_class[c->ev_used / 2] = cls;
+    c->ev_used += 2;
+    c->pending_work[cls] += work;
+    c->pending_count[cls] += 1;
+  }
+};
+
+// Algorithmic work of the step's kernels (bytes a kernel must move, or FLOPs),
+// the units the timing classes are credited with.
+double rms_fwd_bytes(const Dims &D) { return (double)D.N * D.d * (4 + D.ab) + 4.0 * D.N; }
+double rms_bwd_bytes(const Dims &D, bool dres, bool act) {
+  return (double)D.N * D.d * (4.0 * (dres ? 4 : 3) + (act ? D.ab : 0)) + 4.0 * D.N;
+}
+double attn_flops(const Dims &D, double mult) {  // causal: T (T + 1) / 2 pairs
+  return mult * D.B * D.H * ((double)D.T * (D.T + 1) / 2.0) * D.hd;
+}
+
+// Tensor-core GEMM launch; when timing is on, timed as class GEMM with its
+// algorithmic FLOPs (unpadded sizes).
 bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
             int64_t ldr, int splits, int epi, double alg_flops) {
   if (!c->tc) return false;
-  cudaEvent_t e0 = nullptr, e1 = nullptr;
-  if (c->timing) {
-    while (c->ev_pool.size() < c->ev_used + 2) {
-      cudaEvent_t e;
-      if (cudaEventCreate(&e) != cudaSuccess) break;
-      c->ev_pool.push_back(e);
-    }
-    if (c->ev_pool.size() >= c->ev_used + 2) {
-      e0 = c->ev_pool[c->ev_used];
-      e1 = c->ev_pool[c->ev_used + 1];
-      cudaEventRecord(e0, c->cur);
-    }
-  }
-  bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->cur);
-  if (e0) {
-    cudaEventRecord(e1, c->cur);
-    if (ok) {
-      c->ev_used += 2;
-      c->pending_flops += alg_flops;
-      c->pending_launches += 1;
-    }
-  }
+  KTimer kt(c, LLM_KT_GEMM, alg_flops);
+  const bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->cur);
+  if (!ok) kt.drop();
   return ok;
 }
 
@@ -686,7 +722,10 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
   void *wqkv = A(c->w_qkv, l, d * D.qkvw), *wo = A(c->w_o, l, d * d);
   void *w13 = A(c->w_13, l, d * 2 * D.hp), *w2 = A(c->w_2, l, D.hp * d);
   // x1 = x + Attn(RMSNorm_g1(x))
-  rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
+  {
+    KTimer kt(c, LLM_KT_RMSNORM_FWD, rms_fwd_bytes(D));
+    rmsnorm_fwd(x, p + O.g1(l), xn1, D.dt, rstd1, N, D.d, c->cfg.rms_eps, s);
+  }
   {
     GemmOperands g{(int)N, (int)D.qkvw, D.d, xn1, d, true, wqkv, D.qkvw, false, D.dt};
     bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
@@ -702,17 +741,26 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
          nullptr, 0, 1, 2.0 * N * d * d);
     drop_add(x, c->dtmp, x1, N * d, drop_args(c, 2, l), s);
   } else {
-    attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
+    {
+      KTimer kt(c, LLM_KT_ATTN_FWD, attn_flops(D, 4.0));
+      attention_fwd(c->tc, qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s);
+    }
     gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_ADD_F32, x1, d,
          x, d, 1, 2.0 * N * d * d);
   }
   // x2 = x1 + SwiGLU(RMSNorm_g2(x1))
-  rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
+  {
+    KTimer kt(c, LLM_KT_RMSNORM_FWD, rms_fwd_bytes(D));
+    rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
+  }
   // W13 GEMM into the interleaved [a|b], then u = silu(a) * b (a separate
   // full-occupancy pass: cheaper than the same math in the GEMM epilogue)
   gemm(c, GemmOperands{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt},
        OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
-  swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
+  {
+    KTimer kt(c, LLM_KT_SWIGLU_FWD, 3.0 * N * D.h * ab);  // read a, b; write u
+    swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
+  }
   if (!out) return;  // the recomputation stops here: x2 exists
   if (drop) {  // x2 = x1 + f * (u W2)
     gemm(c, GemmOperands{(int)N, D.d, (int)D.hp, u, D.hp, true, w2, d, false, D.dt}, OUT_F32,
@@ -735,20 +783,30 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok, bool train) {
   cudaStream_t s = c->s;
   const int64_t N = D.N, d = D.d;
   // low-precision (or float32) padded copies of the weight matrices
-  if (D.L > 0) {
-    cast_weight(p + O.wqkv(0), c->w_qkv, D.dt, d, D.qkvw, d, D.qkvw, 0, 0, 0, D.L, D.layer_sz,
-                d * D.qkvw, s);
-    cast_weight(p + O.wo(0), c->w_o, D.dt, d, d, d, d, 0, 0, 0, D.L, D.layer_sz, d * d, s);
-    cast_weight(p + O.w13(0), c->w_13, D.dt, d, 2LL * D.h, d, 2 * D.hp, 1, D.h, D.hp, D.L,
-                D.layer_sz, d * 2 * D.hp, s);
-    cast_weight(p + O.w2(0), c->w_2, D.dt, D.h, d, D.hp, d, 0, 0, 0, D.L, D.layer_sz, D.hp * d, s);
+  {
+    const double M = (double)D.L * (d * D.qkvw + d * d + d * 2.0 * D.h + D.h * d) + d * D.V;
+    KTimer kt(c, LLM_KT_WEIGHT_CAST, M * (4 + D.ab));
+    if (D.L > 0) {
+      cast_weight(p + O.wqkv(0), c->w_qkv, D.dt, d, D.qkvw, d, D.qkvw, 0, 0, 0, D.L, D.layer_sz,
+                  d * D.qkvw, s);
+      cast_weight(p + O.wo(0), c->w_o, D.dt, d, d, d, d, 0, 0, 0, D.L, D.layer_sz, d * d, s);
+      cast_weight(p + O.w13(0), c->w_13, D.dt, d, 2LL * D.h, d, 2 * D.hp, 1, D.h, D.hp, D.L,
+                  D.layer_sz, d * 2 * D.hp, s);
+      cast_weight(p + O.w2(0), c->w_2, D.dt, D.h, d, D.hp, d, 0, 0, 0, D.L, D.layer_sz, D.hp * d, s);
+    }
+    cast_weight(p + O.wlm(), c->w_lm, D.dt, d, D.V, d, D.Vp, 0, 0, 0, 1, 0, 0, s);
   }
-  cast_weight(p + O.wlm(), c->w_lm, D.dt, d, D.V, d, D.Vp, 0, 0, 0, 1, 0, 0, s);
-  embed_fwd(p, tok, c->xs, N, D.d, D.V, c->flag_step, s);
+  {
+    KTimer kt(c, LLM_KT_EMBED_FWD, 8.0 * N * d + 4.0 * N);
+    embed_fwd(p, tok, c->xs, N, D.d, D.V, c->flag_step, s);
+  }
   if (drop) drop_rows(c->xs, N * d, drop_args(c, 0, 0), s);
   for (int l = 0; l < D.L; l++) layer_fwd(c, p, l, D.rc ? 0 : l, drop, true);
   float *xL = c->xs + D.L * N * d;
-  rmsnorm_fwd(xL, p + O.gf(), c->xf, D.dt, c->rstdf, N, D.d, c->cfg.rms_eps, s);
+  {
+    KTimer kt(c, LLM_KT_RMSNORM_FWD, rms_fwd_bytes(D));
+    rmsnorm_fwd(xL, p + O.gf(), c->xf, D.dt, c->rstdf, N, D.d, c->cfg.rms_eps, s);
+  }
   gemm(c, GemmOperands{(int)N, (int)D.Vp, D.d, c->xf, d, true, c->w_lm, D.Vp, false, D.dt},
        OUT_ACT, c->logits, D.Vp, nullptr, 0, 1, 2.0 * N * d * D.V);
 }
@@ -761,6 +819,7 @@ void wgrad(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, 
   int splits = wgrad_splits(D, M, Ncols);
   GemmOperands g{(int)M, (int)Ncols, (int)D.N, X, ldx, false, dY, ldy, false, D.dt};
   gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits, 2.0 * rows * cols * D.N);
+  KTimer kt(c, LLM_KT_WGRAD_FINISH, 4.0 * splits * M * Ncols + 4.0 * rows * cols);
   wgrad_finish(c->part, splits, M, Ncols, grad, rows, cols, mode, D.h, c->cur);
 }
 
@@ -813,9 +872,12 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
   gemm(c, GemmOperands{(int)N, D.d, (int)D.Vp, c->logits, D.Vp, true, c->w_lm, D.Vp, true, D.dt},
        OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.V * d);
   float *xL = c->xs + D.L * N * d;
-  nb = rmsnorm_bwd(xL, c->rstdf, p + O.gf(), c->dtmp, nullptr, c->dx, dxact, D.dt, c->dgpart, N,
-                   D.d, s);
-  reduce_partials(c->dgpart, nb, D.d, gr + O.gf(), s);
+  {
+    KTimer kt(c, LLM_KT_RMSNORM_BWD, rms_bwd_bytes(D, false, dxact != nullptr));
+    nb = rmsnorm_bwd(xL, c->rstdf, p + O.gf(), c->dtmp, nullptr, c->dx, dxact, D.dt, c->dgpart, N,
+                     D.d, s);
+    reduce_partials(c->dgpart, nb, D.d, gr + O.gf(), s);
+  }
   for (int l = D.L - 1; l >= 0; l--) {
     // with recompute, the layer's activations come back from its input first
     // (the side stream finished with the slot at the end of layer l + 1)
@@ -833,7 +895,10 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
     wgrad_side(c, u, D.hp, dxop, d, D.hp, d, gr + O.w2(l), D.h, d, 0);
     gemm(c, GemmOperands{(int)N, (int)D.hp, D.d, dxop, d, true, w2, d, true, D.dt}, OUT_ACT, c->du,
          D.hp, nullptr, 0, 1, 2.0 * N * d * D.h);
-    swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
+    {
+      KTimer kt(c, LLM_KT_SWIGLU_BWD, 5.0 * N * D.h * ab);  // read a, b, du; write da, db
+      swiglu_bwd(abuf, c->du, c->dab, D.dt, N, D.hp, s);
+    }
     fork_side(c);  // dab is ready
     wgrad_side(c, xn2, d, c->dab, 2 * D.hp, d, 2 * D.hp, gr + O.w13(l), d, 2LL * D.h, 1);
     gemm(c, GemmOperands{(int)N, D.d, (int)(2 * D.hp), c->dab, 2 * D.hp, true, w13, 2 * D.hp,
@@ -841,9 +906,12 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
          OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * 2 * D.h * d);
     join_side(c);  // the RMSNorm backward overwrites dx2 (dxA)
     if (buckets && l == D.L - 1) cudaEventRecord(c->ev_bucket[0], s);  // gf, Wlm
-    nb = rmsnorm_bwd(x1, rstd2, p + O.g2(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
-                     D.d, s);
-    reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
+    {
+      KTimer kt(c, LLM_KT_RMSNORM_BWD, rms_bwd_bytes(D, true, dxact != nullptr));
+      nb = rmsnorm_bwd(x1, rstd2, p + O.g2(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
+                       D.d, s);
+      reduce_partials(c->dgpart, nb, D.d, gr + O.g2(l), s);
+    }
     // attention branch
     if (drop) drop_to_act(c->dx, c->dxA, D.dt, N * d, drop_args(c, 2, l), s);
     gemm(c, GemmOperands{(int)N, D.d, D.d, dxop, d, true, wo, d, true, D.dt}, OUT_ACT, c->dO, d,
@@ -853,6 +921,7 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
                     drop_args(c, 1, l));
       rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);
     } else {
+      KTimer kt(c, LLM_KT_ATTN_BWD, attn_flops(D, 8.0));
       attention_bwd(c->tc, qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd,
                     c->cos_t, c->sin_t, s);
     }
@@ -863,13 +932,19 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
                          D.dt},
          OUT_F32, c->dtmp, d, nullptr, 0, 1, 2.0 * N * D.qkvw * d);
     join_side(c);  // the RMSNorm backward overwrites dx1 (dxA); the next layer dqkv
-    nb = rmsnorm_bwd(x, rstd1, p + O.g1(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N, D.d,
-                     s);
-    reduce_partials(c->dgpart, nb, D.d, gr + O.g1(l), s);
+    {
+      KTimer kt(c, LLM_KT_RMSNORM_BWD, rms_bwd_bytes(D, true, dxact != nullptr));
+      nb = rmsnorm_bwd(x, rstd1, p + O.g1(l), c->dtmp, c->dx, c->dx, dxact, D.dt, c->dgpart, N,
+                       D.d, s);
+      reduce_partials(c->dgpart, nb, D.d, gr + O.g1(l), s);
+    }
     if (buckets) cudaEventRecord(c->ev_bucket[D.L - l], s);  // layer l
   }
   if (drop) drop_rows(c->dx, N * d, drop_args(c, 0, 0), s);
-  embed_bwd(tok, c->dx, gr, N, D.d, D.V, c->sort_scratch, s);
+  {
+    KTimer kt(c, LLM_KT_EMBED_BWD, 4.0 * N * d + 4.0 * D.V * d + 4.0 * N);
+    embed_bwd(tok, c->dx, gr, N, D.d, D.V, c->sort_scratch, s);
+  }
   join_side(c);  // every weight gradient is in place before AdamW
   if (buckets) {
     if (D.L == 0) cudaEventRecord(c->ev_bucket[0], s);
@@ -975,13 +1050,20 @@ int llm_step(llm_ctx *c, float *d_params, float *d_grads, float *d_m, float *d_v
   auto body = [&]() {
     set_flag_zero(c->flag_step, c->s);
     forward(c, d_params, d_tokens, true);
-    cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
-                  c->flag_step, c->s);
-    loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
+    {
+      // logits read and written once (the gradient over them in place), row losses
+      KTimer kt(c, LLM_KT_CROSS_ENTROPY, 2.0 * D.N * D.V * D.ab + 8.0 * D.N);
+      cross_entropy(c->logits, D.dt, d_targets, c->rowloss, D.N, D.V, D.Vp, 1.0f / (float)D.N,
+                    c->flag_step, c->s);
+      loss_reduce(c->rowloss, D.N, d_loss, c->flag_step, c->s);
+    }
     backward(c, d_params, d_grads, d_tokens);
     if (c->clip > 0.f) clip_step(c, d_grads);
-    adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2,
-          c->cfg.adam_eps, c->flag_step, c->s);
+    {
+      KTimer kt(c, LLM_KT_ADAMW, 28.0 * D.P);  // read p, g, m, v; write p, m, v
+      adamw(d_params, d_grads, d_m, d_v, D.P, c->hyper, c->cfg.beta1, c->cfg.beta2,
+            c->cfg.adam_eps, c->flag_step, c->s);
+    }
     or_flag(c->flag_step, c->flag_sticky, c->s);
   };
   if (c->clip > 0.f) c->have_norm = true;

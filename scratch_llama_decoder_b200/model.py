@@ -255,6 +255,20 @@ class LlamaStep:
         L.check(L.lib.llm_set_graphs(self.ctx, int(bool(enable))), "llm_set_graphs")
 
     @_on_device
+    def read_kernel_class_timing(self):
+        """{class name: (device ms, algorithmic work, launches)} since the last
+        reset (llm_read_kernel_class_timing); read before read_kernel_timing,
+        which resets."""
+        out = {}
+        for k, (name, _) in enumerate(L.KERNEL_CLASSES):
+            ms, w, n = C.c_double(0), C.c_double(0), C.c_int64(0)
+            L.check(L.lib.llm_read_kernel_class_timing(self.ctx, k, C.byref(ms), C.byref(w),
+                                                       C.byref(n)),
+                    "llm_read_kernel_class_timing")
+            out[name] = (ms.value, w.value, n.value)
+        return out
+
+    @_on_device
     def read_kernel_timing(self):
         """(device ms, algorithmic FLOPs, launches) of the timed GEMM launches."""
         ms, fl, n = C.c_double(0), C.c_double(0), C.c_int64(0)
