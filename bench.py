@@ -211,6 +211,7 @@ def step_bytes(cfg):
     return N * L * per_tok_layer + per_step
 
 
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # nominal dense TF32 / BF16 tensor rates (1.1 and 2.25 PFLOP/s): a float32
 # workload's contractions are bounded by the TF32 rate at best
 TF32_OF_BF16 = 1.1 / 2.25
@@ -579,7 +580,11 @@ def kernel_rates(classes, steps, pk, src):
         ms, work, n = classes.get(name, (0.0, 0.0, 0))
         if n == 0 or ms <= 0:
             continue
-        if unit == "flop":
+        if unit == "flop" and name == "gemm_cuda_core":
+            # float32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 FLOPs x 1.965 GHz
+            rate, peak, u = work / (ms / 1e3) / 1e12, FP32_SIMT_TFLOPS, "TFLOP/s"
+            ps = "nominal float32 CUDA-core FMA rate"
+        elif unit == "flop":
             rate, peak, u = work / (ms / 1e3) / 1e12, peak_tc, "TFLOP/s"
             ps = f"{src} bf16_tflops_sustained"
         else:
@@ -631,15 +636,25 @@ def time_workload(name, steps, warmup, dev, local_rank, pk):
     torch.cuda.synchronize()
     clk = clocks.stop()
     assert model.status() == 0, name
+    # kernel classes: the same steps again as individual timed launches
+    model.set_kernel_timing(True)
+    for _ in range(steps):
+        t += 1
+        model.step(P, G, Mo, Vo, t, tok, tgt, cfg["lr"], cfg["wd"], loss)
+    classes = model.read_kernel_class_timing()
+    model.read_kernel_timing()
+    model.set_kernel_timing(False)
     ms = ev[0].elapsed_time(ev[-1]) / steps
     per_step = sorted(ev[k].elapsed_time(ev[k + 1]) for k in range(steps))
     roof = step_roofline(cfg, pk, ms)
+    src = "measured" if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else "fallback"
     out = {"workload": cfg["name"], "ms_per_step": ms, "value": N / (ms / 1e3),
            "unit": "tokens/s", "dtype": "bf16" if cfg["compute"] == "bf16" else "f32",
            "tokens_per_step": N, "frac_of_roofline": roof["frac_of_roofline"],
            "step_roofline": roof, "median_ms": per_step[len(per_step) // 2],
            "best_ms": per_step[0], "gpu_launches": launches * steps,
            "loss": float(loss.item()), "clocks": clk,
+           "kernels": kernel_rates(classes, steps, pk, src),
            "l2": "inputs larger than L2 (saved activations of the step); no flush"}
     model.close()
     del P, G, Mo, Vo, model

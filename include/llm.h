@@ -434,8 +434,9 @@ int llm_set_graphs(llm_ctx *ctx, int enable);
 /* Measurement hooks (strata, bench harness: time what is claimed).  With
  * timing enabled, the launches of later llm_step calls are bracketed by CUDA
  * events on the context's stream, per kernel class, and each bracket is
- * credited with its algorithmic work: FLOPs for the contractions (GEMM:
- * 2*M*N*K with unpadded sizes; attention: the causal T(T+1)/2 (query, key)
+ * credited with its algorithmic work: FLOPs for the contractions (GEMM, on
+ * tensor cores or, for float32 operands, CUDA cores: 2*M*N*K with unpadded
+ * sizes; attention: the causal T(T+1)/2 (query, key)
  * pairs per (sequence, head) times 4 hd FLOPs forward, 8 hd backward), bytes
  * for the memory-bound passes (what the pass must read and write once:
  * RMSNorm forward 4 + ab bytes per element plus the rstd, backward the float32
@@ -468,7 +469,8 @@ enum {
   LLM_KT_ADAMW = 10,
   LLM_KT_WEIGHT_CAST = 11,
   LLM_KT_WGRAD_FINISH = 12,
-  LLM_KT_CLASSES = 13
+  LLM_KT_GEMM_CUDA_CORE = 13, /* float32 projection GEMMs on CUDA cores (FLOPs) */
+  LLM_KT_CLASSES = 14
 };
 int llm_set_kernel_timing(llm_ctx *ctx, int enable);
 int llm_read_kernel_timing(llm_ctx *ctx, double *ms, double *flops, int64_t *launches);

@@ -44,7 +44,7 @@ KERNEL_CLASSES = [("gemm", "flop"), ("attention_fwd", "flop"), ("attention_bwd",
                   ("rmsnorm_fwd", "byte"), ("rmsnorm_bwd", "byte"), ("swiglu_fwd", "byte"),
                   ("swiglu_bwd", "byte"), ("cross_entropy", "byte"), ("embed_fwd", "byte"),
                   ("embed_bwd", "byte"), ("adamw", "byte"), ("weight_cast", "byte"),
-                  ("wgrad_finish", "byte")]
+                  ("wgrad_finish", "byte"), ("gemm_cuda_core", "flop")]
 LR_SHAPES = {"constant": LLM_LR_CONSTANT, "cosine": LLM_LR_COSINE, "linear": LLM_LR_LINEAR}
 
 

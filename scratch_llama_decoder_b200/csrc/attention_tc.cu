@@ -39,7 +39,7 @@ using namespace tc;
 
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
-constexpr int STAGES = 2;
+constexpr int STAGES = 4;  // K and V rings: deep enough to cover the TMA latency under load
 constexpr int NQ = 4;             // key groups of a block (independent softmaxes)
 constexpr int KW = 128 / NQ;      // keys per group (softmax thread)
 constexpr int SM_WARPS = 4 * NQ;  // softmax warps: 4 lane quarters x NQ groups
@@ -54,7 +54,8 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
 // shared memory: Q | K[2] | V[2] | barriers | red
-constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + 256 + 2 * NQ * 128 * 4 + 1024;
+constexpr int BAR_BYTES = 512;  // 48 mbarrier slots, then the TMEM address and abort words
+constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + BAR_BYTES + 2 * NQ * 128 * 4 + 1024;
 
 // Named barrier of the softmax warps (id 1) that ANDs a flag over them.
 LLM_DEV bool softmax_all(bool v) {
@@ -75,16 +76,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = smem, *sK = smem + TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
-  uint32_t *tmem_sh = (uint32_t *)(bars + 24);
+  uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
-  float *red = (float *)(bars + 32);  // [2][NQ][128]: m_g, then l_g per row
+  float *red = (float *)(bars + BAR_BYTES / 8);  // [2][NQ][128]: m_g, then l_g per row
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
-                 v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
-                 p_full = b0 + 8 * 11,             // [NQ]: one per key group
+  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * STAGES,
+                 v_full = k_empty + 8 * STAGES, v_empty = v_full + 8 * STAGES,
+                 s_full = v_empty + 8 * STAGES, s_free = s_full + 8,
+                 p_full = s_free + 8,              // [NQ]: one per key group
                  o_done = p_full + 8 * NQ,         // [NQ]
                  drain = o_done + 8 * NQ;          // [2]: one per MMA warp
-  static_assert(11 + 2 * NQ + 2 <= 24, "barriers overlap the TMEM address word");
+  static_assert(3 + 4 * STAGES + 2 * NQ + 2 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;

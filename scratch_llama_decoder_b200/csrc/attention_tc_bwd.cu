@@ -47,7 +47,7 @@ using namespace tc;
 
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
-constexpr int STAGES = 2;
+constexpr int STAGES = 4;  // streamed-operand rings: deep enough to cover the TMA latency
 constexpr int EW_WARPS = 16;  // elementwise warps: 4 lane quarters x NCQ column groups
 constexpr int NCQ = EW_WARPS / 4;  // column groups of a row (2 or 4)
 constexpr int CW = 128 / NCQ;      // score columns per thread
@@ -59,11 +59,12 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 // dQ kernel: TMEM columns; shared memory Q | dO | K[2] | V[2] | barriers | red
 constexpr int DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DS = 256, DQ_COL_DQA = 320, DQ_COL_DQB = 384;
-constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + 256 + NCQ * 128 * 4;
+constexpr int BAR_BYTES = 512;  // 48 mbarrier slots, then the TMEM address and abort words
+constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + BAR_BYTES + NCQ * 128 * 4;
 // dK/dV kernel: TMEM columns; shared memory K | V | Q[2] | dO[2] | L[2] | D[2] | barriers
 constexpr int KV_COL_S = 0, KV_COL_DP = 128, KV_COL_P = 256, KV_COL_DS = 320, KV_COL_DV = 384,
               KV_COL_DK = 448;
-constexpr int KV_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + 256 + 1024;
+constexpr int KV_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + BAR_BYTES + 1024;
 
 // Named barrier of the elementwise warps (id 1).
 LLM_DEV void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EW_WARPS) : "memory"); }
@@ -127,15 +128,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t *sQ = smem, *sdO = smem + TILE_BYTES, *sK = smem + 2 * TILE_BYTES,
           *sV = sK + STAGES * TILE_BYTES;
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
-  uint32_t *tmem_sh = (uint32_t *)(bars + 24);
+  uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
-  float *red = (float *)(bars + 32);  // [2][128] half-row partial dot products
+  float *red = (float *)(bars + BAR_BYTES / 8);  // [NCQ][128] partial dot products
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 8 * 3, v_full = b0 + 8 * 5,
-                 v_empty = b0 + 8 * 7, s_full = b0 + 8 * 9, s_free = b0 + 8 * 10,
-                 ds_full = b0 + 8 * 11,  // [2]: key half a, b
-                 dq_done = b0 + 8 * 13,  // [2]
-                 drain = b0 + 8 * 15;    // [2]: one per MMA warp
+  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * STAGES,
+                 v_full = k_empty + 8 * STAGES, v_empty = v_full + 8 * STAGES,
+                 s_full = v_empty + 8 * STAGES, s_free = s_full + 8,
+                 ds_full = s_free + 8,   // [2]: key half a, b
+                 dq_done = ds_full + 16, // [2]
+                 drain = dq_done + 16;   // [2]: one per MMA warp
+  static_assert(3 + 4 * STAGES + 6 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -376,12 +379,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float *sL = (float *)(sdO + STAGES * TILE_BYTES);  // [STAGES][128] L * log2(e)
   float *sD = sL + STAGES * 128;                      // [STAGES][128] D
   uint64_t *bars = (uint64_t *)(sD + STAGES * 128);
-  uint32_t *tmem_sh = (uint32_t *)(bars + 24);
+  uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t kv_full = b0, q_full = b0 + 8, q_empty = b0 + 8 * 3, ld_full = b0 + 8 * 5,
-                 s_full = b0 + 8 * 7, s_free = b0 + 8 * 8, p_full = b0 + 8 * 9,
-                 pv_done = b0 + 8 * 10, drain = b0 + 8 * 11;  // drain [2]: one per MMA warp
+  const uint32_t kv_full = b0, q_full = b0 + 8, q_empty = q_full + 8 * STAGES,
+                 ld_full = q_empty + 8 * STAGES, s_full = ld_full + 8 * STAGES,
+                 s_free = s_full + 8, p_full = s_free + 8, pv_done = p_full + 8,
+                 drain = pv_done + 8;  // drain [2]: one per MMA warp
+  static_assert(1 + 3 * STAGES + 6 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nkb = gridDim.z, kb = blockIdx.z;
   const int g = blockIdx.x, b = blockIdx.y;
@@ -531,17 +536,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) mbar_arrive(s_free);
       const int qc0 = qb * BQ + cq * CW;
       const bool diag = (qb == kb);  // keys >= T occur only in this case, above the diagonal
-      const float *Ls = sL + s * 128 + cq * CW, *Ds = sD + s * 128 + cq * CW;
+      // the step's per-query L and D: the same addresses in every lane (a
+      // broadcast), read as 16-byte vectors
+      float Lv[CW], Dl[CW];
+      {
+        const float4 *L4 = reinterpret_cast<const float4 *>(sL + s * 128 + cq * CW);
+        const float4 *D4 = reinterpret_cast<const float4 *>(sD + s * 128 + cq * CW);
+#pragma unroll
+        for (int i = 0; i < CW / 4; i++) {
+          const float4 a = L4[i], c = D4[i];
+          Lv[4 * i] = a.x; Lv[4 * i + 1] = a.y; Lv[4 * i + 2] = a.z; Lv[4 * i + 3] = a.w;
+          Dl[4 * i] = c.x; Dl[4 * i + 1] = c.y; Dl[4 * i + 2] = c.z; Dl[4 * i + 3] = c.w;
+        }
+      }
       uint32_t wp[CW / 2], wd[CW / 2];
 #pragma unroll
       for (int i = 0; i < CW; i += 2) {
-        float p0 = ex2(fmaf(sv[i], sl2, -Ls[i])), p1 = ex2(fmaf(sv[i + 1], sl2, -Ls[i + 1]));
+        float p0 = ex2(fmaf(sv[i], sl2, -Lv[i])), p1 = ex2(fmaf(sv[i + 1], sl2, -Lv[i + 1]));
         if (diag) {
           if (kj > qc0 + i) p0 = 0.f;
           if (kj > qc0 + i + 1) p1 = 0.f;
         }
         wp[i / 2] = pack_bf16(p0, p1);
-        wd[i / 2] = pack_bf16(p0 * (dv[i] - Ds[i]), p1 * (dv[i + 1] - Ds[i + 1]));
+        wd[i / 2] = pack_bf16(p0 * (dv[i] - Dl[i]), p1 * (dv[i + 1] - Dl[i + 1]));
       }
       // P^T and dS^T of the previous step are free once its products completed
       if (st > 0) {

@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace llm {
 
@@ -150,6 +151,17 @@ void embed_fwd(const float *wte, const int32_t *tok, float *x, int64_t N, int d,
   count_launch();
 }
 
+// Four values to 4 consecutive elements: one 8-byte store for bf16, one
+// 16-byte store for float (dst aligned to the element group).
+LLM_DEV void store4(__nv_bfloat16 *dst, float4 o) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+  uint2 q;
+  q.x = *reinterpret_cast<uint32_t *>(&lo);
+  q.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = q;
+}
+LLM_DEV void store4(float *dst, float4 o) { *reinterpret_cast<float4 *>(dst) = o; }
+
 // -------------------------------------------------------------- RMSNorm fwd
 // Hephaistos, Architecture at a glance (Normalization); MicroGPT in Rust,
 // RMSNorm: r = (mean_j x_j^2 + eps)^-1/2, y = g * x * r; r is cached.
@@ -177,9 +189,57 @@ __global__ void k_rmsnorm_fwd(const float *__restrict__ x, const float *__restri
   A *yr = y + row * d;
   for (int j = lane; j < d; j += 32) yr[j] = from_f<A>(g[j] * xr[j] * r);
 }
+// d = 128 * VPL: one warp per row, each lane holding VPL float4 of the row
+// (one read), the normalised row written with 8-byte (bf16) or 16-byte stores.
+template <typename A, int VPL>
+__global__ void __launch_bounds__(256) k_rmsnorm_fwd_v(const float *__restrict__ x,
+                                                       const float *__restrict__ g,
+                                                       A *__restrict__ y, float *__restrict__ rstd,
+                                                       int64_t N, float eps) {
+  constexpr int d = 128 * VPL;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const float4 *xr = reinterpret_cast<const float4 *>(x + row * d);
+  float4 v[VPL];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPL; k++) {
+    v[k] = xr[lane + 32 * k];
+    ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)d + eps);
+  if (lane == 0) rstd[row] = r;
+#pragma unroll
+  for (int k = 0; k < VPL; k++) {
+    const float4 gv = reinterpret_cast<const float4 *>(g)[lane + 32 * k];
+    float4 o;
+    o.x = gv.x * v[k].x * r; o.y = gv.y * v[k].y * r; o.z = gv.z * v[k].z * r; o.w = gv.w * v[k].w * r;
+    store4(y + row * d + 4 * (lane + 32 * k), o);
+  }
+}
 void rmsnorm_fwd(const float *x, const float *g, void *y, DType dt, float *rstd, int64_t N, int d,
                  float eps, cudaStream_t s) {
   unsigned grid = cdiv(N, 8);
+  if ((d == 128 || d == 256 || d == 512 || d == 1024) && ((uintptr_t)x & 15) == 0 &&
+      ((uintptr_t)g & 15) == 0 && ((uintptr_t)y & 15) == 0) {
+#define RF(VPL)                                                                                  \
+  do {                                                                                           \
+    if (dt == DT_BF16)                                                                           \
+      k_rmsnorm_fwd_v<__nv_bfloat16, VPL><<<grid, 256, 0, s>>>(x, g, (__nv_bfloat16 *)y, rstd, N, \
+                                                                eps);                            \
+    else                                                                                         \
+      k_rmsnorm_fwd_v<float, VPL><<<grid, 256, 0, s>>>(x, g, (float *)y, rstd, N, eps);         \
+  } while (0)
+    if (d == 128) RF(1);
+    else if (d == 256) RF(2);
+    else if (d == 512) RF(4);
+    else RF(8);
+#undef RF
+    count_launch();
+    return;
+  }
   if (dt == DT_BF16)
     k_rmsnorm_fwd<<<grid, 256, 0, s>>>(x, g, (__nv_bfloat16 *)y, rstd, N, d, eps);
   else
@@ -229,16 +289,6 @@ __global__ void k_rmsnorm_bwd(const float *__restrict__ x, const float *__restri
     part[(int64_t)blockIdx.x * d + j] = s;
   }
 }
-// Four values to 4 consecutive elements: one 8-byte store for bf16, one
-// 16-byte store for float (dst aligned to the element group).
-LLM_DEV void store4(__nv_bfloat16 *dst, float4 o) {
-  __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
-  uint2 q;
-  q.x = *reinterpret_cast<uint32_t *>(&lo);
-  q.y = *reinterpret_cast<uint32_t *>(&hi);
-  *reinterpret_cast<uint2 *>(dst) = q;
-}
-LLM_DEV void store4(float *dst, float4 o) { *reinterpret_cast<float4 *>(dst) = o; }
 
 // Vectorised form for d = 128 * VPL: each lane owns VPL float4 columns of a
 // row, keeps its gain-gradient partial sums in registers, and the block adds
@@ -459,35 +509,38 @@ LLM_DEV uint4 pack8(const float (&f)[8]) {
   }
   return q;
 }
+// sigmoid by the fast exponential and reciprocal intrinsics (relative error
+// ~1e-6, far below the bf16 rounding of the results)
+LLM_DEV float sigmoid_fast(float a) { return __fdividef(1.0f, 1.0f + __expf(-a)); }
+// Grid-stride over (row, 8-unit group) items with 32-bit index arithmetic
+// (the launcher keeps N * hp / 8 below 2^31).
 __global__ void k_swiglu_fwd_v8(const __nv_bfloat16 *__restrict__ ab, __nv_bfloat16 *__restrict__ u,
                                 int64_t N, int64_t hp) {
-  const int64_t per_row = hp / 8, n = N * per_row;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / per_row, j = (i % per_row) * 8;
-    const __nv_bfloat16 *r = ab + row * 2 * hp + w1_col(j);
+  const uint32_t per_row = (uint32_t)(hp / 8), n = (uint32_t)(N * (hp / 8));
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const uint32_t row = i / per_row, j = (i - row * per_row) * 8;
+    const __nv_bfloat16 *r = ab + (int64_t)row * 2 * hp + w1_col(j);
     float a[8], b[8], o[8];
     unpack8(*reinterpret_cast<const uint4 *>(r), a);
     unpack8(*reinterpret_cast<const uint4 *>(r + SWIGLU_BLOCK), b);
 #pragma unroll
-    for (int k = 0; k < 8; k++) o[k] = a[k] * sigmoidf_(a[k]) * b[k];
-    *reinterpret_cast<uint4 *>(u + row * hp + j) = pack8(o);
+    for (int k = 0; k < 8; k++) o[k] = a[k] * sigmoid_fast(a[k]) * b[k];
+    *reinterpret_cast<uint4 *>(u + (int64_t)row * hp + j) = pack8(o);
   }
 }
 __global__ void k_swiglu_bwd_v8(const __nv_bfloat16 *__restrict__ ab, const __nv_bfloat16 *__restrict__ du,
                                 __nv_bfloat16 *__restrict__ dab, int64_t N, int64_t hp) {
-  const int64_t per_row = hp / 8, n = N * per_row;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / per_row, j = (i % per_row) * 8;
-    const int64_t ca = row * 2 * hp + w1_col(j);
+  const uint32_t per_row = (uint32_t)(hp / 8), n = (uint32_t)(N * (hp / 8));
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const uint32_t row = i / per_row, j = (i - row * per_row) * 8;
+    const int64_t ca = (int64_t)row * 2 * hp + w1_col(j);
     float a[8], b[8], g[8], da[8], db[8];
     unpack8(*reinterpret_cast<const uint4 *>(ab + ca), a);
     unpack8(*reinterpret_cast<const uint4 *>(ab + ca + SWIGLU_BLOCK), b);
-    unpack8(*reinterpret_cast<const uint4 *>(du + row * hp + j), g);
+    unpack8(*reinterpret_cast<const uint4 *>(du + (int64_t)row * hp + j), g);
 #pragma unroll
     for (int k = 0; k < 8; k++) {
-      float sg = sigmoidf_(a[k]);
+      float sg = sigmoid_fast(a[k]);
       da[k] = g[k] * b[k] * sg * (1.f + a[k] * (1.f - sg));
       db[k] = g[k] * a[k] * sg;
     }
@@ -497,7 +550,8 @@ __global__ void k_swiglu_bwd_v8(const __nv_bfloat16 *__restrict__ ab, const __nv
 }
 
 void swiglu_fwd(const void *ab, void *u, DType dt, int64_t N, int64_t hp, cudaStream_t s) {
-  if (dt == DT_BF16 && hp % 8 == 0 && ((uintptr_t)ab & 15) == 0 && ((uintptr_t)u & 15) == 0) {
+  if (dt == DT_BF16 && hp % 8 == 0 && ((uintptr_t)ab & 15) == 0 && ((uintptr_t)u & 15) == 0 &&
+      N * (hp / 8) < ((int64_t)1 << 31)) {
     k_swiglu_fwd_v8<<<min(cdiv(N * hp / 8, 256), 148u * 16), 256, 0, s>>>(
         (const __nv_bfloat16 *)ab, (__nv_bfloat16 *)u, N, hp);
     count_launch();
@@ -513,7 +567,7 @@ void swiglu_fwd(const void *ab, void *u, DType dt, int64_t N, int64_t hp, cudaSt
 void swiglu_bwd(const void *ab, const void *du, void *dab, DType dt, int64_t N, int64_t hp,
                 cudaStream_t s) {
   if (dt == DT_BF16 && hp % 8 == 0 && ((uintptr_t)ab & 15) == 0 && ((uintptr_t)du & 15) == 0 &&
-      ((uintptr_t)dab & 15) == 0) {
+      ((uintptr_t)dab & 15) == 0 && N * (hp / 8) < ((int64_t)1 << 31)) {
     k_swiglu_bwd_v8<<<min(cdiv(N * hp / 8, 256), 148u * 16), 256, 0, s>>>(
         (const __nv_bfloat16 *)ab, (const __nv_bfloat16 *)du, (__nv_bfloat16 *)dab, N, hp);
     count_launch();
@@ -599,14 +653,30 @@ __global__ void __launch_bounds__(NT) k_cross_entropy(A *__restrict__ z, const i
   }
 }
 // bf16 rows held in registers: each thread keeps R 16-byte vectors (8
-// logits each, vector i = threadIdx.x + NT * k) from one read of the row;
-// max, then the sum of 2^(z log2 e - M log2 e), then the gradient, written
-// back once.  Exponentials by the single-instruction ex2 (relative error of a
-// few ulp).  Columns >= V inside the row (padding) get gradient 0.
+// logits each, vector i = threadIdx.x + NT * k) from one read of the row and
+// writes the gradient back over them once.  One exponential per logit: each
+// thread takes its own maximum m_t and sum s_t = sum 2^((z - m_t) log2 e) over
+// its logits, keeping the terms e = 2^((z - m_t) log2 e) (rounded to bf16, in
+// the registers that held the logits); one block reduction of the (m_t, s_t)
+// pairs in a fixed tree order gives the row's maximum M and sum S (the sum
+// from the float32 terms), and the gradient is e * 2^((m_t - M) log2 e) / S
+// minus 1 at the target, times 1/N.  Storing e rounds it once more than
+// computing it afresh would (relative 2^-9, the bf16 output's own rounding).
+// Exponentials by the single-instruction ex2 (relative error of a few ulp).
+// Columns >= V inside the row (padding) get gradient 0.
 LLM_DEV float ex2_fast(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// (m, s) pairs with s relative to 2^(m log2 e): the pair of the union.
+LLM_DEV void ms_combine(float &m, float &s, float m2, float s2) {
+  constexpr float L2E = 1.4426950408889634f;
+  const float mm = fmaxf(m, m2);
+  if (mm == -INFINITY) return;  // both empty
+  s = (m == -INFINITY ? 0.f : s * ex2_fast((m - mm) * L2E)) +
+      (m2 == -INFINITY ? 0.f : s2 * ex2_fast((m2 - mm) * L2E));
+  m = mm;
 }
 template <int NT, int R>
 __global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restrict__ z,
@@ -614,8 +684,8 @@ __global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restr
                                                           float *__restrict__ rowloss, int V,
                                                           int64_t ldz, float inv_n, int *flag) {
   constexpr float L2E = 1.4426950408889634f;
-  __shared__ float red[NT / 32];
-  __shared__ float bcast;
+  __shared__ float red_m[NT / 32], red_s[NT / 32];
+  __shared__ float bc_m, bc_s;
   const int64_t row = blockIdx.x;
   __nv_bfloat16 *zr = z + row * ldz;
   const int nvec = (int)(ldz / 8);
@@ -632,8 +702,8 @@ __global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restr
     y = 0;
   }
   const float zy = __bfloat162float(zr[y]);
-  // row maximum
-  float m = -INFINITY;
+  // this thread's maximum
+  float mt = -INFINITY;
 #pragma unroll
   for (int k = 0; k < R; k++) {
     const int v0 = 8 * (threadIdx.x + NT * k);
@@ -641,49 +711,50 @@ __global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restr
 #pragma unroll
     for (int t = 0; t < 4; t++) {
       const float2 f = __bfloat1622float2(e[t]);
-      if (v0 + 2 * t < V) m = fmaxf(m, f.x);
-      if (v0 + 2 * t + 1 < V) m = fmaxf(m, f.y);
+      if (v0 + 2 * t < V) mt = fmaxf(mt, f.x);
+      if (v0 + 2 * t + 1 < V) mt = fmaxf(mt, f.y);
     }
   }
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[w] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float mm = red[0];
-    for (int i = 1; i < NT / 32; i++) mm = fmaxf(mm, red[i]);
-    bcast = mm;
-  }
-  __syncthreads();
-  const float M2 = bcast * L2E;
-  // sum of exponentials (fixed order: thread, then warp shuffle tree, then warps)
-  float sum = 0.f;
+  // terms relative to mt, kept as bf16 in place of the logits; their sum
+  const float mt2 = mt == -INFINITY ? 0.f : mt * L2E;
+  float st = 0.f;
 #pragma unroll
   for (int k = 0; k < R; k++) {
     const int v0 = 8 * (threadIdx.x + NT * k);
-    const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&q[k]);
+    __nv_bfloat162 *e = reinterpret_cast<__nv_bfloat162 *>(&q[k]);
 #pragma unroll
     for (int t = 0; t < 4; t++) {
       const float2 f = __bfloat1622float2(e[t]);
-      if (v0 + 2 * t < V) sum += ex2_fast(fmaf(f.x, L2E, -M2));
-      if (v0 + 2 * t + 1 < V) sum += ex2_fast(fmaf(f.y, L2E, -M2));
+      const float ea = v0 + 2 * t < V ? ex2_fast(fmaf(f.x, L2E, -mt2)) : 0.f;
+      const float eb = v0 + 2 * t + 1 < V ? ex2_fast(fmaf(f.y, L2E, -mt2)) : 0.f;
+      st += ea + eb;
+      e[t] = __floats2bfloat162_rn(ea, eb);
     }
   }
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  __syncthreads();  // every warp has read bcast before red is reused
-  if (lane == 0) red[w] = sum;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float ss = 0.f;
-    for (int i = 0; i < NT / 32; i++) ss += red[i];
-    bcast = ss;
+  // the row's (M, S): warp tree, then the warps in order by thread 0
+  float m = mt, sm = st;
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+    ms_combine(m, sm, m2, s2);
+  }
+  if (lane == 0) {
+    red_m[w] = m;
+    red_s[w] = sm;
   }
   __syncthreads();
-  const float S = bcast;
-  const float lse = M2 / L2E + logf(S);
+  if (threadIdx.x == 0) {
+    float M = red_m[0], S = red_s[0];
+    for (int i = 1; i < NT / 32; i++) ms_combine(M, S, red_m[i], red_s[i]);
+    bc_m = M;
+    bc_s = S;
+  }
+  __syncthreads();
+  const float M = bc_m, S = bc_s;
+  const float lse = M + logf(S);
   if (threadIdx.x == 0) rowloss[row] = lse - zy;
-  const float LSE2 = lse * L2E;
   // every thread read z[y] (above) before any vector is written back: the
-  // block barriers of the two reductions order the read before these stores
+  // block barriers of the reduction order the read before these stores
+  const float fac = mt == -INFINITY ? 0.f : ex2_fast((mt - M) * L2E) / S * inv_n;
 #pragma unroll
   for (int k = 0; k < R; k++) {
     const int i = threadIdx.x + NT * k;
@@ -694,17 +765,209 @@ __global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restr
     for (int t = 0; t < 4; t++) {
       const float2 f = __bfloat1622float2(e[t]);
       const int va = v0 + 2 * t, vb = va + 1;
-      const float ga = va < V ? (ex2_fast(fmaf(f.x, L2E, -LSE2)) - (va == y ? 1.f : 0.f)) * inv_n : 0.f;
-      const float gb = vb < V ? (ex2_fast(fmaf(f.y, L2E, -LSE2)) - (vb == y ? 1.f : 0.f)) * inv_n : 0.f;
+      const float ga = f.x * fac - (va == y ? inv_n : 0.f);
+      const float gb = f.y * fac - (vb == y ? inv_n : 0.f);
       e[t] = __floats2bfloat162_rn(ga, gb);
     }
     reinterpret_cast<uint4 *>(zr)[i] = q[k];
   }
 }
 
+// Streaming form (bf16, rows of at most 32768 columns): a persistent grid of
+// one 512-thread block per SM walks groups of G = 16 / WPR consecutive rows
+// (WPR warps per row, at most 8 vectors of 8 logits per thread).  Each group
+// comes into one of two 64 KiB shared-memory buffers by one bulk copy
+// (cp.async.bulk, completion counted on an mbarrier), so the next groups load
+// while the current one is reduced and its gradient stored; the row
+// arithmetic is the register form's above (one exponential per logit, the
+// terms kept as bf16, one (m, s) reduction per row in a fixed order).  Every
+// wait is bounded: on time-out the block records FLAG_TIMEOUT, waits (again
+// bounded) for its own copies and leaves.
+constexpr int CES_THREADS = 512, CES_R = 8, CES_BUF = 64 * 1024;
+template <int WPR>
+__global__ void __launch_bounds__(CES_THREADS, 1)
+    k_cross_entropy_stream(__nv_bfloat16 *__restrict__ z, const int32_t *__restrict__ tgt,
+                           float *__restrict__ rowloss, int64_t N, int V, int64_t ldz,
+                           float inv_n, int *flag) {
+  constexpr float L2E = 1.4426950408889634f;
+  constexpr int G = 16 / WPR, TPR = 32 * WPR;
+  extern __shared__ __align__(1024) uint8_t ce_buf[];  // [2][CES_BUF]
+  __shared__ uint64_t full[2];
+  __shared__ float red_m[16], red_s[16];
+  __shared__ int stop_sh;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int grow = warp / WPR, t = threadIdx.x - grow * TPR;
+  const int64_t row_bytes = ldz * 2, ngroups = (N + G - 1) / G;
+  const int nvec = (int)(ldz / 8);
+  const uint32_t fb0 = tc::smem_u32(&full[0]);
+  if (threadIdx.x == 0) {
+    tc::mbar_init(fb0, 1);
+    tc::mbar_init(fb0 + 8, 1);
+    stop_sh = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // thread 0's record of the copy in flight into each buffer (for the drain)
+  uint32_t issued = 0, par[2] = {0, 0};
+  auto issue = [&](int64_t gi, int b) {
+    const int64_t rows = min((int64_t)G, N - gi * G);
+    const uint32_t bytes = (uint32_t)(rows * row_bytes);
+    const uint32_t bar = fb0 + 8 * b;
+    tc::mbar_arrive_expect_tx(bar, bytes);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            tc::smem_u32(ce_buf + b * CES_BUF)),
+        "l"(z + gi * G * ldz), "r"(bytes), "r"(bar)
+        : "memory");
+    issued |= 1u << b;
+  };
+  if (threadIdx.x == 0) {
+    if (blockIdx.x < ngroups) issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < ngroups) issue(blockIdx.x + gridDim.x, 1);
+  }
+  int k = 0;
+  for (int64_t gi = blockIdx.x; gi < ngroups; gi += gridDim.x, k++) {
+    const int b = k & 1;
+    const uint32_t ph = (k >> 1) & 1;
+    // bounded wait for this group's rows, then a block-wide verdict
+    bool ok = tc::mbar_try(fb0 + 8 * b, ph);
+    if (!ok) {
+      const unsigned long long t0 = tc::gtimer();
+      while (!(ok = tc::mbar_try(fb0 + 8 * b, ph)) && tc::gtimer() - t0 < tc::WAIT_NS) {
+      }
+    }
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) {
+        atomicOr(flag, FLAG_TIMEOUT);
+        for (int bb = 0; bb < 2; bb++)
+          if (issued & (1u << bb)) {
+            const unsigned long long t0 = tc::gtimer();
+            while (!tc::mbar_try(fb0 + 8 * bb, par[bb]) && tc::gtimer() - t0 < tc::WAIT_NS) {
+            }
+          }
+      }
+      return;
+    }
+    if (threadIdx.x == 0) {
+      issued &= ~(1u << b);
+      par[b] ^= 1u;
+    }
+    const int64_t row = gi * G + grow;
+    const bool valid = row < N;
+    const uint8_t *src = ce_buf + b * CES_BUF + grow * row_bytes;
+    uint4 q[CES_R];
+#pragma unroll
+    for (int kk = 0; kk < CES_R; kk++) {
+      const int i = t + TPR * kk;
+      q[kk] = (valid && i < nvec) ? reinterpret_cast<const uint4 *>(src)[i] : make_uint4(0, 0, 0, 0);
+    }
+    int y = valid ? tgt[row] : 0;
+    if (y < 0 || y >= V) {
+      if (valid && t == 0) atomicOr(flag, FLAG_TOKEN);
+      y = 0;
+    }
+    const float zy = valid ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(src)[y]) : 0.f;
+    __syncthreads();  // buffer b is read: the group after next may land in it
+    if (threadIdx.x == 0 && gi + 2 * (int64_t)gridDim.x < ngroups) issue(gi + 2 * gridDim.x, b);
+    // this thread's maximum, its terms (kept as bf16) and their sum
+    float mt = -INFINITY;
+#pragma unroll
+    for (int kk = 0; kk < CES_R; kk++) {
+      const int v0 = 8 * (t + TPR * kk);
+      const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&q[kk]);
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const float2 f = __bfloat1622float2(e[u]);
+        if (v0 + 2 * u < V) mt = fmaxf(mt, f.x);
+        if (v0 + 2 * u + 1 < V) mt = fmaxf(mt, f.y);
+      }
+    }
+    const float mt2 = mt == -INFINITY ? 0.f : mt * L2E;
+    float st = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < CES_R; kk++) {
+      const int v0 = 8 * (t + TPR * kk);
+      __nv_bfloat162 *e = reinterpret_cast<__nv_bfloat162 *>(&q[kk]);
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const float2 f = __bfloat1622float2(e[u]);
+        const float ea = v0 + 2 * u < V ? ex2_fast(fmaf(f.x, L2E, -mt2)) : 0.f;
+        const float eb = v0 + 2 * u + 1 < V ? ex2_fast(fmaf(f.y, L2E, -mt2)) : 0.f;
+        st += ea + eb;
+        e[u] = __floats2bfloat162_rn(ea, eb);
+      }
+    }
+    // the row's (M, S): warp tree, then the row's warps in order
+    float M = mt, S = st;
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, M, o), s2 = __shfl_xor_sync(0xffffffffu, S, o);
+      ms_combine(M, S, m2, s2);
+    }
+    if (WPR > 1) {
+      if (lane == 0) {
+        red_m[warp] = M;
+        red_s[warp] = S;
+      }
+      __syncthreads();
+      M = red_m[grow * WPR];
+      S = red_s[grow * WPR];
+      for (int w = 1; w < WPR; w++) ms_combine(M, S, red_m[grow * WPR + w], red_s[grow * WPR + w]);
+      __syncthreads();  // red is reused by the next group
+    }
+    if (!valid) continue;
+    const float lse = M + logf(S);
+    if (t == 0) rowloss[row] = lse - zy;
+    const float fac = mt == -INFINITY ? 0.f : ex2_fast((mt - M) * L2E) / S * inv_n;
+    __nv_bfloat16 *zr = z + row * ldz;
+#pragma unroll
+    for (int kk = 0; kk < CES_R; kk++) {
+      const int i = t + TPR * kk;
+      if (i >= nvec) continue;
+      const int v0 = 8 * i;
+      __nv_bfloat162 *e = reinterpret_cast<__nv_bfloat162 *>(&q[kk]);
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const float2 f = __bfloat1622float2(e[u]);
+        const int va = v0 + 2 * u, vb = va + 1;
+        e[u] = __floats2bfloat162_rn(f.x * fac - (va == y ? inv_n : 0.f),
+                                     f.y * fac - (vb == y ? inv_n : 0.f));
+      }
+      reinterpret_cast<uint4 *>(zr)[i] = q[kk];
+    }
+  }
+}
+
 void cross_entropy(void *logits, DType dt, const int32_t *tgt, float *rowloss, int64_t N, int V,
                    int64_t ldz, float inv_n, int *flag, cudaStream_t s) {
   constexpr int NT = 256, R = 16;
+  if (dt == DT_BF16 && ldz % 8 == 0 && ((uintptr_t)logits & 15) == 0 && ldz <= 32768) {
+    // warps per row: the fewest (a power of two) that keep 8 vectors a thread
+    const int64_t nvec = ldz / 8;
+    int wpr = 1;
+    while ((int64_t)32 * wpr * CES_R < nvec) wpr *= 2;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t groups = (N + 16 / wpr - 1) / (16 / wpr);
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(groups, sms));
+    const int smem = 2 * CES_BUF;
+#define CES(W)                                                                                    \
+  do {                                                                                            \
+    smem_optin((const void *)k_cross_entropy_stream<W>, smem);                                   \
+    k_cross_entropy_stream<W><<<grid, CES_THREADS, smem, s>>>((__nv_bfloat16 *)logits, tgt,      \
+                                                             rowloss, N, V, ldz, inv_n, flag);   \
+  } while (0)
+    switch (wpr) {
+      case 1: CES(1); break;
+      case 2: CES(2); break;
+      case 4: CES(4); break;
+      case 8: CES(8); break;
+      default: CES(16); break;
+    }
+#undef CES
+    count_launch();
+    return;
+  }
   if (dt == DT_BF16 && ldz % 8 == 0 && ((uintptr_t)logits & 15) == 0 && ldz <= (int64_t)NT * R * 8) {
     k_cross_entropy_reg<NT, R><<<(unsigned)N, NT, 0, s>>>((__nv_bfloat16 *)logits, tgt, rowloss, V,
                                                          ldz, inv_n, flag);
@@ -833,10 +1096,23 @@ __global__ void k_wgrad_finish(const float *__restrict__ part, int splits, int64
     for (int64_t c = 4 * (int64_t)threadIdx.x; c < cols; c += 4 * (int64_t)blockDim.x) {
       if (vec && c + 4 <= cols) {
         const int64_t cp = mode == 1 ? ((c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK) : c;
-        float4 acc = *reinterpret_cast<const float4 *>(pr + cp);
-        for (int k = 1; k < splits; k++) {
-          const float4 q = *reinterpret_cast<const float4 *>(pr + k * pstride + cp);
-          acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+        // up to 8 splits' loads in flight at once, added in split order
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k0 = 0; k0 < splits; k0 += 8) {
+          float4 q[8];
+#pragma unroll
+          for (int u = 0; u < 8; u++)
+            if (k0 + u < splits)
+              q[u] = *reinterpret_cast<const float4 *>(pr + (k0 + u) * pstride + cp);
+#pragma unroll
+          for (int u = 0; u < 8; u++) {
+            if (k0 + u >= splits) break;
+            if (k0 + u == 0) {
+              acc = q[u];
+            } else {
+              acc.x += q[u].x; acc.y += q[u].y; acc.z += q[u].z; acc.w += q[u].w;
+            }
+          }
         }
         *reinterpret_cast<float4 *>(gr + c) = acc;
       } else {

@@ -678,6 +678,7 @@ bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
 void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
           int64_t ldr, int splits, double alg_flops) {
   if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, alg_flops)) return;
+  KTimer kt(c, LLM_KT_GEMM_CUDA_CORE, alg_flops);
   gemm_simt(g, out, C, ldc, R, ldr, splits, c->cur);
 }
 
@@ -731,7 +732,10 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
     bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
                         2.0 * N * d * D.qkvw);
     if (!fused) {
-      gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
+      {
+        KTimer kt(c, LLM_KT_GEMM_CUDA_CORE, 2.0 * N * d * D.qkvw);
+        gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
+      }
       rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
     }
   }
