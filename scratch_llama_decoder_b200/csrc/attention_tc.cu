@@ -5,29 +5,36 @@
 //
 // One CTA = 128 queries of one (batch, head); key blocks of 128, split into
 // NQ key groups of KW = 128 / NQ keys.  Warps:
-//   warp 0          TMA producer: the Q tile once, K and V tiles into 2-deep
-//                   rings;
+//   warp 0          TMA producer: the Q tile once, K and V tiles into
+//                   STAGES-deep rings;
 //   warp 1          TMEM allocation and MMA issuer A:
-//                     S    = Q K^T       (M 128, N 128, K 64; both operands
-//                                         K-major in shared memory) -> TMEM S
+//                     S_j  = Q K_j^T     (M 128, N 128, K 64; both operands
+//                                         K-major in shared memory) into TMEM
+//                                         buffer j % 2
 //                     O_g += P_g V_g     for key groups g < NQ/2 (M 128, N 64,
 //                                         K KW; A = P_g from TMEM, B = the V
 //                                         rows of group g, MN-major) -> TMEM O_g
 //   last warp       MMA issuer B: O_g += P_g V_g for groups g >= NQ/2;
 //   4 NQ warps      softmax, NQ per TMEM lane quarter: thread = one query row
 //                   (TMEM lane) and one key group.
-// The key groups are NQ independent online softmaxes (split-K inside the CTA):
-// each (row, group) thread keeps its own running maximum m_g, sum l_g and
-// accumulator O_g, so no thread waits for another inside the key loop; the
-// groups meet once at the end, O = sum_g 2^(m_g-m) O_g / sum_g 2^(m_g-m) l_g
-// with m = max_g m_g.  The running maximum is lazy: the reference of a
-// (row, group) moves only when a block's maximum exceeds it by more than 2^8,
-// so P stays below 256 and O_g is rescaled only then; O_g and l_g always share
-// one reference.  The group's scores are read from TMEM in one round trip and
-// S is released at once, so Q K_{j+1}^T runs during block j's exponentials.
-// MMAs are issued by whole converged warps (one elected lane), from two warps
-// because one warp issues a tcgen05.mma only every ~127 cycles whatever N is.
-// Every wait is bounded (FLAG_TIMEOUT, then drain and free TMEM).
+// S is double-buffered in TMEM and each group's P of a block is written back,
+// packed bf16, over the first KW/2 of that group's own S columns once read:
+// S_{j+1} is computed into the other buffer as soon as the P V products of
+// block j - 1 (which read that buffer) have completed, so a softmax thread
+// finishing block j finds S_{j+1} ready and never waits for the slowest
+// thread to release its S; it waits for the P V products only before a rare
+// rescale of its accumulator.  The key groups are NQ independent online
+// softmaxes (split-K inside the CTA): each (row, group) thread keeps its own
+// running maximum m_g, sum l_g and accumulator O_g; the groups meet once at
+// the end, O = sum_g 2^(m_g-m) O_g / sum_g 2^(m_g-m) l_g with m = max_g m_g.
+// The running maximum is lazy: the reference of a (row, group) moves only when
+// a block's maximum exceeds it by more than 2^8, so P stays below 256 and O_g
+// is rescaled only then.  The maximum is taken on the raw scores (the log2
+// scale is positive) and only the diagonal block runs the causal mask, so an
+// off-diagonal block costs a maximum and one fused multiply-add and one
+// exponential per score.  MMAs are issued by whole converged warps (one
+// elected lane).  Every wait is bounded (FLAG_TIMEOUT, then drain and free
+// TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "tcgen05.cuh"
@@ -46,9 +53,10 @@ constexpr int SM_WARPS = 4 * NQ;  // softmax warps: 4 lane quarters x NQ groups
 constexpr int MMA_B_WARP = 2 + SM_WARPS;
 constexpr int NTHREADS = 32 * (MMA_B_WARP + 1);
 constexpr int TMEM_COLS = 512;
-// TMEM columns: S [0,128), P (packed bf16, group g at COL_P + g KW/2), O_g at
-// COL_O + 64 g
-constexpr int COL_S = 0, COL_P = 128, COL_O = 192;
+// TMEM columns: two S buffers [0,128) and [128,256) (block j in buffer j % 2;
+// group g's P of that block, packed bf16, over the first KW/2 of the group's
+// own S columns once read), O_g at COL_O + 64 g
+constexpr int COL_S = 0, COL_O = 256;
 static_assert(COL_O + 64 * NQ <= TMEM_COLS, "TMEM columns");
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -82,11 +90,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t b0 = smem_u32(bars);
   const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * STAGES,
                  v_full = k_empty + 8 * STAGES, v_empty = v_full + 8 * STAGES,
-                 s_full = v_empty + 8 * STAGES, s_free = s_full + 8,
-                 p_full = s_free + 8,              // [NQ]: one per key group
+                 s_full = v_empty + 8 * STAGES,    // [2]: one per S buffer
+                 buf_free = s_full + 16,           // [2]: the buffer's P V products done
+                 p_full = buf_free + 16,           // [NQ]: one per key group
                  o_done = p_full + 8 * NQ,         // [NQ]
                  drain = o_done + 8 * NQ;          // [2]: one per MMA warp
-  static_assert(3 + 4 * STAGES + 2 * NQ + 2 <= 48, "barriers overlap the TMEM address word");
+  static_assert(5 + 4 * STAGES + 2 * NQ + 2 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -104,8 +113,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(v_full + 8 * s, 1);
       mbar_init(v_empty + 8 * s, 2);  // both P V halves read V_j
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, SM_WARPS);
+    for (int bb = 0; bb < 2; bb++) {
+      mbar_init(s_full + 8 * bb, 1);
+      mbar_init(buf_free + 8 * bb, 2);  // both MMA warps' P V products of the block
+    }
     for (int g2 = 0; g2 < NQ; g2++) {
       mbar_init(p_full + 8 * g2, 4);  // the group's four lane-quarter warps
       mbar_init(o_done + 8 * g2, 1);
@@ -164,14 +175,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
     constexpr uint32_t ID_O = idesc_mn(128, HD, false, true);
     const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
-    auto issue_s = [&](int j) {  // S = Q K_j^T
+    auto issue_s = [&](int j) {  // S = Q K_j^T into buffer j % 2
       const int s = j % STAGES;
       const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < HD / 16; kk++)
-        mma_bf16_e(tmem + COL_S, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), ID_S,
-                   kk > 0 ? 1u : 0u);
-      mma_commit_e(s_full);
+        mma_bf16_e(tmem + COL_S + 128 * (j & 1), qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2),
+                   ID_S, kk > 0 ? 1u : 0u);
+      mma_commit_e(s_full + 8 * (j & 1));
       mma_commit_e(k_empty + 8 * s);
     };
     bool ok = true;
@@ -186,11 +197,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int s = j % STAGES;
       const uint32_t ph = (j / STAGES) & 1;
       if (x == 0 && j + 1 < nj) {
-        // next block's scores once the softmax has read this block's S
+        // next block's scores into the other buffer once its P V products
+        // (block j - 1) have completed
         const int s1 = (j + 1) % STAGES;
         const uint32_t ph1 = ((j + 1) / STAGES) & 1;
         if (!warp_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
-            !warp_wait(s_free, j & 1, abort_sh, gflag)) {
+            (j >= 1 && !warp_wait(buf_free + 8 * ((j + 1) & 1), ((j - 1) >> 1) & 1, abort_sh,
+                                  gflag))) {
           ok = false;
           break;
         }
@@ -213,13 +226,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_after();
 #pragma unroll
         for (int kk = 0; kk < KW / 16; kk++)
-          mma_ts_e(tmem + COL_O + 64 * grp, tmem + COL_P + grp * (KW / 2) + kk * 8,
+          mma_ts_e(tmem + COL_O + 64 * grp, tmem + COL_S + 128 * (j & 1) + grp * KW + kk * 8,
                    vd + (uint64_t)((grp * (KW / 16) + kk) * 128), ID_O,
                    (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit_e(o_done + 8 * grp);
       }
       if (!ok) break;
       mma_commit_e(v_empty + 8 * s);
+      mma_commit_e(buf_free + 8 * (j & 1));
     }
     mma_commit_e(drain + 8 * x);
     if (lane == 0) {
@@ -240,7 +254,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nj && ok; j++) {
-      if (!warp_wait(s_full, j & 1, abort_sh, gflag)) {
+      const uint32_t col_s = COL_S + 128 * (j & 1) + grp * KW;  // this group's S, then P
+      if (!warp_wait(s_full + 8 * (j & 1), (j >> 1) & 1, abort_sh, gflag)) {
         ok = false;
         break;
       }
@@ -248,30 +263,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int k0 = j * BK + grp * KW;
       const bool diag = (j * BK + BK > q0);  // only the diagonal block (or T) masks
       float sv[KW];
-      tmem_ldn<KW>(tmem + lane_off + COL_S + grp * KW, sv);
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);  // the MMA warp may overwrite S now
-      // this group's block maximum (log2 units), 4 independent chains
+      tmem_ldn<KW>(tmem + lane_off + col_s, sv);
+      // this group's block maximum on the raw scores (the log2 factor sl2 > 0
+      // keeps the order), 4 independent chains; masked scores become -inf
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (diag) {  // the diagonal block (and keys past T): mask, then the maximum
 #pragma unroll
-      for (int i = 0; i < KW; i++) {
-        float x = sv[i] * sl2;
-        if (diag && (k0 + i > qi || k0 + i >= T)) x = -INFINITY;
-        sv[i] = x;
-        m4[i & 3] = fmaxf(m4[i & 3], x);
+        for (int i = 0; i < KW; i++) {
+          if (k0 + i > qi || k0 + i >= T) sv[i] = -INFINITY;
+          m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < KW; i++) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
       }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       // true on the first block with an unmasked key (m_ref = -inf until then)
       const bool need = mx > m_ref + LAZY;
-      // P_g and O_g of the previous block are free once its P V has completed
-      if (j > 0) {
+      // O_g is rescaled only after the previous block's P V into it completed
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
         if (!warp_wait(o_done + 8 * grp, (j - 1) & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        {
           const float corr = need ? ex2(m_ref - mx) : 1.f;  // 0 while m_ref = -inf
 #pragma unroll
           for (int c = 0; c < 4; c++) {
@@ -296,14 +312,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < KW; i += 2) {
-        const float p0 = ex2(sv[i] - mr), p1 = ex2(sv[i + 1] - mr);
+        const float p0 = ex2(fmaf(sv[i], sl2, -mr)), p1 = ex2(fmaf(sv[i + 1], sl2, -mr));
         l4[(i >> 1) & 3] += p0 + p1;
         w[i / 2] = pack_bf16(p0, p1);
       }
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
 #pragma unroll
       for (int c = 0; c < KW / 2; c += 16)
-        tmem_stn<(KW / 2 < 16 ? KW / 2 : 16)>(tmem + lane_off + COL_P + grp * (KW / 2) + c, w + c);
+        tmem_stn<(KW / 2 < 16 ? KW / 2 : 16)>(tmem + lane_off + col_s + c, w + c);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       fence_before();
       __syncwarp();

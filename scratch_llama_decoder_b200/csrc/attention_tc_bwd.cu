@@ -308,14 +308,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int k0 = j * BK + cq * CW;
       const bool diag = (j == qb);  // only the diagonal block masks (keys >= T lie above it)
       uint32_t w[CW / 2];
+      if (diag) {  // the causal mask only on the diagonal block
 #pragma unroll
-      for (int i = 0; i < CW; i += 2) {
-        float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
-        if (diag) {
+        for (int i = 0; i < CW; i += 2) {
+          float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
           if (k0 + i > qi) p0 = 0.f;
           if (k0 + i + 1 > qi) p1 = 0.f;
+          w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
         }
-        w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
+      } else {
+#pragma unroll
+        for (int i = 0; i < CW; i += 2) {
+          const float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
+          w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
+        }
       }
       // this half's dS of the previous block is free once its dQ product completed
       if (j > 0) {
@@ -536,29 +542,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) mbar_arrive(s_free);
       const int qc0 = qb * BQ + cq * CW;
       const bool diag = (qb == kb);  // keys >= T occur only in this case, above the diagonal
-      // the step's per-query L and D: the same addresses in every lane (a
-      // broadcast), read as 16-byte vectors
-      float Lv[CW], Dl[CW];
-      {
-        const float4 *L4 = reinterpret_cast<const float4 *>(sL + s * 128 + cq * CW);
-        const float4 *D4 = reinterpret_cast<const float4 *>(sD + s * 128 + cq * CW);
-#pragma unroll
-        for (int i = 0; i < CW / 4; i++) {
-          const float4 a = L4[i], c = D4[i];
-          Lv[4 * i] = a.x; Lv[4 * i + 1] = a.y; Lv[4 * i + 2] = a.z; Lv[4 * i + 3] = a.w;
-          Dl[4 * i] = c.x; Dl[4 * i + 1] = c.y; Dl[4 * i + 2] = c.z; Dl[4 * i + 3] = c.w;
-        }
-      }
+      const float4 *L4 = reinterpret_cast<const float4 *>(sL + s * 128 + cq * CW);
+      const float4 *D4 = reinterpret_cast<const float4 *>(sD + s * 128 + cq * CW);
       uint32_t wp[CW / 2], wd[CW / 2];
 #pragma unroll
-      for (int i = 0; i < CW; i += 2) {
-        float p0 = ex2(fmaf(sv[i], sl2, -Lv[i])), p1 = ex2(fmaf(sv[i + 1], sl2, -Lv[i + 1]));
+      for (int i = 0; i < CW; i += 4) {
+        const float4 lq = L4[i / 4], dq = D4[i / 4];
+        float p0 = ex2(fmaf(sv[i], sl2, -lq.x)), p1 = ex2(fmaf(sv[i + 1], sl2, -lq.y));
+        float p2 = ex2(fmaf(sv[i + 2], sl2, -lq.z)), p3 = ex2(fmaf(sv[i + 3], sl2, -lq.w));
         if (diag) {
           if (kj > qc0 + i) p0 = 0.f;
           if (kj > qc0 + i + 1) p1 = 0.f;
+          if (kj > qc0 + i + 2) p2 = 0.f;
+          if (kj > qc0 + i + 3) p3 = 0.f;
         }
         wp[i / 2] = pack_bf16(p0, p1);
-        wd[i / 2] = pack_bf16(p0 * (dv[i] - Dl[i]), p1 * (dv[i + 1] - Dl[i + 1]));
+        wp[i / 2 + 1] = pack_bf16(p2, p3);
+        wd[i / 2] = pack_bf16(p0 * (dv[i] - dq.x), p1 * (dv[i + 1] - dq.y));
+        wd[i / 2 + 1] = pack_bf16(p2 * (dv[i + 2] - dq.z), p3 * (dv[i + 3] - dq.w));
       }
       // P^T and dS^T of the previous step are free once its products completed
       if (st > 0) {

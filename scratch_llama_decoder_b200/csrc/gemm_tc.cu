@@ -15,7 +15,9 @@
 //               (a residual comes in through bulk tensor loads of the same
 //               square).
 // Two accumulators of 256 columns alternate so the epilogue of one tile
-// overlaps the main loop of the next.  Operands may be K-major or MN-major
+// overlaps the main loop of the next.  Products with M and N of at least 512
+// run on CTA pairs instead (k_gemm_tc2 below: 256 x 256 tiles on two SMs,
+// tcgen05.mma.cta_group::2), the rest on single CTAs.  Operands may be K-major or MN-major
 // (both supported by the UMMA descriptors), which covers the forward
 // (x W), data-gradient (dy W^T) and weight-gradient (x^T dy) orientations
 // without transposed copies.  Every mbarrier wait is bounded; on time-out the
@@ -427,6 +429,281 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+// ------------------------------------------------- CTA-pair (cta_group::2)
+// A cluster of two CTAs on two SMs computes one 256 x 256 tile: CTA r loads
+// rows [m0 + 128 r, m0 + 128 r + 128) of A and columns [n0 + 128 r, ...) of
+// B (32 KiB per stage, no multicast), and the leader (r = 0) issues
+// tcgen05.mma.cta_group::2 (M 256, N 256, K 16), which reads A's halves and
+// B's halves from both CTAs' shared memory at the same offsets and leaves rows
+// 128 r .. 128 r + 127 of the tile in CTA r's TMEM.  Per output element each
+// SM moves a third fewer operand bytes than the single-CTA 128 x 256 tile.
+//   full[s] (leader): both CTAs' copies of stage s complete on it (the
+//     cta_group::2 form of the tensor copy takes the leader's barrier), armed
+//     once by the leader for both CTAs' bytes;
+//   empty[s], tfull[b]: the leader's commits arrive on both CTAs' barriers
+//     (commit multicast);
+//   tempty[b] (leader): both CTAs' epilogue warps arrive (the peer's remotely).
+// (A first form let each CTA's copies complete on its own barrier and had the
+// peer relay the completion to the leader: measured at half the rate of the
+// single-CTA kernel, the relay hop serialising every stage.)  The leader's
+// drain waits on its full barriers, which count both CTAs' bytes, and the
+// final cluster barrier keeps the peer resident until then.  Both CTAs walk
+// the same work items; every wait is bounded.
+constexpr int STAGES2 = 6;
+constexpr int HALF_BYTES = 128 * BK * 2;          // 16 KB: 128 rows x 64 K
+constexpr int STAGE2_BYTES = 2 * HALF_BYTES;      // this CTA's A rows and B columns
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + STAGING_BYTES + 512;
+
+LLM_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared-memory address of the same object in CTA `rank` of the cluster.
+LLM_DEV uint32_t cluster_addr(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+// TMA load into this CTA's shared memory whose bytes complete on the barrier
+// at cluster address `bar` (the leader's), cta_group::2 form.
+LLM_DEV void tma_load_2d_pair_e(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n}\n" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+LLM_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+LLM_DEV void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+LLM_DEV void mma_pair_e(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(ad), "l"(bd), "r"(id), "r"(acc)
+      : "memory");
+}
+// Arrive (when the leader's prior MMAs complete) on the barrier at offset
+// `bar` in both CTAs of the pair.
+LLM_DEV void commit_pair_both_e(uint32_t bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n}\n" ::"r"(bar),
+      "h"((unsigned short)3)
+      : "memory");
+}
+
+// Arrive on this CTA's barrier when the leader's prior pair MMAs complete.
+LLM_DEV void commit_pair_e(uint32_t bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(
+          bar)
+      : "memory");
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_gemm_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
+               const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = (uint64_t *)(smem + STAGES2 * STAGE2_BYTES + STAGING_BYTES);
+  // bars: full[S2], empty[S2], tfull[2], tempty[2], drain, rbar[EPI_WARPS]
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * STAGES2;
+  const uint32_t tfull0 = empty0 + 8 * STAGES2, tempty0 = tfull0 + 16, drain = tempty0 + 16;
+  const uint32_t rbar0 = drain + 8;
+  static_assert(8 * (2 * STAGES2 + 5 + EPI_WARPS) <= 512, "barrier space");
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    for (int s = 0; s < STAGES2; s++) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 2 * EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    for (int w = 0; w < EPI_WARPS; w++) mbar_init(rbar0 + 8 * w, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base_sh)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+  fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int tiles_mn = a.tiles_m * a.tiles_n;  // tiles of 256 x 256
+  const int kblocks_total = (a.K + BK - 1) / BK;
+  const int cid = blockIdx.x / 2, ncl = gridDim.x / 2;
+  auto kblocks_of = [&](int split, int &kb0) {
+    int kb_per = a.kchunk / BK;
+    kb0 = split * kb_per;
+    int kb1 = min(kblocks_total, kb0 + kb_per);
+    return max(0, kb1 - kb0);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------ TMA producer (each CTA, its halves)
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t issued_parity[STAGES2];
+    bool issued[STAGES2];
+    for (int i = 0; i < STAGES2; i++) issued[i] = false;
+    bool ok = true;
+    const uint32_t lead_full0 = cluster_addr(full0, 0);
+    for (int w = cid; w < a.total && ok; w += ncl) {
+      const int split = w / tiles_mn, tile = w % tiles_mn;
+      const int m0 = (tile % a.tiles_m) * 256 + 128 * (int)rank;
+      const int n0 = (tile / a.tiles_m) * 256 + 128 * (int)rank;
+      int kb0, nkb = kblocks_of(split, kb0);
+      for (int kb = 0; kb < nkb; kb++) {
+        if (!warp_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) { ok = false; break; }
+        // both CTAs' bytes complete on the leader's full[s], armed once for both
+        const uint32_t fb = lead_full0 + 8 * s;
+        if (leader) mbar_arrive_expect_tx_e(full0 + 8 * s, 2 * STAGE2_BYTES);
+        const uint32_t sa = smem_u32(smem + s * STAGE2_BYTES), sb = sa + HALF_BYTES;
+        const int k0 = (kb0 + kb) * BK;
+        if (A_MN) {
+          tma_load_2d_pair_e(sa, &tmA, m0, k0, fb);
+          tma_load_2d_pair_e(sa + 8192, &tmA, m0 + 64, k0, fb);
+        } else {
+          tma_load_2d_pair_e(sa, &tmA, k0, m0, fb);
+        }
+        if (B_MN) {
+          tma_load_2d_pair_e(sb, &tmB, n0, k0, fb);
+          tma_load_2d_pair_e(sb + 8192, &tmB, n0 + 64, k0, fb);
+        } else {
+          tma_load_2d_pair_e(sb, &tmB, k0, n0, fb);
+        }
+        issued[s] = true;
+        issued_parity[s] = ph;
+        if (++s == STAGES2) { s = 0; ph ^= 1; }
+      }
+    }
+    // both CTAs' copies complete on the leader's full barriers: the leader
+    // waits for them before the pair may exit (normally they were consumed
+    // already); the final cluster barrier holds the peer until then
+    if (lane == 0 && leader)
+      for (int i = 0; i < STAGES2; i++)
+        if (issued[i]) {
+          const unsigned long long t0 = gtimer();
+          while (!mbar_try(full0 + 8 * i, issued_parity[i]) && gtimer() - t0 < WAIT_NS) {
+          }
+        }
+    __syncwarp();
+  } else if (warp == 1 && !leader) {
+    // the peer's warp 1 only shares the TMEM allocation
+  } else if (warp == 1) {
+    // ------------------------------------ MMA issuer (leader)
+    constexpr uint32_t ID = idesc_mn(256, BN, A_MN, B_MN);
+    int s = 0;
+    uint32_t ph = 0;
+    int acc = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    for (int w = cid; w < a.total && ok; w += ncl) {
+      const int split = w / tiles_mn;
+      int kb0, nkb = kblocks_of(split, kb0);
+      if (nkb == 0) continue;  // the epilogues write zeros without waiting
+      if (!warp_wait(tempty0 + 8 * acc, aph ^ 1, &abort_sh, a.flag)) break;
+      fence_after();
+      const uint32_t td = tmem + acc * BN;
+      for (int kb = 0; kb < nkb; kb++) {
+        if (!warp_wait(full0 + 8 * s, ph, &abort_sh, a.flag)) { ok = false; break; }
+        fence_after();
+        const uint32_t sa = smem_u32(smem + s * STAGE2_BYTES), sb = sa + HALF_BYTES;
+        const uint64_t ad = A_MN ? sdesc(sa, 8192, 1024) : sdesc(sa, 16, 1024);
+        const uint64_t bd = B_MN ? sdesc(sb, 8192, 1024) : sdesc(sb, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; kk++) {
+          const uint64_t da = (uint64_t)(A_MN ? kk * 128 : kk * 2);
+          const uint64_t db = (uint64_t)(B_MN ? kk * 128 : kk * 2);
+          mma_pair_e(td, ad + da, bd + db, ID, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        commit_pair_both_e(empty0 + 8 * s);  // frees the stage in both CTAs
+        if (++s == STAGES2) { s = 0; ph ^= 1; }
+      }
+      if (!ok) break;
+      commit_pair_both_e(tfull0 + 8 * acc);  // accumulator ready in both CTAs
+      if (++acc == 2) { acc = 0; aph ^= 1; }
+    }
+    commit_pair_e(drain);
+    if (lane == 0) {
+      const unsigned long long t0 = gtimer();
+      while (!mbar_try(drain, 0) && gtimer() - t0 < WAIT_NS) {
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 2) {
+    // ------------------------------------ epilogue warps (each CTA, its rows)
+    const int quarter = warp & 3;
+    const int ew = warp - 2;
+    const int c_lo = (ew / 4) * (BN / 2);
+    float *stg = reinterpret_cast<float *>(smem + STAGES2 * STAGE2_BYTES) + ew * STG_BUFS * 32 * 32;
+    int sb = 0;
+    uint32_t rph = 0;
+    const uint32_t rbar = rbar0 + 8 * ew;
+    const uint32_t lead_tempty0 = cluster_addr(tempty0, 0);
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int w = cid; w < a.total; w += ncl) {
+      const int split = w / tiles_mn, tile = w % tiles_mn;
+      const int m0 = (tile % a.tiles_m) * 256 + 128 * (int)rank;
+      const int n0 = (tile / a.tiles_m) * 256;
+      int kb0, nkb = kblocks_of(split, kb0);
+      const int row0 = m0 + quarter * 32;
+      if (nkb == 0) {
+        epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, 0, row0, n0, c_lo, split, true, stg,
+                      sb);
+        continue;
+      }
+      if (!warp_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag)) break;
+      fence_after();
+      const uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
+      epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, tm, row0, n0, c_lo, split, false, stg,
+                    sb);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead_tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; aph ^= 1; }
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no arrival may target a CTA that has left
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 }  // namespace tc
 
 // ------------------------------------------------------------------ host side
@@ -437,6 +714,7 @@ struct TcPlan {
   int T, hd;
   int64_t rot_cols, hp;
   int *flag = nullptr;  // device flag word for time-outs (set by the owner)
+  bool pairs = true;  // CTA-pair kernel for large shapes
   std::mutex mu;
   struct Key {
     const void *p;
@@ -523,7 +801,11 @@ TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, 
   cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, dev);
   p->cos_t = cos_t; p->sin_t = sin_t; p->T = T; p->hd = hd; p->rot_cols = rot_cols; p->hp = hp;
   // the plan's device is current here: opt every variant in on it
-  if (!smem_optin((const void *)tc::k_gemm_tc<false, false>, tc::SMEM_BYTES) ||
+  if (!smem_optin((const void *)tc::k_gemm_tc2<false, false>, tc::SMEM2_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc2<false, true>, tc::SMEM2_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc2<true, false>, tc::SMEM2_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc2<true, true>, tc::SMEM2_BYTES) ||
+      !smem_optin((const void *)tc::k_gemm_tc<false, false>, tc::SMEM_BYTES) ||
       !smem_optin((const void *)tc::k_gemm_tc<false, true>, tc::SMEM_BYTES) ||
       !smem_optin((const void *)tc::k_gemm_tc<true, false>, tc::SMEM_BYTES) ||
       !smem_optin((const void *)tc::k_gemm_tc<true, true>, tc::SMEM_BYTES)) {
@@ -531,6 +813,12 @@ TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, 
     return nullptr;
   }
   return p;
+}
+
+// CTA pairs (256 x 256 tiles) once both sides span at least two tiles of
+// the pair kernel: smaller problems keep the 128 x 256 tiles' parallelism.
+bool tc_gemm_pairs(const TcPlan *p, int64_t M, int64_t N) {
+  return p && p->pairs && M >= 512 && N >= 512;
 }
 
 void tc_plan_set_flag(TcPlan *p, int *flag) {
@@ -580,8 +868,34 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   a.out = out; a.epi = epi; a.C = C; a.ldc = ldc; a.R = R; a.ldr = ldr;
   a.cos_t = p->cos_t; a.sin_t = p->sin_t; a.T = p->T; a.hd = p->hd; a.rot_cols = (int)p->rot_cols;
   a.flag = p->flag;
-  int grid = min(a.total, p->num_sms);
   bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
+  if (tc_gemm_pairs(p, g.M, g.N)) {
+    // CTA pairs: B boxes of 128 rows (K-major), tiles of 256 x 256
+    if (g.b_kmajor && !p->map(g.B, g.K, g.N, g.ldb, 64, 128, &tb)) return false;
+    a.tiles_m = (g.M + 255) / 256;
+    a.tiles_n = (g.N + BN - 1) / BN;
+    a.total = a.tiles_m * a.tiles_n * a.splits;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (unsigned)min(a.total, p->num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (!amn && !bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<false, false>, ta, tb, tcm, trm, a);
+    else if (!amn && bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<false, true>, ta, tb, tcm, trm, a);
+    else if (amn && !bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<true, false>, ta, tb, tcm, trm, a);
+    else e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<true, true>, ta, tb, tcm, trm, a);
+    count_launch();
+    return e == cudaSuccess;
+  }
+  int grid = min(a.total, p->num_sms);
   if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
   else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
   else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);

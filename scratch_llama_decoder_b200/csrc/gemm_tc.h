@@ -21,6 +21,9 @@ void tc_plan_destroy(TcPlan *p);
 void tc_plan_set_flag(TcPlan *p, int *flag);
 bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
              int64_t ldr, int splits, int epi, cudaStream_t s);
+// Whether tc_gemm runs an [M, N] product on CTA pairs (256 x 256 tiles, 74
+// pairs on 148 SMs) rather than single CTAs (128 x 256 tiles).
+bool tc_gemm_pairs(const TcPlan *p, int64_t M, int64_t N);
 
 // Attention dispatch: tensor-core kernels when the plan covers the head size,
 // else the SIMT kernels.

@@ -1096,23 +1096,10 @@ __global__ void k_wgrad_finish(const float *__restrict__ part, int splits, int64
     for (int64_t c = 4 * (int64_t)threadIdx.x; c < cols; c += 4 * (int64_t)blockDim.x) {
       if (vec && c + 4 <= cols) {
         const int64_t cp = mode == 1 ? ((c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK) : c;
-        // up to 8 splits' loads in flight at once, added in split order
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k0 = 0; k0 < splits; k0 += 8) {
-          float4 q[8];
-#pragma unroll
-          for (int u = 0; u < 8; u++)
-            if (k0 + u < splits)
-              q[u] = *reinterpret_cast<const float4 *>(pr + (k0 + u) * pstride + cp);
-#pragma unroll
-          for (int u = 0; u < 8; u++) {
-            if (k0 + u >= splits) break;
-            if (k0 + u == 0) {
-              acc = q[u];
-            } else {
-              acc.x += q[u].x; acc.y += q[u].y; acc.z += q[u].z; acc.w += q[u].w;
-            }
-          }
+        float4 acc = *reinterpret_cast<const float4 *>(pr + cp);
+        for (int k = 1; k < splits; k++) {
+          const float4 q = *reinterpret_cast<const float4 *>(pr + k * pstride + cp);
+          acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
         }
         *reinterpret_cast<float4 *>(gr + c) = acc;
       } else {
@@ -1158,26 +1145,49 @@ __global__ void k_radix_hist(const int32_t *__restrict__ keys, int64_t N, int sh
   __syncthreads();
   hist[(int64_t)threadIdx.x * nblk + blockIdx.x] = cnt[threadIdx.x];
 }
-// Exclusive scan of n ints in place (one block of 1024 threads).
-__global__ void k_scan_excl(int32_t *a, int64_t n) {
-  __shared__ int32_t sh[1024];
+// Exclusive scan of n ints in place (one block of 1024 threads): chunks of
+// 4096, four consecutive elements per thread, a warp-shuffle scan of the
+// thread sums, then one warp scans the 32 warp totals; the running total of
+// the chunks before carries over.  Integer sums: the result is exact.
+__global__ void __launch_bounds__(1024) k_scan_excl(int32_t *a, int64_t n) {
+  __shared__ int32_t wtot[32];
   __shared__ int32_t carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  for (int64_t base = 0; base < n; base += 1024) {
-    int64_t i = base + threadIdx.x;
-    int32_t v = (i < n) ? a[i] : 0;
-    sh[threadIdx.x] = v;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-      int32_t t = (threadIdx.x >= (unsigned)o) ? sh[threadIdx.x - o] : 0;
-      __syncthreads();
-      sh[threadIdx.x] += t;
-      __syncthreads();
+  for (int64_t base = 0; base < n; base += 4096) {
+    const int64_t i0 = base + 4 * (int64_t)threadIdx.x;
+    int32_t v[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) v[k] = i0 + k < n ? a[i0 + k] : 0;
+    const int32_t t = v[0] + v[1] + v[2] + v[3];
+    int32_t inc = t;  // inclusive scan of the thread sums within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += u;
     }
-    if (i < n) a[i] = carry + sh[threadIdx.x] - v;
+    if (lane == 31) wtot[warp] = inc;
     __syncthreads();
-    if (threadIdx.x == 1023) carry += sh[1023];
+    if (warp == 0) {
+      const int32_t w = wtot[lane];
+      int32_t wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += u;
+      }
+      wtot[lane] = wi - w;  // exclusive warp offsets
+    }
+    __syncthreads();
+    int32_t run = carry + wtot[warp] + inc - t;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      if (i0 + k < n) a[i0 + k] = run;
+      run += v[k];
+    }
+    __syncthreads();  // every thread read carry and wtot
+    if (threadIdx.x == 1023) carry = run;  // the last thread's running total is the chunk's end
     __syncthreads();
   }
 }

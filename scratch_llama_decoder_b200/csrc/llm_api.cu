@@ -88,15 +88,19 @@ struct POff {
 // 64 at the tensor rate, 1.9 GHz) plus the partial sums' extra HBM traffic
 // (written by the GEMM, read by the finish pass, 6.5 TB/s); every split keeps
 // at least 8 k-blocks, at most 32 splits.
-int wgrad_splits(const Dims &D, int64_t M, int64_t Ncols) {
-  const int64_t tiles = ((M + 127) / 128) * ((Ncols + 255) / 256);
+// With CTA pairs (pairs = true) an item is a 256 x 256 tile on two SMs, so
+// 74 items run at once and each takes the same time per k-block.
+int wgrad_splits(const Dims &D, int64_t M, int64_t Ncols, bool pairs = false) {
+  const int64_t tiles = pairs ? ((M + 255) / 256) * ((Ncols + 255) / 256)
+                              : ((M + 127) / 128) * ((Ncols + 255) / 256);
+  const int64_t units = pairs ? 74 : 148;
   const int64_t kb = (D.N + 63) / 64;
   int best = 1;
   double best_us = 1e300;
   for (int s = 1; s <= 32; s++) {
     const int64_t kbs = (kb + s - 1) / s;
     if (s > 1 && kbs < 8) break;
-    const double waves = (double)((tiles * s + 147) / 148);
+    const double waves = (double)((tiles * s + units - 1) / units);
     const double us = waves * (double)kbs * 520.0 / 1900.0 +
                       2.0 * s * (double)M * (double)Ncols * 4.0 / 6.5e6;
     if (us < best_us * (1.0 - 1e-9)) {
@@ -240,7 +244,9 @@ int64_t llm_ctx::carve(char *base) {
   dqkv = c.take(ab * N * D_.qkvw);
   int64_t part_elems = 0;
   auto need = [&](int64_t M, int64_t Nc) {
-    part_elems = std::max<int64_t>(part_elems, (int64_t)wgrad_splits(D_, M, Nc) * M * Nc);
+    // room for the split count of either kernel (single CTAs or CTA pairs)
+    const int64_t sp = std::max(wgrad_splits(D_, M, Nc, false), wgrad_splits(D_, M, Nc, true));
+    part_elems = std::max<int64_t>(part_elems, sp * M * Nc);
   };
   need(d, D_.Vp); need(D_.hp, d); need(d, 2 * D_.hp); need(d, d); need(d, D_.qkvw);
   part = (float *)c.take(4 * part_elems);
@@ -820,7 +826,7 @@ void forward(llm_ctx *c, const float *p, const int32_t *tok, bool train) {
 void wgrad(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, int64_t M,
            int64_t Ncols, float *grad, int64_t rows, int64_t cols, int mode) {
   const Dims &D = c->D;
-  int splits = wgrad_splits(D, M, Ncols);
+  int splits = wgrad_splits(D, M, Ncols, tc_gemm_pairs(c->tc, M, Ncols));
   GemmOperands g{(int)M, (int)Ncols, (int)D.N, X, ldx, false, dY, ldy, false, D.dt};
   gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits, 2.0 * rows * cols * D.N);
   KTimer kt(c, LLM_KT_WGRAD_FINISH, 4.0 * splits * M * Ncols + 4.0 * rows * cols);
