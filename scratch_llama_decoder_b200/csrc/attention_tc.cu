@@ -31,9 +31,11 @@
 // a block's maximum exceeds it by more than 2^8, so P stays below 256 and O_g
 // is rescaled only then.  The maximum is taken on the raw scores (the log2
 // scale is positive) and only the diagonal block runs the causal mask, so an
-// off-diagonal block costs a maximum and one fused multiply-add and one
-// exponential per score.  MMAs are issued by whole converged warps (one
-// elected lane).  Every wait is bounded (FLAG_TIMEOUT, then drain and free
+// off-diagonal block costs half a three-input maximum, half a packed f32x2
+// multiply-add and one exponential per score; 5 of every 16 pairs of
+// exponentials run as a polynomial on the FMA pipe (exp2_poly2), the rest on
+// the SFU, whose 16 results per clock and SM would otherwise bound the
+// softmax.  MMAs are issued by whole converged warps (one elected lane).  Every wait is bounded (FLAG_TIMEOUT, then drain and free
 // TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
@@ -61,9 +63,27 @@ static_assert(COL_O + 64 * NQ <= TMEM_COLS, "TMEM columns");
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
-// shared memory: Q | K[2] | V[2] | barriers | red
+// shared memory: Q[2] | K[STAGES] | V[STAGES] | barriers | red[2]
 constexpr int BAR_BYTES = 512;  // 48 mbarrier slots, then the TMEM address and abort words
-constexpr int SMEM_BYTES = (1 + 2 * STAGES) * TILE_BYTES + BAR_BYTES + 2 * NQ * 128 * 4 + 1024;
+constexpr int SMEM_BYTES = (2 + 2 * STAGES) * TILE_BYTES + BAR_BYTES + 2 * 2 * NQ * 128 * 4 + 1024;
+
+// P = 2^(s sl2 - mr) for the KW scores of one (row, group), packed bf16 into
+// w; returns their sum.  Pairs in packed f32x2 arithmetic; with FMA_EXP some
+// pairs take the polynomial 2^x, the rest the SFU.
+template <bool FMA_EXP>
+LLM_DEV float exp_pack(const float (&sv)[KW], float sl2, float mr, uint32_t (&w)[KW / 2]) {
+  float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < KW; i += 2) {
+    const float2 x = __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2),
+                                make_float2(-mr, -mr));
+    const float2 p = FMA_EXP ? exp2_pair(x, i / 2) : make_float2(ex2(x.x), ex2(x.y));
+    if ((i >> 1) & 1) lb = __fadd2_rn(lb, p);
+    else la = __fadd2_rn(la, p);
+    w[i / 2] = pack_bf16(p.x, p.y);
+  }
+  return (la.x + lb.x) + (la.y + lb.y);
+}
 
 // Named barrier of the softmax warps (id 1) that ANDs a flag over them.
 LLM_DEV bool softmax_all(bool v) {
@@ -77,36 +97,49 @@ LLM_DEV bool softmax_all(bool v) {
   return r != 0;
 }
 
+// Named barrier of the softmax warps (id 1).
+LLM_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * SM_WARPS) : "memory"); }
+
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16 *__restrict__ o,
-                  float *__restrict__ lse, int T, int H, int Hkv, float scale, int *gflag) {
+                  float *__restrict__ lse, int B, int T, int H, int Hkv, float scale, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sQ = smem, *sK = smem + TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
+  uint8_t *sQ = smem, *sK = smem + 2 * TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
   uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
   float *red = (float *)(bars + BAR_BYTES / 8);  // [2][NQ][128]: m_g, then l_g per row
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * STAGES,
+  const uint32_t q_full = b0, q_empty = b0 + 16,  // [2]: Q slot
+                 k_full = b0 + 32, k_empty = k_full + 8 * STAGES,
                  v_full = k_empty + 8 * STAGES, v_empty = v_full + 8 * STAGES,
                  s_full = v_empty + 8 * STAGES,    // [2]: one per S buffer
                  buf_free = s_full + 16,           // [2]: the buffer's P V products done
-                 p_full = buf_free + 16,           // [NQ]: one per key group
-                 o_done = p_full + 8 * NQ,         // [NQ]
+                 // [2][NQ]: per S buffer and key group, so that a group's arrivals for
+                 // blocks j and j + 1 (other buffer) can never alias one phase
+                 p_full = buf_free + 16,
+                 o_done = p_full + 16 * NQ,        // [NQ]
                  drain = o_done + 8 * NQ;          // [2]: one per MMA warp
-  static_assert(5 + 4 * STAGES + 2 * NQ + 2 <= 48, "barriers overlap the TMEM address word");
+  static_assert(4 + 4 * STAGES + 4 + 3 * NQ + 2 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int g = h / (H / Hkv), d = H * HD, kvd = Hkv * HD;
-  const int q0 = qb * BQ;
-  const int nj = min(qb + 1, (T + BK - 1) / BK);  // causal: key blocks up to the diagonal
-  const int row_base = b * T;
+  const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int d = H * HD, kvd = Hkv * HD;
+  // item -> (query block, head, batch), longest rows (last query blocks) first
+  auto decode = [&](int item, int &qb, int &h, int &b) {
+    const int z = item / (H * B), rem = item - z * (H * B);
+    qb = nqb - 1 - z;
+    h = rem % H;
+    b = rem / H;
+  };
 
   if (threadIdx.x == 0) {
     *abort_sh = 0;
-    mbar_init(q_full, 1);
+    for (int x = 0; x < 2; x++) {
+      mbar_init(q_full + 8 * x, 1);
+      mbar_init(q_empty + 8 * x, 1);  // the item's last S product on the slot
+    }
     for (int s = 0; s < STAGES; s++) {
       mbar_init(k_full + 8 * s, 1);
       mbar_init(k_empty + 8 * s, 1);
@@ -117,10 +150,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(s_full + 8 * bb, 1);
       mbar_init(buf_free + 8 * bb, 2);  // both MMA warps' P V products of the block
     }
-    for (int g2 = 0; g2 < NQ; g2++) {
-      mbar_init(p_full + 8 * g2, 4);  // the group's four lane-quarter warps
-      mbar_init(o_done + 8 * g2, 1);
-    }
+    for (int g2 = 0; g2 < 2 * NQ; g2++) mbar_init(p_full + 8 * g2, 4);  // 4 lane-quarter warps
+    for (int g2 = 0; g2 < NQ; g2++) mbar_init(o_done + 8 * g2, 1);
     mbar_init(drain, 1);
     mbar_init(drain + 8, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -140,33 +171,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer
+      int gb = 0, nq = 0;  // key blocks and Q tiles issued
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      tma_load_2d(smem_u32(sQ), &tm_qkv, h * HD, row_base + q0, q_full);
-      for (int j = 0; j < nj && ok; j++) {
-        const int s = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
-        if (!mbar_wait(k_empty + 8 * s, ph ^ 1, abort_sh, gflag)) { ok = false; break; }
-        mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
-        tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
-                    k_full + 8 * s);
-        if (!mbar_wait(v_empty + 8 * s, ph ^ 1, abort_sh, gflag)) { ok = false; break; }
-        mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
-        tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD, row_base + j * BK,
-                    v_full + 8 * s);
+      for (int r = 0, it = 0; ok; r++, it++) {
+        const int item = sched_item(r, G, cta);
+        if (item >= n_items) break;
+        int qb, h, b;
+        decode(item, qb, h, b);
+        const int row_base = b * T, g = h / (H / Hkv), slot = it & 1;
+        // Q into the slot of item it - 2 once its last S product completed
+        if (!mbar_wait(q_empty + 8 * slot, ((it >> 1) & 1) ^ 1, abort_sh, gflag)) break;
+        mbar_arrive_expect_tx(q_full + 8 * slot, TILE_BYTES);
+        tma_load_2d(smem_u32(sQ + slot * TILE_BYTES), &tm_qkv, h * HD, row_base + qb * BQ,
+                    q_full + 8 * slot);
+        nq = it + 1;
+        for (int j = 0; j <= qb; j++) {
+          const int s = gb % STAGES;
+          const uint32_t ph = (gb / STAGES) & 1;
+          if (!mbar_wait(k_empty + 8 * s, ph ^ 1, abort_sh, gflag) ||
+              !mbar_wait(v_empty + 8 * s, ph ^ 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
+          tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
+                      k_full + 8 * s);
+          mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
+          tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD,
+                      row_base + j * BK, v_full + 8 * s);
+          gb++;
+        }
       }
       // every copy this thread issued has landed before the CTA may exit
-      unsigned long long t0 = gtimer();
-      while (!mbar_try(q_full, 0) && gtimer() - t0 < WAIT_NS) {
-      }
-      for (int j = max(0, nj - STAGES); j < nj; j++) {
-        const int s = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
-        t0 = gtimer();
-        while (!mbar_try(k_full + 8 * s, ph) && gtimer() - t0 < WAIT_NS) {
-        }
-        while (!mbar_try(v_full + 8 * s, ph) && gtimer() - t0 < WAIT_NS) {
-        }
+      for (int i = max(0, nq - 2); i < nq; i++) drain_wait(q_full + 8 * (i & 1), (i >> 1) & 1);
+      for (int i = max(0, gb - STAGES); i < gb; i++) {
+        drain_wait(k_full + 8 * (i % STAGES), (i / STAGES) & 1);
+        drain_wait(v_full + 8 * (i % STAGES), (i / STAGES) & 1);
       }
     }
   } else if (warp == 1 || warp == MMA_B_WARP) {
@@ -174,66 +214,87 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int x = warp == 1 ? 0 : 1;  // which key half's P V this warp issues
     constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
     constexpr uint32_t ID_O = idesc_mn(128, HD, false, true);
-    const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
-    auto issue_s = [&](int j) {  // S = Q K_j^T into buffer j % 2
-      const int s = j % STAGES;
+    auto issue_s = [&](int slot, int gbn) {  // S = Q K^T of global block gbn into buffer gbn % 2
+      const int s = gbn % STAGES;
+      const uint64_t qd = sdesc(smem_u32(sQ + slot * TILE_BYTES), 16, 1024);
       const uint64_t kd = sdesc(smem_u32(sK + s * TILE_BYTES), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < HD / 16; kk++)
-        mma_bf16_e(tmem + COL_S + 128 * (j & 1), qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2),
-                   ID_S, kk > 0 ? 1u : 0u);
-      mma_commit_e(s_full + 8 * (j & 1));
+        mma_bf16_e(tmem + COL_S + 128 * (gbn & 1), qd + (uint64_t)(kk * 2),
+                   kd + (uint64_t)(kk * 2), ID_S, kk > 0 ? 1u : 0u);
+      mma_commit_e(s_full + 8 * (gbn & 1));
       mma_commit_e(k_empty + 8 * s);
     };
     bool ok = true;
-    if (x == 0) {
+    int gb = 0;
+    int item = sched_item(0, G, cta);
+    if (x == 0 && item < n_items) {  // scores of the first block
+      int qb, h, b;
+      decode(item, qb, h, b);
       ok = warp_wait(q_full, 0, abort_sh, gflag) && warp_wait(k_full, 0, abort_sh, gflag);
       if (ok) {
         fence_after();
-        issue_s(0);
+        issue_s(0, 0);
+        if (qb == 0) mma_commit_e(q_empty);  // the item's last S product on slot 0
       }
     }
-    for (int j = 0; j < nj && ok; j++) {
-      const int s = j % STAGES;
-      const uint32_t ph = (j / STAGES) & 1;
-      if (x == 0 && j + 1 < nj) {
-        // next block's scores into the other buffer once its P V products
-        // (block j - 1) have completed
-        const int s1 = (j + 1) % STAGES;
-        const uint32_t ph1 = ((j + 1) / STAGES) & 1;
-        if (!warp_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
-            (j >= 1 && !warp_wait(buf_free + 8 * ((j + 1) & 1), ((j - 1) >> 1) & 1, abort_sh,
-                                  gflag))) {
+    for (int r = 0, it = 0; item < n_items && ok; r++, it++) {
+      int qb, h, b;
+      decode(item, qb, h, b);
+      const int nj = qb + 1, slot = it & 1;
+      const int next = sched_item(r + 1, G, cta);
+      int qb_next = 0, hn, bn;
+      if (next < n_items) decode(next, qb_next, hn, bn);
+      for (int j = 0; j < nj && ok; j++, gb++) {
+        const int s = gb % STAGES;
+        const uint32_t ph = (gb / STAGES) & 1;
+        const bool here = j + 1 < nj;
+        if (x == 0 && (here || next < n_items)) {
+          // scores of block gb + 1 (this item's next, or the next item's
+          // first) into the other buffer once its P V products (block gb - 1)
+          // have completed
+          const int slot1 = here ? slot : slot ^ 1;
+          const int s1 = (gb + 1) % STAGES;
+          const uint32_t ph1 = ((gb + 1) / STAGES) & 1;
+          if ((!here && !warp_wait(q_full + 8 * slot1, ((it + 1) >> 1) & 1, abort_sh, gflag)) ||
+              !warp_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
+              (gb >= 1 && !warp_wait(buf_free + 8 * ((gb + 1) & 1), ((gb - 1) >> 1) & 1, abort_sh,
+                                     gflag))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          issue_s(slot1, gb + 1);
+          if (here ? (j + 1 == nj - 1) : (qb_next == 0)) mma_commit_e(q_empty + 8 * slot1);
+        }
+        if (!warp_wait(v_full + 8 * s, ph, abort_sh, gflag)) {
           ok = false;
           break;
         }
-        fence_after();
-        issue_s(j + 1);
-      }
-      if (!warp_wait(v_full + 8 * s, ph, abort_sh, gflag)) {
-        ok = false;
-        break;
-      }
-      const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 8192, 1024);
-      // O_g += P_g V[g KW : g KW + KW] for this warp's groups: KW / 16 K-steps
+        const uint64_t vd = sdesc(smem_u32(sV + s * TILE_BYTES), 8192, 1024);
+        // O_g += P_g V[g KW : g KW + KW] for this warp's groups: KW / 16 K-steps
+        // (at an item's first block the softmax warps arrive only after the
+        // previous item's accumulators were read out)
 #pragma unroll
-      for (int gg = 0; gg < NQ / 2; gg++) {
-        const int grp = x * (NQ / 2) + gg;
-        if (!warp_wait(p_full + 8 * grp, j & 1, abort_sh, gflag)) {
-          ok = false;
-          break;
+        for (int gg = 0; gg < NQ / 2; gg++) {
+          const int grp = x * (NQ / 2) + gg;
+          if (!warp_wait(p_full + 8 * ((gb & 1) * NQ + grp), (gb >> 1) & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+#pragma unroll
+          for (int kk = 0; kk < KW / 16; kk++)
+            mma_ts_e(tmem + COL_O + 64 * grp, tmem + COL_S + 128 * (gb & 1) + grp * KW + kk * 8,
+                     vd + (uint64_t)((grp * (KW / 16) + kk) * 128), ID_O,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_e(o_done + 8 * grp);
         }
-        fence_after();
-#pragma unroll
-        for (int kk = 0; kk < KW / 16; kk++)
-          mma_ts_e(tmem + COL_O + 64 * grp, tmem + COL_S + 128 * (j & 1) + grp * KW + kk * 8,
-                   vd + (uint64_t)((grp * (KW / 16) + kk) * 128), ID_O,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit_e(o_done + 8 * grp);
+        if (!ok) break;
+        mma_commit_e(v_empty + 8 * s);
+        mma_commit_e(buf_free + 8 * (gb & 1));
       }
-      if (!ok) break;
-      mma_commit_e(v_empty + 8 * s);
-      mma_commit_e(buf_free + 8 * (j & 1));
+      item = next;
     }
     mma_commit_e(drain + 8 * x);
     if (lane == 0) {
@@ -247,103 +308,110 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quarter = warp & 3;
     const int grp = (warp - 2) >> 2;    // key group: keys [grp KW, grp KW + KW) of a block
     const int r = quarter * 32 + lane;  // row of the tile = TMEM lane
-    const int qi = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t col_o = COL_O + 64 * grp;
     const float sl2 = scale * LOG2E;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nj && ok; j++) {
-      const uint32_t col_s = COL_S + 128 * (j & 1) + grp * KW;  // this group's S, then P
-      if (!warp_wait(s_full + 8 * (j & 1), (j >> 1) & 1, abort_sh, gflag)) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      const int k0 = j * BK + grp * KW;
-      const bool diag = (j * BK + BK > q0);  // only the diagonal block (or T) masks
-      float sv[KW];
-      tmem_ldn<KW>(tmem + lane_off + col_s, sv);
-      // this group's block maximum on the raw scores (the log2 factor sl2 > 0
-      // keeps the order), 4 independent chains; masked scores become -inf
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (diag) {  // the diagonal block (and keys past T): mask, then the maximum
-#pragma unroll
-        for (int i = 0; i < KW; i++) {
-          if (k0 + i > qi || k0 + i >= T) sv[i] = -INFINITY;
-          m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < KW; i++) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
-      }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
-      // true on the first block with an unmasked key (m_ref = -inf until then)
-      const bool need = mx > m_ref + LAZY;
-      // O_g is rescaled only after the previous block's P V into it completed
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        if (!warp_wait(o_done + 8 * grp, (j - 1) & 1, abort_sh, gflag)) {
+    int gb = 0;
+    for (int rr = 0, it = 0;; rr++, it++) {
+      const int item = sched_item(rr, G, cta);
+      if (item >= n_items) break;
+      int qb, h, b;
+      decode(item, qb, h, b);
+      const int q0 = qb * BQ, row_base = b * T, nj = qb + 1;
+      const int qi = q0 + r;
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nj && ok; j++, gb++) {
+        const uint32_t col_s = COL_S + 128 * (gb & 1) + grp * KW;  // this group's S, then P
+        if (!warp_wait(s_full + 8 * (gb & 1), (gb >> 1) & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-        {
-          const float corr = need ? ex2(m_ref - mx) : 1.f;  // 0 while m_ref = -inf
+        const int k0 = j * BK + grp * KW;
+        const bool diag = (j * BK + BK > q0);  // only the diagonal block (or T) masks
+        float sv[KW];
+        tmem_ldn<KW>(tmem + lane_off + col_s, sv);
+        // this group's block maximum on the raw scores (the log2 factor sl2 > 0
+        // keeps the order), 4 independent chains; masked scores become -inf
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (diag) {  // the diagonal block (and keys past T): mask, then the maximum
 #pragma unroll
-          for (int c = 0; c < 4; c++) {
-            float v[16];
-            uint32_t u[16];
-            tmem_ld16(tmem + lane_off + col_o + c * 16, v);
-#pragma unroll
-            for (int i = 0; i < 16; i++) u[i] = __float_as_uint(v[i] * corr);
-            tmem_st16(tmem + lane_off + col_o + c * 16, u);
+          for (int i = 0; i < KW; i++) {
+            if (k0 + i > qi || k0 + i >= T) sv[i] = -INFINITY;
+            m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
           }
-          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        } else {  // three-input maxima, 4 independent chains
+#pragma unroll
+          for (int i = 0; i < KW; i += 2)
+            m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], sv[i], sv[i + 1]);
         }
-      }
-      if (need) {
-        if (m_ref != -INFINITY) l *= ex2(m_ref - mx);
-        m_ref = mx;
-      }
-      // P = 2^(s - m_ref), packed bf16 into this group's KW/2 TMEM columns; a
-      // (row, group) with no unmasked key yet (m_ref = -inf) gets P = 0
-      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-      uint32_t w[KW / 2];
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+        // true on the first block with an unmasked key (m_ref = -inf until then)
+        const bool need = mx > m_ref + LAZY;
+        // O_g is rescaled only after the previous block's P V into it completed
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          if (!warp_wait(o_done + 8 * grp, (gb - 1) & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          {
+            const float corr = need ? ex2(m_ref - mx) : 1.f;  // 0 while m_ref = -inf
 #pragma unroll
-      for (int i = 0; i < KW; i += 2) {
-        const float p0 = ex2(fmaf(sv[i], sl2, -mr)), p1 = ex2(fmaf(sv[i + 1], sl2, -mr));
-        l4[(i >> 1) & 3] += p0 + p1;
-        w[i / 2] = pack_bf16(p0, p1);
+            for (int c = 0; c < 4; c++) {
+              float v[16];
+              uint32_t u[16];
+              tmem_ld16(tmem + lane_off + col_o + c * 16, v);
+#pragma unroll
+              for (int i = 0; i < 16; i++) u[i] = __float_as_uint(v[i] * corr);
+              tmem_st16(tmem + lane_off + col_o + c * 16, u);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          }
+        }
+        if (need) {
+          if (m_ref != -INFINITY) l *= ex2(m_ref - mx);
+          m_ref = mx;
+        }
+        // P = 2^(s - m_ref), packed bf16 into this group's KW/2 TMEM columns; a
+        // (row, group) with no unmasked key yet (m_ref = -inf) gets P = 0
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+        uint32_t w[KW / 2];
+        // the diagonal block on the SFU alone (its masked scores give exact
+        // zeros); elsewhere some pairs on the FMA pipe (exp2_pair)
+        l += diag ? exp_pack<false>(sv, sl2, mr, w) : exp_pack<true>(sv, sl2, mr, w);
+#pragma unroll
+        for (int c = 0; c < KW / 2; c += 16)
+          tmem_stn<(KW / 2 < 16 ? KW / 2 : 16)>(tmem + lane_off + col_s + c, w + c);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + 8 * ((gb & 1) * NQ + grp));
       }
-      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      // the groups meet: shared reference m, combined sum and output; every
+      // accumulator is complete once every o_done phase of the item's last
+      // block is
 #pragma unroll
-      for (int c = 0; c < KW / 2; c += 16)
-        tmem_stn<(KW / 2 < 16 ? KW / 2 : 16)>(tmem + lane_off + col_s + c, w + c);
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + 8 * grp);
-    }
-    // the groups meet: shared reference m, combined sum and output; every
-    // accumulator is complete once every o_done phase of the last block is
-#pragma unroll
-    for (int g2 = 0; g2 < NQ; g2++)
-      if (ok) ok = warp_wait(o_done + 8 * g2, (nj - 1) & 1, abort_sh, gflag);
-    red[grp * 128 + r] = m_ref;
-    red[(NQ + grp) * 128 + r] = l;
-    // barrier of the softmax warps that also tells whether every one finished
-    if (softmax_all(ok)) {
+      for (int g2 = 0; g2 < NQ; g2++)
+        if (ok) ok = warp_wait(o_done + 8 * g2, (gb - 1) & 1, abort_sh, gflag);
+      float *rd = red + (it & 1) * 2 * NQ * 128;
+      rd[grp * 128 + r] = m_ref;
+      rd[(NQ + grp) * 128 + r] = l;
+      // barrier of the softmax warps that also tells whether every one
+      // finished (each warp reaches it once per item, also after a failed
+      // wait, so all of them leave together)
+      if (!softmax_all(ok)) break;
       fence_after();
       float m = -INFINITY;
 #pragma unroll
-      for (int g2 = 0; g2 < NQ; g2++) m = fmaxf(m, red[g2 * 128 + r]);
+      for (int g2 = 0; g2 < NQ; g2++) m = fmaxf(m, rd[g2 * 128 + r]);
       float f[NQ], lt = 0.f;
 #pragma unroll
       for (int g2 = 0; g2 < NQ; g2++) {
-        const float mg = red[g2 * 128 + r];
+        const float mg = rd[g2 * 128 + r];
         f[g2] = mg == -INFINITY ? 0.f : ex2(mg - m);
-        lt += red[(NQ + g2) * 128 + r] * f[g2];
+        lt += rd[(NQ + g2) * 128 + r] * f[g2];
       }
       const float inv = 1.f / lt;
       // this thread's 64 / NQ output columns: [grp 64/NQ, grp 64/NQ + 64/NQ)
@@ -359,6 +427,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int i = 0; i < OW; i++) acc[i] += v[i] * cg;
       }
+      // every softmax warp has read every accumulator before any of them
+      // releases the next item's first P (whose P V overwrites O_g)
+      fence_before();
+      softmax_sync();
       if (qi < T) {
         __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + grp * OW;
 #pragma unroll
@@ -396,9 +468,9 @@ bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int 
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd;
   CUtensorMap map;
   if (!tc::tile_map_bf16(&map, qkv, qkvw, (int64_t)B * T, qkvw, 128)) return false;
-  dim3 grid(H, B, (T + BQ - 1) / BQ);
-  k_attn_fwd_tc<<<grid, NTHREADS, SMEM_BYTES, s>>>(map, (__nv_bfloat16 *)o, lse, T, H, Hkv,
-                                                   1.0f / sqrtf((float)hd), flag);
+  const int items = ((T + BQ - 1) / BQ) * H * B;
+  k_attn_fwd_tc<<<min(items, device_sms()), NTHREADS, SMEM_BYTES, s>>>(
+      map, (__nv_bfloat16 *)o, lse, B, T, H, Hkv, 1.0f / sqrtf((float)hd), flag);
   count_launch();
   return true;
 }

@@ -8,10 +8,9 @@
 // recomputed block by block so no T x T matrix reaches memory.  Two kernels,
 // both with 128 x 128 blocks, one CTA per SM (512 TMEM columns), 19 warps:
 //   warp 0      TMA producer (Q/dO or K/V once, the other pair through a
-//               2-deep ring);
-//   warps 1, 18 MMA issuers A and B (whole converged warps, one elected lane;
-//               one warp issues a tcgen05.mma only every ~127 cycles whatever
-//               N is, so the products are split between two warps); warp 1
+//               STAGES-deep ring);
+//   warps 1, 18 MMA issuers A and B (whole converged warps, one elected lane),
+//               each waiting only on the barriers of its own products; warp 1
 //               also allocates TMEM;
 //   warps 2..17 elementwise warps, four per TMEM lane quarter: thread = one
 //               row of the block (TMEM lane) and one column group (32 of the
@@ -31,11 +30,15 @@
 //   S^T = K Q^T (A) and dP^T = V dO^T (B) into TMEM; P^T and dS^T back into
 //   TMEM as bf16; dV += P^T dO (A) and dK += dS^T Q (B) (A operands from
 //   TMEM, B = dO / Q MN-major).
-//   The per-query L and D of each step travel with its Q/dO tiles.
+//   The per-query -L (log2 units) and -D of each step travel with its Q/dO
+//   tiles.
 // dQ and dK leave through the backward of the rotate-half RoPE (when tables
 // are given), then scale, bf16.  No atomics: every output element is written
-// once by the CTA that owns its row.  Every wait is bounded (FLAG_TIMEOUT,
-// then drain and free TMEM).
+// once by the CTA that owns its row.  The elementwise arithmetic runs on
+// packed f32x2 pairs, and 5 of every 16 pairs of exponentials take the
+// polynomial 2^x on the FMA pipe (exp2_poly2) so that the SFU (16 results per
+// clock and SM) does not bound the loop alone.  Every wait is bounded
+// (FLAG_TIMEOUT, then drain and free TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "tcgen05.cuh"
@@ -57,17 +60,17 @@ constexpr int NTHREADS = 32 * (MMA_B_WARP + 1);
 constexpr int TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 
-// dQ kernel: TMEM columns; shared memory Q | dO | K[2] | V[2] | barriers | red
+// dQ kernel: TMEM columns; shared memory Q[2] | dO[2] | O | K[STAGES] | V[STAGES] |
+// barriers | red[2] | -L
 constexpr int DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DS = 256, DQ_COL_DQA = 320, DQ_COL_DQB = 384;
 constexpr int BAR_BYTES = 512;  // 48 mbarrier slots, then the TMEM address and abort words
-constexpr int DQ_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 1024 + BAR_BYTES + NCQ * 128 * 4;
-// dK/dV kernel: TMEM columns; shared memory K | V | Q[2] | dO[2] | L[2] | D[2] | barriers
+constexpr int DQ_SMEM =
+    (5 + 2 * STAGES) * TILE_BYTES + 1024 + BAR_BYTES + 2 * NCQ * 128 * 4 + 128 * 4;
+// dK/dV kernel: TMEM columns; shared memory K[2] | V[2] | Q[STAGES] | dO[STAGES] |
+// L[STAGES] | D[STAGES] | barriers
 constexpr int KV_COL_S = 0, KV_COL_DP = 128, KV_COL_P = 256, KV_COL_DS = 320, KV_COL_DV = 384,
               KV_COL_DK = 448;
-constexpr int KV_SMEM = (2 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + BAR_BYTES + 1024;
-
-// Named barrier of the elementwise warps (id 1).
-LLM_DEV void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EW_WARPS) : "memory"); }
+constexpr int KV_SMEM = (4 + 2 * STAGES) * TILE_BYTES + 2 * STAGES * 128 * 4 + BAR_BYTES + 1024;
 
 // Backward of the rotate-half RoPE on N column pairs (c, c + 32) of one row:
 // (x, y) <- (x cos + y sin, y cos - x sin), angle table entries ct[i], st[i].
@@ -98,6 +101,16 @@ LLM_DEV void store_n(__nv_bfloat16 *dst, const float (&v)[N], float mul) {
                    pack_bf16(v[i + 4] * mul, v[i + 5] * mul), pack_bf16(v[i + 6] * mul, v[i + 7] * mul));
 }
 
+// N (8) values times mul as bf16 into 16-byte chunk c of a 128-byte row r of a
+// tile in the 128-byte-swizzle layout of its tensor map (chunk c at c ^ (r & 7)).
+template <int N>
+LLM_DEV void stage_n(uint8_t *row, int c, int r, const float (&v)[N], float mul) {
+  static_assert(N == 8, "one 16-byte chunk");
+  *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) =
+      make_uint4(pack_bf16(v[0] * mul, v[1] * mul), pack_bf16(v[2] * mul, v[3] * mul),
+                 pack_bf16(v[4] * mul, v[5] * mul), pack_bf16(v[6] * mul, v[7] * mul));
+}
+
 LLM_DEV void tmem_alloc_512(uint32_t *dst) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst)),
@@ -109,48 +122,64 @@ LLM_DEV void tmem_free_512(uint32_t tmem) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                : "memory");
 }
-// Bounded wait used only on the way out (the copies / MMAs of this thread).
-LLM_DEV void drain_wait(uint32_t bar, uint32_t parity) {
-  const unsigned long long t0 = gtimer();
-  while (!mbar_try(bar, parity) && gtimer() - t0 < WAIT_NS) {
-  }
-}
 
 // ------------------------------------------------------------------- dQ
+// Persistent: gridDim.x CTAs (one per SM) walk the items (query block, head,
+// batch), longest rows first, in the snake of sched_item.  Per item the
+// producer loads Q and dO into slot it % 2, O (for D) and -L into single
+// buffers, then streams the item's K_j, V_j through the ring.  The ring, the
+// S/dP and dS barriers count key blocks over all of a CTA's items (gb), so
+// the next item's tiles land and its first products run while this item's
+// last blocks and epilogue are still in flight.
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_dq_tc(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                 const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dout,
-                 const float *__restrict__ lse, float *__restrict__ Dv,
-                 __nv_bfloat16 *__restrict__ dqkv, const float *__restrict__ cos_t,
-                 const float *__restrict__ sin_t, int T, int H, int Hkv, float scale, int *gflag) {
+                 const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_st,
+                 const float *__restrict__ lse,
+                 float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
+                 const float *__restrict__ cos_t, const float *__restrict__ sin_t, int B, int T,
+                 int H, int Hkv, float scale, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sQ = smem, *sdO = smem + TILE_BYTES, *sK = smem + 2 * TILE_BYTES,
-          *sV = sK + STAGES * TILE_BYTES;
+  uint8_t *sQ = smem, *sdO = smem + 2 * TILE_BYTES, *sO = smem + 4 * TILE_BYTES,
+          *sK = smem + 5 * TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
   uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
-  float *red = (float *)(bars + BAR_BYTES / 8);  // [NCQ][128] partial dot products
+  float *red = (float *)(bars + BAR_BYTES / 8);  // [2][NCQ][128] partial dot products
+  float *sNL = red + 2 * NCQ * 128;              // [128] -L log2(e) of the item's rows
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t q_full = b0, k_full = b0 + 8, k_empty = k_full + 8 * STAGES,
-                 v_full = k_empty + 8 * STAGES, v_empty = v_full + 8 * STAGES,
-                 s_full = v_empty + 8 * STAGES, s_free = s_full + 8,
-                 ds_full = s_free + 8,   // [2]: key half a, b
-                 dq_done = ds_full + 16, // [2]
-                 drain = dq_done + 16;   // [2]: one per MMA warp
-  static_assert(3 + 4 * STAGES + 6 <= 48, "barriers overlap the TMEM address word");
+  const uint32_t qd_full = b0, qd_empty = b0 + 16,  // [2]: Q/dO slot
+                 o_full = b0 + 32, o_empty = b0 + 40, k_full = b0 + 48,
+                 k_empty = k_full + 8 * STAGES, v_full = k_empty + 8 * STAGES,
+                 v_empty = v_full + 8 * STAGES, s_full = v_empty + 8 * STAGES, s_free = s_full + 8,
+                 ds_full = s_free + 8,    // [2]: key half a, b
+                 dq_done = ds_full + 16,  // [2]
+                 red_full = dq_done + 16, acc_free = red_full + 8,
+                 drain = acc_free + 8,    // [2]: one per MMA warp
+                 qsync = drain + 16;      // [4]: per lane quarter, its rows of dQ staged
+  static_assert(6 + 4 * STAGES + 14 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int nqb = gridDim.z, qb = nqb - 1 - blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int g = h / (H / Hkv), d = H * HD, kvd = Hkv * HD;
-  const int64_t ld = d + 2 * kvd;
-  const int q0 = qb * BQ;
-  const int nj = qb + 1;  // causal: key blocks 0..qb (block qb holds the diagonal)
-  const int row_base = b * T;
+  const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int d = H * HD, kvd = Hkv * HD;
+  // item -> (query block, head, batch), longest rows (last query blocks) first
+  auto decode = [&](int item, int &qb, int &h, int &b) {
+    const int z = item / (H * B), rem = item - z * (H * B);
+    qb = nqb - 1 - z;
+    h = rem % H;
+    b = rem / H;
+  };
 
   if (threadIdx.x == 0) {
     *abort_sh = 0;
-    mbar_init(q_full, 1);
+    for (int x = 0; x < 2; x++) {
+      mbar_init(qd_full + 8 * x, 1);
+      // both products' last MMAs on the slot, every elementwise thread's D,
+      // and the bulk stores of dQ staged in the slot's Q tile (one per warp)
+      mbar_init(qd_empty + 8 * x, 2 + 32 * EW_WARPS + EW_WARPS);
+    }
+    mbar_init(o_full, 1 + 32);  // the tile's expect-tx arrival and the 32 lanes writing -L
+    mbar_init(o_empty, 32 * EW_WARPS);  // every elementwise thread read its O row and -L
     for (int s = 0; s < STAGES; s++) {
       mbar_init(k_full + 8 * s, 1);
       mbar_init(k_empty + 8 * s, 2);  // dQ_a and dQ_b read K_j
@@ -164,6 +193,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(dq_done + 8 * x, 1);
       mbar_init(drain + 8 * x, 1);
     }
+    mbar_init(red_full, 32 * EW_WARPS);
+    mbar_init(acc_free, EW_WARPS);  // the accumulators of the item were read out
+    for (int q = 0; q < 4; q++) mbar_init(qsync + 8 * q, 32 * NCQ);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_512(tmem_sh);
@@ -173,44 +205,80 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_sh;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------ TMA producer
-      int issued = 0;
-      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
-      tma_load_2d(smem_u32(sQ), &tm_qkv, h * HD, row_base + q0, q_full);
-      tma_load_2d(smem_u32(sdO), &tm_do, h * HD, row_base + q0, q_full);
-      for (int j = 0; j < nj; j++) {
-        const int s = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
-        if (!mbar_wait(k_empty + 8 * s, ph ^ 1, abort_sh, gflag)) break;
-        if (!mbar_wait(v_empty + 8 * s, ph ^ 1, abort_sh, gflag)) break;
-        mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
-        tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
-                    k_full + 8 * s);
-        mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
-        tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD, row_base + j * BK,
-                    v_full + 8 * s);
-        issued = j + 1;
+    // ---------------------------------------------- TMA producer (warp)
+    int gb = 0, nqd = 0, no = 0;  // key blocks, Q/dO tiles and O tiles issued
+    bool ok = true;
+    for (int r = 0, it = 0; ok; r++, it++) {
+      const int item = sched_item(r, G, cta);
+      if (item >= n_items) break;
+      int qb, h, b;
+      decode(item, qb, h, b);
+      const int q0 = qb * BQ, row_base = b * T, g = h / (H / Hkv), slot = it & 1;
+      // Q, dO into the slot of item it - 2 once it was released
+      if (!warp_wait(qd_empty + 8 * slot, ((it >> 1) & 1) ^ 1, abort_sh, gflag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(qd_full + 8 * slot, 2 * TILE_BYTES);
+        tma_load_2d(smem_u32(sQ + slot * TILE_BYTES), &tm_qkv, h * HD, row_base + q0,
+                    qd_full + 8 * slot);
+        tma_load_2d(smem_u32(sdO + slot * TILE_BYTES), &tm_do, h * HD, row_base + q0,
+                    qd_full + 8 * slot);
       }
-      // every copy this thread issued has landed before the CTA may exit
-      drain_wait(q_full, 0);
-      for (int j = max(0, issued - STAGES); j < issued; j++) {
-        drain_wait(k_full + 8 * (j % STAGES), (j / STAGES) & 1);
-        drain_wait(v_full + 8 * (j % STAGES), (j / STAGES) & 1);
+      nqd = it + 1;
+      // O and -L once the elementwise warps have formed D of item it - 1
+      if (!warp_wait(o_empty, (it & 1) ^ 1, abort_sh, gflag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(o_full, TILE_BYTES);
+        tma_load_2d(smem_u32(sO), &tm_o, h * HD, row_base + q0, o_full);
+      }
+      const int64_t lbase = ((int64_t)b * H + h) * T;
+      for (int i = lane; i < BQ; i += 32) {
+        const int qi = q0 + i;
+        // rows past T get -L = -inf, so every P of theirs is 0
+        sNL[i] = qi < T ? -lse[lbase + qi] * LOG2E : -INFINITY;
+      }
+      mbar_arrive(o_full);
+      no = it + 1;
+      for (int j = 0; j <= qb; j++) {
+        const int s = gb % STAGES;
+        const uint32_t ph = (gb / STAGES) & 1;
+        if (!warp_wait(k_empty + 8 * s, ph ^ 1, abort_sh, gflag) ||
+            !warp_wait(v_empty + 8 * s, ph ^ 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
+          tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
+                      k_full + 8 * s);
+          mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
+          tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD,
+                      row_base + j * BK, v_full + 8 * s);
+        }
+        gb++;
       }
     }
+    // every copy this warp issued has landed before the CTA may exit
+    if (lane == 0) {
+      for (int i = max(0, nqd - 2); i < nqd; i++) drain_wait(qd_full + 8 * (i & 1), (i >> 1) & 1);
+      if (no > 0) drain_wait(o_full, (no - 1) & 1);
+      for (int i = max(0, gb - STAGES); i < gb; i++) {
+        drain_wait(k_full + 8 * (i % STAGES), (i / STAGES) & 1);
+        drain_wait(v_full + 8 * (i % STAGES), (i / STAGES) & 1);
+      }
+    }
+    __syncwarp();
   } else if (warp == 1 || warp == MMA_B_WARP) {
     // ------------------------------------- MMA issuers (whole warps)
     // A: S = Q K_j^T, dQ_a += dS_a K_j[0:64];  B: dP = dO V_j^T, dQ_b += dS_b K_j[64:128]
     const int x = warp == 1 ? 0 : 1;
     constexpr uint32_t ID_S = idesc_mn(128, BK, false, false);
     constexpr uint32_t ID_DQ = idesc_mn(128, HD, false, true);
-    const uint64_t ad = sdesc(smem_u32(x ? sdO : sQ), 16, 1024);
+    uint8_t *sA = x ? sdO : sQ;
     uint8_t *sB = x ? sV : sK;
     const uint32_t b_full = x ? v_full : k_full;
     const uint32_t col = x ? DQ_COL_DP : DQ_COL_S;
-    auto issue_prod = [&](int j) {
-      const int s = j % STAGES;
+    auto issue_prod = [&](int slot, int s) {
+      const uint64_t ad = sdesc(smem_u32(sA + slot * TILE_BYTES), 16, 1024);
       const uint64_t bd = sdesc(smem_u32(sB + s * TILE_BYTES), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < HD / 16; kk++)
@@ -219,39 +287,64 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mma_commit_e(s_full);
       if (x) mma_commit_e(v_empty + 8 * s);  // V_j is not read again
     };
-    bool ok = warp_wait(q_full, 0, abort_sh, gflag) && warp_wait(b_full, 0, abort_sh, gflag);
-    if (ok) {
-      fence_after();
-      issue_prod(0);
+    bool ok = true;
+    int gb = 0;
+    int item = sched_item(0, G, cta);
+    if (item < n_items) {  // products of the first block
+      int qb, h, b;
+      decode(item, qb, h, b);
+      ok = warp_wait(qd_full, 0, abort_sh, gflag) && warp_wait(b_full, 0, abort_sh, gflag);
+      if (ok) {
+        fence_after();
+        issue_prod(0, 0);
+        if (qb == 0) mma_commit_e(qd_empty);  // the item's last products on slot 0
+      }
     }
-    for (int j = 0; j < nj && ok; j++) {
-      const int s = j % STAGES;
-      const uint32_t ph = (j / STAGES) & 1;
-      if (j + 1 < nj) {
-        // next block's products once the elementwise warps have read S, dP
-        const int s1 = (j + 1) % STAGES;
-        const uint32_t ph1 = ((j + 1) / STAGES) & 1;
-        if (!warp_wait(b_full + 8 * s1, ph1, abort_sh, gflag) ||
-            !warp_wait(s_free, j & 1, abort_sh, gflag)) {
+    for (int r = 0, it = 0; item < n_items && ok; r++, it++) {
+      int qb, h, b;
+      decode(item, qb, h, b);
+      const int nj = qb + 1, slot = it & 1;
+      const int next = sched_item(r + 1, G, cta);
+      int qb_next = 0, hn, bn;
+      if (next < n_items) decode(next, qb_next, hn, bn);
+      for (int j = 0; j < nj && ok; j++, gb++) {
+        const int s = gb % STAGES;
+        const uint32_t ph = (gb / STAGES) & 1;
+        // products of block gb + 1 (this item's next, or the next item's first)
+        // once the elementwise warps have read S and dP of block gb
+        const bool here = j + 1 < nj;
+        if (here || next < n_items) {
+          const int slot1 = here ? slot : slot ^ 1;
+          const int s1 = (gb + 1) % STAGES;
+          const uint32_t ph1 = ((gb + 1) / STAGES) & 1;
+          if ((!here && !warp_wait(qd_full + 8 * slot1, ((it + 1) >> 1) & 1, abort_sh, gflag)) ||
+              !warp_wait(b_full + 8 * s1, ph1, abort_sh, gflag) ||
+              !warp_wait(s_free, gb & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          issue_prod(slot1, s1);
+          // the last products that read this Q/dO slot
+          if (here ? (j + 1 == nj - 1) : (qb_next == 0)) mma_commit_e(qd_empty + 8 * slot1);
+        }
+        // dQ_x += dS_x K_j[x half]; the accumulators of the previous item were read out
+        if ((j == 0 && it > 0 && !warp_wait(acc_free, (it - 1) & 1, abort_sh, gflag)) ||
+            !warp_wait(ds_full + 8 * x, gb & 1, abort_sh, gflag) ||
+            (x && !warp_wait(k_full + 8 * s, ph, abort_sh, gflag))) {
           ok = false;
           break;
         }
         fence_after();
-        issue_prod(j + 1);
-      }
-      if (!warp_wait(ds_full + 8 * x, j & 1, abort_sh, gflag) ||
-          (x && !warp_wait(k_full + 8 * s, ph, abort_sh, gflag))) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      const uint64_t kmd = sdesc(smem_u32(sK + s * TILE_BYTES), 8192, 1024);
+        const uint64_t kmd = sdesc(smem_u32(sK + s * TILE_BYTES), 8192, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 4; kk++)
-        mma_ts_e(tmem + (x ? DQ_COL_DQB : DQ_COL_DQA), tmem + DQ_COL_DS + x * 32 + kk * 8,
-                 kmd + (uint64_t)((x * 4 + kk) * 128), ID_DQ, (j > 0 || kk > 0) ? 1u : 0u);
-      mma_commit_e(k_empty + 8 * s);
-      mma_commit_e(dq_done + 8 * x);
+        for (int kk = 0; kk < 4; kk++)
+          mma_ts_e(tmem + (x ? DQ_COL_DQB : DQ_COL_DQA), tmem + DQ_COL_DS + x * 32 + kk * 8,
+                   kmd + (uint64_t)((x * 4 + kk) * 128), ID_DQ, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_e(k_empty + 8 * s);
+        mma_commit_e(dq_done + 8 * x);
+      }
+      item = next;
     }
     mma_commit_e(drain + 8 * x);
     if (lane == 0) drain_wait(drain + 8 * x, 0);
@@ -262,87 +355,116 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int cq = (warp - 2) >> 2;  // column group: keys [cq CW, cq CW + CW) of the block
     const int x = cq / (NCQ / 2);    // key half (dQ_a or dQ_b) this group feeds
     const int r = quarter * 32 + lane;
-    const int qi = q0 + r;
-    const bool valid = qi < T;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = scale * LOG2E;
-    // D_i = dO_i . O_i, each thread over 64 / NCQ of the 64 head columns
-    float dpart = 0.f;
-    if (valid) {
-      const int64_t off = ((int64_t)row_base + qi) * d + h * HD + cq * (HD / NCQ);
-      const uint4 *po = reinterpret_cast<const uint4 *>(o + off);
-      const uint4 *pd = reinterpret_cast<const uint4 *>(dout + off);
-#pragma unroll
-      for (int e = 0; e < HD / NCQ / 8; e++) {
-        const uint4 a = po[e], c = pd[e];
-        const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
-        const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&c);
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-          const float2 fa = __bfloat1622float2(ha[k]), fc = __bfloat1622float2(hc[k]);
-          dpart += fa.x * fc.x + fa.y * fc.y;
-        }
-      }
-    }
-    red[cq * 128 + r] = dpart;
-    ew_sync();
-    float Di = 0.f;
-#pragma unroll
-    for (int c = 0; c < NCQ; c++) Di += red[c * 128 + r];
-    // rows past T get L = +inf, so every P of theirs is 0
-    const float L2 = valid ? lse[((int64_t)b * H + h) * T + qi] * LOG2E : INFINITY;
-    if (cq == 0 && valid) Dv[((int64_t)b * H + h) * T + qi] = Di;
     bool ok = true;
-    for (int j = 0; j < nj && ok; j++) {
-      if (!warp_wait(s_full, j & 1, abort_sh, gflag)) {
+    int gb = 0;
+    for (int rr = 0, it = 0; ok; rr++, it++) {
+      const int item = sched_item(rr, G, cta);
+      if (item >= n_items) break;
+      int qb, h, b;
+      decode(item, qb, h, b);
+      const int q0 = qb * BQ, nj = qb + 1, slot = it & 1;
+      const int qi = q0 + r;
+      const bool valid = qi < T;
+      if (!warp_wait(o_full, it & 1, abort_sh, gflag) ||
+          !warp_wait(qd_full + 8 * slot, (it >> 1) & 1, abort_sh, gflag)) {
         ok = false;
         break;
       }
-      fence_after();
-      float sv[CW], dv[CW];
-      tmem_ldn<CW>(tmem + lane_off + DQ_COL_S + cq * CW, sv);
-      tmem_ldn<CW>(tmem + lane_off + DQ_COL_DP + cq * CW, dv);
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);  // the MMA warps may overwrite S and dP now
-      const int k0 = j * BK + cq * CW;
-      const bool diag = (j == qb);  // only the diagonal block masks (keys >= T lie above it)
-      uint32_t w[CW / 2];
-      if (diag) {  // the causal mask only on the diagonal block
+      // D_i = dO_i . O_i over this thread's 64 / NCQ head columns, from the
+      // tiles in shared memory (128-byte swizzle: 16-byte chunk c of row r at
+      // position c ^ (r & 7))
+      float dpart = 0.f;
+      {
+        const uint8_t *ro = sO + r * 128, *rdo = sdO + slot * TILE_BYTES + r * 128;
 #pragma unroll
-        for (int i = 0; i < CW; i += 2) {
-          float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
-          if (k0 + i > qi) p0 = 0.f;
-          if (k0 + i + 1 > qi) p1 = 0.f;
-          w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
-        }
-      } else {
+        for (int e = 0; e < HD / NCQ / 8; e++) {
+          const int c = ((cq * (HD / NCQ / 8) + e) ^ (r & 7)) << 4;
+          const uint4 a = *reinterpret_cast<const uint4 *>(ro + c);
+          const uint4 cc = *reinterpret_cast<const uint4 *>(rdo + c);
+          const __nv_bfloat162 *ha = reinterpret_cast<const __nv_bfloat162 *>(&a);
+          const __nv_bfloat162 *hc = reinterpret_cast<const __nv_bfloat162 *>(&cc);
 #pragma unroll
-        for (int i = 0; i < CW; i += 2) {
-          const float p0 = ex2(fmaf(sv[i], sl2, -L2)), p1 = ex2(fmaf(sv[i + 1], sl2, -L2));
-          w[i / 2] = pack_bf16(p0 * (dv[i] - Di), p1 * (dv[i + 1] - Di));
+          for (int k = 0; k < 4; k++) {
+            const float2 fa = __bfloat1622float2(ha[k]), fc = __bfloat1622float2(hc[k]);
+            dpart += fa.x * fc.x + fa.y * fc.y;
+          }
         }
       }
-      // this half's dS of the previous block is free once its dQ product completed
-      if (j > 0) {
-        if (!warp_wait(dq_done + 8 * x, (j - 1) & 1, abort_sh, gflag)) {
+      const float nl2 = sNL[r];
+      mbar_arrive(o_empty);              // this thread's O row and -L consumed
+      mbar_arrive(qd_empty + 8 * slot);  // and its dO row
+      float *rd = red + (it & 1) * NCQ * 128;
+      rd[cq * 128 + r] = dpart;
+      mbar_arrive(red_full);
+      if (!warp_wait(red_full, it & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
+      float Di = 0.f;
+#pragma unroll
+      for (int c = 0; c < NCQ; c++) Di += rd[c * 128 + r];
+      if (cq == 0 && valid) Dv[((int64_t)b * H + h) * T + qi] = Di;
+      const float2 nl = make_float2(nl2, nl2), nd = make_float2(-Di, -Di);
+      for (int j = 0; j < nj && ok; j++, gb++) {
+        if (!warp_wait(s_full, gb & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-      }
+        float sv[CW], dv[CW];
+        tmem_ldn<CW>(tmem + lane_off + DQ_COL_S + cq * CW, sv);
+        tmem_ldn<CW>(tmem + lane_off + DQ_COL_DP + cq * CW, dv);
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);  // the MMA warps may overwrite S and dP now
+        const int k0 = j * BK + cq * CW;
+        const bool diag = (j == qb);  // only the diagonal block masks (keys >= T lie above it)
+        uint32_t w[CW / 2];
+        if (diag) {  // the causal mask only on the diagonal block
 #pragma unroll
-      for (int c = 0; c < CW / 2; c += 16)
-        tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + DQ_COL_DS + cq * (CW / 2) + c, w + c);
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full + 8 * x);
-    }
-    if (ok)
-      ok = warp_wait(dq_done, (nj - 1) & 1, abort_sh, gflag) &&
-           warp_wait(dq_done + 8, (nj - 1) & 1, abort_sh, gflag);
-    if (ok) {
+          for (int i = 0; i < CW; i += 2) {
+            float2 p = exp2_pair(
+                __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2), nl), i / 2);
+            if (k0 + i > qi) p.x = 0.f;
+            if (k0 + i + 1 > qi) p.y = 0.f;
+            const float2 ds = __fmul2_rn(p, __fadd2_rn(make_float2(dv[i], dv[i + 1]), nd));
+            w[i / 2] = pack_bf16(ds.x, ds.y);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < CW; i += 2) {
+            const float2 p = exp2_pair(
+                __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2), nl), i / 2);
+            const float2 ds = __fmul2_rn(p, __fadd2_rn(make_float2(dv[i], dv[i + 1]), nd));
+            w[i / 2] = pack_bf16(ds.x, ds.y);
+          }
+        }
+        // this half's dS of the previous block is free once its dQ product
+        // completed (at an item's first block the epilogue already waited)
+        if (j > 0) {
+          if (!warp_wait(dq_done + 8 * x, (gb - 1) & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+        }
+#pragma unroll
+        for (int c = 0; c < CW / 2; c += 16)
+          tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + DQ_COL_DS + cq * (CW / 2) + c,
+                                               w + c);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full + 8 * x);
+      }
+      if (!ok) break;
+      if (!warp_wait(dq_done, (gb - 1) & 1, abort_sh, gflag) ||
+          !warp_wait(dq_done + 8, (gb - 1) & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
       fence_after();
       // column pairs (c, c + 32) of RoPE: this group takes c in [cq HW, cq HW + HW)
       float xa[HW], ya[HW], xb[HW], yb[HW];
@@ -350,20 +472,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + 32 + cq * HW, ya);
       tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + cq * HW, xb);
       tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + 32 + cq * HW, yb);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_free);  // the next item's dQ products may start
 #pragma unroll
       for (int i = 0; i < HW; i++) {
         xa[i] += xb[i];
         ya[i] += yb[i];
       }
-      if (valid) {
-        if (cos_t)
-          rope_bwd_n<HW>(xa, ya, cos_t + (int64_t)qi * (HD / 2) + cq * HW,
-                         sin_t + (int64_t)qi * (HD / 2) + cq * HW);
-        __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + qi) * ld + h * HD + cq * HW;
-        store_n<HW>(dst, xa, scale);
-        store_n<HW>(dst + 32, ya, scale);
+      if (valid && cos_t)
+        rope_bwd_n<HW>(xa, ya, cos_t + (int64_t)qi * (HD / 2) + cq * HW,
+                       sin_t + (int64_t)qi * (HD / 2) + cq * HW);
+      // dQ rows through the item's Q tile (its products are complete): the
+      // 128-byte-swizzle image of the tile, then each warp stores 8 whole rows
+      // of its lane quarter with one bulk tensor copy (rows past T clipped)
+      uint8_t *srow = sQ + slot * TILE_BYTES + r * 128;
+      stage_n<HW>(srow, cq, r, xa, scale);
+      stage_n<HW>(srow, 4 + cq, r, ya, scale);
+      fence_proxy_async();
+      mbar_arrive(qsync + 8 * quarter);
+      if (!warp_wait(qsync + 8 * quarter, it & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
       }
+      if (lane == 0) {
+        const int r0 = quarter * 32 + cq * 8;
+        tma_store_3d(&tm_st, smem_u32(sQ + slot * TILE_BYTES + r0 * 128), h * HD, q0 + r0, b);
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(qd_empty + 8 * slot);
+      }
+      __syncwarp();
     }
+    if (lane == 0) bulk_wait_all();
   }
   fence_before();
   __syncthreads();
@@ -372,40 +513,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // ---------------------------------------------------------------- dK, dV
+// Persistent like the dQ kernel: items (key block, kv head, batch), first key
+// blocks (the most query blocks) first; K and V of item it in slot it % 2,
+// the (query head, query block) steps of all of a CTA's items through one
+// ring (global step gs), so the next item's first products start while this
+// item's last accumulations and epilogue run.
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_dkv_tc(const __grid_constant__ CUtensorMap tm_qkv,
-                  const __grid_constant__ CUtensorMap tm_do, const float *__restrict__ lse,
+                  const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_st,
+                  const float *__restrict__ lse,
                   const float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
-                  const float *__restrict__ cos_t, const float *__restrict__ sin_t, int T, int H,
-                  int Hkv, float scale, int *gflag) {
+                  const float *__restrict__ cos_t, const float *__restrict__ sin_t, int B, int T,
+                  int H, int Hkv, float scale, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sK = smem, *sV = smem + TILE_BYTES, *sQ = smem + 2 * TILE_BYTES,
+  uint8_t *sK = smem, *sV = smem + 2 * TILE_BYTES, *sQ = smem + 4 * TILE_BYTES,
           *sdO = sQ + STAGES * TILE_BYTES;
-  float *sL = (float *)(sdO + STAGES * TILE_BYTES);  // [STAGES][128] L * log2(e)
-  float *sD = sL + STAGES * 128;                      // [STAGES][128] D
+  float *sL = (float *)(sdO + STAGES * TILE_BYTES);  // [STAGES][128] -L * log2(e)
+  float *sD = sL + STAGES * 128;                      // [STAGES][128] -D
   uint64_t *bars = (uint64_t *)(sD + STAGES * 128);
   uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t kv_full = b0, q_full = b0 + 8, q_empty = q_full + 8 * STAGES,
+  const uint32_t kv_full = b0, kv_empty = b0 + 16,  // [2]: K/V slot
+                 q_full = b0 + 32, q_empty = q_full + 8 * STAGES,
                  ld_full = q_empty + 8 * STAGES, s_full = ld_full + 8 * STAGES,
                  s_free = s_full + 8, p_full = s_free + 8, pv_done = p_full + 8,
-                 drain = pv_done + 8;  // drain [2]: one per MMA warp
-  static_assert(1 + 3 * STAGES + 6 <= 48, "barriers overlap the TMEM address word");
+                 drain = pv_done + 8,  // drain [2]: one per MMA warp
+                 qsync = drain + 16;   // [4]: per lane quarter, its rows of dK, dV staged
+  static_assert(4 + 3 * STAGES + 10 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int nkb = gridDim.z, kb = blockIdx.z;
-  const int g = blockIdx.x, b = blockIdx.y;
+  const int nkb = (T + BK - 1) / BK, n_items = nkb * Hkv * B;
+  const int G = gridDim.x, cta = blockIdx.x;
   const int grp = H / Hkv, d = H * HD, kvd = Hkv * HD;
-  const int64_t ld = d + 2 * kvd;
-  const int k0 = kb * BK;
-  const int nq = nkb - kb;       // query blocks kb..nkb-1 see this key block
-  const int nsteps = grp * nq;   // (query head of the group, query block) pairs
-  const int row_base = b * T;
+  // item -> (key block, kv head, batch); steps = grp (nkb - kb)
+  auto decode = [&](int item, int &kb, int &g, int &b) {
+    kb = item / (Hkv * B);
+    const int rem = item - kb * (Hkv * B);
+    g = rem % Hkv;
+    b = rem / Hkv;
+  };
 
   if (threadIdx.x == 0) {
     *abort_sh = 0;
-    mbar_init(kv_full, 1);
+    for (int x = 0; x < 2; x++) {
+      mbar_init(kv_full + 8 * x, 1);
+      // both MMA warps' last products on the slot, and the bulk stores of dK
+      // and dV staged in the slot (one per elementwise warp)
+      mbar_init(kv_empty + 8 * x, 2 + EW_WARPS);
+    }
     for (int s = 0; s < STAGES; s++) {
       mbar_init(q_full + 8 * s, 1);
       mbar_init(q_empty + 8 * s, 2);  // both MMA warps read Q_s and dO_s
@@ -417,6 +573,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(pv_done, 2);  // dV and dK
     mbar_init(drain, 1);
     mbar_init(drain + 8, 1);
+    for (int q = 0; q < 4; q++) mbar_init(qsync + 8 * q, 32 * NCQ);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_512(tmem_sh);
@@ -427,54 +584,71 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (warp)
-    if (lane == 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * TILE_BYTES);
-      tma_load_2d(smem_u32(sK), &tm_qkv, d + g * HD, row_base + k0, kv_full);
-      tma_load_2d(smem_u32(sV), &tm_qkv, d + kvd + g * HD, row_base + k0, kv_full);
-    }
-    int issued = 0;
-    for (int st = 0; st < nsteps; st++) {
-      const int s = st % STAGES;
-      const uint32_t ph = (st / STAGES) & 1;
-      const int hq = g * grp + st / nq, qb = kb + st % nq;
-      // the slot (tiles and L, D) of step st - 2 is free once its products completed
-      if (!warp_wait(q_empty + 8 * s, ph ^ 1, abort_sh, gflag)) break;
+    int gs = 0, nkv = 0;  // steps and K/V tiles issued
+    bool ok = true;
+    for (int r = 0, it = 0; ok; r++, it++) {
+      const int item = sched_item(r, G, cta);
+      if (item >= n_items) break;
+      int kb, g, b;
+      decode(item, kb, g, b);
+      const int k0 = kb * BK, row_base = b * T, nq = nkb - kb, slot = it & 1;
+      if (!warp_wait(kv_empty + 8 * slot, ((it >> 1) & 1) ^ 1, abort_sh, gflag)) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full + 8 * s, 2 * TILE_BYTES);
-        tma_load_2d(smem_u32(sQ + s * TILE_BYTES), &tm_qkv, hq * HD, row_base + qb * BQ,
-                    q_full + 8 * s);
-        tma_load_2d(smem_u32(sdO + s * TILE_BYTES), &tm_do, hq * HD, row_base + qb * BQ,
-                    q_full + 8 * s);
+        mbar_arrive_expect_tx(kv_full + 8 * slot, 2 * TILE_BYTES);
+        tma_load_2d(smem_u32(sK + slot * TILE_BYTES), &tm_qkv, d + g * HD, row_base + k0,
+                    kv_full + 8 * slot);
+        tma_load_2d(smem_u32(sV + slot * TILE_BYTES), &tm_qkv, d + kvd + g * HD, row_base + k0,
+                    kv_full + 8 * slot);
       }
-      const int64_t base = ((int64_t)b * H + hq) * T;
+      nkv = it + 1;
+      for (int st = 0; st < grp * nq; st++) {
+        const int s = gs % STAGES;
+        const uint32_t ph = (gs / STAGES) & 1;
+        const int hq = g * grp + st / nq, qb = kb + st % nq;
+        // the slot (tiles and L, D) of step gs - STAGES is free once its products completed
+        if (!warp_wait(q_empty + 8 * s, ph ^ 1, abort_sh, gflag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full + 8 * s, 2 * TILE_BYTES);
+          tma_load_2d(smem_u32(sQ + s * TILE_BYTES), &tm_qkv, hq * HD, row_base + qb * BQ,
+                      q_full + 8 * s);
+          tma_load_2d(smem_u32(sdO + s * TILE_BYTES), &tm_do, hq * HD, row_base + qb * BQ,
+                      q_full + 8 * s);
+        }
+        const int64_t base = ((int64_t)b * H + hq) * T;
 #pragma unroll
-      for (int i = lane; i < BQ; i += 32) {
-        const int qi = qb * BQ + i;
-        // queries past T get L = +inf, so every P of theirs is 0
-        sL[s * 128 + i] = qi < T ? lse[base + qi] * LOG2E : INFINITY;
-        sD[s * 128 + i] = qi < T ? Dv[base + qi] : 0.f;
+        for (int i = lane; i < BQ; i += 32) {
+          const int qi = qb * BQ + i;
+          // queries past T get -L = -inf, so their P is 0 (below 2^-125 where
+          // the polynomial exponential takes the pair)
+          sL[s * 128 + i] = qi < T ? -lse[base + qi] * LOG2E : -INFINITY;
+          sD[s * 128 + i] = qi < T ? -Dv[base + qi] : 0.f;
+        }
+        mbar_arrive(ld_full + 8 * s);
+        gs++;
       }
-      mbar_arrive(ld_full + 8 * s);
-      issued = st + 1;
     }
     if (lane == 0) {
-      drain_wait(kv_full, 0);
-      for (int st = max(0, issued - STAGES); st < issued; st++)
-        drain_wait(q_full + 8 * (st % STAGES), (st / STAGES) & 1);
+      for (int i = max(0, nkv - 2); i < nkv; i++) drain_wait(kv_full + 8 * (i & 1), (i >> 1) & 1);
+      for (int i = max(0, gs - STAGES); i < gs; i++)
+        drain_wait(q_full + 8 * (i % STAGES), (i / STAGES) & 1);
     }
+    __syncwarp();
   } else if (warp == 1 || warp == MMA_B_WARP) {
     // ------------------------------------- MMA issuers (whole warps)
     // A: S^T = K Q^T, dV += P^T dO;  B: dP^T = V dO^T, dK += dS^T Q
     const int x = warp == 1 ? 0 : 1;
     constexpr uint32_t ID_S = idesc_mn(128, BQ, false, false);
     constexpr uint32_t ID_KV = idesc_mn(128, HD, false, true);
-    const uint64_t ad = sdesc(smem_u32(x ? sV : sK), 16, 1024);
+    uint8_t *sA = x ? sV : sK;     // A of the scores product, slot by item
     uint8_t *sB = x ? sdO : sQ;    // B of the scores product (K-major)
     uint8_t *sB2 = x ? sQ : sdO;   // B of the accumulation (MN-major)
     const uint32_t col = x ? KV_COL_DP : KV_COL_S;
     const uint32_t col_a2 = x ? KV_COL_DS : KV_COL_P, col_acc = x ? KV_COL_DK : KV_COL_DV;
-    auto issue_prod = [&](int st) {
-      const int s = st % STAGES;
+    auto issue_prod = [&](int slot, int s) {
+      const uint64_t ad = sdesc(smem_u32(sA + slot * TILE_BYTES), 16, 1024);
       const uint64_t bd = sdesc(smem_u32(sB + s * TILE_BYTES), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < HD / 16; kk++)
@@ -482,36 +656,61 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    kk > 0 ? 1u : 0u);
       mma_commit_e(s_full);
     };
-    bool ok = warp_wait(kv_full, 0, abort_sh, gflag) && warp_wait(q_full, 0, abort_sh, gflag);
-    if (ok) {
-      fence_after();
-      issue_prod(0);
+    bool ok = true;
+    int gs = 0;
+    int item = sched_item(0, G, cta);
+    if (item < n_items) {  // products of the first step
+      int kb, g, b;
+      decode(item, kb, g, b);
+      ok = warp_wait(kv_full, 0, abort_sh, gflag) && warp_wait(q_full, 0, abort_sh, gflag);
+      if (ok) {
+        fence_after();
+        issue_prod(0, 0);
+        if (grp * (nkb - kb) == 1) mma_commit_e(kv_empty);  // the item's last products on slot 0
+      }
     }
-    for (int st = 0; st < nsteps && ok; st++) {
-      const int s = st % STAGES;
-      if (st + 1 < nsteps) {
-        const int s1 = (st + 1) % STAGES;
-        const uint32_t ph1 = ((st + 1) / STAGES) & 1;
-        if (!warp_wait(q_full + 8 * s1, ph1, abort_sh, gflag) ||
-            !warp_wait(s_free, st & 1, abort_sh, gflag)) {
+    for (int r = 0, it = 0; item < n_items && ok; r++, it++) {
+      int kb, g, b;
+      decode(item, kb, g, b);
+      const int nsteps = grp * (nkb - kb), slot = it & 1;
+      const int next = sched_item(r + 1, G, cta);
+      int kb_next = nkb - 1, gn, bn;
+      if (next < n_items) decode(next, kb_next, gn, bn);
+      const int nsteps_next = grp * (nkb - kb_next);
+      for (int st = 0; st < nsteps && ok; st++, gs++) {
+        const int s = gs % STAGES;
+        // products of step gs + 1 (this item's next, or the next item's first)
+        // once the elementwise warps have read S^T and dP^T of step gs
+        const bool here = st + 1 < nsteps;
+        if (here || next < n_items) {
+          const int slot1 = here ? slot : slot ^ 1;
+          const int s1 = (gs + 1) % STAGES;
+          const uint32_t ph1 = ((gs + 1) / STAGES) & 1;
+          if ((!here && !warp_wait(kv_full + 8 * slot1, ((it + 1) >> 1) & 1, abort_sh, gflag)) ||
+              !warp_wait(q_full + 8 * s1, ph1, abort_sh, gflag) ||
+              !warp_wait(s_free, gs & 1, abort_sh, gflag)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          issue_prod(slot1, s1);
+          // the last products that read this K/V slot
+          if (here ? (st + 1 == nsteps - 1) : (nsteps_next == 1)) mma_commit_e(kv_empty + 8 * slot1);
+        }
+        if (!warp_wait(p_full, gs & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-        issue_prod(st + 1);
-      }
-      if (!warp_wait(p_full, st & 1, abort_sh, gflag)) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      const uint64_t bm = sdesc(smem_u32(sB2 + s * TILE_BYTES), 8192, 1024);
+        const uint64_t bm = sdesc(smem_u32(sB2 + s * TILE_BYTES), 8192, 1024);
 #pragma unroll
-      for (int kk = 0; kk < BQ / 16; kk++)
-        mma_ts_e(tmem + col_acc, tmem + col_a2 + kk * 8, bm + (uint64_t)(kk * 128), ID_KV,
-                 (st > 0 || kk > 0) ? 1u : 0u);
-      mma_commit_e(q_empty + 8 * s);
-      mma_commit_e(pv_done);
+        for (int kk = 0; kk < BQ / 16; kk++)
+          mma_ts_e(tmem + col_acc, tmem + col_a2 + kk * 8, bm + (uint64_t)(kk * 128), ID_KV,
+                   (st > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_e(q_empty + 8 * s);
+        mma_commit_e(pv_done);
+      }
+      item = next;
     }
     mma_commit_e(drain + 8 * x);
     if (lane == 0) drain_wait(drain + 8 * x, 0);
@@ -521,86 +720,131 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quarter = warp & 3;
     const int cq = (warp - 2) >> 2;  // column group: queries [cq CW, cq CW + CW) of the block
     const int r = quarter * 32 + lane;
-    const int kj = k0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool ok = true;
-    for (int st = 0; st < nsteps && ok; st++) {
-      const int s = st % STAGES;
-      const int qb = kb + st % nq;
-      if (!warp_wait(s_full, st & 1, abort_sh, gflag) ||
-          !warp_wait(ld_full + 8 * s, (st / STAGES) & 1, abort_sh, gflag)) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      float sv[CW], dv[CW];
-      tmem_ldn<CW>(tmem + lane_off + KV_COL_S + cq * CW, sv);
-      tmem_ldn<CW>(tmem + lane_off + KV_COL_DP + cq * CW, dv);
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      const int qc0 = qb * BQ + cq * CW;
-      const bool diag = (qb == kb);  // keys >= T occur only in this case, above the diagonal
-      const float4 *L4 = reinterpret_cast<const float4 *>(sL + s * 128 + cq * CW);
-      const float4 *D4 = reinterpret_cast<const float4 *>(sD + s * 128 + cq * CW);
-      uint32_t wp[CW / 2], wd[CW / 2];
-#pragma unroll
-      for (int i = 0; i < CW; i += 4) {
-        const float4 lq = L4[i / 4], dq = D4[i / 4];
-        float p0 = ex2(fmaf(sv[i], sl2, -lq.x)), p1 = ex2(fmaf(sv[i + 1], sl2, -lq.y));
-        float p2 = ex2(fmaf(sv[i + 2], sl2, -lq.z)), p3 = ex2(fmaf(sv[i + 3], sl2, -lq.w));
-        if (diag) {
-          if (kj > qc0 + i) p0 = 0.f;
-          if (kj > qc0 + i + 1) p1 = 0.f;
-          if (kj > qc0 + i + 2) p2 = 0.f;
-          if (kj > qc0 + i + 3) p3 = 0.f;
-        }
-        wp[i / 2] = pack_bf16(p0, p1);
-        wp[i / 2 + 1] = pack_bf16(p2, p3);
-        wd[i / 2] = pack_bf16(p0 * (dv[i] - dq.x), p1 * (dv[i + 1] - dq.y));
-        wd[i / 2 + 1] = pack_bf16(p2 * (dv[i + 2] - dq.z), p3 * (dv[i + 3] - dq.w));
-      }
-      // P^T and dS^T of the previous step are free once its products completed
-      if (st > 0) {
-        if (!warp_wait(pv_done, (st - 1) & 1, abort_sh, gflag)) {
+    int gs = 0;
+    for (int rr = 0, it = 0; ok; rr++, it++) {
+      const int item = sched_item(rr, G, cta);
+      if (item >= n_items) break;
+      int kb, g, b;
+      decode(item, kb, g, b);
+      const int k0 = kb * BK, kj = k0 + r, nq = nkb - kb, slot = it & 1;
+      const int nsteps = grp * nq;
+      // the accumulators of the previous item were read out before this
+      // warp's first P^T / dS^T arrival below (program order), so the
+      // item's first accumulations (accumulate = 0) cannot overwrite them early
+      for (int st = 0; st < nsteps && ok; st++, gs++) {
+        const int s = gs % STAGES;
+        const int qb = kb + st % nq;
+        if (!warp_wait(s_full, gs & 1, abort_sh, gflag) ||
+            !warp_wait(ld_full + 8 * s, (gs / STAGES) & 1, abort_sh, gflag)) {
           ok = false;
           break;
         }
         fence_after();
-      }
+        const int qc0 = qb * BQ + cq * CW;
+        const bool diag = (qb == kb);  // keys >= T occur only in this case, above the diagonal
+        const float4 *L4 = reinterpret_cast<const float4 *>(sL + s * 128 + cq * CW);
+        const float4 *D4 = reinterpret_cast<const float4 *>(sD + s * 128 + cq * CW);
+        // two halves of the thread's CW queries, each read from TMEM, packed
+        // and stored before the next (fewer live registers); S^T and dP^T are
+        // released once the second half is read; P^T and dS^T of the previous
+        // step are free once its products completed (at an item's first step
+        // the epilogue already waited)
 #pragma unroll
-      for (int c = 0; c < CW / 2; c += 16) {
-        tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + KV_COL_P + cq * (CW / 2) + c, wp + c);
-        tmem_stn<(CW / 2 < 16 ? CW / 2 : 16)>(tmem + lane_off + KV_COL_DS + cq * (CW / 2) + c, wd + c);
+        for (int hf = 0; hf < 2; hf++) {
+          constexpr int HC = CW / 2;
+          float sv[HC], dv[HC];
+          tmem_ldn<HC>(tmem + lane_off + KV_COL_S + cq * CW + hf * HC, sv);
+          tmem_ldn<HC>(tmem + lane_off + KV_COL_DP + cq * CW + hf * HC, dv);
+          if (hf == 1) {
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+          }
+          uint32_t wp[HC / 2], wd[HC / 2];
+#pragma unroll
+          for (int i = 0; i < HC; i += 4) {
+            const int c = hf * HC + i;  // query column within the thread's CW
+            const float4 nl = L4[c / 4], nd = D4[c / 4];  // -L (log2 units), -D of 4 queries
+            const float2 x01 = __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2),
+                                          make_float2(nl.x, nl.y));
+            const float2 x23 = __ffma2_rn(make_float2(sv[i + 2], sv[i + 3]),
+                                          make_float2(sl2, sl2), make_float2(nl.z, nl.w));
+            float2 p01 = exp2_pair(x01, c / 2), p23 = exp2_pair(x23, c / 2 + 1);
+            if (diag) {
+              if (kj > qc0 + c) p01.x = 0.f;
+              if (kj > qc0 + c + 1) p01.y = 0.f;
+              if (kj > qc0 + c + 2) p23.x = 0.f;
+              if (kj > qc0 + c + 3) p23.y = 0.f;
+            }
+            wp[i / 2] = pack_bf16(p01.x, p01.y);
+            wp[i / 2 + 1] = pack_bf16(p23.x, p23.y);
+            const float2 d01 = __fmul2_rn(p01, __fadd2_rn(make_float2(dv[i], dv[i + 1]),
+                                                          make_float2(nd.x, nd.y)));
+            const float2 d23 = __fmul2_rn(p23, __fadd2_rn(make_float2(dv[i + 2], dv[i + 3]),
+                                                          make_float2(nd.z, nd.w)));
+            wd[i / 2] = pack_bf16(d01.x, d01.y);
+            wd[i / 2 + 1] = pack_bf16(d23.x, d23.y);
+          }
+          if (hf == 0 && st > 0) {
+            if (!warp_wait(pv_done, (gs - 1) & 1, abort_sh, gflag)) {
+              ok = false;
+              break;
+            }
+            fence_after();
+          }
+          tmem_stn<HC / 2>(tmem + lane_off + KV_COL_P + cq * (CW / 2) + hf * (HC / 2), wp);
+          tmem_stn<HC / 2>(tmem + lane_off + KV_COL_DS + cq * (CW / 2) + hf * (HC / 2), wd);
+        }
+        if (!ok) break;
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
       }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (ok) ok = warp_wait(pv_done, (nsteps - 1) & 1, abort_sh, gflag);
-    if (ok) {
+      if (!ok) break;
+      if (!warp_wait(pv_done, (gs - 1) & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
+      }
       fence_after();
       // column pairs (c, c + 32) of RoPE: this group takes c in [cq HW, cq HW + HW)
-      float xx[HW], yy[HW];
-      __nv_bfloat16 *dst = dqkv + ((int64_t)row_base + kj) * ld + d + g * HD + cq * HW;
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + cq * HW, xx);
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + 32 + cq * HW, yy);
-      if (kj < T) {
-        if (cos_t)
-          rope_bwd_n<HW>(xx, yy, cos_t + (int64_t)kj * (HD / 2) + cq * HW,
-                         sin_t + (int64_t)kj * (HD / 2) + cq * HW);
-        store_n<HW>(dst, xx, scale);
-        store_n<HW>(dst + 32, yy, scale);
+      float xk[HW], yk[HW], xv[HW], yv[HW];
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + cq * HW, xk);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + 32 + cq * HW, yk);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + cq * HW, xv);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + 32 + cq * HW, yv);
+      if (kj < T && cos_t)
+        rope_bwd_n<HW>(xk, yk, cos_t + (int64_t)kj * (HD / 2) + cq * HW,
+                       sin_t + (int64_t)kj * (HD / 2) + cq * HW);
+      // dK, dV rows through the item's K and V tiles (their products are
+      // complete), then each warp stores 8 whole rows of its lane quarter of
+      // both with bulk tensor copies (rows past T clipped)
+      uint8_t *rk = sK + slot * TILE_BYTES + r * 128, *rv = sV + slot * TILE_BYTES + r * 128;
+      stage_n<HW>(rk, cq, r, xk, scale);
+      stage_n<HW>(rk, 4 + cq, r, yk, scale);
+      stage_n<HW>(rv, cq, r, xv, 1.f);
+      stage_n<HW>(rv, 4 + cq, r, yv, 1.f);
+      fence_proxy_async();
+      mbar_arrive(qsync + 8 * quarter);
+      if (!warp_wait(qsync + 8 * quarter, it & 1, abort_sh, gflag)) {
+        ok = false;
+        break;
       }
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + cq * HW, xx);
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + 32 + cq * HW, yy);
-      if (kj < T) {
-        store_n<HW>(dst + kvd, xx, 1.f);
-        store_n<HW>(dst + kvd + 32, yy, 1.f);
+      if (lane == 0) {
+        const int r0 = quarter * 32 + cq * 8;
+        tma_store_3d(&tm_st, smem_u32(sK + slot * TILE_BYTES + r0 * 128), d + g * HD, k0 + r0, b);
+        tma_store_3d(&tm_st, smem_u32(sV + slot * TILE_BYTES + r0 * 128), d + kvd + g * HD,
+                     k0 + r0, b);
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(kv_empty + 8 * slot);
       }
+      __syncwarp();
     }
+    if (lane == 0) bulk_wait_all();
   }
   fence_before();
   __syncthreads();
@@ -609,6 +853,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 }  // namespace attn_tc_bwd
+
 
 // Host side: tensor maps over qkv [B*T, qkvw] and dout [B*T, H*hd] (box 64 x
 // 128); the dQ kernel runs first (it also writes D), then the dK/dV kernel.
@@ -623,18 +868,18 @@ bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *
       !smem_optin((const void *)k_attn_dkv_tc, KV_SMEM))
     return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd, dw = (int64_t)H * hd;
-  CUtensorMap mq, md;
+  CUtensorMap mq, md, mo, mst;
   if (!tc::tile_map_bf16(&mq, qkv, qkvw, (int64_t)B * T, qkvw, 128) ||
-      !tc::tile_map_bf16(&md, dout, dw, (int64_t)B * T, dw, 128))
+      !tc::tile_map_bf16(&md, dout, dw, (int64_t)B * T, dw, 128) ||
+      !tc::tile_map_bf16(&mo, o, dw, (int64_t)B * T, dw, 128) ||
+      !tc::tile_map_bf16_3d(&mst, dqkv, qkvw, T, B, qkvw, 8))
     return false;
-  const int nb = (T + BQ - 1) / BQ;
+  const int nb = (T + BQ - 1) / BQ, sms = device_sms();
   const float scale = 1.0f / sqrtf((float)hd);
-  k_attn_dq_tc<<<dim3(H, B, nb), NTHREADS, DQ_SMEM, s>>>(
-      mq, md, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dout, lse, Dbuf,
-      (__nv_bfloat16 *)dqkv, cos_t, sin_t, T, H, Hkv, scale, flag);
-  k_attn_dkv_tc<<<dim3(Hkv, B, nb), NTHREADS, KV_SMEM, s>>>(mq, md, lse, Dbuf,
-                                                            (__nv_bfloat16 *)dqkv, cos_t, sin_t,
-                                                            T, H, Hkv, scale, flag);
+  k_attn_dq_tc<<<min(nb * H * B, sms), NTHREADS, DQ_SMEM, s>>>(
+      mq, md, mo, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, flag);
+  k_attn_dkv_tc<<<min(nb * Hkv * B, sms), NTHREADS, KV_SMEM, s>>>(
+      mq, md, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, flag);
   count_launch(2);
   return true;
 }

@@ -222,6 +222,8 @@ void set_device_int(int *p, int v, cudaStream_t s);
 // The attribute belongs to the device's context, so it is set once per
 // (device, kernel), under a lock; false when the runtime refuses it.
 bool smem_optin(const void *func, int bytes);
+// Streaming multiprocessors of the current device (cached per device).
+int device_sms();
 
 // Launch counter (kernels enqueued by the current call).
 extern thread_local int g_launches;

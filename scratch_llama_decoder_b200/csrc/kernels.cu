@@ -29,6 +29,21 @@ bool smem_optin(const void *func, int bytes) {
   return true;
 }
 
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  static std::mutex mu;
+  static std::map<int, int> sms;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = sms.find(dev);
+  if (it != sms.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    n = 1;
+  sms[dev] = n;
+  return n;
+}
+
 static inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
 
 // ------------------------------------------------------------------ RoPE table

@@ -49,6 +49,12 @@ LLM_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, 
     }
   }
 }
+// Bounded wait used only on the way out (the copies / MMAs of this thread).
+LLM_DEV void drain_wait(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = gtimer();
+  while (!mbar_try(bar, parity) && gtimer() - t0 < WAIT_NS) {
+  }
+}
 LLM_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
@@ -128,6 +134,52 @@ LLM_DEV float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// 2^x for a pair on the FMA pipe instead of the SFU, so that a softmax loop
+// can split its exponentials between the two units.  Range reduction in the
+// style of Cody and Waite (Software Manual for the Elementary Functions,
+// 1980): x = k + f with k = round(x) taken by adding 1.5 * 2^23 (the rounded
+// sum holds k in its low mantissa bits), f in [-1/2, 1/2]; 2^f by the degree-3
+// polynomial that minimises the maximum relative error on that interval
+// (Remez exchange, fitted by exp2_poly_fit.py beside this file: 7.5e-5, well
+// under half a bf16 ulp); 2^k applied by adding k to the exponent field.
+// Domain x <= 126 (the softmax loops pass x <= 8); x is clamped below at
+// -126, where the result is a tiny positive number (under 2^-125) rather
+// than 0.
+constexpr float EXP2_C0 = 0.9999280571937561f, EXP2_C1 = 0.6932609677314758f,
+                EXP2_C2 = 0.2426111251115799f, EXP2_C3 = 0.0551716685295105f;
+LLM_DEV float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 k = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(k, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
+  p = __ffma2_rn(p, f, make_float2(EXP2_C0, EXP2_C0));
+  // t's bit pattern is that of 1.5 * 2^23 plus k: shifted left by 23 bits,
+  // only k << 23 remains (mod 2^32), the exponent-field increment
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+// Whether pair `i` (of the 16 pairs of a 32-score chunk) of a softmax loop
+// takes the polynomial: 5 of 16, spread over the chunk, which balanced the
+// SFU against the FMA pipe and the issue slots best in a measured sweep.
+LLM_DEV constexpr bool exp2_on_fma(int i) { return ((i & 15) * 5) % 16 < 5; }
+// 2^x for a pair: the polynomial or the SFU, by the pair's index.
+LLM_DEV float2 exp2_pair(float2 x, int i) {
+  return exp2_on_fma(i) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+}
+// Work item of a persistent kernel in scheduling round r: the G CTAs take
+// the items (ordered heaviest first) in a snake, CTA c taking item r G + c in
+// even rounds and r G + G - 1 - c in odd ones, which evens out the summed
+// weights of a CTA's items when the weights fall in steps.
+LLM_DEV int sched_item(int r, int G, int c) { return r * G + ((r & 1) ? G - 1 - c : c); }
+// max(a, b, c) in one instruction.
+LLM_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 // tcgen05.mma with the A operand in TMEM (bf16 pairs packed in 32-bit
 // columns: K 16 = 8 columns) and B in shared memory.
@@ -315,6 +367,46 @@ inline bool tile_map_bf16(CUtensorMap *map, const void *base, int64_t cols, int6
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// Tensor map over a [batches, rows, cols] bf16 array (row stride ld
+// elements, batch stride rows * ld) with a box of 64 columns x box_rows rows
+// x 1 batch and 128-byte swizzle: a bulk store through it clips at the end of
+// each batch's rows, not only at the end of the array.
+inline bool tile_map_bf16_3d(CUtensorMap *map, const void *base, int64_t cols, int64_t rows,
+                             int64_t batches, int64_t ld, int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
+    cudaDriverEntryPointQueryResult q;
+    void *fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  }();
+  if (!encode || ((uintptr_t)base & 15) || (ld * 2) % 16) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batches};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(ld * rows * 2)};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Bulk tensor store of a box from shared memory (3-D map), its commit, and
+// the wait until every committed store of this thread has read its source.
+LLM_DEV void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+          (uint64_t)map),
+      "r"(x), "r"(y), "r"(z), "r"(src)
+      : "memory");
+}
+LLM_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+LLM_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+LLM_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+LLM_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 }  // namespace tc
 }  // namespace llm
