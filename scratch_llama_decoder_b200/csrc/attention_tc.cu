@@ -101,7 +101,7 @@ LLM_DEV bool softmax_all(bool v) {
 LLM_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * SM_WARPS) : "memory"); }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
-    k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, __nv_bfloat16 *__restrict__ o,
+    k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_o,
                   float *__restrict__ lse, int B, int T, int H, int Hkv, float scale, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -126,19 +126,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
   const int G = gridDim.x, cta = blockIdx.x;
   const int d = H * HD, kvd = Hkv * HD;
-  // item -> (query block, head, batch), longest rows (last query blocks) first
+  // item -> (query block, head, batch): longest rows (last query blocks) first,
+  // in bands of 4 query blocks taken pair by pair (band_item)
   auto decode = [&](int item, int &qb, int &h, int &b) {
-    const int z = item / (H * B), rem = item - z * (H * B);
+    int z, pr;
+    band_item(item, nqb, H * B, z, pr);
     qb = nqb - 1 - z;
-    h = rem % H;
-    b = rem / H;
+    h = pr % H;
+    b = pr / H;
   };
 
   if (threadIdx.x == 0) {
     *abort_sh = 0;
     for (int x = 0; x < 2; x++) {
       mbar_init(q_full + 8 * x, 1);
-      mbar_init(q_empty + 8 * x, 1);  // the item's last S product on the slot
+      // the item's last S product on the slot, then the bulk stores of O
+      // staged in it (one per softmax warp)
+      mbar_init(q_empty + 8 * x, 1 + SM_WARPS);
     }
     for (int s = 0; s < STAGES; s++) {
       mbar_init(k_full + 8 * s, 1);
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (item >= n_items) break;
       int qb, h, b;
       decode(item, qb, h, b);
-      const int q0 = qb * BQ, row_base = b * T, nj = qb + 1;
+      const int q0 = qb * BQ, nj = qb + 1;
       const int qi = q0 + r;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
@@ -427,22 +431,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int i = 0; i < OW; i++) acc[i] += v[i] * cg;
       }
-      // every softmax warp has read every accumulator before any of them
-      // releases the next item's first P (whose P V overwrites O_g)
+      // O rows through the item's Q tile (its last S product is complete):
+      // this thread's two 16-byte chunks of row r in the tile's
+      // 128-byte-swizzle image
+      uint8_t *srow = sQ + (it & 1) * TILE_BYTES + r * 128;
+#pragma unroll
+      for (int c = 0; c < OW / 8; c++) {
+        const int ch = grp * (OW / 8) + c;
+        *reinterpret_cast<uint4 *>(srow + ((ch ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16(acc[8 * c], acc[8 * c + 1]), pack_bf16(acc[8 * c + 2], acc[8 * c + 3]),
+                       pack_bf16(acc[8 * c + 4], acc[8 * c + 5]),
+                       pack_bf16(acc[8 * c + 6], acc[8 * c + 7]));
+      }
+      fence_proxy_async();
+      // every softmax warp has read every accumulator (before any of them
+      // releases the next item's first P, whose P V overwrites O_g) and staged
+      // its part of O
       fence_before();
       softmax_sync();
-      if (qi < T) {
-        __nv_bfloat16 *dst = o + ((int64_t)row_base + qi) * d + h * HD + grp * OW;
-#pragma unroll
-        for (int i = 0; i < OW; i += 8) {
-          uint32_t wv[4];
-#pragma unroll
-          for (int e = 0; e < 4; e++) wv[e] = pack_bf16(acc[i + 2 * e], acc[i + 2 * e + 1]);
-          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        }
-        if (grp == 0) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
+      if (lane == 0) {  // 8 whole rows of this warp's lane quarter (rows past T clipped)
+        const int r0 = quarter * 32 + grp * 8;
+        tma_store_3d(&tm_o, smem_u32(sQ + (it & 1) * TILE_BYTES + r0 * 128), h * HD, q0 + r0, b);
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(q_empty + 8 * (it & 1));
       }
+      __syncwarp();
+      if (grp == 0 && qi < T) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
     }
+    if (lane == 0) bulk_wait_all();
   }
   fence_before();
   __syncthreads();
@@ -466,11 +483,13 @@ bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int 
   if (hd != HD || !flag) return false;
   if (!smem_optin((const void *)k_attn_fwd_tc, SMEM_BYTES)) return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd;
-  CUtensorMap map;
-  if (!tc::tile_map_bf16(&map, qkv, qkvw, (int64_t)B * T, qkvw, 128)) return false;
+  CUtensorMap map, mo;
+  if (!tc::tile_map_bf16(&map, qkv, qkvw, (int64_t)B * T, qkvw, 128) ||
+      !tc::tile_map_bf16_3d(&mo, o, (int64_t)H * hd, T, B, (int64_t)H * hd, 8))
+    return false;
   const int items = ((T + BQ - 1) / BQ) * H * B;
   k_attn_fwd_tc<<<min(items, device_sms()), NTHREADS, SMEM_BYTES, s>>>(
-      map, (__nv_bfloat16 *)o, lse, B, T, H, Hkv, 1.0f / sqrtf((float)hd), flag);
+      map, mo, lse, B, T, H, Hkv, 1.0f / sqrtf((float)hd), flag);
   count_launch();
   return true;
 }

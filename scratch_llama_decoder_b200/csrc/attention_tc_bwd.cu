@@ -30,8 +30,8 @@
 //   S^T = K Q^T (A) and dP^T = V dO^T (B) into TMEM; P^T and dS^T back into
 //   TMEM as bf16; dV += P^T dO (A) and dK += dS^T Q (B) (A operands from
 //   TMEM, B = dO / Q MN-major).
-//   The per-query -L (log2 units) and -D of each step travel with its Q/dO
-//   tiles.
+//   The per-query L and D of each step travel with its Q/dO tiles (bulk
+//   copies completing on the same barrier).
 // dQ and dK leave through the backward of the rotate-half RoPE (when tables
 // are given), then scale, bf16.  No atomics: every output element is written
 // once by the CTA that owns its row.  The elementwise arithmetic runs on
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  const float *__restrict__ lse,
                  float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
                  const float *__restrict__ cos_t, const float *__restrict__ sin_t, int B, int T,
-                 int H, int Hkv, float scale, int *gflag) {
+                 int H, int Hkv, float scale, int bulk_l, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = smem, *sdO = smem + 2 * TILE_BYTES, *sO = smem + 4 * TILE_BYTES,
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
   float *red = (float *)(bars + BAR_BYTES / 8);  // [2][NCQ][128] partial dot products
-  float *sNL = red + 2 * NCQ * 128;              // [128] -L log2(e) of the item's rows
+  float *sNL = red + 2 * NCQ * 128;              // [128] L of the item's rows (rows < T)
   const uint32_t b0 = smem_u32(bars);
   const uint32_t qd_full = b0, qd_empty = b0 + 16,  // [2]: Q/dO slot
                  o_full = b0 + 32, o_empty = b0 + 40, k_full = b0 + 48,
@@ -162,12 +162,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
   const int G = gridDim.x, cta = blockIdx.x;
   const int d = H * HD, kvd = Hkv * HD;
-  // item -> (query block, head, batch), longest rows (last query blocks) first
+  // item -> (query block, head, batch): longest rows (last query blocks) first,
+  // in bands of 4 query blocks taken pair by pair (band_item)
   auto decode = [&](int item, int &qb, int &h, int &b) {
-    const int z = item / (H * B), rem = item - z * (H * B);
+    int z, pr;
+    band_item(item, nqb, H * B, z, pr);
     qb = nqb - 1 - z;
-    h = rem % H;
-    b = rem / H;
+    h = pr % H;
+    b = pr / H;
   };
 
   if (threadIdx.x == 0) {
@@ -224,18 +226,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     qd_full + 8 * slot);
       }
       nqd = it + 1;
-      // O and -L once the elementwise warps have formed D of item it - 1
+      // O and L once the elementwise warps have formed D of item it - 1; L
+      // by a bulk copy when its rows are 16-byte aligned (T % 4 == 0), else
+      // by the lanes
       if (!warp_wait(o_empty, (it & 1) ^ 1, abort_sh, gflag)) break;
+      const float *lrow = lse + ((int64_t)b * H + h) * T + q0;
+      const int nvalid = min(BQ, T - q0);
       if (lane == 0) {
-        mbar_arrive_expect_tx(o_full, TILE_BYTES);
+        mbar_arrive_expect_tx(o_full, TILE_BYTES + (bulk_l ? nvalid * 4 : 0));
         tma_load_2d(smem_u32(sO), &tm_o, h * HD, row_base + q0, o_full);
+        if (bulk_l) bulk_load(smem_u32(sNL), lrow, nvalid * 4, o_full);
       }
-      const int64_t lbase = ((int64_t)b * H + h) * T;
-      for (int i = lane; i < BQ; i += 32) {
-        const int qi = q0 + i;
-        // rows past T get -L = -inf, so every P of theirs is 0
-        sNL[i] = qi < T ? -lse[lbase + qi] * LOG2E : -INFINITY;
-      }
+      if (!bulk_l)
+        for (int i = lane; i < nvalid; i += 32) sNL[i] = lrow[i];
       mbar_arrive(o_full);
       no = it + 1;
       for (int j = 0; j <= qb; j++) {
@@ -392,7 +395,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      const float nl2 = sNL[r];
+      // rows past T get -L = -inf, so every P of theirs is 0
+      const float nl2 = valid ? -sNL[r] * LOG2E : -INFINITY;
       mbar_arrive(o_empty);              // this thread's O row and -L consumed
       mbar_arrive(qd_empty + 8 * slot);  // and its dO row
       float *rd = red + (it & 1) * NCQ * 128;
@@ -524,13 +528,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                   const float *__restrict__ lse,
                   const float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
                   const float *__restrict__ cos_t, const float *__restrict__ sin_t, int B, int T,
-                  int H, int Hkv, float scale, int *gflag) {
+                  int H, int Hkv, float scale, int bulk_l, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sK = smem, *sV = smem + 2 * TILE_BYTES, *sQ = smem + 4 * TILE_BYTES,
           *sdO = sQ + STAGES * TILE_BYTES;
-  float *sL = (float *)(sdO + STAGES * TILE_BYTES);  // [STAGES][128] -L * log2(e)
-  float *sD = sL + STAGES * 128;                      // [STAGES][128] -D
+  float *sL = (float *)(sdO + STAGES * TILE_BYTES);  // [STAGES][128] L (+inf past T)
+  float *sD = sL + STAGES * 128;                      // [STAGES][128] D (0 past T)
   uint64_t *bars = (uint64_t *)(sD + STAGES * 128);
   uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
@@ -546,12 +550,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int nkb = (T + BK - 1) / BK, n_items = nkb * Hkv * B;
   const int G = gridDim.x, cta = blockIdx.x;
   const int grp = H / Hkv, d = H * HD, kvd = Hkv * HD;
-  // item -> (key block, kv head, batch); steps = grp (nkb - kb)
+  // item -> (key block, kv head, batch), first key blocks first in bands of 4
+  // taken pair by pair (band_item); steps = grp (nkb - kb)
   auto decode = [&](int item, int &kb, int &g, int &b) {
-    kb = item / (Hkv * B);
-    const int rem = item - kb * (Hkv * B);
-    g = rem % Hkv;
-    b = rem / Hkv;
+    int pr;
+    band_item(item, nkb, Hkv * B, kb, pr);
+    g = pr % Hkv;
+    b = pr / Hkv;
   };
 
   if (threadIdx.x == 0) {
@@ -610,21 +615,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
+        // the step's L and D rows by bulk copies when 16-byte aligned (T % 4
+        // == 0), else by the lanes; queries past T get L = +inf, so their P is
+        // 0 (below 2^-125 where the polynomial exponential takes the pair), and D = 0
+        const int64_t base = ((int64_t)b * H + hq) * T + qb * BQ;
+        const int nvalid = min(BQ, T - qb * BQ);
         if (lane == 0) {
-          mbar_arrive_expect_tx(q_full + 8 * s, 2 * TILE_BYTES);
+          mbar_arrive_expect_tx(q_full + 8 * s, 2 * TILE_BYTES + (bulk_l ? 8 * nvalid : 0));
           tma_load_2d(smem_u32(sQ + s * TILE_BYTES), &tm_qkv, hq * HD, row_base + qb * BQ,
                       q_full + 8 * s);
           tma_load_2d(smem_u32(sdO + s * TILE_BYTES), &tm_do, hq * HD, row_base + qb * BQ,
                       q_full + 8 * s);
+          if (bulk_l) {
+            bulk_load(smem_u32(sL + s * 128), lse + base, nvalid * 4, q_full + 8 * s);
+            bulk_load(smem_u32(sD + s * 128), Dv + base, nvalid * 4, q_full + 8 * s);
+          }
         }
-        const int64_t base = ((int64_t)b * H + hq) * T;
 #pragma unroll
         for (int i = lane; i < BQ; i += 32) {
-          const int qi = qb * BQ + i;
-          // queries past T get -L = -inf, so their P is 0 (below 2^-125 where
-          // the polynomial exponential takes the pair)
-          sL[s * 128 + i] = qi < T ? -lse[base + qi] * LOG2E : -INFINITY;
-          sD[s * 128 + i] = qi < T ? -Dv[base + qi] : 0.f;
+          if (i >= nvalid) {
+            sL[s * 128 + i] = INFINITY;
+            sD[s * 128 + i] = 0.f;
+          } else if (!bulk_l) {
+            sL[s * 128 + i] = lse[base + i];
+            sD[s * 128 + i] = Dv[base + i];
+          }
         }
         mbar_arrive(ld_full + 8 * s);
         gs++;
@@ -738,6 +753,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = gs % STAGES;
         const int qb = kb + st % nq;
         if (!warp_wait(s_full, gs & 1, abort_sh, gflag) ||
+            !warp_wait(q_full + 8 * s, (gs / STAGES) & 1, abort_sh, gflag) ||
             !warp_wait(ld_full + 8 * s, (gs / STAGES) & 1, abort_sh, gflag)) {
           ok = false;
           break;
@@ -767,11 +783,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int i = 0; i < HC; i += 4) {
             const int c = hf * HC + i;  // query column within the thread's CW
-            const float4 nl = L4[c / 4], nd = D4[c / 4];  // -L (log2 units), -D of 4 queries
+            const float4 lq = L4[c / 4], dq = D4[c / 4];  // L and D of 4 queries
+            const float2 nl01 = __fmul2_rn(make_float2(lq.x, lq.y), make_float2(-LOG2E, -LOG2E));
+            const float2 nl23 = __fmul2_rn(make_float2(lq.z, lq.w), make_float2(-LOG2E, -LOG2E));
             const float2 x01 = __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2),
-                                          make_float2(nl.x, nl.y));
+                                          nl01);
             const float2 x23 = __ffma2_rn(make_float2(sv[i + 2], sv[i + 3]),
-                                          make_float2(sl2, sl2), make_float2(nl.z, nl.w));
+                                          make_float2(sl2, sl2), nl23);
             float2 p01 = exp2_pair(x01, c / 2), p23 = exp2_pair(x23, c / 2 + 1);
             if (diag) {
               if (kj > qc0 + c) p01.x = 0.f;
@@ -781,10 +799,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             wp[i / 2] = pack_bf16(p01.x, p01.y);
             wp[i / 2 + 1] = pack_bf16(p23.x, p23.y);
-            const float2 d01 = __fmul2_rn(p01, __fadd2_rn(make_float2(dv[i], dv[i + 1]),
-                                                          make_float2(nd.x, nd.y)));
-            const float2 d23 = __fmul2_rn(p23, __fadd2_rn(make_float2(dv[i + 2], dv[i + 3]),
-                                                          make_float2(nd.z, nd.w)));
+            const float2 d01 = __fmul2_rn(p01, __ffma2_rn(make_float2(dq.x, dq.y), make_float2(-1.f, -1.f),
+                                                          make_float2(dv[i], dv[i + 1])));
+            const float2 d23 = __fmul2_rn(p23, __ffma2_rn(make_float2(dq.z, dq.w), make_float2(-1.f, -1.f),
+                                                          make_float2(dv[i + 2], dv[i + 3])));
             wd[i / 2] = pack_bf16(d01.x, d01.y);
             wd[i / 2 + 1] = pack_bf16(d23.x, d23.y);
           }
@@ -876,10 +894,14 @@ bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *
     return false;
   const int nb = (T + BQ - 1) / BQ, sms = device_sms();
   const float scale = 1.0f / sqrtf((float)hd);
+  // L and D rows of a (batch, head) start 16-byte aligned when T % 4 == 0
+  const int bulk_l = (T % 4 == 0) && !((uintptr_t)lse & 15) && !((uintptr_t)Dbuf & 15);
   k_attn_dq_tc<<<min(nb * H * B, sms), NTHREADS, DQ_SMEM, s>>>(
-      mq, md, mo, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, flag);
+      mq, md, mo, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, bulk_l,
+      flag);
   k_attn_dkv_tc<<<min(nb * Hkv * B, sms), NTHREADS, KV_SMEM, s>>>(
-      mq, md, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, flag);
+      mq, md, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, bulk_l,
+      flag);
   count_launch(2);
   return true;
 }

@@ -175,6 +175,18 @@ LLM_DEV float2 exp2_pair(float2 x, int i) {
 // even rounds and r G + G - 1 - c in odd ones, which evens out the summed
 // weights of a CTA's items when the weights fall in steps.
 LLM_DEV int sched_item(int r, int G, int c) { return r * G + ((r & 1) ? G - 1 - c : c); }
+// Work item -> (weight class z, pair p) for nz classes (z = 0 heaviest) of np
+// pairs: classes in bands of 4, pair-major inside a band, so that the CTAs
+// that work at one time on a pair's classes stream the same tiles and share
+// them in L2, while the weights still fall band by band for the snake.
+LLM_DEV void band_item(int item, int nz, int np, int &z, int &p) {
+  constexpr int BW = 4;
+  const int band = item / (BW * np);
+  const int rem = item - band * BW * np;
+  const int nbb = min(BW, nz - band * BW);
+  p = rem / nbb;
+  z = band * BW + rem - p * nbb;
+}
 // max(a, b, c) in one instruction.
 LLM_DEV float fmax3(float a, float b, float c) {
   float d;
@@ -401,6 +413,15 @@ LLM_DEV void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, in
       "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
           (uint64_t)map),
       "r"(x), "r"(y), "r"(z), "r"(src)
+      : "memory");
+}
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from global to shared memory, completing on `bar`'s transaction count.
+LLM_DEV void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 LLM_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
