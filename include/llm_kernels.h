@@ -57,6 +57,18 @@ int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o, const void
                                   int ctx, int n_head, int n_kv_head, int head_dim,
                                   int tensor_cores, void *stream);
 
+/* The same attention in float32 (the float32 configurations): d_qkv, d_o,
+ * d_dout, d_dqkv float32 with the layouts above, d_lse and d_D as above.
+ * tiled = 1 selects the tiled CUDA-core kernels (head_dim 32 or 64; rows
+ * 16-byte aligned: pointers 16-byte aligned), 0 the one-warp-per-row
+ * kernels (any head_dim); LLM_ERR_ARG otherwise.  Asynchronous on `stream`. */
+int llm_kernel_attention_fwd_f32(const float *d_qkv, float *d_o, float *d_lse, int batch, int ctx,
+                                 int n_head, int n_kv_head, int head_dim, int tiled, void *stream);
+int llm_kernel_attention_bwd_f32(const float *d_qkv, const float *d_o, const float *d_dout,
+                                 const float *d_lse, float *d_D, float *d_dqkv, int batch,
+                                 int ctx, int n_head, int n_kv_head, int head_dim, int tiled,
+                                 void *stream);
+
 /* Embedding backward (Hephaistos, Architecture at a glance: token embedding;
  * its gradient is a scatter-add): dwte[v,:] = sum over positions i with
  * tokens[i] = v of dx[i,:], summed in increasing i (deterministic), zero for

@@ -108,6 +108,9 @@ EXPORTS = {
     "llm_kernel_attention_fwd_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "llm_kernel_attention_bwd_bf16": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                            _vp]),
+    "llm_kernel_attention_fwd_f32": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "llm_kernel_attention_bwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                          _vp]),
     "llm_kernel_embed_bwd_scratch_bytes": (_i, [_i64, _i, C.POINTER(_i64)]),
     "llm_kernel_embed_bwd": (_i, [_vp, _vp, _vp, _i64, _i, _i, _vp, _i64, _vp]),
     "llm_kernel_embed_bwd_noalloc": (_i, [_vp, _vp, _vp, _i64, _i, _i, _vp]),

@@ -129,6 +129,18 @@ void or_flag(const int *src, int *dst, cudaStream_t s);
 // of the site): o uses P f, the backward uses the same f.
 void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
                    int hd, cudaStream_t s, DropArgs drop = DropArgs{});
+// float32 tiled kernels (head size 32 or 64; false otherwise) and the
+// one-warp-per-row kernels alone.
+bool attn_fwd_f32_tiled(const float *qkv, float *o, float *lse, int B, int T, int H, int Hkv,
+                        int hd, cudaStream_t s);
+bool attn_bwd_f32_tiled(const float *qkv, const float *o, const float *dout, const float *lse,
+                        float *Dbuf, float *dqkv, int B, int T, int H, int Hkv, int hd,
+                        cudaStream_t s);
+void attn_fwd_rows(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
+                   int hd, cudaStream_t s, DropArgs drop);
+void attn_bwd_rows(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
+                   void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s,
+                   DropArgs drop);
 void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
                    void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s,
                    DropArgs drop = DropArgs{});

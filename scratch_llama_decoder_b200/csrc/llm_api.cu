@@ -1481,6 +1481,49 @@ extern "C" int llm_kernel_attention_fwd_bf16(const void *d_qkv, void *d_o, float
   return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
 }
 
+extern "C" int llm_kernel_attention_fwd_f32(const float *d_qkv, float *d_o, float *d_lse, int batch,
+                                            int ctx, int n_head, int n_kv_head, int head_dim,
+                                            int tiled, void *stream) {
+  if (!attn_args_ok(d_qkv, d_o, batch, ctx, n_head, n_kv_head, head_dim) || !d_lse)
+    return LLM_ERR_ARG;
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
+  g_launches = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (tiled) {
+    if (((uintptr_t)d_qkv | (uintptr_t)d_o) & 15) return LLM_ERR_ARG;
+    if (!attn_fwd_f32_tiled(d_qkv, d_o, d_lse, batch, ctx, n_head, n_kv_head, head_dim, s))
+      return LLM_ERR_ARG;
+  } else {
+    attn_fwd_rows(d_qkv, d_o, d_lse, DT_F32, batch, ctx, n_head, n_kv_head, head_dim, s,
+                  DropArgs{});
+  }
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+extern "C" int llm_kernel_attention_bwd_f32(const float *d_qkv, const float *d_o,
+                                            const float *d_dout, const float *d_lse, float *d_D,
+                                            float *d_dqkv, int batch, int ctx, int n_head,
+                                            int n_kv_head, int head_dim, int tiled,
+                                            void *stream) {
+  if (!attn_args_ok(d_qkv, d_o, batch, ctx, n_head, n_kv_head, head_dim) || !d_dout || !d_lse ||
+      !d_D || !d_dqkv)
+    return LLM_ERR_ARG;
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
+  g_launches = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (tiled) {
+    if (((uintptr_t)d_qkv | (uintptr_t)d_o | (uintptr_t)d_dout | (uintptr_t)d_dqkv) & 15)
+      return LLM_ERR_ARG;
+    if (!attn_bwd_f32_tiled(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, batch, ctx, n_head,
+                            n_kv_head, head_dim, s))
+      return LLM_ERR_ARG;
+  } else {
+    attn_bwd_rows(d_qkv, d_o, d_dout, d_lse, d_D, d_dqkv, DT_F32, batch, ctx, n_head, n_kv_head,
+                  head_dim, s, DropArgs{});
+  }
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
 extern "C" int llm_kernel_attention_bwd_bf16(const void *d_qkv, const void *d_o,
                                              const void *d_dout, const float *d_lse, float *d_D,
                                              void *d_dqkv, int batch, int ctx, int n_head,

@@ -152,3 +152,62 @@ def test_attention_fwd_bwd_vs_oracle(B, T, H, Hkv, hd, tc):
             ref = dq_ref[:, lo:hi]
             err = np.linalg.norm(dg[b][:, lo:hi] - ref) / max(np.linalg.norm(ref), 1e-3 * full)
             assert err < 2e-2, (b, lo, err)
+
+
+# float32 attention (the float32 configurations): head sizes 32 and 64 with
+# tile multiples, ragged lengths, one position, GQA and MQA, the C2 shape
+ATTN32 = [(1, 64, 2, 2, 32), (2, 200, 4, 2, 32), (1, 130, 2, 2, 64), (3, 1, 4, 1, 64),
+          (2, 333, 4, 4, 32), (1, 256, 4, 4, 32), (2, 129, 8, 2, 64)]
+
+
+@pytest.mark.parametrize("tiled", [1, 0])
+@pytest.mark.parametrize("B,T,H,Hkv,hd", ATTN32)
+def test_attention_f32_vs_oracle(B, T, H, Hkv, hd, tiled):
+    """tiled: 1 = the tiled CUDA-core kernels, 0 = one warp per row; fp32
+    gates (the float32 configurations' logits and gradient tolerances)."""
+    import scratch_llama_decoder_b200 as P
+    rng = np.random.default_rng(7 * B + T + H + hd)
+    d, kvd = H * hd, Hkv * hd
+    w = d + 2 * kvd
+    qkv = torch.tensor(rng.standard_normal((B * T, w)), dtype=torch.float32)
+    dout = torch.tensor(rng.standard_normal((B * T, d)), dtype=torch.float32)
+    qd, dd = qkv.cuda(), dout.cuda()
+    o = torch.zeros(B * T, d, device="cuda")
+    lse = torch.zeros(B, H, T, device="cuda")
+    Dv = torch.zeros(B, H, T, device="cuda")
+    dq = torch.full((B * T, w), float("nan"), device="cuda")
+    p = lambda t: C.c_void_p(t.data_ptr())
+    assert P.lib.llm_kernel_attention_fwd_f32(p(qd), p(o), p(lse), B, T, H, Hkv, hd, tiled,
+                                              None) == 0
+    assert P.lib.llm_kernel_attention_bwd_f32(p(qd), p(o), p(dd), p(lse), p(Dv), p(dq), B, T, H,
+                                              Hkv, hd, tiled, None) == 0
+    torch.cuda.synchronize()
+    q64 = qkv.double().numpy().reshape(B, T, w)
+    d64 = dout.double().numpy().reshape(B, T, d)
+    og = o.double().cpu().numpy().reshape(B, T, d)
+    lg = lse.double().cpu().numpy()
+    dg = dq.double().cpu().numpy().reshape(B, T, w)
+    assert np.isfinite(dg).all()
+    for b in range(B):
+        o_ref, lse_ref, _ = O.attention_fwd(q64[b], d, H, Hkv)
+        dq_ref = O.attention_bwd(q64[b], d64[b], d, H, Hkv)
+        assert np.linalg.norm(og[b] - o_ref) / np.linalg.norm(o_ref) < 1e-5
+        assert np.abs(lg[b] - lse_ref).max() < 1e-5
+        # a block whose exact value vanishes (T = 1) keeps the fp32 rounding of
+        # D = dO . O against dP = dO . v (O(hd eps) of dP): its floor is a
+        # hundredth of the sequence's gradient scale
+        full = np.linalg.norm(dq_ref)
+        for lo, hi in ((0, d), (d, d + kvd), (d + kvd, w)):
+            ref = dq_ref[:, lo:hi]
+            err = np.linalg.norm(dg[b][:, lo:hi] - ref) / max(np.linalg.norm(ref), 1e-2 * full)
+            assert err < 1e-4, (b, lo, err)
+
+
+def test_attention_f32_tiled_rejects_other_head_sizes():
+    import scratch_llama_decoder_b200 as P
+    x = torch.zeros(64, 3 * 16, device="cuda")
+    o = torch.zeros(64, 16, device="cuda")
+    lse = torch.zeros(1, 1, 64, device="cuda")
+    p = lambda t: C.c_void_p(t.data_ptr())
+    assert P.lib.llm_kernel_attention_fwd_f32(p(x), p(o), p(lse), 1, 64, 1, 1, 16, 1, None) == \
+        P.LLM_ERR_ARG
