@@ -60,9 +60,9 @@ METRIC = "training tokens/sec (fwd+bwd+AdamW) on 1 B200; % of tensor/HBM rooflin
 # DRAM bytes (read + write) per tcgen05 GEMM launch, averaged over the 243
 # GEMM launches of one 350M step (profiles/gemm_dram_traffic_step_350m.md);
 # valid only for the GEMM sources that were captured, identified by hash.
-GEMM_TRAFFIC = {"bytes_per_launch": 256.7e6, "workload": "350m-v32000-d1024-l20-bf16",
-                "sha256": {"gemm_tc.cu": "9838f30d7c2ce88eb8d140bce74b03db53dc827e2a0c68d7882854c62a1ca37d",
-                           "tcgen05.cuh": "062e7fbd85e8e8eb829ae9081c3849a887fdfcfea2721b394d186b20100514a8"}}
+GEMM_TRAFFIC = {"bytes_per_launch": 257.8e6, "workload": "350m-v32000-d1024-l20-bf16",
+                "sha256": {"gemm_tc.cu": "e21de602194e9d98e168e1a9787ac6956b70f4c19bb680a3b3032000f1c58a0c",
+                           "tcgen05.cuh": "3ec0ac326a7fbd3690692656fd8581d42175193edc7eb03dbfaf27afa97b1c4a"}}
 
 
 def gemm_traffic(workload):
