@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t col_o = COL_O + 64 * grp;
     const float sl2 = scale * LOG2E;
-    int gb = 0;
+    int gb = 0, st_slot = -1;  // Q slot whose O store is still to be released
     for (int rr = 0, it = 0;; rr++, it++) {
       const int item = sched_item(rr, G, cta);
       if (item >= n_items) break;
@@ -392,6 +392,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full + 8 * ((gb & 1) * NQ + grp));
+        // the previous item's O store has long read its tile: release the slot
+        if (st_slot >= 0) {
+          if (lane == 0) {
+            bulk_wait_read();
+            mbar_arrive(q_empty + 8 * st_slot);
+          }
+          st_slot = -1;
+        }
       }
       // the groups meet: shared reference m, combined sum and output; every
       // accumulator is complete once every o_done phase of the item's last
@@ -453,10 +461,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int r0 = quarter * 32 + grp * 8;
         tma_store_3d(&tm_o, smem_u32(sQ + (it & 1) * TILE_BYTES + r0 * 128), h * HD, q0 + r0, b);
         bulk_commit();
-        bulk_wait_read();
-        mbar_arrive(q_empty + 8 * (it & 1));
       }
-      __syncwarp();
+      st_slot = it & 1;  // released after the next item's first block
       if (grp == 0 && qi < T) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
     }
     if (lane == 0) bulk_wait_all();

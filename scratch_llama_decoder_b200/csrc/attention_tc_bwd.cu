@@ -154,10 +154,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  v_empty = v_full + 8 * STAGES, s_full = v_empty + 8 * STAGES, s_free = s_full + 8,
                  ds_full = s_free + 8,    // [2]: key half a, b
                  dq_done = ds_full + 16,  // [2]
-                 red_full = dq_done + 16, acc_free = red_full + 8,
+                 acc_free = dq_done + 16,
                  drain = acc_free + 8,    // [2]: one per MMA warp
-                 qsync = drain + 16;      // [4]: per lane quarter, its rows of dQ staged
-  static_assert(6 + 4 * STAGES + 14 <= 48, "barriers overlap the TMEM address word");
+                 qsync = drain + 16,      // [4]: per lane quarter, its rows of dQ staged
+                 qred = qsync + 32;       // [4]: per lane quarter, its rows' D parts written
+  static_assert(6 + 4 * STAGES + 18 <= 48, "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -195,9 +196,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(dq_done + 8 * x, 1);
       mbar_init(drain + 8 * x, 1);
     }
-    mbar_init(red_full, 32 * EW_WARPS);
     mbar_init(acc_free, EW_WARPS);  // the accumulators of the item were read out
-    for (int q = 0; q < 4; q++) mbar_init(qsync + 8 * q, 32 * NCQ);
+    for (int q = 0; q < 4; q++) {
+      mbar_init(qsync + 8 * q, 32 * NCQ);
+      mbar_init(qred + 8 * q, 32 * NCQ);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_512(tmem_sh);
@@ -361,7 +364,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool ok = true;
-    int gb = 0;
+    int gb = 0, st_slot = -1;  // slot whose dQ store is still to be released
     for (int rr = 0, it = 0; ok; rr++, it++) {
       const int item = sched_item(rr, G, cta);
       if (item >= n_items) break;
@@ -401,14 +404,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_arrive(qd_empty + 8 * slot);  // and its dO row
       float *rd = red + (it & 1) * NCQ * 128;
       rd[cq * 128 + r] = dpart;
-      mbar_arrive(red_full);
-      if (!warp_wait(red_full, it & 1, abort_sh, gflag)) {
+      // the row's four column groups are the four warps of this lane quarter
+      mbar_arrive(qred + 8 * quarter);
+      if (!warp_wait(qred + 8 * quarter, it & 1, abort_sh, gflag)) {
         ok = false;
         break;
       }
       float Di = 0.f;
 #pragma unroll
       for (int c = 0; c < NCQ; c++) Di += rd[c * 128 + r];
+      // the previous item's dQ store has long read its tile: release the slot
+      if (st_slot >= 0) {
+        if (lane == 0) {
+          bulk_wait_read();
+          mbar_arrive(qd_empty + 8 * st_slot);
+        }
+        st_slot = -1;
+      }
       if (cq == 0 && valid) Dv[((int64_t)b * H + h) * T + qi] = Di;
       const float2 nl = make_float2(nl2, nl2), nd = make_float2(-Di, -Di);
       for (int j = 0; j < nj && ok; j++, gb++) {
@@ -503,10 +515,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int r0 = quarter * 32 + cq * 8;
         tma_store_3d(&tm_st, smem_u32(sQ + slot * TILE_BYTES + r0 * 128), h * HD, q0 + r0, b);
         bulk_commit();
-        bulk_wait_read();
-        mbar_arrive(qd_empty + 8 * slot);
       }
-      __syncwarp();
+      st_slot = slot;  // released (below) once the store has read the tile
     }
     if (lane == 0) bulk_wait_all();
   }
@@ -738,7 +748,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool ok = true;
-    int gs = 0;
+    int gs = 0, st_slot = -1;  // slot whose dK/dV stores are still to be released
     for (int rr = 0, it = 0; ok; rr++, it++) {
       const int item = sched_item(rr, G, cta);
       if (item >= n_items) break;
@@ -821,6 +831,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
+        // the previous item's dK/dV stores have long read their tiles
+        if (st_slot >= 0) {
+          if (lane == 0) {
+            bulk_wait_read();
+            mbar_arrive(kv_empty + 8 * st_slot);
+          }
+          st_slot = -1;
+        }
       }
       if (!ok) break;
       if (!warp_wait(pv_done, (gs - 1) & 1, abort_sh, gflag)) {
@@ -857,10 +875,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_store_3d(&tm_st, smem_u32(sV + slot * TILE_BYTES + r0 * 128), d + kvd + g * HD,
                      k0 + r0, b);
         bulk_commit();
-        bulk_wait_read();
-        mbar_arrive(kv_empty + 8 * slot);
       }
-      __syncwarp();
+      st_slot = slot;  // released after the next item's first step
     }
     if (lane == 0) bulk_wait_all();
   }
