@@ -32,10 +32,10 @@
 // is rescaled only then.  The maximum is taken on the raw scores (the log2
 // scale is positive) and only the diagonal block runs the causal mask, so an
 // off-diagonal block costs half a three-input maximum, half a packed f32x2
-// multiply-add and one exponential per score; 5 of every 16 pairs of
+// multiply-add and one exponential per score; NP_FWD of every 16 pairs of
 // exponentials run as a polynomial on the FMA pipe (exp2_poly2), the rest on
-// the SFU, whose 16 results per clock and SM would otherwise bound the
-// softmax.  MMAs are issued by whole converged warps (one elected lane).  Every wait is bounded (FLAG_TIMEOUT, then drain and free
+// the SFU (16 results per clock and SM); the split was chosen by measurement
+// (0 to 6 of 16 within 5% of each other, 3 the fastest).  MMAs are issued by whole converged warps (one elected lane).  Every wait is bounded (FLAG_TIMEOUT, then drain and free
 // TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
@@ -45,6 +45,14 @@ namespace llm {
 namespace attn_tc {
 
 using namespace tc;
+
+// 2^x for pair i of a 16-pair chunk: NP of the 16 pairs (spread over the
+// chunk) by the polynomial on the FMA pipe, the rest by the SFU.
+template <int NP>
+LLM_DEV float2 exp2_split(float2 x, int i) {
+  return ((i & 15) * NP) % 16 < NP ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+}
+constexpr int NP_FWD = 3;
 
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
@@ -77,7 +85,7 @@ LLM_DEV float exp_pack(const float (&sv)[KW], float sl2, float mr, uint32_t (&w)
   for (int i = 0; i < KW; i += 2) {
     const float2 x = __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2),
                                 make_float2(-mr, -mr));
-    const float2 p = FMA_EXP ? exp2_pair(x, i / 2) : make_float2(ex2(x.x), ex2(x.y));
+    const float2 p = FMA_EXP ? exp2_split<NP_FWD>(x, i / 2) : make_float2(ex2(x.x), ex2(x.y));
     if ((i >> 1) & 1) lb = __fadd2_rn(lb, p);
     else la = __fadd2_rn(la, p);
     w[i / 2] = pack_bf16(p.x, p.y);
@@ -383,7 +391,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float mr = m_ref == -INFINITY ? 0.f : m_ref;
         uint32_t w[KW / 2];
         // the diagonal block on the SFU alone (its masked scores give exact
-        // zeros); elsewhere some pairs on the FMA pipe (exp2_pair)
+        // zeros); elsewhere some pairs on the FMA pipe (exp2_split)
         l += diag ? exp_pack<false>(sv, sl2, mr, w) : exp_pack<true>(sv, sl2, mr, w);
 #pragma unroll
         for (int c = 0; c < KW / 2; c += 16)

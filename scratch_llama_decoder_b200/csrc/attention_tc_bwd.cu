@@ -35,9 +35,10 @@
 // dQ and dK leave through the backward of the rotate-half RoPE (when tables
 // are given), then scale, bf16.  No atomics: every output element is written
 // once by the CTA that owns its row.  The elementwise arithmetic runs on
-// packed f32x2 pairs, and 5 of every 16 pairs of exponentials take the
-// polynomial 2^x on the FMA pipe (exp2_poly2) so that the SFU (16 results per
-// clock and SM) does not bound the loop alone.  Every wait is bounded
+// packed f32x2 pairs; NP_DQ (dQ) and NP_DKV (dK/dV) of every 16 pairs of
+// exponentials take the polynomial 2^x on the FMA pipe (exp2_poly2), the rest
+// the SFU (splits chosen by measurement: dQ fastest at 3, dK/dV at 0, whose
+// ALU pipe is the busier).  Every wait is bounded
 // (FLAG_TIMEOUT, then drain and free TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
@@ -47,6 +48,15 @@ namespace llm {
 namespace attn_tc_bwd {
 
 using namespace tc;
+
+// 2^x for pair i of a 16-pair chunk: NP of the 16 pairs (spread over the
+// chunk) by the polynomial on the FMA pipe, the rest by the SFU.
+template <int NP>
+LLM_DEV float2 exp2_split(float2 x, int i) {
+  return ((i & 15) * NP) % 16 < NP ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+}
+constexpr int NP_DQ = 3;
+constexpr int NP_DKV = 0;
 
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
@@ -441,7 +451,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (diag) {  // the causal mask only on the diagonal block
 #pragma unroll
           for (int i = 0; i < CW; i += 2) {
-            float2 p = exp2_pair(
+            float2 p = exp2_split<NP_DQ>(
                 __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2), nl), i / 2);
             if (k0 + i > qi) p.x = 0.f;
             if (k0 + i + 1 > qi) p.y = 0.f;
@@ -451,7 +461,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else {
 #pragma unroll
           for (int i = 0; i < CW; i += 2) {
-            const float2 p = exp2_pair(
+            const float2 p = exp2_split<NP_DQ>(
                 __ffma2_rn(make_float2(sv[i], sv[i + 1]), make_float2(sl2, sl2), nl), i / 2);
             const float2 ds = __fmul2_rn(p, __fadd2_rn(make_float2(dv[i], dv[i + 1]), nd));
             w[i / 2] = pack_bf16(ds.x, ds.y);
@@ -800,7 +810,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                           nl01);
             const float2 x23 = __ffma2_rn(make_float2(sv[i + 2], sv[i + 3]),
                                           make_float2(sl2, sl2), nl23);
-            float2 p01 = exp2_pair(x01, c / 2), p23 = exp2_pair(x23, c / 2 + 1);
+            float2 p01 = exp2_split<NP_DKV>(x01, c / 2), p23 = exp2_split<NP_DKV>(x23, c / 2 + 1);
             if (diag) {
               if (kj > qc0 + c) p01.x = 0.f;
               if (kj > qc0 + c + 1) p01.y = 0.f;
