@@ -584,6 +584,11 @@ def kernel_rates(classes, steps, pk, src):
             # float32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 FLOPs x 1.965 GHz
             rate, peak, u = work / (ms / 1e3) / 1e12, FP32_SIMT_TFLOPS, "TFLOP/s"
             ps = "nominal float32 CUDA-core FMA rate"
+        elif unit == "flop" and name == "gemm_tf32":
+            # three tf32 products per float32 product: the bound is a third of
+            # the tf32 rate (the bf16 peak times the nominal tf32/bf16 ratio)
+            rate, peak, u = work / (ms / 1e3) / 1e12, peak_tc * TF32_OF_BF16 / 3, "TFLOP/s"
+            ps = f"{src} bf16_tflops_sustained x 1.1/2.25 / 3 (3xTF32)"
         elif unit == "flop":
             rate, peak, u = work / (ms / 1e3) / 1e12, peak_tc, "TFLOP/s"
             ps = f"{src} bf16_tflops_sustained"

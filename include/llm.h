@@ -470,7 +470,9 @@ enum {
   LLM_KT_WEIGHT_CAST = 11,
   LLM_KT_WGRAD_FINISH = 12,
   LLM_KT_GEMM_CUDA_CORE = 13, /* float32 projection GEMMs on CUDA cores (FLOPs) */
-  LLM_KT_CLASSES = 14
+  LLM_KT_GEMM_TF32 = 14,      /* float32 projection GEMMs on the tensor cores, split
+                                 precision (3xTF32), with their operand split (FLOPs) */
+  LLM_KT_CLASSES = 15
 };
 int llm_set_kernel_timing(llm_ctx *ctx, int enable);
 int llm_read_kernel_timing(llm_ctx *ctx, double *ms, double *flops, int64_t *launches);

@@ -30,6 +30,20 @@ int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_t lda, int 
                          const void *d_B, int64_t ldb, int b_kmajor, float *d_C, int64_t ldc,
                          int tensor_cores, int *d_flag, void *stream);
 
+/* The same product with float32 operands (the float32 configurations):
+ * tensor_cores = 1 runs the split-precision tensor-core kernel (3xTF32: each
+ * operand split into a tf32 part and a float32 remainder, three tcgen05
+ * kind::tf32 products accumulated in float32; relative error about 2^-21
+ * per product), which first writes both parts of A and B, K-major, into
+ * d_scratch: at least llm_kernel_gemm_f32_scratch_floats(M, N, K) floats,
+ * 16-byte aligned, contents need no initialisation, LLM_ERR_ARG if smaller;
+ * 0 runs the CUDA-core kernel (d_scratch unused).  d_flag as above. */
+int llm_kernel_gemm_f32_scratch_floats(int M, int N, int K, int64_t *floats);
+int llm_kernel_gemm_f32(int M, int N, int K, const float *d_A, int64_t lda, int a_kmajor,
+                        const float *d_B, int64_t ldb, int b_kmajor, float *d_C, int64_t ldc,
+                        int tensor_cores, float *d_scratch, int64_t scratch_floats, int *d_flag,
+                        void *stream);
+
 /* Causal self-attention of the step, bfloat16 operands and float32 softmax
  * (Hephaistos, Architecture at a glance: causal multi-head attention with a
  * numerically stable softmax; strata: n_head and n_kv_head independent,

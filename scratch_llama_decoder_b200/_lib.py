@@ -44,7 +44,7 @@ KERNEL_CLASSES = [("gemm", "flop"), ("attention_fwd", "flop"), ("attention_bwd",
                   ("rmsnorm_fwd", "byte"), ("rmsnorm_bwd", "byte"), ("swiglu_fwd", "byte"),
                   ("swiglu_bwd", "byte"), ("cross_entropy", "byte"), ("embed_fwd", "byte"),
                   ("embed_bwd", "byte"), ("adamw", "byte"), ("weight_cast", "byte"),
-                  ("wgrad_finish", "byte"), ("gemm_cuda_core", "flop")]
+                  ("wgrad_finish", "byte"), ("gemm_cuda_core", "flop"), ("gemm_tf32", "flop")]
 LR_SHAPES = {"constant": LLM_LR_CONSTANT, "cosine": LLM_LR_COSINE, "linear": LLM_LR_LINEAR}
 
 
@@ -105,6 +105,9 @@ EXPORTS = {
     # include/llm_kernels.h
     "llm_kernel_gemm_bf16": (_i, [_i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp,
                                   _vp]),
+    "llm_kernel_gemm_f32_scratch_floats": (_i, [_i, _i, _i, C.POINTER(_i64)]),
+    "llm_kernel_gemm_f32": (_i, [_i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp,
+                                 _i64, _vp, _vp]),
     "llm_kernel_attention_fwd_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "llm_kernel_attention_bwd_bf16": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                            _vp]),

@@ -40,6 +40,13 @@ enum GemmOut {
   OUT_ADD_F32 = 2,  // C (float) = R + acc
   OUT_PARTIAL = 3   // C (float) [split][M][ldc] = partial sum over the split's K range
 };
+// float32 GEMM on the tensor cores in split precision (3xTF32, gemm_tf32.cu):
+// false (nothing launched) unless A, B are float32 and the scratch holds
+// gemm_tf32_scratch_floats(M, N, K) floats (16-byte aligned).  Counts launches.
+int64_t gemm_tf32_scratch_floats(int64_t M, int64_t N, int64_t K);
+bool gemm_tf32(const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
+               int64_t ldr, int splits, float *scratch, int64_t scratch_floats, int *flag,
+               cudaStream_t s);
 // SIMT (CUDA-core) GEMM: any shape, float32 accumulation.  Counts launches.
 void gemm_simt(const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
                int64_t ldr, int splits, cudaStream_t s);

@@ -148,6 +148,11 @@ struct llm_ctx {
   void *xf, *logits;
   float *rstdf, *rowloss;
   float *dx, *dtmp, *Dbuf, *part, *dgpart;
+  // float32 configurations: split-precision operand copies of the tensor-core
+  // GEMM, one region per stream (the side stream's weight gradients run
+  // concurrently with the main stream's GEMMs)
+  float *tf32_scratch[2] = {nullptr, nullptr};
+  int64_t tf32_floats = 0;
   void *dxA, *du, *dab, *dO, *dqkv;
   int32_t *sort_scratch;
   TcPlan *tc = nullptr;
@@ -250,6 +255,22 @@ int64_t llm_ctx::carve(char *base) {
   };
   need(d, D_.Vp); need(D_.hp, d); need(d, 2 * D_.hp); need(d, d); need(d, D_.qkvw);
   part = (float *)c.take(4 * part_elems);
+  if (D_.dt == DT_F32) {
+    // every GEMM of the step: forward (M = tokens), data gradients, weight
+    // gradients (K = tokens)
+    int64_t tf = 0;
+    auto tneed = [&](int64_t M, int64_t Nn, int64_t K) {
+      tf = std::max<int64_t>(tf, gemm_tf32_scratch_floats(M, Nn, K));
+    };
+    tneed(N, D_.qkvw, d); tneed(N, d, d); tneed(N, 2 * D_.hp, d); tneed(N, d, D_.hp);
+    tneed(N, D_.Vp, d); tneed(N, d, D_.Vp); tneed(N, D_.hp, d); tneed(N, d, 2 * D_.hp);
+    tneed(N, d, D_.qkvw);
+    tneed(d, D_.Vp, N); tneed(D_.hp, d, N); tneed(d, 2 * D_.hp, N); tneed(d, d, N);
+    tneed(d, D_.qkvw, N);
+    tf32_floats = tf;
+    tf32_scratch[0] = (float *)c.take(4 * tf);
+    tf32_scratch[1] = (float *)c.take(4 * tf);
+  }
   dgpart = (float *)c.take(4 * (int64_t)rmsnorm_bwd_blocks(N) * d);
   sort_scratch = (int32_t *)c.take(4 * embed_bwd_scratch_ints(N, D_.V));
   // decode: the four matrix-vector shapes of a layer and the lm_head
@@ -684,6 +705,13 @@ bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
 void gemm(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
           int64_t ldr, int splits, double alg_flops) {
   if (run_tc(c, g, out, C, ldc, R, ldr, splits, TC_EPI_NONE, alg_flops)) return;
+  if (g.in == DT_F32 && c->tf32_floats > 0) {
+    KTimer kt(c, LLM_KT_GEMM_TF32, alg_flops);
+    float *scr = c->tf32_scratch[c->cur == c->s2 && c->s2 ? 1 : 0];
+    if (gemm_tf32(g, out, C, ldc, R, ldr, splits, scr, c->tf32_floats, c->flag_step, c->cur))
+      return;
+    kt.drop();
+  }
   KTimer kt(c, LLM_KT_GEMM_CUDA_CORE, alg_flops);
   gemm_simt(g, out, C, ldc, R, ldr, splits, c->cur);
 }
@@ -738,10 +766,7 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
     bool fused = run_tc(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, TC_EPI_ROPE,
                         2.0 * N * d * D.qkvw);
     if (!fused) {
-      {
-        KTimer kt(c, LLM_KT_GEMM_CUDA_CORE, 2.0 * N * d * D.qkvw);
-        gemm_simt(g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, s);
-      }
+      gemm(c, g, OUT_ACT, qkv, D.qkvw, nullptr, 0, 1, 2.0 * N * d * D.qkvw);
       rope_apply(qkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, 1, s);
     }
   }
@@ -1418,6 +1443,34 @@ extern "C" int llm_kernel_gemm_bf16(int M, int N, int K, const void *d_A, int64_
     if (!plan) return LLM_ERR_ARG;
     tc_plan_set_flag(plan, d_flag);
     if (!tc_gemm(plan, g, OUT_F32, d_C, ldc, nullptr, 0, 1, TC_EPI_NONE, s))
+      return LLM_ERR_ARG;
+  } else {
+    gemm_simt(g, OUT_F32, d_C, ldc, nullptr, 0, 1, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? LLM_OK : LLM_ERR_CUDA;
+}
+
+extern "C" int llm_kernel_gemm_f32_scratch_floats(int M, int N, int K, int64_t *floats) {
+  if (M < 1 || N < 1 || K < 1 || !floats) return LLM_ERR_ARG;
+  *floats = gemm_tf32_scratch_floats(M, N, K);
+  return LLM_OK;
+}
+
+extern "C" int llm_kernel_gemm_f32(int M, int N, int K, const float *d_A, int64_t lda,
+                                   int a_kmajor, const float *d_B, int64_t ldb, int b_kmajor,
+                                   float *d_C, int64_t ldc, int tensor_cores, float *d_scratch,
+                                   int64_t scratch_floats, int *d_flag, void *stream) {
+  if (M < 1 || N < 1 || K < 1 || !d_A || !d_B || !d_C || !d_flag) return LLM_ERR_ARG;
+  if (lda < (a_kmajor ? K : M) || ldb < (b_kmajor ? K : N) || ldc < N) return LLM_ERR_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  GemmOperands g{M, N, K, d_A, lda, a_kmajor != 0, d_B, ldb, b_kmajor != 0, DT_F32};
+  if (!claim_device(nullptr)) return LLM_ERR_ARG;  // one device per process
+  g_launches = 0;
+  if (tensor_cores) {
+    if (!d_scratch || scratch_floats < gemm_tf32_scratch_floats(M, N, K) ||
+        ((uintptr_t)d_scratch & 15))
+      return LLM_ERR_ARG;
+    if (!gemm_tf32(g, OUT_F32, d_C, ldc, nullptr, 0, 1, d_scratch, scratch_floats, d_flag, s))
       return LLM_ERR_ARG;
   } else {
     gemm_simt(g, OUT_F32, d_C, ldc, nullptr, 0, 1, s);

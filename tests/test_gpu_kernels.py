@@ -55,6 +55,65 @@ def test_gemm_bf16(M, N, K, a_k, b_k, tc):
     assert err < 1e-5, err
 
 
+# float32 GEMM shapes: tile multiples, ragged tails, K not a multiple of 32,
+# the float32 workload's (tokens x 384 x 128, weight gradient over tokens)
+SHAPES32 = [(128, 128, 32), (200, 300, 136), (1, 8, 8), (640, 768, 500), (16384, 384, 128),
+            (128, 500, 16384), (333, 129, 77)]
+
+
+@pytest.mark.parametrize("a_k,b_k", [(1, 0), (1, 1), (0, 0), (0, 1)])
+@pytest.mark.parametrize("M,N,K", SHAPES32)
+@pytest.mark.parametrize("tc", [1, 0])
+def test_gemm_f32(M, N, K, a_k, b_k, tc):
+    """tc = 1: split-precision tensor-core kernel (3xTF32); 0: CUDA cores.
+    Gate 1e-5 norm-wise: 3xTF32 keeps about 2^-21 per product and the
+    float32 accumulation adds its rounding; a single tf32 product (2^-11) would
+    fail it.  (One TMEM accumulation chain over K = 16384 measured 1.1e-4,
+    four interleaved chains 2.9e-5: the tensor core's float32 accumulation
+    drops low bits per addition, so the kernel drains its accumulator into
+    float32 registers every 512 of K.)"""
+    import scratch_llama_decoder_b200 as P
+    rng = np.random.default_rng(M * 5 + N * 11 + K)
+    A = torch.tensor(rng.standard_normal((M, K) if a_k else (K, M)), dtype=torch.float32)
+    B = torch.tensor(rng.standard_normal((N, K) if b_k else (K, N)), dtype=torch.float32)
+    lda, ldb = A.shape[1], B.shape[1]
+    Ad, Bd = A.cuda().contiguous(), B.cuda().contiguous()
+    ldc = (N + 3) // 4 * 4
+    Cd = torch.full((M, ldc), float("nan"), device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nf = C.c_int64(0)
+    assert P.lib.llm_kernel_gemm_f32_scratch_floats(M, N, K, C.byref(nf)) == 0
+    scratch = torch.empty(max(1, nf.value), device="cuda")
+    rc = P.lib.llm_kernel_gemm_f32(M, N, K, C.c_void_p(Ad.data_ptr()), lda, a_k,
+                                   C.c_void_p(Bd.data_ptr()), ldb, b_k,
+                                   C.c_void_p(Cd.data_ptr()), ldc, tc,
+                                   C.c_void_p(scratch.data_ptr()), nf.value,
+                                   C.c_void_p(flag.data_ptr()), None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    got = Cd[:, :N].double().cpu().numpy()
+    a64, b64 = A.double().numpy(), B.double().numpy()
+    ref = O.mm_nt(a64 if a_k else a64.T, b64 if b_k else b64.T)
+    err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert err < 1e-5, err
+    assert np.abs(got - ref).max() <= 1e-4 * np.abs(ref).max()
+
+
+def test_gemm_f32_scratch_too_small():
+    import scratch_llama_decoder_b200 as P
+    A = torch.zeros(64, 64, device="cuda")
+    Cd = torch.zeros(64, 64, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nf = C.c_int64(0)
+    assert P.lib.llm_kernel_gemm_f32_scratch_floats(64, 64, 64, C.byref(nf)) == 0
+    scratch = torch.empty(nf.value, device="cuda")
+    p = C.c_void_p(A.data_ptr())
+    assert P.lib.llm_kernel_gemm_f32(64, 64, 64, p, 64, 1, p, 64, 1, C.c_void_p(Cd.data_ptr()),
+                                     64, 1, C.c_void_p(scratch.data_ptr()), nf.value - 4,
+                                     C.c_void_p(flag.data_ptr()), None) == P.LLM_ERR_ARG
+
+
 @pytest.mark.parametrize("N,d,V", [(16, 16, 27), (16384, 1024, 32000), (1000, 64, 500),
                                    (300, 48, 70000)])
 def test_embed_bwd_vs_oracle(N, d, V):
