@@ -10,15 +10,18 @@
 //
 // A split pass (k_tf32_split) writes hi and lo of each operand K-major,
 // [rows][Kp] with Kp = K rounded up to 32 (zeros past K), transposing the
-// MN-major operands through shared memory.  The GEMM kernel: one CTA per
-// 128 x 128 output tile (and K split), warp 0 the TMA producer (Ahi, Alo,
+// MN-major operands through shared memory.  The GEMM kernel: persistent, one
+// CTA per SM over the 128 x 128 output tiles (and K splits), warp 0 the TMA
+// producer (Ahi, Alo,
 // Bhi, Blo tiles of 128 rows x 32 floats, 128-byte swizzle, a 3-deep ring),
 // warp 1 allocates TMEM and issues per K step of 8 the three products
 // (tcgen05.mma kind::tf32, M 128, N 128, K 8), warps 2-5 read the
 // accumulator rows from TMEM and write them out (float32, plus a residual,
 // or a split's partial slab).  The accumulation runs in chunks of 16 K blocks
 // in two TMEM buffers, each finished chunk added into float32 registers by the
-// epilogue warps, which bounds the tensor core's own accumulation chains.  Every wait is bounded (2 s, FLAG_TIMEOUT).
+// epilogue warps, which bounds the tensor core's own accumulation chains (and,
+// over a CTA's items, lets one tile's stores overlap the next tile's
+// products).  Every wait is bounded (2 s, FLAG_TIMEOUT).
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -102,6 +105,7 @@ __global__ void __launch_bounds__(256) k_tf32_split(const float *__restrict__ X,
 
 struct Args {
   int M, N, Kp, kchunk;  // kchunk: K floats per split (a multiple of 32)
+  int tiles_n, tiles, splits;  // work items: tiles x splits, tile = (row block, column block)
   int out;               // GemmOut
   float *C;
   int64_t ldc;
@@ -111,6 +115,9 @@ struct Args {
   int *flag;
 };
 
+// Persistent: gridDim.x CTAs take the work items (tile, split) round-robin.
+// The ring stages and the TMEM chunk buffers are counted over all of a CTA's
+// items, so an item's stores overlap the next item's products.
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm_tf32(const __grid_constant__ CUtensorMap tAh, const __grid_constant__ CUtensorMap tAl,
                 const __grid_constant__ CUtensorMap tBh, const __grid_constant__ CUtensorMap tBl,
@@ -125,9 +132,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  tfull = empty0 + 8 * STAGES,  // [2]: chunk of the buffer accumulated
                  tempty = tfull + 16,          // [2]: chunk of the buffer read out
                  drain = tempty + 16;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM, split = blockIdx.z;
-  const int kf0 = split * a.kchunk, kf1 = min(a.Kp, kf0 + a.kchunk);
-  const int nkb = max(0, (kf1 - kf0) / BKF);
+  const int items = a.tiles * a.splits;
+  // item -> output tile origin and the split's K blocks
+  auto item_of = [&](int w, int &m0, int &n0, int &kf0, int &nkb) {
+    const int tile = w % a.tiles, split = w / a.tiles;
+    m0 = (tile / a.tiles_n) * BM;
+    n0 = (tile % a.tiles_n) * BN;
+    kf0 = split * a.kchunk;
+    const int kf1 = min(a.Kp, kf0 + a.kchunk);
+    nkb = max(0, (kf1 - kf0) / BKF);
+  };
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -156,59 +170,76 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    int issued = 0;
-    for (int kb = 0; kb < nkb; kb++) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!warp_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) break;
-      if (lane == 0) {
-        const uint32_t bar = full0 + 8 * s;
-        uint8_t *st = smem + s * STAGE_BYTES;
-        const int kx = kf0 + kb * BKF;
-        mbar_arrive_expect_tx(bar, STAGE_BYTES);
-        tma_load_2d(smem_u32(st), &tAh, kx, m0, bar);
-        tma_load_2d(smem_u32(st + TILE), &tAl, kx, m0, bar);
-        tma_load_2d(smem_u32(st + 2 * TILE), &tBh, kx, n0, bar);
-        tma_load_2d(smem_u32(st + 3 * TILE), &tBl, kx, n0, bar);
+    int gk = 0;  // K blocks issued over all items
+    bool ok = true;
+    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+      int m0, n0, kf0, nkb;
+      item_of(w, m0, n0, kf0, nkb);
+      for (int kb = 0; kb < nkb; kb++) {
+        const int s = gk % STAGES;
+        const uint32_t ph = (gk / STAGES) & 1;
+        if (!warp_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t bar = full0 + 8 * s;
+          uint8_t *st = smem + s * STAGE_BYTES;
+          const int kx = kf0 + kb * BKF;
+          mbar_arrive_expect_tx(bar, STAGE_BYTES);
+          tma_load_2d(smem_u32(st), &tAh, kx, m0, bar);
+          tma_load_2d(smem_u32(st + TILE), &tAl, kx, m0, bar);
+          tma_load_2d(smem_u32(st + 2 * TILE), &tBh, kx, n0, bar);
+          tma_load_2d(smem_u32(st + 3 * TILE), &tBl, kx, n0, bar);
+        }
+        gk++;
       }
-      issued = kb + 1;
     }
     if (lane == 0)
-      for (int kb = max(0, issued - STAGES); kb < issued; kb++)
-        drain_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1);
+      for (int i = max(0, gk - STAGES); i < gk; i++)
+        drain_wait(full0 + 8 * (i % STAGES), (i / STAGES) & 1);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------- MMA issuer (whole warp, elected)
     bool ok = true;
-    for (int kb = 0; kb < nkb && ok; kb++) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!warp_wait(full0 + 8 * s, ph, &abort_sh, a.flag)) {
-        ok = false;
-        break;
-      }
-      const int ci = kb / CH, buf = ci & 1;
-      // a buffer is reused once the epilogue has read its previous chunk
-      if (kb % CH == 0 && ci >= 2 && !warp_wait(tempty + 8 * buf, ((ci >> 1) - 1) & 1, &abort_sh,
-                                                 a.flag)) {
-        ok = false;
-        break;
-      }
-      fence_after();
-      uint8_t *st = smem + s * STAGE_BYTES;
-      const uint64_t ah = sdesc(smem_u32(st), 16, 1024), al = sdesc(smem_u32(st + TILE), 16, 1024);
-      const uint64_t bh = sdesc(smem_u32(st + 2 * TILE), 16, 1024),
-                     bl = sdesc(smem_u32(st + 3 * TILE), 16, 1024);
+    int gk = 0, gc = 0;  // K blocks and TMEM chunks over all items
+    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+      int m0, n0, kf0, nkb;
+      item_of(w, m0, n0, kf0, nkb);
+      for (int kb = 0; kb < nkb && ok; kb++, gk++) {
+        const int s = gk % STAGES;
+        const uint32_t ph = (gk / STAGES) & 1;
+        if (kb % CH == 0) {
+          // a buffer is reused once the epilogue has read its previous chunk
+          if (gc >= 2 && !warp_wait(tempty + 8 * (gc & 1), ((gc >> 1) - 1) & 1, &abort_sh,
+                                    a.flag)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!warp_wait(full0 + 8 * s, ph, &abort_sh, a.flag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        uint8_t *st = smem + s * STAGE_BYTES;
+        const uint64_t ah = sdesc(smem_u32(st), 16, 1024), al = sdesc(smem_u32(st + TILE), 16, 1024);
+        const uint64_t bh = sdesc(smem_u32(st + 2 * TILE), 16, 1024),
+                       bl = sdesc(smem_u32(st + 3 * TILE), 16, 1024);
+        const uint32_t acc = tmem + 128 * (gc & 1);
 #pragma unroll
-      for (int kk = 0; kk < BKF / 8; kk++) {  // K steps of 8 floats = 32 bytes
-        const uint64_t o = (uint64_t)(kk * 2);
-        const uint32_t acc = tmem + 128 * buf;
-        mma_tf32_e(acc, ah + o, bh + o, (kb % CH > 0 || kk > 0) ? 1u : 0u);
-        mma_tf32_e(acc, ah + o, bl + o, 1u);
-        mma_tf32_e(acc, al + o, bh + o, 1u);
+        for (int kk = 0; kk < BKF / 8; kk++) {  // K steps of 8 floats = 32 bytes
+          const uint64_t o = (uint64_t)(kk * 2);
+          mma_tf32_e(acc, ah + o, bh + o, (kb % CH > 0 || kk > 0) ? 1u : 0u);
+          mma_tf32_e(acc, ah + o, bl + o, 1u);
+          mma_tf32_e(acc, al + o, bh + o, 1u);
+        }
+        mma_commit_e(empty0 + 8 * s);
+        if (kb % CH == CH - 1 || kb == nkb - 1) {
+          mma_commit_e(tfull + 8 * (gc & 1));
+          gc++;
+        }
       }
-      mma_commit_e(empty0 + 8 * s);
-      if (kb % CH == CH - 1 || kb == nkb - 1) mma_commit_e(tfull + 8 * buf);
     }
     mma_commit_e(drain);
     if (lane == 0) drain_wait(drain, 0);
@@ -216,44 +247,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // --------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32 quarter .. 32 quarter + 31
-    const int m = m0 + quarter * 32 + lane;
     const uint32_t row_t = tmem + ((uint32_t)(quarter * 32) << 16);
-    float acc[BN];
-#pragma unroll
-    for (int i = 0; i < BN; i++) acc[i] = 0.f;
     bool ok = true;
-    const int nch = (nkb + CH - 1) / CH;
-    for (int ci = 0; ci < nch && ok; ci++) {
-      const int buf = ci & 1;
-      if (!warp_wait(tfull + 8 * buf, (ci >> 1) & 1, &abort_sh, a.flag)) {
-        ok = false;
-        break;
-      }
-      fence_after();
+    int gc = 0;
+    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+      int m0, n0, kf0, nkb;
+      item_of(w, m0, n0, kf0, nkb);
+      const int m = m0 + quarter * 32 + lane, split = w / a.tiles;
+      float acc[BN];
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        float w[32];
-        tmem_ldn<32>(row_t + 128 * buf + c0, w);
+      for (int i = 0; i < BN; i++) acc[i] = 0.f;
+      const int nch = (nkb + CH - 1) / CH;
+      for (int ci = 0; ci < nch; ci++, gc++) {
+        const int buf = gc & 1;
+        if (!warp_wait(tfull + 8 * buf, (gc >> 1) & 1, &abort_sh, a.flag)) {
+          ok = false;
+          break;
+        }
+        fence_after();
 #pragma unroll
-        for (int i = 0; i < 32; i++) acc[c0 + i] += w[i];
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float v[32];
+          tmem_ldn<32>(row_t + 128 * buf + c0, v);
+#pragma unroll
+          for (int i = 0; i < 32; i++) acc[c0 + i] += v[i];
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty + 8 * buf);
       }
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty + 8 * buf);
-    }
-    if (ok && m < a.M) {
+      if (!ok || m >= a.M) continue;
       float *crow = a.C + (a.out == OUT_PARTIAL ? (int64_t)split * a.M * a.ldc : 0) +
                     (int64_t)m * a.ldc;
       const float *rrow = a.R ? a.R + (int64_t)m * a.ldr : nullptr;
       if (a.vec && n0 + BN <= a.N) {
 #pragma unroll
         for (int i = 0; i < BN; i += 4) {
-          float4 w = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+          float4 v = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
           if (a.out == OUT_ADD_F32) {
             const float4 q = *reinterpret_cast<const float4 *>(rrow + n0 + i);
-            w.x += q.x; w.y += q.y; w.z += q.z; w.w += q.w;
+            v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
           }
-          *reinterpret_cast<float4 *>(crow + n0 + i) = w;
+          *reinterpret_cast<float4 *>(crow + n0 + i) = v;
         }
       } else {
 #pragma unroll
@@ -335,7 +370,10 @@ bool gemm_tf32(const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const f
   a.out = out; a.C = (float *)C; a.ldc = ldc; a.R = R; a.ldr = ldr; a.flag = flag;
   a.vec = ((uintptr_t)C & 15) == 0 && ldc % 4 == 0 &&
           (out != OUT_ADD_F32 || (((uintptr_t)R & 15) == 0 && ldr % 4 == 0));
-  dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + BM - 1) / BM), (unsigned)splits);
+  a.tiles_n = (g.N + BN - 1) / BN;
+  a.tiles = a.tiles_n * ((g.M + BM - 1) / BM);
+  a.splits = splits;
+  const int grid = std::min(a.tiles * splits, device_sms());
   k_gemm_tf32<<<grid, NTHREADS, SMEM, s>>>(tAh, tAl, tBh, tBl, a);
   count_launch();
   return true;
