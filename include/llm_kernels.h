@@ -56,7 +56,7 @@ int llm_kernel_gemm_f32(int M, int N, int K, const float *d_A, int64_t lda, int 
  * row.  Backward: from d_o, d_lse and d_dout (bf16, like d_o) writes d_dqkv
  * (bf16, like d_qkv; every element written) and d_D float32 [batch, n_head,
  * ctx] = rowsum(dout * o) as scratch.  tensor_cores selects the kernels:
- * 2 = the tcgen05/TMEM kernels (head_dim 64; pointers 16-byte aligned),
+ * 2 = the tcgen05/TMEM kernels (head_dim 32 or 64; pointers 16-byte aligned),
  * 1 = the warp-level mma kernels (head_dim 32 or 64), 0 = the CUDA-core
  * kernels; LLM_ERR_ARG if the selection does not cover head_dim.  The calls
  * are asynchronous on `stream`.  The tcgen05 kernels bound every internal

@@ -1,7 +1,9 @@
-// tcgen05 flash-attention forward for head size 64 (bf16 operands, fp32
-// softmax and accumulators): strata's online-softmax attention (no T x T
+// tcgen05 flash-attention forward for head sizes 64 and 32 (bf16 operands,
+// fp32 softmax and accumulators): strata's online-softmax attention (no T x T
 // scores in memory, only the row log-sum-exp saved) on the 5th-generation
-// tensor cores.
+// tensor cores.  A head-32 tile is loaded as the head-64 one with its upper
+// 32 columns zero (the tensor maps of attn_tma.cuh), so the same products
+// give the head-32 scores and an O whose upper half is zero and not stored.
 //
 // One CTA = 128 queries of one (batch, head); key blocks of 128, split into
 // NQ key groups of KW = 128 / NQ keys.  Warps:
@@ -39,12 +41,14 @@
 // TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
+#include "attn_tma.cuh"
 #include "tcgen05.cuh"
 
 namespace llm {
 namespace attn_tc {
 
 using namespace tc;
+using namespace attn_maps;
 
 // 2^x for pair i of a 16-pair chunk: NP of the 16 pairs (spread over the
 // chunk) by the polynomial on the FMA pipe, the rest by the SFU.
@@ -57,6 +61,12 @@ constexpr int NP_FWD = 3;
 constexpr int BQ = 128, BK = 128, HD = 64;
 constexpr int TILE_BYTES = 128 * HD * 2;  // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int STAGES = 4;  // K and V rings: deep enough to cover the TMA latency under load
+// Q slots: an item's O is staged in its own Q slot and released after the
+// next item's first block, so the Q of item it + 1 goes into the slot of item
+// it - 2; with two slots the next item's first S (and the MMA warp's P V of
+// this item's last block, issued after it) would wait for that release and a
+// Q load at every item boundary, which dominates items of one or two blocks
+constexpr int QSLOTS = 3;
 constexpr int NQ = 4;             // key groups of a block (independent softmaxes)
 constexpr int KW = 128 / NQ;      // keys per group (softmax thread)
 constexpr int SM_WARPS = 4 * NQ;  // softmax warps: 4 lane quarters x NQ groups
@@ -73,7 +83,8 @@ constexpr float LN2 = 0.6931471805599453f;
 constexpr float LAZY = 8.f;  // log2 units a row maximum may grow before O is rescaled
 // shared memory: Q[2] | K[STAGES] | V[STAGES] | barriers | red[2]
 constexpr int BAR_BYTES = 512;  // 48 mbarrier slots, then the TMEM address and abort words
-constexpr int SMEM_BYTES = (2 + 2 * STAGES) * TILE_BYTES + BAR_BYTES + 2 * 2 * NQ * 128 * 4 + 1024;
+constexpr int SMEM_BYTES =
+    (QSLOTS + 2 * STAGES) * TILE_BYTES + BAR_BYTES + 2 * 2 * NQ * 128 * 4 + 1024;
 
 // P = 2^(s sl2 - mr) for the KW scores of one (row, group), packed bf16 into
 // w; returns their sum.  Pairs in packed f32x2 arithmetic; with FMA_EXP some
@@ -113,14 +124,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                   float *__restrict__ lse, int B, int T, int H, int Hkv, float scale, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sQ = smem, *sK = smem + 2 * TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
+  uint8_t *sQ = smem, *sK = smem + QSLOTS * TILE_BYTES, *sV = sK + STAGES * TILE_BYTES;
   uint64_t *bars = (uint64_t *)(sV + STAGES * TILE_BYTES);
   uint32_t *tmem_sh = (uint32_t *)(bars + 48);
   volatile int *abort_sh = (volatile int *)(tmem_sh + 1);
   float *red = (float *)(bars + BAR_BYTES / 8);  // [2][NQ][128]: m_g, then l_g per row
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t q_full = b0, q_empty = b0 + 16,  // [2]: Q slot
-                 k_full = b0 + 32, k_empty = k_full + 8 * STAGES,
+  const uint32_t q_full = b0, q_empty = b0 + 8 * QSLOTS,  // [QSLOTS]: Q slot
+                 k_full = b0 + 16 * QSLOTS, k_empty = k_full + 8 * STAGES,
                  v_full = k_empty + 8 * STAGES, v_empty = v_full + 8 * STAGES,
                  s_full = v_empty + 8 * STAGES,    // [2]: one per S buffer
                  buf_free = s_full + 16,           // [2]: the buffer's P V products done
@@ -129,11 +140,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  p_full = buf_free + 16,
                  o_done = p_full + 16 * NQ,        // [NQ]
                  drain = o_done + 8 * NQ;          // [2]: one per MMA warp
-  static_assert(4 + 4 * STAGES + 4 + 3 * NQ + 2 <= 48, "barriers overlap the TMEM address word");
+  static_assert(2 * QSLOTS + 4 * STAGES + 4 + 3 * NQ + 2 <= 48,
+                "barriers overlap the TMEM address word");
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
   const int G = gridDim.x, cta = blockIdx.x;
-  const int d = H * HD, kvd = Hkv * HD;
   // item -> (query block, head, batch): longest rows (last query blocks) first,
   // in bands of 4 query blocks taken pair by pair (band_item)
   auto decode = [&](int item, int &qb, int &h, int &b) {
@@ -146,7 +157,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (threadIdx.x == 0) {
     *abort_sh = 0;
-    for (int x = 0; x < 2; x++) {
+    for (int x = 0; x < QSLOTS; x++) {
       mbar_init(q_full + 8 * x, 1);
       // the item's last S product on the slot, then the bulk stores of O
       // staged in it (one per softmax warp)
@@ -190,11 +201,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (item >= n_items) break;
         int qb, h, b;
         decode(item, qb, h, b);
-        const int row_base = b * T, g = h / (H / Hkv), slot = it & 1;
-        // Q into the slot of item it - 2 once its last S product completed
-        if (!mbar_wait(q_empty + 8 * slot, ((it >> 1) & 1) ^ 1, abort_sh, gflag)) break;
+        const int row_base = b * T, g = h / (H / Hkv), slot = it % QSLOTS;
+        // Q into the slot of item it - QSLOTS once its last S product and the
+        // store of its O (staged in the slot) completed
+        if (!mbar_wait(q_empty + 8 * slot, ((it / QSLOTS) & 1) ^ 1, abort_sh, gflag)) break;
         mbar_arrive_expect_tx(q_full + 8 * slot, TILE_BYTES);
-        tma_load_2d(smem_u32(sQ + slot * TILE_BYTES), &tm_qkv, h * HD, row_base + qb * BQ,
+        tma_load_3d(smem_u32(sQ + slot * TILE_BYTES), &tm_qkv, 0, h, row_base + qb * BQ,
                     q_full + 8 * slot);
         nq = it + 1;
         for (int j = 0; j <= qb; j++) {
@@ -206,16 +218,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
-          tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
+          tma_load_3d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, 0, H + g, row_base + j * BK,
                       k_full + 8 * s);
           mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
-          tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD,
+          tma_load_3d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, 0, H + Hkv + g,
                       row_base + j * BK, v_full + 8 * s);
           gb++;
         }
       }
       // every copy this thread issued has landed before the CTA may exit
-      for (int i = max(0, nq - 2); i < nq; i++) drain_wait(q_full + 8 * (i & 1), (i >> 1) & 1);
+      for (int i = max(0, nq - QSLOTS); i < nq; i++)
+        drain_wait(q_full + 8 * (i % QSLOTS), (i / QSLOTS) & 1);
       for (int i = max(0, gb - STAGES); i < gb; i++) {
         drain_wait(k_full + 8 * (i % STAGES), (i / STAGES) & 1);
         drain_wait(v_full + 8 * (i % STAGES), (i / STAGES) & 1);
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int r = 0, it = 0; item < n_items && ok; r++, it++) {
       int qb, h, b;
       decode(item, qb, h, b);
-      const int nj = qb + 1, slot = it & 1;
+      const int nj = qb + 1, slot = it % QSLOTS;
       const int next = sched_item(r + 1, G, cta);
       int qb_next = 0, hn, bn;
       if (next < n_items) decode(next, qb_next, hn, bn);
@@ -265,10 +278,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // scores of block gb + 1 (this item's next, or the next item's
           // first) into the other buffer once its P V products (block gb - 1)
           // have completed
-          const int slot1 = here ? slot : slot ^ 1;
+          const int slot1 = here ? slot : (it + 1) % QSLOTS;
           const int s1 = (gb + 1) % STAGES;
           const uint32_t ph1 = ((gb + 1) / STAGES) & 1;
-          if ((!here && !warp_wait(q_full + 8 * slot1, ((it + 1) >> 1) & 1, abort_sh, gflag)) ||
+          if ((!here && !warp_wait(q_full + 8 * slot1, ((it + 1) / QSLOTS) & 1, abort_sh, gflag)) ||
               !warp_wait(k_full + 8 * s1, ph1, abort_sh, gflag) ||
               (gb >= 1 && !warp_wait(buf_free + 8 * ((gb + 1) & 1), ((gb - 1) >> 1) & 1, abort_sh,
                                      gflag))) {
@@ -450,7 +463,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // O rows through the item's Q tile (its last S product is complete):
       // this thread's two 16-byte chunks of row r in the tile's
       // 128-byte-swizzle image
-      uint8_t *srow = sQ + (it & 1) * TILE_BYTES + r * 128;
+      uint8_t *srow = sQ + (it % QSLOTS) * TILE_BYTES + r * 128;
 #pragma unroll
       for (int c = 0; c < OW / 8; c++) {
         const int ch = grp * (OW / 8) + c;
@@ -467,10 +480,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       softmax_sync();
       if (lane == 0) {  // 8 whole rows of this warp's lane quarter (rows past T clipped)
         const int r0 = quarter * 32 + grp * 8;
-        tma_store_3d(&tm_o, smem_u32(sQ + (it & 1) * TILE_BYTES + r0 * 128), h * HD, q0 + r0, b);
+        tma_store_4d(&tm_o, smem_u32(sQ + (it % QSLOTS) * TILE_BYTES + r0 * 128), 0, h, q0 + r0, b);
         bulk_commit();
       }
-      st_slot = it & 1;  // released after the next item's first block
+      st_slot = it % QSLOTS;  // released after the next item's first block
       if (grp == 0 && qi < T) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
     }
     if (lane == 0) bulk_wait_all();
@@ -487,19 +500,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace attn_tc
 
-bool attn_tc_covers(DType dt, int hd, int T) { return dt == DT_BF16 && hd == 64 && T >= 1; }
+bool attn_tc_covers(DType dt, int hd, int T) {
+  return dt == DT_BF16 && (hd == 64 || hd == 32) && T >= 1;
+}
 
-// Host side: one tensor map over qkv [B*T rows, qkvw columns] serves the Q, K
-// and V tiles (box 64 x 128, 128-byte swizzle).
+// Host side: one tensor map over qkv [B*T rows][H + 2 Hkv heads][hd] serves
+// the Q, K and V tiles (box 64 x 1 head x 128 rows, 128-byte swizzle); O
+// leaves through a [B][T][H][hd] map (box 64 x 1 x 8 rows x 1).
 bool attn_fwd_tc(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
                  int *flag, cudaStream_t s) {
   using namespace attn_tc;
-  if (hd != HD || !flag) return false;
+  if ((hd != 64 && hd != 32) || !flag) return false;
   if (!smem_optin((const void *)k_attn_fwd_tc, SMEM_BYTES)) return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd;
   CUtensorMap map, mo;
-  if (!tc::tile_map_bf16(&map, qkv, qkvw, (int64_t)B * T, qkvw, 128) ||
-      !tc::tile_map_bf16_3d(&mo, o, (int64_t)H * hd, T, B, (int64_t)H * hd, 8))
+  if (!head_map_load(&map, qkv, hd, H + 2 * Hkv, (int64_t)B * T, qkvw, 128) ||
+      !head_map_store(&mo, o, hd, H, T, B, (int64_t)H * hd, 8))
     return false;
   const int items = ((T + BQ - 1) / BQ) * H * B;
   k_attn_fwd_tc<<<min(items, device_sms()), NTHREADS, SMEM_BYTES, s>>>(

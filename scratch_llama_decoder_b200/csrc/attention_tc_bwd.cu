@@ -1,5 +1,7 @@
-// tcgen05 flash-attention backward for head size 64 (bf16 operands, fp32
-// scores and accumulators).  With the forward's saved row log-sum-exp L and
+// tcgen05 flash-attention backward for head sizes 64 and 32 (bf16 operands,
+// fp32 scores and accumulators; a head-32 tile is the head-64 one with its
+// upper 32 columns loaded as zeros, so every product and D below is the
+// head-32 one, and only the head's own columns are stored).  With the forward's saved row log-sum-exp L and
 // D_i = sum_e dO_ie O_ie, the causal softmax backward of strata's flash
 // attention is, per (query i, key j) pair,
 //     P_ij  = exp(scale * q_i.k_j - L_i)          (0 above the diagonal)
@@ -42,12 +44,14 @@
 // (FLAG_TIMEOUT, then drain and free TMEM).
 #include "common.cuh"
 #include "gemm_tc.h"
+#include "attn_tma.cuh"
 #include "tcgen05.cuh"
 
 namespace llm {
 namespace attn_tc_bwd {
 
 using namespace tc;
+using namespace attn_maps;
 
 // 2^x for pair i of a 16-pair chunk: NP of the 16 pairs (spread over the
 // chunk) by the polynomial on the FMA pipe, the rest by the SFU.
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  const float *__restrict__ lse,
                  float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
                  const float *__restrict__ cos_t, const float *__restrict__ sin_t, int B, int T,
-                 int H, int Hkv, float scale, int bulk_l, int *gflag) {
+                 int H, int Hkv, int hd, float scale, int bulk_l, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = smem, *sdO = smem + 2 * TILE_BYTES, *sO = smem + 4 * TILE_BYTES,
@@ -172,7 +176,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nqb = (T + BQ - 1) / BQ, n_items = nqb * H * B;
   const int G = gridDim.x, cta = blockIdx.x;
-  const int d = H * HD, kvd = Hkv * HD;
   // item -> (query block, head, batch): longest rows (last query blocks) first,
   // in bands of 4 query blocks taken pair by pair (band_item)
   auto decode = [&](int item, int &qb, int &h, int &b) {
@@ -233,9 +236,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!warp_wait(qd_empty + 8 * slot, ((it >> 1) & 1) ^ 1, abort_sh, gflag)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(qd_full + 8 * slot, 2 * TILE_BYTES);
-        tma_load_2d(smem_u32(sQ + slot * TILE_BYTES), &tm_qkv, h * HD, row_base + q0,
+        tma_load_3d(smem_u32(sQ + slot * TILE_BYTES), &tm_qkv, 0, h, row_base + q0,
                     qd_full + 8 * slot);
-        tma_load_2d(smem_u32(sdO + slot * TILE_BYTES), &tm_do, h * HD, row_base + q0,
+        tma_load_3d(smem_u32(sdO + slot * TILE_BYTES), &tm_do, 0, h, row_base + q0,
                     qd_full + 8 * slot);
       }
       nqd = it + 1;
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nvalid = min(BQ, T - q0);
       if (lane == 0) {
         mbar_arrive_expect_tx(o_full, TILE_BYTES + (bulk_l ? nvalid * 4 : 0));
-        tma_load_2d(smem_u32(sO), &tm_o, h * HD, row_base + q0, o_full);
+        tma_load_3d(smem_u32(sO), &tm_o, 0, h, row_base + q0, o_full);
         if (bulk_l) bulk_load(smem_u32(sNL), lrow, nvalid * 4, o_full);
       }
       if (!bulk_l)
@@ -264,10 +267,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(k_full + 8 * s, TILE_BYTES);
-          tma_load_2d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, d + g * HD, row_base + j * BK,
+          tma_load_3d(smem_u32(sK + s * TILE_BYTES), &tm_qkv, 0, H + g, row_base + j * BK,
                       k_full + 8 * s);
           mbar_arrive_expect_tx(v_full + 8 * s, TILE_BYTES);
-          tma_load_2d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, d + kvd + g * HD,
+          tma_load_3d(smem_u32(sV + s * TILE_BYTES), &tm_qkv, 0, H + Hkv + g,
                       row_base + j * BK, v_full + 8 * s);
         }
         gb++;
@@ -492,12 +495,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       fence_after();
-      // column pairs (c, c + 32) of RoPE: this group takes c in [cq HW, cq HW + HW)
+      // column pairs (c, c + hd/2) of RoPE: this group takes c in [xc, xc + HW)
+      // (head 32: groups 2 and 3 repeat 0 and 1 and stage nothing)
+      const int half = hd / 2, xc = (hd == 64 ? cq : (cq & 1)) * HW;
       float xa[HW], ya[HW], xb[HW], yb[HW];
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + cq * HW, xa);
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + 32 + cq * HW, ya);
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + cq * HW, xb);
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + 32 + cq * HW, yb);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + xc, xa);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + half + xc, ya);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + xc, xb);
+      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + half + xc, yb);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_free);  // the next item's dQ products may start
@@ -507,14 +512,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ya[i] += yb[i];
       }
       if (valid && cos_t)
-        rope_bwd_n<HW>(xa, ya, cos_t + (int64_t)qi * (HD / 2) + cq * HW,
-                       sin_t + (int64_t)qi * (HD / 2) + cq * HW);
+        rope_bwd_n<HW>(xa, ya, cos_t + (int64_t)qi * half + xc, sin_t + (int64_t)qi * half + xc);
       // dQ rows through the item's Q tile (its products are complete): the
       // 128-byte-swizzle image of the tile, then each warp stores 8 whole rows
       // of its lane quarter with one bulk tensor copy (rows past T clipped)
       uint8_t *srow = sQ + slot * TILE_BYTES + r * 128;
-      stage_n<HW>(srow, cq, r, xa, scale);
-      stage_n<HW>(srow, 4 + cq, r, ya, scale);
+      if (hd == 64 || cq < 2) {
+        stage_n<HW>(srow, xc / 8, r, xa, scale);
+        stage_n<HW>(srow, (half + xc) / 8, r, ya, scale);
+      }
       fence_proxy_async();
       mbar_arrive(qsync + 8 * quarter);
       if (!warp_wait(qsync + 8 * quarter, it & 1, abort_sh, gflag)) {
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (lane == 0) {
         const int r0 = quarter * 32 + cq * 8;
-        tma_store_3d(&tm_st, smem_u32(sQ + slot * TILE_BYTES + r0 * 128), h * HD, q0 + r0, b);
+        tma_store_4d(&tm_st, smem_u32(sQ + slot * TILE_BYTES + r0 * 128), 0, h, q0 + r0, b);
         bulk_commit();
       }
       st_slot = slot;  // released (below) once the store has read the tile
@@ -548,7 +554,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                   const float *__restrict__ lse,
                   const float *__restrict__ Dv, __nv_bfloat16 *__restrict__ dqkv,
                   const float *__restrict__ cos_t, const float *__restrict__ sin_t, int B, int T,
-                  int H, int Hkv, float scale, int bulk_l, int *gflag) {
+                  int H, int Hkv, int hd, float scale, int bulk_l, int *gflag) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sK = smem, *sV = smem + 2 * TILE_BYTES, *sQ = smem + 4 * TILE_BYTES,
@@ -569,7 +575,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nkb = (T + BK - 1) / BK, n_items = nkb * Hkv * B;
   const int G = gridDim.x, cta = blockIdx.x;
-  const int grp = H / Hkv, d = H * HD, kvd = Hkv * HD;
+  const int grp = H / Hkv;
   // item -> (key block, kv head, batch), first key blocks first in bands of 4
   // taken pair by pair (band_item); steps = grp (nkb - kb)
   auto decode = [&](int item, int &kb, int &g, int &b) {
@@ -620,9 +626,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!warp_wait(kv_empty + 8 * slot, ((it >> 1) & 1) ^ 1, abort_sh, gflag)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(kv_full + 8 * slot, 2 * TILE_BYTES);
-        tma_load_2d(smem_u32(sK + slot * TILE_BYTES), &tm_qkv, d + g * HD, row_base + k0,
+        tma_load_3d(smem_u32(sK + slot * TILE_BYTES), &tm_qkv, 0, H + g, row_base + k0,
                     kv_full + 8 * slot);
-        tma_load_2d(smem_u32(sV + slot * TILE_BYTES), &tm_qkv, d + kvd + g * HD, row_base + k0,
+        tma_load_3d(smem_u32(sV + slot * TILE_BYTES), &tm_qkv, 0, H + Hkv + g, row_base + k0,
                     kv_full + 8 * slot);
       }
       nkv = it + 1;
@@ -642,9 +648,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int nvalid = min(BQ, T - qb * BQ);
         if (lane == 0) {
           mbar_arrive_expect_tx(q_full + 8 * s, 2 * TILE_BYTES + (bulk_l ? 8 * nvalid : 0));
-          tma_load_2d(smem_u32(sQ + s * TILE_BYTES), &tm_qkv, hq * HD, row_base + qb * BQ,
+          tma_load_3d(smem_u32(sQ + s * TILE_BYTES), &tm_qkv, 0, hq, row_base + qb * BQ,
                       q_full + 8 * s);
-          tma_load_2d(smem_u32(sdO + s * TILE_BYTES), &tm_do, hq * HD, row_base + qb * BQ,
+          tma_load_3d(smem_u32(sdO + s * TILE_BYTES), &tm_do, 0, hq, row_base + qb * BQ,
                       q_full + 8 * s);
           if (bulk_l) {
             bulk_load(smem_u32(sL + s * 128), lse + base, nvalid * 4, q_full + 8 * s);
@@ -856,21 +862,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       fence_after();
-      // column pairs (c, c + 32) of RoPE: this group takes c in [cq HW, cq HW + HW)
+      // column pairs (c, c + hd/2) of RoPE in dK: this group takes c in
+      // [xc, xc + HW) (head 32: groups 2 and 3 repeat 0 and 1 and stage no dK);
+      // dV: columns [cq HW, cq HW + HW) and 32 more (zero past head 32)
+      const int half = hd / 2, xc = (hd == 64 ? cq : (cq & 1)) * HW;
       float xk[HW], yk[HW], xv[HW], yv[HW];
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + cq * HW, xk);
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + 32 + cq * HW, yk);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + xc, xk);
+      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + half + xc, yk);
       tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + cq * HW, xv);
       tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + 32 + cq * HW, yv);
       if (kj < T && cos_t)
-        rope_bwd_n<HW>(xk, yk, cos_t + (int64_t)kj * (HD / 2) + cq * HW,
-                       sin_t + (int64_t)kj * (HD / 2) + cq * HW);
+        rope_bwd_n<HW>(xk, yk, cos_t + (int64_t)kj * half + xc, sin_t + (int64_t)kj * half + xc);
       // dK, dV rows through the item's K and V tiles (their products are
       // complete), then each warp stores 8 whole rows of its lane quarter of
       // both with bulk tensor copies (rows past T clipped)
       uint8_t *rk = sK + slot * TILE_BYTES + r * 128, *rv = sV + slot * TILE_BYTES + r * 128;
-      stage_n<HW>(rk, cq, r, xk, scale);
-      stage_n<HW>(rk, 4 + cq, r, yk, scale);
+      if (hd == 64 || cq < 2) {
+        stage_n<HW>(rk, xc / 8, r, xk, scale);
+        stage_n<HW>(rk, (half + xc) / 8, r, yk, scale);
+      }
       stage_n<HW>(rv, cq, r, xv, 1.f);
       stage_n<HW>(rv, 4 + cq, r, yv, 1.f);
       fence_proxy_async();
@@ -881,9 +891,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (lane == 0) {
         const int r0 = quarter * 32 + cq * 8;
-        tma_store_3d(&tm_st, smem_u32(sK + slot * TILE_BYTES + r0 * 128), d + g * HD, k0 + r0, b);
-        tma_store_3d(&tm_st, smem_u32(sV + slot * TILE_BYTES + r0 * 128), d + kvd + g * HD,
-                     k0 + r0, b);
+        tma_store_4d(&tm_st, smem_u32(sK + slot * TILE_BYTES + r0 * 128), 0, H + g, k0 + r0, b);
+        tma_store_4d(&tm_st, smem_u32(sV + slot * TILE_BYTES + r0 * 128), 0, H + Hkv + g, k0 + r0,
+                     b);
         bulk_commit();
       }
       st_slot = slot;  // released after the next item's first step
@@ -899,13 +909,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace attn_tc_bwd
 
 
-// Host side: tensor maps over qkv [B*T, qkvw] and dout [B*T, H*hd] (box 64 x
-// 128); the dQ kernel runs first (it also writes D), then the dK/dV kernel.
+// Host side: head-indexed tensor maps (attn_tma.cuh) over qkv [B*T][H + 2 Hkv
+// heads][hd], O and dout [B*T][H][hd] (box 64 x 1 x 128), and dqkv for the
+// stores ([B][T][H + 2 Hkv][hd], box 64 x 1 x 8 x 1); the dQ kernel runs
+// first (it also writes D), then the dK/dV kernel.
 bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
                  void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
                  const float *sin_t, int *flag, cudaStream_t s) {
   using namespace attn_tc_bwd;
-  if (hd != HD || !flag || ((uintptr_t)o & 15) || ((uintptr_t)dqkv & 15) ||
+  if ((hd != 64 && hd != 32) || !flag || ((uintptr_t)o & 15) || ((uintptr_t)dqkv & 15) ||
       ((uintptr_t)cos_t & 15) || ((uintptr_t)sin_t & 15) || (!cos_t != !sin_t))
     return false;
   if (!smem_optin((const void *)k_attn_dq_tc, DQ_SMEM) ||
@@ -913,21 +925,21 @@ bool attn_bwd_tc(const void *qkv, const void *o, const void *dout, const float *
     return false;
   const int64_t qkvw = (int64_t)(H + 2 * Hkv) * hd, dw = (int64_t)H * hd;
   CUtensorMap mq, md, mo, mst;
-  if (!tc::tile_map_bf16(&mq, qkv, qkvw, (int64_t)B * T, qkvw, 128) ||
-      !tc::tile_map_bf16(&md, dout, dw, (int64_t)B * T, dw, 128) ||
-      !tc::tile_map_bf16(&mo, o, dw, (int64_t)B * T, dw, 128) ||
-      !tc::tile_map_bf16_3d(&mst, dqkv, qkvw, T, B, qkvw, 8))
+  if (!head_map_load(&mq, qkv, hd, H + 2 * Hkv, (int64_t)B * T, qkvw, 128) ||
+      !head_map_load(&md, dout, hd, H, (int64_t)B * T, dw, 128) ||
+      !head_map_load(&mo, o, hd, H, (int64_t)B * T, dw, 128) ||
+      !head_map_store(&mst, dqkv, hd, H + 2 * Hkv, T, B, qkvw, 8))
     return false;
   const int nb = (T + BQ - 1) / BQ, sms = device_sms();
   const float scale = 1.0f / sqrtf((float)hd);
   // L and D rows of a (batch, head) start 16-byte aligned when T % 4 == 0
   const int bulk_l = (T % 4 == 0) && !((uintptr_t)lse & 15) && !((uintptr_t)Dbuf & 15);
   k_attn_dq_tc<<<min(nb * H * B, sms), NTHREADS, DQ_SMEM, s>>>(
-      mq, md, mo, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, bulk_l,
-      flag);
+      mq, md, mo, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, hd, scale,
+      bulk_l, flag);
   k_attn_dkv_tc<<<min(nb * Hkv * B, sms), NTHREADS, KV_SMEM, s>>>(
-      mq, md, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, scale, bulk_l,
-      flag);
+      mq, md, mst, lse, Dbuf, (__nv_bfloat16 *)dqkv, cos_t, sin_t, B, T, H, Hkv, hd, scale,
+      bulk_l, flag);
   count_launch(2);
   return true;
 }

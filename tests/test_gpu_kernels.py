@@ -119,7 +119,7 @@ def test_gemm_f32_scratch_too_small():
 def test_embed_bwd_vs_oracle(N, d, V):
     """Scatter-add of the embedding gradient against the oracle; also
     bit-for-bit equal to float32 sums in the kernel's fixed order (a run of
-    at most 64 rows in increasing position order; a longer run as 8
+    at most 64 rows in increasing position order; a longer run as 32
     contiguous parts, each summed in order, then added in part order); zero
     rows for absent ids; Zipf ids put thousands of rows on id 0."""
     import scratch_llama_decoder_b200 as P
@@ -145,7 +145,7 @@ def test_embed_bwd_vs_oracle(N, d, V):
     for v in range(V):
         run = order[bounds[v]:bounds[v + 1]]
         c = run.size
-        parts = 8 if c > 64 else 1
+        parts = 32 if c > 64 else 1
         for k in range(parts):
             s = np.zeros(d, np.float32)
             for i in run[c * k // parts:c * (k + 1) // parts]:
@@ -165,7 +165,8 @@ def test_embed_bwd_vs_oracle(N, d, V):
 # (batch, ctx, n_head, n_kv_head, head_dim): tile multiples, ragged lengths,
 # one position, MHA/GQA/MQA, both head sizes, the longest context
 ATTN = [(1, 64, 2, 2, 64), (2, 200, 4, 2, 64), (1, 130, 8, 8, 32), (3, 1, 4, 1, 64),
-        (2, 512, 8, 2, 64), (1, 2048, 2, 2, 64), (1, 333, 4, 1, 32)]
+        (2, 512, 8, 2, 64), (1, 2048, 2, 2, 64), (1, 333, 4, 1, 32), (2, 384, 8, 2, 32),
+        (3, 1, 4, 1, 32), (1, 1024, 2, 2, 32)]
 
 
 @pytest.mark.parametrize("tc", [2, 1, 0])
@@ -175,8 +176,6 @@ def test_attention_fwd_bwd_vs_oracle(B, T, H, Hkv, hd, tc):
     import scratch_llama_decoder_b200 as P
     if not tc and T > 600:
         pytest.skip("CUDA-core reference kernel: long contexts covered by the step tests")
-    if tc == 2 and hd != 64:
-        pytest.skip("the tcgen05 kernels cover head size 64")
     rng = np.random.default_rng(B * 1000 + T + H + hd)
     d, kvd = H * hd, Hkv * hd
     w = d + 2 * kvd
@@ -211,6 +210,40 @@ def test_attention_fwd_bwd_vs_oracle(B, T, H, Hkv, hd, tc):
             ref = dq_ref[:, lo:hi]
             err = np.linalg.norm(dg[b][:, lo:hi] - ref) / max(np.linalg.norm(ref), 1e-3 * full)
             assert err < 2e-2, (b, lo, err)
+
+
+def test_attention_tc_head32_writes_only_its_head():
+    """Head 32 on the tcgen05 kernels moves 64-wide tiles; their upper 32
+    columns lie outside the head and must never be written: outputs sit in
+    larger buffers whose guard region past the last row and head stays
+    untouched, and O, dq|dk|dv equal the warp-level mma kernels' results to
+    bf16 rounding."""
+    import scratch_llama_decoder_b200 as P
+    B, T, H, Hkv, hd = 2, 200, 4, 2, 32
+    rng = np.random.default_rng(32)
+    d, kvd = H * hd, Hkv * hd
+    w = d + 2 * kvd
+    qd = _bf16(rng, (B * T, w)).cuda()
+    dd = _bf16(rng, (B * T, d)).cuda()
+    p = lambda t: C.c_void_p(t.data_ptr())
+    guard = 4096
+    res = {}
+    for tc in (2, 1):
+        obuf = torch.full((B * T * d + guard,), 7.0, dtype=torch.bfloat16, device="cuda")
+        gbuf = torch.full((B * T * w + guard,), 7.0, dtype=torch.bfloat16, device="cuda")
+        o, dq = obuf[:B * T * d].view(B * T, d), gbuf[:B * T * w].view(B * T, w)
+        lse = torch.zeros(B, H, T, device="cuda")
+        Dv = torch.zeros(B, H, T, device="cuda")
+        assert P.lib.llm_kernel_attention_fwd_bf16(p(qd), p(o), p(lse), B, T, H, Hkv, hd, tc,
+                                                   None) == 0
+        assert P.lib.llm_kernel_attention_bwd_bf16(p(qd), p(o), p(dd), p(lse), p(Dv), p(dq), B, T,
+                                                   H, Hkv, hd, tc, None) == 0
+        torch.cuda.synchronize()
+        assert bool((obuf[B * T * d:] == 7).all()) and bool((gbuf[B * T * w:] == 7).all()), tc
+        res[tc] = (o.float().cpu(), dq.float().cpu())
+    for a, b in zip(res[2], res[1]):
+        assert torch.isfinite(a).all()
+        assert (a - b).norm() / b.norm() < 1e-2
 
 
 # float32 attention (the float32 configurations): head sizes 32 and 64 with
