@@ -411,27 +411,40 @@ int rmsnorm_bwd(const float *x, const float *rstd, const float *g, const float *
   return nblk;
 }
 
-// out[j] = sum over b of part[b][j]: 8 groups of threads add interleaved
-// rows (b = grp, grp+8, ...), then the 8 group sums are added in group order
-// (a fixed order, so the result does not depend on scheduling).
-__global__ void k_reduce_partials(const float *__restrict__ part, int nblk, int d,
-                                  float *__restrict__ out) {
-  __shared__ float sh[8][32];
+// out[j] = sum over b of part[b][j]: RP_GROUPS groups of threads add
+// interleaved rows (b = grp, grp + RP_GROUPS, ...; four loads in flight, added
+// in row order), then the group sums are added in group order (a fixed order,
+// so the result does not depend on scheduling).  One block per 32 columns.
+constexpr int RP_GROUPS = 32;
+__global__ void __launch_bounds__(32 * RP_GROUPS)
+    k_reduce_partials(const float *__restrict__ part, int nblk, int d, float *__restrict__ out) {
+  __shared__ float sh[RP_GROUPS][33];
   const int c = threadIdx.x & 31, grp = threadIdx.x >> 5;
   const int j = blockIdx.x * 32 + c;
   float s = 0.f;
-  if (j < d)
-    for (int b = grp; b < nblk; b += 8) s += part[(int64_t)b * d + j];
+  if (j < d) {
+    int b = grp;
+    for (; b + 3 * RP_GROUPS < nblk; b += 4 * RP_GROUPS) {
+      const float v0 = part[(int64_t)b * d + j], v1 = part[(int64_t)(b + RP_GROUPS) * d + j],
+                  v2 = part[(int64_t)(b + 2 * RP_GROUPS) * d + j],
+                  v3 = part[(int64_t)(b + 3 * RP_GROUPS) * d + j];
+      s += v0;
+      s += v1;
+      s += v2;
+      s += v3;
+    }
+    for (; b < nblk; b += RP_GROUPS) s += part[(int64_t)b * d + j];
+  }
   sh[grp][c] = s;
   __syncthreads();
   if (grp == 0 && j < d) {
     float t = sh[0][c];
-    for (int k = 1; k < 8; k++) t += sh[k][c];
+    for (int k = 1; k < RP_GROUPS; k++) t += sh[k][c];
     out[j] = t;
   }
 }
 void reduce_partials(const float *part, int nblk, int d, float *out, cudaStream_t s) {
-  k_reduce_partials<<<cdiv(d, 32), 256, 0, s>>>(part, nblk, d, out);
+  k_reduce_partials<<<cdiv(d, 32), 32 * RP_GROUPS, 0, s>>>(part, nblk, d, out);
   count_launch();
 }
 
@@ -1098,32 +1111,42 @@ void adamw(float *p, const float *g, float *m, float *v, int64_t n, const float 
 
 // ------------------------------------------------------------ wgrad finish
 // grad[r, c] = sum over splits k (in order) of part[k, r, cp(c)]; mode 1 maps
-// the interleaved W1 | W3 columns back.  One block per row (grid-stride), 4
-// columns per thread: an aligned group of 4 columns has 4 contiguous
-// partial-sum columns in both modes (SWIGLU_BLOCK and h multiples of 4).
-__global__ void k_wgrad_finish(const float *__restrict__ part, int splits, int64_t part_rows,
-                               int64_t ldp, float *__restrict__ grad, int64_t rows, int64_t cols,
-                               int mode, int64_t h, bool vec) {
+// the interleaved W1 | W3 columns back.  One thread per group of 4 columns
+// over the whole [rows, cols] gradient (grid-stride), so rows narrower than a
+// block keep every lane busy: an aligned group of 4 columns has 4 contiguous
+// partial-sum columns in both modes (SWIGLU_BLOCK and h multiples of 4), and
+// four splits' loads are in flight at a time, added in split order.
+LLM_DEV float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+__global__ void __launch_bounds__(256)
+    k_wgrad_finish(const float *__restrict__ part, int splits, int64_t part_rows, int64_t ldp,
+                   float *__restrict__ grad, int64_t rows, int64_t cols, int mode, int64_t h,
+                   bool vec) {
   const int64_t pstride = part_rows * ldp;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+  const int64_t cq = (cols + 3) / 4, n = rows * cq;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / cq, c = 4 * (i - r * cq);
     const float *pr = part + r * ldp;
     float *gr = grad + r * cols;
-    for (int64_t c = 4 * (int64_t)threadIdx.x; c < cols; c += 4 * (int64_t)blockDim.x) {
-      if (vec && c + 4 <= cols) {
-        const int64_t cp = mode == 1 ? ((c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK) : c;
-        float4 acc = *reinterpret_cast<const float4 *>(pr + cp);
-        for (int k = 1; k < splits; k++) {
-          const float4 q = *reinterpret_cast<const float4 *>(pr + k * pstride + cp);
-          acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
-        }
-        *reinterpret_cast<float4 *>(gr + c) = acc;
-      } else {
-        for (int64_t cc = c; cc < c + 4 && cc < cols; cc++) {
-          const int64_t cp = mode == 1 ? ((cc < h) ? w1_col(cc) : w1_col(cc - h) + SWIGLU_BLOCK) : cc;
-          float acc = 0.f;
-          for (int k = 0; k < splits; k++) acc += pr[k * pstride + cp];
-          gr[cc] = acc;
-        }
+    if (vec && c + 4 <= cols) {
+      const int64_t cp = mode == 1 ? ((c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK) : c;
+      const float4 *p4 = reinterpret_cast<const float4 *>(pr + cp);
+      const int64_t ps4 = pstride / 4;
+      float4 acc = p4[0];
+      int k = 1;
+      for (; k + 4 <= splits; k += 4) {
+        const float4 q1 = p4[k * ps4], q2 = p4[(k + 1) * ps4], q3 = p4[(k + 2) * ps4],
+                     q4 = p4[(k + 3) * ps4];
+        acc = add4(add4(add4(add4(acc, q1), q2), q3), q4);
+      }
+      for (; k < splits; k++) acc = add4(acc, p4[k * ps4]);
+      *reinterpret_cast<float4 *>(gr + c) = acc;
+    } else {
+      for (int64_t cc = c; cc < c + 4 && cc < cols; cc++) {
+        const int64_t cp = mode == 1 ? ((cc < h) ? w1_col(cc) : w1_col(cc - h) + SWIGLU_BLOCK) : cc;
+        float acc = 0.f;
+        for (int k = 0; k < splits; k++) acc += pr[k * pstride + cp];
+        gr[cc] = acc;
       }
     }
   }
@@ -1132,7 +1155,8 @@ void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp,
                   int64_t rows, int64_t cols, int mode, int64_t h, cudaStream_t s) {
   const bool vec = ((uintptr_t)part & 15) == 0 && ((uintptr_t)grad & 15) == 0 && ldp % 4 == 0 &&
                    cols % 4 == 0 && (mode == 0 || h % 4 == 0) && (part_rows * ldp) % 4 == 0;
-  unsigned grid = (unsigned)std::min<int64_t>(rows, 148 * 8);
+  const int64_t groups = rows * ((cols + 3) / 4);
+  unsigned grid = (unsigned)std::min<int64_t>((groups + 255) / 256, 148 * 8);
   k_wgrad_finish<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode, h, vec);
   count_launch();
 }
