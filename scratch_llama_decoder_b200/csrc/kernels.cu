@@ -265,10 +265,15 @@ void rmsnorm_fwd(const float *x, const float *g, void *y, DType dt, float *rstd,
 // -------------------------------------------------------------- RMSNorm bwd
 // Backward of y = g x r:  dx = r g dy - x r^3 (1/d) sum_j g_j dy_j x_j, plus
 // the residual gradient dres; dg = sum over rows of dy x r, reduced in a fixed
-// order: each block writes the partial sum of its RMS_ROWS rows, and
-// reduce_partials adds the blocks in index order.
-constexpr int RMS_ROWS = 64;
-int rmsnorm_bwd_blocks(int64_t N) { return (int)cdiv(N, RMS_ROWS); }
+// order: each block writes the partial sum of its rows, and reduce_partials
+// adds the blocks in index order.  The N rows are split evenly over
+// RMS_BLOCKS blocks (at least 16 rows each): two whole waves of the d = 1024
+// kernel, whose 188 registers a thread leave room for one block per SM (64
+// rows a block made 1.73 waves), and one wave at smaller d.
+constexpr int RMS_BLOCKS = 2 * 148;
+int rmsnorm_bwd_blocks(int64_t N) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(N, 16), RMS_BLOCKS));
+}
 
 template <typename A>
 __global__ void k_rmsnorm_bwd(const float *__restrict__ x, const float *__restrict__ rstd,
@@ -279,10 +284,8 @@ __global__ void k_rmsnorm_bwd(const float *__restrict__ x, const float *__restri
   int warp = threadIdx.x / 32, lane = threadIdx.x & 31, nw = blockDim.x / 32;
   float *acc = sacc + (int64_t)warp * d;
   for (int j = lane; j < d; j += 32) acc[j] = 0.f;
-  int64_t r0 = (int64_t)blockIdx.x * RMS_ROWS;
-  for (int rr = warp; rr < RMS_ROWS; rr += nw) {
-    int64_t row = r0 + rr;
-    if (row >= N) break;
+  const int64_t r1 = (blockIdx.x + 1) * N / gridDim.x;
+  for (int64_t row = blockIdx.x * N / gridDim.x + warp; row < r1; row += nw) {
     const float *xr = x + row * d, *dyr = dy + row * d;
     float r = rstd[row];
     float dot = 0.f;
@@ -325,10 +328,8 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bwd_v(const float *__restrict__
     gv[k] = reinterpret_cast<const float4 *>(g)[lane + 32 * k];
     acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const int64_t r0 = (int64_t)blockIdx.x * RMS_ROWS;
-  for (int rr = warp; rr < RMS_ROWS; rr += 8) {
-    const int64_t row = r0 + rr;
-    if (row >= N) break;
+  const int64_t r1 = (blockIdx.x + 1) * N / gridDim.x;
+  for (int64_t row = blockIdx.x * N / gridDim.x + warp; row < r1; row += 8) {
     const float4 *xr = reinterpret_cast<const float4 *>(x + row * d);
     const float4 *dyr = reinterpret_cast<const float4 *>(dy + row * d);
     float4 xv[VPL], dv[VPL], rv[VPL];
@@ -1111,14 +1112,46 @@ void adamw(float *p, const float *g, float *m, float *v, int64_t n, const float 
 
 // ------------------------------------------------------------ wgrad finish
 // grad[r, c] = sum over splits k (in order) of part[k, r, cp(c)]; mode 1 maps
-// the interleaved W1 | W3 columns back.  One thread per group of 4 columns
-// over the whole [rows, cols] gradient (grid-stride), so rows narrower than a
-// block keep every lane busy: an aligned group of 4 columns has 4 contiguous
-// partial-sum columns in both modes (SWIGLU_BLOCK and h multiples of 4), and
-// four splits' loads are in flight at a time, added in split order.
+// the interleaved W1 | W3 columns back.  One block per row (grid-stride), 4
+// columns per thread: an aligned group of 4 columns has 4 contiguous
+// partial-sum columns in both modes (SWIGLU_BLOCK and h multiples of 4).
+// Partial slabs of at most 32 MB (still in L2 from the GEMM that wrote
+// them) go to k_wgrad_finish_flat instead: one thread per group of 4 columns
+// over the whole gradient, four splits' loads in flight, the same sums in the
+// same order.  Measured in the step (per-class CUDA events): the split-K
+// finish of the 512-wide GQA workload 0.356 -> 0.323 ms, of the 256-wide one
+// 0.262 -> 0.239 ms with the flat kernel; at 350M (slabs of 34-131 MB read
+// mostly from HBM) this kernel is faster, 1.48 against 1.64 ms.
+__global__ void k_wgrad_finish(const float *__restrict__ part, int splits, int64_t part_rows,
+                               int64_t ldp, float *__restrict__ grad, int64_t rows, int64_t cols,
+                               int mode, int64_t h, bool vec) {
+  const int64_t pstride = part_rows * ldp;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float *pr = part + r * ldp;
+    float *gr = grad + r * cols;
+    for (int64_t c = 4 * (int64_t)threadIdx.x; c < cols; c += 4 * (int64_t)blockDim.x) {
+      if (vec && c + 4 <= cols) {
+        const int64_t cp = mode == 1 ? ((c < h) ? w1_col(c) : w1_col(c - h) + SWIGLU_BLOCK) : c;
+        float4 acc = *reinterpret_cast<const float4 *>(pr + cp);
+        for (int k = 1; k < splits; k++) {
+          const float4 q = *reinterpret_cast<const float4 *>(pr + k * pstride + cp);
+          acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+        }
+        *reinterpret_cast<float4 *>(gr + c) = acc;
+      } else {
+        for (int64_t cc = c; cc < c + 4 && cc < cols; cc++) {
+          const int64_t cp = mode == 1 ? ((cc < h) ? w1_col(cc) : w1_col(cc - h) + SWIGLU_BLOCK) : cc;
+          float acc = 0.f;
+          for (int k = 0; k < splits; k++) acc += pr[k * pstride + cp];
+          gr[cc] = acc;
+        }
+      }
+    }
+  }
+}
 LLM_DEV float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
 __global__ void __launch_bounds__(256)
-    k_wgrad_finish(const float *__restrict__ part, int splits, int64_t part_rows, int64_t ldp,
+    k_wgrad_finish_flat(const float *__restrict__ part, int splits, int64_t part_rows, int64_t ldp,
                    float *__restrict__ grad, int64_t rows, int64_t cols, int mode, int64_t h,
                    bool vec) {
   const int64_t pstride = part_rows * ldp;
@@ -1155,9 +1188,16 @@ void wgrad_finish(const float *part, int splits, int64_t part_rows, int64_t ldp,
                   int64_t rows, int64_t cols, int mode, int64_t h, cudaStream_t s) {
   const bool vec = ((uintptr_t)part & 15) == 0 && ((uintptr_t)grad & 15) == 0 && ldp % 4 == 0 &&
                    cols % 4 == 0 && (mode == 0 || h % 4 == 0) && (part_rows * ldp) % 4 == 0;
-  const int64_t groups = rows * ((cols + 3) / 4);
-  unsigned grid = (unsigned)std::min<int64_t>((groups + 255) / 256, 148 * 8);
-  k_wgrad_finish<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode, h, vec);
+  if ((int64_t)splits * part_rows * ldp * 4 <= (int64_t(32) << 20)) {
+    const int64_t groups = rows * ((cols + 3) / 4);
+    const unsigned grid = (unsigned)std::min<int64_t>((groups + 255) / 256, 148 * 8);
+    k_wgrad_finish_flat<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode,
+                                             h, vec);
+  } else {
+    const unsigned grid = (unsigned)std::min<int64_t>(rows, 148 * 8);
+    k_wgrad_finish<<<grid, 256, 0, s>>>(part, splits, part_rows, ldp, grad, rows, cols, mode, h,
+                                        vec);
+  }
   count_launch();
 }
 
