@@ -52,6 +52,7 @@ constexpr int NTHREADS = 64 + 32 * EPI_WARPS;
 struct Args {
   int M, N, K;
   int tiles_m, tiles_n, splits, kchunk, total;
+  int nfast;  // tile order of a split: n tiles fastest (1) or m tiles fastest (0)
   int out, epi;
   void *C;
   int64_t ldc;
@@ -61,6 +62,22 @@ struct Args {
   int T, hd, rot_cols;
   int *flag;
 };
+
+// Tile `tile` of a split -> (m tile, n tile).  With few n tiles (a product of
+// N <= 2048 over a long A, e.g. a data gradient dY W with K = vocabulary or
+// hidden width) n runs fastest, so the CTAs at work together take every n tile
+// of the same A rows and read each A panel from HBM once, sharing it in L2 (m
+// fastest re-read every A panel once per n tile: 3.4-3.8x the algorithmic
+// bytes); otherwise m runs fastest and the A operand stays in L2 across n.
+LLM_DEV void tile_mn(const Args &a, int tile, int &mt, int &nt) {
+  if (a.nfast) {
+    mt = tile / a.tiles_n;
+    nt = tile - mt * a.tiles_n;
+  } else {
+    nt = tile / a.tiles_m;
+    mt = tile - nt * a.tiles_m;
+  }
+}
 
 // ------------------------------------------------------------ epilogue stores
 // A warp's 32 x 32 fp32 chunk (lane i holds row i in v) in the per-warp
@@ -302,8 +319,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = 0; i < STAGES; i++) issued[i] = false;
     bool ok = true;
     for (int w = blockIdx.x; w < a.total && ok; w += gridDim.x) {
-      int split = w / tiles_mn, tile = w % tiles_mn;
-      int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
+      int split = w / tiles_mn, tile = w % tiles_mn, mt, nt;
+      tile_mn(a, tile, mt, nt);
+      int m0 = mt * BM, n0 = nt * BN;
       int kb0, nkb = kblocks_of(split, kb0);
       for (int kb = 0; kb < nkb; kb++) {
         if (!warp_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) { ok = false; break; }
@@ -396,8 +414,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int acc = 0;
     uint32_t aph = 0;
     for (int w = blockIdx.x; w < a.total; w += gridDim.x) {
-      int split = w / tiles_mn, tile = w % tiles_mn;
-      int m0 = (tile % a.tiles_m) * BM, n0 = (tile / a.tiles_m) * BN;
+      int split = w / tiles_mn, tile = w % tiles_mn, mt, nt;
+      tile_mn(a, tile, mt, nt);
+      int m0 = mt * BM, n0 = nt * BN;
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
@@ -576,8 +595,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lead_full0 = cluster_addr(full0, 0);
     for (int w = cid; w < a.total && ok; w += ncl) {
       const int split = w / tiles_mn, tile = w % tiles_mn;
-      const int m0 = (tile % a.tiles_m) * 256 + 128 * (int)rank;
-      const int n0 = (tile / a.tiles_m) * 256 + 128 * (int)rank;
+      int mt, nt;
+      tile_mn(a, tile, mt, nt);
+      const int m0 = mt * 256 + 128 * (int)rank;
+      const int n0 = nt * 256 + 128 * (int)rank;
       int kb0, nkb = kblocks_of(split, kb0);
       for (int kb = 0; kb < nkb; kb++) {
         if (!warp_wait(empty0 + 8 * s, ph ^ 1, &abort_sh, a.flag)) { ok = false; break; }
@@ -671,8 +692,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t aph = 0;
     for (int w = cid; w < a.total; w += ncl) {
       const int split = w / tiles_mn, tile = w % tiles_mn;
-      const int m0 = (tile % a.tiles_m) * 256 + 128 * (int)rank;
-      const int n0 = (tile / a.tiles_m) * 256;
+      int mt, nt;
+      tile_mn(a, tile, mt, nt);
+      const int m0 = mt * 256 + 128 * (int)rank;
+      const int n0 = nt * 256;
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
@@ -865,6 +888,7 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   int kc = (g.K + a.splits - 1) / a.splits;
   a.kchunk = ((kc + BK - 1) / BK) * BK;
   a.total = a.tiles_m * a.tiles_n * a.splits;
+  a.nfast = a.tiles_n <= 8;
   a.out = out; a.epi = epi; a.C = C; a.ldc = ldc; a.R = R; a.ldr = ldr;
   a.cos_t = p->cos_t; a.sin_t = p->sin_t; a.T = p->T; a.hd = p->hd; a.rot_cols = (int)p->rot_cols;
   a.flag = p->flag;
@@ -875,6 +899,7 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
     a.tiles_m = (g.M + 255) / 256;
     a.tiles_n = (g.N + BN - 1) / BN;
     a.total = a.tiles_m * a.tiles_n * a.splits;
+    a.nfast = a.tiles_n <= 8;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
