@@ -853,6 +853,13 @@ void wgrad(llm_ctx *c, const void *X, int64_t ldx, const void *dY, int64_t ldy, 
   const Dims &D = c->D;
   int splits = wgrad_splits(D, M, Ncols, tc_gemm_pairs(c->tc, M, Ncols));
   GemmOperands g{(int)M, (int)Ncols, (int)D.N, X, ldx, false, dY, ldy, false, D.dt};
+  // one split, the caller's layout and no padding (the lm_head gradient with
+  // V a multiple of 128): the product goes straight into the gradient
+  if (splits == 1 && mode == 0 && rows == M && cols == Ncols && cols % 4 == 0 &&
+      ((uintptr_t)grad & 15) == 0) {
+    gemm(c, g, OUT_F32, grad, cols, nullptr, 0, 1, 2.0 * rows * cols * D.N);
+    return;
+  }
   gemm(c, g, OUT_PARTIAL, c->part, Ncols, nullptr, 0, splits, 2.0 * rows * cols * D.N);
   KTimer kt(c, LLM_KT_WGRAD_FINISH, 4.0 * splits * M * Ncols + 4.0 * rows * cols);
   wgrad_finish(c->part, splits, M, Ncols, grad, rows, cols, mode, D.h, c->cur);
