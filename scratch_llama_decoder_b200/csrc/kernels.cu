@@ -805,14 +805,16 @@ __global__ void __launch_bounds__(NT) k_cross_entropy_reg(__nv_bfloat16 *__restr
 // Streaming form (bf16, rows of at most 32768 columns): a persistent grid of
 // one 512-thread block per SM walks groups of G = 16 / WPR consecutive rows
 // (WPR warps per row, at most 8 vectors of 8 logits per thread).  Each group
-// comes into one of two 64 KiB shared-memory buffers by one bulk copy
-// (cp.async.bulk, completion counted on an mbarrier), so the next groups load
-// while the current one is reduced and its gradient stored; the row
+// comes into one of CES_NBUF 64 KiB shared-memory buffers by one bulk copy
+// (cp.async.bulk, completion counted on an mbarrier), so the next two groups
+// load while the current one is reduced and its gradient stored (with two
+// buffers, one 64 KiB row in flight per SM left the 350M step's 32000-wide
+// rows at 0.48 of the copy rate); the row
 // arithmetic is the register form's above (one exponential per logit, the
 // terms kept as bf16, one (m, s) reduction per row in a fixed order).  Every
 // wait is bounded: on time-out the block records FLAG_TIMEOUT, waits (again
 // bounded) for its own copies and leaves.
-constexpr int CES_THREADS = 512, CES_R = 8, CES_BUF = 64 * 1024;
+constexpr int CES_THREADS = 512, CES_R = 8, CES_BUF = 64 * 1024, CES_NBUF = 3;
 template <int WPR>
 __global__ void __launch_bounds__(CES_THREADS, 1)
     k_cross_entropy_stream(__nv_bfloat16 *__restrict__ z, const int32_t *__restrict__ tgt,
@@ -820,8 +822,8 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
                            float inv_n, int *flag) {
   constexpr float L2E = 1.4426950408889634f;
   constexpr int G = 16 / WPR, TPR = 32 * WPR;
-  extern __shared__ __align__(1024) uint8_t ce_buf[];  // [2][CES_BUF]
-  __shared__ uint64_t full[2];
+  extern __shared__ __align__(1024) uint8_t ce_buf[];  // [CES_NBUF][CES_BUF]
+  __shared__ uint64_t full[CES_NBUF];
   __shared__ float red_m[16], red_s[16];
   __shared__ int stop_sh;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
@@ -830,14 +832,13 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
   const int nvec = (int)(ldz / 8);
   const uint32_t fb0 = tc::smem_u32(&full[0]);
   if (threadIdx.x == 0) {
-    tc::mbar_init(fb0, 1);
-    tc::mbar_init(fb0 + 8, 1);
+    for (int bb = 0; bb < CES_NBUF; bb++) tc::mbar_init(fb0 + 8 * bb, 1);
     stop_sh = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   // thread 0's record of the copy in flight into each buffer (for the drain)
-  uint32_t issued = 0, par[2] = {0, 0};
+  uint32_t issued = 0, par[CES_NBUF] = {};
   auto issue = [&](int64_t gi, int b) {
     const int64_t rows = min((int64_t)G, N - gi * G);
     const uint32_t bytes = (uint32_t)(rows * row_bytes);
@@ -850,14 +851,13 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
         : "memory");
     issued |= 1u << b;
   };
-  if (threadIdx.x == 0) {
-    if (blockIdx.x < ngroups) issue(blockIdx.x, 0);
-    if (blockIdx.x + gridDim.x < ngroups) issue(blockIdx.x + gridDim.x, 1);
-  }
+  if (threadIdx.x == 0)
+    for (int bb = 0; bb < CES_NBUF; bb++)
+      if (blockIdx.x + (int64_t)bb * gridDim.x < ngroups) issue(blockIdx.x + (int64_t)bb * gridDim.x, bb);
   int k = 0;
   for (int64_t gi = blockIdx.x; gi < ngroups; gi += gridDim.x, k++) {
-    const int b = k & 1;
-    const uint32_t ph = (k >> 1) & 1;
+    const int b = k % CES_NBUF;
+    const uint32_t ph = (k / CES_NBUF) & 1;
     // bounded wait for this group's rows, then a block-wide verdict
     bool ok = tc::mbar_try(fb0 + 8 * b, ph);
     if (!ok) {
@@ -868,7 +868,7 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
     if (__syncthreads_or(!ok)) {
       if (threadIdx.x == 0) {
         atomicOr(flag, FLAG_TIMEOUT);
-        for (int bb = 0; bb < 2; bb++)
+        for (int bb = 0; bb < CES_NBUF; bb++)
           if (issued & (1u << bb)) {
             const unsigned long long t0 = tc::gtimer();
             while (!tc::mbar_try(fb0 + 8 * bb, par[bb]) && tc::gtimer() - t0 < tc::WAIT_NS) {
@@ -896,36 +896,60 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
       y = 0;
     }
     const float zy = valid ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(src)[y]) : 0.f;
-    __syncthreads();  // buffer b is read: the group after next may land in it
-    if (threadIdx.x == 0 && gi + 2 * (int64_t)gridDim.x < ngroups) issue(gi + 2 * gridDim.x, b);
-    // this thread's maximum, its terms (kept as bf16) and their sum
+    __syncthreads();  // buffer b is read: the group CES_NBUF ahead may land in it
+    if (threadIdx.x == 0 && gi + CES_NBUF * (int64_t)gridDim.x < ngroups)
+      issue(gi + CES_NBUF * (int64_t)gridDim.x, b);
+    // this thread's maximum, its terms (kept as bf16) and their sum; a whole
+    // vector inside [0, V) takes the unchecked form: three-input maxima and
+    // packed f32x2 arithmetic (the kernel is issue-bound, not HBM-bound)
     float mt = -INFINITY;
 #pragma unroll
     for (int kk = 0; kk < CES_R; kk++) {
       const int v0 = 8 * (t + TPR * kk);
       const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&q[kk]);
+      if (v0 + 8 <= V) {
 #pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const float2 f = __bfloat1622float2(e[u]);
-        if (v0 + 2 * u < V) mt = fmaxf(mt, f.x);
-        if (v0 + 2 * u + 1 < V) mt = fmaxf(mt, f.y);
+        for (int u = 0; u < 4; u++) {
+          const float2 f = __bfloat1622float2(e[u]);
+          mt = tc::fmax3(mt, f.x, f.y);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+          const float2 f = __bfloat1622float2(e[u]);
+          if (v0 + 2 * u < V) mt = fmaxf(mt, f.x);
+          if (v0 + 2 * u + 1 < V) mt = fmaxf(mt, f.y);
+        }
       }
     }
     const float mt2 = mt == -INFINITY ? 0.f : mt * L2E;
-    float st = 0.f;
+    const float2 l2e2 = make_float2(L2E, L2E), nm2 = make_float2(-mt2, -mt2);
+    float2 st2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int kk = 0; kk < CES_R; kk++) {
       const int v0 = 8 * (t + TPR * kk);
       __nv_bfloat162 *e = reinterpret_cast<__nv_bfloat162 *>(&q[kk]);
+      if (v0 + 8 <= V) {
 #pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const float2 f = __bfloat1622float2(e[u]);
-        const float ea = v0 + 2 * u < V ? ex2_fast(fmaf(f.x, L2E, -mt2)) : 0.f;
-        const float eb = v0 + 2 * u + 1 < V ? ex2_fast(fmaf(f.y, L2E, -mt2)) : 0.f;
-        st += ea + eb;
-        e[u] = __floats2bfloat162_rn(ea, eb);
+        for (int u = 0; u < 4; u++) {
+          const float2 x = __ffma2_rn(__bfloat1622float2(e[u]), l2e2, nm2);
+          const float2 ex = make_float2(ex2_fast(x.x), ex2_fast(x.y));
+          st2 = __fadd2_rn(st2, ex);
+          e[u] = __floats2bfloat162_rn(ex.x, ex.y);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+          const float2 f = __bfloat1622float2(e[u]);
+          const float ea = v0 + 2 * u < V ? ex2_fast(fmaf(f.x, L2E, -mt2)) : 0.f;
+          const float eb = v0 + 2 * u + 1 < V ? ex2_fast(fmaf(f.y, L2E, -mt2)) : 0.f;
+          st2.x += ea;
+          st2.y += eb;
+          e[u] = __floats2bfloat162_rn(ea, eb);
+        }
       }
     }
+    const float st = st2.x + st2.y;
     // the row's (M, S): warp tree, then the row's warps in order
     float M = mt, S = st;
     for (int o = 16; o > 0; o >>= 1) {
@@ -947,6 +971,7 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
     const float lse = M + logf(S);
     if (t == 0) rowloss[row] = lse - zy;
     const float fac = mt == -INFINITY ? 0.f : ex2_fast((mt - M) * L2E) / S * inv_n;
+    const float2 fac2 = make_float2(fac, fac);
     __nv_bfloat16 *zr = z + row * ldz;
 #pragma unroll
     for (int kk = 0; kk < CES_R; kk++) {
@@ -954,12 +979,20 @@ __global__ void __launch_bounds__(CES_THREADS, 1)
       if (i >= nvec) continue;
       const int v0 = 8 * i;
       __nv_bfloat162 *e = reinterpret_cast<__nv_bfloat162 *>(&q[kk]);
+      if ((unsigned)(y - v0) >= 8u) {  // the target is not in this vector
 #pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const float2 f = __bfloat1622float2(e[u]);
-        const int va = v0 + 2 * u, vb = va + 1;
-        e[u] = __floats2bfloat162_rn(f.x * fac - (va == y ? inv_n : 0.f),
-                                     f.y * fac - (vb == y ? inv_n : 0.f));
+        for (int u = 0; u < 4; u++) {
+          const float2 g = __fmul2_rn(__bfloat1622float2(e[u]), fac2);
+          e[u] = __floats2bfloat162_rn(g.x, g.y);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+          const float2 f = __bfloat1622float2(e[u]);
+          const int va = v0 + 2 * u, vb = va + 1;
+          e[u] = __floats2bfloat162_rn(f.x * fac - (va == y ? inv_n : 0.f),
+                                       f.y * fac - (vb == y ? inv_n : 0.f));
+        }
       }
       reinterpret_cast<uint4 *>(zr)[i] = q[kk];
     }
@@ -979,7 +1012,7 @@ void cross_entropy(void *logits, DType dt, const int32_t *tgt, float *rowloss, i
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t groups = (N + 16 / wpr - 1) / (16 / wpr);
     const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(groups, sms));
-    const int smem = 2 * CES_BUF;
+    const int smem = CES_NBUF * CES_BUF;
 #define CES(W)                                                                                    \
   do {                                                                                            \
     smem_optin((const void *)k_cross_entropy_stream<W>, smem);                                   \
