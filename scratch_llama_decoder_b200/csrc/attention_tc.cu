@@ -452,13 +452,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float acc[OW];
 #pragma unroll
       for (int i = 0; i < OW; i++) acc[i] = 0.f;
+      // two groups' loads in flight per wait, added in group order
 #pragma unroll
-      for (int g2 = 0; g2 < NQ; g2++) {
-        float v[OW];
-        tmem_ldn<OW>(tmem + lane_off + COL_O + 64 * g2 + grp * OW, v);
-        const float cg = f[g2] * inv;
+      for (int g2 = 0; g2 < NQ; g2 += 2) {
+        uint32_t va[OW], vb[OW];
+        tmem_ld_raw<OW>(tmem + lane_off + COL_O + 64 * g2 + grp * OW, va);
+        tmem_ld_raw<OW>(tmem + lane_off + COL_O + 64 * (g2 + 1) + grp * OW, vb);
+        tmem_wait_ld();
+        tmem_after_wait(va);
+        tmem_after_wait(vb);
+        const float ca = f[g2] * inv, cb = f[g2 + 1] * inv;
 #pragma unroll
-        for (int i = 0; i < OW; i++) acc[i] += v[i] * cg;
+        for (int i = 0; i < OW; i++) acc[i] += __uint_as_float(va[i]) * ca;
+#pragma unroll
+        for (int i = 0; i < OW; i++) acc[i] += __uint_as_float(vb[i]) * cb;
       }
       // O rows through the item's Q tile (its last S product is complete):
       // this thread's two 16-byte chunks of row r in the tile's
@@ -484,7 +491,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bulk_commit();
       }
       st_slot = it % QSLOTS;  // released after the next item's first block
-      if (grp == 0 && qi < T) lse[((int64_t)b * H + h) * T + qi] = (m + log2f(lt)) * LN2;
+      if (grp == 0 && qi < T) lse[((int64_t)b * H + h) * T + qi] = (m + __log2f(lt)) * LN2;
     }
     if (lane == 0) bulk_wait_all();
   }

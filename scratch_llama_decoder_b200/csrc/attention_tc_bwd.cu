@@ -499,10 +499,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // (head 32: groups 2 and 3 repeat 0 and 1 and stage nothing)
       const int half = hd / 2, xc = (hd == 64 ? cq : (cq & 1)) * HW;
       float xa[HW], ya[HW], xb[HW], yb[HW];
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + xc, xa);
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQA + half + xc, ya);
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + xc, xb);
-      tmem_ldn<HW>(tmem + lane_off + DQ_COL_DQB + half + xc, yb);
+      {  // the four loads in flight together, one wait
+        uint32_t ra[HW], rya[HW], rb[HW], ryb[HW];
+        tmem_ld_raw<HW>(tmem + lane_off + DQ_COL_DQA + xc, ra);
+        tmem_ld_raw<HW>(tmem + lane_off + DQ_COL_DQA + half + xc, rya);
+        tmem_ld_raw<HW>(tmem + lane_off + DQ_COL_DQB + xc, rb);
+        tmem_ld_raw<HW>(tmem + lane_off + DQ_COL_DQB + half + xc, ryb);
+        tmem_wait_ld();
+        tmem_after_wait(ra);
+        tmem_after_wait(rya);
+        tmem_after_wait(rb);
+        tmem_after_wait(ryb);
+#pragma unroll
+        for (int i = 0; i < HW; i++) {
+          xa[i] = __uint_as_float(ra[i]);
+          ya[i] = __uint_as_float(rya[i]);
+          xb[i] = __uint_as_float(rb[i]);
+          yb[i] = __uint_as_float(ryb[i]);
+        }
+      }
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_free);  // the next item's dQ products may start
@@ -867,10 +882,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // dV: columns [cq HW, cq HW + HW) and 32 more (zero past head 32)
       const int half = hd / 2, xc = (hd == 64 ? cq : (cq & 1)) * HW;
       float xk[HW], yk[HW], xv[HW], yv[HW];
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + xc, xk);
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DK + half + xc, yk);
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + cq * HW, xv);
-      tmem_ldn<HW>(tmem + lane_off + KV_COL_DV + 32 + cq * HW, yv);
+      {  // the four loads in flight together, one wait
+        uint32_t rk[HW], ryk[HW], rv[HW], ryv[HW];
+        tmem_ld_raw<HW>(tmem + lane_off + KV_COL_DK + xc, rk);
+        tmem_ld_raw<HW>(tmem + lane_off + KV_COL_DK + half + xc, ryk);
+        tmem_ld_raw<HW>(tmem + lane_off + KV_COL_DV + cq * HW, rv);
+        tmem_ld_raw<HW>(tmem + lane_off + KV_COL_DV + 32 + cq * HW, ryv);
+        tmem_wait_ld();
+        tmem_after_wait(rk);
+        tmem_after_wait(ryk);
+        tmem_after_wait(rv);
+        tmem_after_wait(ryv);
+#pragma unroll
+        for (int i = 0; i < HW; i++) {
+          xk[i] = __uint_as_float(rk[i]);
+          yk[i] = __uint_as_float(ryk[i]);
+          xv[i] = __uint_as_float(rv[i]);
+          yv[i] = __uint_as_float(ryv[i]);
+        }
+      }
       if (kj < T && cos_t)
         rope_bwd_n<HW>(xk, yk, cos_t + (int64_t)kj * half + xc, sin_t + (int64_t)kj * half + xc);
       // dK, dV rows through the item's K and V tiles (their products are

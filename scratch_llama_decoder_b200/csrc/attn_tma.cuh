@@ -1,4 +1,5 @@
-// Head-indexed tensor maps for the tcgen05 attention kernels.
+// Head-indexed tensor maps and TMEM load helpers of the tcgen05 attention
+// kernels.
 //
 // A row of q|k|v (or of O, dO, dq|dk|dv) is a sequence of heads of hd
 // bf16 values; the maps below describe it as [rows][heads][hd], so a tile is
@@ -34,6 +35,35 @@ LLM_DEV void tma_store_4d(const CUtensorMap *map, uint32_t src, int x, int y, in
           (uint64_t)map),
       "r"(x), "r"(y), "r"(z), "r"(w), "r"(src)
       : "memory");
+}
+
+// TMEM loads without their own wait (32x32b shape: lane = row, N columns
+// of 32 bits), so several can be in flight; tmem_wait_regs waits for all of
+// them and re-defines each loaded register after the wait, so no use of one
+// can be scheduled before it.
+template <int N>
+LLM_DEV void tmem_ld_raw(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N == 8 || N == 16, "8 or 16 columns");
+  if constexpr (N == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  } else {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  }
+}
+LLM_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+template <int N>
+LLM_DEV void tmem_after_wait(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; i++) asm volatile("" : "+r"(r[i]));
 }
 
 inline PFN_cuTensorMapEncodeTiled_v12000 encoder() {
