@@ -443,8 +443,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         fence_after();
         float sv[CW], dv[CW];
-        tmem_ldn<CW>(tmem + lane_off + DQ_COL_S + cq * CW, sv);
-        tmem_ldn<CW>(tmem + lane_off + DQ_COL_DP + cq * CW, dv);
+        tmem_ld_pair<CW>(tmem + lane_off + DQ_COL_S + cq * CW, tmem + lane_off + DQ_COL_DP + cq * CW,
+                         sv, dv);
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);  // the MMA warps may overwrite S and dP now
@@ -813,8 +813,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int hf = 0; hf < 2; hf++) {
           constexpr int HC = CW / 2;
           float sv[HC], dv[HC];
-          tmem_ldn<HC>(tmem + lane_off + KV_COL_S + cq * CW + hf * HC, sv);
-          tmem_ldn<HC>(tmem + lane_off + KV_COL_DP + cq * CW + hf * HC, dv);
+          tmem_ld_pair<HC>(tmem + lane_off + KV_COL_S + cq * CW + hf * HC,
+                           tmem + lane_off + KV_COL_DP + cq * CW + hf * HC, sv, dv);
           if (hf == 1) {
             fence_before();
             __syncwarp();

@@ -43,13 +43,13 @@ LLM_DEV void tma_store_4d(const CUtensorMap *map, uint32_t src, int x, int y, in
 // can be scheduled before it.
 template <int N>
 LLM_DEV void tmem_ld_raw(uint32_t taddr, uint32_t (&r)[N]) {
-  static_assert(N == 8 || N == 16, "8 or 16 columns");
+  static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 columns");
   if constexpr (N == 8) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
-  } else {
+  } else if constexpr (N == 16) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
         "%14,%15}, [%16];"
@@ -57,6 +57,30 @@ LLM_DEV void tmem_ld_raw(uint32_t taddr, uint32_t (&r)[N]) {
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+  } else {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+  }
+}
+// A pair of equal loads (two TMEM regions of this thread's lane) under one wait.
+template <int N>
+LLM_DEV void tmem_ld_pair(uint32_t a, uint32_t b, float (&va)[N], float (&vb)[N]) {
+  uint32_t ra[N], rb[N];
+  tmem_ld_raw<N>(a, ra);
+  tmem_ld_raw<N>(b, rb);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < N; i++) {
+    asm volatile("" : "+r"(ra[i]), "+r"(rb[i]));
+    va[i] = __uint_as_float(ra[i]);
+    vb[i] = __uint_as_float(rb[i]);
   }
 }
 LLM_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
