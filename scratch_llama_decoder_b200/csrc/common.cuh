@@ -17,6 +17,15 @@ template <> LLM_DEV float from_f<float>(float x) { return x; }
 template <> LLM_DEV __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 // ---------------------------------------------------------------- reductions
+// sigmoid by the fast exponential and reciprocal intrinsics (relative error
+// ~1e-6, far below the bf16 rounding of the results)
+LLM_DEV float sigmoid_fast(float a) { return __fdividef(1.0f, 1.0f + __expf(-a)); }
+// One SwiGLU unit as the bf16 path computes it: a and b rounded to bf16 (the
+// stored activations), u = a sigmoid(a) b in float32 (rounded by the caller).
+LLM_DEV float swiglu_unit_bf16(float a, float b) {
+  const float ar = __bfloat162float(__float2bfloat16_rn(a)), br = __bfloat162float(__float2bfloat16_rn(b));
+  return ar * sigmoid_fast(ar) * br;
+}
 LLM_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

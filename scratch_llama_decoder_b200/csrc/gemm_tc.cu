@@ -160,6 +160,7 @@ LLM_DEV void rope32(float (&v)[32], const float *cos_row, const float *sin_row) 
 // every tcgen05.ld (warp-uniform control); rows past M and columns past N are
 // clipped only at the stores.
 LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, const CUtensorMap *tmR,
+                           const CUtensorMap *tmU,
                            uint32_t rbar, uint32_t &rph, volatile int *abort_sh, uint32_t tm,
                            int row0, int n0, int c_lo, int split, bool zero, float *stg_base,
                            int &sb) {
@@ -212,6 +213,40 @@ LLM_DEV void epilogue_tile(const Args &a, const CUtensorMap *tmC, const CUtensor
         stage64_bf16(stg, lo, hi);
         bulk_store(stg, tmC, n, row0, 0, false);
       }
+      if (a.epi == TC_EPI_SWIGLU && n0 + c_lo < N) {
+        // the warp's 128 columns are one interleaved block, a for 64 hidden
+        // units then b for the same units: u = silu(a) b from the
+        // accumulator rounded as the stored [a|b] is, 32 units at a time,
+        // into the u tile at hidden column (n0 + c_lo) / 2
+        float u0[32], u1[32];
+        {
+          float av[32], bv[32];
+          if (zero) {
+            for (int i = 0; i < 32; i++) av[i] = bv[i] = 0.f;
+          } else {
+            tmem_ld32(tm + c_lo, av);
+            tmem_ld32(tm + c_lo + 64, bv);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i++) u0[i] = swiglu_unit_bf16(av[i], bv[i]);
+        }
+        {
+          float av[32], bv[32];
+          if (zero) {
+            for (int i = 0; i < 32; i++) av[i] = bv[i] = 0.f;
+          } else {
+            tmem_ld32(tm + c_lo + 32, av);
+            tmem_ld32(tm + c_lo + 96, bv);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i++) u1[i] = swiglu_unit_bf16(av[i], bv[i]);
+        }
+        stg = stg_base + sb * 32 * 32;
+        sb = sb + 1 == STG_BUFS ? 0 : sb + 1;
+        stg_acquire();
+        stage64_bf16(stg, u0, u1);
+        bulk_store(stg, tmU, (n0 + c_lo) / 2, row0, 0, false);
+      }
     } else {
       // fp32 (plain, residual add, or split-K partial into slab `split`), 32
       // columns per store; the residual chunk R[rows, n : n + 32] is brought
@@ -261,7 +296,7 @@ template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
-              const Args a) {
+              const __grid_constant__ CUtensorMap tmU, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t *bars = (uint64_t *)(smem + STAGES * STAGE_BYTES + STAGING_BYTES);
@@ -420,14 +455,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, 0, row0, n0, c_lo, split, true, stg,
+        epilogue_tile(a, &tmC, &tmR, &tmU, rbar, rph, &abort_sh, 0, row0, n0, c_lo, split, true, stg,
                       sb);
         continue;
       }
       if (!warp_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag)) break;
       fence_after();
       uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, tm, row0, n0, c_lo, split, false, stg,
+      epilogue_tile(a, &tmC, &tmR, &tmU, rbar, rph, &abort_sh, tm, row0, n0, c_lo, split, false, stg,
                     sb);
       fence_before();
       __syncwarp();
@@ -533,7 +568,7 @@ template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
-               const Args a) {
+               const __grid_constant__ CUtensorMap tmU, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t *bars = (uint64_t *)(smem + STAGES2 * STAGE2_BYTES + STAGING_BYTES);
@@ -699,14 +734,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int kb0, nkb = kblocks_of(split, kb0);
       const int row0 = m0 + quarter * 32;
       if (nkb == 0) {
-        epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, 0, row0, n0, c_lo, split, true, stg,
+        epilogue_tile(a, &tmC, &tmR, &tmU, rbar, rph, &abort_sh, 0, row0, n0, c_lo, split, true, stg,
                       sb);
         continue;
       }
       if (!warp_wait(tfull0 + 8 * acc, aph, &abort_sh, a.flag)) break;
       fence_after();
       const uint32_t tm = tmem + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile(a, &tmC, &tmR, rbar, rph, &abort_sh, tm, row0, n0, c_lo, split, false, stg,
+      epilogue_tile(a, &tmC, &tmR, &tmU, rbar, rph, &abort_sh, tm, row0, n0, c_lo, split, false, stg,
                     sb);
       fence_before();
       __syncwarp();
@@ -853,7 +888,7 @@ void tc_plan_destroy(TcPlan *p) { delete p; }
 static bool al16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
 bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-             int64_t ldr, int splits, int epi, cudaStream_t s) {
+             int64_t ldr, int splits, int epi, cudaStream_t s, void *U, int64_t ldu) {
   using namespace tc;
   if (!p || g.in != DT_BF16 || !p->flag) return false;
   if (g.M < 1 || g.N < 1 || g.K < 1) return false;
@@ -861,7 +896,11 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
   if (out == OUT_ACT ? (ldc % 8) : (ldc % 4)) return false;
   if (out == OUT_ADD_F32 && (!R || !al16(R) || ldr % 4)) return false;
   if (epi == TC_EPI_ROPE && !(p->hd == 32 || p->hd == 64)) return false;
-  if (epi != TC_EPI_NONE && epi != TC_EPI_ROPE) return false;
+  if (epi != TC_EPI_NONE && epi != TC_EPI_ROPE && epi != TC_EPI_SWIGLU) return false;
+  // SwiGLU: N = 2 hp columns in interleaved blocks of 128 (a then b), u is
+  // [M][hp] bf16 with a 16-byte aligned row stride
+  if (epi == TC_EPI_SWIGLU && (!U || !al16(U) || ldu % 8 || g.N % 128 || ldu < g.N / 2))
+    return false;
   if (epi != TC_EPI_NONE && out != OUT_ACT) return false;
   // tensor maps: A as [rows][K] (K-major) or [K][M] (MN-major); same for B
   CUtensorMap ta, tb;
@@ -880,6 +919,9 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
                   &tcm))
     return false;
   if (out == OUT_ADD_F32 && !p->map_out(R, g.N, g.M, ldr, 1, false, 4, &trm)) return false;
+  CUtensorMap tum;
+  memset(&tum, 0, sizeof(tum));
+  if (epi == TC_EPI_SWIGLU && !p->map_out(U, g.N / 2, g.M, ldu, 1, false, 2, &tum)) return false;
   Args a{};
   a.M = g.M; a.N = g.N; a.K = g.K;
   a.tiles_m = (g.M + BM - 1) / BM;
@@ -913,18 +955,18 @@ bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (!amn && !bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<false, false>, ta, tb, tcm, trm, a);
-    else if (!amn && bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<false, true>, ta, tb, tcm, trm, a);
-    else if (amn && !bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<true, false>, ta, tb, tcm, trm, a);
-    else e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<true, true>, ta, tb, tcm, trm, a);
+    if (!amn && !bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<false, false>, ta, tb, tcm, trm, tum, a);
+    else if (!amn && bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<false, true>, ta, tb, tcm, trm, tum, a);
+    else if (amn && !bmn) e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<true, false>, ta, tb, tcm, trm, tum, a);
+    else e = cudaLaunchKernelEx(&cfg, k_gemm_tc2<true, true>, ta, tb, tcm, trm, tum, a);
     count_launch();
     return e == cudaSuccess;
   }
   int grid = min(a.total, p->num_sms);
-  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
-  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
-  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
-  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, a);
+  if (!amn && !bmn) k_gemm_tc<false, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, tum, a);
+  else if (!amn && bmn) k_gemm_tc<false, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, tum, a);
+  else if (amn && !bmn) k_gemm_tc<true, false><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, tum, a);
+  else k_gemm_tc<true, true><<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tcm, trm, tum, a);
   count_launch();
   return true;
 }

@@ -10,8 +10,9 @@ namespace llm {
 struct TcPlan;
 
 enum TcEpi {
-  TC_EPI_NONE = 0,  // plain output as selected by GemmOut
-  TC_EPI_ROPE = 1   // QKV forward: rotate q and k columns (RoPE) in the epilogue
+  TC_EPI_NONE = 0,   // plain output as selected by GemmOut
+  TC_EPI_ROPE = 1,   // QKV forward: rotate q and k columns (RoPE) in the epilogue
+  TC_EPI_SWIGLU = 2  // W13 forward: besides the interleaved [a|b], u = silu(a) b into U
 };
 
 TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, int hd,
@@ -19,8 +20,10 @@ TcPlan *tc_plan_create(DType dt, const float *cos_t, const float *sin_t, int T, 
 void tc_plan_destroy(TcPlan *p);
 // Device flag word that records a bounded wait giving up (FLAG_TIMEOUT).
 void tc_plan_set_flag(TcPlan *p, int *flag);
+// U, ldu: the SwiGLU output of TC_EPI_SWIGLU (bf16 [M][ldu]; unused otherwise).
 bool tc_gemm(TcPlan *p, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-             int64_t ldr, int splits, int epi, cudaStream_t s);
+             int64_t ldr, int splits, int epi, cudaStream_t s, void *U = nullptr,
+             int64_t ldu = 0);
 // Whether tc_gemm runs an [M, N] product on CTA pairs (256 x 256 tiles, 74
 // pairs on 148 SMs) rather than single CTAs (128 x 256 tiles).
 bool tc_gemm_pairs(const TcPlan *p, int64_t M, int64_t N);

@@ -538,9 +538,6 @@ LLM_DEV uint4 pack8(const float (&f)[8]) {
   }
   return q;
 }
-// sigmoid by the fast exponential and reciprocal intrinsics (relative error
-// ~1e-6, far below the bf16 rounding of the results)
-LLM_DEV float sigmoid_fast(float a) { return __fdividef(1.0f, 1.0f + __expf(-a)); }
 // Grid-stride over (row, 8-unit group) items with 32-bit index arithmetic
 // (the launcher keeps N * hp / 8 below 2^31).
 __global__ void k_swiglu_fwd_v8(const __nv_bfloat16 *__restrict__ ab, __nv_bfloat16 *__restrict__ u,

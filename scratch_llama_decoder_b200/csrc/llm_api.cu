@@ -692,10 +692,11 @@ double attn_flops(const Dims &D, double mult) {  // causal: T (T + 1) / 2 pairs
 // Tensor-core GEMM launch; when timing is on, timed as class GEMM with its
 // algorithmic FLOPs (unpadded sizes).
 bool run_tc(llm_ctx *c, const GemmOperands &g, GemmOut out, void *C, int64_t ldc, const float *R,
-            int64_t ldr, int splits, int epi, double alg_flops) {
+            int64_t ldr, int splits, int epi, double alg_flops, void *U = nullptr,
+            int64_t ldu = 0) {
   if (!c->tc) return false;
   KTimer kt(c, LLM_KT_GEMM, alg_flops);
-  const bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->cur);
+  const bool ok = tc_gemm(c->tc, g, out, C, ldc, R, ldr, splits, epi, c->cur, U, ldu);
   if (!ok) kt.drop();
   return ok;
 }
@@ -788,13 +789,16 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
     KTimer kt(c, LLM_KT_RMSNORM_FWD, rms_fwd_bytes(D));
     rmsnorm_fwd(x1, p + O.g2(l), xn2, D.dt, rstd2, N, D.d, c->cfg.rms_eps, s);
   }
-  // W13 GEMM into the interleaved [a|b], then u = silu(a) * b (a separate
-  // full-occupancy pass: cheaper than the same math in the GEMM epilogue)
-  gemm(c, GemmOperands{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt},
-       OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
+  // W13 GEMM into the interleaved [a|b] with u = silu(a) * b written by the
+  // same epilogue (tensor-core path); else the GEMM, then a separate pass
   {
-    KTimer kt(c, LLM_KT_SWIGLU_FWD, 3.0 * N * D.h * ab);  // read a, b; write u
-    swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
+    const GemmOperands g13{(int)N, (int)(2 * D.hp), D.d, xn2, d, true, w13, 2 * D.hp, false, D.dt};
+    if (!run_tc(c, g13, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, TC_EPI_SWIGLU,
+                2.0 * N * d * 2 * D.h, u, D.hp)) {
+      gemm(c, g13, OUT_ACT, abuf, 2 * D.hp, nullptr, 0, 1, 2.0 * N * d * 2 * D.h);
+      KTimer kt(c, LLM_KT_SWIGLU_FWD, 3.0 * N * D.h * ab);  // read a, b; write u
+      swiglu_fwd(abuf, u, D.dt, N, D.hp, s);
+    }
   }
   if (!out) return;  // the recomputation stops here: x2 exists
   if (drop) {  // x2 = x1 + f * (u W2)
