@@ -20,12 +20,18 @@ template <> LLM_DEV __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __floa
 // sigmoid by the fast exponential and reciprocal intrinsics (relative error
 // ~1e-6, far below the bf16 rounding of the results)
 LLM_DEV float sigmoid_fast(float a) { return __fdividef(1.0f, 1.0f + __expf(-a)); }
-// One SwiGLU unit as the bf16 path computes it: a and b rounded to bf16 (the
-// stored activations), u = a sigmoid(a) b in float32 (rounded by the caller).
-LLM_DEV float swiglu_unit_bf16(float a, float b) {
-  const float ar = __bfloat162float(__float2bfloat16_rn(a)), br = __bfloat162float(__float2bfloat16_rn(b));
-  return ar * sigmoid_fast(ar) * br;
+// One SwiGLU unit, u = a sigmoid(a) b, and its backward (g = du): the one
+// arithmetic of the separate SwiGLU passes and of the GEMM epilogues that
+// take them over, so both give the same bits.
+LLM_DEV float swiglu_unit(float a, float b) { return a * sigmoid_fast(a) * b; }
+LLM_DEV void swiglu_bwd_unit(float a, float b, float g, float &da, float &db) {
+  const float sg = sigmoid_fast(a);
+  da = g * b * sg * (1.f + a * (1.f - sg));
+  db = g * a * sg;
 }
+LLM_DEV float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+// The forward unit from float32 a and b rounded as the stored [a|b] is.
+LLM_DEV float swiglu_unit_bf16(float a, float b) { return swiglu_unit(round_bf16(a), round_bf16(b)); }
 LLM_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

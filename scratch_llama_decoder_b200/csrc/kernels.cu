@@ -550,7 +550,7 @@ __global__ void k_swiglu_fwd_v8(const __nv_bfloat16 *__restrict__ ab, __nv_bfloa
     unpack8(*reinterpret_cast<const uint4 *>(r), a);
     unpack8(*reinterpret_cast<const uint4 *>(r + SWIGLU_BLOCK), b);
 #pragma unroll
-    for (int k = 0; k < 8; k++) o[k] = a[k] * sigmoid_fast(a[k]) * b[k];
+    for (int k = 0; k < 8; k++) o[k] = swiglu_unit(a[k], b[k]);
     *reinterpret_cast<uint4 *>(u + (int64_t)row * hp + j) = pack8(o);
   }
 }
@@ -565,11 +565,7 @@ __global__ void k_swiglu_bwd_v8(const __nv_bfloat16 *__restrict__ ab, const __nv
     unpack8(*reinterpret_cast<const uint4 *>(ab + ca + SWIGLU_BLOCK), b);
     unpack8(*reinterpret_cast<const uint4 *>(du + (int64_t)row * hp + j), g);
 #pragma unroll
-    for (int k = 0; k < 8; k++) {
-      float sg = sigmoid_fast(a[k]);
-      da[k] = g[k] * b[k] * sg * (1.f + a[k] * (1.f - sg));
-      db[k] = g[k] * a[k] * sg;
-    }
+    for (int k = 0; k < 8; k++) swiglu_bwd_unit(a[k], b[k], g[k], da[k], db[k]);
     *reinterpret_cast<uint4 *>(dab + ca) = pack8(da);
     *reinterpret_cast<uint4 *>(dab + ca + SWIGLU_BLOCK) = pack8(db);
   }
