@@ -26,7 +26,8 @@ events around every GEMM launch over K more steps run right after the timed
 region as individual launches (events cannot time nodes of a replayed graph;
 the kernels are the same).  e2e repeats the timed loop through the same C ABI
 with the step's tokens and targets copied from pinned host memory each step
-and the loss read back each step.  cpu_baseline times the float64 CPU oracle
+and the loss read back each step (one step in flight: the host reads step i's
+loss after launching step i + 1).  cpu_baseline times the float64 CPU oracle
 on a bounded sample of the same workload.
 
 Decode (--decode): generation throughput of the same workload's model with a
@@ -494,15 +495,27 @@ def run_ours(args, rank, world, local_rank):
                 train_step(t)
                 loss_pin.copy_(loss, non_blocking=True)
                 stream.synchronize()
+            # one step in flight: step i + 1's inputs are copied (behind step
+            # i on the stream, so step i has read its own) and its graph
+            # launched before the host reads step i's loss from its pinned slot
+            loss_slots = [torch.zeros(1).pin_memory() for _ in range(2)]
+            done = [torch.cuda.Event() for _ in range(2)]
+            seen = []
             f0.record(stream)
-            for _ in range(args.steps):
+            for i in range(args.steps):
                 t += 1
                 tok.copy_(tok_pin, non_blocking=True)
                 tgt.copy_(tgt_pin, non_blocking=True)
                 train_step(t)
-                loss_pin.copy_(loss, non_blocking=True)
-                stream.synchronize()
+                loss_slots[i % 2].copy_(loss, non_blocking=True)
+                done[i % 2].record(stream)
+                if i > 0:
+                    done[(i - 1) % 2].synchronize()
+                    seen.append(float(loss_slots[(i - 1) % 2].item()))
             f1.record(stream)
+            done[(args.steps - 1) % 2].synchronize()
+            seen.append(float(loss_slots[(args.steps - 1) % 2].item()))
+            assert len(seen) == args.steps and all(x == x for x in seen), seen
         torch.cuda.synchronize()
         barrier()
         ems = f0.elapsed_time(f1)
