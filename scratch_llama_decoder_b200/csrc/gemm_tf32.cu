@@ -103,6 +103,39 @@ __global__ void __launch_bounds__(256) k_tf32_split(const float *__restrict__ X,
   }
 }
 
+// The K-major split as a grid-stride pass, one thread per 4 consecutive
+// elements of a row (Kp a multiple of 32, so a row is whole float4 groups):
+// 16-byte loads when X is 16-byte aligned with ld a multiple of 4, and 16-byte
+// stores of hi and lo (the tiled kernel above moved 4 KiB per 256-thread
+// block, which left it launch-bound).
+__global__ void __launch_bounds__(256) k_tf32_split_rows(const float *__restrict__ X, int64_t ld,
+                                                         int rows, int K, int Kp, bool vec,
+                                                         float *__restrict__ hi,
+                                                         float *__restrict__ lo) {
+  const uint32_t q = (uint32_t)Kp / 4, n = (uint32_t)rows * q;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const uint32_t r = i / q;
+    const int k = 4 * (int)(i - r * q);
+    const float *xr = X + (int64_t)r * ld;
+    float x[4];
+    if (vec && k + 4 <= K) {
+      const float4 v = *reinterpret_cast<const float4 *>(xr + k);
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; e++) x[e] = k + e < K ? xr[k + e] : 0.f;
+    }
+    float h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      h[e] = tf32_round(x[e]);
+      l[e] = x[e] - h[e];
+    }
+    *reinterpret_cast<float4 *>(hi + (int64_t)r * Kp + k) = make_float4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<float4 *>(lo + (int64_t)r * Kp + k) = make_float4(l[0], l[1], l[2], l[3]);
+  }
+}
+
 struct Args {
   int M, N, Kp, kchunk;  // kchunk: K floats per split (a multiple of 32)
   int tiles_n, tiles, splits;  // work items: tiles x splits, tile = (row block, column block)
@@ -332,8 +365,16 @@ static bool tile_map_f32(CUtensorMap *map, const float *base, int64_t Kp, int64_
 static void split(const float *X, int64_t ld, bool kmajor, int rows, int K, int Kp, float *hi,
                   float *lo, cudaStream_t s) {
   dim3 grid((unsigned)(Kp / 32), (unsigned)((rows + 31) / 32));
-  if (kmajor) k_tf32_split<true><<<grid, 256, 0, s>>>(X, ld, rows, K, Kp, hi, lo);
-  else k_tf32_split<false><<<grid, 256, 0, s>>>(X, ld, rows, K, Kp, hi, lo);
+  if (kmajor && (int64_t)rows * (Kp / 4) < (int64_t(1) << 31)) {
+    const bool vec = ((uintptr_t)X & 15) == 0 && ld % 4 == 0;
+    const int64_t groups = (int64_t)rows * (Kp / 4);
+    const unsigned g1 = (unsigned)std::min<int64_t>((groups + 255) / 256, 148 * 16);
+    k_tf32_split_rows<<<g1, 256, 0, s>>>(X, ld, rows, K, Kp, vec, hi, lo);
+  } else if (kmajor) {
+    k_tf32_split<true><<<grid, 256, 0, s>>>(X, ld, rows, K, Kp, hi, lo);
+  } else {
+    k_tf32_split<false><<<grid, 256, 0, s>>>(X, ld, rows, K, Kp, hi, lo);
+  }
   count_launch();
 }
 
