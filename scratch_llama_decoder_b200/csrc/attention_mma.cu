@@ -176,8 +176,9 @@ template <int HD>
 __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict__ qkv,
                                                  __nv_bfloat16 *__restrict__ o,
                                                  float *__restrict__ lse, int T, int H, int Hkv,
-                                                 float scale) {
+                                                 float scale, const DropArgs drop) {
   __shared__ Tile<HD> Qs, Ks[2], Vs[2];
+  const uint32_t dstep = drop.on ? (uint32_t)*drop.step : 0u;
   // grid (H, B, query blocks): blocks are dispatched x-fastest, so the last
   // (longest) query blocks of every head start first
   const int nqb = gridDim.z;
@@ -254,6 +255,17 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
         acc[i][2 * r + 1] *= corr;
       }
     }
+    if (drop.on) {  // P V with the dropped probabilities P f; l keeps P's sums
+#pragma unroll
+      for (int nt = 0; nt < 8; nt++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const int qi = row0 + (e >> 1) * 8;
+          const int kj = k0 + nt * 8 + (lane & 3) * 2 + (e & 1);
+          if (kj <= qi && kj < T && qi < T)
+            s[nt][e] *= drop_factor(drop, (((uint64_t)b * H + h) * T + qi) * T + kj, dstep);
+        }
+    }
     uint32_t pf[4][4];
     c_to_a(s, pf);
     mma_ab<HD>(acc, pf, Vs[cur]);
@@ -288,9 +300,10 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
                                                 __nv_bfloat16 *__restrict__ dqkv,
                                                 const float *__restrict__ cos_t,
                                                 const float *__restrict__ sin_t, int T, int H,
-                                                int Hkv, float scale) {
+                                                int Hkv, float scale, const DropArgs drop) {
   __shared__ Tile<HD> Ks[2], Vs[2];
   __shared__ float Dsh[64];
+  const uint32_t dstep = drop.on ? (uint32_t)*drop.step : 0u;
   const int nqb = gridDim.z;
   const int qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -377,8 +390,13 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
         int r = e >> 1;
         int qi = row0 + r * 8;
         int kj = k0 + nt * 8 + (lane & 3) * 2 + (e & 1);
-        float p = (kj > qi || kj >= T || qi >= T) ? 0.f : tc::ex2(s[nt][e] * sl2 - L2[r]);
-        s[nt][e] = p * (dp[nt][e] - Dr[r]);  // dS
+        const bool valid = !(kj > qi || kj >= T || qi >= T);
+        float p = valid ? tc::ex2(s[nt][e] * sl2 - L2[r]) : 0.f;
+        float dpv = dp[nt][e];
+        // with dropout dP = f (dO . v), the forward having multiplied v by P f
+        if (drop.on && valid)
+          dpv *= drop_factor(drop, (((uint64_t)b * H + h) * T + qi) * T + kj, dstep);
+        s[nt][e] = p * (dpv - Dr[r]);  // dS
       }
     }
     uint32_t sf[4][4];
@@ -407,8 +425,9 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
                                                  __nv_bfloat16 *__restrict__ dqkv,
                                                  const float *__restrict__ cos_t,
                                                  const float *__restrict__ sin_t, int T, int H,
-                                                 int Hkv, float scale) {
+                                                 int Hkv, float scale, const DropArgs drop) {
   __shared__ Tile<HD> KVs, Qs[2], dOs[2];
+  const uint32_t dstep = drop.on ? (uint32_t)*drop.step : 0u;
   __shared__ float Ls[2][64], Ds[2][64];
   // grid (Hkv, B, key blocks): the first key blocks see the most query
   // blocks, and blocks are dispatched x-fastest, so they start first
@@ -460,7 +479,7 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
   cp_commit();
   for (int step = 0; step < nsteps; step++) {
     const int cur = step & 1;
-    const int qb = kb + step % (nqb - kb);
+    const int qb = kb + step % (nqb - kb), hq = g * grp + step / (nqb - kb);
     if (step + 1 < nsteps) issue(step + 1, cur ^ 1);
     cp_commit();
     cp_wait<1>();
@@ -484,9 +503,13 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
           int kj = key0 + (e >> 1) * 8;
           int col = hf * 32 + nt * 8 + (lane & 3) * 2 + (e & 1);
           int qi = q0 + col;
-          float p = (kj > qi || qi >= T || kj >= T) ? 0.f : tc::ex2(s[nt][e] * sl2 - Ls[cur][col]);
-          s[nt][e] = p;                                // P^T
-          dp[nt][e] = p * (dp[nt][e] - Ds[cur][col]);  // dS^T
+          const bool valid = !(kj > qi || qi >= T || kj >= T);
+          float p = valid ? tc::ex2(s[nt][e] * sl2 - Ls[cur][col]) : 0.f;
+          float f = 1.f;  // the forward multiplied v by P f: dV takes P f, dP takes f
+          if (drop.on && valid)
+            f = drop_factor(drop, (((uint64_t)b * H + hq) * T + qi) * T + kj, dstep);
+          s[nt][e] = p * f;                                // (P f)^T
+          dp[nt][e] = p * (dp[nt][e] * f - Ds[cur][col]);  // dS^T
         }
       }
       uint32_t pf[2][4], sf[2][4];
@@ -517,22 +540,22 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
 bool attn_mma_covers(DType dt, int hd) { return dt == DT_BF16 && (hd == 32 || hd == 64); }
 
 void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
-                  cudaStream_t s) {
+                  cudaStream_t s, DropArgs drop) {
   using namespace attn;
   dim3 grid(H, B, (T + BQ - 1) / BQ);
   float scale = 1.0f / sqrtf((float)hd);
   if (hd == 64)
     k_attn_fwd<64><<<grid, NT, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, T, H,
-                                       Hkv, scale);
+                                       Hkv, scale, drop);
   else
     k_attn_fwd<32><<<grid, NT, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, T, H,
-                                       Hkv, scale);
+                                       Hkv, scale, drop);
   count_launch();
 }
 
 void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
                   void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
-                  const float *sin_t, cudaStream_t s) {
+                  const float *sin_t, cudaStream_t s, DropArgs drop) {
   using namespace attn;
   float scale = 1.0f / sqrtf((float)hd);
   const __nv_bfloat16 *q = (const __nv_bfloat16 *)qkv, *oo = (const __nv_bfloat16 *)o,
@@ -540,11 +563,11 @@ void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float 
   __nv_bfloat16 *dq = (__nv_bfloat16 *)dqkv;
   dim3 gq(H, B, (T + BQ - 1) / BQ), gkv(Hkv, B, (T + BKV - 1) / BKV);
   if (hd == 64) {
-    k_attn_dq<64><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
-    k_attn_dkv<64><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
+    k_attn_dq<64><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
+    k_attn_dkv<64><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
   } else {
-    k_attn_dq<32><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
-    k_attn_dkv<32><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale);
+    k_attn_dq<32><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
+    k_attn_dkv<32><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
   }
   count_launch(2);
 }

@@ -154,13 +154,15 @@ void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float
 
 // Tensor-core (mma.sync, bf16) kernels for head sizes 32 and 64.
 bool attn_mma_covers(DType dt, int hd);
+// drop: inverted dropout on the attention probabilities (the masks of the
+// CUDA-core kernels, element ((b H + h) T + i) T + j); off by default.
 void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int Hkv, int hd,
-                  cudaStream_t s);
+                  cudaStream_t s, DropArgs drop = DropArgs{});
 // With cos_t/sin_t (RoPE tables [T, hd/2]) non-null, dq and dk are rotated
 // back by -angle before they are stored.
 void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
                   void *dqkv, int B, int T, int H, int Hkv, int hd, const float *cos_t,
-                  const float *sin_t, cudaStream_t s);
+                  const float *sin_t, cudaStream_t s, DropArgs drop = DropArgs{});
 
 // tcgen05 flash-attention forward (bf16, head size 64); false when it does not
 // cover the arguments.  flag: device word for FLAG_TIMEOUT.

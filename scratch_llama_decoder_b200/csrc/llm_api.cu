@@ -772,7 +772,12 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
     }
   }
   if (drop) {  // x1 = x + f * (o Wo), o from dropped probabilities
-    attn_fwd_simt(qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
+    if (attn_mma_covers(D.dt, D.hd)) {
+      KTimer kt(c, LLM_KT_ATTN_FWD, attn_flops(D, 4.0));
+      attn_fwd_mma(qkv, o, lse, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
+    } else {
+      attn_fwd_simt(qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
+    }
     gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_F32, c->dtmp, d,
          nullptr, 0, 1, 2.0 * N * d * d);
     drop_add(x, c->dtmp, x1, N * d, drop_args(c, 2, l), s);
@@ -962,7 +967,11 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
     if (drop) drop_to_act(c->dx, c->dxA, D.dt, N * d, drop_args(c, 2, l), s);
     gemm(c, GemmOperands{(int)N, D.d, D.d, dxop, d, true, wo, d, true, D.dt}, OUT_ACT, c->dO, d,
          nullptr, 0, 1, 2.0 * N * d * d);
-    if (drop) {  // the same probability masks, then RoPE backward on dq, dk
+    if (drop && attn_mma_covers(D.dt, D.hd)) {  // the same probability masks, RoPE fused
+      KTimer kt(c, LLM_KT_ATTN_BWD, attn_flops(D, 8.0));
+      attn_bwd_mma(qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.B, D.T, D.H, D.Hkv, D.hd, c->cos_t,
+                   c->sin_t, s, drop_args(c, 1, l));
+    } else if (drop) {  // the same probability masks, then RoPE backward on dq, dk
       attn_bwd_simt(qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s,
                     drop_args(c, 1, l));
       rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);

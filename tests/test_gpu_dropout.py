@@ -28,7 +28,10 @@ def _setup(cfg, stream=None):
 
 @pytest.mark.parametrize("name,over", [("c1", dict(batch=2)),
                                        ("c3", dict(batch=2, ctx=64, n_layer=2)),
-                                       ("c4", dict(batch=1, ctx=96, n_layer=2))])
+                                       ("c4", dict(batch=1, ctx=96, n_layer=2)),
+                                       # several 64-row tiles with ragged tails (head 32, head 64 GQA)
+                                       ("c3", dict(batch=1, ctx=130, n_layer=1)),
+                                       ("c4", dict(batch=1, ctx=200, n_layer=1))])
 def test_dropout_grads_match_oracle(name, over):
     cfg = get_config(name, **over)
     lay, p, tok, tgt, m = _setup(cfg)
