@@ -52,13 +52,15 @@ typedef struct {
  * embeddings, the attention weights and the attention and MLP outputs; masks
  * drawn by the training forward and reused by its backward).  The masks come
  * from Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
- * easy as 1, 2, 3", SC 2011): key = the seed's two 32-bit halves, counter =
- * (element index low word, element index high word, site + 4 * layer, step),
- * with sites 0 embedding output [B*T, d], 1 attention probabilities
- * [B, H, T, T], 2 attention branch output [B*T, d], 3 MLP branch output
- * [B*T, d] (element index row-major over those shapes).  An element is kept
- * when the first output word is >= floor(p * 2^32); kept elements are scaled
- * by 1 / (1 - p). */
+ * easy as 1, 2, 3", SC 2011), whose one call gives four 32-bit words: the
+ * elements are taken in groups of four consecutive indices, key = the seed's
+ * two 32-bit halves, counter = (group index low word, group index high word,
+ * site + 4 * layer, step), group index = element index / 4, with sites 0
+ * embedding output [B*T, d], 1 attention probabilities [B, H, T, T],
+ * 2 attention branch output [B*T, d], 3 MLP branch output [B*T, d] (element
+ * index row-major over those shapes).  Element e is kept when output word
+ * e mod 4 of its group's call is >= floor(p * 2^32); kept elements are scaled
+ * by 1 / (1 - p).  The pages fix the rate and the sites, not the generator. */
 void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
   uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3], k0 = key[0], k1 = key[1];
   for (int r = 0; r < 10; r++) {
@@ -80,11 +82,12 @@ typedef struct {
 
 /* 0 or 1/(1-p) for element e of (site, layer) */
 static double drop_factor(const orc_dropout *dr, int site, int layer, uint64_t e) {
-  uint32_t ctr[4] = {(uint32_t)e, (uint32_t)(e >> 32), (uint32_t)(site + 4 * layer), dr->step};
+  const uint64_t g = e / 4;
+  uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), (uint32_t)(site + 4 * layer), dr->step};
   uint32_t key[2] = {(uint32_t)dr->seed, (uint32_t)(dr->seed >> 32)}, out[4];
   orc_philox4x32_10(ctr, key, out);
   const uint64_t thr = (uint64_t)floor(dr->p * 4294967296.0);
-  return (uint64_t)out[0] >= thr ? 1.0 / (1.0 - dr->p) : 0.0;
+  return (uint64_t)out[e % 4] >= thr ? 1.0 / (1.0 - dr->p) : 0.0;
 }
 
 /* ------------------------------------------------------------------ layout */

@@ -171,6 +171,63 @@ LLM_DEV void rope_bwd_row(float (&acc)[HD / 8][4], int r, const float *ct, const
     }
 }
 
+// ------------------------------------------------------------------ dropout
+// Factors of the probabilities (element (hrow + i) T + j of the site, hrow =
+// (b H + h) T) a thread holds in one 8-column tile of a warp's 16-row tile.
+// With T % 4 == 0 the keys 4m .. 4m + 3 of a query are one generator group,
+// so the warp's 32 groups of the tile are drawn once each, one per lane, and
+// the keep bits go to their holders by shuffles; otherwise every element
+// draws its own group.
+//
+// Query-row tiles (forward, dQ): rows r0 + 0..15 are queries, columns k8 +
+// 0..7 keys; a thread holds rows (lane >> 2) + 8 (e >> 1), columns
+// 2 (lane & 3) + (e & 1).  Lane x draws row (x >> 2) + 8 (x & 1), keys
+// 4 ((x >> 1) & 1) .. + 3, so element e's bits are in lane (lane & ~1) |
+// (e >> 1), at bit 2 (lane & 1) + (e & 1).
+LLM_DEV void drop_q_tile(const DropArgs &drop, uint64_t hrow, int T, int r0, int k8, int lane,
+                         uint32_t step, float (&f)[4]) {
+  if ((T & 3) == 0) {
+    const int rx = r0 + (lane >> 2) + (lane & 1) * 8, kx = k8 + ((lane >> 1) & 1) * 4;
+    const uint32_t mine = drop_bits4(drop, ((hrow + rx) * (uint64_t)T + kx) >> 2, step);
+    const uint32_t lo = __shfl_sync(0xffffffffu, mine, lane & ~1);
+    const uint32_t hi = __shfl_sync(0xffffffffu, mine, lane | 1);
+    const int sh = (lane & 1) * 2;
+#pragma unroll
+    for (int e = 0; e < 4; e++)
+      f[e] = (((e >> 1) ? hi : lo) >> (sh + (e & 1))) & 1u ? drop.scale : 0.f;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int qi = r0 + (lane >> 2) + (e >> 1) * 8, kj = k8 + (lane & 3) * 2 + (e & 1);
+      f[e] = drop_factor(drop, (hrow + qi) * (uint64_t)T + kj, step);
+    }
+  }
+}
+// Key-row tiles (dK/dV): rows kr0 + 0..15 are keys, columns q8 + 0..7
+// queries; a thread holds keys (lane >> 2) + 8 (e >> 1), queries
+// 2 (lane & 3) + (e & 1).  Lane x draws query x >> 2, keys 4 (x & 3) .. + 3,
+// so element e's bits are in lane 4 (2 (lane & 3) + (e & 1)) + (lane >> 4) +
+// 2 (e >> 1), at bit (lane >> 2) & 3.
+LLM_DEV void drop_k_tile(const DropArgs &drop, uint64_t hrow, int T, int kr0, int q8, int lane,
+                         uint32_t step, float (&f)[4]) {
+  if ((T & 3) == 0) {
+    const int qx = q8 + (lane >> 2), kx = kr0 + (lane & 3) * 4;
+    const uint32_t mine = drop_bits4(drop, ((hrow + qx) * (uint64_t)T + kx) >> 2, step);
+    const int sh = (lane >> 2) & 3;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int src = 4 * ((lane & 3) * 2 + (e & 1)) + (lane >> 4) + 2 * (e >> 1);
+      f[e] = (__shfl_sync(0xffffffffu, mine, src) >> sh) & 1u ? drop.scale : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int kj = kr0 + (lane >> 2) + (e >> 1) * 8, qi = q8 + (lane & 3) * 2 + (e & 1);
+      f[e] = drop_factor(drop, (hrow + qi) * (uint64_t)T + kj, step);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ forward
 template <int HD>
 __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict__ qkv,
@@ -256,15 +313,14 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
       }
     }
     if (drop.on) {  // P V with the dropped probabilities P f; l keeps P's sums
+      const uint64_t hrow = ((uint64_t)b * H + h) * T;
 #pragma unroll
-      for (int nt = 0; nt < 8; nt++)
+      for (int nt = 0; nt < 8; nt++) {
+        float f[4];
+        drop_q_tile(drop, hrow, T, q0 + w * 16, k0 + nt * 8, lane, dstep, f);
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-          const int qi = row0 + (e >> 1) * 8;
-          const int kj = k0 + nt * 8 + (lane & 3) * 2 + (e & 1);
-          if (kj <= qi && kj < T && qi < T)
-            s[nt][e] *= drop_factor(drop, (((uint64_t)b * H + h) * T + qi) * T + kj, dstep);
-        }
+        for (int e = 0; e < 4; e++) s[nt][e] *= f[e];  // masked entries are 0 already
+      }
     }
     uint32_t pf[4][4];
     c_to_a(s, pf);
@@ -385,6 +441,9 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
     const int k0 = kb * BKV;
 #pragma unroll
     for (int nt = 0; nt < 8; nt++) {
+      float f[4];
+      if (drop.on)
+        drop_q_tile(drop, ((uint64_t)b * H + h) * T, T, q0 + w * 16, k0 + nt * 8, lane, dstep, f);
 #pragma unroll
       for (int e = 0; e < 4; e++) {
         int r = e >> 1;
@@ -394,8 +453,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
         float p = valid ? tc::ex2(s[nt][e] * sl2 - L2[r]) : 0.f;
         float dpv = dp[nt][e];
         // with dropout dP = f (dO . v), the forward having multiplied v by P f
-        if (drop.on && valid)
-          dpv *= drop_factor(drop, (((uint64_t)b * H + h) * T + qi) * T + kj, dstep);
+        if (drop.on) dpv *= f[e];
         s[nt][e] = p * (dpv - Dr[r]);  // dS
       }
     }
@@ -498,6 +556,11 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
       mma_abt<HD, 4>(dp, vf, dOs[cur], hf * 32);
 #pragma unroll
       for (int nt = 0; nt < 4; nt++) {
+        // the forward multiplied v by P f: dV takes P f, dP takes f
+        float f[4] = {1.f, 1.f, 1.f, 1.f};
+        if (drop.on)
+          drop_k_tile(drop, ((uint64_t)b * H + hq) * T, T, k0 + w * 16, q0 + hf * 32 + nt * 8,
+                      lane, dstep, f);
 #pragma unroll
         for (int e = 0; e < 4; e++) {
           int kj = key0 + (e >> 1) * 8;
@@ -505,11 +568,8 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
           int qi = q0 + col;
           const bool valid = !(kj > qi || qi >= T || kj >= T);
           float p = valid ? tc::ex2(s[nt][e] * sl2 - Ls[cur][col]) : 0.f;
-          float f = 1.f;  // the forward multiplied v by P f: dV takes P f, dP takes f
-          if (drop.on && valid)
-            f = drop_factor(drop, (((uint64_t)b * H + hq) * T + qi) * T + kj, dstep);
-          s[nt][e] = p * f;                                // (P f)^T
-          dp[nt][e] = p * (dp[nt][e] * f - Ds[cur][col]);  // dS^T
+          s[nt][e] = p * f[e];                                // (P f)^T
+          dp[nt][e] = p * (dp[nt][e] * f[e] - Ds[cur][col]);  // dS^T
         }
       }
       uint32_t pf[2][4], sf[2][4];

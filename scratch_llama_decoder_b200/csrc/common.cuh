@@ -66,10 +66,17 @@ LLM_DEV void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
     k0 += W0; k1 += W1;
   }
 }
-// 0 or a.scale for element e of the dropout site a (step: *a.step, read once
-// by the caller).
-LLM_DEV float drop_factor(const llm::DropArgs &a, uint64_t e, uint32_t step) {
-  uint32_t c[4] = {(uint32_t)e, (uint32_t)(e >> 32), a.site, step};
+// Keep bits of the elements 4g .. 4g + 3 of the dropout site a (bit j for
+// element 4g + j): one generator call on counter (g, site, step), element
+// 4g + j kept when output word j is >= a.thr (step: *a.step, read once by the
+// caller).
+LLM_DEV uint32_t drop_bits4(const llm::DropArgs &a, uint64_t g, uint32_t step) {
+  uint32_t c[4] = {(uint32_t)g, (uint32_t)(g >> 32), a.site, step};
   philox4x32_10(c, a.k0, a.k1);
-  return c[0] >= a.thr ? a.scale : 0.f;
+  return (uint32_t)(c[0] >= a.thr) | (uint32_t)(c[1] >= a.thr) << 1 |
+         (uint32_t)(c[2] >= a.thr) << 2 | (uint32_t)(c[3] >= a.thr) << 3;
+}
+// 0 or a.scale for element e of the dropout site a.
+LLM_DEV float drop_factor(const llm::DropArgs &a, uint64_t e, uint32_t step) {
+  return (drop_bits4(a, e >> 2, step) >> (e & 3)) & 1u ? a.scale : 0.f;
 }

@@ -1508,39 +1508,56 @@ void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, floa
 // Hephaistos, Architecture at a glance (Regularization): inverted dropout,
 // masks reused by the backward (the factor of an element is a pure function
 // of its index, the site and the step, so the backward draws it again).
+// A thread takes groups of four consecutive elements, one generator call each.
 __global__ void k_drop_rows(float *__restrict__ x, int64_t n, const DropArgs a) {
   const uint32_t step = (uint32_t)*a.step;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    x[i] *= drop_factor(a, (uint64_t)i, step);
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g * 4 < n;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t keep = drop_bits4(a, (uint64_t)g, step);
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+      if (g * 4 + j < n) x[g * 4 + j] *= (keep >> j) & 1u ? a.scale : 0.f;
+  }
 }
 __global__ void k_drop_add(const float *__restrict__ x, const float *__restrict__ y,
                            float *__restrict__ out, int64_t n, const DropArgs a) {
   const uint32_t step = (uint32_t)*a.step;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    out[i] = x[i] + drop_factor(a, (uint64_t)i, step) * y[i];
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g * 4 < n;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t keep = drop_bits4(a, (uint64_t)g, step);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int64_t i = g * 4 + j;
+      if (i < n) out[i] = x[i] + ((keep >> j) & 1u ? a.scale : 0.f) * y[i];
+    }
+  }
 }
 template <typename A>
 __global__ void k_drop_to_act(const float *__restrict__ dx, A *__restrict__ out, int64_t n,
                               const DropArgs a) {
   const uint32_t step = (uint32_t)*a.step;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    out[i] = from_f<A>(drop_factor(a, (uint64_t)i, step) * dx[i]);
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g * 4 < n;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t keep = drop_bits4(a, (uint64_t)g, step);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int64_t i = g * 4 + j;
+      if (i < n) out[i] = from_f<A>(((keep >> j) & 1u ? a.scale : 0.f) * dx[i]);
+    }
+  }
 }
 void drop_rows(float *x, int64_t n, const DropArgs &a, cudaStream_t s) {
-  k_drop_rows<<<min(cdiv(n, 256), 148u * 16), 256, 0, s>>>(x, n, a);
+  k_drop_rows<<<min(cdiv(cdiv(n, 4), 256), 148u * 16), 256, 0, s>>>(x, n, a);
   count_launch();
 }
 void drop_add(const float *x, const float *y, float *out, int64_t n, const DropArgs &a,
               cudaStream_t s) {
-  k_drop_add<<<min(cdiv(n, 256), 148u * 16), 256, 0, s>>>(x, y, out, n, a);
+  k_drop_add<<<min(cdiv(cdiv(n, 4), 256), 148u * 16), 256, 0, s>>>(x, y, out, n, a);
   count_launch();
 }
 void drop_to_act(const float *dx, void *out, DType dt, int64_t n, const DropArgs &a,
                  cudaStream_t s) {
-  const unsigned grid = min(cdiv(n, 256), 148u * 16);
+  const unsigned grid = min(cdiv(cdiv(n, 4), 256), 148u * 16);
   if (dt == DT_BF16) k_drop_to_act<<<grid, 256, 0, s>>>(dx, (__nv_bfloat16 *)out, n, a);
   else k_drop_to_act<<<grid, 256, 0, s>>>(dx, (float *)out, n, a);
   count_launch();

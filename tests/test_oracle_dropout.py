@@ -4,6 +4,9 @@ drawn by the training forward and reused by its backward) and of its mask
 generator, Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC 2011):
 
 - the generator against the published known-answer vectors of Philox4x32-10;
+- the mask of element e is output word e mod 4 of one generator call on the
+  group counter (e / 4, site + 4 layer, step): four elements per call, also
+  past 2^32 groups, and the four words of a group are independent;
 - mask statistics (drop fraction p, unit mean of the inverted factors),
   reproducibility and independence across steps, sites and layers;
 - p = 0 reduces to the training step without dropout;
@@ -60,6 +63,31 @@ def test_mask_statistics_and_independence():
         assert abs(agree - expect) < 0.01, (args, agree)
     # p = 0 keeps everything with factor 1
     np.testing.assert_array_equal(O.dropout_factors(0.0, SEED, STEP, 1, 0, 1000), np.ones(1000))
+
+
+def test_mask_words_are_one_generator_call_per_four_elements():
+    thr = int(np.floor(P_DROP * 2.0 ** 32))
+    key = (SEED & 0xffffffff, SEED >> 32)
+    site, layer = 1, 2
+    for e0 in (0, 4 * 1000 + 2, (1 << 34) + 4 * 5 + 1):  # ragged starts; group high word 1
+        n = 14
+        f = O.dropout_factors(P_DROP, SEED, STEP, site, layer, n, e0=e0)
+        for i in range(n):
+            e = e0 + i
+            g = e // 4
+            words = O.philox4x32_10((g & 0xffffffff, g >> 32, site + 4 * layer, STEP), key)
+            want = 1.0 / (1.0 - P_DROP) if words[e % 4] >= thr else 0.0
+            assert f[i] == want, (e, f[i], want)
+    # the four words of a group are independent: within-group pairs agree as
+    # often as independent draws
+    n = 400_000
+    kept = (O.dropout_factors(P_DROP, SEED, STEP, 3, 0, n) > 0).reshape(-1, 4)
+    expect = P_DROP ** 2 + (1 - P_DROP) ** 2
+    sd = np.sqrt(expect * (1 - expect) / kept.shape[0])
+    for j in range(4):
+        assert abs((1 - kept[:, j].mean()) - P_DROP) < 5 * np.sqrt(P_DROP * (1 - P_DROP) / kept.shape[0])
+        for k in range(j + 1, 4):
+            assert abs((kept[:, j] == kept[:, k]).mean() - expect) < 5 * sd, (j, k)
 
 
 def test_zero_rate_is_the_plain_step():
