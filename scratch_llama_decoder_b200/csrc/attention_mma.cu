@@ -229,13 +229,13 @@ LLM_DEV void drop_k_tile(const DropArgs &drop, uint64_t hrow, int T, int kr0, in
 }
 
 // ------------------------------------------------------------------ forward
-template <int HD>
+template <int HD, bool DROP>
 __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict__ qkv,
                                                  __nv_bfloat16 *__restrict__ o,
                                                  float *__restrict__ lse, int T, int H, int Hkv,
                                                  float scale, const DropArgs drop) {
   __shared__ Tile<HD> Qs, Ks[2], Vs[2];
-  const uint32_t dstep = drop.on ? (uint32_t)*drop.step : 0u;
+  const uint32_t dstep = DROP ? (uint32_t)*drop.step : 0u;
   // grid (H, B, query blocks): blocks are dispatched x-fastest, so the last
   // (longest) query blocks of every head start first
   const int nqb = gridDim.z;
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
         acc[i][2 * r + 1] *= corr;
       }
     }
-    if (drop.on) {  // P V with the dropped probabilities P f; l keeps P's sums
+    if constexpr (DROP) {  // P V with the dropped probabilities P f; l keeps P's sums
       const uint64_t hrow = ((uint64_t)b * H + h) * T;
 #pragma unroll
       for (int nt = 0; nt < 8; nt++) {
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(NT) k_attn_fwd(const __nv_bfloat16 *__restrict
 }
 
 // ---------------------------------------------------------------- backward
-template <int HD>
+template <int HD, bool DROP>
 __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict__ qkv,
                                                 const __nv_bfloat16 *__restrict__ o,
                                                 const __nv_bfloat16 *__restrict__ dout,
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
                                                 int Hkv, float scale, const DropArgs drop) {
   __shared__ Tile<HD> Ks[2], Vs[2];
   __shared__ float Dsh[64];
-  const uint32_t dstep = drop.on ? (uint32_t)*drop.step : 0u;
+  const uint32_t dstep = DROP ? (uint32_t)*drop.step : 0u;
   const int nqb = gridDim.z;
   const int qb = nqb - 1 - blockIdx.z;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
 #pragma unroll
     for (int nt = 0; nt < 8; nt++) {
       float f[4];
-      if (drop.on)
+      if constexpr (DROP)
         drop_q_tile(drop, ((uint64_t)b * H + h) * T, T, q0 + w * 16, k0 + nt * 8, lane, dstep, f);
 #pragma unroll
       for (int e = 0; e < 4; e++) {
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
         float p = valid ? tc::ex2(s[nt][e] * sl2 - L2[r]) : 0.f;
         float dpv = dp[nt][e];
         // with dropout dP = f (dO . v), the forward having multiplied v by P f
-        if (drop.on) dpv *= f[e];
+        if constexpr (DROP) dpv *= f[e];
         s[nt][e] = p * (dpv - Dr[r]);  // dS
       }
     }
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(NT) k_attn_dq(const __nv_bfloat16 *__restrict_
   }
 }
 
-template <int HD>
+template <int HD, bool DROP>
 __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict__ qkv,
                                                  const __nv_bfloat16 *__restrict__ dout,
                                                  const float *__restrict__ lse,
@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
                                                  const float *__restrict__ sin_t, int T, int H,
                                                  int Hkv, float scale, const DropArgs drop) {
   __shared__ Tile<HD> KVs, Qs[2], dOs[2];
-  const uint32_t dstep = drop.on ? (uint32_t)*drop.step : 0u;
+  const uint32_t dstep = DROP ? (uint32_t)*drop.step : 0u;
   __shared__ float Ls[2][64], Ds[2][64];
   // grid (Hkv, B, key blocks): the first key blocks see the most query
   // blocks, and blocks are dispatched x-fastest, so they start first
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(NT) k_attn_dkv(const __nv_bfloat16 *__restrict
       for (int nt = 0; nt < 4; nt++) {
         // the forward multiplied v by P f: dV takes P f, dP takes f
         float f[4] = {1.f, 1.f, 1.f, 1.f};
-        if (drop.on)
+        if constexpr (DROP)
           drop_k_tile(drop, ((uint64_t)b * H + hq) * T, T, k0 + w * 16, q0 + hf * 32 + nt * 8,
                       lane, dstep, f);
 #pragma unroll
@@ -604,12 +604,12 @@ void attn_fwd_mma(const void *qkv, void *o, float *lse, int B, int T, int H, int
   using namespace attn;
   dim3 grid(H, B, (T + BQ - 1) / BQ);
   float scale = 1.0f / sqrtf((float)hd);
-  if (hd == 64)
-    k_attn_fwd<64><<<grid, NT, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, T, H,
-                                       Hkv, scale, drop);
-  else
-    k_attn_fwd<32><<<grid, NT, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, T, H,
-                                       Hkv, scale, drop);
+  auto launch = [&](auto kern) {
+    kern<<<grid, NT, 0, s>>>((const __nv_bfloat16 *)qkv, (__nv_bfloat16 *)o, lse, T, H, Hkv, scale,
+                             drop);
+  };
+  if (hd == 64) drop.on ? launch(k_attn_fwd<64, true>) : launch(k_attn_fwd<64, false>);
+  else drop.on ? launch(k_attn_fwd<32, true>) : launch(k_attn_fwd<32, false>);
   count_launch();
 }
 
@@ -622,13 +622,16 @@ void attn_bwd_mma(const void *qkv, const void *o, const void *dout, const float 
                       *dO = (const __nv_bfloat16 *)dout;
   __nv_bfloat16 *dq = (__nv_bfloat16 *)dqkv;
   dim3 gq(H, B, (T + BQ - 1) / BQ), gkv(Hkv, B, (T + BKV - 1) / BKV);
-  if (hd == 64) {
-    k_attn_dq<64><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
-    k_attn_dkv<64><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
-  } else {
-    k_attn_dq<32><<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
-    k_attn_dkv<32><<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
-  }
+  auto launch = [&](auto kdq, auto kdkv) {
+    kdq<<<gq, NT, 0, s>>>(q, oo, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
+    kdkv<<<gkv, NT, 0, s>>>(q, dO, lse, Dbuf, dq, cos_t, sin_t, T, H, Hkv, scale, drop);
+  };
+  if (hd == 64)
+    drop.on ? launch(k_attn_dq<64, true>, k_attn_dkv<64, true>)
+            : launch(k_attn_dq<64, false>, k_attn_dkv<64, false>);
+  else
+    drop.on ? launch(k_attn_dq<32, true>, k_attn_dkv<32, true>)
+            : launch(k_attn_dq<32, false>, k_attn_dkv<32, false>);
   count_launch(2);
 }
 

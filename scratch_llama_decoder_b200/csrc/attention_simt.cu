@@ -290,16 +290,33 @@ LLM_DEV float half_sum(float v) {
   return v;
 }
 
+// Dropout factors of the keys key0 .. key0 + 3 (key0 % 4 == 0) of query q,
+// element (hrow + q) T + key of the probability site: one generator group
+// when T % 4 == 0, else one group per element.
+LLM_DEV void drop_keys4(const DropArgs &drop, uint64_t hrow, int T, int q, int key0,
+                        uint32_t step, float (&f)[4]) {
+  const uint64_t e0 = (hrow + q) * (uint64_t)T + key0;
+  if ((T & 3) == 0) {
+    const uint32_t keep = drop_bits4(drop, e0 >> 2, step);
+#pragma unroll
+    for (int j = 0; j < 4; j++) f[j] = (keep >> j) & 1u ? drop.scale : 0.f;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; j++) f[j] = drop_factor(drop, e0 + j, step);
+  }
+}
+
 // Forward: grid (query tiles, B*H), last query tiles first.
-template <int HD>
+template <int HD, bool DROP>
 __global__ void __launch_bounds__(TNT) k_attn_fwd_tile(const float *__restrict__ qkv,
                                                         float *__restrict__ o,
                                                         float *__restrict__ lse, int T, int H,
-                                                        int Hkv) {
+                                                        int Hkv, const DropArgs drop) {
   constexpr int CW = HD / 16;
   extern __shared__ float4 sm4[];
   float *Qt = reinterpret_cast<float *>(sm4), *Kt = Qt + HD * TLD, *Vs = Kt + HD * TLD,
         *Pt = Vs + TB * HD;
+  const uint32_t dstep = DROP ? (uint32_t)*drop.step : 0u;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int qb = gridDim.x - 1 - blockIdx.x, b = blockIdx.y / H, h = blockIdx.y % H;
   const int g = h / (H / Hkv), d = H * HD, kvd = Hkv * HD;
@@ -355,6 +372,15 @@ __global__ void __launch_bounds__(TNT) k_attn_fwd_tile(const float *__restrict__
 #pragma unroll
       for (int c = 0; c < CW; c++) acc[r][c] *= corr;
     }
+    if constexpr (DROP) {  // P V with the dropped probabilities P f; the sums lp keep P's
+#pragma unroll
+      for (int r = 0; r < 4; r++) {
+        float f[4];
+        drop_keys4(drop, ((uint64_t)b * H + h) * T, T, q0 + ty * 4 + r, k0 + tx * 4, dstep, f);
+#pragma unroll
+        for (int c = 0; c < 4; c++) pt[c][r] *= f[c];
+      }
+    }
 #pragma unroll
     for (int c = 0; c < 4; c++)
       *reinterpret_cast<float4 *>(Pt + pslot(tx * 4 + c, ty)) =
@@ -376,15 +402,16 @@ __global__ void __launch_bounds__(TNT) k_attn_fwd_tile(const float *__restrict__
 }
 
 // dQ (and D = rowsum(dO o O) into Dbuf): grid (query tiles, B*H).
-template <int HD>
+template <int HD, bool DROP>
 __global__ void __launch_bounds__(TNT) k_attn_dq_tile(const float *__restrict__ qkv,
                                                        const float *__restrict__ o,
                                                        const float *__restrict__ dout,
                                                        const float *__restrict__ lse,
                                                        float *__restrict__ Dbuf,
                                                        float *__restrict__ dqkv, int T, int H,
-                                                       int Hkv) {
+                                                       int Hkv, const DropArgs drop) {
   constexpr int CW = HD / 16;
+  const uint32_t dstep = DROP ? (uint32_t)*drop.step : 0u;
   extern __shared__ float4 sm4[];
   float *Qt = reinterpret_cast<float *>(sm4), *dOt = Qt + HD * TLD, *Kt = dOt + HD * TLD,
         *Vt = Kt + HD * TLD, *Kr = Vt + HD * TLD, *dSt = Kr + TB * HD;
@@ -428,14 +455,19 @@ __global__ void __launch_bounds__(TNT) k_attn_dq_tile(const float *__restrict__ 
     tile_dot<HD>(dOt, Vt, tx, ty, dp);
     float ds[4][4];
 #pragma unroll
-    for (int r = 0; r < 4; r++)
+    for (int r = 0; r < 4; r++) {
+      // with dropout dP = f (dO . v), the forward having multiplied v by P f
+      float f[4] = {1.f, 1.f, 1.f, 1.f};
+      if constexpr (DROP)
+        drop_keys4(drop, ((uint64_t)b * H + h) * T, T, q0 + ty * 4 + r, k0 + tx * 4, dstep, f);
 #pragma unroll
       for (int c = 0; c < 4; c++) {
         const int key = k0 + tx * 4 + c;
         const bool masked = kb == qb && (key > q0 + ty * 4 + r || key >= T);
         const float p = masked ? 0.f : expf(sv[r][c] - Lr[r]);
-        ds[c][r] = p * (dp[r][c] - Dr[r]);
+        ds[c][r] = p * (dp[r][c] * f[c] - Dr[r]);
       }
+    }
 #pragma unroll
     for (int c = 0; c < 4; c++)
       *reinterpret_cast<float4 *>(dSt + pslot(tx * 4 + c, ty)) =
@@ -456,14 +488,15 @@ __global__ void __launch_bounds__(TNT) k_attn_dq_tile(const float *__restrict__ 
 
 // dK, dV: grid (key tiles, B*Hkv), first key tiles first; steps over the
 // group's query heads and the query tiles at or after the key tile.
-template <int HD>
+template <int HD, bool DROP>
 __global__ void __launch_bounds__(TNT) k_attn_dkv_tile(const float *__restrict__ qkv,
                                                         const float *__restrict__ dout,
                                                         const float *__restrict__ lse,
                                                         const float *__restrict__ Dbuf,
                                                         float *__restrict__ dqkv, int T, int H,
-                                                        int Hkv) {
+                                                        int Hkv, const DropArgs drop) {
   constexpr int CW = HD / 16;
+  const uint32_t dstep = DROP ? (uint32_t)*drop.step : 0u;
   extern __shared__ float4 sm4[];
   float *Kt = reinterpret_cast<float *>(sm4), *Vt = Kt + HD * TLD, *Qt = Vt + HD * TLD,
         *dOt = Qt + HD * TLD, *Qr = dOt + HD * TLD, *dOr = Qr + TB * HD, *Ps = dOr + TB * HD,
@@ -497,6 +530,17 @@ __global__ void __launch_bounds__(TNT) k_attn_dkv_tile(const float *__restrict__
       float sv[4][4] = {}, dp[4][4] = {};
       tile_dot<HD>(Kt, Qt, tx, ty, sv);  // S^T: rows keys, columns queries
       tile_dot<HD>(Vt, dOt, tx, ty, dp);
+      // the forward multiplied v by P f: dV takes P f, dP takes f (fk[c][r]:
+      // query q0 + 4 tx + c, key k0 + 4 ty + r)
+      float fk[4][4];
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        if constexpr (DROP)
+          drop_keys4(drop, ((uint64_t)b * H + hq) * T, T, q0 + tx * 4 + c, k0 + ty * 4, dstep,
+                     fk[c]);
+        else
+          fk[c][0] = fk[c][1] = fk[c][2] = fk[c][3] = 1.f;
+      }
       float pq[4][4], dq[4][4];
 #pragma unroll
       for (int r = 0; r < 4; r++)
@@ -505,8 +549,8 @@ __global__ void __launch_bounds__(TNT) k_attn_dkv_tile(const float *__restrict__
           const int key = k0 + ty * 4 + r, q = q0 + tx * 4 + c;
           const bool masked = qb == kb && key > q;
           const float p = masked ? 0.f : expf(sv[r][c] - sL[tx * 4 + c]);
-          pq[c][r] = p;
-          dq[c][r] = p * (dp[r][c] - sD[tx * 4 + c]);
+          pq[c][r] = p * fk[c][r];
+          dq[c][r] = p * (dp[r][c] * fk[c][r] - sD[tx * 4 + c]);
         }
 #pragma unroll
       for (int c = 0; c < 4; c++) {
@@ -540,50 +584,52 @@ template <int HD> constexpr int dq_tile_smem() { return (4 * HD * TLD + TB * HD 
 template <int HD>
 constexpr int dkv_tile_smem() { return (4 * HD * TLD + 2 * TB * HD + 2 * TB * TB + 2 * TB) * 4; }
 
-// The tiled float32 path: head size 32 or 64, no dropout, 16-byte aligned
+// The tiled float32 path: head size 32 or 64, 16-byte aligned
 // rows (every row stride a multiple of 4 floats).
-static bool tile_covers(DType dt, int hd, const DropArgs &drop) {
-  return dt == DT_F32 && (hd == 32 || hd == 64) && !drop.on;
-}
+static bool tile_covers(DType dt, int hd) { return dt == DT_F32 && (hd == 32 || hd == 64); }
 bool attn_tile_covers(int hd) { return hd == 32 || hd == 64; }
 template <int HD>
 static bool attn_fwd_tile(const float *qkv, float *o, float *lse, int B, int T, int H, int Hkv,
-                          cudaStream_t s) {
-  if (!smem_optin((const void *)k_attn_fwd_tile<HD>, fwd_tile_smem<HD>())) return false;
-  k_attn_fwd_tile<HD><<<dim3((T + TB - 1) / TB, B * H), TNT, fwd_tile_smem<HD>(), s>>>(
-      qkv, o, lse, T, H, Hkv);
+                          cudaStream_t s, const DropArgs &drop) {
+  auto kern = drop.on ? k_attn_fwd_tile<HD, true> : k_attn_fwd_tile<HD, false>;
+  if (!smem_optin((const void *)kern, fwd_tile_smem<HD>())) return false;
+  kern<<<dim3((T + TB - 1) / TB, B * H), TNT, fwd_tile_smem<HD>(), s>>>(qkv, o, lse, T, H, Hkv,
+                                                                      drop);
   count_launch();
   return true;
 }
 template <int HD>
 static bool attn_bwd_tile(const float *qkv, const float *o, const float *dout, const float *lse,
-                          float *Dbuf, float *dqkv, int B, int T, int H, int Hkv, cudaStream_t s) {
-  if (!smem_optin((const void *)k_attn_dq_tile<HD>, dq_tile_smem<HD>()) ||
-      !smem_optin((const void *)k_attn_dkv_tile<HD>, dkv_tile_smem<HD>()))
+                          float *Dbuf, float *dqkv, int B, int T, int H, int Hkv, cudaStream_t s,
+                          const DropArgs &drop) {
+  auto kdq = drop.on ? k_attn_dq_tile<HD, true> : k_attn_dq_tile<HD, false>;
+  auto kdkv = drop.on ? k_attn_dkv_tile<HD, true> : k_attn_dkv_tile<HD, false>;
+  if (!smem_optin((const void *)kdq, dq_tile_smem<HD>()) ||
+      !smem_optin((const void *)kdkv, dkv_tile_smem<HD>()))
     return false;
   const int nt = (T + TB - 1) / TB;
-  k_attn_dq_tile<HD><<<dim3(nt, B * H), TNT, dq_tile_smem<HD>(), s>>>(qkv, o, dout, lse, Dbuf,
-                                                                      dqkv, T, H, Hkv);
-  k_attn_dkv_tile<HD><<<dim3(nt, B * Hkv), TNT, dkv_tile_smem<HD>(), s>>>(qkv, dout, lse, Dbuf,
-                                                                          dqkv, T, H, Hkv);
+  kdq<<<dim3(nt, B * H), TNT, dq_tile_smem<HD>(), s>>>(qkv, o, dout, lse, Dbuf, dqkv, T, H, Hkv,
+                                                       drop);
+  kdkv<<<dim3(nt, B * Hkv), TNT, dkv_tile_smem<HD>(), s>>>(qkv, dout, lse, Dbuf, dqkv, T, H, Hkv,
+                                                           drop);
   count_launch(2);
   return true;
 }
 
 bool attn_fwd_f32_tiled(const float *qkv, float *o, float *lse, int B, int T, int H, int Hkv,
-                        int hd, cudaStream_t s) {
+                        int hd, cudaStream_t s, DropArgs drop) {
   if (!attn_tile_covers(hd)) return false;
-  return hd == 32 ? attn_fwd_tile<32>(qkv, o, lse, B, T, H, Hkv, s)
-                  : attn_fwd_tile<64>(qkv, o, lse, B, T, H, Hkv, s);
+  return hd == 32 ? attn_fwd_tile<32>(qkv, o, lse, B, T, H, Hkv, s, drop)
+                  : attn_fwd_tile<64>(qkv, o, lse, B, T, H, Hkv, s, drop);
 }
 bool attn_bwd_f32_tiled(const float *qkv, const float *o, const float *dout, const float *lse,
                         float *Dbuf, float *dqkv, int B, int T, int H, int Hkv, int hd,
-                        cudaStream_t s) {
+                        cudaStream_t s, DropArgs drop) {
   if (!attn_tile_covers(hd)) return false;
-  return hd == 32 ? attn_bwd_tile<32>(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, s)
-                  : attn_bwd_tile<64>(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, s);
+  return hd == 32 ? attn_bwd_tile<32>(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, s, drop)
+                  : attn_bwd_tile<64>(qkv, o, dout, lse, Dbuf, dqkv, B, T, H, Hkv, s, drop);
 }
-// The one-warp-per-row kernels alone (any head size, dropout).
+// The one-warp-per-row kernels alone (any head size).
 void attn_fwd_rows(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
                    int hd, cudaStream_t s, DropArgs drop);
 void attn_bwd_rows(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
@@ -592,17 +638,17 @@ void attn_bwd_rows(const void *qkv, const void *o, const void *dout, const float
 
 void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
                    int hd, cudaStream_t s, DropArgs drop) {
-  if (tile_covers(dt, hd, drop) &&
-      attn_fwd_f32_tiled((const float *)qkv, (float *)o, lse, B, T, H, Hkv, hd, s))
+  if (tile_covers(dt, hd) &&
+      attn_fwd_f32_tiled((const float *)qkv, (float *)o, lse, B, T, H, Hkv, hd, s, drop))
     return;
   attn_fwd_rows(qkv, o, lse, dt, B, T, H, Hkv, hd, s, drop);
 }
 void attn_bwd_simt(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,
                    void *dqkv, DType dt, int B, int T, int H, int Hkv, int hd, cudaStream_t s,
                    DropArgs drop) {
-  if (tile_covers(dt, hd, drop) &&
+  if (tile_covers(dt, hd) &&
       attn_bwd_f32_tiled((const float *)qkv, (const float *)o, (const float *)dout, lse, Dbuf,
-                         (float *)dqkv, B, T, H, Hkv, hd, s))
+                         (float *)dqkv, B, T, H, Hkv, hd, s, drop))
     return;
   attn_bwd_rows(qkv, o, dout, lse, Dbuf, dqkv, dt, B, T, H, Hkv, hd, s, drop);
 }

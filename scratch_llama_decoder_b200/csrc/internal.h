@@ -139,10 +139,10 @@ void attn_fwd_simt(const void *qkv, void *o, float *lse, DType dt, int B, int T,
 // float32 tiled kernels (head size 32 or 64; false otherwise) and the
 // one-warp-per-row kernels alone.
 bool attn_fwd_f32_tiled(const float *qkv, float *o, float *lse, int B, int T, int H, int Hkv,
-                        int hd, cudaStream_t s);
+                        int hd, cudaStream_t s, DropArgs drop = DropArgs{});
 bool attn_bwd_f32_tiled(const float *qkv, const float *o, const float *dout, const float *lse,
                         float *Dbuf, float *dqkv, int B, int T, int H, int Hkv, int hd,
-                        cudaStream_t s);
+                        cudaStream_t s, DropArgs drop = DropArgs{});
 void attn_fwd_rows(const void *qkv, void *o, float *lse, DType dt, int B, int T, int H, int Hkv,
                    int hd, cudaStream_t s, DropArgs drop);
 void attn_bwd_rows(const void *qkv, const void *o, const void *dout, const float *lse, float *Dbuf,

@@ -776,6 +776,7 @@ void layer_fwd(llm_ctx *c, const float *p, int l, int sl, bool drop, bool out) {
       KTimer kt(c, LLM_KT_ATTN_FWD, attn_flops(D, 4.0));
       attn_fwd_mma(qkv, o, lse, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
     } else {
+      KTimer kt(c, LLM_KT_ATTN_FWD, attn_flops(D, 4.0));
       attn_fwd_simt(qkv, o, lse, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s, drop_args(c, 1, l));
     }
     gemm(c, GemmOperands{(int)N, D.d, D.d, o, d, true, wo, d, false, D.dt}, OUT_F32, c->dtmp, d,
@@ -972,8 +973,11 @@ void backward(llm_ctx *c, const float *p, float *gr, const int32_t *tok, bool bu
       attn_bwd_mma(qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.B, D.T, D.H, D.Hkv, D.hd, c->cos_t,
                    c->sin_t, s, drop_args(c, 1, l));
     } else if (drop) {  // the same probability masks, then RoPE backward on dq, dk
-      attn_bwd_simt(qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s,
-                    drop_args(c, 1, l));
+      {
+        KTimer kt(c, LLM_KT_ATTN_BWD, attn_flops(D, 8.0));
+        attn_bwd_simt(qkv, o, c->dO, lse, c->Dbuf, c->dqkv, D.dt, D.B, D.T, D.H, D.Hkv, D.hd, s,
+                      drop_args(c, 1, l));
+      }
       rope_apply(c->dqkv, D.dt, c->cos_t, c->sin_t, N, D.T, D.d + D.kvd, D.qkvw, D.hd, -1, s);
     } else {
       KTimer kt(c, LLM_KT_ATTN_BWD, attn_flops(D, 8.0));

@@ -31,7 +31,11 @@ def _setup(cfg, stream=None):
                                        ("c4", dict(batch=1, ctx=96, n_layer=2)),
                                        # several 64-row tiles with ragged tails (head 32, head 64 GQA)
                                        ("c3", dict(batch=1, ctx=130, n_layer=1)),
-                                       ("c4", dict(batch=1, ctx=200, n_layer=1))])
+                                       ("c4", dict(batch=1, ctx=200, n_layer=1)),
+                                       # the tiled fp32 kernels: T % 4 == 0 (a mask group
+                                       # per 4 keys) and T % 4 != 0 (a group per element)
+                                       ("c2", dict(batch=2, ctx=68, n_layer=2)),
+                                       ("c2", dict(batch=1, ctx=131, n_layer=1))])
 def test_dropout_grads_match_oracle(name, over):
     cfg = get_config(name, **over)
     lay, p, tok, tgt, m = _setup(cfg)
