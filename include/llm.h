@@ -368,15 +368,19 @@ int llm_set_rope_scale(llm_ctx *ctx, float factor);
  * of the embedding output [B*T, d], the attention probabilities [B, H, T, T],
  * and the attention and MLP branch outputs [B*T, d] (before their residual
  * adds) is kept with probability 1 - p and scaled by 1 / (1 - p).  The masks
- * come from Philox4x32-10 (Salmon et al., SC 2011): key = the seed's two
- * 32-bit halves, counter = (element index low word, high word, site + 4 *
- * layer, n) with sites 0 embedding, 1 attention probabilities, 2 attention
- * output, 3 MLP output, element indices row-major over those shapes, n = the
- * number of training calls (llm_step or llm_grad) since the last
- * llm_set_dropout; an element is kept when the first output word is >=
- * floor(p * 2^32).  llm_forward and llm_decode never drop.  While dropout is
- * on, attention runs in the CUDA-core kernels (the tensor-core kernels draw no
- * masks).  p = 0 turns it off (the default).  A changed setting frees the
+ * come from Philox4x32-10 (Salmon et al., SC 2011), one call per group of
+ * four consecutive elements: key = the seed's two 32-bit halves, counter =
+ * (group index low word, high word, site + 4 * layer, n), group index =
+ * element index / 4, with sites 0 embedding, 1 attention probabilities,
+ * 2 attention output, 3 MLP output, element indices row-major over those
+ * shapes, n = the number of training calls (llm_step or llm_grad) since the
+ * last llm_set_dropout; element e is kept when output word e mod 4 of its
+ * group's call is >= floor(p * 2^32).  llm_forward and llm_decode never drop.
+ * While dropout is on, bf16 attention with head size 32 or 64 runs in the
+ * mma.sync kernels and fp32 attention with those head sizes in the tiled
+ * CUDA-core kernels, both drawing the masks inside; other head sizes use the
+ * one-warp-per-row kernels (the tcgen05 kernels draw no masks).  p = 0 turns
+ * it off (the default).  A changed setting frees the
  * captured step graph; every call restarts n at 0.  LLM_ERR_ARG unless
  * 0 <= p < 1. */
 int llm_set_dropout(llm_ctx *ctx, float p, uint64_t seed);
