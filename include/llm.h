@@ -394,6 +394,16 @@ int llm_set_dropout(llm_ctx *ctx, float p, uint64_t seed);
 int llm_get_dropout_calls(llm_ctx *ctx, int64_t *n);
 int llm_set_dropout_calls(llm_ctx *ctx, int64_t n);
 
+/* The index b0 of the context's first sequence in the whole batch of a
+ * data-parallel step (default 0).  The masks of llm_set_dropout are indexed
+ * over the whole batch: the context's sequence b draws those of sequence
+ * b0 + b, so ranks whose contexts hold consecutive shares of the batch
+ * (b0 = rank * batch) draw together the masks of one context over the whole
+ * batch, and no two ranks draw the same ones.  A changed offset frees the
+ * captured step graph.  LLM_ERR_ARG for a null pointer, b0 outside
+ * [0, 2^31), or a context whose device is not current. */
+int llm_set_dropout_offset(llm_ctx *ctx, int64_t b0);
+
 /* The norm clipping uses: LLM_CLIP_L2, the Euclidean norm of the whole
  * gradient (the default), or LLM_CLIP_LINF, its largest absolute element
  * (randyGPT, Training: gradient clipping by the L-infinity norm at 1.0); the

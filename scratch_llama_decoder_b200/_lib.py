@@ -81,6 +81,7 @@ EXPORTS = {
     "llm_set_grad_buckets": (_i, [_vp, _i]),
     "llm_get_dropout_calls": (_i, [_vp, C.POINTER(_i64)]),
     "llm_set_dropout_calls": (_i, [_vp, _i64]),
+    "llm_set_dropout_offset": (_i, [_vp, _i64]),
     "llm_grad_bucket_wait": (_i, [_vp, _i, _vp]),
     "llm_decode": (_i, [_vp, _vp, _vp, _i, _vp]),
     "llm_sample": (_i, [_vp, _vp, _i64, _i, _f, _i, _vp, _vp]),

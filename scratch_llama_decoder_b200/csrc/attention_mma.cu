@@ -174,7 +174,8 @@ LLM_DEV void rope_bwd_row(float (&acc)[HD / 8][4], int r, const float *ct, const
 // ------------------------------------------------------------------ dropout
 // Factors of the probabilities (element (hrow + i) T + j of the site, hrow =
 // (b H + h) T) a thread holds in one 8-column tile of a warp's 16-row tile.
-// With T % 4 == 0 the keys 4m .. 4m + 3 of a query are one generator group,
+// With T % 4 == 0 the keys 4m .. 4m + 3 of a query are one generator group
+// (the context's offset drop.e0, a multiple of H T^2, keeps them aligned),
 // so the warp's 32 groups of the tile are drawn once each, one per lane, and
 // the keep bits go to their holders by shuffles; otherwise every element
 // draws its own group.
@@ -188,7 +189,7 @@ LLM_DEV void drop_q_tile(const DropArgs &drop, uint64_t hrow, int T, int r0, int
                          uint32_t step, float (&f)[4]) {
   if ((T & 3) == 0) {
     const int rx = r0 + (lane >> 2) + (lane & 1) * 8, kx = k8 + ((lane >> 1) & 1) * 4;
-    const uint32_t mine = drop_bits4(drop, ((hrow + rx) * (uint64_t)T + kx) >> 2, step);
+    const uint32_t mine = drop_bits4(drop, (drop.e0 + (hrow + rx) * (uint64_t)T + kx) >> 2, step);
     const uint32_t lo = __shfl_sync(0xffffffffu, mine, lane & ~1);
     const uint32_t hi = __shfl_sync(0xffffffffu, mine, lane | 1);
     const int sh = (lane & 1) * 2;
@@ -212,7 +213,7 @@ LLM_DEV void drop_k_tile(const DropArgs &drop, uint64_t hrow, int T, int kr0, in
                          uint32_t step, float (&f)[4]) {
   if ((T & 3) == 0) {
     const int qx = q8 + (lane >> 2), kx = kr0 + (lane & 3) * 4;
-    const uint32_t mine = drop_bits4(drop, ((hrow + qx) * (uint64_t)T + kx) >> 2, step);
+    const uint32_t mine = drop_bits4(drop, (drop.e0 + (hrow + qx) * (uint64_t)T + kx) >> 2, step);
     const int sh = (lane >> 2) & 3;
 #pragma unroll
     for (int e = 0; e < 4; e++) {

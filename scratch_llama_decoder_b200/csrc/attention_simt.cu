@@ -295,14 +295,14 @@ LLM_DEV float half_sum(float v) {
 // when T % 4 == 0, else one group per element.
 LLM_DEV void drop_keys4(const DropArgs &drop, uint64_t hrow, int T, int q, int key0,
                         uint32_t step, float (&f)[4]) {
-  const uint64_t e0 = (hrow + q) * (uint64_t)T + key0;
-  if ((T & 3) == 0) {
-    const uint32_t keep = drop_bits4(drop, e0 >> 2, step);
+  const uint64_t e = (hrow + q) * (uint64_t)T + key0;
+  if ((T & 3) == 0) {  // drop.e0, a multiple of H T^2, keeps the group aligned
+    const uint32_t keep = drop_bits4(drop, (drop.e0 + e) >> 2, step);
 #pragma unroll
     for (int j = 0; j < 4; j++) f[j] = (keep >> j) & 1u ? drop.scale : 0.f;
   } else {
 #pragma unroll
-    for (int j = 0; j < 4; j++) f[j] = drop_factor(drop, e0 + j, step);
+    for (int j = 0; j < 4; j++) f[j] = drop_factor(drop, e + j, step);
   }
 }
 

@@ -76,7 +76,9 @@ LLM_DEV uint32_t drop_bits4(const llm::DropArgs &a, uint64_t g, uint32_t step) {
   return (uint32_t)(c[0] >= a.thr) | (uint32_t)(c[1] >= a.thr) << 1 |
          (uint32_t)(c[2] >= a.thr) << 2 | (uint32_t)(c[3] >= a.thr) << 3;
 }
-// 0 or a.scale for element e of the dropout site a.
+// 0 or a.scale for element e of the context's part of the dropout site a
+// (whole-batch element a.e0 + e).
 LLM_DEV float drop_factor(const llm::DropArgs &a, uint64_t e, uint32_t step) {
-  return (drop_bits4(a, e >> 2, step) >> (e & 3)) & 1u ? a.scale : 0.f;
+  const uint64_t E = a.e0 + e;
+  return (drop_bits4(a, E >> 2, step) >> (E & 3)) & 1u ? a.scale : 0.f;
 }

@@ -22,6 +22,10 @@ struct DropArgs {
   uint32_t thr = 0, k0 = 0, k1 = 0, site = 0;
   float scale = 1.f;
   const int *step = nullptr;  // device word: the training forward's number
+  // index of the context's first element of the site in the whole batch (its
+  // first sequence's offset, llm_set_dropout_offset, times the elements a
+  // sequence has at the site); kernels index masks at e0 + their own index
+  uint64_t e0 = 0;
 };
 
 // ------------------------------------------------------------ GEMM (shared)

@@ -1508,56 +1508,51 @@ void init_params(float *p, int64_t n, uint64_t seed, uint64_t counter_base, floa
 // Hephaistos, Architecture at a glance (Regularization): inverted dropout,
 // masks reused by the backward (the factor of an element is a pure function
 // of its index, the site and the step, so the backward draws it again).
-// A thread takes groups of four consecutive elements, one generator call each.
-__global__ void k_drop_rows(float *__restrict__ x, int64_t n, const DropArgs a) {
+// A thread takes whole-batch groups of four consecutive elements, one
+// generator call each: the context's elements are a.e0 .. a.e0 + n - 1, so
+// group g holds its local elements 4g - a.e0 .. 4g - a.e0 + 3 that lie in
+// [0, n) (a.e0 need not be a multiple of 4).
+template <typename F>
+LLM_DEV void for_drop_groups(const DropArgs &a, int64_t n, F f) {
   const uint32_t step = (uint32_t)*a.step;
-  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g * 4 < n;
-       g += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t keep = drop_bits4(a, (uint64_t)g, step);
+  const uint64_t g0 = a.e0 >> 2;
+  const int64_t ng = (int64_t)(((a.e0 + (uint64_t)n + 3) >> 2) - g0);
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < ng;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const uint64_t g = g0 + (uint64_t)t;
+    const uint32_t keep = drop_bits4(a, g, step);
+    const int64_t i0 = (int64_t)(g * 4) - (int64_t)a.e0;
 #pragma unroll
     for (int j = 0; j < 4; j++)
-      if (g * 4 + j < n) x[g * 4 + j] *= (keep >> j) & 1u ? a.scale : 0.f;
+      if (i0 + j >= 0 && i0 + j < n) f(i0 + j, (keep >> j) & 1u ? a.scale : 0.f);
   }
+}
+__global__ void k_drop_rows(float *__restrict__ x, int64_t n, const DropArgs a) {
+  for_drop_groups(a, n, [&](int64_t i, float fac) { x[i] *= fac; });
 }
 __global__ void k_drop_add(const float *__restrict__ x, const float *__restrict__ y,
                            float *__restrict__ out, int64_t n, const DropArgs a) {
-  const uint32_t step = (uint32_t)*a.step;
-  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g * 4 < n;
-       g += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t keep = drop_bits4(a, (uint64_t)g, step);
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const int64_t i = g * 4 + j;
-      if (i < n) out[i] = x[i] + ((keep >> j) & 1u ? a.scale : 0.f) * y[i];
-    }
-  }
+  for_drop_groups(a, n, [&](int64_t i, float fac) { out[i] = x[i] + fac * y[i]; });
 }
 template <typename A>
 __global__ void k_drop_to_act(const float *__restrict__ dx, A *__restrict__ out, int64_t n,
                               const DropArgs a) {
-  const uint32_t step = (uint32_t)*a.step;
-  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g * 4 < n;
-       g += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t keep = drop_bits4(a, (uint64_t)g, step);
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const int64_t i = g * 4 + j;
-      if (i < n) out[i] = from_f<A>(((keep >> j) & 1u ? a.scale : 0.f) * dx[i]);
-    }
-  }
+  for_drop_groups(a, n, [&](int64_t i, float fac) { out[i] = from_f<A>(fac * dx[i]); });
 }
+// groups of the launch: at most n / 4 + 2 (n = 0 still launches one block)
+static unsigned drop_grid(int64_t n) { return min(cdiv(n / 4 + 2, 256), 148u * 16); }
 void drop_rows(float *x, int64_t n, const DropArgs &a, cudaStream_t s) {
-  k_drop_rows<<<min(cdiv(cdiv(n, 4), 256), 148u * 16), 256, 0, s>>>(x, n, a);
+  k_drop_rows<<<drop_grid(n), 256, 0, s>>>(x, n, a);
   count_launch();
 }
 void drop_add(const float *x, const float *y, float *out, int64_t n, const DropArgs &a,
               cudaStream_t s) {
-  k_drop_add<<<min(cdiv(cdiv(n, 4), 256), 148u * 16), 256, 0, s>>>(x, y, out, n, a);
+  k_drop_add<<<drop_grid(n), 256, 0, s>>>(x, y, out, n, a);
   count_launch();
 }
 void drop_to_act(const float *dx, void *out, DType dt, int64_t n, const DropArgs &a,
                  cudaStream_t s) {
-  const unsigned grid = min(cdiv(cdiv(n, 4), 256), 148u * 16);
+  const unsigned grid = drop_grid(n);
   if (dt == DT_BF16) k_drop_to_act<<<grid, 256, 0, s>>>(dx, (__nv_bfloat16 *)out, n, a);
   else k_drop_to_act<<<grid, 256, 0, s>>>(dx, (float *)out, n, a);
   count_launch();

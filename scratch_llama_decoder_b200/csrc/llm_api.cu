@@ -196,6 +196,7 @@ struct llm_ctx {
   uint64_t drop_seed = 0;
   int64_t train_calls = 0;
   int *drop_step = nullptr;
+  int64_t drop_b0 = 0;  // llm_set_dropout_offset: first sequence's index in the whole batch
   // gradient buckets (llm_set_grad_buckets): one event per bucket, recorded by
   // llm_grad's backward on the main stream once the bucket's gradients are final
   std::vector<cudaEvent_t> ev_bucket;
@@ -516,6 +517,22 @@ int llm_set_dropout_calls(llm_ctx *c, int64_t n) {
   return LLM_OK;
 }
 
+int llm_set_dropout_offset(llm_ctx *c, int64_t b0) {
+  if (!c || b0 < 0 || b0 > INT32_MAX) return LLM_ERR_ARG;
+  if (!on_device(c)) return LLM_ERR_ARG;
+  if (b0 != c->drop_b0) {
+    // the offsets are baked into a captured step: drop the graph
+    if (c->gexec) {
+      if (cudaStreamSynchronize(c->s) != cudaSuccess) return LLM_ERR_CUDA;
+      cudaGraphExecDestroy(c->gexec);
+      c->gexec = nullptr;
+    }
+    c->have_prev = false;
+    c->drop_b0 = b0;
+  }
+  return LLM_OK;
+}
+
 int llm_set_grad_clip_mode(llm_ctx *c, int mode) {
   if (!c || (mode != LLM_CLIP_L2 && mode != LLM_CLIP_LINF)) return LLM_ERR_ARG;
   if (!on_device(c)) return LLM_ERR_ARG;
@@ -737,6 +754,10 @@ DropArgs drop_args(const llm_ctx *c, int site, int layer) {
   a.k1 = (uint32_t)(c->drop_seed >> 32);
   a.site = (uint32_t)(site + 4 * layer);
   a.step = c->drop_step;
+  // site 1 is [B, H, T, T], the others [B*T, d]
+  const Dims &D = c->D;
+  a.e0 = (uint64_t)c->drop_b0 *
+         (site == 1 ? (uint64_t)D.H * D.T * D.T : (uint64_t)D.T * D.d);
   return a;
 }
 bool dropping(const llm_ctx *c) { return c->drop_p > 0.f; }

@@ -15,6 +15,10 @@ sequences on every rank) and the same parameters.  A step is:
 The ranks' losses are summed too: the returned tensor holds the sum of the
 ranks' mean losses (divided by the rank count it is the batch mean).
 
+Dropout masks are indexed over the whole batch: the wrapper sets the engine's
+sequence offset to rank * (its batch), so the ranks together draw the masks
+one context over the whole batch would draw, and no two ranks share masks.
+
 The engine is a LlamaStep (or any object with its grad / adamw / flag_out /
 flag_in methods, a device and, for CUDA, a stream); collectives are issued on
 the engine's stream so that they follow its kernels in order.
@@ -40,6 +44,9 @@ class DataParallelStep:
         self.world = (dist.get_world_size(group)
                       if dist.is_available() and dist.is_initialized() else 1)
         self.flag = torch.zeros(1, dtype=torch.int32, device=engine.device)
+        set_offset = getattr(engine, "set_dropout_offset", None)
+        if set_offset is not None and self.world > 1:
+            set_offset(dist.get_rank(group) * int(engine.cfg["batch"]))
         self.overlap = bool(overlap) and self.world > 1
         self._comm = None
         if self.overlap:

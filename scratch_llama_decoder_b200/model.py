@@ -219,6 +219,12 @@ class LlamaStep:
         L.check(L.lib.llm_set_dropout_calls(self.ctx, int(n)), "llm_set_dropout_calls")
 
     @_on_device
+    def set_dropout_offset(self, b0):
+        """Index of this context's first sequence in the whole batch: masks are
+        drawn at whole-batch positions (llm_set_dropout_offset)."""
+        L.check(L.lib.llm_set_dropout_offset(self.ctx, int(b0)), "llm_set_dropout_offset")
+
+    @_on_device
     def set_grad_clip(self, max_norm):
         """Global-norm gradient clipping in later steps (llm_set_grad_clip)."""
         L.check(L.lib.llm_set_grad_clip(self.ctx, float(max_norm)), "llm_set_grad_clip")

@@ -218,6 +218,57 @@ def _two_ranks(full_cfg, steps, fail_rank=-1, fail_at=None, overlap=False):
     return res
 
 
+class OffsetEngine:
+    """Records the dropout sequence offset a wrapper gives it."""
+    device = torch.device("cpu")
+
+    def __init__(self, batch):
+        self.cfg = {"batch": batch}
+        self.drop_b0 = None
+
+    def set_dropout_offset(self, b0):
+        self.drop_b0 = b0
+
+
+def _rank_offsets(rank, world, port, batch, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from scratch_llama_decoder_b200.dp import DataParallelStep, ShardedDataParallelStep
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        a, b = OffsetEngine(batch), OffsetEngine(batch)
+        DataParallelStep(a)
+        ShardedDataParallelStep(b, 100)
+        q.put((rank, (a.drop_b0, b.drop_b0)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ranks_draw_dropout_masks_at_whole_batch_positions(world):
+    """Rank r's share starts at sequence r * batch of the whole batch; one
+    process (no group) keeps the engine's own offset."""
+    from scratch_llama_decoder_b200.dp import DataParallelStep
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_offsets, args=(r, world, port, 3, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=300) for _ in range(world))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    assert res == {r: (3 * r, 3 * r) for r in range(world)}
+    e = OffsetEngine(3)
+    DataParallelStep(e)
+    assert e.drop_b0 is None
+
+
 def test_two_ranks_equal_one_process_on_the_whole_batch():
     from synth import get_config
     from scratch_llama_decoder_b200.dp import DataParallelStep

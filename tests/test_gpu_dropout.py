@@ -2,7 +2,9 @@
 the float64 oracle with the same masks: the loss and gradients of training
 calls 0 and 1 (different masks) at fp32 and bf16, MHA and GQA; rate 0 is the
 step without dropout bit for bit; evaluation (llm_forward) never drops; a
-replayed step graph draws the same masks as individual launches."""
+replayed step graph draws the same masks as individual launches; contexts over
+halves of a batch with sequence offsets (llm_set_dropout_offset, as the
+data-parallel wrappers set them) draw the whole batch's masks."""
 import numpy as np
 import pytest
 import torch
@@ -121,4 +123,57 @@ def test_set_dropout_arguments():
     for bad in (1.0, -0.1, float("nan"), 1.5):
         assert L.lib.llm_set_dropout(m.ctx, bad, 1) == L.LLM_ERR_ARG
     assert L.lib.llm_set_dropout(m.ctx, 0.0, 1) == 0
+    m.close()
+
+
+@pytest.mark.parametrize("name,over", [("c4", dict(batch=2, ctx=96, n_layer=1)),   # mma, T % 4 == 0
+                                       ("c3", dict(batch=2, ctx=66, n_layer=1)),   # mma, T % 4 != 0
+                                       ("c2", dict(batch=2, ctx=68, n_layer=1))])  # fp32 tiled
+def test_halves_with_offsets_draw_the_whole_batch_masks(name, over):
+    from scratch_llama_decoder_b200 import LlamaStep
+    full = get_config(name, **over)
+    half = dict(full, batch=full["batch"] // 2)
+    hb = half["batch"]
+    lay = O.param_layout(full)
+    p = make_params(full, lay)
+    tok, tgt = make_batch(full)
+    tok, tgt = tok.reshape(full["batch"], -1), tgt.reshape(full["batch"], -1)
+    tol = TOL[full["compute"]]
+    ranks = [LlamaStep(half), LlamaStep(half)]
+    P = torch.tensor(p, device="cuda")
+    lr_, _, gr_ = O.forward_backward(full, p, tok, tgt, want_logits=False,
+                                     dropout=(float(np.float32(P_DROP)), SEED, 0))
+
+    def halves(offsets):
+        G, loss = torch.zeros_like(P), 0.0
+        for r, m in enumerate(ranks):
+            m.set_dropout(P_DROP, SEED)  # the mask counter restarts at 0
+            m.set_dropout_offset(offsets[r])
+            Gr = torch.zeros_like(P)
+            td = torch.tensor(tok[r * hb:(r + 1) * hb], device="cuda").contiguous()
+            yd = torch.tensor(tgt[r * hb:(r + 1) * hb], device="cuda").contiguous()
+            loss += float(m.grad(P, Gr, td, yd).item()) / 2
+            assert m.status() == 0
+            G += Gr
+        return (G / 2).double().cpu().numpy(), loss
+
+    g, loss = halves([0, hb])  # the mean of the halves' mean gradients
+    assert abs(loss - lr_) <= tol["loss"] * abs(lr_), (loss, lr_)
+    for nm, off, rows, cols in lay:
+        e = rel(g[off:off + rows * cols], gr_[off:off + rows * cols])
+        assert e <= tol["grads"], (nm, e)
+    # without the offset the second half draws the first half's masks
+    g0, _ = halves([0, 0])
+    assert rel(g0, gr_) > 10 * tol["grads"]
+    for m in ranks:
+        m.close()
+
+
+def test_dropout_offset_arguments():
+    import scratch_llama_decoder_b200 as L
+    lay, p, tok, tgt, m = _setup(get_config("c1"))
+    assert L.lib.llm_set_dropout_offset(m.ctx, -1) == L.LLM_ERR_ARG
+    assert L.lib.llm_set_dropout_offset(m.ctx, 1 << 31) == L.LLM_ERR_ARG
+    assert L.lib.llm_set_dropout_offset(None, 0) == L.LLM_ERR_ARG
+    assert L.lib.llm_set_dropout_offset(m.ctx, 5) == 0
     m.close()
