@@ -373,7 +373,8 @@ int llm_set_rope_scale(llm_ctx *ctx, float factor);
  * (group index low word, high word, site + 4 * layer, n), group index =
  * element index / 4, with sites 0 embedding, 1 attention probabilities,
  * 2 attention output, 3 MLP output, element indices row-major over those
- * shapes, n = the number of training calls (llm_step or llm_grad) since the
+ * shapes of the whole batch (the context's sequences start at the offset of
+ * llm_set_dropout_offset, 0 by default), n = the number of training calls (llm_step or llm_grad) since the
  * last llm_set_dropout; element e is kept when output word e mod 4 of its
  * group's call is >= floor(p * 2^32).  llm_forward and llm_decode never drop.
  * While dropout is on, bf16 attention with head size 32 or 64 runs in the
